@@ -1,0 +1,214 @@
+"""B200-native QLoRA: NF4 + Double Quantization storage and the QLoRA linear layer.
+
+Python face of libqlora.so (include/qlora.h).  PyTorch provides device
+memory and streams only; every step of the quantizer, doubleDequant and the
+linear forward/backward runs in the library's sm_100a kernels.  The functions
+here allocate outputs and workspaces with torch and pass raw pointers through
+the C ABI.  There is no CPU or PyTorch fallback: without a CUDA device or the
+built library the calls raise.
+
+Paper: "QLoRA: Efficient Finetuning of Quantized LLMs"
+(aiingo.vercel.app/paper/paper-2305-14314), §2 Eqs. 1-3, §3 Eqs. 4-6,
+Appendix E.
+"""
+
+from __future__ import annotations
+
+from dataclasses import dataclass
+
+import torch
+
+from . import _lib
+from ._lib import QLoRAError  # noqa: F401
+
+__all__ = [
+    "NF4Tensor",
+    "quantize_nf4_dq",
+    "dequant",
+    "linear_fwd",
+    "linear_bwd",
+    "last_device_error",
+    "QLoRAError",
+]
+
+
+def _stream(device: torch.device) -> int:
+    return torch.cuda.current_stream(device).cuda_stream
+
+
+def _ptr(t: torch.Tensor | None) -> int | None:
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("qlora: tensors must live on a CUDA device")
+    if not t.is_contiguous():
+        raise ValueError("qlora: tensors must be contiguous")
+    return t.data_ptr()
+
+
+def _bits(t: torch.Tensor) -> torch.Tensor:
+    if t.dtype != torch.bfloat16:
+        raise TypeError(f"qlora: expected a bfloat16 tensor, got {t.dtype}")
+    return t
+
+
+@dataclass
+class NF4Tensor:
+    """A weight in the QLoRA storage format (device buffers owned by torch).
+
+    codes   uint8 [ceil(numel/2)]   NF4 codes, 2 per byte (even element low nibble)
+    c2_fp8  uint8 [ceil(numel/64)]  E4M3 codes of the mean-centred block absmax
+    c1      fp32  [ceil(nblk/256)]  second-level constants
+    c2_mean fp32  [1]               mean of the first-level constants
+    """
+
+    n_out: int
+    k_in: int
+    codes: torch.Tensor
+    c2_fp8: torch.Tensor
+    c1: torch.Tensor
+    c2_mean: torch.Tensor
+
+    @property
+    def shape(self):
+        return (self.n_out, self.k_in)
+
+    @property
+    def device(self):
+        return self.codes.device
+
+    def as_struct(self) -> _lib.NF4DQ:
+        return _lib.NF4DQ(self.n_out, self.k_in, _ptr(self.codes), _ptr(self.c2_fp8), _ptr(self.c1),
+                          _ptr(self.c2_mean))
+
+    def nbytes(self) -> int:
+        return sum(t.numel() * t.element_size() for t in (self.codes, self.c2_fp8, self.c1, self.c2_mean))
+
+
+def _empty_nf4(n_out: int, k_in: int, device) -> NF4Tensor:
+    numel = n_out * k_in
+    nblk = (numel + 63) // 64
+    return NF4Tensor(
+        n_out, k_in,
+        torch.empty((numel + 1) // 2, dtype=torch.uint8, device=device),
+        torch.empty(nblk, dtype=torch.uint8, device=device),
+        torch.empty((nblk + 255) // 256, dtype=torch.float32, device=device),
+        torch.empty(1, dtype=torch.float32, device=device),
+    )
+
+
+def quantize_nf4_dq(W: torch.Tensor, out: NF4Tensor | None = None) -> NF4Tensor:
+    """Quantize a 2-D fp32 or bf16 CUDA weight [n_out, k_in] to NF4 + DQ."""
+    lib = _lib.load()
+    if W.dim() != 2:
+        raise ValueError("qlora: W must be 2-D [n_out, k_in]")
+    if W.dtype == torch.float32:
+        wdt = _lib.QLORA_DTYPE_F32
+    elif W.dtype == torch.bfloat16:
+        wdt = _lib.QLORA_DTYPE_BF16
+    else:
+        raise TypeError("qlora: W must be float32 or bfloat16")
+    n_out, k_in = W.shape
+    q = out if out is not None else _empty_nf4(n_out, k_in, W.device)
+    ws_bytes = lib.qlora_quantize_workspace_size(n_out * k_in)
+    ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=W.device)
+    _lib.check(lib.qlora_quantize_nf4_dq(_ptr(W), wdt, n_out, k_in, _ptr(q.codes), _ptr(q.c2_fp8), _ptr(q.c1),
+                                         _ptr(q.c2_mean), _ptr(ws), ws_bytes, _stream(W.device)),
+               "qlora_quantize_nf4_dq")
+    return q
+
+
+def dequant(q: NF4Tensor, out: torch.Tensor | None = None) -> torch.Tensor:
+    """doubleDequant (Eq. 6): the bf16 weight [n_out, k_in]."""
+    lib = _lib.load()
+    if out is None:
+        out = torch.empty(q.shape, dtype=torch.bfloat16, device=q.device)
+    st = q.as_struct()
+    _lib.check(lib.qlora_dequant(st, _ptr(_bits(out)), _stream(q.device)), "qlora_dequant")
+    return out
+
+
+class _Workspace:
+    """Grow-only scratch buffers, one per (device, stream), reused across calls.
+
+    Calls on one stream run in order, so they can share a buffer; a different
+    stream gets its own.
+    """
+
+    def __init__(self):
+        self.buf: dict = {}
+
+    def get(self, nbytes: int, device) -> torch.Tensor:
+        dev = torch.device(device)
+        key = (dev, _stream(dev))
+        b = self.buf.get(key)
+        if b is None or b.numel() < nbytes:
+            b = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=dev)
+            self.buf[key] = b
+        return b
+
+
+_WS = _Workspace()
+
+
+def linear_fwd(X: torch.Tensor, q: NF4Tensor, L1: torch.Tensor, L2: torch.Tensor, s: float,
+               save_T: bool = True, Y: torch.Tensor | None = None, T: torch.Tensor | None = None):
+    """Y = X doubleDequant(W)^T + s X L1 L2 (Eq. 3 / Eq. 5).  Returns (Y, T or None).
+
+    X [M, K] bf16, L1 [K, r] bf16, L2 [r, N] bf16; T = s X L1 [M, r] bf16.
+    """
+    lib = _lib.load()
+    M, K = X.shape
+    r = L1.shape[1]
+    N = q.n_out
+    if K != q.k_in or L1.shape[0] != K or tuple(L2.shape) != (r, N):
+        raise ValueError("qlora: shape mismatch")
+    dev = X.device
+    if Y is None:
+        Y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    if save_T and T is None:
+        T = torch.empty((M, r), dtype=torch.bfloat16, device=dev)
+    ws_bytes = lib.qlora_linear_fwd_workspace_size(M, N, K, r)
+    ws = _WS.get(ws_bytes, dev)
+    _lib.check(lib.qlora_linear_fwd(_ptr(_bits(X)), M, q.as_struct(), _ptr(_bits(L1)), _ptr(_bits(L2)), r, float(s),
+                                    _ptr(_bits(Y)), _ptr(T) if save_T else None, _ptr(ws), ws.numel(),
+                                    _stream(dev)), "qlora_linear_fwd")
+    return Y, (T if save_T else None)
+
+
+def linear_bwd(dY: torch.Tensor, X: torch.Tensor, T: torch.Tensor | None, q: NF4Tensor, L1: torch.Tensor,
+               L2: torch.Tensor, s: float, need_dX: bool = True, grad_dtype=torch.bfloat16,
+               dX: torch.Tensor | None = None, dL1: torch.Tensor | None = None, dL2: torch.Tensor | None = None):
+    """Adapter-only backward.  Returns (dX or None, dL1 [K, r], dL2 [r, N])."""
+    lib = _lib.load()
+    M, N = dY.shape
+    K = q.k_in
+    r = L1.shape[1]
+    if N != q.n_out or tuple(X.shape) != (M, K) or tuple(L2.shape) != (r, N):
+        raise ValueError("qlora: shape mismatch")
+    if grad_dtype == torch.bfloat16:
+        gdt = _lib.QLORA_DTYPE_BF16
+    elif grad_dtype == torch.float32:
+        gdt = _lib.QLORA_DTYPE_F32
+    else:
+        raise TypeError("qlora: grad_dtype must be bfloat16 or float32")
+    dev = dY.device
+    if need_dX and dX is None:
+        dX = torch.empty((M, K), dtype=torch.bfloat16, device=dev)
+    if dL1 is None:
+        dL1 = torch.empty((K, r), dtype=grad_dtype, device=dev)
+    if dL2 is None:
+        dL2 = torch.empty((r, N), dtype=grad_dtype, device=dev)
+    ws_bytes = lib.qlora_linear_bwd_workspace_size(M, N, K, r)
+    ws = _WS.get(ws_bytes, dev)
+    _lib.check(lib.qlora_linear_bwd(_ptr(_bits(dY)), _ptr(_bits(X)), _ptr(T), M, q.as_struct(), _ptr(_bits(L1)),
+                                    _ptr(_bits(L2)), r, float(s), _ptr(dX) if need_dX else None, _ptr(dL1),
+                                    _ptr(dL2), gdt, _ptr(ws), ws.numel(), _stream(dev)), "qlora_linear_bwd")
+    return (dX if need_dX else None), dL1, dL2
+
+
+def last_device_error(device=None) -> int:
+    """Synchronize the current stream and return/clear the library's device error word."""
+    lib = _lib.load()
+    dev = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
+    return lib.qlora_get_last_device_error(_stream(dev))

@@ -1,0 +1,470 @@
+// libqlora: host side of the C ABI declared in include/qlora.h.
+//
+// One translation unit: the kernels live in the included .cuh files.
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <cstring>
+#include <mutex>
+
+#include "qlora.h"
+#include "common.cuh"
+#include "quant.cuh"
+#include "tc_gemm.cuh"
+
+namespace qlora {
+
+__device__ int g_dev_err;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceInfo {
+  bool init = false;
+  int sms = 0;
+  int *err = nullptr;        // device address of g_dev_err
+  bool gemm_attr[3] = {false, false, false};
+};
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_mu;
+
+int current_device_info(DeviceInfo **out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return QLORA_ERR_CUDA;
+  DeviceInfo &d = g_dev[dev];
+  if (!d.init) {
+    std::lock_guard<std::mutex> lock(g_mu);
+    if (!d.init) {
+      if (cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return QLORA_ERR_CUDA;
+      if (cudaGetSymbolAddress(reinterpret_cast<void **>(&d.err), g_dev_err) != cudaSuccess) return QLORA_ERR_CUDA;
+      d.init = true;
+    }
+  }
+  *out = &d;
+  return QLORA_OK;
+}
+
+bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+size_t align_up(size_t x, size_t a = 256) { return (x + a - 1) / a * a; }
+
+int launch_status() { return cudaGetLastError() == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA; }
+
+// ---------------------------------------------------------------- TMA maps
+using EncodeTiledFn = PFN_cuTensorMapEncodeTiled_v12000;
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// A bf16 operand of the GEMM engine.  K-major: `rows` x `kext` with row stride
+// `ld` elements, contiguous along the reduction.  MN-major: `kext` rows of
+// `rows` contiguous elements (row stride `ld`), i.e. contiguous along M or N.
+struct Operand {
+  const void *ptr;
+  int64_t rows;   // extent along the output dimension (M for A, N for B)
+  int64_t kext;   // extent along the reduction
+  int64_t ld;     // elements between consecutive rows of the stored matrix
+  int mn_major;
+};
+
+int make_tmap(CUtensorMap *m, const Operand &o, int box_rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return QLORA_ERR_CUDA;
+  cuuint64_t dims[2], strides[1];
+  cuuint32_t box[2], estr[2] = {1, 1};
+  if (!o.mn_major) {
+    dims[0] = (cuuint64_t)o.kext;
+    dims[1] = (cuuint64_t)o.rows;
+    box[0] = 64;
+    box[1] = (cuuint32_t)box_rows;
+  } else {
+    dims[0] = (cuuint64_t)o.rows;
+    dims[1] = (cuuint64_t)o.kext;
+    box[0] = 64;
+    box[1] = 64;
+  }
+  strides[0] = (cuuint64_t)o.ld * 2;
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(o.ptr), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? QLORA_OK : QLORA_ERR_CUDA;
+}
+
+struct GemmSeg {
+  Operand A, B;   // A.kext == B.kext
+};
+
+int pick_bn(int64_t N) { return N <= 64 ? 64 : (N <= 128 ? 128 : 256); }
+
+// Split-K factor for a single-segment product whose tile grid leaves SMs idle.
+void choose_splits(int64_t tiles, int64_t nkb, int sms, bool allow, int *splits, int *kbps) {
+  int s = 1;
+  if (allow && tiles < sms && nkb > 1) {
+    s = (int)std::min<int64_t>(nkb, (2 * (int64_t)sms + tiles - 1) / tiles);
+  }
+  int k = (int)((nkb + s - 1) / s);
+  if (k < 1) k = 1;
+  *kbps = k;
+  *splits = (int)((nkb + k - 1) / k);
+  if (*splits < 1) *splits = 1;
+}
+
+size_t gemm_split_ws_bytes(int64_t M, int64_t N, int64_t K, int sms, bool allow) {
+  const int bn = pick_bn(N);
+  const int64_t tiles = ((M + kBM - 1) / kBM) * ((N + bn - 1) / bn);
+  int splits, kbps;
+  choose_splits(tiles, (K + kBK - 1) / kBK, sms, allow, &splits, &kbps);
+  return splits > 1 ? align_up((size_t)splits * (size_t)M * (size_t)N * 4) : 0;
+}
+
+template <int BN>
+int launch_gemm_bn(const CUtensorMap *maps, TcGemmArgs &args, int sms, DeviceInfo *dev, cudaStream_t st) {
+  using Cfg = TcCfg<BN>;
+  const int idx = BN == 64 ? 0 : (BN == 128 ? 1 : 2);
+  if (!dev->gemm_attr[idx]) {
+    if (cudaFuncSetAttribute(tc_gemm_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes) !=
+        cudaSuccess)
+      return QLORA_ERR_CUDA;
+    dev->gemm_attr[idx] = true;
+  }
+  const int units = args.m_tiles * args.n_tiles * args.splits;
+  const int grid = std::max(1, std::min(units, sms));
+  tc_gemm_kernel<BN><<<grid, kGemmThreads, Cfg::kSmemBytes, st>>>(maps[0], maps[1], maps[2], maps[3], args);
+  return launch_status();
+}
+
+// D[M x N] = alpha * sum_seg A_seg B_seg^T, written to `out` with strides
+// (ld_row, ld_col) as bf16 or fp32.  If `split_ws` is given and the tile grid
+// is small, segment 0's reduction is split and the fp32 partials (dense, in
+// the output's strides) are summed by a finalize pass; the output must then be
+// dense: ld_row * ld_col products cover M*N elements exactly.
+int tc_gemm(cudaStream_t st, DeviceInfo *dev, int64_t M, int64_t N, int nseg, const GemmSeg *segs, float alpha,
+            void *out, int64_t ld_row, int64_t ld_col, int out_f32, float *split_ws) {
+  if (M <= 0 || N <= 0) return QLORA_OK;
+  if (M > (int64_t)INT32_MAX / 2 || N > (int64_t)INT32_MAX / 2) return QLORA_ERR_UNSUPPORTED_SHAPE;
+  const int bn = pick_bn(N);
+  CUtensorMap maps[4];
+  std::memset(maps, 0, sizeof(maps));
+  TcGemmArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.M = (int)M;
+  a.N = (int)N;
+  a.m_tiles = (int)((M + kBM - 1) / kBM);
+  a.n_tiles = (int)((N + bn - 1) / bn);
+  a.nseg = nseg;
+  for (int s = 0; s < nseg; ++s) {
+    a.seg[s].nkb = (int)((segs[s].A.kext + kBK - 1) / kBK);
+    a.seg[s].a_mn = segs[s].A.mn_major;
+    a.seg[s].b_mn = segs[s].B.mn_major;
+    int rc = make_tmap(&maps[2 * s], segs[s].A, kBM);
+    if (rc) return rc;
+    rc = make_tmap(&maps[2 * s + 1], segs[s].B, bn);
+    if (rc) return rc;
+  }
+  if (nseg == 1) maps[2] = maps[0], maps[3] = maps[1];
+  int splits, kbps;
+  choose_splits((int64_t)a.m_tiles * a.n_tiles, a.seg[0].nkb, dev->sms, split_ws != nullptr && nseg == 1, &splits,
+                &kbps);
+  a.splits = splits;
+  a.kb_per_split = kbps;
+  a.err = dev->err;
+  a.ld_row = ld_row;
+  a.ld_col = ld_col;
+  if (splits > 1) {
+    a.alpha = 1.f;
+    a.out = split_ws;
+    a.out_f32 = 1;
+    a.split_stride = M * N;
+  } else {
+    a.alpha = alpha;
+    a.out = out;
+    a.out_f32 = out_f32;
+    a.split_stride = 0;
+  }
+  int rc;
+  switch (bn) {
+    case 64: rc = launch_gemm_bn<64>(maps, a, dev->sms, dev, st); break;
+    case 128: rc = launch_gemm_bn<128>(maps, a, dev->sms, dev, st); break;
+    default: rc = launch_gemm_bn<256>(maps, a, dev->sms, dev, st); break;
+  }
+  if (rc || splits == 1) return rc;
+  const int64_t count = M * N;
+  const int grid = (int)std::min<int64_t>((count + 255) / 256, (int64_t)dev->sms * 8);
+  splitk_finalize_kernel<<<grid, 256, 0, st>>>(split_ws, splits, M * N, count, alpha, out, out_f32);
+  return launch_status();
+}
+
+int dequant_launch(const qlora_nf4dq_t *W, __nv_bfloat16 *out, cudaStream_t st, int sms) {
+  const int64_t numel = W->n_out * W->k_in;
+  if (numel == 0) return QLORA_OK;
+  const int64_t n8 = numel >> 3;
+  const int grid = (int)std::max<int64_t>(1, std::min<int64_t>((n8 + 255) / 256, (int64_t)sms * 16));
+  nf4_dequant_kernel<<<grid, 256, 0, st>>>(W->codes, W->c2_fp8, W->c1, W->c2_mean, numel, out);
+  return launch_status();
+}
+
+int check_weight(const qlora_nf4dq_t *W) {
+  if (!W || !W->codes || !W->c2_fp8 || !W->c1 || !W->c2_mean) return QLORA_ERR_INVALID_ARG;
+  if (W->n_out < 0 || W->k_in < 0) return QLORA_ERR_INVALID_ARG;
+  if (!aligned(W->codes, 16) || !aligned(W->c2_fp8, 16) || !aligned(W->c1, 16) || !aligned(W->c2_mean, 4))
+    return QLORA_ERR_MISALIGNED;
+  return QLORA_OK;
+}
+
+// Common validation of the linear entry points.
+int check_linear(int64_t M, const qlora_nf4dq_t *W, int r) {
+  int rc = check_weight(W);
+  if (rc) return rc;
+  if (M < 0 || r <= 0) return QLORA_ERR_INVALID_ARG;
+  if (W->k_in <= 0 || W->n_out <= 0) return QLORA_ERR_INVALID_ARG;
+  if (W->k_in % 64 || W->n_out % 8 || r % 8 || r > QLORA_MAX_RANK) return QLORA_ERR_UNSUPPORTED_SHAPE;
+  if (M > (int64_t)1 << 30 || W->k_in > (int64_t)1 << 30 || W->n_out > (int64_t)1 << 30)
+    return QLORA_ERR_UNSUPPORTED_SHAPE;
+  return QLORA_OK;
+}
+
+struct FwdLayout {
+  size_t w_hat, t, split, total;
+};
+
+FwdLayout fwd_layout(int64_t M, int64_t N, int64_t K, int r, int sms) {
+  FwdLayout L;
+  L.w_hat = 0;
+  L.t = align_up((size_t)N * K * 2);
+  L.split = L.t + align_up((size_t)M * r * 2);
+  L.total = L.split + gemm_split_ws_bytes(M, r, K, sms, true);
+  return L;
+}
+
+struct BwdLayout {
+  size_t w_hat, g, t, split, total;
+};
+
+BwdLayout bwd_layout(int64_t M, int64_t N, int64_t K, int r, int sms) {
+  BwdLayout L;
+  L.w_hat = 0;
+  L.g = align_up((size_t)N * K * 2);
+  L.t = L.g + align_up((size_t)M * r * 2);
+  L.split = L.t + align_up((size_t)M * r * 2);
+  size_t sw = 0;
+  sw = std::max(sw, gemm_split_ws_bytes(M, r, K, sms, true));   // T = s X L1
+  sw = std::max(sw, gemm_split_ws_bytes(M, r, N, sms, true));   // G = s dY L2^T
+  sw = std::max(sw, gemm_split_ws_bytes(N, r, M, sms, true));   // dL2^T = dY^T T
+  sw = std::max(sw, gemm_split_ws_bytes(K, r, M, sms, true));   // dL1 = X^T G
+  L.total = L.split + sw;
+  return L;
+}
+
+}  // namespace
+}  // namespace qlora
+
+using namespace qlora;
+
+extern "C" {
+
+int qlora_version(void) { return 100; }
+
+const char *qlora_status_str(int status) {
+  switch (status) {
+    case QLORA_OK: return "ok";
+    case QLORA_ERR_INVALID_ARG: return "invalid argument";
+    case QLORA_ERR_MISALIGNED: return "misaligned pointer (16-byte alignment required)";
+    case QLORA_ERR_UNSUPPORTED_SHAPE: return "unsupported shape (k_in % 64, n_out % 8, r % 8, r <= 256)";
+    case QLORA_ERR_CUDA: return "CUDA runtime error";
+    case QLORA_ERR_DEVICE_TIMEOUT: return "a kernel's bounded wait expired";
+    case QLORA_ERR_WORKSPACE: return "workspace missing or too small";
+    default: return "unknown status";
+  }
+}
+
+int qlora_get_last_device_error(void *stream) {
+  DeviceInfo *dev;
+  int rc = current_device_info(&dev);
+  if (rc) return rc;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  int h = 0;
+  if (cudaMemcpyAsync(&h, dev->err, sizeof(int), cudaMemcpyDeviceToHost, st) != cudaSuccess) return QLORA_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return QLORA_ERR_CUDA;
+  if (h != 0) {
+    if (cudaMemsetAsync(dev->err, 0, sizeof(int), st) != cudaSuccess) return QLORA_ERR_CUDA;
+    if (cudaStreamSynchronize(st) != cudaSuccess) return QLORA_ERR_CUDA;
+    return QLORA_ERR_DEVICE_TIMEOUT;
+  }
+  return QLORA_OK;
+}
+
+size_t qlora_quantize_workspace_size(int64_t numel) {
+  if (numel < 0) return 0;
+  const int64_t nblk = (numel + 63) / 64;
+  return align_up((size_t)nblk * 4) + align_up((size_t)kQuantMaxCtas * 8);
+}
+
+int qlora_quantize_nf4_dq(const void *W, int w_dtype, int64_t n_out, int64_t k_in, uint8_t *codes, uint8_t *c2_fp8,
+                          float *c1, float *c2_mean, void *ws, size_t ws_bytes, void *stream) {
+  if (n_out < 0 || k_in < 0) return QLORA_ERR_INVALID_ARG;
+  if (w_dtype != QLORA_DTYPE_F32 && w_dtype != QLORA_DTYPE_BF16) return QLORA_ERR_INVALID_ARG;
+  if (k_in > 0 && n_out > INT64_MAX / k_in) return QLORA_ERR_UNSUPPORTED_SHAPE;
+  const int64_t numel = n_out * k_in;
+  if (!c2_mean) return QLORA_ERR_INVALID_ARG;
+  if (!aligned(c2_mean, 4)) return QLORA_ERR_MISALIGNED;
+  DeviceInfo *dev;
+  int rc = current_device_info(&dev);
+  if (rc) return rc;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (numel == 0) return cudaMemsetAsync(c2_mean, 0, sizeof(float), st) == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+  if (!W || !codes || !c2_fp8 || !c1) return QLORA_ERR_INVALID_ARG;
+  if (!aligned(W, 16) || !aligned(codes, 16) || !aligned(c2_fp8, 16) || !aligned(c1, 16)) return QLORA_ERR_MISALIGNED;
+  if (!ws || ws_bytes < qlora_quantize_workspace_size(numel)) return QLORA_ERR_WORKSPACE;
+  if (!aligned(ws, 16)) return QLORA_ERR_MISALIGNED;
+  const int64_t nblk = (numel + 63) / 64;
+  float *c2 = reinterpret_cast<float *>(ws);
+  double *partial = reinterpret_cast<double *>(reinterpret_cast<uint8_t *>(ws) + align_up((size_t)nblk * 4));
+  const int64_t ngroups = numel >> 8;
+  const int grid1 = (int)std::max<int64_t>(1, std::min<int64_t>((ngroups + 7) / 8, kQuantMaxCtas));
+  if (w_dtype == QLORA_DTYPE_F32)
+    nf4_quantize_kernel<float><<<grid1, kQuantThreads, 0, st>>>(reinterpret_cast<const float *>(W), numel, codes, c2,
+                                                               partial);
+  else
+    nf4_quantize_kernel<__nv_bfloat16><<<grid1, kQuantThreads, 0, st>>>(
+        reinterpret_cast<const __nv_bfloat16 *>(W), numel, codes, c2, partial);
+  rc = launch_status();
+  if (rc) return rc;
+  const int64_t nb256 = (nblk + 255) / 256;
+  const int grid2 = (int)std::max<int64_t>(1, std::min<int64_t>(nb256, (int64_t)dev->sms * 4));
+  dq_constants_kernel<<<grid2, 256, 0, st>>>(c2, nblk, partial, grid1, c2_fp8, c1, c2_mean);
+  return launch_status();
+}
+
+int qlora_dequant(const qlora_nf4dq_t *W, uint16_t *W_out, void *stream) {
+  int rc = check_weight(W);
+  if (rc) return rc;
+  if (W->k_in > 0 && W->n_out > INT64_MAX / W->k_in) return QLORA_ERR_UNSUPPORTED_SHAPE;
+  if (W->n_out * W->k_in == 0) return QLORA_OK;
+  if (!W_out) return QLORA_ERR_INVALID_ARG;
+  if (!aligned(W_out, 16)) return QLORA_ERR_MISALIGNED;
+  DeviceInfo *dev;
+  rc = current_device_info(&dev);
+  if (rc) return rc;
+  return dequant_launch(W, reinterpret_cast<__nv_bfloat16 *>(W_out), reinterpret_cast<cudaStream_t>(stream),
+                        dev->sms);
+}
+
+size_t qlora_linear_fwd_workspace_size(int64_t M, int64_t n_out, int64_t k_in, int r) {
+  if (M < 0 || n_out <= 0 || k_in <= 0 || r <= 0) return 0;
+  DeviceInfo *dev;
+  const int sms = current_device_info(&dev) == QLORA_OK ? dev->sms : 148;
+  return fwd_layout(M, n_out, k_in, r, sms).total;
+}
+
+size_t qlora_linear_bwd_workspace_size(int64_t M, int64_t n_out, int64_t k_in, int r) {
+  if (M < 0 || n_out <= 0 || k_in <= 0 || r <= 0) return 0;
+  DeviceInfo *dev;
+  const int sms = current_device_info(&dev) == QLORA_OK ? dev->sms : 148;
+  return bwd_layout(M, n_out, k_in, r, sms).total;
+}
+
+int qlora_linear_fwd(const uint16_t *X, int64_t M, const qlora_nf4dq_t *W, const uint16_t *L1, const uint16_t *L2,
+                     int r, float s, uint16_t *Y, uint16_t *T_save, void *ws, size_t ws_bytes, void *stream) {
+  int rc = check_linear(M, W, r);
+  if (rc) return rc;
+  if (M == 0) return QLORA_OK;
+  if (!X || !L1 || !L2 || !Y) return QLORA_ERR_INVALID_ARG;
+  if (!aligned(X, 16) || !aligned(L1, 16) || !aligned(L2, 16) || !aligned(Y, 16) || (T_save && !aligned(T_save, 16)))
+    return QLORA_ERR_MISALIGNED;
+  DeviceInfo *dev;
+  rc = current_device_info(&dev);
+  if (rc) return rc;
+  const int64_t N = W->n_out, K = W->k_in;
+  const FwdLayout L = fwd_layout(M, N, K, r, dev->sms);
+  if (!ws || ws_bytes < L.total) return QLORA_ERR_WORKSPACE;
+  if (!aligned(ws, 256)) return QLORA_ERR_MISALIGNED;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t *w8 = reinterpret_cast<uint8_t *>(ws);
+  __nv_bfloat16 *w_hat = reinterpret_cast<__nv_bfloat16 *>(w8 + L.w_hat);
+  uint16_t *T = T_save ? T_save : reinterpret_cast<uint16_t *>(w8 + L.t);
+  float *split_ws = reinterpret_cast<float *>(w8 + L.split);
+
+  // 1. doubleDequant of the frozen weight into the bf16 workspace (Eq. 6).
+  rc = dequant_launch(W, w_hat, st, dev->sms);
+  if (rc) return rc;
+  // 2. T = s X L1 (the adapter's down-projection; L1 read MN-major).
+  GemmSeg sT = {{X, M, K, K, 0}, {L1, r, K, r, 1}};
+  rc = tc_gemm(st, dev, M, r, 1, &sT, s, T, r, 1, 0, split_ws);
+  if (rc) return rc;
+  // 3. Y = X W_hat^T + T L2 (the LoRA up-projection as extra K-steps).
+  GemmSeg sY[2] = {{{X, M, K, K, 0}, {w_hat, N, K, K, 0}}, {{T, M, r, r, 0}, {L2, N, r, N, 1}}};
+  return tc_gemm(st, dev, M, N, 2, sY, 1.f, Y, N, 1, 0, nullptr);
+}
+
+int qlora_linear_bwd(const uint16_t *dY, const uint16_t *X, const uint16_t *T_saved, int64_t M,
+                     const qlora_nf4dq_t *W, const uint16_t *L1, const uint16_t *L2, int r, float s, uint16_t *dX,
+                     void *dL1, void *dL2, int grad_dtype, void *ws, size_t ws_bytes, void *stream) {
+  int rc = check_linear(M, W, r);
+  if (rc) return rc;
+  if (grad_dtype != QLORA_DTYPE_F32 && grad_dtype != QLORA_DTYPE_BF16) return QLORA_ERR_INVALID_ARG;
+  if (!L1 || !L2 || !dL1 || !dL2) return QLORA_ERR_INVALID_ARG;
+  if (M > 0 && (!dY || !X)) return QLORA_ERR_INVALID_ARG;
+  if (!aligned(L1, 16) || !aligned(L2, 16) || !aligned(dL1, 16) || !aligned(dL2, 16) || (dY && !aligned(dY, 16)) ||
+      (X && !aligned(X, 16)) || (dX && !aligned(dX, 16)) || (T_saved && !aligned(T_saved, 16)))
+    return QLORA_ERR_MISALIGNED;
+  DeviceInfo *dev;
+  rc = current_device_info(&dev);
+  if (rc) return rc;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int64_t N = W->n_out, K = W->k_in;
+  const size_t gsz = grad_dtype == QLORA_DTYPE_F32 ? 4 : 2;
+  if (M == 0) {  // no tokens: the adapter gradients are zero
+    if (cudaMemsetAsync(dL1, 0, (size_t)K * r * gsz, st) != cudaSuccess) return QLORA_ERR_CUDA;
+    if (cudaMemsetAsync(dL2, 0, (size_t)r * N * gsz, st) != cudaSuccess) return QLORA_ERR_CUDA;
+    return QLORA_OK;
+  }
+  const BwdLayout L = bwd_layout(M, N, K, r, dev->sms);
+  if (!ws || ws_bytes < L.total) return QLORA_ERR_WORKSPACE;
+  if (!aligned(ws, 256)) return QLORA_ERR_MISALIGNED;
+  uint8_t *w8 = reinterpret_cast<uint8_t *>(ws);
+  __nv_bfloat16 *w_hat = reinterpret_cast<__nv_bfloat16 *>(w8 + L.w_hat);
+  uint16_t *G = reinterpret_cast<uint16_t *>(w8 + L.g);
+  float *split_ws = reinterpret_cast<float *>(w8 + L.split);
+  const uint16_t *T = T_saved;
+  const int out_f32 = grad_dtype == QLORA_DTYPE_F32;
+
+  if (!T) {  // recompute T = s X L1
+    uint16_t *Tw = reinterpret_cast<uint16_t *>(w8 + L.t);
+    GemmSeg sT = {{X, M, K, K, 0}, {L1, r, K, r, 1}};
+    rc = tc_gemm(st, dev, M, r, 1, &sT, s, Tw, r, 1, 0, split_ws);
+    if (rc) return rc;
+    T = Tw;
+  }
+  // G = s dY L2^T  (L2 [r x N] is K-major for this product).
+  GemmSeg sG = {{dY, M, N, N, 0}, {L2, r, N, N, 0}};
+  rc = tc_gemm(st, dev, M, r, 1, &sG, s, G, r, 1, 0, split_ws);
+  if (rc) return rc;
+  if (dX) {
+    // dX = dY W_hat + G L1^T: W_hat [N x K] is read in place as an MN-major B.
+    rc = dequant_launch(W, w_hat, st, dev->sms);
+    if (rc) return rc;
+    GemmSeg sX[2] = {{{dY, M, N, N, 0}, {w_hat, K, N, K, 1}}, {{G, M, r, r, 0}, {L1, K, r, r, 0}}};
+    rc = tc_gemm(st, dev, M, K, 2, sX, 1.f, dX, K, 1, 0, nullptr);
+    if (rc) return rc;
+  }
+  // dL2 = T^T dY, computed as dL2^T [N x r] = dY^T T with a transposed store.
+  GemmSeg s2 = {{dY, N, M, N, 1}, {T, r, M, r, 1}};
+  rc = tc_gemm(st, dev, N, r, 1, &s2, 1.f, dL2, 1, N, out_f32, split_ws);
+  if (rc) return rc;
+  // dL1 = X^T G [K x r].
+  GemmSeg s1 = {{X, K, M, K, 1}, {G, r, M, r, 1}};
+  return tc_gemm(st, dev, K, r, 1, &s1, 1.f, dL1, r, 1, out_f32, split_ws);
+}
+
+}  // extern "C"

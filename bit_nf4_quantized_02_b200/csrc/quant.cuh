@@ -1,0 +1,273 @@
+// NF4 blockwise quantizer, Double Quantization and doubleDequant kernels.
+//
+// QLoRA paper (aiingo.vercel.app/paper/paper-2305-14314):
+//   §2 "Block-wise k-bit Quantization": flatten, cut into blocks of B, one
+//      absmax constant per block (Eqs. 1-2);
+//   §3 "4-bit NormalFloat Quantization" + Appendix E: the 16 NF4 levels;
+//   §3 "Double Quantization": the fp32 constants c2 are mean-centred and
+//      quantized to 8-bit floats in blocks of 256, giving c2_fp8 and c1;
+//   §3 "QLoRA", Eq. 6: doubleDequant(c1, c2, W) = dequant(dequant(c1, c2), W).
+//
+// Storage format produced here (the library's on-device NF4 tensor):
+//   codes   uint8 [ceil(numel/2)]  element 2i in the low nibble of byte i,
+//                                  element 2i+1 in the high nibble;
+//   c2_fp8  uint8 [nblk]           OCP E4M3 code of (c2_b - mu) / c1_beta;
+//   c1      fp32  [ceil(nblk/256)] absmax(c2 - mu) / 448 per 256-block;
+//   mu      fp32  [1]              mean of c2 over the whole tensor;
+// with nblk = ceil(numel/64) and c2_b = max |w| over block b.
+#pragma once
+
+#include <cuda_fp8.h>
+
+#include "common.cuh"
+
+namespace qlora {
+
+// The 16 NF4 levels of Appendix E, in code order (all exact in fp32).
+__constant__ float kNF4[16] = {
+    -1.0f,
+    -0.6961928009986877f,
+    -0.5250730514526367f,
+    -0.39491748809814453f,
+    -0.28444138169288635f,
+    -0.18477343022823334f,
+    -0.09105003625154495f,
+    0.0f,
+    0.07958029955625534f,
+    0.16093020141124725f,
+    0.24611230194568634f,
+    0.33791524171829224f,
+    0.44070982933044434f,
+    0.5626170039176941f,
+    0.7229568362236023f,
+    1.0f,
+};
+
+constexpr int kQuantThreads = 256;
+constexpr int kQuantMaxCtas = 148 * 8;
+
+// Decision thresholds for the nearest-level search.  Level j+1 beats level j
+// exactly when x exceeds their midpoint m_j = (q_j + q_{j+1}) / 2, which is
+// exact in fp64; ties stay at the lower level.  For an fp32 x,
+// "x > m_j"  <=>  "x > RD_fp32(m_j)", so comparing against the midpoint
+// rounded toward -inf keeps the decision exact in fp32.
+struct NF4Thresholds {
+  float t[15];
+  __device__ __forceinline__ void init() {
+#pragma unroll
+    for (int j = 0; j < 15; ++j) t[j] = __double2float_rd(((double)kNF4[j] + (double)kNF4[j + 1]) * 0.5);
+  }
+  // code = #{ j : x > m_j } by a 4-step binary search over the sorted thresholds.
+  __device__ __forceinline__ uint32_t encode(float x) const {
+    const bool b3 = x > t[7];
+    const float s2 = b3 ? t[11] : t[3];
+    const bool b2 = x > s2;
+    const float s1 = b3 ? (b2 ? t[13] : t[9]) : (b2 ? t[5] : t[1]);
+    const bool b1 = x > s1;
+    const float s0 = b3 ? (b2 ? (b1 ? t[14] : t[12]) : (b1 ? t[10] : t[8]))
+                        : (b2 ? (b1 ? t[6] : t[4]) : (b1 ? t[2] : t[0]));
+    const bool b0 = x > s0;
+    return ((uint32_t)b3 << 3) | ((uint32_t)b2 << 2) | ((uint32_t)b1 << 1) | (uint32_t)b0;
+  }
+};
+
+__device__ __forceinline__ void load8(const float *__restrict__ p, float (&v)[8]) {
+  const float4 a = __ldg(reinterpret_cast<const float4 *>(p));
+  const float4 b = __ldg(reinterpret_cast<const float4 *>(p) + 1);
+  v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+  v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+}
+
+__device__ __forceinline__ void load8(const __nv_bfloat16 *__restrict__ p, float (&v)[8]) {
+  const uint4 a = __ldg(reinterpret_cast<const uint4 *>(p));
+  const uint32_t w[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    v[2 * i] = __uint_as_float(w[i] << 16);
+    v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+  }
+}
+
+__device__ __forceinline__ float load1(const float *p) { return __ldg(p); }
+__device__ __forceinline__ float load1(const __nv_bfloat16 *p) { return __bfloat162float(*p); }
+
+// Deterministic CTA-wide fp64 sum (fixed reduction tree).
+__device__ __forceinline__ double cta_sum_f64(double v, double *scratch) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_down_sync(0xFFFFFFFFu, v, o);
+  if (lane_id() == 0) scratch[warp_id()] = v;
+  __syncthreads();
+  double s = 0.0;
+  if (threadIdx.x == 0)
+    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) s += scratch[w];
+  __syncthreads();
+  return s;  // valid in thread 0
+}
+
+// K1: per 64-block absmax c2, nearest-level codes, nibble packing, and one
+// fp64 partial sum of c2 per CTA (for the Double-Quantization mean).
+//
+// A warp processes groups of four 64-blocks (256 elements): lane l owns
+// elements [8l, 8l+8) of the group, i.e. 8 lanes per block; the block absmax
+// is reduced over those 8 lanes.  The (at most four) blocks after the last
+// full group are handled by the last CTA, one warp per block.
+template <typename TW>
+__global__ void __launch_bounds__(kQuantThreads) nf4_quantize_kernel(const TW *__restrict__ W, int64_t numel,
+                                                                    uint8_t *__restrict__ codes,
+                                                                    float *__restrict__ c2,
+                                                                    double *__restrict__ partial) {
+  __shared__ double red[kQuantThreads / 32];
+  NF4Thresholds th;
+  th.init();
+  const int lane = lane_id();
+  const int64_t ngroups = numel >> 8;
+  const int64_t nwarps = (int64_t)gridDim.x * (kQuantThreads / 32);
+  double acc = 0.0;
+
+  for (int64_t g = (int64_t)blockIdx.x * (kQuantThreads / 32) + warp_id(); g < ngroups; g += nwarps) {
+    const int64_t base = (g << 8) + (lane << 3);
+    float v[8];
+    load8(W + base, v);
+    float amax = 0.f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[i]));
+    amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 1));
+    amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 2));
+    amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 4));
+    uint32_t packed = 0;
+    if (amax == 0.f) {
+      packed = 0x77777777u;  // all-zero block: every element is the exact-zero level
+    } else {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) packed |= th.encode(__fdiv_rn(v[i], amax)) << (4 * i);
+    }
+    reinterpret_cast<uint32_t *>(codes)[(g << 5) + lane] = packed;
+    if ((lane & 7) == 0) {
+      c2[(g << 2) + (lane >> 3)] = amax;
+      acc += (double)amax;
+    }
+  }
+
+  // Tail: blocks [4*ngroups, nblk), at most 4, one warp each in the last CTA.
+  if (blockIdx.x == gridDim.x - 1) {
+    const int64_t nblk = (numel + 63) >> 6;
+    const int64_t b = (ngroups << 2) + warp_id();
+    if (b < nblk) {
+      const int64_t s = b << 6;
+      const int64_t i0 = s + 2 * lane, i1 = i0 + 1;
+      const float v0 = i0 < numel ? load1(W + i0) : 0.f;
+      const float v1 = i1 < numel ? load1(W + i1) : 0.f;
+      float amax = fmaxf(fabsf(v0), fabsf(v1));
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
+      uint32_t k0 = 7, k1 = 7;
+      if (amax != 0.f) {
+        k0 = th.encode(__fdiv_rn(v0, amax));
+        k1 = i1 < numel ? th.encode(__fdiv_rn(v1, amax)) : 0u;
+      } else if (i1 >= numel) {
+        k1 = 0;
+      }
+      if (i0 < numel) codes[i0 >> 1] = (uint8_t)(k0 | (k1 << 4));
+      if (lane == 0) {
+        c2[b] = amax;
+        acc += (double)amax;
+      }
+    }
+  }
+
+  const double s = cta_sum_f64(acc, red);
+  if (threadIdx.x == 0) partial[blockIdx.x] = s;
+}
+
+// E4M3 (OCP, finite-only) encode with round-to-nearest-even and saturation to
+// +/-448, by the hardware conversion.
+__device__ __forceinline__ uint8_t f32_to_e4m3_satfinite(float x) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(x), "f"(x));
+  return (uint8_t)(r & 0xFFu);
+}
+
+__device__ __forceinline__ float e4m3_to_f32(uint8_t code) {
+  const __half_raw h = __nv_cvt_fp8_to_halfraw((__nv_fp8_storage_t)code, __NV_E4M3);
+  return __half2float(__half(h));
+}
+
+// K2: Double Quantization of c2.  Every CTA first forms the same mean mu from
+// the K1 partials in a fixed order (so mu is deterministic and identical in
+// all CTAs), then quantizes 256-blocks of c2 - mu:
+//   c1 = absmax(c2 - mu) / 448,  code8 = E4M3(fp32((c2 - mu) / c1)).
+__global__ void __launch_bounds__(256) dq_constants_kernel(const float *__restrict__ c2, int64_t nblk,
+                                                           const double *__restrict__ partial, int npartial,
+                                                           uint8_t *__restrict__ c2_fp8, float *__restrict__ c1,
+                                                           float *__restrict__ mu_out) {
+  __shared__ double red[8];
+  __shared__ float mu_s;
+  __shared__ float wmax[8];
+  double acc = 0.0;
+  for (int i = threadIdx.x; i < npartial; i += blockDim.x) acc += partial[i];
+  const double total = cta_sum_f64(acc, red);
+  if (threadIdx.x == 0) {
+    mu_s = __double2float_rn(__ddiv_rn(total, (double)nblk));
+    if (blockIdx.x == 0) *mu_out = mu_s;
+  }
+  __syncthreads();
+  const float mu = mu_s;
+  const int64_t nb256 = (nblk + 255) >> 8;
+  for (int64_t beta = blockIdx.x; beta < nb256; beta += gridDim.x) {
+    const int64_t idx = (beta << 8) + threadIdx.x;
+    const float d = idx < nblk ? __fsub_rn(__ldg(c2 + idx), mu) : 0.f;
+    float a = fabsf(d);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, o));
+    if (lane_id() == 0) wmax[warp_id()] = a;
+    __syncthreads();
+    float A = wmax[0];
+#pragma unroll
+    for (int w = 1; w < 8; ++w) A = fmaxf(A, wmax[w]);
+    __syncthreads();
+    const float c1v = __fdiv_rn(A, 448.0f);
+    if (idx < nblk) c2_fp8[idx] = (c1v == 0.f) ? (uint8_t)0 : f32_to_e4m3_satfinite(__fdiv_rn(d, c1v));
+    if (threadIdx.x == 0) c1[beta] = c1v;
+  }
+}
+
+// K3: doubleDequant (Eq. 6) to bf16:
+//   c2_hat = fma(E4M3(code8_b), c1_beta, mu)   (one rounding)
+//   W_hat  = bf16_rne(fp32(NF4[code] * c2_hat))
+// Each thread converts 8 elements (one 32-bit word of nibbles -> one 16-byte
+// store); a scalar path finishes a numel that is not a multiple of 8.
+__global__ void __launch_bounds__(256) nf4_dequant_kernel(const uint8_t *__restrict__ codes,
+                                                          const uint8_t *__restrict__ c2_fp8,
+                                                          const float *__restrict__ c1,
+                                                          const float *__restrict__ mu_p, int64_t numel,
+                                                          __nv_bfloat16 *__restrict__ out) {
+  __shared__ float lut[16];
+  if (threadIdx.x < 16) lut[threadIdx.x] = kNF4[threadIdx.x];
+  __syncthreads();
+  const float mu = __ldg(mu_p);
+  const int64_t n8 = numel >> 3;
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < n8; e += stride) {
+    const uint32_t q = __ldg(reinterpret_cast<const uint32_t *>(codes) + e);
+    const int64_t b = e >> 3;
+    const float c2h = __fmaf_rn(e4m3_to_f32(__ldg(c2_fp8 + b)), __ldg(c1 + (b >> 8)), mu);
+    uint32_t o[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float lo = __fmul_rn(lut[(q >> (8 * i)) & 0xF], c2h);
+      const float hi = __fmul_rn(lut[(q >> (8 * i + 4)) & 0xF], c2h);
+      const __nv_bfloat162 p = __floats2bfloat162_rn(lo, hi);
+      o[i] = *reinterpret_cast<const uint32_t *>(&p);
+    }
+    reinterpret_cast<uint4 *>(out)[e] = make_uint4(o[0], o[1], o[2], o[3]);
+  }
+  if (blockIdx.x == 0 && threadIdx.x < (numel & 7)) {
+    const int64_t i = (n8 << 3) + threadIdx.x;
+    const int64_t b = i >> 6;
+    const float c2h = __fmaf_rn(e4m3_to_f32(c2_fp8[b]), c1[b >> 8], mu);
+    const uint32_t code = (codes[i >> 1] >> ((i & 1) * 4)) & 0xF;
+    out[i] = __float2bfloat16_rn(__fmul_rn(lut[code], c2h));
+  }
+}
+
+}  // namespace qlora

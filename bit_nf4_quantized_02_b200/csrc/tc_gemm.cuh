@@ -1,0 +1,320 @@
+// Persistent tcgen05 GEMM engine for every dense product of the QLoRA linear.
+//
+//   D[M x N] = alpha * sum_seg A_seg[M x K_seg] * B_seg[N x K_seg]^T
+//
+// One kernel, warp-specialised, one CTA per SM:
+//   warp 0        TMA producer: 128-byte-swizzled tiles of A and B into a ring
+//                 of shared-memory stages (mbarrier full/empty pairs);
+//   warp 1        allocates TMEM, one thread issues tcgen05.mma (bf16 in, fp32
+//                 accumulate) into one of two TMEM accumulators;
+//   warps 2..5    epilogue: tcgen05.ld the accumulator, scale, convert, store;
+//                 the second accumulator lets the next tile's MMAs overlap.
+// Each segment has its own operand major-ness (K-major = contiguous along the
+// reduction; MN-major = contiguous along the output rows/columns), selected
+// per MMA through the instruction descriptor, so X*W^T, dY*W (W read in its
+// stored layout), X^T*G and the LoRA extra K-steps all run on this engine.
+// A segment-0 split of the reduction (split-K) writes fp32 partials that a
+// finalize kernel sums in a fixed order.
+#pragma once
+
+#include "common.cuh"
+
+namespace qlora {
+
+constexpr int kBM = 128;   // MMA M (TMEM lanes)
+constexpr int kBK = 64;    // one 128-byte swizzle row of bf16
+constexpr int kGemmThreads = 192;
+
+struct TcSeg {
+  int nkb;   // 64-wide k-blocks in this segment
+  int a_mn;  // A is MN-major (contiguous along M)
+  int b_mn;  // B is MN-major (contiguous along N)
+};
+
+struct TcGemmArgs {
+  int M, N;
+  int m_tiles, n_tiles, splits, kb_per_split;
+  int nseg;
+  TcSeg seg[2];
+  float alpha;
+  void *out;
+  int64_t ld_row, ld_col;   // element strides of D(i, j) in `out`
+  int64_t split_stride;     // elements between split-K partial outputs
+  int out_f32;              // 1: fp32 output, 0: bf16
+  int *err;
+};
+
+template <int BN>
+struct TcCfg {
+  static constexpr int kABytes = kBM * kBK * 2;
+  static constexpr int kBBytes = BN * kBK * 2;
+  static constexpr int kStageBytes = kABytes + kBBytes;
+  static constexpr int kStages = BN == 256 ? 4 : (BN == 128 ? 6 : 8);
+  static constexpr int kTmemCols = 2 * BN;
+  static constexpr int kBarBytes = 256;
+  static constexpr int kSmemBytes = kStages * kStageBytes + kBarBytes + 1024;
+};
+
+__device__ __forceinline__ void tc_unit_coords(int u, const TcGemmArgs &p, int &mt, int &nt, int &split) {
+  const int tiles = p.m_tiles * p.n_tiles;
+  split = u / tiles;
+  const int t = u - split * tiles;
+  constexpr int kGroupM = 8;  // sweep 8 M-tiles across all N-tiles: B panels stay in L2
+  const int per_group = kGroupM * p.n_tiles;
+  const int group = t / per_group;
+  const int first_m = group * kGroupM;
+  const int gm = min(p.m_tiles - first_m, kGroupM);
+  const int r = t - group * per_group;
+  mt = first_m + r % gm;
+  nt = r / gm;
+}
+
+__device__ __forceinline__ void tc_seg_range(const TcGemmArgs &p, int s, int split, int &kb0, int &kb1) {
+  if (s == 0) {
+    kb0 = split * p.kb_per_split;
+    kb1 = min(p.seg[0].nkb, kb0 + p.kb_per_split);
+  } else {
+    kb0 = 0;
+    kb1 = split == 0 ? p.seg[1].nkb : 0;
+  }
+}
+
+template <int BN>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    tc_gemm_kernel(const __grid_constant__ CUtensorMap tA0, const __grid_constant__ CUtensorMap tB0,
+                   const __grid_constant__ CUtensorMap tA1, const __grid_constant__ CUtensorMap tB1,
+                   const TcGemmArgs p) {
+  using Cfg = TcCfg<BN>;
+  constexpr int S = Cfg::kStages;
+  extern __shared__ uint8_t smem_raw[];
+  // 1024-byte alignment: the 128B-swizzle pattern repeats every 8 rows of 128 B.
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t *bar_area = smem + S * Cfg::kStageBytes;
+  uint64_t *full_bar = reinterpret_cast<uint64_t *>(bar_area);
+  uint64_t *empty_bar = full_bar + S;
+  uint64_t *tfull_bar = empty_bar + S;       // [2]
+  uint64_t *tempty_bar = tfull_bar + 2;      // [2]
+  uint64_t *done_bar = tempty_bar + 2;       // [1]
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(done_bar + 1);
+
+  const int warp = warp_id();
+  const int lane = lane_id();
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < S; ++i) {
+      mbar_init(smem_u32(full_bar + i), 1);
+      mbar_init(smem_u32(empty_bar + i), 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(smem_u32(tfull_bar + i), 1);
+      mbar_init(smem_u32(tempty_bar + i), 4 * 32);
+    }
+    mbar_init(smem_u32(done_bar), 1);
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tA0);
+    tma_prefetch_desc(&tB0);
+    if (p.nseg > 1) {
+      tma_prefetch_desc(&tA1);
+      tma_prefetch_desc(&tB1);
+    }
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), Cfg::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  const int units = p.m_tiles * p.n_tiles * p.splits;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t used = 0;           // stages that received at least one load
+      uint32_t last_parity = 0;    // parity of the last load issued into each stage
+      bool ok = true;
+      for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
+        int mt, nt, split;
+        tc_unit_coords(u, p, mt, nt, split);
+        for (int s = 0; s < p.nseg && ok; ++s) {
+          const CUtensorMap *ta = s == 0 ? &tA0 : &tA1;
+          const CUtensorMap *tb = s == 0 ? &tB0 : &tB1;
+          int kb0, kb1;
+          tc_seg_range(p, s, split, kb0, kb1);
+          for (int kb = kb0; kb < kb1; ++kb) {
+            if (!mbar_wait(smem_u32(empty_bar + stage), phase ^ 1, p.err, DEV_TIMEOUT_PRODUCER)) {
+              ok = false;
+              break;
+            }
+            const uint32_t fb = smem_u32(full_bar + stage);
+            mbar_arrive_expect_tx(fb, Cfg::kStageBytes);
+            const uint32_t sa = smem_u32(smem + stage * Cfg::kStageBytes);
+            const uint32_t sb = sa + Cfg::kABytes;
+            if (!p.seg[s].a_mn) {
+              tma_load_2d(sa, ta, fb, kb * kBK, mt * kBM);
+            } else {
+              tma_load_2d(sa, ta, fb, mt * kBM, kb * kBK);
+              tma_load_2d(sa + 8192, ta, fb, mt * kBM + 64, kb * kBK);
+            }
+            if (!p.seg[s].b_mn) {
+              tma_load_2d(sb, tb, fb, kb * kBK, nt * BN);
+            } else {
+#pragma unroll
+              for (int j = 0; j < BN / 64; ++j) tma_load_2d(sb + j * 8192, tb, fb, nt * BN + 64 * j, kb * kBK);
+            }
+            used |= 1u << stage;
+            last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
+            if (++stage == S) {
+              stage = 0;
+              phase ^= 1;
+            }
+          }
+        }
+      }
+      // Drain: never leave the CTA while a tensor copy is still landing in
+      // shared memory.
+      for (int i = 0; i < S; ++i)
+        if (used & (1u << i)) mbar_wait(smem_u32(full_bar + i), (last_parity >> i) & 1u, p.err, DEV_TIMEOUT_DRAIN);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      uint32_t idesc[2];
+      for (int s = 0; s < 2; ++s) idesc[s] = idesc_bf16_f32(kBM, BN, p.seg[s].a_mn, p.seg[s].b_mn);
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      int t = 0;
+      for (int u = blockIdx.x; u < units && ok; u += gridDim.x, ++t) {
+        int mt, nt, split;
+        tc_unit_coords(u, p, mt, nt, split);
+        const int acc = t & 1;
+        const uint32_t use = (uint32_t)(t >> 1);
+        if (!mbar_wait(smem_u32(tempty_bar + acc), (use & 1u) ^ 1u, p.err, DEV_TIMEOUT_MMA)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
+        uint32_t accumulate = 0;
+        for (int s = 0; s < p.nseg && ok; ++s) {
+          int kb0, kb1;
+          tc_seg_range(p, s, split, kb0, kb1);
+          const int a_mn = p.seg[s].a_mn, b_mn = p.seg[s].b_mn;
+          for (int kb = kb0; kb < kb1; ++kb) {
+            if (!mbar_wait(smem_u32(full_bar + stage), phase, p.err, DEV_TIMEOUT_MMA)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t sa = smem_u32(smem + stage * Cfg::kStageBytes);
+            const uint32_t sb = sa + Cfg::kABytes;
+#pragma unroll
+            for (int k = 0; k < kBK / 16; ++k) {
+              // K-major: the 16-wide k-slice starts 32 B into each swizzled row.
+              // MN-major: it starts 16 rows (2 KB) further down the tile.
+              const uint64_t ad = a_mn ? smem_desc_sw128(sa + k * 2048, 8192, 1024) : smem_desc_sw128(sa + k * 32, 16, 1024);
+              const uint64_t bd = b_mn ? smem_desc_sw128(sb + k * 2048, 8192, 1024) : smem_desc_sw128(sb + k * 32, 16, 1024);
+              tc_mma_f16(d_tmem, ad, bd, idesc[s], accumulate);
+              accumulate = 1;
+            }
+            tc_commit(smem_u32(empty_bar + stage));  // frees the stage once these MMAs have read it
+            if (++stage == S) {
+              stage = 0;
+              phase ^= 1;
+            }
+          }
+        }
+        tc_commit(smem_u32(tfull_bar + acc));        // accumulator ready for the epilogue
+      }
+      // All MMAs issued by this thread must finish before TMEM is released.
+      tc_commit(smem_u32(done_bar));
+      mbar_wait(smem_u32(done_bar), 0, p.err, DEV_TIMEOUT_DRAIN);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;  // TMEM lane quarter this warp may access
+    int t = 0;
+    for (int u = blockIdx.x; u < units; u += gridDim.x, ++t) {
+      int mt, nt, split;
+      tc_unit_coords(u, p, mt, nt, split);
+      const int acc = t & 1;
+      const uint32_t use = (uint32_t)(t >> 1);
+      if (!mbar_wait(smem_u32(tfull_bar + acc), use & 1u, p.err, DEV_TIMEOUT_EPILOGUE)) break;
+      tc_fence_after();
+      const int row = mt * kBM + q * 32 + lane;
+      const bool row_ok = row < p.M;
+      const float alpha = p.alpha;
+#pragma unroll 1
+      for (int c = 0; c < BN; c += 32) {
+        uint32_t r[32];
+        tmem_ld_32x32b_x32(tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN + c), r);
+        tmem_wait_ld();
+        const int col0 = nt * BN + c;
+        if (!row_ok || col0 >= p.N) continue;
+        if (p.out_f32) {
+          float *o = reinterpret_cast<float *>(p.out) + (int64_t)split * p.split_stride;
+          if (p.ld_col == 1 && col0 + 32 <= p.N) {
+            float4 *dst = reinterpret_cast<float4 *>(o + (int64_t)row * p.ld_row + col0);
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+              dst[j] = make_float4(alpha * __uint_as_float(r[4 * j]), alpha * __uint_as_float(r[4 * j + 1]),
+                                   alpha * __uint_as_float(r[4 * j + 2]), alpha * __uint_as_float(r[4 * j + 3]));
+          } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              if (col0 + j < p.N) o[(int64_t)row * p.ld_row + (int64_t)(col0 + j) * p.ld_col] = alpha * __uint_as_float(r[j]);
+          }
+        } else {
+          __nv_bfloat16 *o = reinterpret_cast<__nv_bfloat16 *>(p.out);
+          if (p.ld_col == 1 && col0 + 32 <= p.N) {
+            uint4 *dst = reinterpret_cast<uint4 *>(o + (int64_t)row * p.ld_row + col0);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              uint32_t w[4];
+#pragma unroll
+              for (int h = 0; h < 4; ++h) {
+                const __nv_bfloat162 b2 = __floats2bfloat162_rn(alpha * __uint_as_float(r[8 * j + 2 * h]),
+                                                                alpha * __uint_as_float(r[8 * j + 2 * h + 1]));
+                w[h] = *reinterpret_cast<const uint32_t *>(&b2);
+              }
+              dst[j] = make_uint4(w[0], w[1], w[2], w[3]);
+            }
+          } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              if (col0 + j < p.N)
+                o[(int64_t)row * p.ld_row + (int64_t)(col0 + j) * p.ld_col] = __float2bfloat16_rn(alpha * __uint_as_float(r[j]));
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(smem_u32(tempty_bar + acc));
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem_base, Cfg::kTmemCols);
+}
+
+// Fixed-order sum of split-K partials: dst[i] = alpha * sum_s part[s * stride + i].
+__global__ void __launch_bounds__(256) splitk_finalize_kernel(const float *__restrict__ part, int splits,
+                                                              int64_t stride, int64_t count, float alpha,
+                                                              void *dst, int dst_f32) {
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < count; i += (int64_t)gridDim.x * blockDim.x) {
+    float s = 0.f;
+    for (int k = 0; k < splits; ++k) s += __ldg(part + (int64_t)k * stride + i);
+    s *= alpha;
+    if (dst_f32)
+      reinterpret_cast<float *>(dst)[i] = s;
+    else
+      reinterpret_cast<__nv_bfloat16 *>(dst)[i] = __float2bfloat16_rn(s);
+  }
+}
+
+}  // namespace qlora

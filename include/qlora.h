@@ -1,0 +1,167 @@
+/*
+ * qlora.h -- C ABI of the B200 (sm_100a) QLoRA NF4 library (libqlora.so).
+ *
+ * The operations are those of "QLoRA: Efficient Finetuning of Quantized LLMs"
+ * (Dettmers et al.; page aiingo.vercel.app/paper/paper-2305-14314):
+ *   - blockwise absmax quantization of a frozen weight to the 4-bit NormalFloat
+ *     type (§2 "Block-wise k-bit Quantization"; §3 "4-bit NormalFloat
+ *     Quantization", Eq. 4; exact levels in Appendix E), block size 64;
+ *   - Double Quantization of the per-block fp32 constants to 8-bit floats in
+ *     blocks of 256 after subtracting their mean (§3 "Double Quantization");
+ *   - doubleDequant to bfloat16 (§3 "QLoRA", Eq. 6);
+ *   - the QLoRA linear layer Y = X doubleDequant(c1, c2, W) + s X L1 L2
+ *     (§2 Eq. 3, §3 Eq. 5) and its backward, which produces dX through the
+ *     dequantized frozen weight and gradients for the adapter L1, L2 only
+ *     (§3, paragraph after Eq. 6).  There is no dW.
+ *
+ * Conventions shared by every entry point
+ *   - Memory: every pointer argument is a DEVICE pointer owned by the caller,
+ *     except where a parameter says otherwise.  The library never allocates
+ *     device memory: scratch space is passed in as (ws, ws_bytes) and must be
+ *     at least the size the matching *_workspace_size() function returns.
+ *   - Streams: `stream` is a cudaStream_t (NULL = legacy default stream).
+ *     Every call only enqueues work on that stream and never synchronizes it;
+ *     outputs are valid once the stream has reached that point.
+ *   - bfloat16 data is passed as uint16_t bit patterns.
+ *   - Alignment: every device pointer must be 16-byte aligned (W->c2_mean and
+ *     c2_mean only need 4 bytes).
+ *   - Errors: every call returns an int status (QLORA_OK = 0 or a negative
+ *     QLORA_ERR_*); argument errors are detected on the host before anything
+ *     is enqueued.  A kernel never traps: if a pipeline wait inside a kernel
+ *     exceeds its time bound the kernel records a device error and returns,
+ *     which qlora_get_last_device_error() reports.
+ *   - Shapes: W is stored as [n_out x k_in] row-major (a PyTorch Linear.weight;
+ *     the paper's W in R^{h x o} transposed).  Blocks of 64 run along the
+ *     row-major flattening, so with k_in % 64 == 0 every block lies inside one
+ *     output row.
+ */
+#ifndef QLORA_H_
+#define QLORA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define QLORA_API __attribute__((visibility("default")))
+#else
+#define QLORA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---- status codes ------------------------------------------------------ */
+#define QLORA_OK 0
+#define QLORA_ERR_INVALID_ARG (-1)       /* null pointer, negative size, bad dtype, bad rank */
+#define QLORA_ERR_MISALIGNED (-2)        /* a pointer violates the alignment rule above */
+#define QLORA_ERR_UNSUPPORTED_SHAPE (-3) /* k_in % 64, n_out % 8 or r % 8 not 0, r > 256, size limits */
+#define QLORA_ERR_CUDA (-4)              /* a CUDA runtime call or launch failed */
+#define QLORA_ERR_DEVICE_TIMEOUT (-5)    /* a kernel's bounded wait expired (see below) */
+#define QLORA_ERR_WORKSPACE (-6)         /* ws is NULL or smaller than required */
+
+/* ---- dtypes ---------------------------------------------------------------- */
+#define QLORA_DTYPE_F32 0
+#define QLORA_DTYPE_BF16 1
+
+/* Largest LoRA rank supported by the linear entry points. */
+#define QLORA_MAX_RANK 256
+
+/*
+ * A quantized weight: a view of caller-owned device buffers (not owned).
+ * n = n_out * k_in elements, nblk = ceil(n / 64) blocks, n1 = ceil(nblk / 256).
+ */
+typedef struct {
+  int64_t n_out, k_in;    /* logical shape of W: [n_out x k_in] row-major            */
+  const uint8_t *codes;   /* [ceil(n/2)] NF4 codes, 2 per byte: element 2i in the low
+                             nibble of byte i, element 2i+1 in the high nibble         */
+  const uint8_t *c2_fp8;  /* [nblk] OCP E4M3 code of (c2_b - mean) / c1               */
+  const float *c1;        /* [n1] second-level constants: absmax(c2 - mean) / 448    */
+  const float *c2_mean;   /* [1] mean of the first-level constants c2                 */
+} qlora_nf4dq_t;
+
+/* ---- quantizer -------------------------------------------------------------- */
+
+/* Scratch bytes qlora_quantize_nf4_dq needs for a tensor of `numel` elements. */
+QLORA_API size_t qlora_quantize_workspace_size(int64_t numel);
+
+/*
+ * NF4 + Double Quantization of a frozen weight (§2 blockwise quantization,
+ * §3 NF4 and Double Quantization, Appendix E levels).
+ *   W        [n_out x k_in] fp32 or bf16 (w_dtype), finite values.
+ *   For each 64-block b of the row-major flattening: c2_b = max |w|;
+ *   code = nearest NF4 level to fp32(w / c2_b) (IEEE division; exact ties go to
+ *   the lower level; an all-zero block gets the exact-zero code 7); codes are
+ *   packed two per byte (see qlora_nf4dq_t).
+ *   Then mean = fp32(sum c2 / nblk) (deterministic fp64 sum) and for each
+ *   256-block beta of c2: d = fp32(c2 - mean), c1_beta = fp32(max|d| / 448),
+ *   c2_fp8 = E4M3 round-to-nearest-even, saturating, of fp32(d / c1_beta)
+ *   (code 0 when c1_beta == 0).
+ *   Outputs: codes [ceil(n/2)], c2_fp8 [nblk], c1 [n1], c2_mean [1].
+ *   Any n_out, k_in >= 0 (a final partial block uses only its real elements).
+ */
+QLORA_API int qlora_quantize_nf4_dq(const void *W, int w_dtype, int64_t n_out, int64_t k_in, uint8_t *codes,
+                          uint8_t *c2_fp8, float *c1, float *c2_mean, void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * doubleDequant (§3 Eq. 6) of the whole weight to bf16:
+ *   c2_hat = fma_fp32(E4M3(c2_fp8_b), c1_beta, mean)  (one rounding),
+ *   W_out  = bf16_rne(fp32(NF4[code] * c2_hat)).
+ *   W_out  [n_out x k_in] bf16, row-major.  No workspace.
+ */
+QLORA_API int qlora_dequant(const qlora_nf4dq_t *W, uint16_t *W_out, void *stream);
+
+/* ---- QLoRA linear ------------------------------------------------------------ */
+
+/* Scratch bytes for qlora_linear_fwd / qlora_linear_bwd at these sizes. */
+QLORA_API size_t qlora_linear_fwd_workspace_size(int64_t M, int64_t n_out, int64_t k_in, int r);
+QLORA_API size_t qlora_linear_bwd_workspace_size(int64_t M, int64_t n_out, int64_t k_in, int r);
+
+/*
+ * Forward (§2 Eq. 3 / §3 Eq. 5 with the scale s of Eq. 3):
+ *   Y = X doubleDequant(W)^T + T L2,  T = s X L1.
+ *   X [M x K] bf16, L1 [K x r] bf16, L2 [r x N] bf16, Y [M x N] bf16 (out),
+ *   T_save [M x r] bf16 (out, may be NULL): the adapter down-projection s X L1
+ *   as used by the forward, for the backward.
+ *   K = W->k_in (multiple of 64), N = W->n_out (multiple of 8), r a multiple of
+ *   8 in [8, 256].  All products accumulate in fp32 on the tensor cores.
+ */
+QLORA_API int qlora_linear_fwd(const uint16_t *X, int64_t M, const qlora_nf4dq_t *W, const uint16_t *L1, const uint16_t *L2,
+                     int r, float s, uint16_t *Y, uint16_t *T_save, void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * Backward (§3, paragraph after Eq. 6: adapter gradients only, the gradient
+ * passing through the weight dequantized to bf16):
+ *   G   = s dY L2^T                  [M x r] (internal, bf16)
+ *   dX  = dY doubleDequant(W) + G L1^T   [M x K] bf16 (out; may be NULL to skip)
+ *   dL2 = T^T dY                     [r x N] (out)
+ *   dL1 = X^T G                      [K x r] (out)
+ *   T_saved [M x r] bf16 from the forward, or NULL to recompute T = s X L1.
+ *   dL1, dL2 are written (not accumulated) as grad_dtype (QLORA_DTYPE_BF16 or
+ *   QLORA_DTYPE_F32).  Shape rules as for the forward.
+ */
+QLORA_API int qlora_linear_bwd(const uint16_t *dY, const uint16_t *X, const uint16_t *T_saved, int64_t M,
+                     const qlora_nf4dq_t *W, const uint16_t *L1, const uint16_t *L2, int r, float s, uint16_t *dX,
+                     void *dL1, void *dL2, int grad_dtype, void *ws, size_t ws_bytes, void *stream);
+
+/* ---- diagnostics ----------------------------------------------------------------- */
+
+/* Static description of a status code. */
+QLORA_API const char *qlora_status_str(int status);
+
+/*
+ * Synchronizes `stream`, then returns and clears the device error word of the
+ * current device: QLORA_OK, or QLORA_ERR_DEVICE_TIMEOUT if a kernel gave up a
+ * bounded wait since the last call (the kernel's outputs are then invalid),
+ * or QLORA_ERR_CUDA if the synchronization itself failed.
+ */
+QLORA_API int qlora_get_last_device_error(void *stream);
+
+/* Library version (major * 10000 + minor * 100 + patch). */
+QLORA_API int qlora_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QLORA_H_ */

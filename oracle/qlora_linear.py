@@ -66,3 +66,12 @@ def backward_dx_rows(dY_rows, W_hat, L1, L2, s: float):
     dY_rows, W_hat, L1, L2 = map(_f64, (dY_rows, W_hat, L1, L2))
     G = s * (dY_rows @ L2.T)
     return dY_rows @ W_hat + G @ L1.T
+
+
+def adapter_grads(dY, X, L1, L2, s: float):
+    """(dL1, dL2) of ``backward`` alone; they do not involve the frozen weight."""
+    dY, X, L1, L2 = map(_f64, (dY, X, L1, L2))
+    G = s * (dY @ L2.T)
+    dL2 = s * ((X @ L1).T @ dY)
+    dL1 = X.T @ G
+    return dL1, dL2

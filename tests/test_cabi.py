@@ -1,0 +1,84 @@
+"""The C-ABI library loads, exports every entry point declared in
+include/qlora.h, and rejects bad arguments on the host (no GPU needed)."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+from conftest import ROOT
+
+HEADER = os.path.join(ROOT, "include", "qlora.h")
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(qlora_\w+)\s*\(", src)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from bit_nf4_quantized_02_b200 import _lib, build
+    build.build()
+    return _lib.load()
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for required in ("qlora_quantize_nf4_dq", "qlora_dequant", "qlora_linear_fwd", "qlora_linear_bwd"):
+        assert required in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+
+
+def test_binding_covers_every_declared_symbol():
+    from bit_nf4_quantized_02_b200 import _lib
+    assert set(declared_functions()) <= set(_lib.SIGNATURES)
+
+
+def test_exported_symbols_are_only_the_c_abi(lib):
+    import subprocess
+    out = subprocess.run(["nm", "-D", "--defined-only", lib._name], capture_output=True, text=True).stdout
+    exported = {l.split()[-1] for l in out.splitlines() if " T " in l}
+    assert exported == set(declared_functions())
+
+
+def test_status_strings_and_version(lib):
+    assert lib.qlora_version() >= 100
+    for code in (0, -1, -2, -3, -4, -5, -6):
+        assert lib.qlora_status_str(code)
+
+
+def test_host_argument_validation(lib):
+    from bit_nf4_quantized_02_b200 import _lib
+    # bad dtype / negative sizes are rejected before any CUDA call
+    assert lib.qlora_quantize_nf4_dq(None, 7, 4, 64, None, None, None, None, None, 0, None) == _lib.QLORA_ERR_INVALID_ARG
+    assert lib.qlora_quantize_nf4_dq(None, 0, -1, 64, None, None, None, None, None, 0, None) == _lib.QLORA_ERR_INVALID_ARG
+    # a weight view with missing buffers
+    w = _lib.NF4DQ(8, 64, None, None, None, None)
+    assert lib.qlora_dequant(ctypes.byref(w), None, None) == _lib.QLORA_ERR_INVALID_ARG
+    # shape rules of the linear: K % 64, N % 8, r % 8, r <= 256
+    fake = 1 << 20  # aligned non-null placeholders: validation fails before any use
+    for n_out, k_in, r, want in ((8, 60, 8, _lib.QLORA_ERR_UNSUPPORTED_SHAPE),
+                                 (12, 64, 8, _lib.QLORA_ERR_UNSUPPORTED_SHAPE),
+                                 (8, 64, 12, _lib.QLORA_ERR_UNSUPPORTED_SHAPE),
+                                 (8, 64, 264, _lib.QLORA_ERR_UNSUPPORTED_SHAPE),
+                                 (8, 64, 0, _lib.QLORA_ERR_INVALID_ARG)):
+        wq = _lib.NF4DQ(n_out, k_in, fake, fake, fake, fake)
+        rc = lib.qlora_linear_fwd(fake, 4, ctypes.byref(wq), fake, fake, r, 1.0, fake, None, fake, 1 << 30, None)
+        assert rc == want, (n_out, k_in, r, rc)
+    # misaligned weight buffers
+    wq = _lib.NF4DQ(8, 64, fake + 4, fake, fake, fake)
+    assert lib.qlora_linear_fwd(fake, 4, ctypes.byref(wq), fake, fake, 8, 1.0, fake, None, fake, 1 << 30,
+                                None) == _lib.QLORA_ERR_MISALIGNED
+
+
+def test_workspace_sizes_are_host_only(lib):
+    assert lib.qlora_quantize_workspace_size(1 << 20) >= (1 << 20) // 64 * 4
+    assert lib.qlora_linear_fwd_workspace_size(8192, 4096, 4096, 64) >= 4096 * 4096 * 2
+    assert lib.qlora_linear_bwd_workspace_size(8192, 4096, 4096, 64) >= 4096 * 4096 * 2 + 2 * 8192 * 64 * 2

@@ -82,3 +82,10 @@ def test_finite_differences():
             args_m[which][idx] -= h
             num[idx] = (E(*args_p) - E(*args_m)) / (2 * h)
         assert np.allclose(num, grad, rtol=1e-6, atol=1e-8)
+
+
+def test_adapter_grads_equal_backward():
+    X, W, L1, L2, dY = _case(36)
+    _, dL1, dL2 = qlora_linear.backward(dY, X, W, L1, L2, 0.3)
+    a1, a2 = qlora_linear.adapter_grads(dY, X, L1, L2, 0.3)
+    assert np.array_equal(a1, dL1) and np.array_equal(a2, dL2)
