@@ -1,0 +1,427 @@
+#!/usr/bin/env python
+"""Benchmark of the QLoRA NF4 + DQ linear layer on B200.
+
+Workload (one "step"): the seven linears of a LLaMA-7B layer (q, k, v, o:
+4096x4096; gate, up: 4096->11008; down: 11008->4096), LoRA r=64, alpha=16
+(s=0.25), 16x512 = 8192 tokens, synthetic seeded inputs:
+  1. NF4 + Double-Quantization of the seven fp32 N(0, 0.02^2) weights,
+  2. forward of the seven linears (Y = X W_hat^T + s X L1 L2),
+  3. backward in reverse order (dX, dL1, dL2; no dW),
+  4. with N > 1 ranks: all-reduce of the adapter gradients (data parallel).
+Metric: algorithmic TFLOP/s of the linear forward+backward (4MKN + 6Mr(K+N)
+per linear; quantization and dequantization work not counted), whole job.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Prints one JSON line (rank 0).
+"""
+
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+from synth import inputs, workloads  # noqa: E402
+
+WL = workloads.LLAMA7B_LAYER
+METRIC = "QLoRA NF4 linear fwd+bwd TFLOP/s"
+UNIT = "TFLOP/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def linear_flops(M, N, K, r):
+    base = 2 * M * K * N
+    lora = 2 * M * r * (K + N)
+    return {"fwd": base + lora, "bwd": base + 2 * lora, "fwd_bwd": 2 * base + 3 * lora,
+            "gemm_Y": base + 2 * M * r * N, "gemm_dX": base + 2 * M * r * K}
+
+
+def step_flops(M=WL.M, r=WL.r):
+    return sum(linear_flops(M, l.n_out, l.k_in, r)["fwd_bwd"] for l in WL.linears)
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+def source_hash(*names):
+    h = hashlib.sha256()
+    for n in names:
+        with open(os.path.join(ROOT, "bit_nf4_quantized_02_b200", "csrc", n), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+# --------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_indices):
+        self.gpus = gpu_indices
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except OSError:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.t.join(timeout=5)
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                idx = int(parts[0])
+            except ValueError:
+                continue
+            if self.gpus and idx not in self.gpus:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# --------------------------------------------------------------------------- our arm
+class Linear:
+    def __init__(self, lin, X, dev, seed):
+        M, r = WL.M, WL.r
+        self.lin = lin
+        N, K = lin.n_out, lin.k_in
+        self.W = inputs.device_normal((N, K), inputs.WEIGHT_STD, seed, dev)
+        self.L1 = inputs.device_normal((K, r), 1.0 / np.sqrt(K), seed + 1, dev, torch.bfloat16)
+        self.L2 = inputs.device_normal((r, N), inputs.L2_STD, seed + 2, dev, torch.bfloat16)
+        self.X = X
+        self.dY = inputs.device_normal((M, N), 1.0, seed + 3, dev, torch.bfloat16)
+        self.Y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+        self.T = torch.empty(M, 2 * r, dtype=torch.bfloat16, device=dev)
+        self.dX = torch.empty(M, K, dtype=torch.bfloat16, device=dev)
+        self.q = None
+
+
+def build_layer(dev, rank):
+    M = WL.M
+    base = WL.seed + 1000 * rank
+    H = inputs.device_normal((M, 4096), 1.0, base + 11, dev, torch.bfloat16)      # q, k, v, gate, up
+    A = inputs.device_normal((M, 4096), 1.0, base + 12, dev, torch.bfloat16)      # o
+    U = inputs.device_normal((M, 11008), 1.0, base + 13, dev, torch.bfloat16)     # down
+    xs = {"q": H, "k": H, "v": H, "o": A, "gate": H, "up": H, "down": U}
+    lins = [Linear(l, xs[l.name], dev, WL.seed + 100 * i) for i, l in enumerate(WL.linears)]
+    # adapter gradients as views of one flat fp32 buffer (one all-reduce per step)
+    sizes = [l.lin.k_in * WL.r + WL.r * l.lin.n_out for l in lins]
+    flat = torch.zeros(sum(sizes), dtype=torch.float32, device=dev)
+    off = 0
+    for l in lins:
+        K, N, r = l.lin.k_in, l.lin.n_out, WL.r
+        l.dL1 = flat[off:off + K * r].view(K, r)
+        l.dL2 = flat[off + K * r:off + K * r + r * N].view(r, N)
+        off += K * r + r * N
+    return lins, flat, (H, A, U)
+
+
+def make_step(qlora, lins, flat, world):
+    def step():
+        for l in lins:
+            l.q = qlora.quantize_nf4_dq(l.W, out=l.q)
+        for l in lins:
+            qlora.linear_fwd(l.X, l.q, l.L1, l.L2, WL.s, Y=l.Y, T=l.T)
+        for l in reversed(lins):
+            qlora.linear_bwd(l.dY, l.X, l.T, l.q, l.L1, l.L2, WL.s, grad_dtype=torch.float32,
+                             dX=l.dX, dL1=l.dL1, dL2=l.dL2)
+        if world > 1:
+            torch.distributed.all_reduce(flat)
+    return step
+
+
+def run_ours(args, rank, world, local_rank):
+    import bit_nf4_quantized_02_b200 as qlora
+    from bit_nf4_quantized_02_b200 import _lib
+
+    _lib.load()
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    lins, flat, acts = build_layer(dev, rank)
+    for l in lins:  # allocate the quantized buffers once
+        l.q = qlora.quantize_nf4_dq(l.W)
+    step = make_step(qlora, lins, flat, world)
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if qlora.last_device_error() != 0:
+        raise RuntimeError("device error during warm-up")
+
+    sampler = ClockSampler(list(range(world)) if world > 1 else [local_rank]) if rank == 0 else None
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    if sampler:
+        sampler.start()
+        time.sleep(0.5)
+    qlora.profile_start(args.steps * 200 + 64)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        step()
+    e1.record()
+    torch.cuda.synchronize()
+    launches = qlora.profile_stop()
+    if world > 1:
+        torch.distributed.barrier()
+    clocks = sampler.stop() if sampler else None
+    ms = e0.elapsed_time(e1) / args.steps
+    t = torch.tensor([ms], device=dev)
+    if world > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    ms = float(t.item())
+    if qlora.last_device_error() != 0:
+        raise RuntimeError("device error during the timed region")
+
+    # ---------------- end to end: host inputs in, adapter gradients out
+    pinned_in = [torch.empty(a.shape, dtype=a.dtype, pin_memory=True) for a in acts]
+    pinned_dy = [torch.empty(l.dY.shape, dtype=l.dY.dtype, pin_memory=True) for l in lins]
+    for h, a in zip(pinned_in, acts):
+        h.copy_(a)
+    for h, l in zip(pinned_dy, lins):
+        h.copy_(l.dY)
+    grads_host = torch.empty(flat.shape, dtype=flat.dtype, pin_memory=True)
+    h2d = sum(t.numel() * t.element_size() for t in pinned_in + pinned_dy)
+    d2h = grads_host.numel() * grads_host.element_size()
+
+    def e2e_step():
+        for h, a in zip(pinned_in, acts):
+            a.copy_(h, non_blocking=True)
+        for h, l in zip(pinned_dy, lins):
+            l.dY.copy_(h, non_blocking=True)
+        step()
+        grads_host.copy_(flat, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    e0.record()
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record()
+    torch.cuda.synchronize()
+    ms_e2e = e0.elapsed_time(e1) / args.steps
+    t = torch.tensor([ms_e2e], device=dev)
+    if world > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    ms_e2e = float(t.item())
+
+    if rank != 0:
+        return None
+    flops = step_flops() * world
+    value = flops / (ms * 1e-3) / 1e12
+    peaks, peak_src = load_peaks()
+    # dominant kernel: the tcgen05 GEMM launches of the Y and dX products
+    per_kind = {}
+    for kind, kms in launches:
+        c = per_kind.setdefault(kind, [0, 0.0])
+        c[0] += 1
+        c[1] += kms
+    dom_ms = per_kind.get("gemm_Y", [0, 0.0])[1] + per_kind.get("gemm_dX", [0, 0.0])[1]
+    dom_n = per_kind.get("gemm_Y", [0, 0.0])[0] + per_kind.get("gemm_dX", [0, 0.0])[0]
+    dom_flops = args.steps * sum(linear_flops(WL.M, l.n_out, l.k_in, WL.r)["gemm_Y"] +
+                                 linear_flops(WL.M, l.n_out, l.k_in, WL.r)["gemm_dX"] for l in WL.linears)
+    achieved = dom_flops / (dom_ms * 1e-3) / 1e12 if dom_ms > 0 else None
+    peak = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+    traffic = None
+    tp = os.path.join(ROOT, "profiles", "tc_gemm_traffic.json")
+    if os.path.exists(tp):
+        with open(tp) as f:
+            tr = json.load(f)
+        if tr.get("source_hash") == source_hash("tc_gemm.cuh", "common.cuh"):
+            traffic = tr.get("bytes_per_launch")
+    total_kernel_ms = sum(v[1] for v in per_kind.values())
+    kernels = {k: {"launches_per_step": v[0] / args.steps, "ms_per_step": v[1] / args.steps,
+                   "share": v[1] / total_kernel_ms if total_kernel_ms else None}
+               for k, v in sorted(per_kind.items(), key=lambda kv: -kv[1][1])}
+    out = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": WL.name, "model": "llama7b-layer-linears", "global_batch": 16 * world,
+                   "seq_len": 512, "tokens_per_rank": WL.M, "lora_r": WL.r, "lora_alpha": WL.alpha,
+                   "parallelism": f"dp{world}" if world > 1 else "single",
+                   "step": "quantize 7 fp32 weights to NF4+DQ, fwd + bwd of the 7 QLoRA linears"
+                           + (", all-reduce of adapter grads" if world > 1 else ""),
+                   "l2": "inputs larger than L2 (>1 GB touched per step), no flush"},
+        "e2e": {"value": flops / (ms_e2e * 1e-3) / 1e12, "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "gpu_launches": len(launches),
+        "roofline": {"bound": "tensor", "kernel": "tc_gemm (Y = X W^T + T L2 and dX = dY W + G L1^T)",
+                     "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                     "frac": achieved / peak if achieved else None, "traffic": traffic,
+                     "peak_source": f"{peak_src} bf16_tflops_sustained",
+                     "launches_timed": dom_n, "avg_launch_ms": dom_ms / dom_n if dom_n else None},
+        "kernels": kernels,
+        "clocks": clocks,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline()
+    return out
+
+
+# --------------------------------------------------------------------------- oracle timing
+SAMPLE_SLICE = 64   # the CPU sample is 1/64 of a step: 128 of the 8192 tokens, 1/64 of each weight's rows
+
+
+def _oracle_sample_setup():
+    g = inputs.rng(WL.seed + 7)
+    Ms = WL.M // SAMPLE_SLICE
+    data = []
+    for lin in WL.linears:
+        N, K = lin.n_out, lin.k_in
+        rows = N // SAMPLE_SLICE
+        data.append({
+            "W_rows": inputs.weight_f32(g, rows, K),
+            # a seeded stand-in for the dequantized weight (the oracle's cost does not depend on values)
+            "W_hat": inputs.normal_bf16(g, (N, K), 0.02).float().numpy(),
+            "X": inputs.normal_bf16(g, (Ms, K)).float().numpy(),
+            "dY": inputs.normal_bf16(g, (Ms, N)).float().numpy(),
+            "L1": inputs.normal_bf16(g, (K, WL.r), 1 / np.sqrt(K)).float().numpy(),
+            "L2": inputs.normal_bf16(g, (WL.r, N), 0.01).float().numpy(),
+        })
+    return data
+
+
+def _oracle_sample_step(data):
+    from oracle import nf4dq, qlora_linear
+    for d in data:
+        nf4dq.quantize_nf4_dq(d["W_rows"])
+        qlora_linear.forward(d["X"], d["W_hat"], d["L1"], d["L2"], WL.s)
+    for d in reversed(data):
+        qlora_linear.backward(d["dY"], d["X"], d["W_hat"], d["L1"], d["L2"], WL.s)
+
+
+def _cores():
+    try:
+        from threadpoolctl import threadpool_info
+        n = max((i.get("num_threads", 1) for i in threadpool_info()), default=1)
+        return int(n)
+    except Exception:
+        return os.cpu_count() or 1
+
+
+SAMPLE_DESC = (f"1/{SAMPLE_SLICE} of a step: NF4+DQ of 1/{SAMPLE_SLICE} of each weight's rows and fp64 fwd+bwd "
+               f"of the 7 linears at {WL.M // SAMPLE_SLICE} of {WL.M} tokens; full-step time = {SAMPLE_SLICE} x sample")
+
+
+def cpu_baseline(reps=1):
+    data = _oracle_sample_setup()
+    t0 = time.perf_counter()
+    for _ in range(reps):
+        _oracle_sample_step(data)
+    dt = (time.perf_counter() - t0) / reps
+    step_s = dt * SAMPLE_SLICE
+    return {"value": step_flops() / step_s / 1e12, "unit": UNIT, "cores": _cores(), "kind": "oracle",
+            "sample": SAMPLE_DESC, "sample_seconds": dt}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return None
+    data = _oracle_sample_setup()
+    for _ in range(args.warmup):
+        _oracle_sample_step(data)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        _oracle_sample_step(data)
+    dt = (time.perf_counter() - t0) / args.steps
+    step_s = dt * SAMPLE_SLICE
+    value = step_flops() / step_s / 1e12
+    cores = _cores()
+    return {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_s * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": WL.name, "model": "llama7b-layer-linears", "global_batch": 16, "seq_len": 512,
+                   "lora_r": WL.r, "lora_alpha": WL.alpha, "parallelism": "single (rank 0 only)"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": SAMPLE_DESC},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        args.warmup = 3
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        out = run_reference(args, rank, world)
+    else:
+        if world > 1:
+            torch.cuda.set_device(local_rank)
+            torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                                 device_id=torch.device("cuda", local_rank))
+        try:
+            out = run_ours(args, rank, world, local_rank)
+        finally:
+            if world > 1:
+                torch.distributed.destroy_process_group()
+    if out is not None and rank == 0:
+        print(json.dumps(out), flush=True)
+
+
+if __name__ == "__main__":
+    main()

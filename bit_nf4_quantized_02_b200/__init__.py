@@ -28,6 +28,9 @@ __all__ = [
     "linear_fwd",
     "linear_bwd",
     "last_device_error",
+    "t_value",
+    "profile_start",
+    "profile_stop",
     "QLoRAError",
 ]
 
@@ -155,7 +158,8 @@ def linear_fwd(X: torch.Tensor, q: NF4Tensor, L1: torch.Tensor, L2: torch.Tensor
                save_T: bool = True, Y: torch.Tensor | None = None, T: torch.Tensor | None = None):
     """Y = X doubleDequant(W)^T + s X L1 L2 (Eq. 3 / Eq. 5).  Returns (Y, T or None).
 
-    X [M, K] bf16, L1 [K, r] bf16, L2 [r, N] bf16; T = s X L1 [M, r] bf16.
+    X [M, K] bf16, L1 [K, r] bf16, L2 [r, N] bf16.  T [M, 2r] bf16 holds
+    T = s X L1 as a hi/lo pair: T ~= T[:, :r] + T[:, r:] (see ``t_value``).
     """
     lib = _lib.load()
     M, K = X.shape
@@ -167,13 +171,19 @@ def linear_fwd(X: torch.Tensor, q: NF4Tensor, L1: torch.Tensor, L2: torch.Tensor
     if Y is None:
         Y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
     if save_T and T is None:
-        T = torch.empty((M, r), dtype=torch.bfloat16, device=dev)
+        T = torch.empty((M, 2 * r), dtype=torch.bfloat16, device=dev)
     ws_bytes = lib.qlora_linear_fwd_workspace_size(M, N, K, r)
     ws = _WS.get(ws_bytes, dev)
     _lib.check(lib.qlora_linear_fwd(_ptr(_bits(X)), M, q.as_struct(), _ptr(_bits(L1)), _ptr(_bits(L2)), r, float(s),
                                     _ptr(_bits(Y)), _ptr(T) if save_T else None, _ptr(ws), ws.numel(),
                                     _stream(dev)), "qlora_linear_fwd")
     return Y, (T if save_T else None)
+
+
+def t_value(T: torch.Tensor) -> torch.Tensor:
+    """The fp32 value of a hi/lo pair T [M, 2r] saved by ``linear_fwd``."""
+    r = T.shape[1] // 2
+    return T[:, :r].float() + T[:, r:].float()
 
 
 def linear_bwd(dY: torch.Tensor, X: torch.Tensor, T: torch.Tensor | None, q: NF4Tensor, L1: torch.Tensor,
@@ -205,6 +215,27 @@ def linear_bwd(dY: torch.Tensor, X: torch.Tensor, T: torch.Tensor | None, q: NF4
                                     _ptr(_bits(L2)), r, float(s), _ptr(dX) if need_dX else None, _ptr(dL1),
                                     _ptr(dL2), gdt, _ptr(ws), ws.numel(), _stream(dev)), "qlora_linear_bwd")
     return (dX if need_dX else None), dL1, dL2
+
+
+def profile_start(capacity: int = 4096) -> None:
+    """Start logging the library's kernel launches with CUDA events (diagnostics)."""
+    _lib.check(_lib.load().qlora_profile_start(capacity), "qlora_profile_start")
+
+
+def profile_stop() -> list:
+    """Stop logging; returns [(kernel kind name, milliseconds), ...] in launch order.
+
+    Waits for the logged launches to finish.
+    """
+    import ctypes
+    lib = _lib.load()
+    n = lib.qlora_profile_stop()
+    out = []
+    kind, ms = ctypes.c_int(), ctypes.c_float()
+    for i in range(n):
+        _lib.check(lib.qlora_profile_read(i, ctypes.byref(kind), ctypes.byref(ms)), "qlora_profile_read")
+        out.append((_lib.KERNEL_KINDS.get(kind.value, str(kind.value)), ms.value))
+    return out
 
 
 def last_device_error(device=None) -> int:

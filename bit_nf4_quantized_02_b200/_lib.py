@@ -24,6 +24,12 @@ QLORA_DTYPE_F32 = 0
 QLORA_DTYPE_BF16 = 1
 QLORA_MAX_RANK = 256
 
+KERNEL_KINDS = {
+    1: "quantize", 2: "dq_constants", 3: "dequant",
+    10: "gemm_T", 11: "gemm_Y", 12: "gemm_G", 13: "gemm_dX", 14: "gemm_dL2", 15: "gemm_dL1",
+    20: "splitk_finalize", 30: "gemv_fwd",
+}
+
 
 class NF4DQ(ctypes.Structure):
     """Mirror of qlora_nf4dq_t."""
@@ -41,6 +47,9 @@ class NF4DQ(ctypes.Structure):
 # name -> (restype, argtypes)
 SIGNATURES = {
     "qlora_version": (c_int, []),
+    "qlora_profile_start": (c_int, [c_int]),
+    "qlora_profile_stop": (c_int, []),
+    "qlora_profile_read": (c_int, [c_int, POINTER(c_int), POINTER(c_float)]),
     "qlora_status_str": (ctypes.c_char_p, [c_int]),
     "qlora_get_last_device_error": (c_int, [c_void_p]),
     "qlora_quantize_workspace_size": (c_size_t, [c_int64]),

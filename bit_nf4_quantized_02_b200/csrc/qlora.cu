@@ -45,6 +45,36 @@ int current_device_info(DeviceInfo **out) {
   return QLORA_OK;
 }
 
+// ---------------------------------------------------------------- event log
+// Opt-in timing of the library's own kernel launches: while enabled, every
+// launch is bracketed by a pair of CUDA events recorded on its stream.
+struct ProfLog {
+  bool on = false;
+  int used = 0;
+  int cap = 0;
+  int dev = -1;
+  cudaEvent_t *ev = nullptr;  // 2 * cap events
+  int *kind = nullptr;        // cap
+};
+ProfLog g_prof;
+std::mutex g_prof_mu;
+
+struct ProfScope {
+  int slot = -1;
+  cudaStream_t st;
+  ProfScope(int kind, cudaStream_t s) : st(s) {
+    if (!g_prof.on) return;
+    std::lock_guard<std::mutex> lock(g_prof_mu);
+    if (!g_prof.on || g_prof.used >= g_prof.cap) return;
+    slot = g_prof.used++;
+    g_prof.kind[slot] = kind;
+    cudaEventRecord(g_prof.ev[2 * slot], st);
+  }
+  ~ProfScope() {
+    if (slot >= 0) cudaEventRecord(g_prof.ev[2 * slot + 1], st);
+  }
+};
+
 bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 
 size_t align_up(size_t x, size_t a = 256) { return (x + a - 1) / a * a; }
@@ -110,7 +140,7 @@ int pick_bn(int64_t N) { return N <= 64 ? 64 : (N <= 128 ? 128 : 256); }
 // Split-K factor for a single-segment product whose tile grid leaves SMs idle.
 void choose_splits(int64_t tiles, int64_t nkb, int sms, bool allow, int *splits, int *kbps) {
   int s = 1;
-  if (allow && tiles < sms && nkb > 1) {
+  if (allow && tiles > 0 && tiles < sms && nkb > 1) {
     s = (int)std::min<int64_t>(nkb, (2 * (int64_t)sms + tiles - 1) / tiles);
   }
   int k = (int)((nkb + s - 1) / s);
@@ -121,6 +151,7 @@ void choose_splits(int64_t tiles, int64_t nkb, int sms, bool allow, int *splits,
 }
 
 size_t gemm_split_ws_bytes(int64_t M, int64_t N, int64_t K, int sms, bool allow) {
+  if (M <= 0 || N <= 0 || K <= 0) return 0;
   const int bn = pick_bn(N);
   const int64_t tiles = ((M + kBM - 1) / kBM) * ((N + bn - 1) / bn);
   int splits, kbps;
@@ -129,7 +160,7 @@ size_t gemm_split_ws_bytes(int64_t M, int64_t N, int64_t K, int sms, bool allow)
 }
 
 template <int BN>
-int launch_gemm_bn(const CUtensorMap *maps, TcGemmArgs &args, int sms, DeviceInfo *dev, cudaStream_t st) {
+int launch_gemm_bn(const CUtensorMap *maps, TcGemmArgs &args, int sms, DeviceInfo *dev, cudaStream_t st, int kind) {
   using Cfg = TcCfg<BN>;
   const int idx = BN == 64 ? 0 : (BN == 128 ? 1 : 2);
   if (!dev->gemm_attr[idx]) {
@@ -140,17 +171,19 @@ int launch_gemm_bn(const CUtensorMap *maps, TcGemmArgs &args, int sms, DeviceInf
   }
   const int units = args.m_tiles * args.n_tiles * args.splits;
   const int grid = std::max(1, std::min(units, sms));
+  ProfScope prof(kind, st);
   tc_gemm_kernel<BN><<<grid, kGemmThreads, Cfg::kSmemBytes, st>>>(maps[0], maps[1], maps[2], maps[3], args);
   return launch_status();
 }
 
 // D[M x N] = alpha * sum_seg A_seg B_seg^T, written to `out` with strides
-// (ld_row, ld_col) as bf16 or fp32.  If `split_ws` is given and the tile grid
-// is small, segment 0's reduction is split and the fp32 partials (dense, in
-// the output's strides) are summed by a finalize pass; the output must then be
-// dense: ld_row * ld_col products cover M*N elements exactly.
+// (ld_row, ld_col) as bf16 (optionally with a lo part at +lo_off) or fp32.
+// If `split_ws` is given and the tile grid leaves SMs idle, the reduction is
+// split (segment 0 only, or every segment when `split_all`), the fp32
+// partials go to split_ws and a finalize pass sums them in a fixed order.
 int tc_gemm(cudaStream_t st, DeviceInfo *dev, int64_t M, int64_t N, int nseg, const GemmSeg *segs, float alpha,
-            void *out, int64_t ld_row, int64_t ld_col, int out_f32, float *split_ws) {
+            void *out, int64_t ld_row, int64_t ld_col, int out_f32, float *split_ws, int kind, int64_t lo_off = 0,
+            bool split_all = false) {
   if (M <= 0 || N <= 0) return QLORA_OK;
   if (M > (int64_t)INT32_MAX / 2 || N > (int64_t)INT32_MAX / 2) return QLORA_ERR_UNSUPPORTED_SHAPE;
   const int bn = pick_bn(N);
@@ -173,35 +206,38 @@ int tc_gemm(cudaStream_t st, DeviceInfo *dev, int64_t M, int64_t N, int nseg, co
     if (rc) return rc;
   }
   if (nseg == 1) maps[2] = maps[0], maps[3] = maps[1];
+  if (split_all && (nseg < 2 || a.seg[1].nkb != a.seg[0].nkb)) split_all = false;
   int splits, kbps;
-  choose_splits((int64_t)a.m_tiles * a.n_tiles, a.seg[0].nkb, dev->sms, split_ws != nullptr && nseg == 1, &splits,
-                &kbps);
+  choose_splits((int64_t)a.m_tiles * a.n_tiles, a.seg[0].nkb, dev->sms,
+                split_ws != nullptr && (nseg == 1 || split_all), &splits, &kbps);
   a.splits = splits;
   a.kb_per_split = kbps;
+  a.split_all = split_all ? 1 : 0;
   a.err = dev->err;
   a.ld_row = ld_row;
   a.ld_col = ld_col;
+  a.lo_off = lo_off;
   if (splits > 1) {
     a.alpha = 1.f;
     a.out = split_ws;
     a.out_f32 = 1;
-    a.split_stride = M * N;
   } else {
     a.alpha = alpha;
     a.out = out;
     a.out_f32 = out_f32;
-    a.split_stride = 0;
   }
   int rc;
   switch (bn) {
-    case 64: rc = launch_gemm_bn<64>(maps, a, dev->sms, dev, st); break;
-    case 128: rc = launch_gemm_bn<128>(maps, a, dev->sms, dev, st); break;
-    default: rc = launch_gemm_bn<256>(maps, a, dev->sms, dev, st); break;
+    case 64: rc = launch_gemm_bn<64>(maps, a, dev->sms, dev, st, kind); break;
+    case 128: rc = launch_gemm_bn<128>(maps, a, dev->sms, dev, st, kind); break;
+    default: rc = launch_gemm_bn<256>(maps, a, dev->sms, dev, st, kind); break;
   }
   if (rc || splits == 1) return rc;
   const int64_t count = M * N;
   const int grid = (int)std::min<int64_t>((count + 255) / 256, (int64_t)dev->sms * 8);
-  splitk_finalize_kernel<<<grid, 256, 0, st>>>(split_ws, splits, M * N, count, alpha, out, out_f32);
+  ProfScope prof(QLORA_KERNEL_SPLITK_FINALIZE, st);
+  splitk_finalize_kernel<<<grid, 256, 0, st>>>(split_ws, splits, (int)M, (int)N, alpha, out, ld_row, ld_col, lo_off,
+                                               out_f32);
   return launch_status();
 }
 
@@ -210,6 +246,7 @@ int dequant_launch(const qlora_nf4dq_t *W, __nv_bfloat16 *out, cudaStream_t st, 
   if (numel == 0) return QLORA_OK;
   const int64_t n8 = numel >> 3;
   const int grid = (int)std::max<int64_t>(1, std::min<int64_t>((n8 + 255) / 256, (int64_t)sms * 16));
+  ProfScope prof(QLORA_KERNEL_DEQUANT, st);
   nf4_dequant_kernel<<<grid, 256, 0, st>>>(W->codes, W->c2_fp8, W->c1, W->c2_mean, numel, out);
   return launch_status();
 }
@@ -242,7 +279,7 @@ FwdLayout fwd_layout(int64_t M, int64_t N, int64_t K, int r, int sms) {
   FwdLayout L;
   L.w_hat = 0;
   L.t = align_up((size_t)N * K * 2);
-  L.split = L.t + align_up((size_t)M * r * 2);
+  L.split = L.t + align_up((size_t)M * 2 * r * 2);
   L.total = L.split + gemm_split_ws_bytes(M, r, K, sms, true);
   return L;
 }
@@ -255,8 +292,8 @@ BwdLayout bwd_layout(int64_t M, int64_t N, int64_t K, int r, int sms) {
   BwdLayout L;
   L.w_hat = 0;
   L.g = align_up((size_t)N * K * 2);
-  L.t = L.g + align_up((size_t)M * r * 2);
-  L.split = L.t + align_up((size_t)M * r * 2);
+  L.t = L.g + align_up((size_t)M * 2 * r * 2);
+  L.split = L.t + align_up((size_t)M * 2 * r * 2);
   size_t sw = 0;
   sw = std::max(sw, gemm_split_ws_bytes(M, r, K, sms, true));   // T = s X L1
   sw = std::max(sw, gemm_split_ws_bytes(M, r, N, sms, true));   // G = s dY L2^T
@@ -274,6 +311,50 @@ using namespace qlora;
 extern "C" {
 
 int qlora_version(void) { return 100; }
+
+int qlora_profile_start(int capacity) {
+  if (capacity <= 0 || capacity > (1 << 20)) return QLORA_ERR_INVALID_ARG;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return QLORA_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_prof_mu);
+  if (g_prof.cap < capacity || g_prof.dev != dev) {
+    if (g_prof.ev) {
+      int cur = 0;
+      cudaGetDevice(&cur);
+      cudaSetDevice(g_prof.dev);
+      for (int i = 0; i < 2 * g_prof.cap; ++i) cudaEventDestroy(g_prof.ev[i]);
+      cudaSetDevice(cur);
+      delete[] g_prof.ev;
+      delete[] g_prof.kind;
+      g_prof.ev = nullptr;
+      g_prof.kind = nullptr;
+      g_prof.cap = 0;
+    }
+    g_prof.ev = new cudaEvent_t[2 * capacity];
+    g_prof.kind = new int[capacity];
+    for (int i = 0; i < 2 * capacity; ++i)
+      if (cudaEventCreate(&g_prof.ev[i]) != cudaSuccess) return QLORA_ERR_CUDA;
+    g_prof.cap = capacity;
+    g_prof.dev = dev;
+  }
+  g_prof.used = 0;
+  g_prof.on = true;
+  return QLORA_OK;
+}
+
+int qlora_profile_stop(void) {
+  std::lock_guard<std::mutex> lock(g_prof_mu);
+  g_prof.on = false;
+  return g_prof.used;
+}
+
+int qlora_profile_read(int i, int *kind, float *ms) {
+  std::lock_guard<std::mutex> lock(g_prof_mu);
+  if (i < 0 || i >= g_prof.used || !kind || !ms) return QLORA_ERR_INVALID_ARG;
+  *kind = g_prof.kind[i];
+  if (cudaEventSynchronize(g_prof.ev[2 * i + 1]) != cudaSuccess) return QLORA_ERR_CUDA;
+  return cudaEventElapsedTime(ms, g_prof.ev[2 * i], g_prof.ev[2 * i + 1]) == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+}
 
 const char *qlora_status_str(int status) {
   switch (status) {
@@ -332,16 +413,20 @@ int qlora_quantize_nf4_dq(const void *W, int w_dtype, int64_t n_out, int64_t k_i
   double *partial = reinterpret_cast<double *>(reinterpret_cast<uint8_t *>(ws) + align_up((size_t)nblk * 4));
   const int64_t ngroups = numel >> 8;
   const int grid1 = (int)std::max<int64_t>(1, std::min<int64_t>((ngroups + 7) / 8, kQuantMaxCtas));
+  {
+  ProfScope prof(QLORA_KERNEL_QUANTIZE, st);
   if (w_dtype == QLORA_DTYPE_F32)
     nf4_quantize_kernel<float><<<grid1, kQuantThreads, 0, st>>>(reinterpret_cast<const float *>(W), numel, codes, c2,
                                                                partial);
   else
     nf4_quantize_kernel<__nv_bfloat16><<<grid1, kQuantThreads, 0, st>>>(
         reinterpret_cast<const __nv_bfloat16 *>(W), numel, codes, c2, partial);
+  }
   rc = launch_status();
   if (rc) return rc;
   const int64_t nb256 = (nblk + 255) / 256;
   const int grid2 = (int)std::max<int64_t>(1, std::min<int64_t>(nb256, (int64_t)dev->sms * 4));
+  ProfScope prof(QLORA_KERNEL_DQ_CONSTANTS, st);
   dq_constants_kernel<<<grid2, 256, 0, st>>>(c2, nblk, partial, grid1, c2_fp8, c1, c2_mean);
   return launch_status();
 }
@@ -398,13 +483,14 @@ int qlora_linear_fwd(const uint16_t *X, int64_t M, const qlora_nf4dq_t *W, const
   // 1. doubleDequant of the frozen weight into the bf16 workspace (Eq. 6).
   rc = dequant_launch(W, w_hat, st, dev->sms);
   if (rc) return rc;
-  // 2. T = s X L1 (the adapter's down-projection; L1 read MN-major).
+  // 2. T = s X L1 (the adapter's down-projection; L1 read MN-major), stored
+  //    as a bf16 hi/lo pair [M x 2r]: T ~= T[:, :r] + T[:, r:].
   GemmSeg sT = {{X, M, K, K, 0}, {L1, r, K, r, 1}};
-  rc = tc_gemm(st, dev, M, r, 1, &sT, s, T, r, 1, 0, split_ws);
+  rc = tc_gemm(st, dev, M, r, 1, &sT, s, T, 2 * r, 1, 0, split_ws, QLORA_KERNEL_GEMM_T, r);
   if (rc) return rc;
-  // 3. Y = X W_hat^T + T L2 (the LoRA up-projection as extra K-steps).
-  GemmSeg sY[2] = {{{X, M, K, K, 0}, {w_hat, N, K, K, 0}}, {{T, M, r, r, 0}, {L2, N, r, N, 1}}};
-  return tc_gemm(st, dev, M, N, 2, sY, 1.f, Y, N, 1, 0, nullptr);
+  // 3. Y = X W_hat^T + T_hi L2 (the LoRA up-projection as extra K-steps).
+  GemmSeg sY[2] = {{{X, M, K, K, 0}, {w_hat, N, K, K, 0}}, {{T, M, r, 2 * r, 0}, {L2, N, r, N, 1}}};
+  return tc_gemm(st, dev, M, N, 2, sY, 1.f, Y, N, 1, 0, nullptr, QLORA_KERNEL_GEMM_Y);
 }
 
 int qlora_linear_bwd(const uint16_t *dY, const uint16_t *X, const uint16_t *T_saved, int64_t M,
@@ -439,32 +525,35 @@ int qlora_linear_bwd(const uint16_t *dY, const uint16_t *X, const uint16_t *T_sa
   const uint16_t *T = T_saved;
   const int out_f32 = grad_dtype == QLORA_DTYPE_F32;
 
-  if (!T) {  // recompute T = s X L1
+  if (!T) {  // recompute T = s X L1 (hi/lo pair)
     uint16_t *Tw = reinterpret_cast<uint16_t *>(w8 + L.t);
     GemmSeg sT = {{X, M, K, K, 0}, {L1, r, K, r, 1}};
-    rc = tc_gemm(st, dev, M, r, 1, &sT, s, Tw, r, 1, 0, split_ws);
+    rc = tc_gemm(st, dev, M, r, 1, &sT, s, Tw, 2 * r, 1, 0, split_ws, QLORA_KERNEL_GEMM_T, r);
     if (rc) return rc;
     T = Tw;
   }
-  // G = s dY L2^T  (L2 [r x N] is K-major for this product).
+  // G = s dY L2^T (L2 [r x N] is K-major for this product), as a hi/lo pair.
   GemmSeg sG = {{dY, M, N, N, 0}, {L2, r, N, N, 0}};
-  rc = tc_gemm(st, dev, M, r, 1, &sG, s, G, r, 1, 0, split_ws);
+  rc = tc_gemm(st, dev, M, r, 1, &sG, s, G, 2 * r, 1, 0, split_ws, QLORA_KERNEL_GEMM_G, r);
   if (rc) return rc;
   if (dX) {
-    // dX = dY W_hat + G L1^T: W_hat [N x K] is read in place as an MN-major B.
+    // dX = dY W_hat + G_hi L1^T: W_hat [N x K] is read in place as an MN-major B.
     rc = dequant_launch(W, w_hat, st, dev->sms);
     if (rc) return rc;
-    GemmSeg sX[2] = {{{dY, M, N, N, 0}, {w_hat, K, N, K, 1}}, {{G, M, r, r, 0}, {L1, K, r, r, 0}}};
-    rc = tc_gemm(st, dev, M, K, 2, sX, 1.f, dX, K, 1, 0, nullptr);
+    GemmSeg sX[2] = {{{dY, M, N, N, 0}, {w_hat, K, N, K, 1}}, {{G, M, r, 2 * r, 0}, {L1, K, r, r, 0}}};
+    rc = tc_gemm(st, dev, M, K, 2, sX, 1.f, dX, K, 1, 0, nullptr, QLORA_KERNEL_GEMM_DX);
     if (rc) return rc;
   }
-  // dL2 = T^T dY, computed as dL2^T [N x r] = dY^T T with a transposed store.
-  GemmSeg s2 = {{dY, N, M, N, 1}, {T, r, M, r, 1}};
-  rc = tc_gemm(st, dev, N, r, 1, &s2, 1.f, dL2, 1, N, out_f32, split_ws);
+  // dL2 = T^T dY as dL2^T [N x r] = dY^T (T_hi + T_lo): two accumulated
+  // segments over the tokens, written transposed.
+  const uint16_t *T_lo = T + r;
+  GemmSeg s2[2] = {{{dY, N, M, N, 1}, {T, r, M, 2 * r, 1}}, {{dY, N, M, N, 1}, {T_lo, r, M, 2 * r, 1}}};
+  rc = tc_gemm(st, dev, N, r, 2, s2, 1.f, dL2, 1, N, out_f32, split_ws, QLORA_KERNEL_GEMM_DL2, 0, true);
   if (rc) return rc;
-  // dL1 = X^T G [K x r].
-  GemmSeg s1 = {{X, K, M, K, 1}, {G, r, M, r, 1}};
-  return tc_gemm(st, dev, K, r, 1, &s1, 1.f, dL1, r, 1, out_f32, split_ws);
+  // dL1 = X^T (G_hi + G_lo) [K x r].
+  const uint16_t *G_lo = G + r;
+  GemmSeg s1[2] = {{{X, K, M, K, 1}, {G, r, M, 2 * r, 1}}, {{X, K, M, K, 1}, {G_lo, r, M, 2 * r, 1}}};
+  return tc_gemm(st, dev, K, r, 2, s1, 1.f, dL1, r, 1, out_f32, split_ws, QLORA_KERNEL_GEMM_DL1, 0, true);
 }
 
 }  // extern "C"

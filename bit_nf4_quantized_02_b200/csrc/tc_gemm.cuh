@@ -13,8 +13,11 @@
 // reduction; MN-major = contiguous along the output rows/columns), selected
 // per MMA through the instruction descriptor, so X*W^T, dY*W (W read in its
 // stored layout), X^T*G and the LoRA extra K-steps all run on this engine.
-// A segment-0 split of the reduction (split-K) writes fp32 partials that a
-// finalize kernel sums in a fixed order.
+// A split of the reduction (split-K; of segment 0, or of every segment when
+// they have equal lengths) writes fp32 partials that a finalize kernel sums
+// in a fixed order.  A bf16 output can also be stored as a hi/lo pair
+// (hi = bf16(v), lo = bf16(v - hi)) so that a later product can consume it
+// at nearly fp32 accuracy as two bf16 operands.
 #pragma once
 
 #include "common.cuh"
@@ -35,11 +38,12 @@ struct TcGemmArgs {
   int M, N;
   int m_tiles, n_tiles, splits, kb_per_split;
   int nseg;
+  int split_all;            // split-K applies to every segment (equal k-block counts)
   TcSeg seg[2];
   float alpha;
   void *out;
-  int64_t ld_row, ld_col;   // element strides of D(i, j) in `out`
-  int64_t split_stride;     // elements between split-K partial outputs
+  int64_t ld_row, ld_col;   // element strides of D(i, j) in `out` (unsplit output)
+  int64_t lo_off;           // bf16 output only: if > 0 also store lo = bf16(v - hi) at +lo_off
   int out_f32;              // 1: fp32 output, 0: bf16
   int *err;
 };
@@ -70,9 +74,9 @@ __device__ __forceinline__ void tc_unit_coords(int u, const TcGemmArgs &p, int &
 }
 
 __device__ __forceinline__ void tc_seg_range(const TcGemmArgs &p, int s, int split, int &kb0, int &kb1) {
-  if (s == 0) {
+  if (s == 0 || p.split_all) {
     kb0 = split * p.kb_per_split;
-    kb1 = min(p.seg[0].nkb, kb0 + p.kb_per_split);
+    kb1 = min(p.seg[s].nkb, kb0 + p.kb_per_split);
   } else {
     kb0 = 0;
     kb1 = split == 0 ? p.seg[1].nkb : 0;
@@ -243,7 +247,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       tc_unit_coords(u, p, mt, nt, split);
       const int acc = t & 1;
       const uint32_t use = (uint32_t)(t >> 1);
-      if (!mbar_wait(smem_u32(tfull_bar + acc), use & 1u, p.err, DEV_TIMEOUT_EPILOGUE)) break;
+      // Warp-uniform wait: tcgen05.ld below must be executed by all 32 lanes.
+      const bool got = mbar_wait(smem_u32(tfull_bar + acc), use & 1u, p.err, DEV_TIMEOUT_EPILOGUE);
+      if (!__all_sync(0xFFFFFFFFu, got)) break;
       tc_fence_after();
       const int row = mt * kBM + q * 32 + lane;
       const bool row_ok = row < p.M;
@@ -255,9 +261,22 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         tmem_wait_ld();
         const int col0 = nt * BN + c;
         if (!row_ok || col0 >= p.N) continue;
-        if (p.out_f32) {
-          float *o = reinterpret_cast<float *>(p.out) + (int64_t)split * p.split_stride;
-          if (p.ld_col == 1 && col0 + 32 <= p.N) {
+        if (p.splits > 1) {
+          // split-K partial: dense fp32 [split][M][N], summed by the finalize pass
+          float *o = reinterpret_cast<float *>(p.out) + ((int64_t)split * p.M + row) * p.N + col0;
+          if (col0 + 32 <= p.N && (p.N & 3) == 0) {
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+              reinterpret_cast<float4 *>(o)[j] = make_float4(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1]),
+                                                             __uint_as_float(r[4 * j + 2]), __uint_as_float(r[4 * j + 3]));
+          } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              if (col0 + j < p.N) o[j] = __uint_as_float(r[j]);
+          }
+        } else if (p.out_f32) {
+          float *o = reinterpret_cast<float *>(p.out);
+          if (p.ld_col == 1 && col0 + 32 <= p.N && (p.ld_row & 3) == 0) {
             float4 *dst = reinterpret_cast<float4 *>(o + (int64_t)row * p.ld_row + col0);
 #pragma unroll
             for (int j = 0; j < 8; ++j)
@@ -270,24 +289,35 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           }
         } else {
           __nv_bfloat16 *o = reinterpret_cast<__nv_bfloat16 *>(p.out);
-          if (p.ld_col == 1 && col0 + 32 <= p.N) {
+          const int64_t lo = p.lo_off;
+          if (p.ld_col == 1 && col0 + 32 <= p.N && (p.ld_row & 7) == 0 && (lo & 7) == 0) {
             uint4 *dst = reinterpret_cast<uint4 *>(o + (int64_t)row * p.ld_row + col0);
+            uint4 *dst_lo = reinterpret_cast<uint4 *>(o + (int64_t)row * p.ld_row + col0 + lo);
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
-              uint32_t w[4];
+              uint32_t w[4], wl[4];
 #pragma unroll
               for (int h = 0; h < 4; ++h) {
-                const __nv_bfloat162 b2 = __floats2bfloat162_rn(alpha * __uint_as_float(r[8 * j + 2 * h]),
-                                                                alpha * __uint_as_float(r[8 * j + 2 * h + 1]));
+                const float v0 = alpha * __uint_as_float(r[8 * j + 2 * h]);
+                const float v1 = alpha * __uint_as_float(r[8 * j + 2 * h + 1]);
+                const __nv_bfloat162 b2 = __floats2bfloat162_rn(v0, v1);
                 w[h] = *reinterpret_cast<const uint32_t *>(&b2);
+                const __nv_bfloat162 l2 = __floats2bfloat162_rn(v0 - __low2float(b2), v1 - __high2float(b2));
+                wl[h] = *reinterpret_cast<const uint32_t *>(&l2);
               }
               dst[j] = make_uint4(w[0], w[1], w[2], w[3]);
+              if (lo > 0) dst_lo[j] = make_uint4(wl[0], wl[1], wl[2], wl[3]);
             }
           } else {
 #pragma unroll
             for (int j = 0; j < 32; ++j)
-              if (col0 + j < p.N)
-                o[(int64_t)row * p.ld_row + (int64_t)(col0 + j) * p.ld_col] = __float2bfloat16_rn(alpha * __uint_as_float(r[j]));
+              if (col0 + j < p.N) {
+                const float v = alpha * __uint_as_float(r[j]);
+                const __nv_bfloat16 hb = __float2bfloat16_rn(v);
+                const int64_t off = (int64_t)row * p.ld_row + (int64_t)(col0 + j) * p.ld_col;
+                o[off] = hb;
+                if (lo > 0) o[off + lo] = __float2bfloat16_rn(v - __bfloat162float(hb));
+              }
           }
         }
       }
@@ -302,18 +332,27 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   if (warp == 1) tmem_dealloc(tmem_base, Cfg::kTmemCols);
 }
 
-// Fixed-order sum of split-K partials: dst[i] = alpha * sum_s part[s * stride + i].
-__global__ void __launch_bounds__(256) splitk_finalize_kernel(const float *__restrict__ part, int splits,
-                                                              int64_t stride, int64_t count, float alpha,
-                                                              void *dst, int dst_f32) {
+// Fixed-order sum of split-K partials (dense fp32 [splits][M][N]) into the
+// output D(i, j) at dst + i*ld_row + j*ld_col, with the same bf16 hi/lo and
+// fp32 options as the GEMM epilogue.
+__global__ void __launch_bounds__(256) splitk_finalize_kernel(const float *__restrict__ part, int splits, int M,
+                                                              int N, float alpha, void *dst, int64_t ld_row,
+                                                              int64_t ld_col, int64_t lo_off, int dst_f32) {
+  const int64_t count = (int64_t)M * N;
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < count; i += (int64_t)gridDim.x * blockDim.x) {
     float s = 0.f;
-    for (int k = 0; k < splits; ++k) s += __ldg(part + (int64_t)k * stride + i);
+    for (int k = 0; k < splits; ++k) s += __ldg(part + (int64_t)k * count + i);
     s *= alpha;
-    if (dst_f32)
-      reinterpret_cast<float *>(dst)[i] = s;
-    else
-      reinterpret_cast<__nv_bfloat16 *>(dst)[i] = __float2bfloat16_rn(s);
+    const int64_t row = i / N, col = i - row * N;
+    const int64_t off = row * ld_row + col * ld_col;
+    if (dst_f32) {
+      reinterpret_cast<float *>(dst)[off] = s;
+    } else {
+      __nv_bfloat16 *o = reinterpret_cast<__nv_bfloat16 *>(dst);
+      const __nv_bfloat16 hb = __float2bfloat16_rn(s);
+      o[off] = hb;
+      if (lo_off > 0) o[off + lo_off] = __float2bfloat16_rn(s - __bfloat162float(hb));
+    }
   }
 }
 

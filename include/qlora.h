@@ -120,9 +120,13 @@ QLORA_API size_t qlora_linear_bwd_workspace_size(int64_t M, int64_t n_out, int64
 /*
  * Forward (§2 Eq. 3 / §3 Eq. 5 with the scale s of Eq. 3):
  *   Y = X doubleDequant(W)^T + T L2,  T = s X L1.
- *   X [M x K] bf16, L1 [K x r] bf16, L2 [r x N] bf16, Y [M x N] bf16 (out),
- *   T_save [M x r] bf16 (out, may be NULL): the adapter down-projection s X L1
- *   as used by the forward, for the backward.
+ *   X [M x K] bf16, L1 [K x r] bf16, L2 [r x N] bf16, Y [M x N] bf16 (out).
+ *   T_save [M x 2r] bf16 (out, may be NULL): the adapter down-projection
+ *   T = s X L1 (fp32 accumulation) kept for the backward as a pair of bf16
+ *   halves, T ~= T_save[:, :r] + T_save[:, r:] (hi = bf16(T),
+ *   lo = bf16(T - hi); relative error about 2^-17).  The forward's up-projection
+ *   uses the hi half; the backward's dL2 = T^T dY uses both, so that the long
+ *   reduction over tokens does not amplify a bf16 rounding of T.
  *   K = W->k_in (multiple of 64), N = W->n_out (multiple of 8), r a multiple of
  *   8 in [8, 256].  All products accumulate in fp32 on the tensor cores.
  */
@@ -132,11 +136,11 @@ QLORA_API int qlora_linear_fwd(const uint16_t *X, int64_t M, const qlora_nf4dq_t
 /*
  * Backward (§3, paragraph after Eq. 6: adapter gradients only, the gradient
  * passing through the weight dequantized to bf16):
- *   G   = s dY L2^T                  [M x r] (internal, bf16)
+ *   G   = s dY L2^T                  [M x r] (internal, bf16 hi/lo pair)
  *   dX  = dY doubleDequant(W) + G L1^T   [M x K] bf16 (out; may be NULL to skip)
  *   dL2 = T^T dY                     [r x N] (out)
  *   dL1 = X^T G                      [K x r] (out)
- *   T_saved [M x r] bf16 from the forward, or NULL to recompute T = s X L1.
+ *   T_saved [M x 2r] bf16 (hi/lo pair) from the forward, or NULL to recompute.
  *   dL1, dL2 are written (not accumulated) as grad_dtype (QLORA_DTYPE_BF16 or
  *   QLORA_DTYPE_F32).  Shape rules as for the forward.
  */
@@ -156,6 +160,31 @@ QLORA_API const char *qlora_status_str(int status);
  * or QLORA_ERR_CUDA if the synchronization itself failed.
  */
 QLORA_API int qlora_get_last_device_error(void *stream);
+
+/*
+ * Kernel timing log (diagnostics).  qlora_profile_start(capacity) enables it
+ * for the current device: each subsequent kernel launch of this library is
+ * bracketed by two CUDA events recorded on the launch's stream, for the first
+ * `capacity` launches (later ones are not logged).  qlora_profile_stop()
+ * disables it and returns the number of logged launches.  qlora_profile_read(i)
+ * then returns launch i's kernel kind (QLORA_KERNEL_*) and its elapsed
+ * milliseconds (waiting for its end event).  The log's events are host-side
+ * CUDA objects created by start(); no device memory is allocated.
+ */
+#define QLORA_KERNEL_QUANTIZE 1
+#define QLORA_KERNEL_DQ_CONSTANTS 2
+#define QLORA_KERNEL_DEQUANT 3
+#define QLORA_KERNEL_GEMM_T 10      /* T = s X L1 */
+#define QLORA_KERNEL_GEMM_Y 11      /* Y = X W_hat^T + T L2 */
+#define QLORA_KERNEL_GEMM_G 12      /* G = s dY L2^T */
+#define QLORA_KERNEL_GEMM_DX 13     /* dX = dY W_hat + G L1^T */
+#define QLORA_KERNEL_GEMM_DL2 14    /* dL2 = T^T dY */
+#define QLORA_KERNEL_GEMM_DL1 15    /* dL1 = X^T G */
+#define QLORA_KERNEL_SPLITK_FINALIZE 20
+#define QLORA_KERNEL_GEMV_FWD 30    /* fused decode + product for few tokens */
+QLORA_API int qlora_profile_start(int capacity);
+QLORA_API int qlora_profile_stop(void);
+QLORA_API int qlora_profile_read(int i, int *kind, float *ms);
 
 /* Library version (major * 10000 + minor * 100 + patch). */
 QLORA_API int qlora_version(void);

@@ -79,6 +79,10 @@ def test_host_argument_validation(lib):
 
 
 def test_workspace_sizes_are_host_only(lib):
+    # degenerate sizes never divide by zero
+    assert lib.qlora_linear_fwd_workspace_size(0, 64, 128, 8) >= 0
+    assert lib.qlora_linear_bwd_workspace_size(0, 64, 128, 8) >= 0
+    assert lib.qlora_linear_fwd_workspace_size(1, 8, 64, 8) > 0
     assert lib.qlora_quantize_workspace_size(1 << 20) >= (1 << 20) // 64 * 4
     assert lib.qlora_linear_fwd_workspace_size(8192, 4096, 4096, 64) >= 4096 * 4096 * 2
     assert lib.qlora_linear_bwd_workspace_size(8192, 4096, 4096, 64) >= 4096 * 4096 * 2 + 2 * 8192 * 64 * 2
