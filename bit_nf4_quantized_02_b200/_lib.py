@@ -19,6 +19,8 @@ QLORA_ERR_UNSUPPORTED_SHAPE = -3
 QLORA_ERR_CUDA = -4
 QLORA_ERR_DEVICE_TIMEOUT = -5
 QLORA_ERR_WORKSPACE = -6
+QLORA_ERR_SCRATCH_LIMIT = -7
+QLORA_NOALLOC_MAX_NUMEL = 1 << 28
 
 QLORA_DTYPE_F32 = 0
 QLORA_DTYPE_BF16 = 1
@@ -55,6 +57,8 @@ SIGNATURES = {
     "qlora_quantize_workspace_size": (c_size_t, [c_int64]),
     "qlora_quantize_nf4_dq": (c_int, [c_void_p, c_int, c_int64, c_int64, c_void_p, c_void_p, c_void_p, c_void_p,
                                       c_void_p, c_size_t, c_void_p]),
+    "qlora_quantize_nf4_dq_noalloc": (c_int, [c_void_p, c_int, c_int64, c_int64, c_void_p, c_void_p, c_void_p,
+                                              c_void_p, c_void_p]),
     "qlora_dequant": (c_int, [POINTER(NF4DQ), c_void_p, c_void_p]),
     "qlora_linear_fwd_workspace_size": (c_size_t, [c_int64, c_int64, c_int64, c_int]),
     "qlora_linear_bwd_workspace_size": (c_size_t, [c_int64, c_int64, c_int64, c_int]),

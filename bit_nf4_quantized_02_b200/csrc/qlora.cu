@@ -304,6 +304,34 @@ BwdLayout bwd_layout(int64_t M, int64_t N, int64_t K, int r, int sms) {
 }
 
 }  // namespace
+
+// ----------------------------------------------------- no-allocation scratch
+// Fixed scratch of qlora_quantize_nf4_dq_noalloc: fp32 block constants for up
+// to 2^22 blocks of 64 (16 MiB), then the fp64 per-CTA partial sums (16 KiB).
+constexpr int64_t kNoallocMaxBlocks = QLORA_NOALLOC_MAX_NUMEL / 64;
+constexpr size_t kNoallocC2Bytes = (size_t)kNoallocMaxBlocks * 4;
+static_assert(kNoallocC2Bytes + (size_t)kQuantMaxCtas * 8 <= QLORA_NOALLOC_SCRATCH_BYTES, "scratch too small");
+static __device__ __align__(256) unsigned char g_noalloc_scratch[QLORA_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+void *g_noalloc_addr[kMaxDevices];
+std::mutex g_noalloc_mu;
+
+// Device address of the static scratch on the current device, looked up once
+// per device with that device current (host code cannot use the symbol itself).
+int noalloc_scratch(unsigned char **out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return QLORA_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_addr[dev]) {
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return QLORA_ERR_CUDA;
+    g_noalloc_addr[dev] = p;
+  }
+  *out = reinterpret_cast<unsigned char *>(g_noalloc_addr[dev]);
+  return QLORA_OK;
+}
+}  // namespace
 }  // namespace qlora
 
 using namespace qlora;
@@ -365,6 +393,7 @@ const char *qlora_status_str(int status) {
     case QLORA_ERR_CUDA: return "CUDA runtime error";
     case QLORA_ERR_DEVICE_TIMEOUT: return "a kernel's bounded wait expired";
     case QLORA_ERR_WORKSPACE: return "workspace missing or too small";
+    case QLORA_ERR_SCRATCH_LIMIT: return "tensor larger than the fixed scratch of the no-allocation entry point";
     default: return "unknown status";
   }
 }
@@ -427,6 +456,43 @@ int qlora_quantize_nf4_dq(const void *W, int w_dtype, int64_t n_out, int64_t k_i
   const int64_t nb256 = (nblk + 255) / 256;
   const int grid2 = (int)std::max<int64_t>(1, std::min<int64_t>(nb256, (int64_t)dev->sms * 4));
   ProfScope prof(QLORA_KERNEL_DQ_CONSTANTS, st);
+  dq_constants_kernel<<<grid2, 256, 0, st>>>(c2, nblk, partial, grid1, c2_fp8, c1, c2_mean);
+  return launch_status();
+}
+
+int qlora_quantize_nf4_dq_noalloc(const void *W, int w_dtype, int64_t n_out, int64_t k_in, uint8_t *codes,
+                                  uint8_t *c2_fp8, float *c1, float *c2_mean, void *stream) {
+  if (n_out < 0 || k_in < 0) return QLORA_ERR_INVALID_ARG;
+  if (w_dtype != QLORA_DTYPE_F32 && w_dtype != QLORA_DTYPE_BF16) return QLORA_ERR_INVALID_ARG;
+  if (k_in > 0 && n_out > QLORA_NOALLOC_MAX_NUMEL / k_in) return QLORA_ERR_SCRATCH_LIMIT;
+  const int64_t numel = n_out * k_in;
+  if (!c2_mean) return QLORA_ERR_INVALID_ARG;
+  if (!aligned(c2_mean, 4)) return QLORA_ERR_MISALIGNED;
+  DeviceInfo *dev;
+  int rc = current_device_info(&dev);
+  if (rc) return rc;
+  unsigned char *scratch;
+  rc = noalloc_scratch(&scratch);
+  if (rc) return rc;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (numel == 0) return cudaMemsetAsync(c2_mean, 0, sizeof(float), st) == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+  if (!W || !codes || !c2_fp8 || !c1) return QLORA_ERR_INVALID_ARG;
+  if (!aligned(W, 16) || !aligned(codes, 16) || !aligned(c2_fp8, 16) || !aligned(c1, 16)) return QLORA_ERR_MISALIGNED;
+  const int64_t nblk = (numel + 63) / 64;
+  float *c2 = reinterpret_cast<float *>(scratch);
+  double *partial = reinterpret_cast<double *>(scratch + kNoallocC2Bytes);
+  const int64_t ngroups = numel >> 8;
+  const int grid1 = (int)std::max<int64_t>(1, std::min<int64_t>((ngroups + 7) / 8, kQuantMaxCtas));
+  if (w_dtype == QLORA_DTYPE_F32)
+    nf4_quantize_kernel<float><<<grid1, kQuantThreads, 0, st>>>(reinterpret_cast<const float *>(W), numel, codes, c2,
+                                                               partial);
+  else
+    nf4_quantize_kernel<__nv_bfloat16><<<grid1, kQuantThreads, 0, st>>>(
+        reinterpret_cast<const __nv_bfloat16 *>(W), numel, codes, c2, partial);
+  rc = launch_status();
+  if (rc) return rc;
+  const int64_t nb256 = (nblk + 255) / 256;
+  const int grid2 = (int)std::max<int64_t>(1, std::min<int64_t>(nb256, (int64_t)dev->sms * 4));
   dq_constants_kernel<<<grid2, 256, 0, st>>>(c2, nblk, partial, grid1, c2_fp8, c1, c2_mean);
   return launch_status();
 }

@@ -59,6 +59,7 @@ extern "C" {
 #define QLORA_ERR_CUDA (-4)              /* a CUDA runtime call or launch failed */
 #define QLORA_ERR_DEVICE_TIMEOUT (-5)    /* a kernel's bounded wait expired (see below) */
 #define QLORA_ERR_WORKSPACE (-6)         /* ws is NULL or smaller than required */
+#define QLORA_ERR_SCRATCH_LIMIT (-7)     /* too large for the fixed scratch of a no-allocation entry point */
 
 /* ---- dtypes ---------------------------------------------------------------- */
 #define QLORA_DTYPE_F32 0
@@ -102,6 +103,38 @@ QLORA_API size_t qlora_quantize_workspace_size(int64_t numel);
  */
 QLORA_API int qlora_quantize_nf4_dq(const void *W, int w_dtype, int64_t n_out, int64_t k_in, uint8_t *codes,
                           uint8_t *c2_fp8, float *c1, float *c2_mean, void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * qlora_quantize_nf4_dq without a workspace argument.  The paper has no
+ * counterpart: this is a convenience of the library.
+ *
+ * Who needs it: callers that cannot allocate device memory at the point where
+ * they quantize -- for example code that runs under a framework which owns all
+ * device memory through its own pool (allocating behind its back breaks its
+ * accounting and limits), or latency-critical code that must not pay for
+ * cudaMalloc's implicit device-wide synchronization.  Such callers pass only
+ * the inputs and outputs.
+ *
+ * Scratch: the fp32 block constants and the fp64 partial sums live in one
+ * static device array inside the library, QLORA_NOALLOC_SCRATCH_BYTES long.
+ * Every GPU on which the library is loaded holds that array until the process
+ * exits.  Limit: n_out * k_in <= QLORA_NOALLOC_MAX_NUMEL (2^28 weights, e.g. a
+ * 16384 x 16384 matrix); larger tensors return QLORA_ERR_SCRATCH_LIMIT before
+ * anything is enqueued.  This entry point never allocates or frees device
+ * memory.
+ *
+ * Set-up: the first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress) with that device current; make that first call before
+ * any stream capture.  Concurrency: all calls share the one array and it keeps
+ * the last call's contents, so calls that may overlap on the GPU (different
+ * streams without ordering) race and must be serialized by the caller.  Every
+ * scratch entry a call reads is first written by the same call.
+ * Outputs, rules and results are identical to qlora_quantize_nf4_dq.
+ */
+#define QLORA_NOALLOC_MAX_NUMEL ((int64_t)1 << 28)
+#define QLORA_NOALLOC_SCRATCH_BYTES (((size_t)1 << 24) + 16384)
+QLORA_API int qlora_quantize_nf4_dq_noalloc(const void *W, int w_dtype, int64_t n_out, int64_t k_in, uint8_t *codes,
+                                            uint8_t *c2_fp8, float *c1, float *c2_mean, void *stream);
 
 /*
  * doubleDequant (§3 Eq. 6) of the whole weight to bf16:
