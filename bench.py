@@ -50,8 +50,8 @@ def linear_flops(M, N, K, r):
             "gemm_Y": base + 2 * M * r * N, "gemm_dX": base + 2 * M * r * K}
 
 
-def step_flops(M=WL.M, r=WL.r):
-    return sum(linear_flops(M, l.n_out, l.k_in, r)["fwd_bwd"] for l in WL.linears)
+def step_flops(linears=None, M=WL.M, r=WL.r):
+    return sum(linear_flops(M, l.n_out, l.k_in, r)["fwd_bwd"] for l in (linears or WL.linears))
 
 
 def load_peaks():
@@ -183,6 +183,43 @@ def make_step(qlora, lins, flat, world):
     return step
 
 
+def run_e2e(args, step, lins, flat, acts, dev, world, e0, e1):
+    """Same step with host buffers: X and dY copied in, adapter gradients copied out."""
+    pinned_in = [torch.empty(a.shape, dtype=a.dtype, pin_memory=True) for a in acts]
+    pinned_dy = [torch.empty(l.dY.shape, dtype=l.dY.dtype, pin_memory=True) for l in lins]
+    for h, a in zip(pinned_in, acts):
+        h.copy_(a)
+    for h, l in zip(pinned_dy, lins):
+        h.copy_(l.dY)
+    grads_host = torch.empty(flat.shape, dtype=flat.dtype, pin_memory=True)
+    h2d = sum(t.numel() * t.element_size() for t in pinned_in + pinned_dy)
+    d2h = grads_host.numel() * grads_host.element_size()
+
+    def e2e_step():
+        for h, a in zip(pinned_in, acts):
+            a.copy_(h, non_blocking=True)
+        for h, l in zip(pinned_dy, lins):
+            l.dY.copy_(h, non_blocking=True)
+        step()
+        grads_host.copy_(flat, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    e0.record()
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record()
+    torch.cuda.synchronize()
+    ms_e2e = e0.elapsed_time(e1) / args.steps
+    t = torch.tensor([ms_e2e], device=dev)
+    if world > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    ms_e2e = float(t.item())
+
+    return ms_e2e, h2d, d2h
+
 def run_ours(args, rank, world, local_rank):
     import bit_nf4_quantized_02_b200 as qlora
     from bit_nf4_quantized_02_b200 import _lib
@@ -191,6 +228,8 @@ def run_ours(args, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     lins, flat, acts = build_layer(dev, rank)
+    if args.linear:
+        lins = [l for l in lins if l.lin.name == args.linear]
     for l in lins:  # allocate the quantized buffers once
         l.q = qlora.quantize_nf4_dq(l.W)
     step = make_step(qlora, lins, flat, world)
@@ -227,42 +266,15 @@ def run_ours(args, rank, world, local_rank):
         raise RuntimeError("device error during the timed region")
 
     # ---------------- end to end: host inputs in, adapter gradients out
-    pinned_in = [torch.empty(a.shape, dtype=a.dtype, pin_memory=True) for a in acts]
-    pinned_dy = [torch.empty(l.dY.shape, dtype=l.dY.dtype, pin_memory=True) for l in lins]
-    for h, a in zip(pinned_in, acts):
-        h.copy_(a)
-    for h, l in zip(pinned_dy, lins):
-        h.copy_(l.dY)
-    grads_host = torch.empty(flat.shape, dtype=flat.dtype, pin_memory=True)
-    h2d = sum(t.numel() * t.element_size() for t in pinned_in + pinned_dy)
-    d2h = grads_host.numel() * grads_host.element_size()
-
-    def e2e_step():
-        for h, a in zip(pinned_in, acts):
-            a.copy_(h, non_blocking=True)
-        for h, l in zip(pinned_dy, lins):
-            l.dY.copy_(h, non_blocking=True)
-        step()
-        grads_host.copy_(flat, non_blocking=True)
-
-    e2e_step()
-    torch.cuda.synchronize()
-    if world > 1:
-        torch.distributed.barrier()
-    e0.record()
-    for _ in range(args.steps):
-        e2e_step()
-    e1.record()
-    torch.cuda.synchronize()
-    ms_e2e = e0.elapsed_time(e1) / args.steps
-    t = torch.tensor([ms_e2e], device=dev)
-    if world > 1:
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-    ms_e2e = float(t.item())
+    if args.no_e2e:
+        ms_e2e, h2d, d2h = None, None, None
+    else:
+        ms_e2e, h2d, d2h = run_e2e(args, step, lins, flat, acts, dev, world, e0, e1)
 
     if rank != 0:
         return None
-    flops = step_flops() * world
+    sel = [l.lin for l in lins]
+    flops = step_flops(sel) * world
     value = flops / (ms * 1e-3) / 1e12
     peaks, peak_src = load_peaks()
     # dominant kernel: the tcgen05 GEMM launches of the Y and dX products
@@ -274,7 +286,7 @@ def run_ours(args, rank, world, local_rank):
     dom_ms = per_kind.get("gemm_Y", [0, 0.0])[1] + per_kind.get("gemm_dX", [0, 0.0])[1]
     dom_n = per_kind.get("gemm_Y", [0, 0.0])[0] + per_kind.get("gemm_dX", [0, 0.0])[0]
     dom_flops = args.steps * sum(linear_flops(WL.M, l.n_out, l.k_in, WL.r)["gemm_Y"] +
-                                 linear_flops(WL.M, l.n_out, l.k_in, WL.r)["gemm_dX"] for l in WL.linears)
+                                 linear_flops(WL.M, l.n_out, l.k_in, WL.r)["gemm_dX"] for l in sel)
     achieved = dom_flops / (dom_ms * 1e-3) / 1e12 if dom_ms > 0 else None
     peak = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
     traffic = None
@@ -292,14 +304,15 @@ def run_ours(args, rank, world, local_rank):
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": WL.name, "model": "llama7b-layer-linears", "global_batch": 16 * world,
+        "config": {"workload": WL.name + (f"[{args.linear} only]" if args.linear else ""),
+                   "model": "llama7b-layer-linears", "global_batch": 16 * world,
                    "seq_len": 512, "tokens_per_rank": WL.M, "lora_r": WL.r, "lora_alpha": WL.alpha,
                    "parallelism": f"dp{world}" if world > 1 else "single",
                    "step": "quantize 7 fp32 weights to NF4+DQ, fwd + bwd of the 7 QLoRA linears"
                            + (", all-reduce of adapter grads" if world > 1 else ""),
                    "l2": "inputs larger than L2 (>1 GB touched per step), no flush"},
-        "e2e": {"value": flops / (ms_e2e * 1e-3) / 1e12, "unit": UNIT, "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h},
+        "e2e": ({"value": flops / (ms_e2e * 1e-3) / 1e12, "unit": UNIT, "h2d_bytes_per_step": h2d,
+                 "d2h_bytes_per_step": d2h} if ms_e2e else None),
         "gpu_launches": len(launches),
         "roofline": {"bound": "tensor", "kernel": "tc_gemm (Y = X W^T + T L2 and dX = dY W + G L1^T)",
                      "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
@@ -309,7 +322,7 @@ def run_ours(args, rank, world, local_rank):
         "kernels": kernels,
         "clocks": clocks,
     }
-    if world == 1 and not args.no_cpu_baseline:
+    if world == 1 and not args.no_cpu_baseline and not args.linear:
         out["cpu_baseline"] = cpu_baseline()
     return out
 
@@ -401,6 +414,9 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end (host buffers) measurement")
+    ap.add_argument("--linear", choices=[l.name for l in WL.linears], default=None,
+                    help="restrict the step to one linear of the layer (profiling runs)")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3
