@@ -289,13 +289,19 @@ def run_ours(args, rank, world, local_rank):
                                  linear_flops(WL.M, l.n_out, l.k_in, WL.r)["gemm_dX"] for l in sel)
     achieved = dom_flops / (dom_ms * 1e-3) / 1e12 if dom_ms > 0 else None
     peak = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+    # DRAM traffic per launch: the ncu-measured ratio of DRAM bytes to algorithmic
+    # bytes for these launches (captured at the q shape), applied to the average
+    # algorithmic bytes of the timed launches; null once the kernel source changed.
     traffic = None
-    tp = os.path.join(ROOT, "profiles", "tc_gemm_traffic.json")
+    tp = os.path.join(ROOT, "profiles", "tc_gemm_traffic.txt")
     if os.path.exists(tp):
         with open(tp) as f:
             tr = json.load(f)
         if tr.get("source_hash") == source_hash("tc_gemm.cuh", "common.cuh"):
-            traffic = tr.get("bytes_per_launch")
+            M, r = WL.M, WL.r
+            alg = [2 * M * l.k_in + 2 * l.n_out * l.k_in + 2 * M * l.n_out + 2 * M * r + 2 * r * l.n_out for l in sel]
+            alg += [2 * M * l.n_out + 2 * l.n_out * l.k_in + 2 * M * l.k_in + 2 * M * r + 2 * r * l.k_in for l in sel]
+            traffic = tr["traffic_over_algorithmic"] * sum(alg) / len(alg)
     total_kernel_ms = sum(v[1] for v in per_kind.values())
     kernels = {k: {"launches_per_step": v[0] / args.steps, "ms_per_step": v[1] / args.steps,
                    "share": v[1] / total_kernel_ms if total_kernel_ms else None}
@@ -315,6 +321,7 @@ def run_ours(args, rank, world, local_rank):
                  "d2h_bytes_per_step": d2h} if ms_e2e else None),
         "gpu_launches": len(launches),
         "roofline": {"bound": "tensor", "kernel": "tc_gemm (Y = X W^T + T L2 and dX = dY W + G L1^T)",
+                     "traffic_unit": "bytes per launch (DRAM read + write)",
                      "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                      "frac": achieved / peak if achieved else None, "traffic": traffic,
                      "peak_source": f"{peak_src} bf16_tflops_sustained",
