@@ -1,0 +1,386 @@
+// Fused doubleDequant + product for few tokens (QLoRA §3 Eq. 5 / Eq. 6 at
+// decode-sized M): the frozen-weight bytes dominate, so every NF4 weight is
+// read once from HBM and decoded in registers straight into tensor-core
+// fragments -- no bf16 copy of the weight is ever written.
+//
+//   Y[M x N] = bf16( X W_hat^T + (s X L1) L2 ),   M <= 8*NT (NT in {1, 2, 4})
+//
+// One persistent kernel, 160 threads per CTA (2 CTAs per SM):
+//   * every CTA first adds a thin K-slice of X L1 into an fp32 accumulator
+//     (red.global.add) and counts itself done; the last one writes
+//     T = s X L1 as a bf16 hi/lo pair for the backward.
+//   * warp 4 is a TMA producer: per stage, 64 weight rows x 256 K of packed
+//     codes (128-byte swizzle) and the matching X tile (3-D view of X,
+//     [token][64-block][64], 128-byte swizzle) into a ring of mbarrier stages;
+//   * warps 0..3 each own 16 weight rows.  Lane (g, j) decodes rows g and g+8
+//     of NF4 block j of the stage -- 64 weights per row, all under one
+//     constant -- through a 16-entry bf16 table T_b[c] = bf16(NF4[c] * c2_hat)
+//     (bit-identical to qlora_dequant) held as byte planes and indexed with
+//     byte permutes, and feeds them as the A operand of mma.sync m16n8k16
+//     (bf16 in, fp32 accumulate) against X as the B operand.
+//   * The K positions inside a stage are permuted consistently for A and B:
+//     logical k-step s, slot u of lane-column j <-> physical k = 64 j + 4 s + u,
+//     so each lane's codes are one contiguous 32-byte run per row and its X
+//     operand is one 16-byte run per two steps; both are bank-conflict free
+//     under the 128-byte swizzle.
+//   * A unit is 64 rows x 512 K; partial products are added into an fp32
+//     [M x N] accumulator with red.global.add (L2 resident).  The CTA that
+//     completes a 64-row block (counter) waits for T, adds T L2 and writes Y.
+// The accumulator, counters and T accumulator must be zero at launch (the
+// host clears them with one memset in stream order).  Split-K additions make
+// the low bits of Y depend on the order in which CTAs finish.
+#pragma once
+
+#include "common.cuh"
+#include "quant.cuh"
+
+namespace qlora {
+
+constexpr int kGvRows = 64;          // weight rows per unit (4 warps x 16)
+constexpr int kGvStageK = 256;       // K per pipeline stage
+constexpr int kGvUnitK = 512;        // K per unit (2 stages)
+constexpr int kGvThreads = 160;      // 4 decode/MMA warps + 1 producer warp
+constexpr int kGvMaxM = 32;
+
+template <int NT>
+struct GvCfg {
+  static constexpr int kCodeBytes = kGvRows * 128;          // 64 rows x 256 codes
+  static constexpr int kXBytes = 8 * NT * kGvStageK * 2;    // padded tokens x 256 bf16
+  static constexpr int kStageBytes = kCodeBytes + kXBytes;
+  static constexpr int kStages = NT == 1 ? 8 : (NT == 2 ? 6 : 4);
+  // + 1024 alignment slack + 256 barrier/flag area; the launch adds M*r*4 bytes
+  // for s*T (used by the finisher).
+  static constexpr int kSmemBytes = kStages * kStageBytes + 1024 + 256;
+};
+
+struct GvArgs {
+  int M, N, K, r;
+  int nks;               // units per 64-row block
+  int units;
+  float s;
+  const uint8_t *c2_fp8;
+  const float *c1;
+  const float *mu;
+  const __nv_bfloat16 *X;    // [M x K]
+  const __nv_bfloat16 *L1;   // [K x r]
+  const __nv_bfloat16 *L2;   // [r x N]
+  float *acc;            // [M x N] fp32, zero at launch
+  float *tacc;           // [M x r] fp32 (unscaled X L1), zero at launch
+  unsigned *counters;    // [ceil(N/64)], zero at launch
+  unsigned *tdone;       // [1], zero at launch
+  __nv_bfloat16 *Y;      // [M x N]
+  __nv_bfloat16 *T_save; // [M x 2r] hi/lo or nullptr
+  int *err;
+};
+
+__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// prmt in its default mode, where a selector nibble with bit 3 set replicates
+// the sign bit of the selected byte.
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t d;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+  return d;
+}
+
+__device__ __forceinline__ uint4 lds128(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+  return v;
+}
+
+__device__ __forceinline__ void red_add_f32(float *p, float v) {
+  asm volatile("red.global.add.f32 [%0], %1;" ::"l"(p), "f"(v) : "memory");
+}
+
+__device__ __forceinline__ void named_bar_sync(int id, int n) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+
+// The 16 decoded values of one 64-block, bf16(NF4[c] * c2_hat), stored as two
+// byte planes: lo[i] holds the low bytes of entries 4i..4i+3, hi[i] the high
+// bytes.
+struct BlockTable {
+  uint32_t lo[4], hi[4];
+  __device__ __forceinline__ void build(float c2h) {
+    uint32_t e[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const __nv_bfloat162 p = __floats2bfloat162_rn(__fmul_rn(kNF4[2 * i], c2h), __fmul_rn(kNF4[2 * i + 1], c2h));
+      e[i] = *reinterpret_cast<const uint32_t *>(&p);
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      lo[i] = __byte_perm(e[2 * i], e[2 * i + 1], 0x6420);
+      hi[i] = __byte_perm(e[2 * i], e[2 * i + 1], 0x7531);
+    }
+  }
+  // Four codes (nibbles of the low 16 bits of `sel7`, bit 3 cleared) whose
+  // bit-3 flags are the byte mask `m8` -> two bf16x2 words {T[c0],T[c1]},
+  // {T[c2],T[c3]}.
+  __device__ __forceinline__ void lookup4(uint32_t sel7, uint32_t m8, uint32_t &p01, uint32_t &p23) const {
+    const uint32_t la = __byte_perm(lo[0], lo[1], sel7);
+    const uint32_t lb = __byte_perm(lo[2], lo[3], sel7);
+    const uint32_t ha = __byte_perm(hi[0], hi[1], sel7);
+    const uint32_t hb = __byte_perm(hi[2], hi[3], sel7);
+    const uint32_t l = (lb & m8) | (la & ~m8);
+    const uint32_t h = (hb & m8) | (ha & ~m8);
+    p01 = __byte_perm(l, h, 0x5140);
+    p23 = __byte_perm(l, h, 0x7362);
+  }
+};
+
+// c2_hat of 64-block b (flattened index): fma(E4M3(code8_b), c1_{b/256}, mu).
+__device__ __forceinline__ float gv_c2hat(const GvArgs &p, int64_t b, float mu) {
+  return __fmaf_rn(e4m3_to_f32(__ldg(p.c2_fp8 + b)), __ldg(p.c1 + (b >> 8)), mu);
+}
+
+template <int NT>
+__global__ void __launch_bounds__(kGvThreads, 2)
+    gemv_fwd_kernel(const __grid_constant__ CUtensorMap tmCodes, const __grid_constant__ CUtensorMap tmX,
+                    const GvArgs p) {
+  using Cfg = GvCfg<NT>;
+  constexpr int S = Cfg::kStages;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t *full_bar = reinterpret_cast<uint64_t *>(smem + S * Cfg::kStageBytes);
+  uint64_t *empty_bar = full_bar + S;
+  unsigned *flag = reinterpret_cast<unsigned *>(empty_bar + S);
+  float *t_s = reinterpret_cast<float *>(smem + S * Cfg::kStageBytes + 256);  // [M x r] s*T
+  bool t_loaded = false;
+
+  const int warp = warp_id();
+  const int lane = lane_id();
+  const int kblocks = p.K >> 6;
+
+  // ---------------------------------------------------------------- T = X L1
+  // Every CTA adds X[:, k0:k1] L1[k0:k1, :] for its own thin K-slice into the
+  // fp32 accumulator; thread (token group of 4, column j) keeps 4 sums.
+  {
+    const int kper = ((p.K + 8 * (int)gridDim.x - 1) / (8 * (int)gridDim.x)) * 8;
+    const int k0 = min(p.K, (int)blockIdx.x * kper);
+    const int k1 = min(p.K, k0 + kper);
+    const int groups = (p.M + 3) >> 2;
+    for (int o = threadIdx.x; o < groups * p.r && k0 < k1; o += blockDim.x) {
+      const int tg = o / p.r, jj = o - tg * p.r;
+      float t[4] = {0.f, 0.f, 0.f, 0.f};
+      for (int k = k0; k < k1; ++k) {
+        const float l1 = __bfloat162float(p.L1[(int64_t)k * p.r + jj]);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int m = 4 * tg + i;
+          if (m < p.M) t[i] = __fmaf_rn(__bfloat162float(p.X[(int64_t)m * p.K + k]), l1, t[i]);
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        if (4 * tg + i < p.M) red_add_f32(p.tacc + (4 * tg + i) * p.r + jj, t[i]);
+    }
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) *flag = atomicAdd(p.tdone, 1u);
+    __syncthreads();
+    if (*flag == gridDim.x - 1 && p.T_save) {
+      __threadfence();
+      for (int i = threadIdx.x; i < p.M * p.r; i += blockDim.x) {
+        const float v = p.s * __ldcg(p.tacc + i);
+        const int m = i / p.r, jj = i - m * p.r;
+        const __nv_bfloat16 hb = __float2bfloat16_rn(v);
+        p.T_save[(int64_t)m * 2 * p.r + jj] = hb;
+        p.T_save[(int64_t)m * 2 * p.r + p.r + jj] = __float2bfloat16_rn(v - __bfloat162float(hb));
+      }
+    }
+    __syncthreads();
+  }
+
+  // ---------------------------------------------------------------- main loop
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < S; ++i) {
+      mbar_init(smem_u32(full_bar + i), 1);
+      mbar_init(smem_u32(empty_bar + i), 4);
+    }
+    fence_mbar_init();
+  }
+  __syncthreads();
+
+  if (warp == 4) {
+    if (lane == 0) {
+      tma_prefetch_desc(&tmCodes);
+      tma_prefetch_desc(&tmX);
+      int stage = 0;
+      uint32_t phase = 0, used = 0, last_parity = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < p.units && ok; u += gridDim.x) {
+        const int rb = u / p.nks, ks = u - rb * p.nks;
+        const int kbeg = ks * kGvUnitK;
+        const int nst = min(kGvUnitK, p.K - kbeg) > kGvStageK ? 2 : 1;
+        for (int st = 0; st < nst; ++st) {
+          if (!mbar_wait(smem_u32(empty_bar + stage), phase ^ 1, p.err, DEV_TIMEOUT_PRODUCER)) {
+            ok = false;
+            break;
+          }
+          const uint32_t fb = smem_u32(full_bar + stage);
+          mbar_arrive_expect_tx(fb, Cfg::kStageBytes);
+          const uint32_t sc = smem_u32(smem + stage * Cfg::kStageBytes);
+          const int k0 = kbeg + st * kGvStageK;
+          tma_load_2d(sc, &tmCodes, fb, k0 >> 1, rb * kGvRows);
+          asm volatile(
+              "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5}], "
+              "[%2];" ::"r"(sc + Cfg::kCodeBytes),
+              "l"(reinterpret_cast<uint64_t>(&tmX)), "r"(fb), "r"(0), "r"(k0 >> 6), "r"(0)
+              : "memory");
+          used |= 1u << stage;
+          last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
+          if (++stage == S) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+      for (int i = 0; i < S; ++i)
+        if (used & (1u << i)) mbar_wait(smem_u32(full_bar + i), (last_parity >> i) & 1u, p.err, DEV_TIMEOUT_DRAIN);
+    }
+  } else {
+    const int g = lane >> 2, j = lane & 3;
+    const int r0 = warp * 16 + g;  // row of this lane inside the unit (and r0 + 8)
+    const float mu = __ldg(p.mu);
+    int stage = 0;
+    uint32_t phase = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; u < p.units && ok; u += gridDim.x) {
+      const int rb = u / p.nks, ks = u - rb * p.nks;
+      const int kbeg = ks * kGvUnitK;
+      const int nst = min(kGvUnitK, p.K - kbeg) > kGvStageK ? 2 : 1;
+      const int n0 = rb * kGvRows + r0, n1 = n0 + 8;
+      float d[NT][4];
+#pragma unroll
+      for (int t = 0; t < NT; ++t) d[t][0] = d[t][1] = d[t][2] = d[t][3] = 0.f;
+      for (int st = 0; st < nst; ++st) {
+        // the lane's 64-block in this stage and its two tables
+        const int kb = ((kbeg + st * kGvStageK) >> 6) + j;
+        BlockTable tb0, tb1;
+        const bool kok = kb < kblocks;
+        tb0.build(kok && n0 < p.N ? gv_c2hat(p, (int64_t)n0 * kblocks + kb, mu) : 0.f);
+        tb1.build(kok && n1 < p.N ? gv_c2hat(p, (int64_t)n1 * kblocks + kb, mu) : 0.f);
+        if (!mbar_wait(smem_u32(full_bar + stage), phase, p.err, DEV_TIMEOUT_MMA)) {
+          ok = false;
+          break;
+        }
+        const uint32_t sc = smem_u32(smem + stage * Cfg::kStageBytes);
+        const uint32_t sx = sc + Cfg::kCodeBytes;
+        // codes of rows r0, r0+8: 16-byte chunks 2j, 2j+1 of their 128-byte lines
+        uint32_t q0[8], q1[8];
+        {
+          const uint4 a = lds128(sc + r0 * 128 + (((2 * j) ^ (r0 & 7)) << 4));
+          const uint4 b = lds128(sc + r0 * 128 + (((2 * j + 1) ^ (r0 & 7)) << 4));
+          const uint4 c = lds128(sc + (r0 + 8) * 128 + (((2 * j) ^ (r0 & 7)) << 4));
+          const uint4 e = lds128(sc + (r0 + 8) * 128 + (((2 * j + 1) ^ (r0 & 7)) << 4));
+          q0[0] = a.x; q0[1] = a.y; q0[2] = a.z; q0[3] = a.w; q0[4] = b.x; q0[5] = b.y; q0[6] = b.z; q0[7] = b.w;
+          q1[0] = c.x; q1[1] = c.y; q1[2] = c.z; q1[3] = c.w; q1[4] = e.x; q1[5] = e.y; q1[6] = e.z; q1[7] = e.w;
+        }
+#pragma unroll
+        for (int w = 0; w < 8; ++w) {
+          // X operand for steps 2w, 2w+1: token g + 8t, line (token*4 + j), chunk w
+          uint4 xb[NT];
+#pragma unroll
+          for (int t = 0; t < NT; ++t) {
+            const int line = (g + 8 * t) * 4 + j;
+            xb[t] = lds128(sx + line * 128 + ((w ^ (line & 7)) << 4));
+          }
+          const uint32_t m0 = q0[w] & 0x77777777u, m1 = q1[w] & 0x77777777u;
+          const uint32_t s0 = q0[w] << 4, s1 = q1[w] << 4;
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            uint32_t a[4];
+            const uint32_t msel = h ? 0xFBEAu : 0xD9C8u;
+            tb0.lookup4(h ? (m0 >> 16) : m0, prmt(s0, q0[w], msel), a[0], a[2]);
+            tb1.lookup4(h ? (m1 >> 16) : m1, prmt(s1, q1[w], msel), a[1], a[3]);
+#pragma unroll
+            for (int t = 0; t < NT; ++t) {
+              const uint32_t b0 = h ? xb[t].z : xb[t].x;
+              const uint32_t b1 = h ? xb[t].w : xb[t].y;
+              mma_bf16_16816(d[t], a, b0, b1);
+            }
+          }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(empty_bar + stage));
+        if (++stage == S) {
+          stage = 0;
+          phase ^= 1;
+        }
+      }
+      if (!ok) break;
+      // add this unit's partial products into the accumulator
+#pragma unroll
+      for (int t = 0; t < NT; ++t) {
+        const int tok = 8 * t + 2 * j;
+        if (tok < p.M) {
+          if (n0 < p.N) red_add_f32(p.acc + (int64_t)tok * p.N + n0, d[t][0]);
+          if (n1 < p.N) red_add_f32(p.acc + (int64_t)tok * p.N + n1, d[t][2]);
+        }
+        if (tok + 1 < p.M) {
+          if (n0 < p.N) red_add_f32(p.acc + (int64_t)(tok + 1) * p.N + n0, d[t][1]);
+          if (n1 < p.N) red_add_f32(p.acc + (int64_t)(tok + 1) * p.N + n1, d[t][3]);
+        }
+      }
+      __threadfence();
+      named_bar_sync(1, 128);
+      if (threadIdx.x == 0) {
+        const unsigned done = atomicAdd(p.counters + rb, 1u);
+        unsigned last = done == (unsigned)p.nks - 1;
+        if (last) {
+          // T must be complete before the LoRA term is added.
+          const uint64_t t0 = globaltimer_ns();
+          while (atomicAdd(p.tdone, 0u) < gridDim.x) {
+            if (globaltimer_ns() - t0 > kWaitLimitNs) {
+              record_error(p.err, DEV_TIMEOUT_EPILOGUE);
+              last = 0;
+              break;
+            }
+          }
+        }
+        *flag = last;
+      }
+      named_bar_sync(1, 128);
+      if (*flag) {
+        __threadfence();
+        if (!t_loaded) {  // s*T, complete once every CTA has added its slice
+          for (int i = threadIdx.x; i < p.M * p.r; i += 128) t_s[i] = p.s * __ldcg(p.tacc + i);
+          t_loaded = true;
+          named_bar_sync(1, 128);
+        }
+        // Y[tok][n] = bf16(acc + sum_j (s*T)[tok][j] * L2[j][n]) for this 64-row block
+        const int n = rb * kGvRows + (threadIdx.x & 63);
+        const int tok0 = threadIdx.x >> 6;  // 0 or 1: tokens tok0, tok0 + 2, ...
+        if (n < p.N) {
+          float y[4 * NT];
+#pragma unroll
+          for (int i = 0; i < 4 * NT; ++i) y[i] = 0.f;
+          for (int jj = 0; jj < p.r; ++jj) {
+            const float l2 = __bfloat162float(p.L2[(int64_t)jj * p.N + n]);
+#pragma unroll
+            for (int i = 0; i < 4 * NT; ++i) {
+              const int tok = tok0 + 2 * i;
+              if (tok < p.M) y[i] = __fmaf_rn(t_s[tok * p.r + jj], l2, y[i]);
+            }
+          }
+#pragma unroll
+          for (int i = 0; i < 4 * NT; ++i) {
+            const int tok = tok0 + 2 * i;
+            if (tok < p.M)
+              p.Y[(int64_t)tok * p.N + n] = __float2bfloat16_rn(__ldcg(p.acc + (int64_t)tok * p.N + n) + y[i]);
+          }
+        }
+      }
+    }
+  }
+}
+
+}  // namespace qlora

@@ -11,6 +11,7 @@
 #include "common.cuh"
 #include "quant.cuh"
 #include "tc_gemm.cuh"
+#include "gemv.cuh"
 
 namespace qlora {
 
@@ -25,6 +26,7 @@ struct DeviceInfo {
   int sms = 0;
   int *err = nullptr;        // device address of g_dev_err
   bool gemm_attr[3] = {false, false, false};
+  int gemv_smem_set[3] = {0, 0, 0};   // dynamic smem limit set per NT variant
 };
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_mu;
@@ -271,6 +273,95 @@ int check_linear(int64_t M, const qlora_nf4dq_t *W, int r) {
   return QLORA_OK;
 }
 
+int encode_tmap(CUtensorMap *m, CUtensorMapDataType dt, int rank, const void *ptr, const cuuint64_t *dims,
+                const cuuint64_t *strides, const cuuint32_t *box) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return QLORA_ERR_CUDA;
+  const cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(m, dt, rank, const_cast<void *>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? QLORA_OK : QLORA_ERR_CUDA;
+}
+
+// Workspace of the few-token forward: [acc M*N f32 | tacc M*r f32 | counters | tdone], all zeroed per call.
+struct GemvLayout {
+  size_t acc, tacc, counters, tdone, zero_bytes, total;
+};
+
+GemvLayout gemv_layout(int64_t M, int64_t N, int r) {
+  GemvLayout L;
+  L.acc = 0;
+  L.tacc = align_up((size_t)M * N * 4, 16);
+  L.counters = L.tacc + align_up((size_t)M * r * 4, 16);
+  L.tdone = L.counters + (size_t)((N + kGvRows - 1) / kGvRows) * 4;
+  L.zero_bytes = L.tdone + 4;
+  L.total = align_up(L.zero_bytes);
+  return L;
+}
+
+template <int NT>
+int launch_gemv(const qlora_nf4dq_t *W, const uint16_t *X, int64_t M, const uint16_t *L1, const uint16_t *L2, int r,
+                float s, uint16_t *Y, uint16_t *T_save, uint8_t *ws, DeviceInfo *dev, cudaStream_t st) {
+  using Cfg = GvCfg<NT>;
+  const int64_t N = W->n_out, K = W->k_in;
+  const GemvLayout L = gemv_layout(M, N, r);
+  if (cudaMemsetAsync(ws, 0, L.zero_bytes, st) != cudaSuccess) return QLORA_ERR_CUDA;
+  CUtensorMap tm_codes, tm_x;
+  {
+    const cuuint64_t dims[2] = {(cuuint64_t)(K / 2), (cuuint64_t)N};
+    const cuuint64_t strides[1] = {(cuuint64_t)(K / 2)};
+    const cuuint32_t box[2] = {128, (cuuint32_t)kGvRows};
+    int rc = encode_tmap(&tm_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, W->codes, dims, strides, box);
+    if (rc) return rc;
+  }
+  {
+    const cuuint64_t dims[3] = {64, (cuuint64_t)(K / 64), (cuuint64_t)M};
+    const cuuint64_t strides[2] = {128, (cuuint64_t)K * 2};
+    const cuuint32_t box[3] = {64, 4, (cuuint32_t)(8 * NT)};
+    int rc = encode_tmap(&tm_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, X, dims, strides, box);
+    if (rc) return rc;
+  }
+  const int smem = Cfg::kSmemBytes + (int)(M * r * 4);
+  const int idx = NT == 1 ? 0 : (NT == 2 ? 1 : 2);
+  if (dev->gemv_smem_set[idx] < smem) {
+    if (cudaFuncSetAttribute(gemv_fwd_kernel<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+      return QLORA_ERR_CUDA;
+    dev->gemv_smem_set[idx] = smem;
+  }
+  // Every CTA must be resident at once: the finishing CTAs wait for all CTAs'
+  // share of T, so the grid never exceeds what fits on the device together.
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, gemv_fwd_kernel<NT>, kGvThreads, smem) != cudaSuccess ||
+      per_sm < 1)
+    return QLORA_ERR_CUDA;
+  GvArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.M = (int)M;
+  a.N = (int)N;
+  a.K = (int)K;
+  a.r = r;
+  a.nks = (int)((K + kGvUnitK - 1) / kGvUnitK);
+  a.units = (int)((N + kGvRows - 1) / kGvRows) * a.nks;
+  a.s = s;
+  a.c2_fp8 = W->c2_fp8;
+  a.c1 = W->c1;
+  a.mu = W->c2_mean;
+  a.X = reinterpret_cast<const __nv_bfloat16 *>(X);
+  a.L1 = reinterpret_cast<const __nv_bfloat16 *>(L1);
+  a.L2 = reinterpret_cast<const __nv_bfloat16 *>(L2);
+  a.acc = reinterpret_cast<float *>(ws + L.acc);
+  a.tacc = reinterpret_cast<float *>(ws + L.tacc);
+  a.counters = reinterpret_cast<unsigned *>(ws + L.counters);
+  a.tdone = reinterpret_cast<unsigned *>(ws + L.tdone);
+  a.Y = reinterpret_cast<__nv_bfloat16 *>(Y);
+  a.T_save = reinterpret_cast<__nv_bfloat16 *>(T_save);
+  a.err = dev->err;
+  const int grid = std::max(1, std::min(a.units, per_sm * dev->sms));
+  ProfScope prof(QLORA_KERNEL_GEMV_FWD, st);
+  gemv_fwd_kernel<NT><<<grid, kGvThreads, smem, st>>>(tm_codes, tm_x, a);
+  return launch_status();
+}
+
 struct FwdLayout {
   size_t w_hat, t, split, total;
 };
@@ -513,6 +604,7 @@ int qlora_dequant(const qlora_nf4dq_t *W, uint16_t *W_out, void *stream) {
 
 size_t qlora_linear_fwd_workspace_size(int64_t M, int64_t n_out, int64_t k_in, int r) {
   if (M < 0 || n_out <= 0 || k_in <= 0 || r <= 0) return 0;
+  if (M <= kGvMaxM) return gemv_layout(M, n_out, r).total;
   DeviceInfo *dev;
   const int sms = current_device_info(&dev) == QLORA_OK ? dev->sms : 148;
   return fwd_layout(M, n_out, k_in, r, sms).total;
@@ -537,10 +629,19 @@ int qlora_linear_fwd(const uint16_t *X, int64_t M, const qlora_nf4dq_t *W, const
   rc = current_device_info(&dev);
   if (rc) return rc;
   const int64_t N = W->n_out, K = W->k_in;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (M <= kGvMaxM) {
+    // Few tokens: the weight bytes dominate; one fused decode + product pass.
+    if (!ws || ws_bytes < gemv_layout(M, N, r).total) return QLORA_ERR_WORKSPACE;
+    if (!aligned(ws, 256)) return QLORA_ERR_MISALIGNED;
+    uint8_t *w8 = reinterpret_cast<uint8_t *>(ws);
+    if (M <= 8) return launch_gemv<1>(W, X, M, L1, L2, r, s, Y, T_save, w8, dev, st);
+    if (M <= 16) return launch_gemv<2>(W, X, M, L1, L2, r, s, Y, T_save, w8, dev, st);
+    return launch_gemv<4>(W, X, M, L1, L2, r, s, Y, T_save, w8, dev, st);
+  }
   const FwdLayout L = fwd_layout(M, N, K, r, dev->sms);
   if (!ws || ws_bytes < L.total) return QLORA_ERR_WORKSPACE;
   if (!aligned(ws, 256)) return QLORA_ERR_MISALIGNED;
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   uint8_t *w8 = reinterpret_cast<uint8_t *>(ws);
   __nv_bfloat16 *w_hat = reinterpret_cast<__nv_bfloat16 *>(w8 + L.w_hat);
   uint16_t *T = T_save ? T_save : reinterpret_cast<uint16_t *>(w8 + L.t);

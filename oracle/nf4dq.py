@@ -350,6 +350,35 @@ def dequantize(q) -> np.ndarray:
     return bf16_bits_to_f32(bits)
 
 
+def dequantize_rows(w, rows) -> np.ndarray:
+    """doubleDequant of selected rows of a 2-D weight, for sampled checks.
+
+    The same steps as ``quantize_nf4_dq`` + ``dequantize``: every block's c2
+    (the mean needs all of them), then the second-level constants of the
+    256-groups holding the selected rows' blocks, then those rows' codes.
+    Requires k_in % 64 == 0 (blocks do not straddle rows).
+    """
+    w = f32(w)
+    n_out, k_in = w.shape
+    if k_in % W_BLOCK:
+        raise ValueError("dequantize_rows: k_in must be a multiple of 64")
+    c2 = block_absmax(w.reshape(-1), W_BLOCK)
+    mu = dq_mean(c2)
+    bpr = k_in // W_BLOCK
+    out = np.empty((len(rows), k_in), np.float32)
+    for i, row in enumerate(rows):
+        b0, b1 = row * bpr, (row + 1) * bpr
+        g0, g1 = b0 // C2_BLOCK, (b1 - 1) // C2_BLOCK + 1
+        seg = c2[g0 * C2_BLOCK: min(c2.size, g1 * C2_BLOCK)]
+        code8, c1, _ = double_quantize(seg, mu)
+        c2_hat = dequant_c2(code8, c1, mu)[b0 - g0 * C2_BLOCK: b1 - g0 * C2_BLOCK]
+        codes, c2_row = quantize_nf4(w[row])
+        assert np.array_equal(c2_row, c2[b0:b1])
+        prod = (NF4_VALUES[codes] * np.repeat(c2_hat, W_BLOCK)).astype(np.float32)
+        out[i] = bf16_bits_to_f32(bf16_rne_bits(prod))
+    return out
+
+
 def dequant_nf4_no_dq(codes, c2, shape) -> np.ndarray:
     """First-level dequant only (Eq. 2 with the absmax constant), float64."""
     codes = np.asarray(codes, dtype=np.uint8).reshape(-1)

@@ -142,3 +142,11 @@ def test_double_dequant_codes7_is_zero():
     q = nf4dq.quantize_nf4_dq(w)
     assert np.all(q["codes"] == 7)
     assert np.all(nf4dq.dequantize(q) == 0.0)
+
+
+def test_dequantize_rows_equals_full_dequantize():
+    g = inputs.rng(26)
+    w = inputs.normal_f32(g, (40, 1024), 0.02)   # 640 blocks: rows straddle 256-groups
+    full = nf4dq.dequantize(nf4dq.quantize_nf4_dq(w))
+    rows = [0, 3, 4, 17, 39]
+    assert np.array_equal(nf4dq.dequantize_rows(w, rows), full[rows])
