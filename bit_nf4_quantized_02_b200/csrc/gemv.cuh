@@ -5,10 +5,11 @@
 //
 //   Y[M x N] = bf16( X W_hat^T + (s X L1) L2 ),   M <= 8*NT (NT in {1, 2, 4})
 //
-// One persistent kernel, 160 threads per CTA (2 CTAs per SM):
-//   * every CTA first adds a thin K-slice of X L1 into an fp32 accumulator
-//     (red.global.add) and counts itself done; the last one writes
-//     T = s X L1 as a bf16 hi/lo pair for the backward.
+// Two launches per linear: lora_down_small_kernel adds K-slices of X L1 into
+// an fp32 accumulator; gemv_fwd_kernel is launched as its programmatic
+// dependent, so it streams the weight concurrently and only its finishing
+// CTAs wait (griddepcontrol.wait) for T before adding the LoRA term.
+// gemv_fwd_kernel, persistent, 160 threads per CTA (2 CTAs per SM):
 //   * warp 4 is a TMA producer: per stage, 64 weight rows x 256 K of packed
 //     codes (128-byte swizzle) and the matching X tile (3-D view of X,
 //     [token][64-block][64], 128-byte swizzle) into a ring of mbarrier stages;
@@ -25,7 +26,9 @@
 //     under the 128-byte swizzle.
 //   * A unit is 64 rows x 512 K; partial products are added into an fp32
 //     [M x N] accumulator with red.global.add (L2 resident).  The CTA that
-//     completes a 64-row block (counter) waits for T, adds T L2 and writes Y.
+//     completes a 64-row block (counter) waits for T, adds s T L2 and writes
+//     Y; the finisher of row block 0 also writes T = s X L1 as a bf16 hi/lo
+//     pair for the backward.
 // The accumulator, counters and T accumulator must be zero at launch (the
 // host clears them with one memset in stream order).  Split-K additions make
 // the low bits of Y depend on the order in which CTAs finish.
@@ -67,7 +70,6 @@ struct GvArgs {
   float *acc;            // [M x N] fp32, zero at launch
   float *tacc;           // [M x r] fp32 (unscaled X L1), zero at launch
   unsigned *counters;    // [ceil(N/64)], zero at launch
-  unsigned *tdone;       // [1], zero at launch
   __nv_bfloat16 *Y;      // [M x N]
   __nv_bfloat16 *T_save; // [M x 2r] hi/lo or nullptr
   int *err;
@@ -136,10 +138,37 @@ struct BlockTable {
   }
 };
 
-// c2_hat of 64-block b (flattened index): fma(E4M3(code8_b), c1_{b/256}, mu).
-__device__ __forceinline__ float gv_c2hat(const GvArgs &p, int64_t b, float mu) {
-  return __fmaf_rn(e4m3_to_f32(__ldg(p.c2_fp8 + b)), __ldg(p.c1 + (b >> 8)), mu);
-}
+// Raw constants of a lane's two (row, block) pairs for one (unit, stage) item.
+struct ConstPrefetch {
+  uint32_t code8[2];
+  float c1[2];
+  bool ok[2];
+  __device__ __forceinline__ void load(const GvArgs &p, int u, int st, int r0, int j, int kblocks) {
+    ok[0] = ok[1] = false;
+    code8[0] = code8[1] = 0;
+    c1[0] = c1[1] = 0.f;
+    if (u >= p.units) return;
+    const int rb = u / p.nks, ks = u - rb * p.nks;
+    const int kb = ((ks * kGvUnitK + st * kGvStageK) >> 6) + j;
+    if (kb >= kblocks) return;
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      const int n = rb * kGvRows + r0 + 8 * i;
+      if (n < p.N) {
+        const int64_t b = (int64_t)n * kblocks + kb;
+        code8[i] = __ldg(p.c2_fp8 + b);
+        c1[i] = __ldg(p.c1 + (b >> 8));
+        ok[i] = true;
+      }
+    }
+  }
+  __device__ __forceinline__ float c2hat(int i, float mu) const {
+    return ok[i] ? __fmaf_rn(e4m3_to_f32((uint8_t)code8[i]), c1[i], mu) : 0.f;
+  }
+};
+
+template <int NT>
+__device__ __noinline__ void gv_finish(const GvArgs &p, int rb, float *t_s, bool &t_loaded);
 
 template <int NT>
 __global__ void __launch_bounds__(kGvThreads, 2)
@@ -158,46 +187,6 @@ __global__ void __launch_bounds__(kGvThreads, 2)
   const int warp = warp_id();
   const int lane = lane_id();
   const int kblocks = p.K >> 6;
-
-  // ---------------------------------------------------------------- T = X L1
-  // Every CTA adds X[:, k0:k1] L1[k0:k1, :] for its own thin K-slice into the
-  // fp32 accumulator; thread (token group of 4, column j) keeps 4 sums.
-  {
-    const int kper = ((p.K + 8 * (int)gridDim.x - 1) / (8 * (int)gridDim.x)) * 8;
-    const int k0 = min(p.K, (int)blockIdx.x * kper);
-    const int k1 = min(p.K, k0 + kper);
-    const int groups = (p.M + 3) >> 2;
-    for (int o = threadIdx.x; o < groups * p.r && k0 < k1; o += blockDim.x) {
-      const int tg = o / p.r, jj = o - tg * p.r;
-      float t[4] = {0.f, 0.f, 0.f, 0.f};
-      for (int k = k0; k < k1; ++k) {
-        const float l1 = __bfloat162float(p.L1[(int64_t)k * p.r + jj]);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int m = 4 * tg + i;
-          if (m < p.M) t[i] = __fmaf_rn(__bfloat162float(p.X[(int64_t)m * p.K + k]), l1, t[i]);
-        }
-      }
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-        if (4 * tg + i < p.M) red_add_f32(p.tacc + (4 * tg + i) * p.r + jj, t[i]);
-    }
-    __threadfence();
-    __syncthreads();
-    if (threadIdx.x == 0) *flag = atomicAdd(p.tdone, 1u);
-    __syncthreads();
-    if (*flag == gridDim.x - 1 && p.T_save) {
-      __threadfence();
-      for (int i = threadIdx.x; i < p.M * p.r; i += blockDim.x) {
-        const float v = p.s * __ldcg(p.tacc + i);
-        const int m = i / p.r, jj = i - m * p.r;
-        const __nv_bfloat16 hb = __float2bfloat16_rn(v);
-        p.T_save[(int64_t)m * 2 * p.r + jj] = hb;
-        p.T_save[(int64_t)m * 2 * p.r + p.r + jj] = __float2bfloat16_rn(v - __bfloat162float(hb));
-      }
-    }
-    __syncthreads();
-  }
 
   // ---------------------------------------------------------------- main loop
   if (threadIdx.x == 0) {
@@ -252,133 +241,191 @@ __global__ void __launch_bounds__(kGvThreads, 2)
     const float mu = __ldg(p.mu);
     int stage = 0;
     uint32_t phase = 0;
-    bool ok = true;
-    for (int u = blockIdx.x; u < p.units && ok; u += gridDim.x) {
+    // Flat walk over this CTA's (unit, stage) items; the block constants of
+    // the next item are loaded one item ahead so their latency hides under
+    // the current item's decode.
+    int u = blockIdx.x, st = 0;
+    ConstPrefetch pre, nxt;
+    pre.load(p, u, st, r0, j, kblocks);
+    float d[NT][4];
+    while (u < p.units) {
       const int rb = u / p.nks, ks = u - rb * p.nks;
       const int kbeg = ks * kGvUnitK;
       const int nst = min(kGvUnitK, p.K - kbeg) > kGvStageK ? 2 : 1;
       const int n0 = rb * kGvRows + r0, n1 = n0 + 8;
-      float d[NT][4];
+      if (st == 0) {
 #pragma unroll
-      for (int t = 0; t < NT; ++t) d[t][0] = d[t][1] = d[t][2] = d[t][3] = 0.f;
-      for (int st = 0; st < nst; ++st) {
-        // the lane's 64-block in this stage and its two tables
-        const int kb = ((kbeg + st * kGvStageK) >> 6) + j;
-        BlockTable tb0, tb1;
-        const bool kok = kb < kblocks;
-        tb0.build(kok && n0 < p.N ? gv_c2hat(p, (int64_t)n0 * kblocks + kb, mu) : 0.f);
-        tb1.build(kok && n1 < p.N ? gv_c2hat(p, (int64_t)n1 * kblocks + kb, mu) : 0.f);
-        if (!mbar_wait(smem_u32(full_bar + stage), phase, p.err, DEV_TIMEOUT_MMA)) {
-          ok = false;
-          break;
-        }
-        const uint32_t sc = smem_u32(smem + stage * Cfg::kStageBytes);
-        const uint32_t sx = sc + Cfg::kCodeBytes;
-        // codes of rows r0, r0+8: 16-byte chunks 2j, 2j+1 of their 128-byte lines
-        uint32_t q0[8], q1[8];
-        {
-          const uint4 a = lds128(sc + r0 * 128 + (((2 * j) ^ (r0 & 7)) << 4));
-          const uint4 b = lds128(sc + r0 * 128 + (((2 * j + 1) ^ (r0 & 7)) << 4));
-          const uint4 c = lds128(sc + (r0 + 8) * 128 + (((2 * j) ^ (r0 & 7)) << 4));
-          const uint4 e = lds128(sc + (r0 + 8) * 128 + (((2 * j + 1) ^ (r0 & 7)) << 4));
-          q0[0] = a.x; q0[1] = a.y; q0[2] = a.z; q0[3] = a.w; q0[4] = b.x; q0[5] = b.y; q0[6] = b.z; q0[7] = b.w;
-          q1[0] = c.x; q1[1] = c.y; q1[2] = c.z; q1[3] = c.w; q1[4] = e.x; q1[5] = e.y; q1[6] = e.z; q1[7] = e.w;
-        }
+        for (int t = 0; t < NT; ++t) d[t][0] = d[t][1] = d[t][2] = d[t][3] = 0.f;
+      }
+      BlockTable tb0, tb1;
+      tb0.build(pre.c2hat(0, mu));
+      tb1.build(pre.c2hat(1, mu));
+      int nu = u, nstn = st + 1;
+      if (nstn == nst) {
+        nu = u + gridDim.x;
+        nstn = 0;
+      }
+      nxt.load(p, nu, nstn, r0, j, kblocks);
+      if (!mbar_wait(smem_u32(full_bar + stage), phase, p.err, DEV_TIMEOUT_MMA)) break;
+      const uint32_t sc = smem_u32(smem + stage * Cfg::kStageBytes);
+      const uint32_t sx = sc + Cfg::kCodeBytes;
+      // codes of rows r0, r0+8: 16-byte chunks 2j, 2j+1 of their 128-byte lines
+      uint32_t q0[8], q1[8];
+      {
+        const uint4 a = lds128(sc + r0 * 128 + (((2 * j) ^ (r0 & 7)) << 4));
+        const uint4 b = lds128(sc + r0 * 128 + (((2 * j + 1) ^ (r0 & 7)) << 4));
+        const uint4 c = lds128(sc + (r0 + 8) * 128 + (((2 * j) ^ (r0 & 7)) << 4));
+        const uint4 e = lds128(sc + (r0 + 8) * 128 + (((2 * j + 1) ^ (r0 & 7)) << 4));
+        q0[0] = a.x; q0[1] = a.y; q0[2] = a.z; q0[3] = a.w; q0[4] = b.x; q0[5] = b.y; q0[6] = b.z; q0[7] = b.w;
+        q1[0] = c.x; q1[1] = c.y; q1[2] = c.z; q1[3] = c.w; q1[4] = e.x; q1[5] = e.y; q1[6] = e.z; q1[7] = e.w;
+      }
 #pragma unroll
-        for (int w = 0; w < 8; ++w) {
-          // X operand for steps 2w, 2w+1: token g + 8t, line (token*4 + j), chunk w
-          uint4 xb[NT];
+      for (int w = 0; w < 8; ++w) {
+        // X operand for steps 2w, 2w+1: token g + 8t, line (token*4 + j), chunk w
+        uint4 xb[NT];
+#pragma unroll
+        for (int t = 0; t < NT; ++t) {
+          const int line = (g + 8 * t) * 4 + j;
+          xb[t] = lds128(sx + line * 128 + ((w ^ (line & 7)) << 4));
+        }
+        const uint32_t m0 = q0[w] & 0x77777777u, m1 = q1[w] & 0x77777777u;
+        const uint32_t s0 = q0[w] << 4, s1 = q1[w] << 4;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          uint32_t a[4];
+          const uint32_t msel = h ? 0xFBEAu : 0xD9C8u;
+          tb0.lookup4(h ? (m0 >> 16) : m0, prmt(s0, q0[w], msel), a[0], a[2]);
+          tb1.lookup4(h ? (m1 >> 16) : m1, prmt(s1, q1[w], msel), a[1], a[3]);
 #pragma unroll
           for (int t = 0; t < NT; ++t) {
-            const int line = (g + 8 * t) * 4 + j;
-            xb[t] = lds128(sx + line * 128 + ((w ^ (line & 7)) << 4));
-          }
-          const uint32_t m0 = q0[w] & 0x77777777u, m1 = q1[w] & 0x77777777u;
-          const uint32_t s0 = q0[w] << 4, s1 = q1[w] << 4;
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            uint32_t a[4];
-            const uint32_t msel = h ? 0xFBEAu : 0xD9C8u;
-            tb0.lookup4(h ? (m0 >> 16) : m0, prmt(s0, q0[w], msel), a[0], a[2]);
-            tb1.lookup4(h ? (m1 >> 16) : m1, prmt(s1, q1[w], msel), a[1], a[3]);
-#pragma unroll
-            for (int t = 0; t < NT; ++t) {
-              const uint32_t b0 = h ? xb[t].z : xb[t].x;
-              const uint32_t b1 = h ? xb[t].w : xb[t].y;
-              mma_bf16_16816(d[t], a, b0, b1);
-            }
+            const uint32_t b0 = h ? xb[t].z : xb[t].x;
+            const uint32_t b1 = h ? xb[t].w : xb[t].y;
+            mma_bf16_16816(d[t], a, b0, b1);
           }
         }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(smem_u32(empty_bar + stage));
-        if (++stage == S) {
-          stage = 0;
-          phase ^= 1;
-        }
       }
-      if (!ok) break;
-      // add this unit's partial products into the accumulator
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(empty_bar + stage));
+      if (++stage == S) {
+        stage = 0;
+        phase ^= 1;
+      }
+      if (st == nst - 1) {
+        // the unit is complete: add its partial products into the accumulator
 #pragma unroll
-      for (int t = 0; t < NT; ++t) {
-        const int tok = 8 * t + 2 * j;
-        if (tok < p.M) {
-          if (n0 < p.N) red_add_f32(p.acc + (int64_t)tok * p.N + n0, d[t][0]);
-          if (n1 < p.N) red_add_f32(p.acc + (int64_t)tok * p.N + n1, d[t][2]);
-        }
-        if (tok + 1 < p.M) {
-          if (n0 < p.N) red_add_f32(p.acc + (int64_t)(tok + 1) * p.N + n0, d[t][1]);
-          if (n1 < p.N) red_add_f32(p.acc + (int64_t)(tok + 1) * p.N + n1, d[t][3]);
-        }
-      }
-      __threadfence();
-      named_bar_sync(1, 128);
-      if (threadIdx.x == 0) {
-        const unsigned done = atomicAdd(p.counters + rb, 1u);
-        unsigned last = done == (unsigned)p.nks - 1;
-        if (last) {
-          // T must be complete before the LoRA term is added.
-          const uint64_t t0 = globaltimer_ns();
-          while (atomicAdd(p.tdone, 0u) < gridDim.x) {
-            if (globaltimer_ns() - t0 > kWaitLimitNs) {
-              record_error(p.err, DEV_TIMEOUT_EPILOGUE);
-              last = 0;
-              break;
-            }
+        for (int t = 0; t < NT; ++t) {
+          const int tok = 8 * t + 2 * j;
+          if (tok < p.M) {
+            if (n0 < p.N) red_add_f32(p.acc + (int64_t)tok * p.N + n0, d[t][0]);
+            if (n1 < p.N) red_add_f32(p.acc + (int64_t)tok * p.N + n1, d[t][2]);
+          }
+          if (tok + 1 < p.M) {
+            if (n0 < p.N) red_add_f32(p.acc + (int64_t)(tok + 1) * p.N + n0, d[t][1]);
+            if (n1 < p.N) red_add_f32(p.acc + (int64_t)(tok + 1) * p.N + n1, d[t][3]);
           }
         }
-        *flag = last;
-      }
-      named_bar_sync(1, 128);
-      if (*flag) {
         __threadfence();
-        if (!t_loaded) {  // s*T, complete once every CTA has added its slice
-          for (int i = threadIdx.x; i < p.M * p.r; i += 128) t_s[i] = p.s * __ldcg(p.tacc + i);
-          t_loaded = true;
-          named_bar_sync(1, 128);
-        }
-        // Y[tok][n] = bf16(acc + sum_j (s*T)[tok][j] * L2[j][n]) for this 64-row block
-        const int n = rb * kGvRows + (threadIdx.x & 63);
-        const int tok0 = threadIdx.x >> 6;  // 0 or 1: tokens tok0, tok0 + 2, ...
-        if (n < p.N) {
-          float y[4 * NT];
-#pragma unroll
-          for (int i = 0; i < 4 * NT; ++i) y[i] = 0.f;
-          for (int jj = 0; jj < p.r; ++jj) {
-            const float l2 = __bfloat162float(p.L2[(int64_t)jj * p.N + n]);
-#pragma unroll
-            for (int i = 0; i < 4 * NT; ++i) {
-              const int tok = tok0 + 2 * i;
-              if (tok < p.M) y[i] = __fmaf_rn(t_s[tok * p.r + jj], l2, y[i]);
-            }
-          }
-#pragma unroll
-          for (int i = 0; i < 4 * NT; ++i) {
-            const int tok = tok0 + 2 * i;
-            if (tok < p.M)
-              p.Y[(int64_t)tok * p.N + n] = __float2bfloat16_rn(__ldcg(p.acc + (int64_t)tok * p.N + n) + y[i]);
-          }
-        }
+        named_bar_sync(1, 128);
+        if (threadIdx.x == 0) *flag = atomicAdd(p.counters + rb, 1u) == (unsigned)p.nks - 1;
+        named_bar_sync(1, 128);
+        if (*flag) gv_finish<NT>(p, rb, t_s, t_loaded);
       }
+      u = nu;
+      st = nstn;
+      pre = nxt;
+    }
+  }
+}
+
+// Adds the LoRA term to a completed 64-row block of the accumulator and writes
+// Y: Y[tok][n] = bf16(acc[tok][n] + sum_j (s T)[tok][j] L2[j][n]).  Runs on
+// the 128 decode threads of the CTA that completed the block.
+template <int NT>
+__device__ __noinline__ void gv_finish(const GvArgs &p, int rb, float *t_s, bool &t_loaded) {
+  __threadfence();
+  if (!t_loaded) {
+    // T comes from the preceding (programmatic-dependent) launch.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    for (int i = threadIdx.x; i < p.M * p.r; i += 128) t_s[i] = p.s * __ldcg(p.tacc + i);
+    t_loaded = true;
+    named_bar_sync(1, 128);
+  }
+  if (rb == 0 && p.T_save) {
+    for (int i = threadIdx.x; i < p.M * p.r; i += 128) {
+      const float v = t_s[i];
+      const int m = i / p.r, jj = i - m * p.r;
+      const __nv_bfloat16 hb = __float2bfloat16_rn(v);
+      p.T_save[(int64_t)m * 2 * p.r + jj] = hb;
+      p.T_save[(int64_t)m * 2 * p.r + p.r + jj] = __float2bfloat16_rn(v - __bfloat162float(hb));
+    }
+  }
+  const int n = rb * kGvRows + (threadIdx.x & 63);
+  const int tok0 = threadIdx.x >> 6;  // 0 or 1: tokens tok0, tok0 + 2, ...
+  if (n >= p.N) return;
+  float y[4 * NT];
+#pragma unroll
+  for (int i = 0; i < 4 * NT; ++i) {
+    const int tok = tok0 + 2 * i;
+    y[i] = tok < p.M ? __ldcg(p.acc + (int64_t)tok * p.N + n) : 0.f;
+  }
+  for (int j0 = 0; j0 < p.r; j0 += 8) {
+    float l2[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) l2[q] = __bfloat162float(p.L2[(int64_t)(j0 + q) * p.N + n]);
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+#pragma unroll
+      for (int i = 0; i < 4 * NT; ++i) {
+        const int tok = tok0 + 2 * i;
+        if (tok < p.M) y[i] = __fmaf_rn(t_s[tok * p.r + j0 + q], l2[q], y[i]);
+      }
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < 4 * NT; ++i) {
+    const int tok = tok0 + 2 * i;
+    if (tok < p.M) p.Y[(int64_t)tok * p.N + n] = __float2bfloat16_rn(y[i]);
+  }
+}
+
+// T accumulation for few tokens: tacc[M x r] += X[:, k-slice] L1[k-slice, :]
+// for a 64-wide K slice per CTA (blockIdx.x) and a 64-wide column slice
+// (blockIdx.y).  Inputs are staged in shared memory with coalesced loads, then
+// each thread forms 4 tokens x 1 column over the slice and adds it with
+// red.global.add.  Lets its dependent launch start immediately.
+constexpr int kTSliceK = 64;
+
+__global__ void __launch_bounds__(256) lora_down_small_kernel(const __nv_bfloat16 *__restrict__ X,
+                                                              const __nv_bfloat16 *__restrict__ L1, int M, int K,
+                                                              int r, float *__restrict__ tacc) {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  __shared__ float xs[kGvMaxM][kTSliceK + 1];
+  __shared__ float ls[kTSliceK][65];
+  const int k0 = blockIdx.x * kTSliceK;
+  const int kn = min(kTSliceK, K - k0);
+  const int j0 = blockIdx.y * 64;
+  const int jn = min(64, r - j0);
+  for (int i = threadIdx.x; i < kGvMaxM * kTSliceK; i += blockDim.x) {
+    const int m = i / kTSliceK, k = i - m * kTSliceK;
+    xs[m][k] = (m < M && k < kn) ? __bfloat162float(X[(int64_t)m * K + k0 + k]) : 0.f;
+  }
+  for (int i = threadIdx.x; i < kTSliceK * 64; i += blockDim.x) {
+    const int k = i >> 6, jj = i & 63;
+    ls[k][jj] = (k < kn && jj < jn) ? __bfloat162float(L1[(int64_t)(k0 + k) * r + j0 + jj]) : 0.f;
+  }
+  __syncthreads();
+  const int jj = threadIdx.x & 63;
+  for (int m0 = (threadIdx.x >> 6) * 4; m0 < M; m0 += 16) {
+    float t[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int k = 0; k < kn; ++k) {
+      const float l = ls[k][jj];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) t[i] = __fmaf_rn(xs[m0 + i][k], l, t[i]);
+    }
+    if (jj < jn) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        if (m0 + i < M) red_add_f32(tacc + (m0 + i) * r + j0 + jj, t[i]);
     }
   }
 }

@@ -283,9 +283,9 @@ int encode_tmap(CUtensorMap *m, CUtensorMapDataType dt, int rank, const void *pt
   return r == CUDA_SUCCESS ? QLORA_OK : QLORA_ERR_CUDA;
 }
 
-// Workspace of the few-token forward: [acc M*N f32 | tacc M*r f32 | counters | tdone], all zeroed per call.
+// Workspace of the few-token forward: [acc M*N f32 | tacc M*r f32 | counters], all zeroed per call.
 struct GemvLayout {
-  size_t acc, tacc, counters, tdone, zero_bytes, total;
+  size_t acc, tacc, counters, zero_bytes, total;
 };
 
 GemvLayout gemv_layout(int64_t M, int64_t N, int r) {
@@ -293,8 +293,7 @@ GemvLayout gemv_layout(int64_t M, int64_t N, int r) {
   L.acc = 0;
   L.tacc = align_up((size_t)M * N * 4, 16);
   L.counters = L.tacc + align_up((size_t)M * r * 4, 16);
-  L.tdone = L.counters + (size_t)((N + kGvRows - 1) / kGvRows) * 4;
-  L.zero_bytes = L.tdone + 4;
+  L.zero_bytes = L.counters + (size_t)((N + kGvRows - 1) / kGvRows) * 4;
   L.total = align_up(L.zero_bytes);
   return L;
 }
@@ -328,8 +327,6 @@ int launch_gemv(const qlora_nf4dq_t *W, const uint16_t *X, int64_t M, const uint
       return QLORA_ERR_CUDA;
     dev->gemv_smem_set[idx] = smem;
   }
-  // Every CTA must be resident at once: the finishing CTAs wait for all CTAs'
-  // share of T, so the grid never exceeds what fits on the device together.
   int per_sm = 0;
   if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, gemv_fwd_kernel<NT>, kGvThreads, smem) != cudaSuccess ||
       per_sm < 1)
@@ -346,19 +343,35 @@ int launch_gemv(const qlora_nf4dq_t *W, const uint16_t *X, int64_t M, const uint
   a.c2_fp8 = W->c2_fp8;
   a.c1 = W->c1;
   a.mu = W->c2_mean;
-  a.X = reinterpret_cast<const __nv_bfloat16 *>(X);
-  a.L1 = reinterpret_cast<const __nv_bfloat16 *>(L1);
   a.L2 = reinterpret_cast<const __nv_bfloat16 *>(L2);
   a.acc = reinterpret_cast<float *>(ws + L.acc);
   a.tacc = reinterpret_cast<float *>(ws + L.tacc);
   a.counters = reinterpret_cast<unsigned *>(ws + L.counters);
-  a.tdone = reinterpret_cast<unsigned *>(ws + L.tdone);
   a.Y = reinterpret_cast<__nv_bfloat16 *>(Y);
   a.T_save = reinterpret_cast<__nv_bfloat16 *>(T_save);
   a.err = dev->err;
   const int grid = std::max(1, std::min(a.units, per_sm * dev->sms));
   ProfScope prof(QLORA_KERNEL_GEMV_FWD, st);
-  gemv_fwd_kernel<NT><<<grid, kGvThreads, smem, st>>>(tm_codes, tm_x, a);
+  // T accumulation first; the product kernel is its programmatic dependent and
+  // overlaps it, waiting for T only where the LoRA term is added.
+  const dim3 tgrid((unsigned)((K + kTSliceK - 1) / kTSliceK), (unsigned)((r + 63) / 64));
+  lora_down_small_kernel<<<tgrid, 256, 0, st>>>(reinterpret_cast<const __nv_bfloat16 *>(X),
+                                                reinterpret_cast<const __nv_bfloat16 *>(L1), (int)M, (int)K, r,
+                                                a.tacc);
+  int rc = launch_status();
+  if (rc) return rc;
+  cudaLaunchConfig_t cfg;
+  std::memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kGvThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, gemv_fwd_kernel<NT>, tm_codes, tm_x, a) != cudaSuccess) return QLORA_ERR_CUDA;
   return launch_status();
 }
 
