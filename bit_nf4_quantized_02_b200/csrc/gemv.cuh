@@ -52,7 +52,7 @@ struct GvCfg {
   static constexpr int kStageBytes = kCodeBytes + kXBytes;
   static constexpr int kStages = NT == 1 ? 8 : (NT == 2 ? 6 : 4);
   // + 1024 alignment slack + 256 barrier/flag area; the launch adds M*r*4 bytes
-  // for s*T (used by the finisher).
+  // for s*T and r*128 bytes for a 64-column slice of L2 (used by the finisher).
   static constexpr int kSmemBytes = kStages * kStageBytes + 1024 + 256;
 };
 
@@ -168,12 +168,150 @@ struct ConstPrefetch {
 };
 
 template <int NT>
-__device__ __noinline__ void gv_finish(const GvArgs &p, int rb, float *t_s, bool &t_loaded);
+__device__ __forceinline__ bool gv_finish(const GvArgs &p, int rb, float *t_s, bool t_loaded);
+
+// State of one decode/MMA warp of gemv_fwd_kernel.
+template <int NT>
+struct GvConsumer {
+  using Cfg = GvCfg<NT>;
+  const GvArgs *p;
+  uint8_t *smem;
+  uint64_t *full_bar, *empty_bar;
+  unsigned *flag;
+  float *t_s;
+  bool t_loaded;
+  int kblocks, g, j, r0, lane;
+  int stage;
+  uint32_t phase;
+  int u, st;
+  float mu;
+  float d[2][NT][4];  // two accumulator chains (even / odd k-steps)
+
+  __device__ __forceinline__ void init(const GvArgs &pp, uint8_t *sm, uint64_t *fb, uint64_t *eb, unsigned *fl,
+                                       float *ts, int kb) {
+    p = &pp;
+    smem = sm;
+    full_bar = fb;
+    empty_bar = eb;
+    flag = fl;
+    t_s = ts;
+    t_loaded = false;
+    kblocks = kb;
+    lane = lane_id();
+    g = lane >> 2;
+    j = lane & 3;
+    r0 = warp_id() * 16 + g;
+    stage = 0;
+    phase = 0;
+    u = blockIdx.x;
+    st = 0;
+    mu = __ldg(pp.mu);
+  }
+
+  // Process item (u, st) whose constants are in `cur`; start loading the next
+  // item's constants into `nxt`.  Returns false on a pipeline timeout.
+  __device__ __forceinline__ bool item(const ConstPrefetch &cur, ConstPrefetch &nxt) {
+    const GvArgs &P = *p;
+    const int rb = u / P.nks, ks = u - rb * P.nks;
+    const int kbeg = ks * kGvUnitK;
+    const int nst = min(kGvUnitK, P.K - kbeg) > kGvStageK ? 2 : 1;
+    const int n0 = rb * kGvRows + r0, n1 = n0 + 8;
+    if (st == 0) {
+#pragma unroll
+      for (int c = 0; c < 2; ++c)
+#pragma unroll
+        for (int t = 0; t < NT; ++t) d[c][t][0] = d[c][t][1] = d[c][t][2] = d[c][t][3] = 0.f;
+    }
+    BlockTable tb0, tb1;
+    tb0.build(cur.c2hat(0, mu));
+    tb1.build(cur.c2hat(1, mu));
+    int nu = u, nstn = st + 1;
+    if (nstn == nst) {
+      nu = u + gridDim.x;
+      nstn = 0;
+    }
+    nxt.load(P, nu, nstn, r0, j, kblocks);
+    if (!mbar_wait(smem_u32(full_bar + stage), phase, P.err, DEV_TIMEOUT_MMA)) return false;
+    const uint32_t sc = smem_u32(smem + stage * Cfg::kStageBytes);
+    const uint32_t sx = sc + Cfg::kCodeBytes;
+    // codes of rows r0, r0+8: 16-byte chunks 2j, 2j+1 of their 128-byte lines
+    uint32_t q0[8], q1[8];
+    {
+      const uint4 a = lds128(sc + r0 * 128 + (((2 * j) ^ (r0 & 7)) << 4));
+      const uint4 b = lds128(sc + r0 * 128 + (((2 * j + 1) ^ (r0 & 7)) << 4));
+      const uint4 c = lds128(sc + (r0 + 8) * 128 + (((2 * j) ^ (r0 & 7)) << 4));
+      const uint4 e = lds128(sc + (r0 + 8) * 128 + (((2 * j + 1) ^ (r0 & 7)) << 4));
+      q0[0] = a.x; q0[1] = a.y; q0[2] = a.z; q0[3] = a.w; q0[4] = b.x; q0[5] = b.y; q0[6] = b.z; q0[7] = b.w;
+      q1[0] = c.x; q1[1] = c.y; q1[2] = c.z; q1[3] = c.w; q1[4] = e.x; q1[5] = e.y; q1[6] = e.z; q1[7] = e.w;
+    }
+#pragma unroll
+    for (int w = 0; w < 8; ++w) {
+      // X operand for steps 2w, 2w+1: token g + 8t, line (token*4 + j), chunk w
+      uint4 xb[NT];
+#pragma unroll
+      for (int t = 0; t < NT; ++t) {
+        const int line = (g + 8 * t) * 4 + j;
+        xb[t] = lds128(sx + line * 128 + ((w ^ (line & 7)) << 4));
+      }
+      const uint32_t m0 = q0[w] & 0x77777777u, m1 = q1[w] & 0x77777777u;
+      const uint32_t s0 = q0[w] << 4, s1 = q1[w] << 4;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        uint32_t a[4];
+        const uint32_t msel = h ? 0xFBEAu : 0xD9C8u;
+        tb0.lookup4(h ? (m0 >> 16) : m0, prmt(s0, q0[w], msel), a[0], a[2]);
+        tb1.lookup4(h ? (m1 >> 16) : m1, prmt(s1, q1[w], msel), a[1], a[3]);
+#pragma unroll
+        for (int t = 0; t < NT; ++t) {
+          const uint32_t b0 = h ? xb[t].z : xb[t].x;
+          const uint32_t b1 = h ? xb[t].w : xb[t].y;
+          mma_bf16_16816(d[h][t], a, b0, b1);
+        }
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(smem_u32(empty_bar + stage));
+    if (++stage == Cfg::kStages) {
+      stage = 0;
+      phase ^= 1;
+    }
+    if (st == nst - 1) {
+      // the unit is complete: add its partial products into the accumulator
+#pragma unroll
+      for (int t = 0; t < NT; ++t) {
+        const int tok = 8 * t + 2 * j;
+        const float v0 = d[0][t][0] + d[1][t][0], v1 = d[0][t][1] + d[1][t][1];
+        const float v2 = d[0][t][2] + d[1][t][2], v3 = d[0][t][3] + d[1][t][3];
+        if (tok < P.M) {
+          if (n0 < P.N) red_add_f32(P.acc + (int64_t)tok * P.N + n0, v0);
+          if (n1 < P.N) red_add_f32(P.acc + (int64_t)tok * P.N + n1, v2);
+        }
+        if (tok + 1 < P.M) {
+          if (n0 < P.N) red_add_f32(P.acc + (int64_t)(tok + 1) * P.N + n0, v1);
+          if (n1 < P.N) red_add_f32(P.acc + (int64_t)(tok + 1) * P.N + n1, v3);
+        }
+      }
+      // The barrier orders every thread's additions before thread 0's fence
+      // and counter increment (cumulativity); the last of the unit's row
+      // block finishes it.
+      named_bar_sync(1, 128);
+      if (threadIdx.x == 0) {
+        __threadfence();
+        *flag = atomicAdd(P.counters + rb, 1u) == (unsigned)P.nks - 1;
+      }
+      named_bar_sync(1, 128);
+      if (*flag) t_loaded = gv_finish<NT>(P, rb, t_s, t_loaded);
+    }
+    u = nu;
+    st = nstn;
+    return true;
+  }
+};
 
 template <int NT>
 __global__ void __launch_bounds__(kGvThreads, 2)
     gemv_fwd_kernel(const __grid_constant__ CUtensorMap tmCodes, const __grid_constant__ CUtensorMap tmX,
-                    const GvArgs p) {
+                    const __grid_constant__ GvArgs p) {
   using Cfg = GvCfg<NT>;
   constexpr int S = Cfg::kStages;
   extern __shared__ uint8_t smem_raw[];
@@ -199,140 +337,67 @@ __global__ void __launch_bounds__(kGvThreads, 2)
   __syncthreads();
 
   if (warp == 4) {
+    // Lane 0 drives the TMA ring; all lanes prefetch the next stage's block
+    // constants (one code8 run per weight row) into L2 for the decode warps.
     if (lane == 0) {
       tma_prefetch_desc(&tmCodes);
       tma_prefetch_desc(&tmX);
-      int stage = 0;
-      uint32_t phase = 0, used = 0, last_parity = 0;
-      bool ok = true;
-      for (int u = blockIdx.x; u < p.units && ok; u += gridDim.x) {
-        const int rb = u / p.nks, ks = u - rb * p.nks;
-        const int kbeg = ks * kGvUnitK;
-        const int nst = min(kGvUnitK, p.K - kbeg) > kGvStageK ? 2 : 1;
-        for (int st = 0; st < nst; ++st) {
-          if (!mbar_wait(smem_u32(empty_bar + stage), phase ^ 1, p.err, DEV_TIMEOUT_PRODUCER)) {
-            ok = false;
-            break;
-          }
-          const uint32_t fb = smem_u32(full_bar + stage);
-          mbar_arrive_expect_tx(fb, Cfg::kStageBytes);
-          const uint32_t sc = smem_u32(smem + stage * Cfg::kStageBytes);
-          const int k0 = kbeg + st * kGvStageK;
-          tma_load_2d(sc, &tmCodes, fb, k0 >> 1, rb * kGvRows);
-          asm volatile(
-              "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5}], "
-              "[%2];" ::"r"(sc + Cfg::kCodeBytes),
-              "l"(reinterpret_cast<uint64_t>(&tmX)), "r"(fb), "r"(0), "r"(k0 >> 6), "r"(0)
-              : "memory");
-          used |= 1u << stage;
-          last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
-          if (++stage == S) {
-            stage = 0;
-            phase ^= 1;
-          }
-        }
-      }
-      for (int i = 0; i < S; ++i)
-        if (used & (1u << i)) mbar_wait(smem_u32(full_bar + i), (last_parity >> i) & 1u, p.err, DEV_TIMEOUT_DRAIN);
     }
-  } else {
-    const int g = lane >> 2, j = lane & 3;
-    const int r0 = warp * 16 + g;  // row of this lane inside the unit (and r0 + 8)
-    const float mu = __ldg(p.mu);
     int stage = 0;
-    uint32_t phase = 0;
-    // Flat walk over this CTA's (unit, stage) items; the block constants of
-    // the next item are loaded one item ahead so their latency hides under
-    // the current item's decode.
-    int u = blockIdx.x, st = 0;
-    ConstPrefetch pre, nxt;
-    pre.load(p, u, st, r0, j, kblocks);
-    float d[NT][4];
-    while (u < p.units) {
+    uint32_t phase = 0, used = 0, last_parity = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; u < p.units && ok; u += gridDim.x) {
       const int rb = u / p.nks, ks = u - rb * p.nks;
       const int kbeg = ks * kGvUnitK;
       const int nst = min(kGvUnitK, p.K - kbeg) > kGvStageK ? 2 : 1;
-      const int n0 = rb * kGvRows + r0, n1 = n0 + 8;
-      if (st == 0) {
 #pragma unroll
-        for (int t = 0; t < NT; ++t) d[t][0] = d[t][1] = d[t][2] = d[t][3] = 0.f;
+      for (int i = 0; i < 2; ++i) {
+        const int n = rb * kGvRows + lane + 32 * i;
+        if (n < p.N) asm volatile("prefetch.global.L2 [%0];" ::"l"(p.c2_fp8 + (int64_t)n * kblocks + (kbeg >> 6)));
       }
-      BlockTable tb0, tb1;
-      tb0.build(pre.c2hat(0, mu));
-      tb1.build(pre.c2hat(1, mu));
-      int nu = u, nstn = st + 1;
-      if (nstn == nst) {
-        nu = u + gridDim.x;
-        nstn = 0;
-      }
-      nxt.load(p, nu, nstn, r0, j, kblocks);
-      if (!mbar_wait(smem_u32(full_bar + stage), phase, p.err, DEV_TIMEOUT_MMA)) break;
-      const uint32_t sc = smem_u32(smem + stage * Cfg::kStageBytes);
-      const uint32_t sx = sc + Cfg::kCodeBytes;
-      // codes of rows r0, r0+8: 16-byte chunks 2j, 2j+1 of their 128-byte lines
-      uint32_t q0[8], q1[8];
-      {
-        const uint4 a = lds128(sc + r0 * 128 + (((2 * j) ^ (r0 & 7)) << 4));
-        const uint4 b = lds128(sc + r0 * 128 + (((2 * j + 1) ^ (r0 & 7)) << 4));
-        const uint4 c = lds128(sc + (r0 + 8) * 128 + (((2 * j) ^ (r0 & 7)) << 4));
-        const uint4 e = lds128(sc + (r0 + 8) * 128 + (((2 * j + 1) ^ (r0 & 7)) << 4));
-        q0[0] = a.x; q0[1] = a.y; q0[2] = a.z; q0[3] = a.w; q0[4] = b.x; q0[5] = b.y; q0[6] = b.z; q0[7] = b.w;
-        q1[0] = c.x; q1[1] = c.y; q1[2] = c.z; q1[3] = c.w; q1[4] = e.x; q1[5] = e.y; q1[6] = e.z; q1[7] = e.w;
-      }
-#pragma unroll
-      for (int w = 0; w < 8; ++w) {
-        // X operand for steps 2w, 2w+1: token g + 8t, line (token*4 + j), chunk w
-        uint4 xb[NT];
-#pragma unroll
-        for (int t = 0; t < NT; ++t) {
-          const int line = (g + 8 * t) * 4 + j;
-          xb[t] = lds128(sx + line * 128 + ((w ^ (line & 7)) << 4));
-        }
-        const uint32_t m0 = q0[w] & 0x77777777u, m1 = q1[w] & 0x77777777u;
-        const uint32_t s0 = q0[w] << 4, s1 = q1[w] << 4;
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          uint32_t a[4];
-          const uint32_t msel = h ? 0xFBEAu : 0xD9C8u;
-          tb0.lookup4(h ? (m0 >> 16) : m0, prmt(s0, q0[w], msel), a[0], a[2]);
-          tb1.lookup4(h ? (m1 >> 16) : m1, prmt(s1, q1[w], msel), a[1], a[3]);
-#pragma unroll
-          for (int t = 0; t < NT; ++t) {
-            const uint32_t b0 = h ? xb[t].z : xb[t].x;
-            const uint32_t b1 = h ? xb[t].w : xb[t].y;
-            mma_bf16_16816(d[t], a, b0, b1);
+      for (int st = 0; st < nst; ++st) {
+        bool got = true;
+        if (lane == 0) {
+          got = mbar_wait(smem_u32(empty_bar + stage), phase ^ 1, p.err, DEV_TIMEOUT_PRODUCER);
+          if (got) {
+            const uint32_t fb = smem_u32(full_bar + stage);
+            mbar_arrive_expect_tx(fb, Cfg::kStageBytes);
+            const uint32_t sc = smem_u32(smem + stage * Cfg::kStageBytes);
+            const int k0 = kbeg + st * kGvStageK;
+            tma_load_2d(sc, &tmCodes, fb, k0 >> 1, rb * kGvRows);
+            asm volatile(
+                "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, "
+                "%5}], [%2];" ::"r"(sc + Cfg::kCodeBytes),
+                "l"(reinterpret_cast<uint64_t>(&tmX)), "r"(fb), "r"(0), "r"(k0 >> 6), "r"(0)
+                : "memory");
+            used |= 1u << stage;
+            last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
           }
         }
-      }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(empty_bar + stage));
-      if (++stage == S) {
-        stage = 0;
-        phase ^= 1;
-      }
-      if (st == nst - 1) {
-        // the unit is complete: add its partial products into the accumulator
-#pragma unroll
-        for (int t = 0; t < NT; ++t) {
-          const int tok = 8 * t + 2 * j;
-          if (tok < p.M) {
-            if (n0 < p.N) red_add_f32(p.acc + (int64_t)tok * p.N + n0, d[t][0]);
-            if (n1 < p.N) red_add_f32(p.acc + (int64_t)tok * p.N + n1, d[t][2]);
-          }
-          if (tok + 1 < p.M) {
-            if (n0 < p.N) red_add_f32(p.acc + (int64_t)(tok + 1) * p.N + n0, d[t][1]);
-            if (n1 < p.N) red_add_f32(p.acc + (int64_t)(tok + 1) * p.N + n1, d[t][3]);
-          }
+        if (!__shfl_sync(0xFFFFFFFFu, got ? 1 : 0, 0)) {
+          ok = false;
+          break;
         }
-        __threadfence();
-        named_bar_sync(1, 128);
-        if (threadIdx.x == 0) *flag = atomicAdd(p.counters + rb, 1u) == (unsigned)p.nks - 1;
-        named_bar_sync(1, 128);
-        if (*flag) gv_finish<NT>(p, rb, t_s, t_loaded);
+        if (++stage == S) {
+          stage = 0;
+          phase ^= 1;
+        }
       }
-      u = nu;
-      st = nstn;
-      pre = nxt;
+    }
+    if (lane == 0)
+      for (int i = 0; i < S; ++i)
+        if (used & (1u << i)) mbar_wait(smem_u32(full_bar + i), (last_parity >> i) & 1u, p.err, DEV_TIMEOUT_DRAIN);
+  } else {
+    GvConsumer<NT> c;
+    c.init(p, smem, full_bar, empty_bar, flag, t_s, kblocks);
+    // Flat walk over this CTA's (unit, stage) items, unrolled by two so the
+    // block constants of the next item load into the other buffer (no copies
+    // of in-flight loads) while the current item is decoded.
+    ConstPrefetch pa, pb;
+    pa.load(p, c.u, c.st, c.r0, c.j, kblocks);
+    while (c.u < p.units) {
+      if (!c.item(pa, pb)) break;
+      if (c.u >= p.units || !c.item(pb, pa)) break;
     }
   }
 }
@@ -341,7 +406,7 @@ __global__ void __launch_bounds__(kGvThreads, 2)
 // Y: Y[tok][n] = bf16(acc[tok][n] + sum_j (s T)[tok][j] L2[j][n]).  Runs on
 // the 128 decode threads of the CTA that completed the block.
 template <int NT>
-__device__ __noinline__ void gv_finish(const GvArgs &p, int rb, float *t_s, bool &t_loaded) {
+__device__ __forceinline__ bool gv_finish(const GvArgs &p, int rb, float *t_s, bool t_loaded) {
   __threadfence();
   if (!t_loaded) {
     // T comes from the preceding (programmatic-dependent) launch.
@@ -359,33 +424,42 @@ __device__ __noinline__ void gv_finish(const GvArgs &p, int rb, float *t_s, bool
       p.T_save[(int64_t)m * 2 * p.r + p.r + jj] = __float2bfloat16_rn(v - __bfloat162float(hb));
     }
   }
-  const int n = rb * kGvRows + (threadIdx.x & 63);
-  const int tok0 = threadIdx.x >> 6;  // 0 or 1: tokens tok0, tok0 + 2, ...
-  if (n >= p.N) return;
-  float y[4 * NT];
-#pragma unroll
-  for (int i = 0; i < 4 * NT; ++i) {
-    const int tok = tok0 + 2 * i;
-    y[i] = tok < p.M ? __ldcg(p.acc + (int64_t)tok * p.N + n) : 0.f;
+  // stage this block's 64 columns of L2 (r rows x 128 B) with one round of loads
+  __nv_bfloat16 *l2s = reinterpret_cast<__nv_bfloat16 *>(t_s + p.M * p.r);
+  const int nb = rb * kGvRows;
+  const int ncols = min(kGvRows, p.N - nb);
+  for (int i = threadIdx.x; i < p.r * 8; i += 128) {
+    const int jj = i >> 3, c = i & 7;  // 16-byte chunk c of row jj
+    uint4 v = make_uint4(0, 0, 0, 0);
+    if (8 * c < ncols) v = __ldg(reinterpret_cast<const uint4 *>(p.L2 + (int64_t)jj * p.N + nb) + c);
+    reinterpret_cast<uint4 *>(l2s + jj * kGvRows)[c] = v;
   }
-  for (int j0 = 0; j0 < p.r; j0 += 8) {
-    float l2[8];
+  named_bar_sync(1, 128);
+  const int n = nb + (threadIdx.x & 63);
+  const int tok0 = threadIdx.x >> 6;  // 0 or 1: tokens tok0, tok0 + 2, ...
+  if (n < p.N) {
+    float y[4 * NT];
 #pragma unroll
-    for (int q = 0; q < 8; ++q) l2[q] = __bfloat162float(p.L2[(int64_t)(j0 + q) * p.N + n]);
-#pragma unroll
-    for (int q = 0; q < 8; ++q) {
+    for (int i = 0; i < 4 * NT; ++i) {
+      const int tok = tok0 + 2 * i;
+      y[i] = tok < p.M ? __ldcg(p.acc + (int64_t)tok * p.N + n) : 0.f;
+    }
+    for (int jj = 0; jj < p.r; ++jj) {
+      const float l2 = __bfloat162float(l2s[jj * kGvRows + (threadIdx.x & 63)]);
 #pragma unroll
       for (int i = 0; i < 4 * NT; ++i) {
         const int tok = tok0 + 2 * i;
-        if (tok < p.M) y[i] = __fmaf_rn(t_s[tok * p.r + j0 + q], l2[q], y[i]);
+        if (tok < p.M) y[i] = __fmaf_rn(t_s[tok * p.r + jj], l2, y[i]);
       }
     }
-  }
 #pragma unroll
-  for (int i = 0; i < 4 * NT; ++i) {
-    const int tok = tok0 + 2 * i;
-    if (tok < p.M) p.Y[(int64_t)tok * p.N + n] = __float2bfloat16_rn(y[i]);
+    for (int i = 0; i < 4 * NT; ++i) {
+      const int tok = tok0 + 2 * i;
+      if (tok < p.M) p.Y[(int64_t)tok * p.N + n] = __float2bfloat16_rn(y[i]);
+    }
   }
+  named_bar_sync(1, 128);  // l2s is reused by the next finish
+  return t_loaded;
 }
 
 // T accumulation for few tokens: tacc[M x r] += X[:, k-slice] L1[k-slice, :]

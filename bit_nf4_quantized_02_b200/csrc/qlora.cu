@@ -320,7 +320,7 @@ int launch_gemv(const qlora_nf4dq_t *W, const uint16_t *X, int64_t M, const uint
     int rc = encode_tmap(&tm_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, X, dims, strides, box);
     if (rc) return rc;
   }
-  const int smem = Cfg::kSmemBytes + (int)(M * r * 4);
+  const int smem = Cfg::kSmemBytes + (int)(M * r * 4) + r * kGvRows * 2;
   const int idx = NT == 1 ? 0 : (NT == 2 ? 1 : 2);
   if (dev->gemv_smem_set[idx] < smem) {
     if (cudaFuncSetAttribute(gemv_fwd_kernel<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
