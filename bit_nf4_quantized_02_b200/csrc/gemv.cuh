@@ -5,10 +5,13 @@
 //
 //   Y[M x N] = bf16( X W_hat^T + (s X L1) L2 ),   M <= 8*NT (NT in {1, 2, 4})
 //
-// Two launches per linear: lora_down_small_kernel adds K-slices of X L1 into
-// an fp32 accumulator; gemv_fwd_kernel is launched as its programmatic
-// dependent, so it streams the weight concurrently and only its finishing
-// CTAs wait (griddepcontrol.wait) for T before adding the LoRA term.
+// Three launches per linear, chained with programmatic dependent launch:
+//   lora_down_small_kernel   adds K-slices of X L1 into an fp32 accumulator;
+//   gemv_fwd_kernel          streams the weight and adds X W_hat^T into an fp32
+//                            [M x N] accumulator (does not need T, so it
+//                            overlaps the first kernel completely);
+//   gemv_epilogue_kernel     Y = bf16(acc + s T L2), and T = s X L1 as a bf16
+//                            hi/lo pair for the backward.
 // gemv_fwd_kernel, persistent, 160 threads per CTA (2 CTAs per SM):
 //   * warp 4 is a TMA producer: per stage, 64 weight rows x 256 K of packed
 //     codes (128-byte swizzle) and the matching X tile (3-D view of X,
@@ -25,13 +28,11 @@
 //     operand is one 16-byte run per two steps; both are bank-conflict free
 //     under the 128-byte swizzle.
 //   * A unit is 64 rows x 512 K; partial products are added into an fp32
-//     [M x N] accumulator with red.global.add (L2 resident).  The CTA that
-//     completes a 64-row block (counter) waits for T, adds s T L2 and writes
-//     Y; the finisher of row block 0 also writes T = s X L1 as a bf16 hi/lo
-//     pair for the backward.
-// The accumulator, counters and T accumulator must be zero at launch (the
-// host clears them with one memset in stream order).  Split-K additions make
-// the low bits of Y depend on the order in which CTAs finish.
+//     [M x N] accumulator with red.global.add (L2 resident); all CTAs do the
+//     same amount of work (no per-block finishing step on the critical path).
+// The two accumulators must be zero at launch (the host clears them with one
+// memset in stream order).  Split-K additions make the low bits of Y depend
+// on the order in which CTAs finish.
 #pragma once
 
 #include "common.cuh"
@@ -51,8 +52,7 @@ struct GvCfg {
   static constexpr int kXBytes = 8 * NT * kGvStageK * 2;    // padded tokens x 256 bf16
   static constexpr int kStageBytes = kCodeBytes + kXBytes;
   static constexpr int kStages = NT == 1 ? 8 : (NT == 2 ? 6 : 4);
-  // + 1024 alignment slack + 256 barrier/flag area; the launch adds M*r*4 bytes
-  // for s*T and r*128 bytes for a 64-column slice of L2 (used by the finisher).
+  // + 1024 alignment slack + 256 barrier area
   static constexpr int kSmemBytes = kStages * kStageBytes + 1024 + 256;
 };
 
@@ -68,10 +68,6 @@ struct GvArgs {
   const __nv_bfloat16 *L1;   // [K x r]
   const __nv_bfloat16 *L2;   // [r x N]
   float *acc;            // [M x N] fp32, zero at launch
-  float *tacc;           // [M x r] fp32 (unscaled X L1), zero at launch
-  unsigned *counters;    // [ceil(N/64)], zero at launch
-  __nv_bfloat16 *Y;      // [M x N]
-  __nv_bfloat16 *T_save; // [M x 2r] hi/lo or nullptr
   int *err;
 };
 
@@ -100,6 +96,10 @@ __device__ __forceinline__ uint4 lds128(uint32_t addr) {
 __device__ __forceinline__ void red_add_f32(float *p, float v) {
   asm volatile("red.global.add.f32 [%0], %1;" ::"l"(p), "f"(v) : "memory");
 }
+
+// Release/acquire fence at GPU scope (lighter than the sequentially
+// consistent fence of __threadfence()).
+__device__ __forceinline__ void fence_acq_rel_gpu() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
 
 __device__ __forceinline__ void named_bar_sync(int id, int n) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
@@ -167,9 +167,6 @@ struct ConstPrefetch {
   }
 };
 
-template <int NT>
-__device__ __forceinline__ bool gv_finish(const GvArgs &p, int rb, float *t_s, bool t_loaded);
-
 // State of one decode/MMA warp of gemv_fwd_kernel.
 template <int NT>
 struct GvConsumer {
@@ -177,9 +174,6 @@ struct GvConsumer {
   const GvArgs *p;
   uint8_t *smem;
   uint64_t *full_bar, *empty_bar;
-  unsigned *flag;
-  float *t_s;
-  bool t_loaded;
   int kblocks, g, j, r0, lane;
   int stage;
   uint32_t phase;
@@ -187,15 +181,11 @@ struct GvConsumer {
   float mu;
   float d[2][NT][4];  // two accumulator chains (even / odd k-steps)
 
-  __device__ __forceinline__ void init(const GvArgs &pp, uint8_t *sm, uint64_t *fb, uint64_t *eb, unsigned *fl,
-                                       float *ts, int kb) {
+  __device__ __forceinline__ void init(const GvArgs &pp, uint8_t *sm, uint64_t *fb, uint64_t *eb, int kb) {
     p = &pp;
     smem = sm;
     full_bar = fb;
     empty_bar = eb;
-    flag = fl;
-    t_s = ts;
-    t_loaded = false;
     kblocks = kb;
     lane = lane_id();
     g = lane >> 2;
@@ -291,16 +281,6 @@ struct GvConsumer {
           if (n1 < P.N) red_add_f32(P.acc + (int64_t)(tok + 1) * P.N + n1, v3);
         }
       }
-      // The barrier orders every thread's additions before thread 0's fence
-      // and counter increment (cumulativity); the last of the unit's row
-      // block finishes it.
-      named_bar_sync(1, 128);
-      if (threadIdx.x == 0) {
-        __threadfence();
-        *flag = atomicAdd(P.counters + rb, 1u) == (unsigned)P.nks - 1;
-      }
-      named_bar_sync(1, 128);
-      if (*flag) t_loaded = gv_finish<NT>(P, rb, t_s, t_loaded);
     }
     u = nu;
     st = nstn;
@@ -318,13 +298,11 @@ __global__ void __launch_bounds__(kGvThreads, 2)
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t *full_bar = reinterpret_cast<uint64_t *>(smem + S * Cfg::kStageBytes);
   uint64_t *empty_bar = full_bar + S;
-  unsigned *flag = reinterpret_cast<unsigned *>(empty_bar + S);
-  float *t_s = reinterpret_cast<float *>(smem + S * Cfg::kStageBytes + 256);  // [M x r] s*T
-  bool t_loaded = false;
 
   const int warp = warp_id();
   const int lane = lane_id();
   const int kblocks = p.K >> 6;
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");  // the epilogue may launch and wait
 
   // ---------------------------------------------------------------- main loop
   if (threadIdx.x == 0) {
@@ -389,7 +367,7 @@ __global__ void __launch_bounds__(kGvThreads, 2)
         if (used & (1u << i)) mbar_wait(smem_u32(full_bar + i), (last_parity >> i) & 1u, p.err, DEV_TIMEOUT_DRAIN);
   } else {
     GvConsumer<NT> c;
-    c.init(p, smem, full_bar, empty_bar, flag, t_s, kblocks);
+    c.init(p, smem, full_bar, empty_bar, kblocks);
     // Flat walk over this CTA's (unit, stage) items, unrolled by two so the
     // block constants of the next item load into the other buffer (no copies
     // of in-flight loads) while the current item is decoded.
@@ -400,66 +378,9 @@ __global__ void __launch_bounds__(kGvThreads, 2)
       if (c.u >= p.units || !c.item(pb, pa)) break;
     }
   }
-}
-
-// Adds the LoRA term to a completed 64-row block of the accumulator and writes
-// Y: Y[tok][n] = bf16(acc[tok][n] + sum_j (s T)[tok][j] L2[j][n]).  Runs on
-// the 128 decode threads of the CTA that completed the block.
-template <int NT>
-__device__ __forceinline__ bool gv_finish(const GvArgs &p, int rb, float *t_s, bool t_loaded) {
-  __threadfence();
-  if (!t_loaded) {
-    // T comes from the preceding (programmatic-dependent) launch.
-    asm volatile("griddepcontrol.wait;" ::: "memory");
-    for (int i = threadIdx.x; i < p.M * p.r; i += 128) t_s[i] = p.s * __ldcg(p.tacc + i);
-    t_loaded = true;
-    named_bar_sync(1, 128);
-  }
-  if (rb == 0 && p.T_save) {
-    for (int i = threadIdx.x; i < p.M * p.r; i += 128) {
-      const float v = t_s[i];
-      const int m = i / p.r, jj = i - m * p.r;
-      const __nv_bfloat16 hb = __float2bfloat16_rn(v);
-      p.T_save[(int64_t)m * 2 * p.r + jj] = hb;
-      p.T_save[(int64_t)m * 2 * p.r + p.r + jj] = __float2bfloat16_rn(v - __bfloat162float(hb));
-    }
-  }
-  // stage this block's 64 columns of L2 (r rows x 128 B) with one round of loads
-  __nv_bfloat16 *l2s = reinterpret_cast<__nv_bfloat16 *>(t_s + p.M * p.r);
-  const int nb = rb * kGvRows;
-  const int ncols = min(kGvRows, p.N - nb);
-  for (int i = threadIdx.x; i < p.r * 8; i += 128) {
-    const int jj = i >> 3, c = i & 7;  // 16-byte chunk c of row jj
-    uint4 v = make_uint4(0, 0, 0, 0);
-    if (8 * c < ncols) v = __ldg(reinterpret_cast<const uint4 *>(p.L2 + (int64_t)jj * p.N + nb) + c);
-    reinterpret_cast<uint4 *>(l2s + jj * kGvRows)[c] = v;
-  }
-  named_bar_sync(1, 128);
-  const int n = nb + (threadIdx.x & 63);
-  const int tok0 = threadIdx.x >> 6;  // 0 or 1: tokens tok0, tok0 + 2, ...
-  if (n < p.N) {
-    float y[4 * NT];
-#pragma unroll
-    for (int i = 0; i < 4 * NT; ++i) {
-      const int tok = tok0 + 2 * i;
-      y[i] = tok < p.M ? __ldcg(p.acc + (int64_t)tok * p.N + n) : 0.f;
-    }
-    for (int jj = 0; jj < p.r; ++jj) {
-      const float l2 = __bfloat162float(l2s[jj * kGvRows + (threadIdx.x & 63)]);
-#pragma unroll
-      for (int i = 0; i < 4 * NT; ++i) {
-        const int tok = tok0 + 2 * i;
-        if (tok < p.M) y[i] = __fmaf_rn(t_s[tok * p.r + jj], l2, y[i]);
-      }
-    }
-#pragma unroll
-    for (int i = 0; i < 4 * NT; ++i) {
-      const int tok = tok0 + 2 * i;
-      if (tok < p.M) p.Y[(int64_t)tok * p.N + n] = __float2bfloat16_rn(y[i]);
-    }
-  }
-  named_bar_sync(1, 128);  // l2s is reused by the next finish
-  return t_loaded;
+  // Complete only after the T launch this grid overlapped has completed, so
+  // that the epilogue launched after this grid sees T.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
 // T accumulation for few tokens: tacc[M x r] += X[:, k-slice] L1[k-slice, :]
@@ -502,6 +423,48 @@ __global__ void __launch_bounds__(256) lora_down_small_kernel(const __nv_bfloat1
         if (m0 + i < M) red_add_f32(tacc + (m0 + i) * r + j0 + jj, t[i]);
     }
   }
+}
+
+// Y[tok][n] = bf16(acc[tok][n] + sum_j (s T)[tok][j] L2[j][n]) for one column
+// per thread; the block with blockIdx.x == 0 also writes T = s X L1 as a bf16
+// hi/lo pair.  Launched as a programmatic dependent of gemv_fwd_kernel: it
+// stages s T and then waits for the accumulator.
+__global__ void __launch_bounds__(256) gemv_epilogue_kernel(const float *__restrict__ acc,
+                                                            const float *__restrict__ tacc,
+                                                            const __nv_bfloat16 *__restrict__ L2, int M, int N, int r,
+                                                            float s, __nv_bfloat16 *__restrict__ Y,
+                                                            __nv_bfloat16 *__restrict__ T_save) {
+  extern __shared__ float ts[];  // [M x r]
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  for (int i = threadIdx.x; i < M * r; i += blockDim.x) ts[i] = s * tacc[i];
+  __syncthreads();
+  if (blockIdx.x == 0 && T_save) {
+    for (int i = threadIdx.x; i < M * r; i += blockDim.x) {
+      const float v = ts[i];
+      const int m = i / r, jj = i - m * r;
+      const __nv_bfloat16 hb = __float2bfloat16_rn(v);
+      T_save[(int64_t)m * 2 * r + jj] = hb;
+      T_save[(int64_t)m * 2 * r + r + jj] = __float2bfloat16_rn(v - __bfloat162float(hb));
+    }
+  }
+  const int n = blockIdx.x * blockDim.x + threadIdx.x;
+  if (n >= N) return;
+  float y[kGvMaxM];
+#pragma unroll
+  for (int m = 0; m < kGvMaxM; ++m) y[m] = m < M ? acc[(int64_t)m * N + n] : 0.f;
+  for (int j0 = 0; j0 < r; j0 += 8) {
+    float l2[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) l2[q] = __bfloat162float(L2[(int64_t)(j0 + q) * N + n]);
+#pragma unroll
+    for (int q = 0; q < 8; ++q)
+#pragma unroll
+      for (int m = 0; m < kGvMaxM; ++m)
+        if (m < M) y[m] = __fmaf_rn(ts[m * r + j0 + q], l2[q], y[m]);
+  }
+#pragma unroll
+  for (int m = 0; m < kGvMaxM; ++m)
+    if (m < M) Y[(int64_t)m * N + n] = __float2bfloat16_rn(y[m]);
 }
 
 }  // namespace qlora

@@ -283,19 +283,36 @@ int encode_tmap(CUtensorMap *m, CUtensorMapDataType dt, int rank, const void *pt
   return r == CUDA_SUCCESS ? QLORA_OK : QLORA_ERR_CUDA;
 }
 
-// Workspace of the few-token forward: [acc M*N f32 | tacc M*r f32 | counters], all zeroed per call.
+// Workspace of the few-token forward: [acc M*N f32 | tacc M*r f32], zeroed per call.
 struct GemvLayout {
-  size_t acc, tacc, counters, zero_bytes, total;
+  size_t acc, tacc, zero_bytes, total;
 };
 
 GemvLayout gemv_layout(int64_t M, int64_t N, int r) {
   GemvLayout L;
   L.acc = 0;
   L.tacc = align_up((size_t)M * N * 4, 16);
-  L.counters = L.tacc + align_up((size_t)M * r * 4, 16);
-  L.zero_bytes = L.counters + (size_t)((N + kGvRows - 1) / kGvRows) * 4;
+  L.zero_bytes = L.tacc + (size_t)M * r * 4;
   L.total = align_up(L.zero_bytes);
   return L;
+}
+
+// Launch `kernel` on `st` as a programmatic dependent of the previous launch.
+template <typename... KArgs, typename... Args>
+int launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, Args... args) {
+  cudaLaunchConfig_t cfg;
+  std::memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kernel, args...) != cudaSuccess) return QLORA_ERR_CUDA;
+  return launch_status();
 }
 
 template <int NT>
@@ -320,7 +337,7 @@ int launch_gemv(const qlora_nf4dq_t *W, const uint16_t *X, int64_t M, const uint
     int rc = encode_tmap(&tm_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, X, dims, strides, box);
     if (rc) return rc;
   }
-  const int smem = Cfg::kSmemBytes + (int)(M * r * 4) + r * kGvRows * 2;
+  const int smem = Cfg::kSmemBytes;
   const int idx = NT == 1 ? 0 : (NT == 2 ? 1 : 2);
   if (dev->gemv_smem_set[idx] < smem) {
     if (cudaFuncSetAttribute(gemv_fwd_kernel<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
@@ -345,34 +362,25 @@ int launch_gemv(const qlora_nf4dq_t *W, const uint16_t *X, int64_t M, const uint
   a.mu = W->c2_mean;
   a.L2 = reinterpret_cast<const __nv_bfloat16 *>(L2);
   a.acc = reinterpret_cast<float *>(ws + L.acc);
-  a.tacc = reinterpret_cast<float *>(ws + L.tacc);
-  a.counters = reinterpret_cast<unsigned *>(ws + L.counters);
-  a.Y = reinterpret_cast<__nv_bfloat16 *>(Y);
-  a.T_save = reinterpret_cast<__nv_bfloat16 *>(T_save);
   a.err = dev->err;
+  float *tacc = reinterpret_cast<float *>(ws + L.tacc);
   const int grid = std::max(1, std::min(a.units, per_sm * dev->sms));
   ProfScope prof(QLORA_KERNEL_GEMV_FWD, st);
-  // T accumulation first; the product kernel is its programmatic dependent and
-  // overlaps it, waiting for T only where the LoRA term is added.
+  // 1. T accumulation; 2. the product, overlapping it; 3. the LoRA epilogue.
   const dim3 tgrid((unsigned)((K + kTSliceK - 1) / kTSliceK), (unsigned)((r + 63) / 64));
   lora_down_small_kernel<<<tgrid, 256, 0, st>>>(reinterpret_cast<const __nv_bfloat16 *>(X),
-                                                reinterpret_cast<const __nv_bfloat16 *>(L1), (int)M, (int)K, r,
-                                                a.tacc);
+                                                reinterpret_cast<const __nv_bfloat16 *>(L1), (int)M, (int)K, r, tacc);
   int rc = launch_status();
   if (rc) return rc;
-  cudaLaunchConfig_t cfg;
-  std::memset(&cfg, 0, sizeof(cfg));
-  cfg.gridDim = dim3(grid);
-  cfg.blockDim = dim3(kGvThreads);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, gemv_fwd_kernel<NT>, tm_codes, tm_x, a) != cudaSuccess) return QLORA_ERR_CUDA;
-  return launch_status();
+  rc = launch_pdl(gemv_fwd_kernel<NT>, dim3(grid), dim3(kGvThreads), (size_t)smem, st, tm_codes, tm_x, a);
+  if (rc) return rc;
+  const size_t esmem = (size_t)M * r * 4;
+  if (esmem > 48 * 1024 &&
+      cudaFuncSetAttribute(gemv_epilogue_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)esmem) != cudaSuccess)
+    return QLORA_ERR_CUDA;
+  return launch_pdl(gemv_epilogue_kernel, dim3((unsigned)((N + 255) / 256)), dim3(256), esmem, st,
+                    (const float *)a.acc, (const float *)tacc, a.L2, (int)M, (int)N, r, s,
+                    reinterpret_cast<__nv_bfloat16 *>(Y), reinterpret_cast<__nv_bfloat16 *>(T_save));
 }
 
 struct FwdLayout {
