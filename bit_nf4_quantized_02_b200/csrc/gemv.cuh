@@ -12,7 +12,7 @@
 //                            overlaps the first kernel completely);
 //   gemv_epilogue_kernel     Y = bf16(acc + s T L2), and T = s X L1 as a bf16
 //                            hi/lo pair for the backward.
-// gemv_fwd_kernel, persistent, 160 threads per CTA (2 CTAs per SM):
+// gemv_fwd_kernel, persistent, 160 threads per CTA (3 CTAs per SM):
 //   * warp 4 is a TMA producer: per stage, 64 weight rows x 256 K of packed
 //     codes (128-byte swizzle) and the matching X tile (3-D view of X,
 //     [token][64-block][64], 128-byte swizzle) into a ring of mbarrier stages;
@@ -51,7 +51,7 @@ struct GvCfg {
   static constexpr int kCodeBytes = kGvRows * 128;          // 64 rows x 256 codes
   static constexpr int kXBytes = 8 * NT * kGvStageK * 2;    // padded tokens x 256 bf16
   static constexpr int kStageBytes = kCodeBytes + kXBytes;
-  static constexpr int kStages = NT == 1 ? 8 : (NT == 2 ? 6 : 4);
+  static constexpr int kStages = NT == 1 ? 5 : (NT == 2 ? 4 : 3);   // ~64 KB: 3 CTAs per SM
   // + 1024 alignment slack + 256 barrier area
   static constexpr int kSmemBytes = kStages * kStageBytes + 1024 + 256;
 };
@@ -289,7 +289,7 @@ struct GvConsumer {
 };
 
 template <int NT>
-__global__ void __launch_bounds__(kGvThreads, 2)
+__global__ void __launch_bounds__(kGvThreads, 3)
     gemv_fwd_kernel(const __grid_constant__ CUtensorMap tmCodes, const __grid_constant__ CUtensorMap tmX,
                     const __grid_constant__ GvArgs p) {
   using Cfg = GvCfg<NT>;
@@ -425,18 +425,29 @@ __global__ void __launch_bounds__(256) lora_down_small_kernel(const __nv_bfloat1
   }
 }
 
-// Y[tok][n] = bf16(acc[tok][n] + sum_j (s T)[tok][j] L2[j][n]) for one column
-// per thread; the block with blockIdx.x == 0 also writes T = s X L1 as a bf16
-// hi/lo pair.  Launched as a programmatic dependent of gemv_fwd_kernel: it
-// stages s T and then waits for the accumulator.
+// Y[tok][n] = bf16(acc[tok][n] + sum_j (s T)[tok][j] L2[j][n]).  A CTA owns 64
+// columns: it stages their L2 slice (r x 64) before waiting for the product
+// kernel (L2 is an input), then s T, then thread (column c, token group q)
+// forms tokens q, q+4, q+8, ...  Block 0 also writes T = s X L1 as a bf16
+// hi/lo pair.  Launched as a programmatic dependent of gemv_fwd_kernel.
 __global__ void __launch_bounds__(256) gemv_epilogue_kernel(const float *__restrict__ acc,
                                                             const float *__restrict__ tacc,
                                                             const __nv_bfloat16 *__restrict__ L2, int M, int N, int r,
                                                             float s, __nv_bfloat16 *__restrict__ Y,
                                                             __nv_bfloat16 *__restrict__ T_save) {
-  extern __shared__ float ts[];  // [M x r]
+  extern __shared__ float esm[];
+  float *ts = esm;                                                 // [M x r] s*T
+  __nv_bfloat16 *l2s = reinterpret_cast<__nv_bfloat16 *>(esm + M * r);  // [r x 64]
+  const int nb = blockIdx.x * 64;
+  const int ncols = min(64, N - nb);
+  for (int i = threadIdx.x; i < r * 8; i += blockDim.x) {
+    const int jj = i >> 3, c = i & 7;  // 16-byte chunk c of row jj of the slice
+    uint4 v = make_uint4(0, 0, 0, 0);
+    if (8 * c < ncols) v = __ldg(reinterpret_cast<const uint4 *>(L2 + (int64_t)jj * N + nb) + c);
+    reinterpret_cast<uint4 *>(l2s + jj * 64)[c] = v;
+  }
   asm volatile("griddepcontrol.wait;" ::: "memory");
-  for (int i = threadIdx.x; i < M * r; i += blockDim.x) ts[i] = s * tacc[i];
+  for (int i = threadIdx.x; i < M * r; i += blockDim.x) ts[i] = s * __ldcg(tacc + i);
   __syncthreads();
   if (blockIdx.x == 0 && T_save) {
     for (int i = threadIdx.x; i < M * r; i += blockDim.x) {
@@ -447,24 +458,29 @@ __global__ void __launch_bounds__(256) gemv_epilogue_kernel(const float *__restr
       T_save[(int64_t)m * 2 * r + r + jj] = __float2bfloat16_rn(v - __bfloat162float(hb));
     }
   }
-  const int n = blockIdx.x * blockDim.x + threadIdx.x;
-  if (n >= N) return;
-  float y[kGvMaxM];
+  const int c = threadIdx.x & 63, q = threadIdx.x >> 6;
+  const int n = nb + c;
+  if (c >= ncols) return;
+  constexpr int kTok = kGvMaxM / 4;
+  float y[kTok];
 #pragma unroll
-  for (int m = 0; m < kGvMaxM; ++m) y[m] = m < M ? acc[(int64_t)m * N + n] : 0.f;
-  for (int j0 = 0; j0 < r; j0 += 8) {
-    float l2[8];
+  for (int i = 0; i < kTok; ++i) {
+    const int m = q + 4 * i;
+    y[i] = m < M ? __ldcg(acc + (int64_t)m * N + n) : 0.f;
+  }
+  for (int jj = 0; jj < r; ++jj) {
+    const float l2 = __bfloat162float(l2s[jj * 64 + c]);
 #pragma unroll
-    for (int q = 0; q < 8; ++q) l2[q] = __bfloat162float(L2[(int64_t)(j0 + q) * N + n]);
-#pragma unroll
-    for (int q = 0; q < 8; ++q)
-#pragma unroll
-      for (int m = 0; m < kGvMaxM; ++m)
-        if (m < M) y[m] = __fmaf_rn(ts[m * r + j0 + q], l2[q], y[m]);
+    for (int i = 0; i < kTok; ++i) {
+      const int m = q + 4 * i;
+      if (m < M) y[i] = __fmaf_rn(ts[m * r + jj], l2, y[i]);
+    }
   }
 #pragma unroll
-  for (int m = 0; m < kGvMaxM; ++m)
-    if (m < M) Y[(int64_t)m * N + n] = __float2bfloat16_rn(y[m]);
+  for (int i = 0; i < kTok; ++i) {
+    const int m = q + 4 * i;
+    if (m < M) Y[(int64_t)m * N + n] = __float2bfloat16_rn(y[i]);
+  }
 }
 
 }  // namespace qlora

@@ -27,6 +27,7 @@ struct DeviceInfo {
   int *err = nullptr;        // device address of g_dev_err
   bool gemm_attr[3] = {false, false, false};
   int gemv_smem_set[3] = {0, 0, 0};   // dynamic smem limit set per NT variant
+  int gemv_per_sm[3] = {0, 0, 0};     // resident CTAs per SM per NT variant
 };
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_mu;
@@ -344,9 +345,10 @@ int launch_gemv(const qlora_nf4dq_t *W, const uint16_t *X, int64_t M, const uint
       return QLORA_ERR_CUDA;
     dev->gemv_smem_set[idx] = smem;
   }
-  int per_sm = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, gemv_fwd_kernel<NT>, kGvThreads, smem) != cudaSuccess ||
-      per_sm < 1)
+  int &per_sm = dev->gemv_per_sm[idx];
+  if (per_sm < 1 &&
+      (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, gemv_fwd_kernel<NT>, kGvThreads, smem) != cudaSuccess ||
+       per_sm < 1))
     return QLORA_ERR_CUDA;
   GvArgs a;
   std::memset(&a, 0, sizeof(a));
@@ -374,11 +376,11 @@ int launch_gemv(const qlora_nf4dq_t *W, const uint16_t *X, int64_t M, const uint
   if (rc) return rc;
   rc = launch_pdl(gemv_fwd_kernel<NT>, dim3(grid), dim3(kGvThreads), (size_t)smem, st, tm_codes, tm_x, a);
   if (rc) return rc;
-  const size_t esmem = (size_t)M * r * 4;
+  const size_t esmem = (size_t)M * r * 4 + (size_t)r * 64 * 2;
   if (esmem > 48 * 1024 &&
       cudaFuncSetAttribute(gemv_epilogue_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)esmem) != cudaSuccess)
     return QLORA_ERR_CUDA;
-  return launch_pdl(gemv_epilogue_kernel, dim3((unsigned)((N + 255) / 256)), dim3(256), esmem, st,
+  return launch_pdl(gemv_epilogue_kernel, dim3((unsigned)((N + 63) / 64)), dim3(256), esmem, st,
                     (const float *)a.acc, (const float *)tacc, a.L2, (int)M, (int)N, r, s,
                     reinterpret_cast<__nv_bfloat16 *>(Y), reinterpret_cast<__nv_bfloat16 *>(T_save));
 }
