@@ -35,6 +35,7 @@ sys.path.insert(0, ROOT)
 import numpy as np  # noqa: E402
 import torch  # noqa: E402
 
+from bit_nf4_quantized_02_b200.dp import FlatGrads  # noqa: E402
 from synth import inputs, workloads  # noqa: E402
 
 WL = workloads.LLAMA7B_LAYER
@@ -158,18 +159,13 @@ def build_layer(dev, rank):
     xs = {"q": H, "k": H, "v": H, "o": A, "gate": H, "up": H, "down": U}
     lins = [Linear(l, xs[l.name], dev, WL.seed + 100 * i) for i, l in enumerate(WL.linears)]
     # adapter gradients as views of one flat fp32 buffer (one all-reduce per step)
-    sizes = [l.lin.k_in * WL.r + WL.r * l.lin.n_out for l in lins]
-    flat = torch.zeros(sum(sizes), dtype=torch.float32, device=dev)
-    off = 0
-    for l in lins:
-        K, N, r = l.lin.k_in, l.lin.n_out, WL.r
-        l.dL1 = flat[off:off + K * r].view(K, r)
-        l.dL2 = flat[off + K * r:off + K * r + r * N].view(r, N)
-        off += K * r + r * N
-    return lins, flat, (H, A, U)
+    grads = FlatGrads([(l.lin.k_in, l.lin.n_out, WL.r) for l in lins], dev)
+    for l, (dl1, dl2) in zip(lins, grads.views):
+        l.dL1, l.dL2 = dl1, dl2
+    return lins, grads, (H, A, U)
 
 
-def make_step(qlora, lins, flat, world):
+def make_step(qlora, lins, grads, world):
     def step():
         for l in lins:
             l.q = qlora.quantize_nf4_dq(l.W, out=l.q)
@@ -178,8 +174,7 @@ def make_step(qlora, lins, flat, world):
         for l in reversed(lins):
             qlora.linear_bwd(l.dY, l.X, l.T, l.q, l.L1, l.L2, WL.s, grad_dtype=torch.float32,
                              dX=l.dX, dL1=l.dL1, dL2=l.dL2)
-        if world > 1:
-            torch.distributed.all_reduce(flat)
+        grads.allreduce()
     return step
 
 
@@ -227,12 +222,13 @@ def run_ours(args, rank, world, local_rank):
     _lib.load()
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
-    lins, flat, acts = build_layer(dev, rank)
+    lins, grads, acts = build_layer(dev, rank)
+    flat = grads.flat
     if args.linear:
         lins = [l for l in lins if l.lin.name == args.linear]
     for l in lins:  # allocate the quantized buffers once
         l.q = qlora.quantize_nf4_dq(l.W)
-    step = make_step(qlora, lins, flat, world)
+    step = make_step(qlora, lins, grads, world)
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
@@ -334,6 +330,179 @@ def run_ours(args, rank, world, local_rank):
     return out
 
 
+# --------------------------------------------------------------------------- other workloads
+def _timed(qlora, step, args, dev, world, rank, local_rank, profile=True):
+    """Warm up, then time args.steps steps with CUDA events (max over ranks)."""
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if qlora.last_device_error() != 0:
+        raise RuntimeError("device error during warm-up")
+    sampler = ClockSampler([local_rank]) if rank == 0 else None
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    if sampler:
+        sampler.start()
+        time.sleep(0.5)
+    if profile:
+        qlora.profile_start(args.steps * 256 + 64)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        step()
+    e1.record()
+    torch.cuda.synchronize()
+    launches = qlora.profile_stop() if profile else []
+    clocks = sampler.stop() if sampler else None
+    ms = e0.elapsed_time(e1) / args.steps
+    t = torch.tensor([ms], device=dev)
+    if world > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    if qlora.last_device_error() != 0:
+        raise RuntimeError("device error during the timed region")
+    return float(t.item()), launches, clocks
+
+
+def _kernel_table(launches, steps):
+    per_kind = {}
+    for kind, kms in launches:
+        c = per_kind.setdefault(kind, [0, 0.0])
+        c[0] += 1
+        c[1] += kms
+    total = sum(v[1] for v in per_kind.values())
+    return per_kind, {k: {"launches_per_step": v[0] / steps, "ms_per_step": v[1] / steps,
+                          "share": v[1] / total if total else None}
+                      for k, v in sorted(per_kind.items(), key=lambda kv: -kv[1][1])}
+
+
+def run_decode(args, rank, world, local_rank):
+    """LLaMA-65B layer forward at 16 tokens: the memory-bound few-token path."""
+    import bit_nf4_quantized_02_b200 as qlora
+    wl = workloads.LLAMA65B_LAYER
+    M, r, s = wl.extra["M_decode"], wl.r, wl.s
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    base = wl.seed + 1000 * rank
+    H = inputs.device_normal((M, 8192), 1.0, base + 1, dev, torch.bfloat16)
+    A = inputs.device_normal((M, 8192), 1.0, base + 2, dev, torch.bfloat16)
+    U = inputs.device_normal((M, 22016), 1.0, base + 3, dev, torch.bfloat16)
+    xs = {"q": H, "k": H, "v": H, "o": A, "gate": H, "up": H, "down": U}
+    lins = []
+    nbytes = 0
+    for i, lin in enumerate(wl.linears):
+        N, K = lin.n_out, lin.k_in
+        W = inputs.device_normal((N, K), inputs.WEIGHT_STD, wl.seed + 100 * i, dev)
+        q = qlora.quantize_nf4_dq(W)
+        del W
+        L1 = inputs.device_normal((K, r), 1.0 / np.sqrt(K), wl.seed + 100 * i + 1, dev, torch.bfloat16)
+        L2 = inputs.device_normal((r, N), inputs.L2_STD, wl.seed + 100 * i + 2, dev, torch.bfloat16)
+        Y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+        T = torch.empty(M, 2 * r, dtype=torch.bfloat16, device=dev)
+        lins.append((xs[lin.name], q, L1, L2, Y, T))
+        # algorithmic bytes: NF4+DQ weight, LoRA factors, X read, Y and T written
+        nbytes += q.nbytes() + 2 * r * (K + N) + 2 * M * K + 2 * M * N + 2 * M * 2 * r
+    torch.cuda.synchronize()
+
+    def step():
+        for X, q, L1, L2, Y, T in lins:
+            qlora.linear_fwd(X, q, L1, L2, s, Y=Y, T=T)
+
+    ms, launches, clocks = _timed(qlora, step, args, dev, world, rank, local_rank)
+    # the same step captured in a CUDA graph (no host launch overhead)
+    g = torch.cuda.CUDAGraph()
+    side = torch.cuda.Stream(dev)
+    side.wait_stream(torch.cuda.current_stream(dev))
+    with torch.cuda.stream(side):
+        step()
+        with torch.cuda.graph(g, stream=side):
+            step()
+    torch.cuda.current_stream(dev).wait_stream(side)
+    for _ in range(3):
+        g.replay()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        g.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    ms_graph = e0.elapsed_time(e1) / args.steps
+    if rank != 0:
+        return None
+    peaks, peak_src = load_peaks()
+    per_kind, kernels = _kernel_table(launches, args.steps)
+    dom = per_kind.get("gemv_fwd", [0, 0.0])
+    achieved = nbytes * args.steps / (dom[1] * 1e-3) / 1e9 if dom[1] > 0 else None
+    peak = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+    return {
+        "metric": "QLoRA NF4 linear forward, NF4-weight-bound GB/s", "value": nbytes * world / (ms * 1e-3) / 1e9,
+        "unit": "GB/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": "llama65b-layer-7-linears-forward-M16-r64", "tokens": M, "lora_r": r,
+                   "bytes_per_step": nbytes, "l2": "weights (418 MB) larger than L2, no flush",
+                   "step": "forward of the 7 QLoRA linears (weights resident, quantized once)"},
+        "graph": {"ms_per_step": ms_graph, "value": nbytes * world / (ms_graph * 1e-3) / 1e9, "unit": "GB/s",
+                  "frac_of_hbm": nbytes / (ms_graph * 1e-3) / 1e9 / peak},
+        "gpu_launches": len(launches),
+        "roofline": {"bound": "hbm", "kernel": "few-token forward chain (lora_down_small + gemv_fwd + epilogue)",
+                     "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak if achieved else None, "traffic": None,
+                     "peak_source": f"{peak_src} hbm_gbs", "launches_timed": dom[0],
+                     "avg_launch_ms": dom[1] / dom[0] if dom[0] else None},
+        "kernels": kernels, "clocks": clocks,
+    }
+
+
+def run_quantizer(args, rank, world, local_rank):
+    """NF4 + DQ quantize, then dequantize, of the LLaMA-7B-shaped bf16 weights (with outliers)."""
+    import bit_nf4_quantized_02_b200 as qlora
+    wl = workloads.QUANTIZER_7B
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    mats = []
+    nbytes_q = nbytes_d = 0
+    for i, lin in enumerate(wl.linears):
+        W = inputs.device_weight_with_outliers(lin.n_out, lin.k_in, wl.seed + 1000 * rank + i, dev)
+        q = qlora.quantize_nf4_dq(W)
+        out = torch.empty_like(W)
+        mats.append((W, q, out))
+        nbytes_q += W.numel() * 2 + q.nbytes()
+        nbytes_d += q.nbytes() + W.numel() * 2
+    torch.cuda.synchronize()
+
+    def step():
+        for W, q, out in mats:
+            qlora.quantize_nf4_dq(W, out=q)
+        for W, q, out in mats:
+            qlora.dequant(q, out=out)
+
+    ms, launches, clocks = _timed(qlora, step, args, dev, world, rank, local_rank)
+    if rank != 0:
+        return None
+    peaks, peak_src = load_peaks()
+    per_kind, kernels = _kernel_table(launches, args.steps)
+    peak = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+    qk, dk = per_kind.get("quantize", [0, 0.0]), per_kind.get("dequant", [0, 0.0])
+    dq = per_kind.get("dq_constants", [0, 0.0])
+    q_ms = qk[1] + dq[1]
+    roof_q = nbytes_q * args.steps / (q_ms * 1e-3) / 1e9 if q_ms else None
+    roof_d = nbytes_d * args.steps / (dk[1] * 1e-3) / 1e9 if dk[1] else None
+    return {
+        "metric": "NF4+DQ quantize + dequantize GB/s", "value": (nbytes_q + nbytes_d) * world / (ms * 1e-3) / 1e9,
+        "unit": "GB/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "u8", "data": "synthetic",
+        "config": {"workload": wl.name, "params": sum(l.n_out * l.k_in for l in wl.linears),
+                   "bytes_quantize": nbytes_q, "bytes_dequant": nbytes_d,
+                   "l2": "weights (667 MB bf16) larger than L2, no flush"},
+        "gpu_launches": len(launches),
+        "roofline": {"bound": "hbm", "kernel": "quantize (K1 + K2) and dequant (K3)",
+                     "achieved": roof_q, "achieved_dequant": roof_d, "peak": peak, "unit": "GB/s",
+                     "frac": roof_q / peak if roof_q else None, "frac_dequant": roof_d / peak if roof_d else None,
+                     "traffic": None, "peak_source": f"{peak_src} hbm_gbs"},
+        "kernels": kernels, "clocks": clocks,
+    }
+
+
 # --------------------------------------------------------------------------- oracle timing
 SAMPLE_SLICE = 64   # the CPU sample is 1/64 of a step: 128 of the 8192 tokens, 1/64 of each weight's rows
 
@@ -424,6 +593,10 @@ def main():
     ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end (host buffers) measurement")
     ap.add_argument("--linear", choices=[l.name for l in WL.linears], default=None,
                     help="restrict the step to one linear of the layer (profiling runs)")
+    ap.add_argument("--workload", choices=["llama7b-train", "llama65b-decode", "quantizer"], default="llama7b-train",
+                    help="llama7b-train (default, the headline): quantize + fwd + bwd of a LLaMA-7B layer at 8192 "
+                         "tokens; llama65b-decode: forward of a LLaMA-65B layer at 16 tokens; quantizer: NF4+DQ "
+                         "quantize and dequantize of LLaMA-7B-shaped bf16 weights")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3
@@ -438,7 +611,12 @@ def main():
             torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
                                                  device_id=torch.device("cuda", local_rank))
         try:
-            out = run_ours(args, rank, world, local_rank)
+            if args.workload == "llama65b-decode":
+                out = run_decode(args, rank, world, local_rank)
+            elif args.workload == "quantizer":
+                out = run_quantizer(args, rank, world, local_rank)
+            else:
+                out = run_ours(args, rank, world, local_rank)
         finally:
             if world > 1:
                 torch.distributed.destroy_process_group()
