@@ -1,9 +1,9 @@
 // Fused doubleDequant + product for few tokens (QLoRA §3 Eq. 5 / Eq. 6 at
 // decode-sized M): the frozen-weight bytes dominate, so every NF4 weight is
-// read once from HBM and decoded on the fly into tensor-core fragments -- no
-// bf16 copy of the weight is ever written.
+// read once from HBM and decoded in registers straight into tensor-core
+// fragments -- no bf16 copy of the weight is ever written.
 //
-//   Y[M x N] = bf16( X W_hat^T + (s X L1) L2 ),   M <= 16*MT (MT in {1, 2})
+//   Y[M x N] = bf16( X W_hat^T + (s X L1) L2 ),   M <= 8*NT (NT in {1, 2, 4})
 //
 // Three launches per linear, chained with programmatic dependent launch:
 //   lora_down_small_kernel   adds K-slices of X L1 into an fp32 accumulator;
@@ -12,32 +12,24 @@
 //                            overlaps the first kernel completely);
 //   gemv_epilogue_kernel     Y = bf16(acc + s T L2), and T = s X L1 as a bf16
 //                            hi/lo pair for the backward.
-//
-// gemv_fwd_kernel: persistent, 160 threads per CTA, 2 CTAs per SM.
-//   * Operands: mma.sync m16n8k16 (bf16 in, fp32 accumulate) with the tokens
-//     as the A operand (16 per tile) and the weight as the B operand (8 output
-//     features per tile), so one X fragment feeds 8 weight tiles.
-//   * Warp 4 (producer): per stage, 64 weight rows x 256 K of packed codes
-//     (TMA, 128-byte swizzle), the X tile ([token][64-block][64], TMA 3-D,
-//     128-byte swizzle) and the 64 x 4 block constants
-//     c2_hat = fma(E4M3(code8), c1, mean) computed by its lanes into shared
-//     memory; the stage's mbarrier completes on the TMA bytes plus the
-//     constants' arrival.
-//   * Warp w in 0..3 (consumers) takes 64-block w of every stage for all 64
-//     rows.  Decode: each byte of codes is two consecutive weights; it indexes
-//     a 256-entry shared table of bf16x2 (NF4[lo nibble], NF4[hi nibble]),
-//     replicated once per lane so every lookup is bank-conflict free, and the
-//     entry is directly a B-fragment register.  The block constant is applied
-//     in fp32 after the block's four MMAs (per-block partial accumulators):
-//     Y = sum_b c2_hat_b (X_b . bf16(NF4[codes_b])).  This equals X W_hat^T up
-//     to bf16 rounding placement: the constant multiplies in fp32 instead of
-//     being folded into a bf16 weight first.
-//   * K inside a block is permuted identically for A and B: lane column j,
-//     k-step s, slot u <-> k = 16 j + 4 s + u, so a lane's codes of a row are
-//     one 8-byte run per block and its X operand one 32-byte run.
-//   * A unit is 64 rows x 512 K (2 stages).  The four warps' partial sums are
-//     reduced through shared memory and added into the fp32 [M x N]
-//     accumulator with red.global.add (L2 resident).
+// gemv_fwd_kernel, persistent, 160 threads per CTA (3 CTAs per SM):
+//   * warp 4 is a TMA producer: per stage, 64 weight rows x 256 K of packed
+//     codes (128-byte swizzle) and the matching X tile (3-D view of X,
+//     [token][64-block][64], 128-byte swizzle) into a ring of mbarrier stages;
+//   * warps 0..3 each own 16 weight rows.  Lane (g, j) decodes rows g and g+8
+//     of NF4 block j of the stage -- 64 weights per row, all under one
+//     constant -- through a 16-entry bf16 table T_b[c] = bf16(NF4[c] * c2_hat)
+//     (bit-identical to qlora_dequant) held as byte planes and indexed with
+//     byte permutes, and feeds them as the A operand of mma.sync m16n8k16
+//     (bf16 in, fp32 accumulate) against X as the B operand.
+//   * The K positions inside a stage are permuted consistently for A and B:
+//     logical k-step s, slot u of lane-column j <-> physical k = 64 j + 4 s + u,
+//     so each lane's codes are one contiguous 32-byte run per row and its X
+//     operand is one 16-byte run per two steps; both are bank-conflict free
+//     under the 128-byte swizzle.
+//   * A unit is 64 rows x 512 K; partial products are added into an fp32
+//     [M x N] accumulator with red.global.add (L2 resident); all CTAs do the
+//     same amount of work (no per-block finishing step on the critical path).
 // The two accumulators must be zero at launch (the host clears them with one
 // memset in stream order).  Split-K additions make the low bits of Y depend
 // on the order in which CTAs finish.
@@ -48,22 +40,20 @@
 
 namespace qlora {
 
-constexpr int kGvRows = 64;          // weight rows per stage / unit
-constexpr int kGvStageK = 256;       // K per pipeline stage (4 blocks of 64)
+constexpr int kGvRows = 64;          // weight rows per unit (4 warps x 16)
+constexpr int kGvStageK = 256;       // K per pipeline stage
 constexpr int kGvUnitK = 512;        // K per unit (2 stages)
 constexpr int kGvThreads = 160;      // 4 decode/MMA warps + 1 producer warp
 constexpr int kGvMaxM = 32;
-constexpr int kGvLutBytes = 256 * 32 * 4;   // 256 entries x 32 lane copies x bf16x2
 
-template <int MT>
+template <int NT>
 struct GvCfg {
   static constexpr int kCodeBytes = kGvRows * 128;          // 64 rows x 256 codes
-  static constexpr int kXBytes = 16 * MT * kGvStageK * 2;   // 16*MT tokens x 256 bf16
-  static constexpr int kScaleBytes = 4 * kGvRows * 4;       // [block][row] fp32
-  static constexpr int kStageBytes = kCodeBytes + kXBytes + kScaleBytes;
-  static constexpr int kStages = MT == 1 ? 3 : 2;
-  static constexpr int kRedBytes = 4 * 32 * 32 * MT * 4;    // per-warp partials, 32 lanes x 32*MT floats
-  static constexpr int kSmemBytes = kGvLutBytes + kStages * kStageBytes + kRedBytes + 256 + 1024;
+  static constexpr int kXBytes = 8 * NT * kGvStageK * 2;    // padded tokens x 256 bf16
+  static constexpr int kStageBytes = kCodeBytes + kXBytes;
+  static constexpr int kStages = NT == 1 ? 5 : (NT == 2 ? 4 : 3);   // ~64 KB: 3 CTAs per SM
+  // + 1024 alignment slack + 256 barrier area
+  static constexpr int kSmemBytes = kStages * kStageBytes + 1024 + 256;
 };
 
 struct GvArgs {
@@ -74,12 +64,13 @@ struct GvArgs {
   const uint8_t *c2_fp8;
   const float *c1;
   const float *mu;
+  const __nv_bfloat16 *X;    // [M x K]
+  const __nv_bfloat16 *L1;   // [K x r]
   const __nv_bfloat16 *L2;   // [r x N]
   float *acc;            // [M x N] fp32, zero at launch
   int *err;
 };
 
-// D += A * B, or D = A * B when `zero` (C read as 0).
 __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
   asm volatile(
       "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
@@ -88,21 +79,17 @@ __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
+// prmt in its default mode, where a selector nibble with bit 3 set replicates
+// the sign bit of the selected byte.
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t d;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+  return d;
+}
+
 __device__ __forceinline__ uint4 lds128(uint32_t addr) {
   uint4 v;
   asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
-  return v;
-}
-
-__device__ __forceinline__ uint2 lds64(uint32_t addr) {
-  uint2 v;
-  asm volatile("ld.shared.v2.b32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr));
-  return v;
-}
-
-__device__ __forceinline__ uint32_t lds32(uint32_t addr) {
-  uint32_t v;
-  asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(addr));
   return v;
 }
 
@@ -110,141 +97,206 @@ __device__ __forceinline__ void red_add_f32(float *p, float v) {
   asm volatile("red.global.add.f32 [%0], %1;" ::"l"(p), "f"(v) : "memory");
 }
 
+// Release/acquire fence at GPU scope (lighter than the sequentially
+// consistent fence of __threadfence()).
+__device__ __forceinline__ void fence_acq_rel_gpu() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
+
 __device__ __forceinline__ void named_bar_sync(int id, int n) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
 }
 
-// bf16x2 decode of one byte of codes through the lane's copy of the table:
-// entry b sits at lut + (b * 32 + lane) * 4.
-__device__ __forceinline__ uint32_t lut_decode(uint32_t lane_base, uint32_t word, int byte) {
-  const uint32_t b = __byte_perm(word, 0u, 0x4440 + byte);   // zero-extended byte
-  return lds32(lane_base + b * 128u);
-}
-
-// Raw block constants of one stage for one producer lane: rows lane and
-// lane + 32 of the 64-row tile, the stage's 4 blocks.
-struct GvConsts {
-  uint32_t code8[8];
-  float c1[8];
-  __device__ __forceinline__ void load(const GvArgs &p, int u, int st, int lane, int kblocks) {
-    int rb = 0, kb0 = 0;
-    const bool live = u < p.units;
-    if (live) {
-      rb = u / p.nks;
-      const int ks = u - rb * p.nks;
-      kb0 = (ks * kGvUnitK + st * kGvStageK) >> 6;
-    }
+// The 16 decoded values of one 64-block, bf16(NF4[c] * c2_hat), stored as two
+// byte planes: lo[i] holds the low bytes of entries 4i..4i+3, hi[i] the high
+// bytes.
+struct BlockTable {
+  uint32_t lo[4], hi[4];
+  __device__ __forceinline__ void build(float c2h) {
+    uint32_t e[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-      const int row = rb * kGvRows + lane + 32 * (i >> 2);
-      const int kb = kb0 + (i & 3);
-      code8[i] = 0;
-      c1[i] = 0.f;
-      if (live && row < p.N && kb < kblocks) {
-        const int64_t b = (int64_t)row * kblocks + kb;
-        code8[i] = __ldg(p.c2_fp8 + b);
-        c1[i] = __ldg(p.c1 + (b >> 8));
-      }
+      const __nv_bfloat162 p = __floats2bfloat162_rn(__fmul_rn(kNF4[2 * i], c2h), __fmul_rn(kNF4[2 * i + 1], c2h));
+      e[i] = *reinterpret_cast<const uint32_t *>(&p);
     }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      lo[i] = __byte_perm(e[2 * i], e[2 * i + 1], 0x6420);
+      hi[i] = __byte_perm(e[2 * i], e[2 * i + 1], 0x7531);
+    }
+  }
+  // Four codes (nibbles of the low 16 bits of `sel7`, bit 3 cleared) whose
+  // bit-3 flags are the byte mask `m8` -> two bf16x2 words {T[c0],T[c1]},
+  // {T[c2],T[c3]}.
+  __device__ __forceinline__ void lookup4(uint32_t sel7, uint32_t m8, uint32_t &p01, uint32_t &p23) const {
+    const uint32_t la = __byte_perm(lo[0], lo[1], sel7);
+    const uint32_t lb = __byte_perm(lo[2], lo[3], sel7);
+    const uint32_t ha = __byte_perm(hi[0], hi[1], sel7);
+    const uint32_t hb = __byte_perm(hi[2], hi[3], sel7);
+    const uint32_t l = (lb & m8) | (la & ~m8);
+    const uint32_t h = (hb & m8) | (ha & ~m8);
+    p01 = __byte_perm(l, h, 0x5140);
+    p23 = __byte_perm(l, h, 0x7362);
   }
 };
 
-template <int MT>
-struct GvProducer {
-  using Cfg = GvCfg<MT>;
-  const GvArgs *p;
-  uint8_t *stage_base;
-  uint64_t *full_bar, *empty_bar;
-  const CUtensorMap *tmCodes, *tmX;
-  int kblocks, lane, stage, u, st;
-  uint32_t phase, used, last_parity;
-  float mu;
+// Raw constants of a lane's two (row, block) pairs for one (unit, stage) item.
+struct ConstPrefetch {
+  uint32_t code8[2];
+  float c1[2];
+  bool ok[2];
+  __device__ __forceinline__ void load(const GvArgs &p, int u, int st, int r0, int j, int kblocks) {
+    ok[0] = ok[1] = false;
+    code8[0] = code8[1] = 0;
+    c1[0] = c1[1] = 0.f;
+    if (u >= p.units) return;
+    const int rb = u / p.nks, ks = u - rb * p.nks;
+    const int kb = ((ks * kGvUnitK + st * kGvStageK) >> 6) + j;
+    if (kb >= kblocks) return;
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      const int n = rb * kGvRows + r0 + 8 * i;
+      if (n < p.N) {
+        const int64_t b = (int64_t)n * kblocks + kb;
+        code8[i] = __ldg(p.c2_fp8 + b);
+        c1[i] = __ldg(p.c1 + (b >> 8));
+        ok[i] = true;
+      }
+    }
+  }
+  __device__ __forceinline__ float c2hat(int i, float mu) const {
+    return ok[i] ? __fmaf_rn(e4m3_to_f32((uint8_t)code8[i]), c1[i], mu) : 0.f;
+  }
+};
 
-  __device__ __forceinline__ void init(const GvArgs &pp, uint8_t *sb, uint64_t *fb, uint64_t *eb,
-                                       const CUtensorMap *tc, const CUtensorMap *tx, int kb) {
+// State of one decode/MMA warp of gemv_fwd_kernel.
+template <int NT>
+struct GvConsumer {
+  using Cfg = GvCfg<NT>;
+  const GvArgs *p;
+  uint8_t *smem;
+  uint64_t *full_bar, *empty_bar;
+  int kblocks, g, j, r0, lane;
+  int stage;
+  uint32_t phase;
+  int u, st;
+  float mu;
+  float d[2][NT][4];  // two accumulator chains (even / odd k-steps)
+
+  __device__ __forceinline__ void init(const GvArgs &pp, uint8_t *sm, uint64_t *fb, uint64_t *eb, int kb) {
     p = &pp;
-    stage_base = sb;
+    smem = sm;
     full_bar = fb;
     empty_bar = eb;
-    tmCodes = tc;
-    tmX = tx;
     kblocks = kb;
     lane = lane_id();
+    g = lane >> 2;
+    j = lane & 3;
+    r0 = warp_id() * 16 + g;
     stage = 0;
-    phase = used = last_parity = 0;
+    phase = 0;
     u = blockIdx.x;
     st = 0;
     mu = __ldg(pp.mu);
   }
 
-  // Issue item (u, st) whose constants are in `cur`; start loading the next
+  // Process item (u, st) whose constants are in `cur`; start loading the next
   // item's constants into `nxt`.  Returns false on a pipeline timeout.
-  __device__ __forceinline__ bool item(const GvConsts &cur, GvConsts &nxt) {
+  __device__ __forceinline__ bool item(const ConstPrefetch &cur, ConstPrefetch &nxt) {
     const GvArgs &P = *p;
     const int rb = u / P.nks, ks = u - rb * P.nks;
     const int kbeg = ks * kGvUnitK;
     const int nst = min(kGvUnitK, P.K - kbeg) > kGvStageK ? 2 : 1;
+    const int n0 = rb * kGvRows + r0, n1 = n0 + 8;
+    if (st == 0) {
+#pragma unroll
+      for (int c = 0; c < 2; ++c)
+#pragma unroll
+        for (int t = 0; t < NT; ++t) d[c][t][0] = d[c][t][1] = d[c][t][2] = d[c][t][3] = 0.f;
+    }
+    BlockTable tb0, tb1;
+    tb0.build(cur.c2hat(0, mu));
+    tb1.build(cur.c2hat(1, mu));
     int nu = u, nstn = st + 1;
     if (nstn == nst) {
       nu = u + gridDim.x;
       nstn = 0;
     }
-    nxt.load(P, nu, nstn, lane, kblocks);
-    const int k0 = kbeg + st * kGvStageK;
-    bool got = true;
-    if (lane == 0) {
-      got = mbar_wait(smem_u32(empty_bar + stage), phase ^ 1, P.err, DEV_TIMEOUT_PRODUCER);
-      if (got) {
-        const uint32_t fb = smem_u32(full_bar + stage);
-        mbar_arrive_expect_tx(fb, Cfg::kCodeBytes + Cfg::kXBytes);
-        const uint32_t sc = smem_u32(stage_base + stage * Cfg::kStageBytes);
-        tma_load_2d(sc, tmCodes, fb, k0 >> 1, rb * kGvRows);
-        asm volatile(
-            "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5}], "
-            "[%2];" ::"r"(sc + Cfg::kCodeBytes),
-            "l"(reinterpret_cast<uint64_t>(tmX)), "r"(fb), "r"(0), "r"(k0 >> 6), "r"(0)
-            : "memory");
-        used |= 1u << stage;
-        last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
+    nxt.load(P, nu, nstn, r0, j, kblocks);
+    if (!mbar_wait(smem_u32(full_bar + stage), phase, P.err, DEV_TIMEOUT_MMA)) return false;
+    const uint32_t sc = smem_u32(smem + stage * Cfg::kStageBytes);
+    const uint32_t sx = sc + Cfg::kCodeBytes;
+    // codes of rows r0, r0+8: 16-byte chunks 2j, 2j+1 of their 128-byte lines
+    uint32_t q0[8], q1[8];
+    {
+      const uint4 a = lds128(sc + r0 * 128 + (((2 * j) ^ (r0 & 7)) << 4));
+      const uint4 b = lds128(sc + r0 * 128 + (((2 * j + 1) ^ (r0 & 7)) << 4));
+      const uint4 c = lds128(sc + (r0 + 8) * 128 + (((2 * j) ^ (r0 & 7)) << 4));
+      const uint4 e = lds128(sc + (r0 + 8) * 128 + (((2 * j + 1) ^ (r0 & 7)) << 4));
+      q0[0] = a.x; q0[1] = a.y; q0[2] = a.z; q0[3] = a.w; q0[4] = b.x; q0[5] = b.y; q0[6] = b.z; q0[7] = b.w;
+      q1[0] = c.x; q1[1] = c.y; q1[2] = c.z; q1[3] = c.w; q1[4] = e.x; q1[5] = e.y; q1[6] = e.z; q1[7] = e.w;
+    }
+#pragma unroll
+    for (int w = 0; w < 8; ++w) {
+      // X operand for steps 2w, 2w+1: token g + 8t, line (token*4 + j), chunk w
+      uint4 xb[NT];
+#pragma unroll
+      for (int t = 0; t < NT; ++t) {
+        const int line = (g + 8 * t) * 4 + j;
+        xb[t] = lds128(sx + line * 128 + ((w ^ (line & 7)) << 4));
+      }
+      const uint32_t m0 = q0[w] & 0x77777777u, m1 = q1[w] & 0x77777777u;
+      const uint32_t s0 = q0[w] << 4, s1 = q1[w] << 4;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        uint32_t a[4];
+        const uint32_t msel = h ? 0xFBEAu : 0xD9C8u;
+        tb0.lookup4(h ? (m0 >> 16) : m0, prmt(s0, q0[w], msel), a[0], a[2]);
+        tb1.lookup4(h ? (m1 >> 16) : m1, prmt(s1, q1[w], msel), a[1], a[3]);
+#pragma unroll
+        for (int t = 0; t < NT; ++t) {
+          const uint32_t b0 = h ? xb[t].z : xb[t].x;
+          const uint32_t b1 = h ? xb[t].w : xb[t].y;
+          mma_bf16_16816(d[h][t], a, b0, b1);
+        }
       }
     }
-    if (!__shfl_sync(0xFFFFFFFFu, got ? 1 : 0, 0)) return false;
-    // block constants -> [block][row] fp32 of the stage (free: the empty wait above)
-    float *scales = reinterpret_cast<float *>(stage_base + stage * Cfg::kStageBytes + Cfg::kCodeBytes + Cfg::kXBytes);
-#pragma unroll
-    for (int i = 0; i < 8; ++i)
-      scales[(i & 3) * kGvRows + lane + 32 * (i >> 2)] = __fmaf_rn(e4m3_to_f32((uint8_t)cur.code8[i]), cur.c1[i], mu);
     __syncwarp();
-    if (lane == 0) mbar_arrive(smem_u32(full_bar + stage));   // constants in place
+    if (lane == 0) mbar_arrive(smem_u32(empty_bar + stage));
     if (++stage == Cfg::kStages) {
       stage = 0;
       phase ^= 1;
+    }
+    if (st == nst - 1) {
+      // the unit is complete: add its partial products into the accumulator
+#pragma unroll
+      for (int t = 0; t < NT; ++t) {
+        const int tok = 8 * t + 2 * j;
+        const float v0 = d[0][t][0] + d[1][t][0], v1 = d[0][t][1] + d[1][t][1];
+        const float v2 = d[0][t][2] + d[1][t][2], v3 = d[0][t][3] + d[1][t][3];
+        if (tok < P.M) {
+          if (n0 < P.N) red_add_f32(P.acc + (int64_t)tok * P.N + n0, v0);
+          if (n1 < P.N) red_add_f32(P.acc + (int64_t)tok * P.N + n1, v2);
+        }
+        if (tok + 1 < P.M) {
+          if (n0 < P.N) red_add_f32(P.acc + (int64_t)(tok + 1) * P.N + n0, v1);
+          if (n1 < P.N) red_add_f32(P.acc + (int64_t)(tok + 1) * P.N + n1, v3);
+        }
+      }
     }
     u = nu;
     st = nstn;
     return true;
   }
-
-  // Never leave the CTA while a tensor copy is still landing in shared memory.
-  __device__ __forceinline__ void drain() {
-    if (lane == 0)
-      for (int i = 0; i < Cfg::kStages; ++i)
-        if (used & (1u << i))
-          mbar_wait(smem_u32(full_bar + i), (last_parity >> i) & 1u, p->err, DEV_TIMEOUT_DRAIN);
-  }
 };
 
-template <int MT>
-__global__ void __launch_bounds__(kGvThreads, 2)
+template <int NT>
+__global__ void __launch_bounds__(kGvThreads, 3)
     gemv_fwd_kernel(const __grid_constant__ CUtensorMap tmCodes, const __grid_constant__ CUtensorMap tmX,
                     const __grid_constant__ GvArgs p) {
-  using Cfg = GvCfg<MT>;
+  using Cfg = GvCfg<NT>;
   constexpr int S = Cfg::kStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t *stage_base = smem + kGvLutBytes;                       // 1024-aligned (LUT is 32 KB)
-  float *red = reinterpret_cast<float *>(stage_base + S * Cfg::kStageBytes);
-  uint64_t *full_bar = reinterpret_cast<uint64_t *>(reinterpret_cast<uint8_t *>(red) + Cfg::kRedBytes);
+  uint64_t *full_bar = reinterpret_cast<uint64_t *>(smem + S * Cfg::kStageBytes);
   uint64_t *empty_bar = full_bar + S;
 
   const int warp = warp_id();
@@ -252,18 +304,10 @@ __global__ void __launch_bounds__(kGvThreads, 2)
   const int kblocks = p.K >> 6;
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");  // the epilogue may launch and wait
 
-  // the byte -> (NF4[lo], NF4[hi]) bf16x2 table, one copy per lane
-  {
-    uint32_t *lut = reinterpret_cast<uint32_t *>(smem);
-    for (int i = threadIdx.x; i < 256 * 32; i += blockDim.x) {
-      const int b = i >> 5;
-      const __nv_bfloat162 v = __floats2bfloat162_rn(kNF4[b & 15], kNF4[b >> 4]);
-      lut[i] = *reinterpret_cast<const uint32_t *>(&v);
-    }
-  }
+  // ---------------------------------------------------------------- main loop
   if (threadIdx.x == 0) {
     for (int i = 0; i < S; ++i) {
-      mbar_init(smem_u32(full_bar + i), 2);   // TMA (with tx) + constants
+      mbar_init(smem_u32(full_bar + i), 1);
       mbar_init(smem_u32(empty_bar + i), 4);
     }
     fence_mbar_init();
@@ -271,122 +315,67 @@ __global__ void __launch_bounds__(kGvThreads, 2)
   __syncthreads();
 
   if (warp == 4) {
-    // ------------------------------------------------------------ producer
+    // Lane 0 drives the TMA ring; all lanes prefetch the next stage's block
+    // constants (one code8 run per weight row) into L2 for the decode warps.
     if (lane == 0) {
       tma_prefetch_desc(&tmCodes);
       tma_prefetch_desc(&tmX);
     }
-    GvProducer<MT> pr;
-    pr.init(p, stage_base, full_bar, empty_bar, &tmCodes, &tmX, kblocks);
-    // Flat walk over (unit, stage) items, unrolled by two: the block constants
-    // of the next item load into the other register set while this one is
-    // issued, so their latency never stalls the ring.
-    GvConsts ca, cb;
-    ca.load(p, pr.u, pr.st, lane, kblocks);
-    while (pr.u < p.units) {
-      if (!pr.item(ca, cb)) break;
-      if (pr.u >= p.units || !pr.item(cb, ca)) break;
-    }
-    pr.drain();
-  } else {
-    // ------------------------------------------------------------ consumers
-    const int g = lane >> 2, j = lane & 3;
-    const uint32_t lane_base = smem_u32(smem) + lane * 4;
     int stage = 0;
-    uint32_t phase = 0;
-    float acc[8][MT][4];
+    uint32_t phase = 0, used = 0, last_parity = 0;
     bool ok = true;
     for (int u = blockIdx.x; u < p.units && ok; u += gridDim.x) {
       const int rb = u / p.nks, ks = u - rb * p.nks;
       const int kbeg = ks * kGvUnitK;
       const int nst = min(kGvUnitK, p.K - kbeg) > kGvStageK ? 2 : 1;
 #pragma unroll
-      for (int t = 0; t < 8; ++t)
-#pragma unroll
-        for (int m = 0; m < MT; ++m) acc[t][m][0] = acc[t][m][1] = acc[t][m][2] = acc[t][m][3] = 0.f;
+      for (int i = 0; i < 2; ++i) {
+        const int n = rb * kGvRows + lane + 32 * i;
+        if (n < p.N) asm volatile("prefetch.global.L2 [%0];" ::"l"(p.c2_fp8 + (int64_t)n * kblocks + (kbeg >> 6)));
+      }
       for (int st = 0; st < nst; ++st) {
-        if (!mbar_wait(smem_u32(full_bar + stage), phase, p.err, DEV_TIMEOUT_MMA)) {
+        bool got = true;
+        if (lane == 0) {
+          got = mbar_wait(smem_u32(empty_bar + stage), phase ^ 1, p.err, DEV_TIMEOUT_PRODUCER);
+          if (got) {
+            const uint32_t fb = smem_u32(full_bar + stage);
+            mbar_arrive_expect_tx(fb, Cfg::kStageBytes);
+            const uint32_t sc = smem_u32(smem + stage * Cfg::kStageBytes);
+            const int k0 = kbeg + st * kGvStageK;
+            tma_load_2d(sc, &tmCodes, fb, k0 >> 1, rb * kGvRows);
+            asm volatile(
+                "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, "
+                "%5}], [%2];" ::"r"(sc + Cfg::kCodeBytes),
+                "l"(reinterpret_cast<uint64_t>(&tmX)), "r"(fb), "r"(0), "r"(k0 >> 6), "r"(0)
+                : "memory");
+            used |= 1u << stage;
+            last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
+          }
+        }
+        if (!__shfl_sync(0xFFFFFFFFu, got ? 1 : 0, 0)) {
           ok = false;
           break;
         }
-        const uint32_t sc = smem_u32(stage_base + stage * Cfg::kStageBytes);
-        const uint32_t sx = sc + Cfg::kCodeBytes;
-        const uint32_t ss = sx + Cfg::kXBytes;
-        // A fragments of block `warp` for its 4 k-steps: tokens g (+16m) and g+8 (+16m),
-        // X[tok][16j .. 16j+15] = chunks 2j, 2j+1 of line (tok*4 + warp)
-        uint32_t afr[MT][4][4];
-#pragma unroll
-        for (int m = 0; m < MT; ++m) {
-          uint4 x[2][2];
-#pragma unroll
-          for (int hh = 0; hh < 2; ++hh) {
-            const int line = (g + 8 * hh + 16 * m) * 4 + warp;
-#pragma unroll
-            for (int c = 0; c < 2; ++c) x[hh][c] = lds128(sx + line * 128 + (((2 * j + c) ^ (line & 7)) << 4));
-          }
-#pragma unroll
-          for (int s = 0; s < 4; ++s) {
-            const uint4 &lo = x[0][s >> 1], &hi = x[1][s >> 1];
-            afr[m][s][0] = (s & 1) ? lo.z : lo.x;   // token g,   k 4s+0..1
-            afr[m][s][1] = (s & 1) ? hi.z : hi.x;   // token g+8, k 4s+0..1
-            afr[m][s][2] = (s & 1) ? lo.w : lo.y;   // token g,   k 4s+2..3
-            afr[m][s][3] = (s & 1) ? hi.w : hi.y;   // token g+8, k 4s+2..3
-          }
-        }
-#pragma unroll
-        for (int t = 0; t < 8; ++t) {
-          // codes of row 8t+g in block `warp`: bytes [8j, 8j+8) = 16 weights
-          const int row = 8 * t + g;
-          const uint32_t boff = warp * 32 + j * 8;             // byte offset in the 128-byte line
-          const uint2 cw = lds64(sc + row * 128 + ((((boff >> 4)) ^ (row & 7)) << 4) + (boff & 15));
-          // block constants of rows 8t+2j, 8t+2j+1 (the D fragment's columns)
-          const uint2 sv = lds64(ss + (warp * kGvRows + 8 * t + 2 * j) * 4);
-          uint32_t bfr[8];
-#pragma unroll
-          for (int b = 0; b < 4; ++b) {
-            bfr[b] = lut_decode(lane_base, cw.x, b);
-            bfr[4 + b] = lut_decode(lane_base, cw.y, b);
-          }
-#pragma unroll
-          for (int m = 0; m < MT; ++m) {
-            float pd[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-            for (int s = 0; s < 4; ++s) mma_bf16_16816(pd, afr[m][s], bfr[2 * s], bfr[2 * s + 1]);
-            const float s0 = __uint_as_float(sv.x), s1 = __uint_as_float(sv.y);
-            acc[t][m][0] = __fmaf_rn(s0, pd[0], acc[t][m][0]);
-            acc[t][m][1] = __fmaf_rn(s1, pd[1], acc[t][m][1]);
-            acc[t][m][2] = __fmaf_rn(s0, pd[2], acc[t][m][2]);
-            acc[t][m][3] = __fmaf_rn(s1, pd[3], acc[t][m][3]);
-          }
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(smem_u32(empty_bar + stage));
         if (++stage == S) {
           stage = 0;
           phase ^= 1;
         }
       }
-      if (!ok) break;
-      // reduce the four warps' partial sums and add them into the accumulator
-      float *myred = red + (warp * 32 + lane) * (32 * MT);
-#pragma unroll
-      for (int t = 0; t < 8; ++t)
-#pragma unroll
-        for (int m = 0; m < MT; ++m)
-#pragma unroll
-          for (int v = 0; v < 4; ++v) myred[(t * MT + m) * 4 + v] = acc[t][m][v];
-      named_bar_sync(1, 128);
-      // thread (lane', warp') sums element e = warp'*8*MT .. of lane' across the 4 warps
-      for (int e = warp * 8 * MT; e < (warp + 1) * 8 * MT; ++e) {
-        float v = 0.f;
-#pragma unroll
-        for (int w2 = 0; w2 < 4; ++w2) v += red[(w2 * 32 + lane) * (32 * MT) + e];
-        const int t = e / (4 * MT), m = (e / 4) % MT, q = e & 3;
-        const int tok = 16 * m + g + ((q & 2) ? 8 : 0);
-        const int row = rb * kGvRows + 8 * t + 2 * j + (q & 1);
-        if (tok < p.M && row < p.N) red_add_f32(p.acc + (int64_t)tok * p.N + row, v);
-      }
-      named_bar_sync(1, 128);
+    }
+    if (lane == 0)
+      for (int i = 0; i < S; ++i)
+        if (used & (1u << i)) mbar_wait(smem_u32(full_bar + i), (last_parity >> i) & 1u, p.err, DEV_TIMEOUT_DRAIN);
+  } else {
+    GvConsumer<NT> c;
+    c.init(p, smem, full_bar, empty_bar, kblocks);
+    // Flat walk over this CTA's (unit, stage) items, unrolled by two so the
+    // block constants of the next item load into the other buffer (no copies
+    // of in-flight loads) while the current item is decoded.
+    ConstPrefetch pa, pb;
+    pa.load(p, c.u, c.st, c.r0, c.j, kblocks);
+    while (c.u < p.units) {
+      if (!c.item(pa, pb)) break;
+      if (c.u >= p.units || !c.item(pb, pa)) break;
     }
   }
   // Complete only after the T launch this grid overlapped has completed, so

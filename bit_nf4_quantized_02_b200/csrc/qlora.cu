@@ -26,8 +26,8 @@ struct DeviceInfo {
   int sms = 0;
   int *err = nullptr;        // device address of g_dev_err
   bool gemm_attr[3] = {false, false, false};
-  int gemv_smem_set[3] = {0, 0, 0};   // dynamic smem limit set per MT variant
-  int gemv_per_sm[3] = {0, 0, 0};     // resident CTAs per SM per MT variant
+  int gemv_smem_set[3] = {0, 0, 0};   // dynamic smem limit set per NT variant
+  int gemv_per_sm[3] = {0, 0, 0};     // resident CTAs per SM per NT variant
 };
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_mu;
@@ -316,10 +316,10 @@ int launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cud
   return launch_status();
 }
 
-template <int MT>
+template <int NT>
 int launch_gemv(const qlora_nf4dq_t *W, const uint16_t *X, int64_t M, const uint16_t *L1, const uint16_t *L2, int r,
                 float s, uint16_t *Y, uint16_t *T_save, uint8_t *ws, DeviceInfo *dev, cudaStream_t st) {
-  using Cfg = GvCfg<MT>;
+  using Cfg = GvCfg<NT>;
   const int64_t N = W->n_out, K = W->k_in;
   const GemvLayout L = gemv_layout(M, N, r);
   if (cudaMemsetAsync(ws, 0, L.zero_bytes, st) != cudaSuccess) return QLORA_ERR_CUDA;
@@ -334,20 +334,20 @@ int launch_gemv(const qlora_nf4dq_t *W, const uint16_t *X, int64_t M, const uint
   {
     const cuuint64_t dims[3] = {64, (cuuint64_t)(K / 64), (cuuint64_t)M};
     const cuuint64_t strides[2] = {128, (cuuint64_t)K * 2};
-    const cuuint32_t box[3] = {64, 4, (cuuint32_t)(16 * MT)};
+    const cuuint32_t box[3] = {64, 4, (cuuint32_t)(8 * NT)};
     int rc = encode_tmap(&tm_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, X, dims, strides, box);
     if (rc) return rc;
   }
   const int smem = Cfg::kSmemBytes;
-  const int idx = MT - 1;
+  const int idx = NT == 1 ? 0 : (NT == 2 ? 1 : 2);
   if (dev->gemv_smem_set[idx] < smem) {
-    if (cudaFuncSetAttribute(gemv_fwd_kernel<MT>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+    if (cudaFuncSetAttribute(gemv_fwd_kernel<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
       return QLORA_ERR_CUDA;
     dev->gemv_smem_set[idx] = smem;
   }
   int &per_sm = dev->gemv_per_sm[idx];
   if (per_sm < 1 &&
-      (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, gemv_fwd_kernel<MT>, kGvThreads, smem) != cudaSuccess ||
+      (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, gemv_fwd_kernel<NT>, kGvThreads, smem) != cudaSuccess ||
        per_sm < 1))
     return QLORA_ERR_CUDA;
   GvArgs a;
@@ -374,7 +374,7 @@ int launch_gemv(const qlora_nf4dq_t *W, const uint16_t *X, int64_t M, const uint
                                                 reinterpret_cast<const __nv_bfloat16 *>(L1), (int)M, (int)K, r, tacc);
   int rc = launch_status();
   if (rc) return rc;
-  rc = launch_pdl(gemv_fwd_kernel<MT>, dim3(grid), dim3(kGvThreads), (size_t)smem, st, tm_codes, tm_x, a);
+  rc = launch_pdl(gemv_fwd_kernel<NT>, dim3(grid), dim3(kGvThreads), (size_t)smem, st, tm_codes, tm_x, a);
   if (rc) return rc;
   const size_t esmem = (size_t)M * r * 4 + (size_t)r * 64 * 2;
   if (esmem > 48 * 1024 &&
@@ -658,8 +658,9 @@ int qlora_linear_fwd(const uint16_t *X, int64_t M, const qlora_nf4dq_t *W, const
     if (!ws || ws_bytes < gemv_layout(M, N, r).total) return QLORA_ERR_WORKSPACE;
     if (!aligned(ws, 256)) return QLORA_ERR_MISALIGNED;
     uint8_t *w8 = reinterpret_cast<uint8_t *>(ws);
-    if (M <= 16) return launch_gemv<1>(W, X, M, L1, L2, r, s, Y, T_save, w8, dev, st);
-    return launch_gemv<2>(W, X, M, L1, L2, r, s, Y, T_save, w8, dev, st);
+    if (M <= 8) return launch_gemv<1>(W, X, M, L1, L2, r, s, Y, T_save, w8, dev, st);
+    if (M <= 16) return launch_gemv<2>(W, X, M, L1, L2, r, s, Y, T_save, w8, dev, st);
+    return launch_gemv<4>(W, X, M, L1, L2, r, s, Y, T_save, w8, dev, st);
   }
   const FwdLayout L = fwd_layout(M, N, K, r, dev->sms);
   if (!ws || ws_bytes < L.total) return QLORA_ERR_WORKSPACE;
