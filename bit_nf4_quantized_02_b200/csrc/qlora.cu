@@ -25,7 +25,8 @@ struct DeviceInfo {
   bool init = false;
   int sms = 0;
   int *err = nullptr;        // device address of g_dev_err
-  bool gemm_attr[3] = {false, false, false};
+  bool gemm_attr[4] = {false, false, false, false};   // BN 64, 128, 256; 256 in CTA pairs
+  int pair_clusters = 0;     // co-resident 2-CTA clusters of the pair GEMM
   int gemv_smem_set[3] = {0, 0, 0};   // dynamic smem limit set per NT variant
   int gemv_per_sm[3] = {0, 0, 0};     // resident CTAs per SM per NT variant
 };
@@ -179,6 +180,45 @@ int launch_gemm_bn(const CUtensorMap *maps, TcGemmArgs &args, int sms, DeviceInf
   return launch_status();
 }
 
+// CTA-pair GEMM (256 x 256 tiles): a persistent grid of 2-CTA clusters, as
+// many as can be resident at once.
+int launch_gemm_pair(const CUtensorMap *maps, TcGemmArgs &args, DeviceInfo *dev, cudaStream_t st, int kind) {
+  constexpr int BN = 256;
+  using Cfg = TcCfg<BN, true>;
+  auto kernel = tc_gemm_kernel<BN, true>;
+  cudaLaunchConfig_t cfg;
+  std::memset(&cfg, 0, sizeof(cfg));
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.blockDim = dim3(kGemmThreads, 1, 1);
+  cfg.dynamicSmemBytes = Cfg::kSmemBytes;
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (!dev->gemm_attr[3]) {
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes) != cudaSuccess)
+      return QLORA_ERR_CUDA;
+    cfg.gridDim = dim3(2 * (unsigned)dev->sms, 1, 1);
+    int clusters = 0;
+    if (cudaOccupancyMaxActiveClusters(&clusters, kernel, &cfg) != cudaSuccess || clusters < 1) return QLORA_ERR_CUDA;
+    dev->pair_clusters = clusters;
+    dev->gemm_attr[3] = true;
+  }
+  const int units = args.m_tiles * args.n_tiles * args.splits;
+  const int clusters = std::max(1, std::min(units, dev->pair_clusters));
+  cfg.gridDim = dim3(2 * (unsigned)clusters, 1, 1);
+  ProfScope prof(kind, st);
+  if (cudaLaunchKernelEx(&cfg, kernel, maps[0], maps[1], maps[2], maps[3], args) != cudaSuccess) return QLORA_ERR_CUDA;
+  return launch_status();
+}
+
+// The CTA-pair form serves the wide products (N > 128) that are not split
+// along K and have at least two 128-row tiles.
+bool use_pair(int bn, int splits, int64_t M) { return bn == 256 && splits == 1 && M > kBM; }
+
 // D[M x N] = alpha * sum_seg A_seg B_seg^T, written to `out` with strides
 // (ld_row, ld_col) as bf16 (optionally with a lo part at +lo_off) or fp32.
 // If `split_ws` is given and the tile grid leaves SMs idle, the reduction is
@@ -199,20 +239,22 @@ int tc_gemm(cudaStream_t st, DeviceInfo *dev, int64_t M, int64_t N, int nseg, co
   a.m_tiles = (int)((M + kBM - 1) / kBM);
   a.n_tiles = (int)((N + bn - 1) / bn);
   a.nseg = nseg;
-  for (int s = 0; s < nseg; ++s) {
-    a.seg[s].nkb = (int)((segs[s].A.kext + kBK - 1) / kBK);
-    a.seg[s].a_mn = segs[s].A.mn_major;
-    a.seg[s].b_mn = segs[s].B.mn_major;
-    int rc = make_tmap(&maps[2 * s], segs[s].A, kBM);
-    if (rc) return rc;
-    rc = make_tmap(&maps[2 * s + 1], segs[s].B, bn);
-    if (rc) return rc;
-  }
-  if (nseg == 1) maps[2] = maps[0], maps[3] = maps[1];
+  for (int s = 0; s < nseg; ++s) a.seg[s].nkb = (int)((segs[s].A.kext + kBK - 1) / kBK);
   if (split_all && (nseg < 2 || a.seg[1].nkb != a.seg[0].nkb)) split_all = false;
   int splits, kbps;
   choose_splits((int64_t)a.m_tiles * a.n_tiles, a.seg[0].nkb, dev->sms,
                 split_ws != nullptr && (nseg == 1 || split_all), &splits, &kbps);
+  const bool pair = use_pair(bn, splits, M);
+  if (pair) a.m_tiles = (int)((M + 2 * kBM - 1) / (2 * kBM));
+  for (int s = 0; s < nseg; ++s) {
+    a.seg[s].a_mn = segs[s].A.mn_major;
+    a.seg[s].b_mn = segs[s].B.mn_major;
+    int rc = make_tmap(&maps[2 * s], segs[s].A, kBM);
+    if (rc) return rc;
+    rc = make_tmap(&maps[2 * s + 1], segs[s].B, pair ? bn / 2 : bn);
+    if (rc) return rc;
+  }
+  if (nseg == 1) maps[2] = maps[0], maps[3] = maps[1];
   a.splits = splits;
   a.kb_per_split = kbps;
   a.split_all = split_all ? 1 : 0;
@@ -230,10 +272,14 @@ int tc_gemm(cudaStream_t st, DeviceInfo *dev, int64_t M, int64_t N, int nseg, co
     a.out_f32 = out_f32;
   }
   int rc;
-  switch (bn) {
-    case 64: rc = launch_gemm_bn<64>(maps, a, dev->sms, dev, st, kind); break;
-    case 128: rc = launch_gemm_bn<128>(maps, a, dev->sms, dev, st, kind); break;
-    default: rc = launch_gemm_bn<256>(maps, a, dev->sms, dev, st, kind); break;
+  if (pair) {
+    rc = launch_gemm_pair(maps, a, dev, st, kind);
+  } else {
+    switch (bn) {
+      case 64: rc = launch_gemm_bn<64>(maps, a, dev->sms, dev, st, kind); break;
+      case 128: rc = launch_gemm_bn<128>(maps, a, dev->sms, dev, st, kind); break;
+      default: rc = launch_gemm_bn<256>(maps, a, dev->sms, dev, st, kind); break;
+    }
   }
   if (rc || splits == 1) return rc;
   const int64_t count = M * N;

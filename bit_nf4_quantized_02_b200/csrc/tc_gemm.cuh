@@ -2,7 +2,7 @@
 //
 //   D[M x N] = alpha * sum_seg A_seg[M x K_seg] * B_seg[N x K_seg]^T
 //
-// One kernel, warp-specialised, one CTA per SM:
+// One kernel, warp-specialised, one CTA per SM (or one CTA pair per two SMs):
 //   warp 0        TMA producer: 128-byte-swizzled tiles of A and B into a ring
 //                 of shared-memory stages (mbarrier full/empty pairs);
 //   warp 1        allocates TMEM, one thread issues tcgen05.mma (bf16 in, fp32
@@ -15,7 +15,12 @@
 // stored layout), X^T*G and the LoRA extra K-steps all run on this engine.
 // A split of the reduction (split-K; of segment 0, or of every segment when
 // they have equal lengths) writes fp32 partials that a finalize kernel sums
-// in a fixed order.  A bf16 output can also be stored as a hi/lo pair
+// in a fixed order.  In the CTA-pair form (cta_group::2, a cluster of two
+// CTAs) the pair computes 256-row tiles: each CTA stages its 128 rows of A
+// and half of B's rows, the leader CTA issues 256-row MMAs that read both
+// CTAs' shared memory, and each CTA's epilogue drains its own 128 rows of
+// the accumulator -- half the B bytes per SM of the single-CTA form.
+// A bf16 output can also be stored as a hi/lo pair
 // (hi = bf16(v), lo = bf16(v - hi)) so that a later product can consume it
 // at nearly fp32 accuracy as two bf16 operands.
 #pragma once
@@ -48,15 +53,21 @@ struct TcGemmArgs {
   int *err;
 };
 
-template <int BN>
+// BN: output columns per tile.  PAIR: tile of 2*kBM rows computed by a CTA
+// pair, each CTA holding kBM rows of A and BN/2 rows of B.
+template <int BN, bool PAIR = false>
 struct TcCfg {
+  static constexpr int kTileM = PAIR ? 2 * kBM : kBM;
+  static constexpr int kBRows = PAIR ? BN / 2 : BN;   // B rows staged by one CTA
   static constexpr int kABytes = kBM * kBK * 2;
-  static constexpr int kBBytes = BN * kBK * 2;
+  static constexpr int kBBytes = kBRows * kBK * 2;
   static constexpr int kStageBytes = kABytes + kBBytes;
-  static constexpr int kStages = BN == 256 ? 4 : (BN == 128 ? 6 : 8);
+  static constexpr int kStages = PAIR ? 7 : (BN == 256 ? 4 : (BN == 128 ? 6 : 8));
   static constexpr int kTmemCols = 2 * BN;
   static constexpr int kBarBytes = 256;
   static constexpr int kSmemBytes = kStages * kStageBytes + kBarBytes + 1024;
+  static_assert(kSmemBytes <= 232448, "shared memory per CTA");
+  static_assert(!PAIR || BN % 128 == 0, "each CTA of a pair stages whole 64-row B atoms");
 };
 
 __device__ __forceinline__ void tc_unit_coords(int u, const TcGemmArgs &p, int &mt, int &nt, int &split) {
@@ -83,13 +94,18 @@ __device__ __forceinline__ void tc_seg_range(const TcGemmArgs &p, int s, int spl
   }
 }
 
-template <int BN>
+template <int BN, bool PAIR = false>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tA0, const __grid_constant__ CUtensorMap tB0,
                    const __grid_constant__ CUtensorMap tA1, const __grid_constant__ CUtensorMap tB1,
                    const TcGemmArgs p) {
-  using Cfg = TcCfg<BN>;
+  using Cfg = TcCfg<BN, PAIR>;
   constexpr int S = Cfg::kStages;
+  // Pair form: the grid is a 1-D array of 2-CTA clusters; CTA rank 0 leads.
+  const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
+  const bool leader = rank == 0;
+  const int first_unit = PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
+  const int unit_stride = PAIR ? (int)(gridDim.x >> 1) : (int)gridDim.x;
   extern __shared__ uint8_t smem_raw[];
   // 1024-byte alignment: the 128B-swizzle pattern repeats every 8 rows of 128 B.
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -111,7 +127,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(smem_u32(tfull_bar + i), 1);
-      mbar_init(smem_u32(tempty_bar + i), 4 * 32);
+      mbar_init(smem_u32(tempty_bar + i), PAIR ? 8 : 4);  // one arrive per epilogue warp (of both CTAs)
     }
     mbar_init(smem_u32(done_bar), 1);
     fence_mbar_init();
@@ -125,11 +141,22 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
   }
   if (warp == 1) {
-    tmem_alloc(smem_u32(tmem_slot), Cfg::kTmemCols);
-    tmem_relinquish();
+    if (PAIR) {
+      tmem_alloc_pair(smem_u32(tmem_slot), Cfg::kTmemCols);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(smem_u32(tmem_slot), Cfg::kTmemCols);
+      tmem_relinquish();
+    }
   }
   tc_fence_before();
-  __syncthreads();
+  // Pair form: neither CTA may touch its peer's barriers before they exist.
+  if (PAIR) {
+    __syncwarp();   // the cluster barrier is warp-aligned: reconverge after the role branches
+    cluster_sync();
+  } else {
+    __syncthreads();
+  }
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
@@ -143,9 +170,18 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       uint32_t used = 0;           // stages that received at least one load
       uint32_t last_parity = 0;    // parity of the last load issued into each stage
       bool ok = true;
-      for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
+      // Loads of either CTA of a pair complete on the leader's full barrier,
+      // which expects both CTAs' bytes.
+      auto load = [&](uint32_t dst, const CUtensorMap *m, uint32_t bar, int x, int y) {
+        if (PAIR) tma_load_2d_pair(dst, m, bar, x, y); else tma_load_2d(dst, m, bar, x, y);
+      };
+      const int a_row0 = (int)rank * kBM;           // this CTA's rows within the tile
+      const int b_row0 = (int)rank * Cfg::kBRows;
+      for (int u = first_unit; u < units && ok; u += unit_stride) {
         int mt, nt, split;
         tc_unit_coords(u, p, mt, nt, split);
+        const int am = mt * Cfg::kTileM + a_row0;
+        const int bn0 = nt * BN + b_row0;
         for (int s = 0; s < p.nseg && ok; ++s) {
           const CUtensorMap *ta = s == 0 ? &tA0 : &tA1;
           const CUtensorMap *tb = s == 0 ? &tB0 : &tB1;
@@ -156,21 +192,22 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
               ok = false;
               break;
             }
-            const uint32_t fb = smem_u32(full_bar + stage);
-            mbar_arrive_expect_tx(fb, Cfg::kStageBytes);
+            const uint32_t fb_local = smem_u32(full_bar + stage);
+            const uint32_t fb = PAIR ? mapa_shared(fb_local, 0) : fb_local;
+            if (leader) mbar_arrive_expect_tx(fb_local, (PAIR ? 2 : 1) * Cfg::kStageBytes);
             const uint32_t sa = smem_u32(smem + stage * Cfg::kStageBytes);
             const uint32_t sb = sa + Cfg::kABytes;
             if (!p.seg[s].a_mn) {
-              tma_load_2d(sa, ta, fb, kb * kBK, mt * kBM);
+              load(sa, ta, fb, kb * kBK, am);
             } else {
-              tma_load_2d(sa, ta, fb, mt * kBM, kb * kBK);
-              tma_load_2d(sa + 8192, ta, fb, mt * kBM + 64, kb * kBK);
+              load(sa, ta, fb, am, kb * kBK);
+              load(sa + 8192, ta, fb, am + 64, kb * kBK);
             }
             if (!p.seg[s].b_mn) {
-              tma_load_2d(sb, tb, fb, kb * kBK, nt * BN);
+              load(sb, tb, fb, kb * kBK, bn0);
             } else {
 #pragma unroll
-              for (int j = 0; j < BN / 64; ++j) tma_load_2d(sb + j * 8192, tb, fb, nt * BN + 64 * j, kb * kBK);
+              for (int j = 0; j < Cfg::kBRows / 64; ++j) load(sb + j * 8192, tb, fb, bn0 + 64 * j, kb * kBK);
             }
             used |= 1u << stage;
             last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
@@ -182,25 +219,36 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
       }
       // Drain: never leave the CTA while a tensor copy is still landing in
-      // shared memory.
-      for (int i = 0; i < S; ++i)
-        if (used & (1u << i)) mbar_wait(smem_u32(full_bar + i), (last_parity >> i) & 1u, p.err, DEV_TIMEOUT_DRAIN);
+      // shared memory.  A single CTA watches its full barriers.  In a pair the
+      // copies complete on the leader's barriers, so each CTA instead waits
+      // until the MMAs have consumed the last fill of every stage (its empty
+      // barrier completes the phase of that fill's parity); after one wait
+      // runs out the rest are skipped, the copies having long landed.
+      for (int i = 0; i < S; ++i) {
+        if (!(used & (1u << i))) continue;
+        const uint32_t par = (last_parity >> i) & 1u;
+        const bool done = PAIR ? mbar_wait(smem_u32(empty_bar + i), par, p.err, DEV_TIMEOUT_DRAIN)
+                               : mbar_wait(smem_u32(full_bar + i), par, p.err, DEV_TIMEOUT_DRAIN);
+        if (!done) break;
+      }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    // Pair form: the leader alone issues; the peer's tensor core works on the
+    // leader's instructions.
+    if (lane == 0 && leader) {
       uint32_t idesc[2];
-      for (int s = 0; s < 2; ++s) idesc[s] = idesc_bf16_f32(kBM, BN, p.seg[s].a_mn, p.seg[s].b_mn);
+      for (int s = 0; s < 2; ++s) idesc[s] = idesc_bf16_f32(Cfg::kTileM, BN, p.seg[s].a_mn, p.seg[s].b_mn);
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
       int t = 0;
-      for (int u = blockIdx.x; u < units && ok; u += gridDim.x, ++t) {
+      for (int u = first_unit; u < units && ok; u += unit_stride, ++t) {
         int mt, nt, split;
         tc_unit_coords(u, p, mt, nt, split);
         const int acc = t & 1;
         const uint32_t use = (uint32_t)(t >> 1);
-        if (!mbar_wait(smem_u32(tempty_bar + acc), (use & 1u) ^ 1u, p.err, DEV_TIMEOUT_MMA)) break;
+        if (!mbar_wait<PAIR>(smem_u32(tempty_bar + acc), (use & 1u) ^ 1u, p.err, DEV_TIMEOUT_MMA)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
         uint32_t accumulate = 0;
@@ -222,27 +270,36 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
               // MN-major: it starts 16 rows (2 KB) further down the tile.
               const uint64_t ad = a_mn ? smem_desc_sw128(sa + k * 2048, 8192, 1024) : smem_desc_sw128(sa + k * 32, 16, 1024);
               const uint64_t bd = b_mn ? smem_desc_sw128(sb + k * 2048, 8192, 1024) : smem_desc_sw128(sb + k * 32, 16, 1024);
-              tc_mma_f16(d_tmem, ad, bd, idesc[s], accumulate);
+              if (PAIR) tc_mma_f16_pair(d_tmem, ad, bd, idesc[s], accumulate);
+              else tc_mma_f16(d_tmem, ad, bd, idesc[s], accumulate);
               accumulate = 1;
             }
-            tc_commit(smem_u32(empty_bar + stage));  // frees the stage once these MMAs have read it
+            // frees the stage (in both CTAs of a pair) once these MMAs have read it
+            if (PAIR) tc_commit_pair(smem_u32(empty_bar + stage), 0x3);
+            else tc_commit(smem_u32(empty_bar + stage));
             if (++stage == S) {
               stage = 0;
               phase ^= 1;
             }
           }
         }
-        tc_commit(smem_u32(tfull_bar + acc));        // accumulator ready for the epilogue
+        // accumulator ready for the epilogue(s)
+        if (PAIR) tc_commit_pair(smem_u32(tfull_bar + acc), 0x3);
+        else tc_commit(smem_u32(tfull_bar + acc));
       }
       // All MMAs issued by this thread must finish before TMEM is released.
-      tc_commit(smem_u32(done_bar));
+      if (PAIR) tc_commit_pair(smem_u32(done_bar), 0x1);
+      else tc_commit(smem_u32(done_bar));
       mbar_wait(smem_u32(done_bar), 0, p.err, DEV_TIMEOUT_DRAIN);
     }
   } else {
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;  // TMEM lane quarter this warp may access
     int t = 0;
-    for (int u = blockIdx.x; u < units; u += gridDim.x, ++t) {
+    // The accumulator is released with one arrive per warp, on the leader's
+    // barrier in the pair form.
+    const uint32_t tempty0 = PAIR ? mapa_shared(smem_u32(tempty_bar), 0) : smem_u32(tempty_bar);
+    for (int u = first_unit; u < units; u += unit_stride, ++t) {
       int mt, nt, split;
       tc_unit_coords(u, p, mt, nt, split);
       const int acc = t & 1;
@@ -251,7 +308,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const bool got = mbar_wait(smem_u32(tfull_bar + acc), use & 1u, p.err, DEV_TIMEOUT_EPILOGUE);
       if (!__all_sync(0xFFFFFFFFu, got)) break;
       tc_fence_after();
-      const int row = mt * kBM + q * 32 + lane;
+      const int row = mt * Cfg::kTileM + (int)rank * kBM + q * 32 + lane;
       const bool row_ok = row < p.M;
       const float alpha = p.alpha;
 #pragma unroll 1
@@ -322,14 +379,28 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
       }
       tc_fence_before();
-      mbar_arrive(smem_u32(tempty_bar + acc));
+      __syncwarp();
+      if (lane == 0) {
+        if (PAIR) mbar_arrive_cluster(tempty0 + 8u * (uint32_t)acc);
+        else mbar_arrive(tempty0 + 8u * (uint32_t)acc);
+      }
     }
   }
 
   tc_fence_before();
-  __syncthreads();
+  // Pair form: no CTA leaves (or frees TMEM) while its peer may still signal
+  // its barriers or its MMAs may still run.
+  if (PAIR) {
+    __syncwarp();   // the cluster barrier is warp-aligned: reconverge after the role branches
+    cluster_sync();
+  } else {
+    __syncthreads();
+  }
   tc_fence_after();
-  if (warp == 1) tmem_dealloc(tmem_base, Cfg::kTmemCols);
+  if (warp == 1) {
+    if (PAIR) tmem_dealloc_pair(tmem_base, Cfg::kTmemCols);
+    else tmem_dealloc(tmem_base, Cfg::kTmemCols);
+  }
 }
 
 // Fixed-order sum of split-K partials (dense fp32 [splits][M][N]) into the
