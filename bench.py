@@ -135,8 +135,8 @@ class ClockSampler:
 
 # --------------------------------------------------------------------------- our arm
 class Linear:
-    def __init__(self, lin, X, dev, seed):
-        M, r = WL.M, WL.r
+    def __init__(self, lin, X, dev, seed, wl=WL):
+        M, r = wl.M, wl.r
         self.lin = lin
         N, K = lin.n_out, lin.k_in
         self.W = inputs.device_normal((N, K), inputs.WEIGHT_STD, seed, dev)
@@ -150,51 +150,49 @@ class Linear:
         self.q = None
 
 
-def build_layer(dev, rank):
-    M = WL.M
-    base = WL.seed + 1000 * rank
-    H = inputs.device_normal((M, 4096), 1.0, base + 11, dev, torch.bfloat16)      # q, k, v, gate, up
-    A = inputs.device_normal((M, 4096), 1.0, base + 12, dev, torch.bfloat16)      # o
-    U = inputs.device_normal((M, 11008), 1.0, base + 13, dev, torch.bfloat16)     # down
+def build_layer(dev, rank, wl=WL):
+    """The seven linears of one layer on independent seeded inputs."""
+    M = wl.M
+    hidden, mlp = wl.linears[0].k_in, wl.linears[4].n_out
+    base = wl.seed + 1000 * rank
+    H = inputs.device_normal((M, hidden), 1.0, base + 11, dev, torch.bfloat16)    # q, k, v, gate, up
+    A = inputs.device_normal((M, hidden), 1.0, base + 12, dev, torch.bfloat16)    # o
+    U = inputs.device_normal((M, mlp), 1.0, base + 13, dev, torch.bfloat16)       # down
     xs = {"q": H, "k": H, "v": H, "o": A, "gate": H, "up": H, "down": U}
-    lins = [Linear(l, xs[l.name], dev, WL.seed + 100 * i) for i, l in enumerate(WL.linears)]
+    lins = [Linear(l, xs[l.name], dev, wl.seed + 100 * i, wl) for i, l in enumerate(wl.linears)]
     # adapter gradients as views of one flat fp32 buffer (one all-reduce per step)
-    grads = FlatGrads([(l.lin.k_in, l.lin.n_out, WL.r) for l in lins], dev)
+    grads = FlatGrads([(l.lin.k_in, l.lin.n_out, wl.r) for l in lins], dev)
     for l, (dl1, dl2) in zip(lins, grads.views):
         l.dL1, l.dL2 = dl1, dl2
-    return lins, grads, (H, A, U)
+    return lins, grads, [H, A, U] + [l.dY for l in lins]
 
 
-def make_step(qlora, lins, grads, world):
+def make_step(qlora, lins, grads, world, wl=WL):
     def step():
         for l in lins:
             l.q = qlora.quantize_nf4_dq(l.W, out=l.q)
         for l in lins:
-            qlora.linear_fwd(l.X, l.q, l.L1, l.L2, WL.s, Y=l.Y, T=l.T)
+            qlora.linear_fwd(l.X, l.q, l.L1, l.L2, wl.s, Y=l.Y, T=l.T)
         for l in reversed(lins):
-            qlora.linear_bwd(l.dY, l.X, l.T, l.q, l.L1, l.L2, WL.s, grad_dtype=torch.float32,
+            qlora.linear_bwd(l.dY, l.X, l.T, l.q, l.L1, l.L2, wl.s, grad_dtype=torch.float32,
                              dX=l.dX, dL1=l.dL1, dL2=l.dL2)
         grads.allreduce()
     return step
 
 
-def run_e2e(args, step, lins, flat, acts, dev, world, e0, e1):
-    """Same step with host buffers: X and dY copied in, adapter gradients copied out."""
+def run_e2e(args, step, flat, acts, dev, world, e0, e1):
+    """Same step with host buffers: the step's activations and output gradients
+    (`acts`) copied in from pinned host memory, adapter gradients copied out."""
     pinned_in = [torch.empty(a.shape, dtype=a.dtype, pin_memory=True) for a in acts]
-    pinned_dy = [torch.empty(l.dY.shape, dtype=l.dY.dtype, pin_memory=True) for l in lins]
     for h, a in zip(pinned_in, acts):
         h.copy_(a)
-    for h, l in zip(pinned_dy, lins):
-        h.copy_(l.dY)
     grads_host = torch.empty(flat.shape, dtype=flat.dtype, pin_memory=True)
-    h2d = sum(t.numel() * t.element_size() for t in pinned_in + pinned_dy)
+    h2d = sum(t.numel() * t.element_size() for t in pinned_in)
     d2h = grads_host.numel() * grads_host.element_size()
 
     def e2e_step():
         for h, a in zip(pinned_in, acts):
             a.copy_(h, non_blocking=True)
-        for h, l in zip(pinned_dy, lins):
-            l.dY.copy_(h, non_blocking=True)
         step()
         grads_host.copy_(flat, non_blocking=True)
 
@@ -215,6 +213,10 @@ def run_e2e(args, step, lins, flat, acts, dev, world, e0, e1):
 
     return ms_e2e, h2d, d2h
 
+TRAIN = {"llama7b-train": workloads.LLAMA7B_LAYER, "llama65b-train": workloads.LLAMA65B_LAYER,
+         "llama33b-stack": workloads.LLAMA33B_STACK}
+
+
 def run_ours(args, rank, world, local_rank):
     import bit_nf4_quantized_02_b200 as qlora
     from bit_nf4_quantized_02_b200 import _lib
@@ -222,13 +224,26 @@ def run_ours(args, rank, world, local_rank):
     _lib.load()
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
-    lins, grads, acts = build_layer(dev, rank)
-    flat = grads.flat
-    if args.linear:
-        lins = [l for l in lins if l.lin.name == args.linear]
-    for l in lins:  # allocate the quantized buffers once
-        l.q = qlora.quantize_nf4_dq(l.W)
-    step = make_step(qlora, lins, grads, world)
+    wl = TRAIN[args.workload]
+    if wl.layers > 1:
+        from bit_nf4_quantized_02_b200.stack import QLoRAStack, SEEDED_DY
+        hidden, mlp = wl.linears[0].n_out, wl.linears[4].n_out
+        st = QLoRAStack(qlora, hidden, mlp, wl.layers, wl.M, wl.r, wl.alpha, wl.seed + 100_000 * rank, dev,
+                        lambda shape, std, seed, dtype: inputs.device_normal(shape, std, seed, dev, dtype))
+        st.quantize()     # allocate the quantized buffers once
+        grads, flat = st.grads, st.grads.flat
+        acts = [st.H[0], st.dH[-1]] + st.R + [st.lin[l][n].dY for l in range(wl.layers) for n in SEEDED_DY]
+        step = st.step
+        sel = wl.linears * wl.layers
+    else:
+        lins, grads, acts = build_layer(dev, rank, wl)
+        flat = grads.flat
+        if args.linear:
+            lins = [l for l in lins if l.lin.name == args.linear]
+        for l in lins:  # allocate the quantized buffers once
+            l.q = qlora.quantize_nf4_dq(l.W)
+        step = make_step(qlora, lins, grads, world, wl)
+        sel = [l.lin for l in lins]
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
@@ -242,7 +257,7 @@ def run_ours(args, rank, world, local_rank):
     if sampler:
         sampler.start()
         time.sleep(0.5)
-    qlora.profile_start(args.steps * 200 + 64)
+    qlora.profile_start(args.steps * 200 * wl.layers + 64)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record()
     for _ in range(args.steps):
@@ -265,12 +280,11 @@ def run_ours(args, rank, world, local_rank):
     if args.no_e2e:
         ms_e2e, h2d, d2h = None, None, None
     else:
-        ms_e2e, h2d, d2h = run_e2e(args, step, lins, flat, acts, dev, world, e0, e1)
+        ms_e2e, h2d, d2h = run_e2e(args, step, flat, acts, dev, world, e0, e1)
 
     if rank != 0:
         return None
-    sel = [l.lin for l in lins]
-    flops = step_flops(sel) * world
+    flops = step_flops(sel, wl.M, wl.r) * world
     value = flops / (ms * 1e-3) / 1e12
     peaks, peak_src = load_peaks()
     # dominant kernel: the tcgen05 GEMM launches of the Y and dX products
@@ -281,8 +295,8 @@ def run_ours(args, rank, world, local_rank):
         c[1] += kms
     dom_ms = per_kind.get("gemm_Y", [0, 0.0])[1] + per_kind.get("gemm_dX", [0, 0.0])[1]
     dom_n = per_kind.get("gemm_Y", [0, 0.0])[0] + per_kind.get("gemm_dX", [0, 0.0])[0]
-    dom_flops = args.steps * sum(linear_flops(WL.M, l.n_out, l.k_in, WL.r)["gemm_Y"] +
-                                 linear_flops(WL.M, l.n_out, l.k_in, WL.r)["gemm_dX"] for l in sel)
+    dom_flops = args.steps * sum(linear_flops(wl.M, l.n_out, l.k_in, wl.r)["gemm_Y"] +
+                                 linear_flops(wl.M, l.n_out, l.k_in, wl.r)["gemm_dX"] for l in sel)
     achieved = dom_flops / (dom_ms * 1e-3) / 1e12 if dom_ms > 0 else None
     peak = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
     # DRAM traffic per launch: the ncu-measured ratio of DRAM bytes to algorithmic
@@ -294,7 +308,7 @@ def run_ours(args, rank, world, local_rank):
         with open(tp) as f:
             tr = json.load(f)
         if tr.get("source_hash") == source_hash("tc_gemm.cuh", "common.cuh"):
-            M, r = WL.M, WL.r
+            M, r = wl.M, wl.r
             alg = [2 * M * l.k_in + 2 * l.n_out * l.k_in + 2 * M * l.n_out + 2 * M * r + 2 * r * l.n_out for l in sel]
             alg += [2 * M * l.n_out + 2 * l.n_out * l.k_in + 2 * M * l.k_in + 2 * M * r + 2 * r * l.k_in for l in sel]
             traffic = tr["traffic_over_algorithmic"] * sum(alg) / len(alg)
@@ -306,11 +320,16 @@ def run_ours(args, rank, world, local_rank):
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": WL.name + (f"[{args.linear} only]" if args.linear else ""),
-                   "model": "llama7b-layer-linears", "global_batch": 16 * world,
-                   "seq_len": 512, "tokens_per_rank": WL.M, "lora_r": WL.r, "lora_alpha": WL.alpha,
+        "config": {"workload": wl.name + (f"[{args.linear} only]" if args.linear else ""),
+                   "model": {"llama7b-train": "llama7b-layer-linears", "llama65b-train": "llama65b-layer-linears",
+                             "llama33b-stack": "llama33b-8-layer-stack"}[args.workload],
+                   "global_batch": (16 if wl.M == 8192 and args.workload == "llama7b-train" else 4) * world,
+                   "seq_len": 512 if args.workload == "llama7b-train" else 2048,
+                   "tokens_per_rank": wl.M, "lora_r": wl.r, "lora_alpha": wl.alpha, "layers": wl.layers,
                    "parallelism": f"dp{world}" if world > 1 else "single",
-                   "step": "quantize 7 fp32 weights to NF4+DQ, fwd + bwd of the 7 QLoRA linears"
+                   "step": f"quantize {7 * wl.layers} fp32 weights to NF4+DQ, fwd + bwd of the "
+                           f"{7 * wl.layers} QLoRA linears"
+                           + (" (layer to layer: H' = bf16(down(up(H)) + R))" if wl.layers > 1 else "")
                            + (", all-reduce of adapter grads" if world > 1 else ""),
                    "l2": "inputs larger than L2 (>1 GB touched per step), no flush"},
         "e2e": ({"value": flops / (ms_e2e * 1e-3) / 1e12, "unit": UNIT, "h2d_bytes_per_step": h2d,
@@ -325,7 +344,7 @@ def run_ours(args, rank, world, local_rank):
         "kernels": kernels,
         "clocks": clocks,
     }
-    if world == 1 and not args.no_cpu_baseline and not args.linear:
+    if world == 1 and not args.no_cpu_baseline and not args.linear and args.workload == "llama7b-train":
         out["cpu_baseline"] = cpu_baseline()
     return out
 
@@ -431,7 +450,7 @@ def run_decode(args, rank, world, local_rank):
         return None
     peaks, peak_src = load_peaks()
     per_kind, kernels = _kernel_table(launches, args.steps)
-    dom = per_kind.get("gemv_fwd", [0, 0.0])
+    dom = per_kind.get("fused_fwd", per_kind.get("gemv_fwd", [0, 0.0]))
     achieved = nbytes * args.steps / (dom[1] * 1e-3) / 1e9 if dom[1] > 0 else None
     peak = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
     return {
@@ -593,10 +612,12 @@ def main():
     ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end (host buffers) measurement")
     ap.add_argument("--linear", choices=[l.name for l in WL.linears], default=None,
                     help="restrict the step to one linear of the layer (profiling runs)")
-    ap.add_argument("--workload", choices=["llama7b-train", "llama65b-decode", "quantizer"], default="llama7b-train",
+    ap.add_argument("--workload", choices=list(TRAIN) + ["llama65b-decode", "quantizer"], default="llama7b-train",
                     help="llama7b-train (default, the headline): quantize + fwd + bwd of a LLaMA-7B layer at 8192 "
-                         "tokens; llama65b-decode: forward of a LLaMA-65B layer at 16 tokens; quantizer: NF4+DQ "
-                         "quantize and dequantize of LLaMA-7B-shaped bf16 weights")
+                         "tokens; llama65b-train: the same for a LLaMA-65B layer at 4x2048 tokens; llama33b-stack: "
+                         "eight LLaMA-33B layers at 4x2048 tokens, forward then backward; llama65b-decode: forward "
+                         "of a LLaMA-65B layer at 16 tokens; quantizer: NF4+DQ quantize and dequantize of "
+                         "LLaMA-7B-shaped bf16 weights")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3

@@ -385,61 +385,71 @@ __global__ void __launch_bounds__(kGvThreads, 3)
 
 // T accumulation for few tokens: tacc[M x r] += X[:, k-slice] L1[k-slice, :]
 // for a 64-wide K slice per CTA (blockIdx.x) and a 64-wide column slice
-// (blockIdx.y).  Inputs are staged in shared memory with coalesced loads, then
-// each thread forms 4 tokens x 1 column over the slice and adds it with
-// red.global.add.  Lets its dependent launch start immediately.
+// (blockIdx.y).  Inputs are staged in shared memory with coalesced loads (X in
+// chunks of 32 tokens), then each thread forms 4 tokens x 1 column over the
+// slice and adds it with red.global.add.  Lets its dependent launch start
+// immediately.
 constexpr int kTSliceK = 64;
+constexpr int kTokChunk = 32;
 
 __global__ void __launch_bounds__(256) lora_down_small_kernel(const __nv_bfloat16 *__restrict__ X,
                                                               const __nv_bfloat16 *__restrict__ L1, int M, int K,
                                                               int r, float *__restrict__ tacc) {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-  __shared__ float xs[kGvMaxM][kTSliceK + 1];
+  __shared__ float xs[kTokChunk][kTSliceK + 1];
   __shared__ float ls[kTSliceK][65];
   const int k0 = blockIdx.x * kTSliceK;
   const int kn = min(kTSliceK, K - k0);
   const int j0 = blockIdx.y * 64;
   const int jn = min(64, r - j0);
-  for (int i = threadIdx.x; i < kGvMaxM * kTSliceK; i += blockDim.x) {
-    const int m = i / kTSliceK, k = i - m * kTSliceK;
-    xs[m][k] = (m < M && k < kn) ? __bfloat162float(X[(int64_t)m * K + k0 + k]) : 0.f;
-  }
   for (int i = threadIdx.x; i < kTSliceK * 64; i += blockDim.x) {
     const int k = i >> 6, jj = i & 63;
     ls[k][jj] = (k < kn && jj < jn) ? __bfloat162float(L1[(int64_t)(k0 + k) * r + j0 + jj]) : 0.f;
   }
-  __syncthreads();
   const int jj = threadIdx.x & 63;
-  for (int m0 = (threadIdx.x >> 6) * 4; m0 < M; m0 += 16) {
-    float t[4] = {0.f, 0.f, 0.f, 0.f};
-    for (int k = 0; k < kn; ++k) {
-      const float l = ls[k][jj];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) t[i] = __fmaf_rn(xs[m0 + i][k], l, t[i]);
+  for (int mc = 0; mc < M; mc += kTokChunk) {
+    const int mn = min(kTokChunk, M - mc);
+    __syncthreads();   // ls staged; the previous chunk's xs no longer read
+    for (int i = threadIdx.x; i < kTokChunk * kTSliceK; i += blockDim.x) {
+      const int m = i / kTSliceK, k = i - m * kTSliceK;
+      xs[m][k] = (m < mn && k < kn) ? __bfloat162float(X[(int64_t)(mc + m) * K + k0 + k]) : 0.f;
     }
-    if (jj < jn) {
+    __syncthreads();
+    for (int m0 = (threadIdx.x >> 6) * 4; m0 < mn; m0 += 16) {
+      float t[4] = {0.f, 0.f, 0.f, 0.f};
+      for (int k = 0; k < kn; ++k) {
+        const float l = ls[k][jj];
 #pragma unroll
-      for (int i = 0; i < 4; ++i)
-        if (m0 + i < M) red_add_f32(tacc + (m0 + i) * r + j0 + jj, t[i]);
+        for (int i = 0; i < 4; ++i) t[i] = __fmaf_rn(xs[m0 + i][k], l, t[i]);
+      }
+      if (jj < jn) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          if (m0 + i < mn) red_add_f32(tacc + (mc + m0 + i) * r + j0 + jj, t[i]);
+      }
     }
   }
 }
 
 // Y[tok][n] = bf16(acc[tok][n] + sum_j (s T)[tok][j] L2[j][n]).  A CTA owns 64
-// columns: it stages their L2 slice (r x 64) before waiting for the product
-// kernel (L2 is an input), then s T, then thread (column c, token group q)
-// forms tokens q, q+4, q+8, ...  Block 0 also writes T = s X L1 as a bf16
-// hi/lo pair.  Launched as a programmatic dependent of gemv_fwd_kernel.
+// columns (blockIdx.x) of 32 tokens (blockIdx.y): it stages their L2 slice
+// (r x 64) before waiting for the product kernel (L2 is an input), then s T
+// of its tokens, then thread (column c, token group q) forms tokens q, q+4,
+// ..., q+28.  Blocks of the first column slice also write T = s X L1 of their
+// tokens as a bf16 hi/lo pair.  Launched as a programmatic dependent of the
+// product kernel.
 __global__ void __launch_bounds__(256) gemv_epilogue_kernel(const float *__restrict__ acc,
                                                             const float *__restrict__ tacc,
                                                             const __nv_bfloat16 *__restrict__ L2, int M, int N, int r,
                                                             float s, __nv_bfloat16 *__restrict__ Y,
                                                             __nv_bfloat16 *__restrict__ T_save) {
   extern __shared__ float esm[];
-  float *ts = esm;                                                 // [M x r] s*T
-  __nv_bfloat16 *l2s = reinterpret_cast<__nv_bfloat16 *>(esm + M * r);  // [r x 64]
+  float *ts = esm;                                                        // [32 x r] s*T
+  __nv_bfloat16 *l2s = reinterpret_cast<__nv_bfloat16 *>(esm + kTokChunk * r);  // [r x 64]
   const int nb = blockIdx.x * 64;
   const int ncols = min(64, N - nb);
+  const int mb = blockIdx.y * kTokChunk;
+  const int mn = min(kTokChunk, M - mb);
   for (int i = threadIdx.x; i < r * 8; i += blockDim.x) {
     const int jj = i >> 3, c = i & 7;  // 16-byte chunk c of row jj of the slice
     uint4 v = make_uint4(0, 0, 0, 0);
@@ -447,12 +457,12 @@ __global__ void __launch_bounds__(256) gemv_epilogue_kernel(const float *__restr
     reinterpret_cast<uint4 *>(l2s + jj * 64)[c] = v;
   }
   asm volatile("griddepcontrol.wait;" ::: "memory");
-  for (int i = threadIdx.x; i < M * r; i += blockDim.x) ts[i] = s * __ldcg(tacc + i);
+  for (int i = threadIdx.x; i < mn * r; i += blockDim.x) ts[i] = s * __ldcg(tacc + (int64_t)mb * r + i);
   __syncthreads();
   if (blockIdx.x == 0 && T_save) {
-    for (int i = threadIdx.x; i < M * r; i += blockDim.x) {
+    for (int i = threadIdx.x; i < mn * r; i += blockDim.x) {
       const float v = ts[i];
-      const int m = i / r, jj = i - m * r;
+      const int m = mb + i / r, jj = i % r;
       const __nv_bfloat16 hb = __float2bfloat16_rn(v);
       T_save[(int64_t)m * 2 * r + jj] = hb;
       T_save[(int64_t)m * 2 * r + r + jj] = __float2bfloat16_rn(v - __bfloat162float(hb));
@@ -461,25 +471,25 @@ __global__ void __launch_bounds__(256) gemv_epilogue_kernel(const float *__restr
   const int c = threadIdx.x & 63, q = threadIdx.x >> 6;
   const int n = nb + c;
   if (c >= ncols) return;
-  constexpr int kTok = kGvMaxM / 4;
+  constexpr int kTok = kTokChunk / 4;
   float y[kTok];
 #pragma unroll
   for (int i = 0; i < kTok; ++i) {
     const int m = q + 4 * i;
-    y[i] = m < M ? __ldcg(acc + (int64_t)m * N + n) : 0.f;
+    y[i] = m < mn ? __ldcg(acc + (int64_t)(mb + m) * N + n) : 0.f;
   }
   for (int jj = 0; jj < r; ++jj) {
     const float l2 = __bfloat162float(l2s[jj * 64 + c]);
 #pragma unroll
     for (int i = 0; i < kTok; ++i) {
       const int m = q + 4 * i;
-      if (m < M) y[i] = __fmaf_rn(ts[m * r + jj], l2, y[i]);
+      if (m < mn) y[i] = __fmaf_rn(ts[m * r + jj], l2, y[i]);
     }
   }
 #pragma unroll
   for (int i = 0; i < kTok; ++i) {
     const int m = q + 4 * i;
-    if (m < M) Y[(int64_t)m * N + n] = __float2bfloat16_rn(y[i]);
+    if (m < mn) Y[(int64_t)(mb + m) * N + n] = __float2bfloat16_rn(y[i]);
   }
 }
 

@@ -12,6 +12,7 @@
 #include "quant.cuh"
 #include "tc_gemm.cuh"
 #include "gemv.cuh"
+#include "fused_fwd.cuh"
 
 namespace qlora {
 
@@ -29,6 +30,7 @@ struct DeviceInfo {
   int pair_clusters = 0;     // co-resident 2-CTA clusters of the pair GEMM
   int gemv_smem_set[3] = {0, 0, 0};   // dynamic smem limit set per NT variant
   int gemv_per_sm[3] = {0, 0, 0};     // resident CTAs per SM per NT variant
+  int fused_smem_set[4] = {0, 0, 0, 0};   // dynamic smem limit set per token-padding variant
 };
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_mu;
@@ -362,6 +364,79 @@ int launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cud
   return launch_status();
 }
 
+// Y = bf16(acc + s T L2) and the T hi/lo pair, as a programmatic dependent of
+// the product kernel just launched.
+int launch_lora_epilogue(const float *acc, const float *tacc, const __nv_bfloat16 *L2, int64_t M, int64_t N, int r,
+                         float s, uint16_t *Y, uint16_t *T_save, cudaStream_t st) {
+  const size_t esmem = (size_t)kTokChunk * r * 4 + (size_t)r * 64 * 2;
+  if (esmem > 48 * 1024 &&
+      cudaFuncSetAttribute(gemv_epilogue_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)esmem) != cudaSuccess)
+    return QLORA_ERR_CUDA;
+  const dim3 grid((unsigned)((N + 63) / 64), (unsigned)((M + kTokChunk - 1) / kTokChunk));
+  return launch_pdl(gemv_epilogue_kernel, grid, dim3(256), esmem, st, acc, tacc, L2, (int)M, (int)N, r, s,
+                    reinterpret_cast<__nv_bfloat16 *>(Y), reinterpret_cast<__nv_bfloat16 *>(T_save));
+}
+
+// Fused doubleDequant + tcgen05 forward for M <= 128 tokens (MP = padded M):
+// T accumulation, then the product (a programmatic dependent of it), then the
+// LoRA epilogue.
+template <int MP>
+int launch_fused_fwd(const qlora_nf4dq_t *W, const uint16_t *X, int64_t M, const uint16_t *L1, const uint16_t *L2,
+                     int r, float s, uint16_t *Y, uint16_t *T_save, uint8_t *ws, DeviceInfo *dev, cudaStream_t st) {
+  using Cfg = FtCfg<MP>;
+  const int64_t N = W->n_out, K = W->k_in;
+  const GemvLayout L = gemv_layout(M, N, r);
+  if (cudaMemsetAsync(ws, 0, L.zero_bytes, st) != cudaSuccess) return QLORA_ERR_CUDA;
+  CUtensorMap tm_codes, tm_x;
+  {
+    const cuuint64_t dims[2] = {(cuuint64_t)(K / 2), (cuuint64_t)N};
+    const cuuint64_t strides[1] = {(cuuint64_t)(K / 2)};
+    const cuuint32_t box[2] = {128, (cuuint32_t)kFtRows};
+    int rc = encode_tmap(&tm_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, W->codes, dims, strides, box);
+    if (rc) return rc;
+  }
+  {
+    // X as [64-block][token][64]: one box = the four K-major atoms of a stage
+    const cuuint64_t dims[3] = {64, (cuuint64_t)M, (cuuint64_t)(K / 64)};
+    const cuuint64_t strides[2] = {(cuuint64_t)K * 2, 128};
+    const cuuint32_t box[3] = {64, (cuuint32_t)MP, 4};
+    int rc = encode_tmap(&tm_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, X, dims, strides, box);
+    if (rc) return rc;
+  }
+  const int idx = MP == 16 ? 0 : (MP == 32 ? 1 : (MP == 64 ? 2 : 3));
+  if (dev->fused_smem_set[idx] < Cfg::kSmemBytes) {
+    if (cudaFuncSetAttribute(nf4_fused_fwd_kernel<MP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             Cfg::kSmemBytes) != cudaSuccess)
+      return QLORA_ERR_CUDA;
+    dev->fused_smem_set[idx] = Cfg::kSmemBytes;
+  }
+  FtArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.M = (int)M;
+  a.N = (int)N;
+  a.K = (int)K;
+  a.kstages = (int)((K + kFtStageK - 1) / kFtStageK);
+  a.items = (int)((N + kFtRows - 1) / kFtRows) * a.kstages;
+  a.c2_fp8 = W->c2_fp8;
+  a.c1 = W->c1;
+  a.mu = W->c2_mean;
+  a.acc = reinterpret_cast<float *>(ws + L.acc);
+  a.err = dev->err;
+  float *tacc = reinterpret_cast<float *>(ws + L.tacc);
+  const int grid = std::max(1, std::min(a.items, dev->sms));
+  ProfScope prof(QLORA_KERNEL_FUSED_FWD, st);
+  // 1. T accumulation; 2. the fused product, overlapping it; 3. the LoRA epilogue.
+  const dim3 tgrid((unsigned)((K + kTSliceK - 1) / kTSliceK), (unsigned)((r + 63) / 64));
+  lora_down_small_kernel<<<tgrid, 256, 0, st>>>(reinterpret_cast<const __nv_bfloat16 *>(X),
+                                                reinterpret_cast<const __nv_bfloat16 *>(L1), (int)M, (int)K, r, tacc);
+  int rc = launch_status();
+  if (rc) return rc;
+  rc = launch_pdl(nf4_fused_fwd_kernel<MP>, dim3(grid), dim3(Cfg::kThreads), (size_t)Cfg::kSmemBytes, st, tm_codes,
+                  tm_x, a);
+  if (rc) return rc;
+  return launch_lora_epilogue(a.acc, tacc, reinterpret_cast<const __nv_bfloat16 *>(L2), M, N, r, s, Y, T_save, st);
+}
+
 template <int NT>
 int launch_gemv(const qlora_nf4dq_t *W, const uint16_t *X, int64_t M, const uint16_t *L1, const uint16_t *L2, int r,
                 float s, uint16_t *Y, uint16_t *T_save, uint8_t *ws, DeviceInfo *dev, cudaStream_t st) {
@@ -422,13 +497,7 @@ int launch_gemv(const qlora_nf4dq_t *W, const uint16_t *X, int64_t M, const uint
   if (rc) return rc;
   rc = launch_pdl(gemv_fwd_kernel<NT>, dim3(grid), dim3(kGvThreads), (size_t)smem, st, tm_codes, tm_x, a);
   if (rc) return rc;
-  const size_t esmem = (size_t)M * r * 4 + (size_t)r * 64 * 2;
-  if (esmem > 48 * 1024 &&
-      cudaFuncSetAttribute(gemv_epilogue_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)esmem) != cudaSuccess)
-    return QLORA_ERR_CUDA;
-  return launch_pdl(gemv_epilogue_kernel, dim3((unsigned)((N + 63) / 64)), dim3(256), esmem, st,
-                    (const float *)a.acc, (const float *)tacc, a.L2, (int)M, (int)N, r, s,
-                    reinterpret_cast<__nv_bfloat16 *>(Y), reinterpret_cast<__nv_bfloat16 *>(T_save));
+  return launch_lora_epilogue(a.acc, tacc, a.L2, M, N, r, s, Y, T_save, st);
 }
 
 struct FwdLayout {
@@ -673,7 +742,7 @@ int qlora_dequant(const qlora_nf4dq_t *W, uint16_t *W_out, void *stream) {
 
 size_t qlora_linear_fwd_workspace_size(int64_t M, int64_t n_out, int64_t k_in, int r) {
   if (M < 0 || n_out <= 0 || k_in <= 0 || r <= 0) return 0;
-  if (M <= kGvMaxM) return gemv_layout(M, n_out, r).total;
+  if (M <= kFtMaxM) return gemv_layout(M, n_out, r).total;
   DeviceInfo *dev;
   const int sms = current_device_info(&dev) == QLORA_OK ? dev->sms : 148;
   return fwd_layout(M, n_out, k_in, r, sms).total;
@@ -699,14 +768,18 @@ int qlora_linear_fwd(const uint16_t *X, int64_t M, const qlora_nf4dq_t *W, const
   if (rc) return rc;
   const int64_t N = W->n_out, K = W->k_in;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  if (M <= kGvMaxM) {
+  if (M <= kFtMaxM) {
     // Few tokens: the weight bytes dominate; one fused decode + product pass.
     if (!ws || ws_bytes < gemv_layout(M, N, r).total) return QLORA_ERR_WORKSPACE;
     if (!aligned(ws, 256)) return QLORA_ERR_MISALIGNED;
     uint8_t *w8 = reinterpret_cast<uint8_t *>(ws);
+    // up to 32 tokens: weight decoded straight into mma.sync fragments (each
+    // warp independent); 33..128: decoded into shared memory for tcgen05
     if (M <= 8) return launch_gemv<1>(W, X, M, L1, L2, r, s, Y, T_save, w8, dev, st);
     if (M <= 16) return launch_gemv<2>(W, X, M, L1, L2, r, s, Y, T_save, w8, dev, st);
-    return launch_gemv<4>(W, X, M, L1, L2, r, s, Y, T_save, w8, dev, st);
+    if (M <= kGvMaxM) return launch_gemv<4>(W, X, M, L1, L2, r, s, Y, T_save, w8, dev, st);
+    if (M <= 64) return launch_fused_fwd<64>(W, X, M, L1, L2, r, s, Y, T_save, w8, dev, st);
+    return launch_fused_fwd<128>(W, X, M, L1, L2, r, s, Y, T_save, w8, dev, st);
   }
   const FwdLayout L = fwd_layout(M, N, K, r, dev->sms);
   if (!ws || ws_bytes < L.total) return QLORA_ERR_WORKSPACE;

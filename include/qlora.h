@@ -214,7 +214,8 @@ QLORA_API int qlora_get_last_device_error(void *stream);
 #define QLORA_KERNEL_GEMM_DL2 14    /* dL2 = T^T dY */
 #define QLORA_KERNEL_GEMM_DL1 15    /* dL1 = X^T G */
 #define QLORA_KERNEL_SPLITK_FINALIZE 20
-#define QLORA_KERNEL_GEMV_FWD 30    /* fused decode + product for few tokens */
+#define QLORA_KERNEL_GEMV_FWD 30    /* fused decode + mma.sync product, up to 32 tokens */
+#define QLORA_KERNEL_FUSED_FWD 31   /* fused decode + tcgen05 product, up to 128 tokens */
 QLORA_API int qlora_profile_start(int capacity);
 QLORA_API int qlora_profile_stop(void);
 QLORA_API int qlora_profile_read(int i, int *kind, float *ms);

@@ -16,10 +16,12 @@ aiingo.vercel.app/paper/paper-2305-14314) defines:
 * ``qlora_linear`` -- the QLoRA linear layer forward (§2 Eq. 3, §3 Eq. 5) and
                       its backward with adapter-only gradients (§3, the
                       paragraph after Eq. 6), in float64.
+* ``stack``        -- the wiring between the layers of a stack of such
+                      linears (a reading: the pages give no model code).
 
 Every function is pinned by ``tests/test_oracle_*.py`` against values the
 paper prints, closed forms, library special cases or brute force.  It shares
 no code, table or constant with the CUDA path.
 """
 
-from . import nf4dq, qlora_linear  # noqa: F401
+from . import nf4dq, qlora_linear, stack  # noqa: F401

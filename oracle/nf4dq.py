@@ -379,6 +379,32 @@ def dequantize_rows(w, rows) -> np.ndarray:
     return out
 
 
+def dequantize_cols(w, cols) -> np.ndarray:
+    """doubleDequant of selected columns of a 2-D weight: [n_out, len(cols)].
+
+    The same steps as ``quantize_nf4_dq`` + ``dequantize``: every block's c2
+    and their Double Quantization (the mean and each 256-group need all of
+    them), then the codes of the selected elements only.  Requires
+    k_in % 64 == 0 (blocks do not straddle rows).
+    """
+    w = f32(w)
+    n_out, k_in = w.shape
+    if k_in % W_BLOCK:
+        raise ValueError("dequantize_cols: k_in must be a multiple of 64")
+    cols = np.asarray(cols, dtype=np.int64)
+    bpr = k_in // W_BLOCK
+    c2 = block_absmax(w.reshape(-1), W_BLOCK)
+    code8, c1, mu = double_quantize(c2)
+    c2_hat = dequant_c2(code8, c1, mu).reshape(n_out, bpr)[:, cols // W_BLOCK]
+    c2_sel = c2.reshape(n_out, bpr)[:, cols // W_BLOCK]
+    with np.errstate(invalid="ignore", divide="ignore"):
+        x = (w[:, cols] / c2_sel).astype(np.float32)      # IEEE float32 quotient
+    codes = nf4_code(np.where(c2_sel == 0, np.float32(0), x))
+    codes = np.where(c2_sel == 0, NF4_ZERO_CODE, codes).astype(np.uint8)
+    prod = (NF4_VALUES[codes] * c2_hat).astype(np.float32)
+    return bf16_bits_to_f32(bf16_rne_bits(prod))
+
+
 def dequant_nf4_no_dq(codes, c2, shape) -> np.ndarray:
     """First-level dequant only (Eq. 2 with the absmax constant), float64."""
     codes = np.asarray(codes, dtype=np.uint8).reshape(-1)

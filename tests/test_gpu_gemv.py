@@ -1,6 +1,7 @@
-"""GPU parity of the fused few-token forward (M <= 32 tokens: the weight is
-decoded in registers and never written as bf16) against the float64 oracle,
-and its consistency with the large-M path's dequantized weight."""
+"""GPU parity of the fused few-token forward (M <= 128 tokens: the weight is
+decoded into shared memory for the tensor core and never written to HBM as
+bf16) against the float64 oracle, and its consistency with the large-M
+path's dequantized weight."""
 
 import numpy as np
 import pytest
@@ -23,8 +24,8 @@ def _case(M, N, K, r, seed):
     return W, X, L1, L2
 
 
-@pytest.mark.parametrize("M", [1, 5, 8, 9, 16, 17, 32])
-@pytest.mark.parametrize("N,K,r", [(72, 320, 8), (520, 1088, 64), (1032, 2048, 136)])
+@pytest.mark.parametrize("M", [1, 5, 8, 9, 16, 17, 32, 33, 64, 65, 100, 128])
+@pytest.mark.parametrize("N,K,r", [(72, 320, 8), (520, 1088, 64), (1032, 2048, 136), (264, 64, 16)])
 def test_few_token_forward_parity(M, N, K, r):
     W, X, L1, L2 = _case(M, N, K, r, 500 + M + N + K + r)
     s = 16.0 / r

@@ -150,3 +150,12 @@ def test_dequantize_rows_equals_full_dequantize():
     full = nf4dq.dequantize(nf4dq.quantize_nf4_dq(w))
     rows = [0, 3, 4, 17, 39]
     assert np.array_equal(nf4dq.dequantize_rows(w, rows), full[rows])
+
+
+def test_dequantize_cols_equals_full_dequantize():
+    g = inputs.rng(27)
+    w = inputs.normal_f32(g, (40, 1024), 0.02)
+    w[5, 128:192] = 0.0                          # an all-zero block: code 7 -> 0
+    full = nf4dq.dequantize(nf4dq.quantize_nf4_dq(w))
+    cols = [0, 63, 64, 130, 131, 700, 1023]
+    assert np.array_equal(nf4dq.dequantize_cols(w, cols), full[:, cols])
