@@ -101,9 +101,6 @@ __device__ __forceinline__ void red_add_f32(float *p, float v) {
 // consistent fence of __threadfence()).
 __device__ __forceinline__ void fence_acq_rel_gpu() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
 
-__device__ __forceinline__ void named_bar_sync(int id, int n) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
-}
 
 // The 16 decoded values of one 64-block, bf16(NF4[c] * c2_hat), stored as two
 // byte planes: lo[i] holds the low bytes of entries 4i..4i+3, hi[i] the high

@@ -26,7 +26,7 @@ struct DeviceInfo {
   bool init = false;
   int sms = 0;
   int *err = nullptr;        // device address of g_dev_err
-  bool gemm_attr[4] = {false, false, false, false};   // BN 64, 128, 256; 256 in CTA pairs
+  bool gemm_attr[7] = {false, false, false, false, false, false, false};  // BN 64/128/256, pair, fold 64/128/256
   int pair_clusters = 0;     // co-resident 2-CTA clusters of the pair GEMM
   int gemv_smem_set[3] = {0, 0, 0};   // dynamic smem limit set per NT variant
   int gemv_per_sm[3] = {0, 0, 0};     // resident CTAs per SM per NT variant
@@ -156,29 +156,35 @@ void choose_splits(int64_t tiles, int64_t nkb, int sms, bool allow, int *splits,
   if (*splits < 1) *splits = 1;
 }
 
-size_t gemm_split_ws_bytes(int64_t M, int64_t N, int64_t K, int sms, bool allow) {
+// Split-K partials of a product with N columns (w output columns after a fold).
+size_t gemm_split_ws_bytes(int64_t M, int64_t N, int64_t K, int sms, bool allow, int64_t w = -1) {
   if (M <= 0 || N <= 0 || K <= 0) return 0;
+  if (w < 0) w = N;
   const int bn = pick_bn(N);
   const int64_t tiles = ((M + kBM - 1) / kBM) * ((N + bn - 1) / bn);
   int splits, kbps;
   choose_splits(tiles, (K + kBK - 1) / kBK, sms, allow, &splits, &kbps);
-  return splits > 1 ? align_up((size_t)splits * (size_t)M * (size_t)N * 4) : 0;
+  return splits > 1 ? align_up((size_t)splits * (size_t)M * (size_t)w * 4) : 0;
 }
 
-template <int BN>
+// The hi/lo fold applies when both halves (2w columns) fit one tile and the
+// epilogue's 32-column chunks line up with the halves.
+bool can_fold(int64_t w) { return w == 8 || w == 16 || (w % 32 == 0 && 2 * w <= 256); }
+
+template <int BN, bool FOLD = false>
 int launch_gemm_bn(const CUtensorMap *maps, TcGemmArgs &args, int sms, DeviceInfo *dev, cudaStream_t st, int kind) {
   using Cfg = TcCfg<BN>;
-  const int idx = BN == 64 ? 0 : (BN == 128 ? 1 : 2);
+  auto kernel = tc_gemm_kernel<BN, false, FOLD>;
+  const int idx = (BN == 64 ? 0 : (BN == 128 ? 1 : 2)) + (FOLD ? 4 : 0);
   if (!dev->gemm_attr[idx]) {
-    if (cudaFuncSetAttribute(tc_gemm_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes) !=
-        cudaSuccess)
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes) != cudaSuccess)
       return QLORA_ERR_CUDA;
     dev->gemm_attr[idx] = true;
   }
   const int units = args.m_tiles * args.n_tiles * args.splits;
   const int grid = std::max(1, std::min(units, sms));
   ProfScope prof(kind, st);
-  tc_gemm_kernel<BN><<<grid, kGemmThreads, Cfg::kSmemBytes, st>>>(maps[0], maps[1], maps[2], maps[3], args);
+  kernel<<<grid, kGemmThreads, Cfg::kSmemBytes, st>>>(maps[0], maps[1], maps[2], maps[3], args);
   return launch_status();
 }
 
@@ -228,7 +234,7 @@ bool use_pair(int bn, int splits, int64_t M) { return bn == 256 && splits == 1 &
 // partials go to split_ws and a finalize pass sums them in a fixed order.
 int tc_gemm(cudaStream_t st, DeviceInfo *dev, int64_t M, int64_t N, int nseg, const GemmSeg *segs, float alpha,
             void *out, int64_t ld_row, int64_t ld_col, int out_f32, float *split_ws, int kind, int64_t lo_off = 0,
-            bool split_all = false) {
+            bool split_all = false, int fold = 0) {
   if (M <= 0 || N <= 0) return QLORA_OK;
   if (M > (int64_t)INT32_MAX / 2 || N > (int64_t)INT32_MAX / 2) return QLORA_ERR_UNSUPPORTED_SHAPE;
   const int bn = pick_bn(N);
@@ -246,7 +252,7 @@ int tc_gemm(cudaStream_t st, DeviceInfo *dev, int64_t M, int64_t N, int nseg, co
   int splits, kbps;
   choose_splits((int64_t)a.m_tiles * a.n_tiles, a.seg[0].nkb, dev->sms,
                 split_ws != nullptr && (nseg == 1 || split_all), &splits, &kbps);
-  const bool pair = use_pair(bn, splits, M);
+  const bool pair = use_pair(bn, splits, M) && fold == 0;
   if (pair) a.m_tiles = (int)((M + 2 * kBM - 1) / (2 * kBM));
   for (int s = 0; s < nseg; ++s) {
     a.seg[s].a_mn = segs[s].A.mn_major;
@@ -264,6 +270,7 @@ int tc_gemm(cudaStream_t st, DeviceInfo *dev, int64_t M, int64_t N, int nseg, co
   a.ld_row = ld_row;
   a.ld_col = ld_col;
   a.lo_off = lo_off;
+  a.fold = fold;
   if (splits > 1) {
     a.alpha = 1.f;
     a.out = split_ws;
@@ -276,6 +283,12 @@ int tc_gemm(cudaStream_t st, DeviceInfo *dev, int64_t M, int64_t N, int nseg, co
   int rc;
   if (pair) {
     rc = launch_gemm_pair(maps, a, dev, st, kind);
+  } else if (fold) {
+    switch (bn) {
+      case 64: rc = launch_gemm_bn<64, true>(maps, a, dev->sms, dev, st, kind); break;
+      case 128: rc = launch_gemm_bn<128, true>(maps, a, dev->sms, dev, st, kind); break;
+      default: rc = launch_gemm_bn<256, true>(maps, a, dev->sms, dev, st, kind); break;
+    }
   } else {
     switch (bn) {
       case 64: rc = launch_gemm_bn<64>(maps, a, dev->sms, dev, st, kind); break;
@@ -284,10 +297,11 @@ int tc_gemm(cudaStream_t st, DeviceInfo *dev, int64_t M, int64_t N, int nseg, co
     }
   }
   if (rc || splits == 1) return rc;
-  const int64_t count = M * N;
+  const int64_t W = fold > 0 ? fold : N;
+  const int64_t count = M * W;
   const int grid = (int)std::min<int64_t>((count + 255) / 256, (int64_t)dev->sms * 8);
   ProfScope prof(QLORA_KERNEL_SPLITK_FINALIZE, st);
-  splitk_finalize_kernel<<<grid, 256, 0, st>>>(split_ws, splits, (int)M, (int)N, alpha, out, ld_row, ld_col, lo_off,
+  splitk_finalize_kernel<<<grid, 256, 0, st>>>(split_ws, splits, (int)M, (int)W, alpha, out, ld_row, ld_col, lo_off,
                                                out_f32);
   return launch_status();
 }
@@ -526,8 +540,13 @@ BwdLayout bwd_layout(int64_t M, int64_t N, int64_t K, int r, int sms) {
   size_t sw = 0;
   sw = std::max(sw, gemm_split_ws_bytes(M, r, K, sms, true));   // T = s X L1
   sw = std::max(sw, gemm_split_ws_bytes(M, r, N, sms, true));   // G = s dY L2^T
-  sw = std::max(sw, gemm_split_ws_bytes(N, r, M, sms, true));   // dL2^T = dY^T T
-  sw = std::max(sw, gemm_split_ws_bytes(K, r, M, sms, true));   // dL1 = X^T G
+  if (can_fold(r)) {
+    sw = std::max(sw, gemm_split_ws_bytes(N, 2 * r, M, sms, true, r));   // dL2^T = dY^T [T_hi | T_lo], folded
+    sw = std::max(sw, gemm_split_ws_bytes(K, 2 * r, M, sms, true, r));   // dL1 = X^T [G_hi | G_lo], folded
+  } else {
+    sw = std::max(sw, gemm_split_ws_bytes(N, r, M, sms, true));   // dL2^T = dY^T T_hi + dY^T T_lo
+    sw = std::max(sw, gemm_split_ws_bytes(K, r, M, sms, true));   // dL1 = X^T G_hi + X^T G_lo
+  }
   L.total = L.split + sw;
   return L;
 }
@@ -853,13 +872,22 @@ int qlora_linear_bwd(const uint16_t *dY, const uint16_t *X, const uint16_t *T_sa
     rc = tc_gemm(st, dev, M, K, 2, sX, 1.f, dX, K, 1, 0, nullptr, QLORA_KERNEL_GEMM_DX);
     if (rc) return rc;
   }
-  // dL2 = T^T dY as dL2^T [N x r] = dY^T (T_hi + T_lo): two accumulated
-  // segments over the tokens, written transposed.
+  // dL2 = T^T dY as dL2^T [N x r] = dY^T (T_hi + T_lo), written transposed,
+  // and dL1 = X^T (G_hi + G_lo) [K x r].  When both halves fit one tile the
+  // product runs against the whole [hi | lo] pair (2r columns) and the
+  // epilogue adds the halves, so dY and X stream once; otherwise as two
+  // accumulated segments over the tokens.
+  if (can_fold(r)) {
+    GemmSeg s2 = {{dY, N, M, N, 1}, {T, 2 * r, M, 2 * r, 1}};
+    rc = tc_gemm(st, dev, N, 2 * r, 1, &s2, 1.f, dL2, 1, N, out_f32, split_ws, QLORA_KERNEL_GEMM_DL2, 0, false, r);
+    if (rc) return rc;
+    GemmSeg s1 = {{X, K, M, K, 1}, {G, 2 * r, M, 2 * r, 1}};
+    return tc_gemm(st, dev, K, 2 * r, 1, &s1, 1.f, dL1, r, 1, out_f32, split_ws, QLORA_KERNEL_GEMM_DL1, 0, false, r);
+  }
   const uint16_t *T_lo = T + r;
   GemmSeg s2[2] = {{{dY, N, M, N, 1}, {T, r, M, 2 * r, 1}}, {{dY, N, M, N, 1}, {T_lo, r, M, 2 * r, 1}}};
   rc = tc_gemm(st, dev, N, r, 2, s2, 1.f, dL2, 1, N, out_f32, split_ws, QLORA_KERNEL_GEMM_DL2, 0, true);
   if (rc) return rc;
-  // dL1 = X^T (G_hi + G_lo) [K x r].
   const uint16_t *G_lo = G + r;
   GemmSeg s1[2] = {{{X, K, M, K, 1}, {G, r, M, 2 * r, 1}}, {{X, K, M, K, 1}, {G_lo, r, M, 2 * r, 1}}};
   return tc_gemm(st, dev, K, r, 2, s1, 1.f, dL1, r, 1, out_f32, split_ws, QLORA_KERNEL_GEMM_DL1, 0, true);

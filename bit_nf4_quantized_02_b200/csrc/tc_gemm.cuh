@@ -15,7 +15,9 @@
 // stored layout), X^T*G and the LoRA extra K-steps all run on this engine.
 // A split of the reduction (split-K; of segment 0, or of every segment when
 // they have equal lengths) writes fp32 partials that a finalize kernel sums
-// in a fixed order.  In the CTA-pair form (cta_group::2, a cluster of two
+// in a fixed order.  The fold form adds accumulator columns j and j + fold,
+// so a product against a [hi | lo] pair of bf16 halves (2 fold columns, one N
+// tile) streams its other operand once.  In the CTA-pair form (cta_group::2, a cluster of two
 // CTAs) the pair computes 256-row tiles: each CTA stages its 128 rows of A
 // and half of B's rows, the leader CTA issues 256-row MMAs that read both
 // CTAs' shared memory, and each CTA's epilogue drains its own 128 rows of
@@ -50,8 +52,37 @@ struct TcGemmArgs {
   int64_t ld_row, ld_col;   // element strides of D(i, j) in `out` (unsplit output)
   int64_t lo_off;           // bf16 output only: if > 0 also store lo = bf16(v - hi) at +lo_off
   int out_f32;              // 1: fp32 output, 0: bf16
+  int fold;                 // fold form: output column j < fold is D(i, j) + D(i, j + fold)
   int *err;
 };
+
+// Fold-form store of 32 consecutive output columns col0.. of row `row` (the
+// values before alpha; split partials go to the dense [split][M][fold] buffer).
+__device__ __forceinline__ void tc_store_fold(const TcGemmArgs &p, int row, int col0, int split, const float (&v)[32]) {
+  const int W = p.fold;
+  if (p.splits > 1) {
+    float *o = reinterpret_cast<float *>(p.out) + ((int64_t)split * p.M + row) * W + col0;
+#pragma unroll
+    for (int j = 0; j < 32; ++j)
+      if (col0 + j < W) o[j] = v[j];
+    return;
+  }
+  const float alpha = p.alpha;
+#pragma unroll
+  for (int j = 0; j < 32; ++j)
+    if (col0 + j < W) {
+      const float x = alpha * v[j];
+      const int64_t off = (int64_t)row * p.ld_row + (int64_t)(col0 + j) * p.ld_col;
+      if (p.out_f32) {
+        reinterpret_cast<float *>(p.out)[off] = x;
+      } else {
+        __nv_bfloat16 *o = reinterpret_cast<__nv_bfloat16 *>(p.out);
+        const __nv_bfloat16 hb = __float2bfloat16_rn(x);
+        o[off] = hb;
+        if (p.lo_off > 0) o[off + p.lo_off] = __float2bfloat16_rn(x - __bfloat162float(hb));
+      }
+    }
+}
 
 // BN: output columns per tile.  PAIR: tile of 2*kBM rows computed by a CTA
 // pair, each CTA holding kBM rows of A and BN/2 rows of B.
@@ -94,7 +125,7 @@ __device__ __forceinline__ void tc_seg_range(const TcGemmArgs &p, int s, int spl
   }
 }
 
-template <int BN, bool PAIR = false>
+template <int BN, bool PAIR = false, bool FOLD = false>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tA0, const __grid_constant__ CUtensorMap tB0,
                    const __grid_constant__ CUtensorMap tA1, const __grid_constant__ CUtensorMap tB1,
@@ -311,6 +342,31 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const int row = mt * Cfg::kTileM + (int)rank * kBM + q * 32 + lane;
       const bool row_ok = row < p.M;
       const float alpha = p.alpha;
+      if constexpr (FOLD) {
+        // one N tile of 2*fold columns: output column j = column j + column j + fold
+        const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
+#pragma unroll 1
+        for (int c = 0; c < (p.fold < 32 ? 32 : p.fold); c += 32) {
+          uint32_t r[32];
+          float v[32];
+          tmem_ld_32x32b_x32(tb + (uint32_t)c, r);
+          tmem_wait_ld();
+          if (p.fold >= 32) {
+            uint32_t r2[32];
+            tmem_ld_32x32b_x32(tb + (uint32_t)(c + p.fold), r2);
+            tmem_wait_ld();
+#pragma unroll
+            for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]) + __uint_as_float(r2[j]);
+          } else if (p.fold == 16) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) v[j] = j < 16 ? __uint_as_float(r[j]) + __uint_as_float(r[j + 16]) : 0.f;
+          } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) v[j] = j < 8 ? __uint_as_float(r[j]) + __uint_as_float(r[j + 8]) : 0.f;
+          }
+          if (row_ok) tc_store_fold(p, row, c, split, v);
+        }
+      } else
 #pragma unroll 1
       for (int c = 0; c < BN; c += 32) {
         uint32_t r[32];
