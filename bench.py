@@ -168,32 +168,61 @@ def build_layer(dev, rank, wl=WL):
 
 
 def make_step(qlora, lins, grads, world, wl=WL):
-    def step():
+    """One step; `ready(t)` (if given) is called before the step first reads input t."""
+    def step(ready=None):
         for l in lins:
             l.q = qlora.quantize_nf4_dq(l.W, out=l.q)
         for l in lins:
+            if ready:
+                ready(l.X)
             qlora.linear_fwd(l.X, l.q, l.L1, l.L2, wl.s, Y=l.Y, T=l.T)
         for l in reversed(lins):
+            if ready:
+                ready(l.dY)
             qlora.linear_bwd(l.dY, l.X, l.T, l.q, l.L1, l.L2, wl.s, grad_dtype=torch.float32,
                              dX=l.dX, dL1=l.dL1, dL2=l.dL2)
         grads.allreduce()
     return step
 
 
-def run_e2e(args, step, flat, acts, dev, world, e0, e1):
+def run_e2e(args, step, flat, acts, dev, world, e0, e1, overlap=False):
     """Same step with host buffers: the step's activations and output gradients
-    (`acts`) copied in from pinned host memory, adapter gradients copied out."""
+    (`acts`, in the order the step first reads them) copied in from pinned host
+    memory, adapter gradients copied out.  With `overlap`, the copies run on a
+    copy stream and the step waits for each input just before it first reads
+    it, so the transfers overlap quantization and the earlier linears."""
     pinned_in = [torch.empty(a.shape, dtype=a.dtype, pin_memory=True) for a in acts]
     for h, a in zip(pinned_in, acts):
         h.copy_(a)
     grads_host = torch.empty(flat.shape, dtype=flat.dtype, pin_memory=True)
     h2d = sum(t.numel() * t.element_size() for t in pinned_in)
     d2h = grads_host.numel() * grads_host.element_size()
+    copy_stream = torch.cuda.Stream(dev)
+    main = torch.cuda.current_stream(dev)
 
     def e2e_step():
-        for h, a in zip(pinned_in, acts):
-            a.copy_(h, non_blocking=True)
-        step()
+        if not overlap:
+            for h, a in zip(pinned_in, acts):
+                a.copy_(h, non_blocking=True)
+            step()
+        else:
+            # the copies may start once the previous step no longer reads the buffers
+            copy_stream.wait_stream(main)
+            done = {}
+            with torch.cuda.stream(copy_stream):
+                for h, a in zip(pinned_in, acts):
+                    a.copy_(h, non_blocking=True)
+                    ev = torch.cuda.Event()
+                    ev.record(copy_stream)
+                    done[a.data_ptr()] = ev
+
+            def ready(t):
+                ev = done.pop(t.data_ptr(), None)
+                if ev is not None:
+                    main.wait_event(ev)
+            step(ready)
+            for ev in done.values():       # inputs the step never read still complete within it
+                main.wait_event(ev)
         grads_host.copy_(flat, non_blocking=True)
 
     e2e_step()
@@ -237,6 +266,8 @@ def run_ours(args, rank, world, local_rank):
         sel = wl.linears * wl.layers
     else:
         lins, grads, acts = build_layer(dev, rank, wl)
+        # copy order for the end-to-end run: the step's first read of each input
+        acts = acts[:3] + acts[3:][::-1]
         flat = grads.flat
         if args.linear:
             lins = [l for l in lins if l.lin.name == args.linear]
@@ -280,7 +311,7 @@ def run_ours(args, rank, world, local_rank):
     if args.no_e2e:
         ms_e2e, h2d, d2h = None, None, None
     else:
-        ms_e2e, h2d, d2h = run_e2e(args, step, flat, acts, dev, world, e0, e1)
+        ms_e2e, h2d, d2h = run_e2e(args, step, flat, acts, dev, world, e0, e1, overlap=wl.layers == 1)
 
     if rank != 0:
         return None
@@ -333,7 +364,10 @@ def run_ours(args, rank, world, local_rank):
                            + (", all-reduce of adapter grads" if world > 1 else ""),
                    "l2": "inputs larger than L2 (>1 GB touched per step), no flush"},
         "e2e": ({"value": flops / (ms_e2e * 1e-3) / 1e12, "unit": UNIT, "h2d_bytes_per_step": h2d,
-                 "d2h_bytes_per_step": d2h} if ms_e2e else None),
+                 "d2h_bytes_per_step": d2h,
+                 "copies": ("host->device copies on a copy stream in the order the step first reads them, "
+                            "overlapping quantization and compute" if wl.layers == 1 else
+                            "host->device copies before the step")} if ms_e2e else None),
         "gpu_launches": len(launches),
         "roofline": {"bound": "tensor", "kernel": "tc_gemm (Y = X W^T + T L2 and dX = dY W + G L1^T)",
                      "traffic_unit": "bytes per launch (DRAM read + write)",
@@ -399,7 +433,7 @@ def run_decode(args, rank, world, local_rank):
     """LLaMA-65B layer forward at 16 tokens: the memory-bound few-token path."""
     import bit_nf4_quantized_02_b200 as qlora
     wl = workloads.LLAMA65B_LAYER
-    M, r, s = wl.extra["M_decode"], wl.r, wl.s
+    M, r, s = args.tokens or wl.extra["M_decode"], wl.r, wl.s
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     base = wl.seed + 1000 * rank
@@ -450,20 +484,21 @@ def run_decode(args, rank, world, local_rank):
         return None
     peaks, peak_src = load_peaks()
     per_kind, kernels = _kernel_table(launches, args.steps)
-    dom = per_kind.get("fused_fwd", per_kind.get("gemv_fwd", [0, 0.0]))
+    dom = per_kind.get("fused_fwd") or per_kind.get("gemv_fwd") or [0, 0.0]
     achieved = nbytes * args.steps / (dom[1] * 1e-3) / 1e9 if dom[1] > 0 else None
     peak = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
     return {
         "metric": "QLoRA NF4 linear forward, NF4-weight-bound GB/s", "value": nbytes * world / (ms * 1e-3) / 1e9,
         "unit": "GB/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": "llama65b-layer-7-linears-forward-M16-r64", "tokens": M, "lora_r": r,
+        "config": {"workload": f"llama65b-layer-7-linears-forward-M{M}-r64", "tokens": M, "lora_r": r,
                    "bytes_per_step": nbytes, "l2": "weights (418 MB) larger than L2, no flush",
                    "step": "forward of the 7 QLoRA linears (weights resident, quantized once)"},
         "graph": {"ms_per_step": ms_graph, "value": nbytes * world / (ms_graph * 1e-3) / 1e9, "unit": "GB/s",
                   "frac_of_hbm": nbytes / (ms_graph * 1e-3) / 1e9 / peak},
         "gpu_launches": len(launches),
-        "roofline": {"bound": "hbm", "kernel": "few-token forward chain (lora_down_small + gemv_fwd + epilogue)",
+        "roofline": {"bound": "hbm", "kernel": ("few-token forward chain (lora_down_small + " +
+                                                ("gemv_fwd" if M <= 32 else "nf4_fused_fwd (tcgen05)") + " + epilogue)"),
                      "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak if achieved else None, "traffic": None,
                      "peak_source": f"{peak_src} hbm_gbs", "launches_timed": dom[0],
@@ -610,6 +645,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end (host buffers) measurement")
+    ap.add_argument("--tokens", type=int, default=None,
+                    help="llama65b-decode: tokens per step (default 16; 33..128 run the tcgen05 fused forward)")
     ap.add_argument("--linear", choices=[l.name for l in WL.linears], default=None,
                     help="restrict the step to one linear of the layer (profiling runs)")
     ap.add_argument("--workload", choices=list(TRAIN) + ["llama65b-decode", "quantizer"], default="llama7b-train",
