@@ -44,6 +44,10 @@ int current_device_info(DeviceInfo **out) {
     if (!d.init) {
       if (cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return QLORA_ERR_CUDA;
       if (cudaGetSymbolAddress(reinterpret_cast<void **>(&d.err), g_dev_err) != cudaSuccess) return QLORA_ERR_CUDA;
+      // One-time fill of the quantizer's code table (a constant of the NF4
+      // levels), completed before any library launch on this device.
+      code_lut_init_kernel<<<kCodeBins / 256, 256>>>();
+      if (cudaGetLastError() != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess) return QLORA_ERR_CUDA;
       d.init = true;
     }
   }

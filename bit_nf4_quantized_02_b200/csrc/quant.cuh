@@ -71,6 +71,53 @@ struct NF4Thresholds {
   }
 };
 
+// Exact nearest-level codes without a division for almost every weight.
+// [-1, 1] is cut into kCodeBins bins of width 2^-13; bin(x) = floor((x + 1) *
+// kCodeBins / 2).  A bin with no decision threshold within two bins of it has
+// one code for every x in those five bins, so any estimate of
+// x = fp32(w / absmax) that is within one bin of x and lands in it (the
+// estimate w * (1/absmax) is within a few ulps, far below a bin) gives the
+// exact code.  The bins near a threshold (5 per threshold, 0.46% of them) are
+// marked, and their weights take the exact division.
+constexpr int kCodeBins = 16384;
+constexpr uint8_t kCodeBoundary = 0xFF;
+
+// The table, filled once per device from the same thresholds the exact path
+// uses (code_lut_init_kernel), and copied into shared memory by each CTA.
+__device__ __align__(16) uint8_t g_code_lut[kCodeBins];
+
+__global__ void __launch_bounds__(256) code_lut_init_kernel() {
+  const int b = blockIdx.x * blockDim.x + threadIdx.x;
+  if (b >= kCodeBins) return;
+  NF4Thresholds th;
+  th.init();
+  uint32_t code = 0;
+  bool edge = false;
+#pragma unroll
+  for (int j = 0; j < 15; ++j) {
+    const int tb = (int)floor(((double)th.t[j] + 1.0) * (kCodeBins / 2));
+    code += tb < b ? 1u : 0u;
+    edge |= tb >= b - 2 && tb <= b + 2;
+  }
+  g_code_lut[b] = edge ? kCodeBoundary : (uint8_t)code;
+}
+
+// Copy the table into shared memory (all threads of the CTA).
+__device__ __forceinline__ void load_code_lut(uint8_t *lut) {
+  for (int i = threadIdx.x; i < kCodeBins / 16; i += blockDim.x)
+    reinterpret_cast<uint4 *>(lut)[i] = reinterpret_cast<const uint4 *>(g_code_lut)[i];
+}
+
+// Code of v / amax given rinv = 1 / amax (amax > 0): table lookup, exact
+// division only in boundary bins.
+__device__ __forceinline__ uint32_t fast_code(float v, float amax, float rinv, const uint8_t *lut,
+                                              const NF4Thresholds &th) {
+  int b = __float2int_rd(__fmaf_rn(v * rinv, (float)(kCodeBins / 2), (float)(kCodeBins / 2)));
+  b = min(max(b, 0), kCodeBins - 1);
+  const uint32_t c = lut[b];
+  return c != kCodeBoundary ? c : th.encode(__fdiv_rn(v, amax));
+}
+
 __device__ __forceinline__ void load8(const float *__restrict__ p, float (&v)[8]) {
   const float4 a = __ldg(reinterpret_cast<const float4 *>(p));
   const float4 b = __ldg(reinterpret_cast<const float4 *>(p) + 1);
@@ -117,8 +164,11 @@ __global__ void __launch_bounds__(kQuantThreads) nf4_quantize_kernel(const TW *_
                                                                     float *__restrict__ c2,
                                                                     double *__restrict__ partial) {
   __shared__ double red[kQuantThreads / 32];
+  __shared__ __align__(16) uint8_t lut[kCodeBins];
   NF4Thresholds th;
   th.init();
+  load_code_lut(lut);
+  __syncthreads();
   const int lane = lane_id();
   const int64_t ngroups = numel >> 8;
   const int64_t nwarps = (int64_t)gridDim.x * (kQuantThreads / 32);
@@ -138,8 +188,9 @@ __global__ void __launch_bounds__(kQuantThreads) nf4_quantize_kernel(const TW *_
     if (amax == 0.f) {
       packed = 0x77777777u;  // all-zero block: every element is the exact-zero level
     } else {
+      const float rinv = __frcp_rn(amax);
 #pragma unroll
-      for (int i = 0; i < 8; ++i) packed |= th.encode(__fdiv_rn(v[i], amax)) << (4 * i);
+      for (int i = 0; i < 8; ++i) packed |= fast_code(v[i], amax, rinv, lut, th) << (4 * i);
     }
     reinterpret_cast<uint32_t *>(codes)[(g << 5) + lane] = packed;
     if ((lane & 7) == 0) {

@@ -21,7 +21,10 @@
  *     at least the size the matching *_workspace_size() function returns.
  *   - Streams: `stream` is a cudaStream_t (NULL = legacy default stream).
  *     Every call only enqueues work on that stream and never synchronizes it;
- *     outputs are valid once the stream has reached that point.
+ *     outputs are valid once the stream has reached that point.  The one
+ *     exception is the first call on a device: it fills a constant table of
+ *     the quantizer (a function of the NF4 levels only) and waits for the
+ *     device once.
  *   - bfloat16 data is passed as uint16_t bit patterns.
  *   - Alignment: every device pointer must be 16-byte aligned (W->c2_mean and
  *     c2_mean only need 4 bytes).
