@@ -329,7 +329,13 @@ def run_ours(args, rank, world, local_rank):
     dom_flops = args.steps * sum(linear_flops(wl.M, l.n_out, l.k_in, wl.r)["gemm_Y"] +
                                  linear_flops(wl.M, l.n_out, l.k_in, wl.r)["gemm_dX"] for l in sel)
     achieved = dom_flops / (dom_ms * 1e-3) / 1e12 if dom_ms > 0 else None
-    peak = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+    # The burst GEMM peak while the SM clock held its maximum through the timed
+    # region; the sustained (power-capped) one once the clock dropped.
+    at_max = bool(clocks and clocks.get("sm_mhz") and clocks.get("sm_max_mhz")
+                  and clocks["sm_mhz"] >= 0.97 * clocks["sm_max_mhz"]
+                  and "sw_power_cap" not in (clocks.get("reasons") or []))
+    peak_key = "bf16_tflops" if at_max else "bf16_tflops_sustained"
+    peak = peaks.get(peak_key, FALLBACK_PEAKS[peak_key])
     # DRAM traffic per launch: the ncu-measured ratio of DRAM bytes to algorithmic
     # bytes for these launches (captured at the q shape), applied to the average
     # algorithmic bytes of the timed launches; null once the kernel source changed.
@@ -373,7 +379,7 @@ def run_ours(args, rank, world, local_rank):
                      "traffic_unit": "bytes per launch (DRAM read + write)",
                      "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                      "frac": achieved / peak if achieved else None, "traffic": traffic,
-                     "peak_source": f"{peak_src} bf16_tflops_sustained",
+                     "peak_source": f"{peak_src} {peak_key}",
                      "launches_timed": dom_n, "avg_launch_ms": dom_ms / dom_n if dom_n else None},
         "kernels": kernels,
         "clocks": clocks,

@@ -26,8 +26,8 @@ struct DeviceInfo {
   bool init = false;
   int sms = 0;
   int *err = nullptr;        // device address of g_dev_err
-  bool gemm_attr[7] = {false, false, false, false, false, false, false};  // BN 64/128/256, pair, fold 64/128/256
-  int pair_clusters = 0;     // co-resident 2-CTA clusters of the pair GEMM
+  bool gemm_attr[16] = {};   // [wide][fold][BN 64/128/256 or 3 = pair]: shared-memory limit set
+  int pair_clusters[2] = {0, 0};   // co-resident 2-CTA clusters of the pair GEMM [wide]
   int gemv_smem_set[3] = {0, 0, 0};   // dynamic smem limit set per NT variant
   int gemv_per_sm[3] = {0, 0, 0};     // resident CTAs per SM per NT variant
   int fused_smem_set[4] = {0, 0, 0, 0};   // dynamic smem limit set per token-padding variant
@@ -141,6 +141,40 @@ int make_tmap(CUtensorMap *m, const Operand &o, int box_rows) {
   return r == CUDA_SUCCESS ? QLORA_OK : QLORA_ERR_CUDA;
 }
 
+// The same operand as 3-D boxes of two k-blocks, for the GEMM's wide stages.
+// K-major: dims {64, rows, kext/64} with the k-block stride 128 B, so a box
+// {64, box_rows, 2} lands as [k-block][row][64].  MN-major: dims {64, kext,
+// rows/64} with the chunk stride 128 B, a box {64, 128, box_rows/64} lands
+// as [chunk][k][64].  Only whole 64-wide blocks may be described this way (a
+// partial one would read into the next row), hence wide_ok().
+bool wide_ok(const Operand &o) { return o.mn_major ? o.rows % 64 == 0 : o.kext % 64 == 0; }
+
+int make_tmap3(CUtensorMap *m, const Operand &o, int box_rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return QLORA_ERR_CUDA;
+  cuuint64_t dims[3], strides[2];
+  cuuint32_t box[3], estr[3] = {1, 1, 1};
+  dims[0] = 64;
+  box[0] = 64;
+  if (!o.mn_major) {
+    dims[1] = (cuuint64_t)o.rows;
+    dims[2] = (cuuint64_t)(o.kext / 64);
+    box[1] = (cuuint32_t)box_rows;
+    box[2] = 2;
+  } else {
+    dims[1] = (cuuint64_t)o.kext;
+    dims[2] = (cuuint64_t)(o.rows / 64);
+    box[1] = 128;
+    box[2] = (cuuint32_t)(box_rows / 64);
+  }
+  strides[0] = (cuuint64_t)o.ld * 2;
+  strides[1] = 128;
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(o.ptr), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? QLORA_OK : QLORA_ERR_CUDA;
+}
+
 struct GemmSeg {
   Operand A, B;   // A.kext == B.kext
 };
@@ -175,11 +209,11 @@ size_t gemm_split_ws_bytes(int64_t M, int64_t N, int64_t K, int sms, bool allow,
 // epilogue's 32-column chunks line up with the halves.
 bool can_fold(int64_t w) { return w == 8 || w == 16 || (w % 32 == 0 && 2 * w <= 256); }
 
-template <int BN, bool FOLD = false>
+template <int BN, bool FOLD, bool WIDE>
 int launch_gemm_bn(const CUtensorMap *maps, TcGemmArgs &args, int sms, DeviceInfo *dev, cudaStream_t st, int kind) {
-  using Cfg = TcCfg<BN>;
-  auto kernel = tc_gemm_kernel<BN, false, FOLD>;
-  const int idx = (BN == 64 ? 0 : (BN == 128 ? 1 : 2)) + (FOLD ? 4 : 0);
+  using Cfg = TcCfg<BN, false, WIDE>;
+  auto kernel = tc_gemm_kernel<BN, false, FOLD, WIDE>;
+  const int idx = (BN == 64 ? 0 : (BN == 128 ? 1 : 2)) + (FOLD ? 4 : 0) + (WIDE ? 8 : 0);
   if (!dev->gemm_attr[idx]) {
     if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes) != cudaSuccess)
       return QLORA_ERR_CUDA;
@@ -194,10 +228,11 @@ int launch_gemm_bn(const CUtensorMap *maps, TcGemmArgs &args, int sms, DeviceInf
 
 // CTA-pair GEMM (256 x 256 tiles): a persistent grid of 2-CTA clusters, as
 // many as can be resident at once.
+template <bool WIDE>
 int launch_gemm_pair(const CUtensorMap *maps, TcGemmArgs &args, DeviceInfo *dev, cudaStream_t st, int kind) {
   constexpr int BN = 256;
-  using Cfg = TcCfg<BN, true>;
-  auto kernel = tc_gemm_kernel<BN, true>;
+  using Cfg = TcCfg<BN, true, WIDE>;
+  auto kernel = tc_gemm_kernel<BN, true, false, WIDE>;
   cudaLaunchConfig_t cfg;
   std::memset(&cfg, 0, sizeof(cfg));
   cudaLaunchAttribute attr[1];
@@ -210,17 +245,18 @@ int launch_gemm_pair(const CUtensorMap *maps, TcGemmArgs &args, DeviceInfo *dev,
   cfg.stream = st;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (!dev->gemm_attr[3]) {
+  const int idx = 3 + (WIDE ? 8 : 0);
+  if (!dev->gemm_attr[idx]) {
     if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes) != cudaSuccess)
       return QLORA_ERR_CUDA;
     cfg.gridDim = dim3(2 * (unsigned)dev->sms, 1, 1);
     int clusters = 0;
     if (cudaOccupancyMaxActiveClusters(&clusters, kernel, &cfg) != cudaSuccess || clusters < 1) return QLORA_ERR_CUDA;
-    dev->pair_clusters = clusters;
-    dev->gemm_attr[3] = true;
+    dev->pair_clusters[WIDE ? 1 : 0] = clusters;
+    dev->gemm_attr[idx] = true;
   }
   const int units = args.m_tiles * args.n_tiles * args.splits;
-  const int clusters = std::max(1, std::min(units, dev->pair_clusters));
+  const int clusters = std::max(1, std::min(units, dev->pair_clusters[WIDE ? 1 : 0]));
   cfg.gridDim = dim3(2 * (unsigned)clusters, 1, 1);
   ProfScope prof(kind, st);
   if (cudaLaunchKernelEx(&cfg, kernel, maps[0], maps[1], maps[2], maps[3], args) != cudaSuccess) return QLORA_ERR_CUDA;
@@ -258,12 +294,21 @@ int tc_gemm(cudaStream_t st, DeviceInfo *dev, int64_t M, int64_t N, int nseg, co
                 split_ws != nullptr && (nseg == 1 || split_all), &splits, &kbps);
   const bool pair = use_pair(bn, splits, M) && fold == 0;
   if (pair) a.m_tiles = (int)((M + 2 * kBM - 1) / (2 * kBM));
+  // Wide stages (two k-blocks per 3-D box) wherever segment 0 allows them;
+  // the single-CTA 256-column form keeps one k-block per stage.
+  bool seg_wide[2] = {false, false};
+  for (int s = 0; s < nseg; ++s)
+    seg_wide[s] = a.seg[s].nkb >= 2 && wide_ok(segs[s].A) && wide_ok(segs[s].B);
+  const bool wide = seg_wide[0] && (pair || bn <= 128);
+  const int brows = pair ? bn / 2 : bn;
   for (int s = 0; s < nseg; ++s) {
     a.seg[s].a_mn = segs[s].A.mn_major;
     a.seg[s].b_mn = segs[s].B.mn_major;
-    int rc = make_tmap(&maps[2 * s], segs[s].A, kBM);
+    a.seg[s].wide = wide && seg_wide[s];
+    int rc = a.seg[s].wide ? make_tmap3(&maps[2 * s], segs[s].A, kBM) : make_tmap(&maps[2 * s], segs[s].A, kBM);
     if (rc) return rc;
-    rc = make_tmap(&maps[2 * s + 1], segs[s].B, pair ? bn / 2 : bn);
+    rc = a.seg[s].wide ? make_tmap3(&maps[2 * s + 1], segs[s].B, brows)
+                       : make_tmap(&maps[2 * s + 1], segs[s].B, brows);
     if (rc) return rc;
   }
   if (nseg == 1) maps[2] = maps[0], maps[3] = maps[1];
@@ -286,18 +331,22 @@ int tc_gemm(cudaStream_t st, DeviceInfo *dev, int64_t M, int64_t N, int nseg, co
   }
   int rc;
   if (pair) {
-    rc = launch_gemm_pair(maps, a, dev, st, kind);
+    rc = wide ? launch_gemm_pair<true>(maps, a, dev, st, kind) : launch_gemm_pair<false>(maps, a, dev, st, kind);
   } else if (fold) {
     switch (bn) {
-      case 64: rc = launch_gemm_bn<64, true>(maps, a, dev->sms, dev, st, kind); break;
-      case 128: rc = launch_gemm_bn<128, true>(maps, a, dev->sms, dev, st, kind); break;
-      default: rc = launch_gemm_bn<256, true>(maps, a, dev->sms, dev, st, kind); break;
+      case 64: rc = wide ? launch_gemm_bn<64, true, true>(maps, a, dev->sms, dev, st, kind)
+                         : launch_gemm_bn<64, true, false>(maps, a, dev->sms, dev, st, kind); break;
+      case 128: rc = wide ? launch_gemm_bn<128, true, true>(maps, a, dev->sms, dev, st, kind)
+                          : launch_gemm_bn<128, true, false>(maps, a, dev->sms, dev, st, kind); break;
+      default: rc = launch_gemm_bn<256, true, false>(maps, a, dev->sms, dev, st, kind); break;
     }
   } else {
     switch (bn) {
-      case 64: rc = launch_gemm_bn<64>(maps, a, dev->sms, dev, st, kind); break;
-      case 128: rc = launch_gemm_bn<128>(maps, a, dev->sms, dev, st, kind); break;
-      default: rc = launch_gemm_bn<256>(maps, a, dev->sms, dev, st, kind); break;
+      case 64: rc = wide ? launch_gemm_bn<64, false, true>(maps, a, dev->sms, dev, st, kind)
+                         : launch_gemm_bn<64, false, false>(maps, a, dev->sms, dev, st, kind); break;
+      case 128: rc = wide ? launch_gemm_bn<128, false, true>(maps, a, dev->sms, dev, st, kind)
+                          : launch_gemm_bn<128, false, false>(maps, a, dev->sms, dev, st, kind); break;
+      default: rc = launch_gemm_bn<256, false, false>(maps, a, dev->sms, dev, st, kind); break;
     }
   }
   if (rc || splits == 1) return rc;

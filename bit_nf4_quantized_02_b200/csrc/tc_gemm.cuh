@@ -39,6 +39,7 @@ struct TcSeg {
   int nkb;   // 64-wide k-blocks in this segment
   int a_mn;  // A is MN-major (contiguous along M)
   int b_mn;  // B is MN-major (contiguous along N)
+  int wide;  // both tensor maps are 3-D boxes of two k-blocks (WIDE kernels only)
 };
 
 struct TcGemmArgs {
@@ -85,15 +86,22 @@ __device__ __forceinline__ void tc_store_fold(const TcGemmArgs &p, int row, int 
 }
 
 // BN: output columns per tile.  PAIR: tile of 2*kBM rows computed by a CTA
-// pair, each CTA holding kBM rows of A and BN/2 rows of B.
-template <int BN, bool PAIR = false>
+// pair, each CTA holding kBM rows of A and BN/2 rows of B.  WIDE: a stage
+// holds two k-blocks, each operand loaded by one 3-D box spanning both (a
+// segment that cannot use 3-D boxes fills only the first k-block of a stage).
+template <int BN, bool PAIR = false, bool WIDE = false>
 struct TcCfg {
   static constexpr int kTileM = PAIR ? 2 * kBM : kBM;
   static constexpr int kBRows = PAIR ? BN / 2 : BN;   // B rows staged by one CTA
-  static constexpr int kABytes = kBM * kBK * 2;
-  static constexpr int kBBytes = kBRows * kBK * 2;
-  static constexpr int kStageBytes = kABytes + kBBytes;
-  static constexpr int kStages = PAIR ? 7 : (BN == 256 ? 4 : (BN == 128 ? 6 : 8));
+  static constexpr int kABytes = kBM * kBK * 2;       // one k-block of A
+  static constexpr int kBBytes = kBRows * kBK * 2;    // one k-block of B
+  static constexpr int kKB = WIDE ? 2 : 1;            // k-blocks per stage
+  static constexpr int kAStage = kKB * kABytes;
+  static constexpr int kStageBytes = kKB * (kABytes + kBBytes);
+  // MN-major operands are stored as 64-element-wide chunks of kKB*64 k-rows.
+  static constexpr int kMnChunk = kKB * 64 * 128;
+  static constexpr int kStages = WIDE ? (PAIR || BN == 128 ? 3 : (BN == 64 ? 4 : 2))
+                                      : (PAIR ? 7 : (BN == 256 ? 4 : (BN == 128 ? 6 : 8)));
   static constexpr int kTmemCols = 2 * BN;
   static constexpr int kBarBytes = 256;
   static constexpr int kSmemBytes = kStages * kStageBytes + kBarBytes + 1024;
@@ -125,12 +133,12 @@ __device__ __forceinline__ void tc_seg_range(const TcGemmArgs &p, int s, int spl
   }
 }
 
-template <int BN, bool PAIR = false, bool FOLD = false>
+template <int BN, bool PAIR = false, bool FOLD = false, bool WIDE = false>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tA0, const __grid_constant__ CUtensorMap tB0,
                    const __grid_constant__ CUtensorMap tA1, const __grid_constant__ CUtensorMap tB1,
                    const TcGemmArgs p) {
-  using Cfg = TcCfg<BN, PAIR>;
+  using Cfg = TcCfg<BN, PAIR, WIDE>;
   constexpr int S = Cfg::kStages;
   // Pair form: the grid is a 1-D array of 2-CTA clusters; CTA rank 0 leads.
   const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
@@ -206,6 +214,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       auto load = [&](uint32_t dst, const CUtensorMap *m, uint32_t bar, int x, int y) {
         if (PAIR) tma_load_2d_pair(dst, m, bar, x, y); else tma_load_2d(dst, m, bar, x, y);
       };
+      auto load3 = [&](uint32_t dst, const CUtensorMap *m, uint32_t bar, int y, int z) {
+        if (PAIR) tma_load_3d_pair(dst, m, bar, 0, y, z); else tma_load_3d(dst, m, bar, 0, y, z);
+      };
       const int a_row0 = (int)rank * kBM;           // this CTA's rows within the tile
       const int b_row0 = (int)rank * Cfg::kBRows;
       for (int u = first_unit; u < units && ok; u += unit_stride) {
@@ -218,27 +229,41 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           const CUtensorMap *tb = s == 0 ? &tB0 : &tB1;
           int kb0, kb1;
           tc_seg_range(p, s, split, kb0, kb1);
-          for (int kb = kb0; kb < kb1; ++kb) {
+          const bool wide = WIDE && p.seg[s].wide;
+          const int step = wide ? 2 : 1;
+          for (int kb = kb0; kb < kb1; kb += step) {
             if (!mbar_wait(smem_u32(empty_bar + stage), phase ^ 1, p.err, DEV_TIMEOUT_PRODUCER)) {
               ok = false;
               break;
             }
             const uint32_t fb_local = smem_u32(full_bar + stage);
             const uint32_t fb = PAIR ? mapa_shared(fb_local, 0) : fb_local;
-            if (leader) mbar_arrive_expect_tx(fb_local, (PAIR ? 2 : 1) * Cfg::kStageBytes);
+            // a box is counted in full, also where it reaches past the
+            // segment (those k-blocks are zero-filled or simply not used)
+            const uint32_t bytes = wide ? Cfg::kStageBytes : Cfg::kABytes + Cfg::kBBytes;
+            if (leader) mbar_arrive_expect_tx(fb_local, (PAIR ? 2 : 1) * bytes);
             const uint32_t sa = smem_u32(smem + stage * Cfg::kStageBytes);
-            const uint32_t sb = sa + Cfg::kABytes;
-            if (!p.seg[s].a_mn) {
-              load(sa, ta, fb, kb * kBK, am);
+            const uint32_t sb = sa + Cfg::kAStage;
+            if (wide) {
+              // K-major maps are {64 k, rows, k-blocks}: smem [k-block][row][64].
+              // MN-major maps are {64 mn, k, 64-wide mn chunks}: smem [chunk][k][64].
+              if (!p.seg[s].a_mn) load3(sa, ta, fb, am, kb);
+              else load3(sa, ta, fb, kb * kBK, am >> 6);
+              if (!p.seg[s].b_mn) load3(sb, tb, fb, bn0, kb);
+              else load3(sb, tb, fb, kb * kBK, bn0 >> 6);
             } else {
-              load(sa, ta, fb, am, kb * kBK);
-              load(sa + 8192, ta, fb, am + 64, kb * kBK);
-            }
-            if (!p.seg[s].b_mn) {
-              load(sb, tb, fb, kb * kBK, bn0);
-            } else {
+              if (!p.seg[s].a_mn) {
+                load(sa, ta, fb, kb * kBK, am);
+              } else {
+                load(sa, ta, fb, am, kb * kBK);
+                load(sa + Cfg::kMnChunk, ta, fb, am + 64, kb * kBK);
+              }
+              if (!p.seg[s].b_mn) {
+                load(sb, tb, fb, kb * kBK, bn0);
+              } else {
 #pragma unroll
-              for (int j = 0; j < Cfg::kBRows / 64; ++j) load(sb + j * 8192, tb, fb, bn0 + 64 * j, kb * kBK);
+                for (int j = 0; j < Cfg::kBRows / 64; ++j) load(sb + j * Cfg::kMnChunk, tb, fb, bn0 + 64 * j, kb * kBK);
+              }
             }
             used |= 1u << stage;
             last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
@@ -287,23 +312,33 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           int kb0, kb1;
           tc_seg_range(p, s, split, kb0, kb1);
           const int a_mn = p.seg[s].a_mn, b_mn = p.seg[s].b_mn;
-          for (int kb = kb0; kb < kb1; ++kb) {
+          const int step = (WIDE && p.seg[s].wide) ? 2 : 1;
+          for (int kb = kb0; kb < kb1; kb += step) {
             if (!mbar_wait(smem_u32(full_bar + stage), phase, p.err, DEV_TIMEOUT_MMA)) {
               ok = false;
               break;
             }
             tc_fence_after();
             const uint32_t sa = smem_u32(smem + stage * Cfg::kStageBytes);
-            const uint32_t sb = sa + Cfg::kABytes;
+            const uint32_t sb = sa + Cfg::kAStage;
+            const int nk = min(step, kb1 - kb);
+            for (int kk = 0; kk < nk; ++kk) {
+              // K-major: k-block kk is the next [rows][64] tile; the 16-wide
+              // k-slice starts 32 B into each swizzled row.  MN-major: k-block
+              // kk starts 64 k-rows (8 KB) into each chunk, the k-slice 16
+              // k-rows (2 KB) further.
+              const uint32_t ak = a_mn ? sa + kk * 8192 : sa + kk * Cfg::kABytes;
+              const uint32_t bk = b_mn ? sb + kk * 8192 : sb + kk * Cfg::kBBytes;
 #pragma unroll
-            for (int k = 0; k < kBK / 16; ++k) {
-              // K-major: the 16-wide k-slice starts 32 B into each swizzled row.
-              // MN-major: it starts 16 rows (2 KB) further down the tile.
-              const uint64_t ad = a_mn ? smem_desc_sw128(sa + k * 2048, 8192, 1024) : smem_desc_sw128(sa + k * 32, 16, 1024);
-              const uint64_t bd = b_mn ? smem_desc_sw128(sb + k * 2048, 8192, 1024) : smem_desc_sw128(sb + k * 32, 16, 1024);
-              if (PAIR) tc_mma_f16_pair(d_tmem, ad, bd, idesc[s], accumulate);
-              else tc_mma_f16(d_tmem, ad, bd, idesc[s], accumulate);
-              accumulate = 1;
+              for (int k = 0; k < kBK / 16; ++k) {
+                const uint64_t ad = a_mn ? smem_desc_sw128(ak + k * 2048, Cfg::kMnChunk, 1024)
+                                         : smem_desc_sw128(ak + k * 32, 16, 1024);
+                const uint64_t bd = b_mn ? smem_desc_sw128(bk + k * 2048, Cfg::kMnChunk, 1024)
+                                         : smem_desc_sw128(bk + k * 32, 16, 1024);
+                if (PAIR) tc_mma_f16_pair(d_tmem, ad, bd, idesc[s], accumulate);
+                else tc_mma_f16(d_tmem, ad, bd, idesc[s], accumulate);
+                accumulate = 1;
+              }
             }
             // frees the stage (in both CTAs of a pair) once these MMAs have read it
             if (PAIR) tc_commit_pair(smem_u32(empty_bar + stage), 0x3);
