@@ -46,7 +46,7 @@ int current_device_info(DeviceInfo **out) {
       if (cudaGetSymbolAddress(reinterpret_cast<void **>(&d.err), g_dev_err) != cudaSuccess) return QLORA_ERR_CUDA;
       // One-time fill of the quantizer's code table (a constant of the NF4
       // levels), completed before any library launch on this device.
-      code_lut_init_kernel<<<kCodeBins / 256, 256>>>();
+      code_lut_init_kernel<<<(kCodeLutBytes + 255) / 256, 256>>>();
       if (cudaGetLastError() != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess) return QLORA_ERR_CUDA;
       d.init = true;
     }
@@ -741,8 +741,8 @@ int qlora_quantize_nf4_dq(const void *W, int w_dtype, int64_t n_out, int64_t k_i
   const int64_t nblk = (numel + 63) / 64;
   float *c2 = reinterpret_cast<float *>(ws);
   double *partial = reinterpret_cast<double *>(reinterpret_cast<uint8_t *>(ws) + align_up((size_t)nblk * 4));
-  const int64_t ngroups = numel >> 8;
-  const int grid1 = (int)std::max<int64_t>(1, std::min<int64_t>((ngroups + 7) / 8, kQuantMaxCtas));
+  const int64_t ngroups = numel >> 9;   // 512-element groups, one per warp iteration
+  const int grid1 = (int)std::max<int64_t>(1, std::min<int64_t>((ngroups + 7) / 8, std::min(kQuantMaxCtas, dev->sms * kQuantCtasPerSm)));
   {
   ProfScope prof(QLORA_KERNEL_QUANTIZE, st);
   if (w_dtype == QLORA_DTYPE_F32)
@@ -782,8 +782,8 @@ int qlora_quantize_nf4_dq_noalloc(const void *W, int w_dtype, int64_t n_out, int
   const int64_t nblk = (numel + 63) / 64;
   float *c2 = reinterpret_cast<float *>(scratch);
   double *partial = reinterpret_cast<double *>(scratch + kNoallocC2Bytes);
-  const int64_t ngroups = numel >> 8;
-  const int grid1 = (int)std::max<int64_t>(1, std::min<int64_t>((ngroups + 7) / 8, kQuantMaxCtas));
+  const int64_t ngroups = numel >> 9;   // 512-element groups, one per warp iteration
+  const int grid1 = (int)std::max<int64_t>(1, std::min<int64_t>((ngroups + 7) / 8, std::min(kQuantMaxCtas, dev->sms * kQuantCtasPerSm)));
   if (w_dtype == QLORA_DTYPE_F32)
     nf4_quantize_kernel<float><<<grid1, kQuantThreads, 0, st>>>(reinterpret_cast<const float *>(W), numel, codes, c2,
                                                                partial);

@@ -44,6 +44,7 @@ __constant__ float kNF4[16] = {
 };
 
 constexpr int kQuantThreads = 256;
+constexpr int kQuantCtasPerSm = 5;     // resident at 48 registers per thread
 constexpr int kQuantMaxCtas = 148 * 8;
 
 // Decision thresholds for the nearest-level search.  Level j+1 beats level j
@@ -77,61 +78,79 @@ struct NF4Thresholds {
 // one code for every x in those five bins, so any estimate of
 // x = fp32(w / absmax) that is within one bin of x and lands in it (the
 // estimate w * (1/absmax) is within a few ulps, far below a bin) gives the
-// exact code.  The bins near a threshold (5 per threshold, 0.46% of them) are
-// marked, and their weights take the exact division.
+// exact code.  The bins near a threshold (5 per threshold, 0.46% of them) hold
+// kCodeBoundary | j, j the index of that threshold (thresholds are hundreds of
+// bins apart, so there is one), and their weights take the exact division:
+// the code is then j + (x > t_j).
+//
+// The table is indexed by b + 1, b the estimated bin, so that the two
+// rounding overshoots b = -1 and b = kCodeBins (x within an ulp of -1 or 1)
+// need no clamp: entry i holds the code of bin min(max(i - 1, 0), kCodeBins - 1).
 constexpr int kCodeBins = 16384;
-constexpr uint8_t kCodeBoundary = 0xFF;
+constexpr int kCodeLutEntries = kCodeBins + 2;
+constexpr int kCodeLutBytes = (kCodeLutEntries + 15) / 16 * 16;
+constexpr uint8_t kCodeBoundary = 0x80;
 
 // The table, filled once per device from the same thresholds the exact path
 // uses (code_lut_init_kernel), and copied into shared memory by each CTA.
-__device__ __align__(16) uint8_t g_code_lut[kCodeBins];
+__device__ __align__(16) uint8_t g_code_lut[kCodeLutBytes];
 
 __global__ void __launch_bounds__(256) code_lut_init_kernel() {
-  const int b = blockIdx.x * blockDim.x + threadIdx.x;
-  if (b >= kCodeBins) return;
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= kCodeLutBytes) return;
+  const int b = min(max(i - 1, 0), kCodeBins - 1);
   NF4Thresholds th;
   th.init();
   uint32_t code = 0;
-  bool edge = false;
+  int edge = -1;
 #pragma unroll
   for (int j = 0; j < 15; ++j) {
     const int tb = (int)floor(((double)th.t[j] + 1.0) * (kCodeBins / 2));
     code += tb < b ? 1u : 0u;
-    edge |= tb >= b - 2 && tb <= b + 2;
+    if (tb >= b - 2 && tb <= b + 2) edge = j;
   }
-  g_code_lut[b] = edge ? kCodeBoundary : (uint8_t)code;
+  g_code_lut[i] = edge >= 0 ? (uint8_t)(kCodeBoundary | edge) : (uint8_t)code;
 }
 
 // Copy the table into shared memory (all threads of the CTA).
 __device__ __forceinline__ void load_code_lut(uint8_t *lut) {
-  for (int i = threadIdx.x; i < kCodeBins / 16; i += blockDim.x)
+  for (int i = threadIdx.x; i < kCodeLutBytes / 16; i += blockDim.x)
     reinterpret_cast<uint4 *>(lut)[i] = reinterpret_cast<const uint4 *>(g_code_lut)[i];
 }
 
-// Code of v / amax given rinv = 1 / amax (amax > 0): table lookup, exact
-// division only in boundary bins.
-__device__ __forceinline__ uint32_t fast_code(float v, float amax, float rinv, const uint8_t *lut,
-                                              const NF4Thresholds &th) {
-  int b = __float2int_rd(__fmaf_rn(v * rinv, (float)(kCodeBins / 2), (float)(kCodeBins / 2)));
-  b = min(max(b, 0), kCodeBins - 1);
-  const uint32_t c = lut[b];
-  return c != kCodeBoundary ? c : th.encode(__fdiv_rn(v, amax));
+// Table index of v given sc = (1/absmax) * kCodeBins/2: the fused multiply-add
+// rounded toward zero lands in [2^23, 2^24), where its bits minus those of
+// 2^23 are floor(v * sc + kCodeBins/2 + 1) = b + 1 exactly.  Any non-finite
+// or out-of-range value (a NaN weight) is clamped into the table.
+__device__ __forceinline__ uint32_t code_lut_index(float v, float sc) {
+  const float y = __fmaf_rz(v, sc, 8388608.0f + (float)(kCodeBins / 2 + 1));
+  return min(__float_as_uint(y) - 0x4B000000u, (uint32_t)(kCodeLutEntries - 1));
 }
 
-__device__ __forceinline__ void load8(const float *__restrict__ p, float (&v)[8]) {
-  const float4 a = __ldg(reinterpret_cast<const float4 *>(p));
-  const float4 b = __ldg(reinterpret_cast<const float4 *>(p) + 1);
-  v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
-  v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+// Exact code of a weight whose table entry marks a boundary bin near threshold j.
+__device__ __forceinline__ uint32_t boundary_code(float v, float amax, uint32_t entry, const float *thr) {
+  const uint32_t j = entry & 0x0Fu;
+  return j + (__fdiv_rn(v, amax) > thr[j] ? 1u : 0u);
 }
 
-__device__ __forceinline__ void load8(const __nv_bfloat16 *__restrict__ p, float (&v)[8]) {
-  const uint4 a = __ldg(reinterpret_cast<const uint4 *>(p));
-  const uint32_t w[4] = {a.x, a.y, a.z, a.w};
+__device__ __forceinline__ void load16(const float *__restrict__ p, float (&v)[16]) {
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    v[2 * i] = __uint_as_float(w[i] << 16);
-    v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+  for (int q = 0; q < 4; ++q) {
+    const float4 a = __ldg(reinterpret_cast<const float4 *>(p) + q);
+    v[4 * q] = a.x; v[4 * q + 1] = a.y; v[4 * q + 2] = a.z; v[4 * q + 3] = a.w;
+  }
+}
+
+__device__ __forceinline__ void load16(const __nv_bfloat16 *__restrict__ p, float (&v)[16]) {
+#pragma unroll
+  for (int q = 0; q < 2; ++q) {
+    const uint4 a = __ldg(reinterpret_cast<const uint4 *>(p) + q);
+    const uint32_t w[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      v[8 * q + 2 * i] = __uint_as_float(w[i] << 16);
+      v[8 * q + 2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+    }
   }
 }
 
@@ -154,55 +173,75 @@ __device__ __forceinline__ double cta_sum_f64(double v, double *scratch) {
 // K1: per 64-block absmax c2, nearest-level codes, nibble packing, and one
 // fp64 partial sum of c2 per CTA (for the Double-Quantization mean).
 //
-// A warp processes groups of four 64-blocks (256 elements): lane l owns
-// elements [8l, 8l+8) of the group, i.e. 8 lanes per block; the block absmax
-// is reduced over those 8 lanes.  The (at most four) blocks after the last
-// full group are handled by the last CTA, one warp per block.
+// A warp processes groups of eight 64-blocks (512 elements): lane l owns
+// elements [16l, 16l+16) of the group, i.e. 4 lanes per block; the block
+// absmax is reduced over those 4 lanes.  The (at most eight) blocks after the
+// last full group are handled by the last CTA, one warp per block.
+constexpr float kTinyAbsmax = 1e-30f;   // below this 1/absmax may overflow: exact division
+
 template <typename TW>
-__global__ void __launch_bounds__(kQuantThreads) nf4_quantize_kernel(const TW *__restrict__ W, int64_t numel,
+__global__ void __launch_bounds__(kQuantThreads, kQuantCtasPerSm) nf4_quantize_kernel(const TW *__restrict__ W, int64_t numel,
                                                                     uint8_t *__restrict__ codes,
                                                                     float *__restrict__ c2,
                                                                     double *__restrict__ partial) {
   __shared__ double red[kQuantThreads / 32];
-  __shared__ __align__(16) uint8_t lut[kCodeBins];
+  __shared__ float thr[16];
+  __shared__ __align__(16) uint8_t lut[kCodeLutBytes];
   NF4Thresholds th;
   th.init();
+  if (threadIdx.x < 15)
+    thr[threadIdx.x] = __double2float_rd(((double)kNF4[threadIdx.x] + (double)kNF4[threadIdx.x + 1]) * 0.5);
   load_code_lut(lut);
   __syncthreads();
   const int lane = lane_id();
-  const int64_t ngroups = numel >> 8;
+  const int64_t ngroups = numel >> 9;
   const int64_t nwarps = (int64_t)gridDim.x * (kQuantThreads / 32);
   double acc = 0.0;
 
   for (int64_t g = (int64_t)blockIdx.x * (kQuantThreads / 32) + warp_id(); g < ngroups; g += nwarps) {
-    const int64_t base = (g << 8) + (lane << 3);
-    float v[8];
-    load8(W + base, v);
+    const int64_t base = (g << 9) + (lane << 4);
+    float v[16];
+    load16(W + base, v);
     float amax = 0.f;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[i]));
+    for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(v[i]));
     amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 1));
     amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 2));
-    amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 4));
-    uint32_t packed = 0;
-    if (amax == 0.f) {
-      packed = 0x77777777u;  // all-zero block: every element is the exact-zero level
-    } else {
-      const float rinv = __frcp_rn(amax);
+    uint32_t pk[2] = {0x77777777u, 0x77777777u};   // all-zero block: every element is the exact-zero level
+    if (amax >= kTinyAbsmax) {
+      const float sc = __frcp_rn(amax) * (float)(kCodeBins / 2);
 #pragma unroll
-      for (int i = 0; i < 8; ++i) packed |= fast_code(v[i], amax, rinv, lut, th) << (4 * i);
+      for (int h = 0; h < 2; ++h) {
+        uint32_t w = 0;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const float x = v[8 * h + i];
+          uint32_t c = lut[code_lut_index(x, sc)];
+          if (c & kCodeBoundary) c = boundary_code(x, amax, c, thr);
+          w |= c << (4 * i);
+        }
+        pk[h] = w;
+      }
+    } else if (amax != 0.f) {
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        uint32_t w = 0;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) w |= th.encode(__fdiv_rn(v[8 * h + i], amax)) << (4 * i);
+        pk[h] = w;
+      }
     }
-    reinterpret_cast<uint32_t *>(codes)[(g << 5) + lane] = packed;
-    if ((lane & 7) == 0) {
-      c2[(g << 2) + (lane >> 3)] = amax;
+    reinterpret_cast<uint2 *>(codes)[(g << 5) + lane] = make_uint2(pk[0], pk[1]);
+    if ((lane & 3) == 0) {
+      c2[(g << 3) + (lane >> 2)] = amax;
       acc += (double)amax;
     }
   }
 
-  // Tail: blocks [4*ngroups, nblk), at most 4, one warp each in the last CTA.
+  // Tail: blocks [8*ngroups, nblk), at most 8, one warp each in the last CTA.
   if (blockIdx.x == gridDim.x - 1) {
     const int64_t nblk = (numel + 63) >> 6;
-    const int64_t b = (ngroups << 2) + warp_id();
+    const int64_t b = (ngroups << 3) + warp_id();
     if (b < nblk) {
       const int64_t s = b << 6;
       const int64_t i0 = s + 2 * lane, i1 = i0 + 1;
