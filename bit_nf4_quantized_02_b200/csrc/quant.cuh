@@ -86,10 +86,14 @@ struct NF4Thresholds {
 // The table is indexed by b + 1, b the estimated bin, so that the two
 // rounding overshoots b = -1 and b = kCodeBins (x within an ulp of -1 or 1)
 // need no clamp: entry i holds the code of bin min(max(i - 1, 0), kCodeBins - 1).
+// In shared memory it is followed by zeros up to kCodeLutSpan entries, the
+// range of the 15-bit index below, so that no value of a weight (a NaN
+// included) can index outside it.
 constexpr int kCodeBins = 16384;
 constexpr int kCodeLutEntries = kCodeBins + 2;
 constexpr int kCodeLutBytes = (kCodeLutEntries + 15) / 16 * 16;
-constexpr uint8_t kCodeBoundary = 0x80;
+constexpr int kCodeLutSpan = 32768;
+constexpr uint32_t kCodeBoundary = 0x80;
 
 // The table, filled once per device from the same thresholds the exact path
 // uses (code_lut_init_kernel), and copied into shared memory by each CTA.
@@ -112,47 +116,83 @@ __global__ void __launch_bounds__(256) code_lut_init_kernel() {
   g_code_lut[i] = edge >= 0 ? (uint8_t)(kCodeBoundary | edge) : (uint8_t)code;
 }
 
-// Copy the table into shared memory (all threads of the CTA).
+// Copy the table into shared memory and zero the rest of its span (all
+// threads of the CTA).
 __device__ __forceinline__ void load_code_lut(uint8_t *lut) {
-  for (int i = threadIdx.x; i < kCodeLutBytes / 16; i += blockDim.x)
-    reinterpret_cast<uint4 *>(lut)[i] = reinterpret_cast<const uint4 *>(g_code_lut)[i];
+  for (int i = threadIdx.x; i < kCodeLutSpan / 16; i += blockDim.x)
+    reinterpret_cast<uint4 *>(lut)[i] =
+        i < kCodeLutBytes / 16 ? reinterpret_cast<const uint4 *>(g_code_lut)[i] : make_uint4(0, 0, 0, 0);
 }
 
 // Table index of v given sc = (1/absmax) * kCodeBins/2: the fused multiply-add
-// rounded toward zero lands in [2^23, 2^24), where its bits minus those of
-// 2^23 are floor(v * sc + kCodeBins/2 + 1) = b + 1 exactly.  Any non-finite
-// or out-of-range value (a NaN weight) is clamped into the table.
+// rounded toward zero lands in [2^23, 2^24), where the low bits of the result
+// are floor(v * sc + kCodeBins/2 + 1) = b + 1 exactly (2^23 has none set).
+// The 15-bit mask keeps any other value (a NaN weight) inside the span.
 __device__ __forceinline__ uint32_t code_lut_index(float v, float sc) {
   const float y = __fmaf_rz(v, sc, 8388608.0f + (float)(kCodeBins / 2 + 1));
-  return min(__float_as_uint(y) - 0x4B000000u, (uint32_t)(kCodeLutEntries - 1));
+  return __float_as_uint(y) & (uint32_t)(kCodeLutSpan - 1);
 }
 
-// Exact code of a weight whose table entry marks a boundary bin near threshold j.
-__device__ __forceinline__ uint32_t boundary_code(float v, float amax, uint32_t entry, const float *thr) {
-  const uint32_t j = entry & 0x0Fu;
-  return j + (__fdiv_rn(v, amax) > thr[j] ? 1u : 0u);
+// Four table entries (bytes) -> one word, entry i in byte i.
+__device__ __forceinline__ uint32_t pack_entries(uint32_t e0, uint32_t e1, uint32_t e2, uint32_t e3) {
+  return __byte_perm(__byte_perm(e0, e1, 0x0040), __byte_perm(e2, e3, 0x0040), 0x5410);
 }
 
-__device__ __forceinline__ void load16(const float *__restrict__ p, float (&v)[16]) {
+// Eight entries in two words -> eight 4-bit codes (the low nibble of each
+// entry; for a boundary entry that is its threshold index j), element i in
+// bits [4i, 4i+4).
+__device__ __forceinline__ uint32_t pack_nibbles(uint32_t a, uint32_t b) {
+  a &= 0x0F0F0F0Fu;
+  b &= 0x0F0F0F0Fu;
+  a |= a >> 4;   // byte 0: e0 | e1 << 4, byte 2: e2 | e3 << 4
+  b |= b >> 4;
+  return __byte_perm(a, b, 0x6420);
+}
+
+// Bit q of the result: entry q of the word is a boundary entry.
+__device__ __forceinline__ uint32_t boundary_bits(uint32_t w) {
+  return (((w & 0x80808080u) >> 7) * 0x01020408u) >> 24;
+}
+
+// Sixteen consecutive weights as loaded (two or four 16-byte loads).  Issuing
+// the next group's loads before processing this one (one more group in
+// flight per warp) was measured slower: the registers it needs drop the
+// kernel from five to four resident CTAs per SM.
+template <typename TW>
+struct Raw16;
+template <>
+struct Raw16<float> {
+  float4 q[4];
+  __device__ __forceinline__ void load(const float *__restrict__ p) {
 #pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    const float4 a = __ldg(reinterpret_cast<const float4 *>(p) + q);
-    v[4 * q] = a.x; v[4 * q + 1] = a.y; v[4 * q + 2] = a.z; v[4 * q + 3] = a.w;
+    for (int i = 0; i < 4; ++i) q[i] = __ldg(reinterpret_cast<const float4 *>(p) + i);
   }
-}
-
-__device__ __forceinline__ void load16(const __nv_bfloat16 *__restrict__ p, float (&v)[16]) {
-#pragma unroll
-  for (int q = 0; q < 2; ++q) {
-    const uint4 a = __ldg(reinterpret_cast<const uint4 *>(p) + q);
-    const uint32_t w[4] = {a.x, a.y, a.z, a.w};
+  __device__ __forceinline__ void unpack(float (&v)[16]) const {
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      v[8 * q + 2 * i] = __uint_as_float(w[i] << 16);
-      v[8 * q + 2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+      v[4 * i] = q[i].x; v[4 * i + 1] = q[i].y; v[4 * i + 2] = q[i].z; v[4 * i + 3] = q[i].w;
     }
   }
-}
+};
+template <>
+struct Raw16<__nv_bfloat16> {
+  uint4 q[2];
+  __device__ __forceinline__ void load(const __nv_bfloat16 *__restrict__ p) {
+#pragma unroll
+    for (int i = 0; i < 2; ++i) q[i] = __ldg(reinterpret_cast<const uint4 *>(p) + i);
+  }
+  __device__ __forceinline__ void unpack(float (&v)[16]) const {
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const uint32_t w[4] = {q[h].x, q[h].y, q[h].z, q[h].w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        v[8 * h + 2 * i] = __uint_as_float(w[i] << 16);
+        v[8 * h + 2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+      }
+    }
+  }
+};
 
 __device__ __forceinline__ float load1(const float *p) { return __ldg(p); }
 __device__ __forceinline__ float load1(const __nv_bfloat16 *p) { return __bfloat162float(*p); }
@@ -186,7 +226,7 @@ __global__ void __launch_bounds__(kQuantThreads, kQuantCtasPerSm) nf4_quantize_k
                                                                     double *__restrict__ partial) {
   __shared__ double red[kQuantThreads / 32];
   __shared__ float thr[16];
-  __shared__ __align__(16) uint8_t lut[kCodeLutBytes];
+  __shared__ __align__(16) uint8_t lut[kCodeLutSpan];
   NF4Thresholds th;
   th.init();
   if (threadIdx.x < 15)
@@ -200,38 +240,47 @@ __global__ void __launch_bounds__(kQuantThreads, kQuantCtasPerSm) nf4_quantize_k
 
   for (int64_t g = (int64_t)blockIdx.x * (kQuantThreads / 32) + warp_id(); g < ngroups; g += nwarps) {
     const int64_t base = (g << 9) + (lane << 4);
+    Raw16<TW> cur;
+    cur.load(W + base);
     float v[16];
-    load16(W + base, v);
+    cur.unpack(v);
     float amax = 0.f;
 #pragma unroll
     for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(v[i]));
     amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 1));
     amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 2));
-    uint32_t pk[2] = {0x77777777u, 0x77777777u};   // all-zero block: every element is the exact-zero level
+    uint32_t pk0 = 0x77777777u, pk1 = 0x77777777u;   // all-zero block: every element is the exact-zero level
     if (amax >= kTinyAbsmax) {
       const float sc = __frcp_rn(amax) * (float)(kCodeBins / 2);
+      uint32_t e[16];
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        uint32_t w = 0;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const float x = v[8 * h + i];
-          uint32_t c = lut[code_lut_index(x, sc)];
-          if (c & kCodeBoundary) c = boundary_code(x, amax, c, thr);
-          w |= c << (4 * i);
+      for (int i = 0; i < 16; ++i) e[i] = lut[code_lut_index(v[i], sc)];
+      const uint32_t w0 = pack_entries(e[0], e[1], e[2], e[3]), w1 = pack_entries(e[4], e[5], e[6], e[7]);
+      const uint32_t w2 = pack_entries(e[8], e[9], e[10], e[11]), w3 = pack_entries(e[12], e[13], e[14], e[15]);
+      pk0 = pack_nibbles(w0, w1);
+      pk1 = pack_nibbles(w2, w3);
+      if ((w0 | w1 | w2 | w3) & 0x80808080u) {
+        // Boundary weights (a few per warp): exact division, code = j + (x > t_j).
+        uint32_t m = boundary_bits(w0) | (boundary_bits(w1) << 4) | (boundary_bits(w2) << 8) | (boundary_bits(w3) << 12);
+        while (m) {
+          const int i = __ffs(m) - 1;
+          m &= m - 1;
+          const int sh = 4 * (i & 7);
+          uint32_t &pk = i < 8 ? pk0 : pk1;
+          const uint32_t j = (pk >> sh) & 0xFu;
+          const uint32_t c = j + (__fdiv_rn(load1(W + base + i), amax) > thr[j] ? 1u : 0u);
+          pk = (pk & ~(0xFu << sh)) | (c << sh);
         }
-        pk[h] = w;
       }
     } else if (amax != 0.f) {
+      pk0 = pk1 = 0;
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        uint32_t w = 0;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) w |= th.encode(__fdiv_rn(v[8 * h + i], amax)) << (4 * i);
-        pk[h] = w;
+      for (int i = 0; i < 8; ++i) {
+        pk0 |= th.encode(__fdiv_rn(v[i], amax)) << (4 * i);
+        pk1 |= th.encode(__fdiv_rn(v[8 + i], amax)) << (4 * i);
       }
     }
-    reinterpret_cast<uint2 *>(codes)[(g << 5) + lane] = make_uint2(pk[0], pk[1]);
+    reinterpret_cast<uint2 *>(codes)[(g << 5) + lane] = make_uint2(pk0, pk1);
     if ((lane & 3) == 0) {
       c2[(g << 3) + (lane >> 2)] = amax;
       acc += (double)amax;

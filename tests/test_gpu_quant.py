@@ -52,6 +52,44 @@ def test_quantize_special_values():
     _check_bit_exact(W)
 
 
+def _near_threshold_blocks(seed: int) -> np.ndarray:
+    """64-blocks whose first element fixes the absmax (alternating sign) and
+    whose others sit at, within 40 ulps of, and within five 2^-13 steps of,
+    every decision threshold, at several absmax scales."""
+    g = np.random.default_rng(seed)
+    xs = []
+    for m in nf4dq.NF4_MIDPOINTS.astype(np.float64):
+        t = np.float32(m)
+        up, down = t, t
+        xs.append(t)
+        for _ in range(40):
+            up = np.nextafter(up, np.float32(np.inf), dtype=np.float32)
+            down = np.nextafter(down, np.float32(-np.inf), dtype=np.float32)
+            xs += [up, down]
+        xs += [np.float32(m + k * 2.0 ** -13 + g.uniform(-2.0 ** -14, 2.0 ** -14)) for k in range(-5, 6)]
+    xs = np.array(xs, dtype=np.float32)
+    blocks = []
+    for amax in (1.0, 0.37, 3.1e-5, 1234.5, 3 * 2.0 ** -20, 7e-3):
+        a = np.float32(amax)
+        v = np.clip((xs.astype(np.float64) * amax).astype(np.float32), -a, a)
+        for n, i in enumerate(range(0, v.size, 63)):
+            blk = np.zeros(64, dtype=np.float32)
+            blk[0] = a if n % 2 == 0 else -a
+            blk[1:1 + v[i:i + 63].size] = v[i:i + 63]
+            blocks.append(blk)
+    return np.stack(blocks)
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_quantize_near_every_threshold(dtype):
+    """Weights at and around each NF4 decision threshold: the nearest-level
+    decision must match the oracle's exact division bit for bit (this drives
+    the boundary bins of the kernel's table and their exact-division path)."""
+    B = _near_threshold_blocks(77)
+    W = torch.from_numpy(B[: B.shape[0] // 8 * 8].reshape(-1, 512).copy())
+    _check_bit_exact(W.to(dtype))
+
+
 def test_quantize_constant_c2_gives_zero_c1():
     W = torch.ones(16, 64 * 256 // 16, dtype=torch.float32) * 0.5
     q, oq = _check_bit_exact(W)
