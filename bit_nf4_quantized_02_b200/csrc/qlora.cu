@@ -755,9 +755,9 @@ int qlora_quantize_nf4_dq(const void *W, int w_dtype, int64_t n_out, int64_t k_i
   rc = launch_status();
   if (rc) return rc;
   const int64_t nb256 = (nblk + 255) / 256;
-  const int grid2 = (int)std::max<int64_t>(1, std::min<int64_t>(nb256, (int64_t)dev->sms * 4));
+  const int grid2 = (int)std::max<int64_t>(1, std::min<int64_t>((nb256 + kDqWarps - 1) / kDqWarps, (int64_t)dev->sms * 4));
   ProfScope prof(QLORA_KERNEL_DQ_CONSTANTS, st);
-  dq_constants_kernel<<<grid2, 256, 0, st>>>(c2, nblk, partial, grid1, c2_fp8, c1, c2_mean);
+  dq_constants_kernel<<<grid2, 32 * kDqWarps, 0, st>>>(c2, nblk, partial, grid1, c2_fp8, c1, c2_mean);
   return launch_status();
 }
 
@@ -793,8 +793,8 @@ int qlora_quantize_nf4_dq_noalloc(const void *W, int w_dtype, int64_t n_out, int
   rc = launch_status();
   if (rc) return rc;
   const int64_t nb256 = (nblk + 255) / 256;
-  const int grid2 = (int)std::max<int64_t>(1, std::min<int64_t>(nb256, (int64_t)dev->sms * 4));
-  dq_constants_kernel<<<grid2, 256, 0, st>>>(c2, nblk, partial, grid1, c2_fp8, c1, c2_mean);
+  const int grid2 = (int)std::max<int64_t>(1, std::min<int64_t>((nb256 + kDqWarps - 1) / kDqWarps, (int64_t)dev->sms * 4));
+  dq_constants_kernel<<<grid2, 32 * kDqWarps, 0, st>>>(c2, nblk, partial, grid1, c2_fp8, c1, c2_mean);
   return launch_status();
 }
 

@@ -333,15 +333,17 @@ __device__ __forceinline__ float e4m3_to_f32(uint8_t code) {
 
 // K2: Double Quantization of c2.  Every CTA first forms the same mean mu from
 // the K1 partials in a fixed order (so mu is deterministic and identical in
-// all CTAs), then quantizes 256-blocks of c2 - mu:
+// all CTAs), then quantizes 256-blocks of c2 - mu, one warp per block (lane l
+// owns entries [8l, 8l+8)):
 //   c1 = absmax(c2 - mu) / 448,  code8 = E4M3(fp32((c2 - mu) / c1)).
-__global__ void __launch_bounds__(256) dq_constants_kernel(const float *__restrict__ c2, int64_t nblk,
-                                                           const double *__restrict__ partial, int npartial,
-                                                           uint8_t *__restrict__ c2_fp8, float *__restrict__ c1,
-                                                           float *__restrict__ mu_out) {
-  __shared__ double red[8];
+constexpr int kDqWarps = 8;
+
+__global__ void __launch_bounds__(32 * kDqWarps) dq_constants_kernel(const float *__restrict__ c2, int64_t nblk,
+                                                                    const double *__restrict__ partial, int npartial,
+                                                                    uint8_t *__restrict__ c2_fp8,
+                                                                    float *__restrict__ c1, float *__restrict__ mu_out) {
+  __shared__ double red[kDqWarps];
   __shared__ float mu_s;
-  __shared__ float wmax[8];
   double acc = 0.0;
   for (int i = threadIdx.x; i < npartial; i += blockDim.x) acc += partial[i];
   const double total = cta_sum_f64(acc, red);
@@ -351,22 +353,40 @@ __global__ void __launch_bounds__(256) dq_constants_kernel(const float *__restri
   }
   __syncthreads();
   const float mu = mu_s;
+  const int lane = lane_id();
   const int64_t nb256 = (nblk + 255) >> 8;
-  for (int64_t beta = blockIdx.x; beta < nb256; beta += gridDim.x) {
-    const int64_t idx = (beta << 8) + threadIdx.x;
-    const float d = idx < nblk ? __fsub_rn(__ldg(c2 + idx), mu) : 0.f;
-    float a = fabsf(d);
+  for (int64_t beta = (int64_t)blockIdx.x * kDqWarps + warp_id(); beta < nb256; beta += (int64_t)gridDim.x * kDqWarps) {
+    const int64_t i0 = (beta << 8) + (lane << 3);
+    const bool full = i0 + 8 <= nblk;
+    float d[8];
+    if (full) {
+      const float4 a = __ldg(reinterpret_cast<const float4 *>(c2 + i0));
+      const float4 b = __ldg(reinterpret_cast<const float4 *>(c2 + i0) + 1);
+      const float x[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, o));
-    if (lane_id() == 0) wmax[warp_id()] = a;
-    __syncthreads();
-    float A = wmax[0];
+      for (int k = 0; k < 8; ++k) d[k] = __fsub_rn(x[k], mu);
+    } else {
 #pragma unroll
-    for (int w = 1; w < 8; ++w) A = fmaxf(A, wmax[w]);
-    __syncthreads();
+      for (int k = 0; k < 8; ++k) d[k] = i0 + k < nblk ? __fsub_rn(__ldg(c2 + i0 + k), mu) : 0.f;
+    }
+    float A = 0.f;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) A = fmaxf(A, fabsf(d[k]));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) A = fmaxf(A, __shfl_xor_sync(0xFFFFFFFFu, A, o));
     const float c1v = __fdiv_rn(A, 448.0f);
-    if (idx < nblk) c2_fp8[idx] = (c1v == 0.f) ? (uint8_t)0 : f32_to_e4m3_satfinite(__fdiv_rn(d, c1v));
-    if (threadIdx.x == 0) c1[beta] = c1v;
+    uint32_t q[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) q[k] = c1v == 0.f ? 0u : (uint32_t)f32_to_e4m3_satfinite(__fdiv_rn(d[k], c1v));
+    if (full) {
+      reinterpret_cast<uint2 *>(c2_fp8 + i0)[0] =
+          make_uint2(q[0] | (q[1] << 8) | (q[2] << 16) | (q[3] << 24), q[4] | (q[5] << 8) | (q[6] << 16) | (q[7] << 24));
+    } else {
+#pragma unroll
+      for (int k = 0; k < 8; ++k)
+        if (i0 + k < nblk) c2_fp8[i0 + k] = (uint8_t)q[k];
+    }
+    if (lane == 0) c1[beta] = c1v;
   }
 }
 
