@@ -181,11 +181,14 @@ struct GemmSeg {
 
 int pick_bn(int64_t N) { return N <= 64 ? 64 : (N <= 128 ? 128 : 256); }
 
-// Split-K factor for a single-segment product whose tile grid leaves SMs idle.
+// Split-K factor for a single-segment product whose tile grid leaves SMs idle:
+// as many splits as fit in one wave, so no CTA runs a second unit (these are
+// the HBM-streaming rank-r products; one longer unit per SM streams faster
+// than more, shorter units over several waves).
 void choose_splits(int64_t tiles, int64_t nkb, int sms, bool allow, int *splits, int *kbps) {
   int s = 1;
   if (allow && tiles > 0 && tiles < sms && nkb > 1) {
-    s = (int)std::min<int64_t>(nkb, (2 * (int64_t)sms + tiles - 1) / tiles);
+    s = (int)std::max<int64_t>(1, std::min<int64_t>(nkb, sms / tiles));
   }
   int k = (int)((nkb + s - 1) / s);
   if (k < 1) k = 1;
