@@ -33,7 +33,8 @@ namespace qlora {
 
 constexpr int kBM = 128;   // MMA M (TMEM lanes)
 constexpr int kBK = 64;    // one 128-byte swizzle row of bf16
-constexpr int kGemmThreads = 192;
+constexpr int kGemmThreads = 224;
+constexpr int kProdBWarp = 6;   // the B producer; warp 0 produces A
 
 struct TcSeg {
   int nkb;   // 64-wide k-blocks in this segment
@@ -161,7 +162,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < S; ++i) {
-      mbar_init(smem_u32(full_bar + i), 1);
+      mbar_init(smem_u32(full_bar + i), 2);    // the A and the B producer (of the leader, in a pair)
       mbar_init(smem_u32(empty_bar + i), 1);
     }
     for (int i = 0; i < 2; ++i) {
@@ -201,9 +202,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
   const int units = p.m_tiles * p.n_tiles * p.splits;
 
-  if (warp == 0) {
-    // ------------------------------------------------------------ producer
+  if (warp == 0 || warp == kProdBWarp) {
+    // ------------------------------------------------------------ producers
+    // One thread streams A and another B: the TMA engine overlaps the copies
+    // of different issuing threads, while one thread's copies are served
+    // largely one after another.  Each arms the full barrier with its own
+    // bytes (in a pair, both CTAs' bytes of its operand).
     if (lane == 0) {
+      const bool isA = warp == 0;
       int stage = 0;
       uint32_t phase = 0;
       uint32_t used = 0;           // stages that received at least one load
@@ -240,24 +246,29 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             const uint32_t fb = PAIR ? mapa_shared(fb_local, 0) : fb_local;
             // a box is counted in full, also where it reaches past the
             // segment (those k-blocks are zero-filled or simply not used)
-            const uint32_t bytes = wide ? Cfg::kStageBytes : Cfg::kABytes + Cfg::kBBytes;
+            const uint32_t bytes = isA ? (wide ? Cfg::kAStage : Cfg::kABytes)
+                                       : (wide ? Cfg::kStageBytes - Cfg::kAStage : Cfg::kBBytes);
             if (leader) mbar_arrive_expect_tx(fb_local, (PAIR ? 2 : 1) * bytes);
             const uint32_t sa = smem_u32(smem + stage * Cfg::kStageBytes);
             const uint32_t sb = sa + Cfg::kAStage;
             if (wide) {
               // K-major maps are {64 k, rows, k-blocks}: smem [k-block][row][64].
               // MN-major maps are {64 mn, k, 64-wide mn chunks}: smem [chunk][k][64].
-              if (!p.seg[s].a_mn) load3(sa, ta, fb, am, kb);
-              else load3(sa, ta, fb, kb * kBK, am >> 6);
-              if (!p.seg[s].b_mn) load3(sb, tb, fb, bn0, kb);
-              else load3(sb, tb, fb, kb * kBK, bn0 >> 6);
-            } else {
+              if (isA) {
+                if (!p.seg[s].a_mn) load3(sa, ta, fb, am, kb);
+                else load3(sa, ta, fb, kb * kBK, am >> 6);
+              } else {
+                if (!p.seg[s].b_mn) load3(sb, tb, fb, bn0, kb);
+                else load3(sb, tb, fb, kb * kBK, bn0 >> 6);
+              }
+            } else if (isA) {
               if (!p.seg[s].a_mn) {
                 load(sa, ta, fb, kb * kBK, am);
               } else {
                 load(sa, ta, fb, am, kb * kBK);
                 load(sa + Cfg::kMnChunk, ta, fb, am + 64, kb * kBK);
               }
+            } else {
               if (!p.seg[s].b_mn) {
                 load(sb, tb, fb, kb * kBK, bn0);
               } else {
@@ -358,7 +369,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       else tc_commit(smem_u32(done_bar));
       mbar_wait(smem_u32(done_bar), 0, p.err, DEV_TIMEOUT_DRAIN);
     }
-  } else {
+  } else if (warp < kProdBWarp) {
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;  // TMEM lane quarter this warp may access
     int t = 0;
