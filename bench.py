@@ -288,12 +288,18 @@ def run_ours(args, rank, world, local_rank):
     if sampler:
         sampler.start()
         time.sleep(0.5)
-    qlora.profile_start(args.steps * 200 * wl.layers + 64)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record()
     for _ in range(args.steps):
         step()
     e1.record()
+    torch.cuda.synchronize()
+    # The per-launch event log (kernel table, roofline) comes from a second
+    # pass of the same steps on every rank: events between launches would
+    # serialise the programmatic dependent launches of the timed pass.
+    qlora.profile_start(args.steps * 200 * wl.layers + 64)
+    for _ in range(args.steps):
+        step()
     torch.cuda.synchronize()
     launches = qlora.profile_stop()
     if world > 1:
@@ -404,15 +410,22 @@ def _timed(qlora, step, args, dev, world, rank, local_rank, profile=True):
     if sampler:
         sampler.start()
         time.sleep(0.5)
-    if profile:
-        qlora.profile_start(args.steps * 256 + 64)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record()
     for _ in range(args.steps):
         step()
     e1.record()
     torch.cuda.synchronize()
-    launches = qlora.profile_stop() if profile else []
+    # The per-launch event log (kernel table, roofline) comes from a second
+    # pass of the same steps: events between launches would serialise the
+    # programmatic dependent launches of the timed pass.
+    launches = []
+    if profile:
+        qlora.profile_start(args.steps * 256 + 64)
+        for _ in range(args.steps):
+            step()
+        torch.cuda.synchronize()
+        launches = qlora.profile_stop()
     clocks = sampler.stop() if sampler else None
     ms = e0.elapsed_time(e1) / args.steps
     t = torch.tensor([ms], device=dev)

@@ -110,6 +110,55 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int *er
 }
 
 // ---------------------------------------------------------------------------
+// Programmatic dependent launch.  A kernel launched as a programmatic
+// dependent may start before the previous kernel in its stream has finished:
+// it must pdl_wait() before its first access to global memory that another
+// kernel writes or reads, and every such kernel waits in every CTA, so that a
+// grid never completes before the grid it follows.  pdl_trigger() lets the
+// next kernel launch (and run up to its own wait) while this one runs.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+// Loads of data that an earlier kernel of the stream wrote, in a kernel that
+// may have started before that kernel finished.  The read-only path (__ldg)
+// lets the compiler treat the data as invariant and schedule the load before
+// pdl_wait(); volatile asm keeps these loads after it (volatile asm is never
+// reordered with other volatile asm), and .cg reads them at L2.
+__device__ __forceinline__ uint4 ld_dep_v4(const void *p) {
+  uint4 v;
+  asm volatile("ld.global.cg.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+__device__ __forceinline__ float4 ld_dep_f4(const float *p) {
+  const uint4 v = ld_dep_v4(p);
+  return make_float4(__uint_as_float(v.x), __uint_as_float(v.y), __uint_as_float(v.z), __uint_as_float(v.w));
+}
+__device__ __forceinline__ uint32_t ld_dep_u32(const void *p) {
+  uint32_t v;
+  asm volatile("ld.global.cg.u32 %0, [%1];" : "=r"(v) : "l"(p));
+  return v;
+}
+__device__ __forceinline__ float ld_dep_f32(const float *p) { return __uint_as_float(ld_dep_u32(p)); }
+__device__ __forceinline__ double ld_dep_f64(const double *p) {
+  double v;
+  asm volatile("ld.global.cg.f64 %0, [%1];" : "=d"(v) : "l"(p));
+  return v;
+}
+__device__ __forceinline__ uint32_t ld_dep_u16(const void *p) {
+  uint16_t v;
+  asm volatile("ld.global.cg.u16 %0, [%1];" : "=h"(v) : "l"(p));
+  return v;
+}
+__device__ __forceinline__ uint32_t ld_dep_u8(const uint8_t *p) {
+  uint16_t v;
+  asm volatile("ld.global.cg.u8 %0, [%1];" : "=h"(v) : "l"(p));
+  return v;
+}
+
+// ---------------------------------------------------------------------------
 // Thread-block clusters
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ uint32_t cluster_ctarank() {

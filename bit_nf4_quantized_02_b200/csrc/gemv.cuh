@@ -454,7 +454,7 @@ __global__ void __launch_bounds__(256) gemv_epilogue_kernel(const float *__restr
     reinterpret_cast<uint4 *>(l2s + jj * 64)[c] = v;
   }
   asm volatile("griddepcontrol.wait;" ::: "memory");
-  for (int i = threadIdx.x; i < mn * r; i += blockDim.x) ts[i] = s * __ldcg(tacc + (int64_t)mb * r + i);
+  for (int i = threadIdx.x; i < mn * r; i += blockDim.x) ts[i] = s * ld_dep_f32(tacc + (int64_t)mb * r + i);
   __syncthreads();
   if (blockIdx.x == 0 && T_save) {
     for (int i = threadIdx.x; i < mn * r; i += blockDim.x) {
@@ -473,7 +473,7 @@ __global__ void __launch_bounds__(256) gemv_epilogue_kernel(const float *__restr
 #pragma unroll
   for (int i = 0; i < kTok; ++i) {
     const int m = q + 4 * i;
-    y[i] = m < mn ? __ldcg(acc + (int64_t)(mb + m) * N + n) : 0.f;
+    y[i] = m < mn ? ld_dep_f32(acc + (int64_t)(mb + m) * N + n) : 0.f;
   }
   for (int jj = 0; jj < r; ++jj) {
     const float l2 = __bfloat162float(l2s[jj * 64 + c]);

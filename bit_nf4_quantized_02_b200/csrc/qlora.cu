@@ -91,6 +91,27 @@ size_t align_up(size_t x, size_t a = 256) { return (x + a - 1) / a * a; }
 
 int launch_status() { return cudaGetLastError() == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA; }
 
+// Launch `kernel` on `st` as a programmatic dependent of the previous launch.
+// Every kernel launched this way waits (griddepcontrol.wait) before it touches
+// memory another kernel writes or reads.
+template <typename... KArgs, typename... Args>
+int launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, Args... args) {
+  cudaLaunchConfig_t cfg;
+  std::memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kernel, args...) != cudaSuccess) return QLORA_ERR_CUDA;
+  return launch_status();
+}
+
+
 // ---------------------------------------------------------------- TMA maps
 using EncodeTiledFn = PFN_cuTensorMapEncodeTiled_v12000;
 
@@ -225,8 +246,8 @@ int launch_gemm_bn(const CUtensorMap *maps, TcGemmArgs &args, int sms, DeviceInf
   const int units = args.m_tiles * args.n_tiles * args.splits;
   const int grid = std::max(1, std::min(units, sms));
   ProfScope prof(kind, st);
-  kernel<<<grid, kGemmThreads, Cfg::kSmemBytes, st>>>(maps[0], maps[1], maps[2], maps[3], args);
-  return launch_status();
+  return launch_pdl(kernel, dim3(grid), dim3(kGemmThreads), Cfg::kSmemBytes, st, maps[0], maps[1], maps[2], maps[3],
+                    args);
 }
 
 // CTA-pair GEMM (256 x 256 tiles): a persistent grid of 2-CTA clusters, as
@@ -238,16 +259,18 @@ int launch_gemm_pair(const CUtensorMap *maps, TcGemmArgs &args, DeviceInfo *dev,
   auto kernel = tc_gemm_kernel<BN, true, false, WIDE>;
   cudaLaunchConfig_t cfg;
   std::memset(&cfg, 0, sizeof(cfg));
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.blockDim = dim3(kGemmThreads, 1, 1);
   cfg.dynamicSmemBytes = Cfg::kSmemBytes;
   cfg.stream = st;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 1;   // the occupancy query takes the cluster shape alone
   const int idx = 3 + (WIDE ? 8 : 0);
   if (!dev->gemm_attr[idx]) {
     if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes) != cudaSuccess)
@@ -261,6 +284,7 @@ int launch_gemm_pair(const CUtensorMap *maps, TcGemmArgs &args, DeviceInfo *dev,
   const int units = args.m_tiles * args.n_tiles * args.splits;
   const int clusters = std::max(1, std::min(units, dev->pair_clusters[WIDE ? 1 : 0]));
   cfg.gridDim = dim3(2 * (unsigned)clusters, 1, 1);
+  cfg.numAttrs = 2;   // launched as a programmatic dependent of the previous kernel
   ProfScope prof(kind, st);
   if (cudaLaunchKernelEx(&cfg, kernel, maps[0], maps[1], maps[2], maps[3], args) != cudaSuccess) return QLORA_ERR_CUDA;
   return launch_status();
@@ -357,9 +381,8 @@ int tc_gemm(cudaStream_t st, DeviceInfo *dev, int64_t M, int64_t N, int nseg, co
   const int64_t count = M * W;
   const int grid = (int)std::min<int64_t>((count + 255) / 256, (int64_t)dev->sms * 8);
   ProfScope prof(QLORA_KERNEL_SPLITK_FINALIZE, st);
-  splitk_finalize_kernel<<<grid, 256, 0, st>>>(split_ws, splits, (int)M, (int)W, alpha, out, ld_row, ld_col, lo_off,
-                                               out_f32);
-  return launch_status();
+  return launch_pdl(splitk_finalize_kernel, dim3(grid), dim3(256), 0, st, (const float *)split_ws, splits, (int)M,
+                    (int)W, alpha, out, ld_row, ld_col, lo_off, out_f32);
 }
 
 int dequant_launch(const qlora_nf4dq_t *W, __nv_bfloat16 *out, cudaStream_t st, int sms) {
@@ -368,8 +391,8 @@ int dequant_launch(const qlora_nf4dq_t *W, __nv_bfloat16 *out, cudaStream_t st, 
   const int64_t n8 = numel >> 3;
   const int grid = (int)std::max<int64_t>(1, std::min<int64_t>((n8 + 255) / 256, (int64_t)sms * 16));
   ProfScope prof(QLORA_KERNEL_DEQUANT, st);
-  nf4_dequant_kernel<<<grid, 256, 0, st>>>(W->codes, W->c2_fp8, W->c1, W->c2_mean, numel, out);
-  return launch_status();
+  return launch_pdl(nf4_dequant_kernel, dim3(grid), dim3(256), 0, st, W->codes, W->c2_fp8, W->c1, W->c2_mean, numel,
+                    out);
 }
 
 int check_weight(const qlora_nf4dq_t *W) {
@@ -414,24 +437,6 @@ GemvLayout gemv_layout(int64_t M, int64_t N, int r) {
   L.zero_bytes = L.tacc + (size_t)M * r * 4;
   L.total = align_up(L.zero_bytes);
   return L;
-}
-
-// Launch `kernel` on `st` as a programmatic dependent of the previous launch.
-template <typename... KArgs, typename... Args>
-int launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, Args... args) {
-  cudaLaunchConfig_t cfg;
-  std::memset(&cfg, 0, sizeof(cfg));
-  cfg.gridDim = grid;
-  cfg.blockDim = block;
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, kernel, args...) != cudaSuccess) return QLORA_ERR_CUDA;
-  return launch_status();
 }
 
 // Y = bf16(acc + s T L2) and the T hi/lo pair, as a programmatic dependent of
@@ -749,19 +754,18 @@ int qlora_quantize_nf4_dq(const void *W, int w_dtype, int64_t n_out, int64_t k_i
   {
   ProfScope prof(QLORA_KERNEL_QUANTIZE, st);
   if (w_dtype == QLORA_DTYPE_F32)
-    nf4_quantize_kernel<float><<<grid1, kQuantThreads, 0, st>>>(reinterpret_cast<const float *>(W), numel, codes, c2,
-                                                               partial);
+    rc = launch_pdl(nf4_quantize_kernel<float>, dim3(grid1), dim3(kQuantThreads), 0, st,
+                    reinterpret_cast<const float *>(W), numel, codes, c2, partial);
   else
-    nf4_quantize_kernel<__nv_bfloat16><<<grid1, kQuantThreads, 0, st>>>(
-        reinterpret_cast<const __nv_bfloat16 *>(W), numel, codes, c2, partial);
+    rc = launch_pdl(nf4_quantize_kernel<__nv_bfloat16>, dim3(grid1), dim3(kQuantThreads), 0, st,
+                    reinterpret_cast<const __nv_bfloat16 *>(W), numel, codes, c2, partial);
   }
-  rc = launch_status();
   if (rc) return rc;
   const int64_t nb256 = (nblk + 255) / 256;
   const int grid2 = (int)std::max<int64_t>(1, std::min<int64_t>((nb256 + kDqWarps - 1) / kDqWarps, (int64_t)dev->sms * 4));
   ProfScope prof(QLORA_KERNEL_DQ_CONSTANTS, st);
-  dq_constants_kernel<<<grid2, 32 * kDqWarps, 0, st>>>(c2, nblk, partial, grid1, c2_fp8, c1, c2_mean);
-  return launch_status();
+  return launch_pdl(dq_constants_kernel, dim3(grid2), dim3(32 * kDqWarps), 0, st, (const float *)c2, nblk,
+                    (const double *)partial, grid1, c2_fp8, c1, c2_mean);
 }
 
 int qlora_quantize_nf4_dq_noalloc(const void *W, int w_dtype, int64_t n_out, int64_t k_in, uint8_t *codes,
@@ -788,17 +792,16 @@ int qlora_quantize_nf4_dq_noalloc(const void *W, int w_dtype, int64_t n_out, int
   const int64_t ngroups = numel >> 9;   // 512-element groups, one per warp iteration
   const int grid1 = (int)std::max<int64_t>(1, std::min<int64_t>((ngroups + 7) / 8, std::min(kQuantMaxCtas, dev->sms * kQuantCtasPerSm)));
   if (w_dtype == QLORA_DTYPE_F32)
-    nf4_quantize_kernel<float><<<grid1, kQuantThreads, 0, st>>>(reinterpret_cast<const float *>(W), numel, codes, c2,
-                                                               partial);
+    rc = launch_pdl(nf4_quantize_kernel<float>, dim3(grid1), dim3(kQuantThreads), 0, st,
+                    reinterpret_cast<const float *>(W), numel, codes, c2, partial);
   else
-    nf4_quantize_kernel<__nv_bfloat16><<<grid1, kQuantThreads, 0, st>>>(
-        reinterpret_cast<const __nv_bfloat16 *>(W), numel, codes, c2, partial);
-  rc = launch_status();
+    rc = launch_pdl(nf4_quantize_kernel<__nv_bfloat16>, dim3(grid1), dim3(kQuantThreads), 0, st,
+                    reinterpret_cast<const __nv_bfloat16 *>(W), numel, codes, c2, partial);
   if (rc) return rc;
   const int64_t nb256 = (nblk + 255) / 256;
   const int grid2 = (int)std::max<int64_t>(1, std::min<int64_t>((nb256 + kDqWarps - 1) / kDqWarps, (int64_t)dev->sms * 4));
-  dq_constants_kernel<<<grid2, 32 * kDqWarps, 0, st>>>(c2, nblk, partial, grid1, c2_fp8, c1, c2_mean);
-  return launch_status();
+  return launch_pdl(dq_constants_kernel, dim3(grid2), dim3(32 * kDqWarps), 0, st, (const float *)c2, nblk,
+                    (const double *)partial, grid1, c2_fp8, c1, c2_mean);
 }
 
 int qlora_dequant(const qlora_nf4dq_t *W, uint16_t *W_out, void *stream) {

@@ -165,7 +165,7 @@ struct Raw16<float> {
   float4 q[4];
   __device__ __forceinline__ void load(const float *__restrict__ p) {
 #pragma unroll
-    for (int i = 0; i < 4; ++i) q[i] = __ldg(reinterpret_cast<const float4 *>(p) + i);
+    for (int i = 0; i < 4; ++i) q[i] = ld_dep_f4(p + 4 * i);
   }
   __device__ __forceinline__ void unpack(float (&v)[16]) const {
 #pragma unroll
@@ -179,7 +179,7 @@ struct Raw16<__nv_bfloat16> {
   uint4 q[2];
   __device__ __forceinline__ void load(const __nv_bfloat16 *__restrict__ p) {
 #pragma unroll
-    for (int i = 0; i < 2; ++i) q[i] = __ldg(reinterpret_cast<const uint4 *>(p) + i);
+    for (int i = 0; i < 2; ++i) q[i] = ld_dep_v4(p + 8 * i);
   }
   __device__ __forceinline__ void unpack(float (&v)[16]) const {
 #pragma unroll
@@ -194,8 +194,8 @@ struct Raw16<__nv_bfloat16> {
   }
 };
 
-__device__ __forceinline__ float load1(const float *p) { return __ldg(p); }
-__device__ __forceinline__ float load1(const __nv_bfloat16 *p) { return __bfloat162float(*p); }
+__device__ __forceinline__ float load1(const float *p) { return ld_dep_f32(p); }
+__device__ __forceinline__ float load1(const __nv_bfloat16 *p) { return __uint_as_float(ld_dep_u16(p) << 16); }
 
 // Deterministic CTA-wide fp64 sum (fixed reduction tree).
 __device__ __forceinline__ double cta_sum_f64(double v, double *scratch) {
@@ -233,6 +233,8 @@ __global__ void __launch_bounds__(kQuantThreads, kQuantCtasPerSm) nf4_quantize_k
     thr[threadIdx.x] = __double2float_rd(((double)kNF4[threadIdx.x] + (double)kNF4[threadIdx.x + 1]) * 0.5);
   load_code_lut(lut);
   __syncthreads();
+  pdl_trigger();
+  pdl_wait();
   const int lane = lane_id();
   const int64_t ngroups = numel >> 9;
   const int64_t nwarps = (int64_t)gridDim.x * (kQuantThreads / 32);
@@ -344,8 +346,10 @@ __global__ void __launch_bounds__(32 * kDqWarps) dq_constants_kernel(const float
                                                                     float *__restrict__ c1, float *__restrict__ mu_out) {
   __shared__ double red[kDqWarps];
   __shared__ float mu_s;
+  pdl_trigger();
+  pdl_wait();
   double acc = 0.0;
-  for (int i = threadIdx.x; i < npartial; i += blockDim.x) acc += partial[i];
+  for (int i = threadIdx.x; i < npartial; i += blockDim.x) acc += ld_dep_f64(partial + i);
   const double total = cta_sum_f64(acc, red);
   if (threadIdx.x == 0) {
     mu_s = __double2float_rn(__ddiv_rn(total, (double)nblk));
@@ -360,14 +364,14 @@ __global__ void __launch_bounds__(32 * kDqWarps) dq_constants_kernel(const float
     const bool full = i0 + 8 <= nblk;
     float d[8];
     if (full) {
-      const float4 a = __ldg(reinterpret_cast<const float4 *>(c2 + i0));
-      const float4 b = __ldg(reinterpret_cast<const float4 *>(c2 + i0) + 1);
+      const float4 a = ld_dep_f4(c2 + i0);
+      const float4 b = ld_dep_f4(c2 + i0 + 4);
       const float x[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
 #pragma unroll
       for (int k = 0; k < 8; ++k) d[k] = __fsub_rn(x[k], mu);
     } else {
 #pragma unroll
-      for (int k = 0; k < 8; ++k) d[k] = i0 + k < nblk ? __fsub_rn(__ldg(c2 + i0 + k), mu) : 0.f;
+      for (int k = 0; k < 8; ++k) d[k] = i0 + k < nblk ? __fsub_rn(ld_dep_f32(c2 + i0 + k), mu) : 0.f;
     }
     float A = 0.f;
 #pragma unroll
@@ -403,13 +407,15 @@ __global__ void __launch_bounds__(256) nf4_dequant_kernel(const uint8_t *__restr
   __shared__ float lut[16];
   if (threadIdx.x < 16) lut[threadIdx.x] = kNF4[threadIdx.x];
   __syncthreads();
-  const float mu = __ldg(mu_p);
+  pdl_trigger();
+  pdl_wait();
+  const float mu = ld_dep_f32(mu_p);
   const int64_t n8 = numel >> 3;
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
   for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < n8; e += stride) {
-    const uint32_t q = __ldg(reinterpret_cast<const uint32_t *>(codes) + e);
+    const uint32_t q = ld_dep_u32(codes + 4 * e);
     const int64_t b = e >> 3;
-    const float c2h = __fmaf_rn(e4m3_to_f32(__ldg(c2_fp8 + b)), __ldg(c1 + (b >> 8)), mu);
+    const float c2h = __fmaf_rn(e4m3_to_f32((uint8_t)ld_dep_u8(c2_fp8 + b)), ld_dep_f32(c1 + (b >> 8)), mu);
     uint32_t o[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
@@ -423,8 +429,8 @@ __global__ void __launch_bounds__(256) nf4_dequant_kernel(const uint8_t *__restr
   if (blockIdx.x == 0 && threadIdx.x < (numel & 7)) {
     const int64_t i = (n8 << 3) + threadIdx.x;
     const int64_t b = i >> 6;
-    const float c2h = __fmaf_rn(e4m3_to_f32(c2_fp8[b]), c1[b >> 8], mu);
-    const uint32_t code = (codes[i >> 1] >> ((i & 1) * 4)) & 0xF;
+    const float c2h = __fmaf_rn(e4m3_to_f32((uint8_t)ld_dep_u8(c2_fp8 + b)), ld_dep_f32(c1 + (b >> 8)), mu);
+    const uint32_t code = (ld_dep_u8(codes + (i >> 1)) >> ((i & 1) * 4)) & 0xF;
     out[i] = __float2bfloat16_rn(__fmul_rn(lut[code], c2h));
   }
 }

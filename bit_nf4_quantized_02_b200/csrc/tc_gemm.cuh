@@ -199,6 +199,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   }
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  // Launched as a programmatic dependent: the set-up above overlapped the
+  // previous kernel; its results are visible after the wait.
+  pdl_trigger();
+  pdl_wait();
 
   const int units = p.m_tiles * p.n_tiles * p.splits;
 
@@ -511,10 +515,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 __global__ void __launch_bounds__(256) splitk_finalize_kernel(const float *__restrict__ part, int splits, int M,
                                                               int N, float alpha, void *dst, int64_t ld_row,
                                                               int64_t ld_col, int64_t lo_off, int dst_f32) {
+  pdl_trigger();
+  pdl_wait();
   const int64_t count = (int64_t)M * N;
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < count; i += (int64_t)gridDim.x * blockDim.x) {
     float s = 0.f;
-    for (int k = 0; k < splits; ++k) s += __ldg(part + (int64_t)k * count + i);
+    for (int k = 0; k < splits; ++k) s += ld_dep_f32(part + (int64_t)k * count + i);
     s *= alpha;
     const int64_t row = i / N, col = i - row * N;
     const int64_t off = row * ld_row + col * ld_col;
