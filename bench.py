@@ -281,27 +281,30 @@ def run_ours(args, rank, world, local_rank):
     if qlora.last_device_error() != 0:
         raise RuntimeError("device error during warm-up")
 
-    sampler = ClockSampler(list(range(world)) if world > 1 else [local_rank]) if rank == 0 else None
-    if world > 1:
-        torch.distributed.barrier()
+    # The per-launch event log (kernel table, roofline) comes from its own pass
+    # of the same steps on every rank, ahead of the timed pass: events between
+    # launches would serialise the programmatic dependent launches there.  A
+    # pause after it lets the GPU leave the power state the pass drove it to.
+    qlora.profile_start(args.steps * 200 * wl.layers + 64)
+    for _ in range(args.steps):
+        step()
     torch.cuda.synchronize()
+    launches = qlora.profile_stop()
+    time.sleep(1.0)
+
+    sampler = ClockSampler(list(range(world)) if world > 1 else [local_rank]) if rank == 0 else None
     if sampler:
         sampler.start()
         time.sleep(0.5)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record()
     for _ in range(args.steps):
         step()
     e1.record()
     torch.cuda.synchronize()
-    # The per-launch event log (kernel table, roofline) comes from a second
-    # pass of the same steps on every rank: events between launches would
-    # serialise the programmatic dependent launches of the timed pass.
-    qlora.profile_start(args.steps * 200 * wl.layers + 64)
-    for _ in range(args.steps):
-        step()
-    torch.cuda.synchronize()
-    launches = qlora.profile_stop()
     if world > 1:
         torch.distributed.barrier()
     clocks = sampler.stop() if sampler else None
@@ -403,22 +406,10 @@ def _timed(qlora, step, args, dev, world, rank, local_rank, profile=True):
     torch.cuda.synchronize()
     if qlora.last_device_error() != 0:
         raise RuntimeError("device error during warm-up")
-    sampler = ClockSampler([local_rank]) if rank == 0 else None
-    if world > 1:
-        torch.distributed.barrier()
-    torch.cuda.synchronize()
-    if sampler:
-        sampler.start()
-        time.sleep(0.5)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for _ in range(args.steps):
-        step()
-    e1.record()
-    torch.cuda.synchronize()
-    # The per-launch event log (kernel table, roofline) comes from a second
-    # pass of the same steps: events between launches would serialise the
-    # programmatic dependent launches of the timed pass.
+    # The per-launch event log (kernel table, roofline) comes from its own pass
+    # of the same steps, ahead of the timed pass: events between launches
+    # would serialise the programmatic dependent launches there.  A pause
+    # after it lets the GPU leave the power state the pass drove it to.
     launches = []
     if profile:
         qlora.profile_start(args.steps * 256 + 64)
@@ -426,6 +417,20 @@ def _timed(qlora, step, args, dev, world, rank, local_rank, profile=True):
             step()
         torch.cuda.synchronize()
         launches = qlora.profile_stop()
+        time.sleep(1.0)
+    sampler = ClockSampler([local_rank]) if rank == 0 else None
+    if sampler:
+        sampler.start()
+        time.sleep(0.5)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        step()
+    e1.record()
+    torch.cuda.synchronize()
     clocks = sampler.stop() if sampler else None
     ms = e0.elapsed_time(e1) / args.steps
     t = torch.tensor([ms], device=dev)

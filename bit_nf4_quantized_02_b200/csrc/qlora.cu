@@ -106,7 +106,9 @@ int launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cud
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  // While the per-launch event log records, the events between launches
+  // serialise them anyway; plain launches then time each kernel alone.
+  cfg.numAttrs = g_prof.on ? 0 : 1;
   if (cudaLaunchKernelEx(&cfg, kernel, args...) != cudaSuccess) return QLORA_ERR_CUDA;
   return launch_status();
 }
@@ -284,7 +286,7 @@ int launch_gemm_pair(const CUtensorMap *maps, TcGemmArgs &args, DeviceInfo *dev,
   const int units = args.m_tiles * args.n_tiles * args.splits;
   const int clusters = std::max(1, std::min(units, dev->pair_clusters[WIDE ? 1 : 0]));
   cfg.gridDim = dim3(2 * (unsigned)clusters, 1, 1);
-  cfg.numAttrs = 2;   // launched as a programmatic dependent of the previous kernel
+  cfg.numAttrs = g_prof.on ? 1 : 2;   // a programmatic dependent of the previous kernel, unless the event log records
   ProfScope prof(kind, st);
   if (cudaLaunchKernelEx(&cfg, kernel, maps[0], maps[1], maps[2], maps[3], args) != cudaSuccess) return QLORA_ERR_CUDA;
   return launch_status();
