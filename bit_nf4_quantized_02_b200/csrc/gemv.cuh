@@ -51,7 +51,10 @@ struct GvCfg {
   static constexpr int kCodeBytes = kGvRows * 128;          // 64 rows x 256 codes
   static constexpr int kXBytes = 8 * NT * kGvStageK * 2;    // padded tokens x 256 bf16
   static constexpr int kStageBytes = kCodeBytes + kXBytes;
-  static constexpr int kStages = NT == 1 ? 5 : (NT == 2 ? 4 : 3);   // ~64 KB: 3 CTAs per SM
+  // 4 CTAs per SM (at most 48 KB and 96 registers each) up to 16 tokens; at
+  // 32 tokens the register cap would spill, so 3 CTAs of 72 KB.
+  static constexpr int kCtasPerSm = NT == 4 ? 3 : 4;
+  static constexpr int kStages = NT == 1 ? 4 : 3;
   // + 1024 alignment slack + 256 barrier area
   static constexpr int kSmemBytes = kStages * kStageBytes + 1024 + 256;
 };
@@ -286,7 +289,7 @@ struct GvConsumer {
 };
 
 template <int NT>
-__global__ void __launch_bounds__(kGvThreads, 3)
+__global__ void __launch_bounds__(kGvThreads, GvCfg<NT>::kCtasPerSm)
     gemv_fwd_kernel(const __grid_constant__ CUtensorMap tmCodes, const __grid_constant__ CUtensorMap tmX,
                     const __grid_constant__ GvArgs p) {
   using Cfg = GvCfg<NT>;
