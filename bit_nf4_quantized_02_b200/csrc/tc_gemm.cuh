@@ -114,7 +114,9 @@ __device__ __forceinline__ void tc_unit_coords(int u, const TcGemmArgs &p, int &
   const int tiles = p.m_tiles * p.n_tiles;
   split = u / tiles;
   const int t = u - split * tiles;
-  constexpr int kGroupM = 8;  // sweep 8 M-tiles across all N-tiles: B panels stay in L2
+  // sweep 16 M-tiles across all N-tiles: B panels stay in L2 (8 re-read them
+  // from DRAM twice as often; 32 let the A panels crowd L2: both slower)
+  constexpr int kGroupM = 16;
   const int per_group = kGroupM * p.n_tiles;
   const int group = t / per_group;
   const int first_m = group * kGroupM;
