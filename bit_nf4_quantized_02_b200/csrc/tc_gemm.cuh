@@ -3,12 +3,15 @@
 //   D[M x N] = alpha * sum_seg A_seg[M x K_seg] * B_seg[N x K_seg]^T
 //
 // One kernel, warp-specialised, one CTA per SM (or one CTA pair per two SMs):
-//   warp 0        TMA producer: 128-byte-swizzled tiles of A and B into a ring
-//                 of shared-memory stages (mbarrier full/empty pairs);
+//   warps 0, 6    TMA producers of A and of B: 128-byte-swizzled tiles into a
+//                 ring of shared-memory stages (mbarrier full/empty pairs);
+//                 a stage holds one or (WIDE) two 64-wide k-blocks;
 //   warp 1        allocates TMEM, one thread issues tcgen05.mma (bf16 in, fp32
 //                 accumulate) into one of two TMEM accumulators;
 //   warps 2..5    epilogue: tcgen05.ld the accumulator, scale, convert, store;
 //                 the second accumulator lets the next tile's MMAs overlap.
+// It is launched as a programmatic dependent: the set-up (barriers, TMEM)
+// overlaps the previous kernel, and every role starts after pdl_wait().
 // Each segment has its own operand major-ness (K-major = contiguous along the
 // reduction; MN-major = contiguous along the output rows/columns), selected
 // per MMA through the instruction descriptor, so X*W^T, dY*W (W read in its

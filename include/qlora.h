@@ -24,7 +24,10 @@
  *     outputs are valid once the stream has reached that point.  The one
  *     exception is the first call on a device: it fills a constant table of
  *     the quantizer (a function of the NF4 levels only) and waits for the
- *     device once.
+ *     device once.  The kernels are launched as programmatic dependents of
+ *     the kernel before them in the stream (they may start their set-up
+ *     while it finishes) and wait for it before touching any memory, so the
+ *     ordering is that of plain stream order.
  *   - bfloat16 data is passed as uint16_t bit patterns.
  *   - Alignment: every device pointer must be 16-byte aligned (W->c2_mean and
  *     c2_mean only need 4 bytes).
