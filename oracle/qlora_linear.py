@@ -75,3 +75,41 @@ def adapter_grads(dY, X, L1, L2, s: float):
     dL2 = s * ((X @ L1).T @ dY)
     dL1 = X.T @ G
     return dL1, dL2
+
+
+# --------------------------------------------------------------------------- LoRA dropout
+# QLoRA Appendix B.2 trains with LoRA dropout (0.1 up to 13B, 0.05 at 33B and
+# 65B).  The pages do not say where it acts; the reading taken is the usual
+# LoRA one: on the adapter's input only,
+#     Y = X W_hat^T + s (drop(X) L1) L2,   drop(X) = X * m / (1 - p),
+# with m a 0/1 keep mask drawn once per step and passed in (it is an input,
+# not drawn here).  The base product sees X unchanged.
+
+def dropped(X, mask, p: float) -> np.ndarray:
+    """drop(X) = X * m / (1 - p) in float64; mask is a 0/1 (or bool) array shaped like X."""
+    return _f64(X) * _f64(mask) / (1.0 - p)
+
+
+def forward_dropout(X, W_hat, L1, L2, s: float, mask, p: float):
+    """Forward with LoRA dropout.  Returns (Y [M, N], T [M, r]) with T = s drop(X) L1."""
+    X, W_hat, L1, L2 = map(_f64, (X, W_hat, L1, L2))
+    T = s * (dropped(X, mask, p) @ L1)
+    Y = X @ W_hat.T + T @ L2
+    return Y, T
+
+
+def backward_dropout(dY, X, W_hat, L1, L2, s: float, mask, p: float):
+    """Adapter-only backward of ``forward_dropout`` (no dW).
+
+    G   = s dY L2^T                          [M, r]
+    dX  = dY W_hat + (G L1^T) * m / (1 - p)  [M, K]  (the mask gates only the adapter path)
+    dL2 = T^T dY, T = s drop(X) L1           [r, N]
+    dL1 = drop(X)^T G                        [K, r]
+    """
+    dY, X, W_hat, L1, L2 = map(_f64, (dY, X, W_hat, L1, L2))
+    Xd = dropped(X, mask, p)
+    G = s * (dY @ L2.T)
+    dX = dY @ W_hat + (G @ L1.T) * _f64(mask) / (1.0 - p)
+    dL2 = (s * (Xd @ L1)).T @ dY
+    dL1 = Xd.T @ G
+    return dX, dL1, dL2

@@ -80,3 +80,26 @@ def device_weight_with_outliers(n_out: int, k_in: int, seed: int, device,
     sign = torch.where(torch.rand(n_out_lier, generator=gen, device=device) < 0.5, -1.0, 1.0)
     w[pos] = sign * (sigmas * std)
     return w.view(n_out, k_in).to(torch.bfloat16)
+
+
+def dropout_mask(g: np.random.Generator, M: int, K: int, p: float) -> np.ndarray:
+    """Keep mask of LoRA dropout, bit-packed: uint32 [M, K/32], bit b of word w
+    of row i keeps element (i, 32 w + b); each element is kept with
+    probability 1 - p, independently.  K must be a multiple of 32."""
+    if K % 32:
+        raise ValueError("K must be a multiple of 32")
+    keep = g.random((M, K), dtype=np.float32) >= np.float32(p)
+    return pack_mask(keep)
+
+
+def pack_mask(keep: np.ndarray) -> np.ndarray:
+    """bool [M, K] -> uint32 [M, K/32] (element 32 w + b in bit b of word w)."""
+    M, K = keep.shape
+    bits = keep.reshape(M, K // 32, 32).astype(np.uint64) << np.arange(32, dtype=np.uint64)
+    return bits.sum(axis=-1).astype(np.uint32)
+
+
+def unpack_mask(words: np.ndarray, K: int) -> np.ndarray:
+    """uint32 [M, K/32] -> bool [M, K], the inverse of pack_mask."""
+    w = np.asarray(words, dtype=np.uint32)
+    return ((w[:, :, None] >> np.arange(32, dtype=np.uint32)) & 1).astype(bool).reshape(w.shape[0], K)
