@@ -154,12 +154,24 @@ class _Workspace:
 _WS = _Workspace()
 
 
+def _mask_arg(mask: torch.Tensor, M: int, K: int, dev) -> torch.Tensor:
+    """Check a LoRA-dropout keep mask: int32/uint32 words [M, K/32] on ``dev``."""
+    if mask.device != torch.device(dev) or mask.dtype not in (torch.int32, torch.uint32) or \
+            tuple(mask.shape) != (M, K // 32) or not mask.is_contiguous():
+        raise ValueError("qlora: dropout mask must be contiguous 32-bit words [M, K/32] on the device")
+    return mask
+
+
 def linear_fwd(X: torch.Tensor, q: NF4Tensor, L1: torch.Tensor, L2: torch.Tensor, s: float,
-               save_T: bool = True, Y: torch.Tensor | None = None, T: torch.Tensor | None = None):
+               save_T: bool = True, Y: torch.Tensor | None = None, T: torch.Tensor | None = None,
+               dropout_mask: torch.Tensor | None = None, dropout_p: float = 0.0):
     """Y = X doubleDequant(W)^T + s X L1 L2 (Eq. 3 / Eq. 5).  Returns (Y, T or None).
 
     X [M, K] bf16, L1 [K, r] bf16, L2 [r, N] bf16.  T [M, 2r] bf16 holds
     T = s X L1 as a hi/lo pair: T ~= T[:, :r] + T[:, r:] (see ``t_value``).
+    With ``dropout_mask`` (keep bits, 32-bit words [M, K/32], element 32 w + b
+    in bit b of word w) LoRA dropout acts on the adapter input:
+    T = s (X * m / (1 - dropout_p)) L1.
     """
     lib = _lib.load()
     M, K = X.shape
@@ -172,6 +184,14 @@ def linear_fwd(X: torch.Tensor, q: NF4Tensor, L1: torch.Tensor, L2: torch.Tensor
         Y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
     if save_T and T is None:
         T = torch.empty((M, 2 * r), dtype=torch.bfloat16, device=dev)
+    if dropout_mask is not None:
+        _mask_arg(dropout_mask, M, K, dev)
+        ws = _WS.get(lib.qlora_linear_fwd_dropout_workspace_size(M, N, K, r), dev)
+        _lib.check(lib.qlora_linear_fwd_dropout(_ptr(_bits(X)), M, q.as_struct(), _ptr(_bits(L1)), _ptr(_bits(L2)), r,
+                                                float(s), _ptr(dropout_mask), float(dropout_p), _ptr(_bits(Y)),
+                                                _ptr(T) if save_T else None, _ptr(ws), ws.numel(), _stream(dev)),
+                   "qlora_linear_fwd_dropout")
+        return Y, (T if save_T else None)
     ws_bytes = lib.qlora_linear_fwd_workspace_size(M, N, K, r)
     ws = _WS.get(ws_bytes, dev)
     _lib.check(lib.qlora_linear_fwd(_ptr(_bits(X)), M, q.as_struct(), _ptr(_bits(L1)), _ptr(_bits(L2)), r, float(s),
@@ -188,8 +208,13 @@ def t_value(T: torch.Tensor) -> torch.Tensor:
 
 def linear_bwd(dY: torch.Tensor, X: torch.Tensor, T: torch.Tensor | None, q: NF4Tensor, L1: torch.Tensor,
                L2: torch.Tensor, s: float, need_dX: bool = True, grad_dtype=torch.bfloat16,
-               dX: torch.Tensor | None = None, dL1: torch.Tensor | None = None, dL2: torch.Tensor | None = None):
-    """Adapter-only backward.  Returns (dX or None, dL1 [K, r], dL2 [r, N])."""
+               dX: torch.Tensor | None = None, dL1: torch.Tensor | None = None, dL2: torch.Tensor | None = None,
+               dropout_mask: torch.Tensor | None = None, dropout_p: float = 0.0):
+    """Adapter-only backward.  Returns (dX or None, dL1 [K, r], dL2 [r, N]).
+
+    With ``dropout_mask`` (the forward's mask) the adapter path goes through
+    the mask: dX = dY W_hat + (G L1^T) m / (1 - p), dL1 = drop(X)^T G.
+    """
     lib = _lib.load()
     M, N = dY.shape
     K = q.k_in
@@ -209,6 +234,15 @@ def linear_bwd(dY: torch.Tensor, X: torch.Tensor, T: torch.Tensor | None, q: NF4
         dL1 = torch.empty((K, r), dtype=grad_dtype, device=dev)
     if dL2 is None:
         dL2 = torch.empty((r, N), dtype=grad_dtype, device=dev)
+    if dropout_mask is not None:
+        _mask_arg(dropout_mask, M, K, dev)
+        ws = _WS.get(lib.qlora_linear_bwd_dropout_workspace_size(M, N, K, r), dev)
+        _lib.check(lib.qlora_linear_bwd_dropout(_ptr(_bits(dY)), _ptr(_bits(X)), _ptr(T), M, q.as_struct(),
+                                                _ptr(_bits(L1)), _ptr(_bits(L2)), r, float(s), _ptr(dropout_mask),
+                                                float(dropout_p), _ptr(dX) if need_dX else None, _ptr(dL1),
+                                                _ptr(dL2), gdt, _ptr(ws), ws.numel(), _stream(dev)),
+                   "qlora_linear_bwd_dropout")
+        return (dX if need_dX else None), dL1, dL2
     ws_bytes = lib.qlora_linear_bwd_workspace_size(M, N, K, r)
     ws = _WS.get(ws_bytes, dev)
     _lib.check(lib.qlora_linear_bwd(_ptr(_bits(dY)), _ptr(_bits(X)), _ptr(T), M, q.as_struct(), _ptr(_bits(L1)),

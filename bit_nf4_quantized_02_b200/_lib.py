@@ -28,8 +28,8 @@ QLORA_MAX_RANK = 256
 
 KERNEL_KINDS = {
     1: "quantize", 2: "dq_constants", 3: "dequant",
-    10: "gemm_T", 11: "gemm_Y", 12: "gemm_G", 13: "gemm_dX", 14: "gemm_dL2", 15: "gemm_dL1",
-    20: "splitk_finalize", 30: "gemv_fwd", 31: "fused_fwd",
+    10: "gemm_T", 11: "gemm_Y", 12: "gemm_G", 13: "gemm_dX", 14: "gemm_dL2", 15: "gemm_dL1", 16: "gemm_Z",
+    20: "splitk_finalize", 30: "gemv_fwd", 31: "fused_fwd", 40: "dropout_mask",
 }
 
 
@@ -66,6 +66,13 @@ SIGNATURES = {
                                  c_void_p, c_void_p, c_size_t, c_void_p]),
     "qlora_linear_bwd": (c_int, [c_void_p, c_void_p, c_void_p, c_int64, POINTER(NF4DQ), c_void_p, c_void_p, c_int,
                                  c_float, c_void_p, c_void_p, c_void_p, c_int, c_void_p, c_size_t, c_void_p]),
+    "qlora_linear_fwd_dropout_workspace_size": (c_size_t, [c_int64, c_int64, c_int64, c_int]),
+    "qlora_linear_bwd_dropout_workspace_size": (c_size_t, [c_int64, c_int64, c_int64, c_int]),
+    "qlora_linear_fwd_dropout": (c_int, [c_void_p, c_int64, POINTER(NF4DQ), c_void_p, c_void_p, c_int, c_float,
+                                         c_void_p, c_float, c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]),
+    "qlora_linear_bwd_dropout": (c_int, [c_void_p, c_void_p, c_void_p, c_int64, POINTER(NF4DQ), c_void_p, c_void_p,
+                                         c_int, c_float, c_void_p, c_float, c_void_p, c_void_p, c_void_p, c_int,
+                                         c_void_p, c_size_t, c_void_p]),
 }
 
 _lib = None

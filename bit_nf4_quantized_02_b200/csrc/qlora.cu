@@ -13,6 +13,7 @@
 #include "tc_gemm.cuh"
 #include "gemv.cuh"
 #include "fused_fwd.cuh"
+#include "dropout.cuh"
 
 namespace qlora {
 
@@ -202,6 +203,14 @@ struct GemmSeg {
   Operand A, B;   // A.kext == B.kext
 };
 
+// Masked addend of a bf16 GEMM output (see TcGemmArgs::add).
+struct GemmAddend {
+  const uint16_t *z;
+  const uint32_t *mask;
+  float scale;
+  int64_t ld;
+};
+
 int pick_bn(int64_t N) { return N <= 64 ? 64 : (N <= 128 ? 128 : 256); }
 
 // Split-K factor for a single-segment product whose tile grid leaves SMs idle:
@@ -303,8 +312,10 @@ bool use_pair(int bn, int splits, int64_t M) { return bn == 256 && splits == 1 &
 // partials go to split_ws and a finalize pass sums them in a fixed order.
 int tc_gemm(cudaStream_t st, DeviceInfo *dev, int64_t M, int64_t N, int nseg, const GemmSeg *segs, float alpha,
             void *out, int64_t ld_row, int64_t ld_col, int out_f32, float *split_ws, int kind, int64_t lo_off = 0,
-            bool split_all = false, int fold = 0) {
+            bool split_all = false, int fold = 0, const GemmAddend *add = nullptr) {
   if (M <= 0 || N <= 0) return QLORA_OK;
+  // the addend is applied by the direct bf16 epilogue only
+  if (add && (split_ws || out_f32 || fold || N % 32)) return QLORA_ERR_UNSUPPORTED_SHAPE;
   if (M > (int64_t)INT32_MAX / 2 || N > (int64_t)INT32_MAX / 2) return QLORA_ERR_UNSUPPORTED_SHAPE;
   const int bn = pick_bn(N);
   CUtensorMap maps[4];
@@ -349,6 +360,12 @@ int tc_gemm(cudaStream_t st, DeviceInfo *dev, int64_t M, int64_t N, int nseg, co
   a.ld_col = ld_col;
   a.lo_off = lo_off;
   a.fold = fold;
+  if (add) {
+    a.add = add->z;
+    a.add_mask = add->mask;
+    a.add_scale = add->scale;
+    a.add_ld = add->ld;
+  }
   if (splits > 1) {
     a.alpha = 1.f;
     a.out = split_ws;
@@ -820,6 +837,120 @@ int qlora_dequant(const qlora_nf4dq_t *W, uint16_t *W_out, void *stream) {
                         dev->sms);
 }
 
+}  // extern "C"
+
+namespace {
+
+// Forward above the few-token sizes: dequant + tcgen05 GEMMs.  The adapter's
+// down-projection reads Xt with scale t_scale: T = t_scale Xt L1 (Xt = X and
+// t_scale = s without dropout).
+int fwd_large(const uint16_t *X, const uint16_t *Xt, float t_scale, int64_t M, const qlora_nf4dq_t *W,
+              const uint16_t *L1, const uint16_t *L2, int r, uint16_t *Y, uint16_t *T_save, uint8_t *w8,
+              const FwdLayout &L, DeviceInfo *dev, cudaStream_t st) {
+  const int64_t N = W->n_out, K = W->k_in;
+  __nv_bfloat16 *w_hat = reinterpret_cast<__nv_bfloat16 *>(w8 + L.w_hat);
+  uint16_t *T = T_save ? T_save : reinterpret_cast<uint16_t *>(w8 + L.t);
+  float *split_ws = reinterpret_cast<float *>(w8 + L.split);
+  // 1. doubleDequant of the frozen weight into the bf16 workspace (Eq. 6).
+  int rc = dequant_launch(W, w_hat, st, dev->sms);
+  if (rc) return rc;
+  // 2. T = s X L1 (the adapter's down-projection; L1 read MN-major), stored
+  //    as a bf16 hi/lo pair [M x 2r]: T ~= T[:, :r] + T[:, r:].
+  GemmSeg sT = {{Xt, M, K, K, 0}, {L1, r, K, r, 1}};
+  rc = tc_gemm(st, dev, M, r, 1, &sT, t_scale, T, 2 * r, 1, 0, split_ws, QLORA_KERNEL_GEMM_T, r);
+  if (rc) return rc;
+  // 3. Y = X W_hat^T + T_hi L2 (the LoRA up-projection as extra K-steps).
+  GemmSeg sY[2] = {{{X, M, K, K, 0}, {w_hat, N, K, K, 0}}, {{T, M, r, 2 * r, 0}, {L2, N, r, N, 1}}};
+  return tc_gemm(st, dev, M, N, 2, sY, 1.f, Y, N, 1, 0, nullptr, QLORA_KERNEL_GEMM_Y);
+}
+
+// Dropout state of a backward: the adapter reads Xt (the masked input) with
+// its scales multiplied by keep = 1/(1 - p), and dX's adapter term goes
+// through the mask via Z = G_hi L1^T, added in the dX epilogue.
+struct BwdDropout {
+  const uint16_t *Xt;
+  float keep;
+  const uint32_t *mask;
+  uint16_t *Z;   // [M x K] workspace
+};
+
+int bwd_large(const uint16_t *dY, const uint16_t *X, const uint16_t *T_saved, int64_t M, const qlora_nf4dq_t *W,
+              const uint16_t *L1, const uint16_t *L2, int r, float s, uint16_t *dX, void *dL1, void *dL2,
+              int out_f32, uint8_t *w8, const BwdLayout &L, const BwdDropout *drop, DeviceInfo *dev,
+              cudaStream_t st) {
+  const int64_t N = W->n_out, K = W->k_in;
+  __nv_bfloat16 *w_hat = reinterpret_cast<__nv_bfloat16 *>(w8 + L.w_hat);
+  uint16_t *G = reinterpret_cast<uint16_t *>(w8 + L.g);
+  float *split_ws = reinterpret_cast<float *>(w8 + L.split);
+  const uint16_t *Xt = drop ? drop->Xt : X;        // what the adapter reads
+  const float keep = drop ? drop->keep : 1.f;
+  const uint16_t *T = T_saved;
+  int rc;
+  if (!T) {  // recompute T = s X L1 (hi/lo pair)
+    uint16_t *Tw = reinterpret_cast<uint16_t *>(w8 + L.t);
+    GemmSeg sT = {{Xt, M, K, K, 0}, {L1, r, K, r, 1}};
+    rc = tc_gemm(st, dev, M, r, 1, &sT, s * keep, Tw, 2 * r, 1, 0, split_ws, QLORA_KERNEL_GEMM_T, r);
+    if (rc) return rc;
+    T = Tw;
+  }
+  // G = s dY L2^T (L2 [r x N] is K-major for this product), as a hi/lo pair.
+  GemmSeg sG = {{dY, M, N, N, 0}, {L2, r, N, N, 0}};
+  rc = tc_gemm(st, dev, M, r, 1, &sG, s, G, 2 * r, 1, 0, split_ws, QLORA_KERNEL_GEMM_G, r);
+  if (rc) return rc;
+  if (dX) {
+    // dX = dY W_hat + G_hi L1^T: W_hat [N x K] is read in place as an MN-major B.
+    rc = dequant_launch(W, w_hat, st, dev->sms);
+    if (rc) return rc;
+    if (!drop) {
+      GemmSeg sX[2] = {{{dY, M, N, N, 0}, {w_hat, K, N, K, 1}}, {{G, M, r, 2 * r, 0}, {L1, K, r, r, 0}}};
+      rc = tc_gemm(st, dev, M, K, 2, sX, 1.f, dX, K, 1, 0, nullptr, QLORA_KERNEL_GEMM_DX);
+    } else {
+      // With dropout the adapter term is gated by the mask: Z = G_hi L1^T
+      // first, then dX = dY W_hat + keep * m * Z, added before the rounding.
+      GemmSeg sZ = {{G, M, r, 2 * r, 0}, {L1, K, r, r, 0}};
+      rc = tc_gemm(st, dev, M, K, 1, &sZ, 1.f, drop->Z, K, 1, 0, nullptr, QLORA_KERNEL_GEMM_Z);
+      if (rc) return rc;
+      GemmSeg sX = {{dY, M, N, N, 0}, {w_hat, K, N, K, 1}};
+      const GemmAddend add = {drop->Z, drop->mask, keep, K};
+      rc = tc_gemm(st, dev, M, K, 1, &sX, 1.f, dX, K, 1, 0, nullptr, QLORA_KERNEL_GEMM_DX, 0, false, 0, &add);
+    }
+    if (rc) return rc;
+  }
+  // dL2 = T^T dY as dL2^T [N x r] = dY^T (T_hi + T_lo), written transposed,
+  // and dL1 = Xt^T (G_hi + G_lo) [K x r] (times keep).  When both halves fit
+  // one tile the product runs against the whole [hi | lo] pair (2r columns)
+  // and the epilogue adds the halves, so dY and X stream once; otherwise as
+  // two accumulated segments over the tokens.
+  if (can_fold(r)) {
+    GemmSeg s2 = {{dY, N, M, N, 1}, {T, 2 * r, M, 2 * r, 1}};
+    rc = tc_gemm(st, dev, N, 2 * r, 1, &s2, 1.f, dL2, 1, N, out_f32, split_ws, QLORA_KERNEL_GEMM_DL2, 0, false, r);
+    if (rc) return rc;
+    GemmSeg s1 = {{Xt, K, M, K, 1}, {G, 2 * r, M, 2 * r, 1}};
+    return tc_gemm(st, dev, K, 2 * r, 1, &s1, keep, dL1, r, 1, out_f32, split_ws, QLORA_KERNEL_GEMM_DL1, 0, false, r);
+  }
+  const uint16_t *T_lo = T + r;
+  GemmSeg s2[2] = {{{dY, N, M, N, 1}, {T, r, M, 2 * r, 1}}, {{dY, N, M, N, 1}, {T_lo, r, M, 2 * r, 1}}};
+  rc = tc_gemm(st, dev, N, r, 2, s2, 1.f, dL2, 1, N, out_f32, split_ws, QLORA_KERNEL_GEMM_DL2, 0, true);
+  if (rc) return rc;
+  const uint16_t *G_lo = G + r;
+  GemmSeg s1[2] = {{{Xt, K, M, K, 1}, {G, r, M, 2 * r, 1}}, {{Xt, K, M, K, 1}, {G_lo, r, M, 2 * r, 1}}};
+  return tc_gemm(st, dev, K, r, 2, s1, keep, dL1, r, 1, out_f32, split_ws, QLORA_KERNEL_GEMM_DL1, 0, true);
+}
+
+// Xm = X * m into the workspace.
+int dropout_launch(const uint16_t *X, const uint32_t *mask, int64_t numel, uint16_t *Xm, DeviceInfo *dev,
+                   cudaStream_t st) {
+  if (numel == 0) return QLORA_OK;
+  const int64_t n8 = numel >> 3;
+  const int grid = (int)std::max<int64_t>(1, std::min<int64_t>((n8 + 255) / 256, (int64_t)dev->sms * 16));
+  ProfScope prof(QLORA_KERNEL_DROPOUT_MASK, st);
+  return launch_pdl(dropout_mask_kernel, dim3(grid), dim3(256), 0, st, X, mask, numel, Xm);
+}
+
+}  // namespace
+
+extern "C" {
+
 size_t qlora_linear_fwd_workspace_size(int64_t M, int64_t n_out, int64_t k_in, int r) {
   if (M < 0 || n_out <= 0 || k_in <= 0 || r <= 0) return 0;
   if (M <= kFtMaxM) return gemv_layout(M, n_out, r).total;
@@ -864,22 +995,7 @@ int qlora_linear_fwd(const uint16_t *X, int64_t M, const qlora_nf4dq_t *W, const
   const FwdLayout L = fwd_layout(M, N, K, r, dev->sms);
   if (!ws || ws_bytes < L.total) return QLORA_ERR_WORKSPACE;
   if (!aligned(ws, 256)) return QLORA_ERR_MISALIGNED;
-  uint8_t *w8 = reinterpret_cast<uint8_t *>(ws);
-  __nv_bfloat16 *w_hat = reinterpret_cast<__nv_bfloat16 *>(w8 + L.w_hat);
-  uint16_t *T = T_save ? T_save : reinterpret_cast<uint16_t *>(w8 + L.t);
-  float *split_ws = reinterpret_cast<float *>(w8 + L.split);
-
-  // 1. doubleDequant of the frozen weight into the bf16 workspace (Eq. 6).
-  rc = dequant_launch(W, w_hat, st, dev->sms);
-  if (rc) return rc;
-  // 2. T = s X L1 (the adapter's down-projection; L1 read MN-major), stored
-  //    as a bf16 hi/lo pair [M x 2r]: T ~= T[:, :r] + T[:, r:].
-  GemmSeg sT = {{X, M, K, K, 0}, {L1, r, K, r, 1}};
-  rc = tc_gemm(st, dev, M, r, 1, &sT, s, T, 2 * r, 1, 0, split_ws, QLORA_KERNEL_GEMM_T, r);
-  if (rc) return rc;
-  // 3. Y = X W_hat^T + T_hi L2 (the LoRA up-projection as extra K-steps).
-  GemmSeg sY[2] = {{{X, M, K, K, 0}, {w_hat, N, K, K, 0}}, {{T, M, r, 2 * r, 0}, {L2, N, r, N, 1}}};
-  return tc_gemm(st, dev, M, N, 2, sY, 1.f, Y, N, 1, 0, nullptr, QLORA_KERNEL_GEMM_Y);
+  return fwd_large(X, X, s, M, W, L1, L2, r, Y, T_save, reinterpret_cast<uint8_t *>(ws), L, dev, st);
 }
 
 int qlora_linear_bwd(const uint16_t *dY, const uint16_t *X, const uint16_t *T_saved, int64_t M,
@@ -907,51 +1023,89 @@ int qlora_linear_bwd(const uint16_t *dY, const uint16_t *X, const uint16_t *T_sa
   const BwdLayout L = bwd_layout(M, N, K, r, dev->sms);
   if (!ws || ws_bytes < L.total) return QLORA_ERR_WORKSPACE;
   if (!aligned(ws, 256)) return QLORA_ERR_MISALIGNED;
-  uint8_t *w8 = reinterpret_cast<uint8_t *>(ws);
-  __nv_bfloat16 *w_hat = reinterpret_cast<__nv_bfloat16 *>(w8 + L.w_hat);
-  uint16_t *G = reinterpret_cast<uint16_t *>(w8 + L.g);
-  float *split_ws = reinterpret_cast<float *>(w8 + L.split);
-  const uint16_t *T = T_saved;
-  const int out_f32 = grad_dtype == QLORA_DTYPE_F32;
+  return bwd_large(dY, X, T_saved, M, W, L1, L2, r, s, dX, dL1, dL2, grad_dtype == QLORA_DTYPE_F32,
+                   reinterpret_cast<uint8_t *>(ws), L, nullptr, dev, st);
+}
 
-  if (!T) {  // recompute T = s X L1 (hi/lo pair)
-    uint16_t *Tw = reinterpret_cast<uint16_t *>(w8 + L.t);
-    GemmSeg sT = {{X, M, K, K, 0}, {L1, r, K, r, 1}};
-    rc = tc_gemm(st, dev, M, r, 1, &sT, s, Tw, 2 * r, 1, 0, split_ws, QLORA_KERNEL_GEMM_T, r);
-    if (rc) return rc;
-    T = Tw;
-  }
-  // G = s dY L2^T (L2 [r x N] is K-major for this product), as a hi/lo pair.
-  GemmSeg sG = {{dY, M, N, N, 0}, {L2, r, N, N, 0}};
-  rc = tc_gemm(st, dev, M, r, 1, &sG, s, G, 2 * r, 1, 0, split_ws, QLORA_KERNEL_GEMM_G, r);
+// ---------------------------------------------------------------- LoRA dropout
+// Workspace: the plain large-M layout, then Xm [M x K] bf16 (and, backward,
+// Z [M x K] bf16).
+size_t qlora_linear_fwd_dropout_workspace_size(int64_t M, int64_t n_out, int64_t k_in, int r) {
+  if (M < 0 || n_out <= 0 || k_in <= 0 || r <= 0) return 0;
+  DeviceInfo *dev;
+  const int sms = current_device_info(&dev) == QLORA_OK ? dev->sms : 148;
+  return fwd_layout(M, n_out, k_in, r, sms).total + align_up((size_t)M * k_in * 2);
+}
+
+size_t qlora_linear_bwd_dropout_workspace_size(int64_t M, int64_t n_out, int64_t k_in, int r) {
+  if (M < 0 || n_out <= 0 || k_in <= 0 || r <= 0) return 0;
+  DeviceInfo *dev;
+  const int sms = current_device_info(&dev) == QLORA_OK ? dev->sms : 148;
+  return bwd_layout(M, n_out, k_in, r, sms).total + 2 * align_up((size_t)M * k_in * 2);
+}
+
+int qlora_linear_fwd_dropout(const uint16_t *X, int64_t M, const qlora_nf4dq_t *W, const uint16_t *L1,
+                             const uint16_t *L2, int r, float s, const uint32_t *mask, float p, uint16_t *Y,
+                             uint16_t *T_save, void *ws, size_t ws_bytes, void *stream) {
+  int rc = check_linear(M, W, r);
   if (rc) return rc;
-  if (dX) {
-    // dX = dY W_hat + G_hi L1^T: W_hat [N x K] is read in place as an MN-major B.
-    rc = dequant_launch(W, w_hat, st, dev->sms);
-    if (rc) return rc;
-    GemmSeg sX[2] = {{{dY, M, N, N, 0}, {w_hat, K, N, K, 1}}, {{G, M, r, 2 * r, 0}, {L1, K, r, r, 0}}};
-    rc = tc_gemm(st, dev, M, K, 2, sX, 1.f, dX, K, 1, 0, nullptr, QLORA_KERNEL_GEMM_DX);
-    if (rc) return rc;
-  }
-  // dL2 = T^T dY as dL2^T [N x r] = dY^T (T_hi + T_lo), written transposed,
-  // and dL1 = X^T (G_hi + G_lo) [K x r].  When both halves fit one tile the
-  // product runs against the whole [hi | lo] pair (2r columns) and the
-  // epilogue adds the halves, so dY and X stream once; otherwise as two
-  // accumulated segments over the tokens.
-  if (can_fold(r)) {
-    GemmSeg s2 = {{dY, N, M, N, 1}, {T, 2 * r, M, 2 * r, 1}};
-    rc = tc_gemm(st, dev, N, 2 * r, 1, &s2, 1.f, dL2, 1, N, out_f32, split_ws, QLORA_KERNEL_GEMM_DL2, 0, false, r);
-    if (rc) return rc;
-    GemmSeg s1 = {{X, K, M, K, 1}, {G, 2 * r, M, 2 * r, 1}};
-    return tc_gemm(st, dev, K, 2 * r, 1, &s1, 1.f, dL1, r, 1, out_f32, split_ws, QLORA_KERNEL_GEMM_DL1, 0, false, r);
-  }
-  const uint16_t *T_lo = T + r;
-  GemmSeg s2[2] = {{{dY, N, M, N, 1}, {T, r, M, 2 * r, 1}}, {{dY, N, M, N, 1}, {T_lo, r, M, 2 * r, 1}}};
-  rc = tc_gemm(st, dev, N, r, 2, s2, 1.f, dL2, 1, N, out_f32, split_ws, QLORA_KERNEL_GEMM_DL2, 0, true);
+  if (!(p >= 0.f && p < 1.f)) return QLORA_ERR_INVALID_ARG;
+  if (M == 0) return QLORA_OK;
+  if (!X || !L1 || !L2 || !Y || !mask) return QLORA_ERR_INVALID_ARG;
+  if (!aligned(X, 16) || !aligned(L1, 16) || !aligned(L2, 16) || !aligned(Y, 16) || !aligned(mask, 16) ||
+      (T_save && !aligned(T_save, 16)))
+    return QLORA_ERR_MISALIGNED;
+  DeviceInfo *dev;
+  rc = current_device_info(&dev);
   if (rc) return rc;
-  const uint16_t *G_lo = G + r;
-  GemmSeg s1[2] = {{{X, K, M, K, 1}, {G, r, M, 2 * r, 1}}, {{X, K, M, K, 1}, {G_lo, r, M, 2 * r, 1}}};
-  return tc_gemm(st, dev, K, r, 2, s1, 1.f, dL1, r, 1, out_f32, split_ws, QLORA_KERNEL_GEMM_DL1, 0, true);
+  const int64_t N = W->n_out, K = W->k_in;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const FwdLayout L = fwd_layout(M, N, K, r, dev->sms);
+  if (!ws || ws_bytes < qlora_linear_fwd_dropout_workspace_size(M, N, K, r)) return QLORA_ERR_WORKSPACE;
+  if (!aligned(ws, 256)) return QLORA_ERR_MISALIGNED;
+  uint8_t *w8 = reinterpret_cast<uint8_t *>(ws);
+  uint16_t *Xm = reinterpret_cast<uint16_t *>(w8 + L.total);
+  rc = dropout_launch(X, mask, M * K, Xm, dev, st);
+  if (rc) return rc;
+  return fwd_large(X, Xm, s / (1.f - p), M, W, L1, L2, r, Y, T_save, w8, L, dev, st);
+}
+
+int qlora_linear_bwd_dropout(const uint16_t *dY, const uint16_t *X, const uint16_t *T_saved, int64_t M,
+                             const qlora_nf4dq_t *W, const uint16_t *L1, const uint16_t *L2, int r, float s,
+                             const uint32_t *mask, float p, uint16_t *dX, void *dL1, void *dL2, int grad_dtype,
+                             void *ws, size_t ws_bytes, void *stream) {
+  int rc = check_linear(M, W, r);
+  if (rc) return rc;
+  if (!(p >= 0.f && p < 1.f)) return QLORA_ERR_INVALID_ARG;
+  if (grad_dtype != QLORA_DTYPE_F32 && grad_dtype != QLORA_DTYPE_BF16) return QLORA_ERR_INVALID_ARG;
+  if (!L1 || !L2 || !dL1 || !dL2) return QLORA_ERR_INVALID_ARG;
+  if (M > 0 && (!dY || !X || !mask)) return QLORA_ERR_INVALID_ARG;
+  if (!aligned(L1, 16) || !aligned(L2, 16) || !aligned(dL1, 16) || !aligned(dL2, 16) || (dY && !aligned(dY, 16)) ||
+      (X && !aligned(X, 16)) || (dX && !aligned(dX, 16)) || (T_saved && !aligned(T_saved, 16)) ||
+      (mask && !aligned(mask, 16)))
+    return QLORA_ERR_MISALIGNED;
+  DeviceInfo *dev;
+  rc = current_device_info(&dev);
+  if (rc) return rc;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int64_t N = W->n_out, K = W->k_in;
+  const size_t gsz = grad_dtype == QLORA_DTYPE_F32 ? 4 : 2;
+  if (M == 0) {
+    if (cudaMemsetAsync(dL1, 0, (size_t)K * r * gsz, st) != cudaSuccess) return QLORA_ERR_CUDA;
+    if (cudaMemsetAsync(dL2, 0, (size_t)r * N * gsz, st) != cudaSuccess) return QLORA_ERR_CUDA;
+    return QLORA_OK;
+  }
+  const BwdLayout L = bwd_layout(M, N, K, r, dev->sms);
+  if (!ws || ws_bytes < qlora_linear_bwd_dropout_workspace_size(M, N, K, r)) return QLORA_ERR_WORKSPACE;
+  if (!aligned(ws, 256)) return QLORA_ERR_MISALIGNED;
+  uint8_t *w8 = reinterpret_cast<uint8_t *>(ws);
+  uint16_t *Xm = reinterpret_cast<uint16_t *>(w8 + L.total);
+  uint16_t *Z = reinterpret_cast<uint16_t *>(w8 + L.total + align_up((size_t)M * K * 2));
+  rc = dropout_launch(X, mask, M * K, Xm, dev, st);
+  if (rc) return rc;
+  const BwdDropout drop = {Xm, 1.f / (1.f - p), mask, Z};
+  return bwd_large(dY, X, T_saved, M, W, L1, L2, r, s, dX, dL1, dL2, grad_dtype == QLORA_DTYPE_F32, w8, L, &drop,
+                   dev, st);
 }
 
 }  // extern "C"

@@ -58,8 +58,39 @@ struct TcGemmArgs {
   int64_t lo_off;           // bf16 output only: if > 0 also store lo = bf16(v - hi) at +lo_off
   int out_f32;              // 1: fp32 output, 0: bf16
   int fold;                 // fold form: output column j < fold is D(i, j) + D(i, j + fold)
+  // Optional masked addend of a bf16 output (unsplit, not folded): before
+  // rounding, D(i, j) += add_scale * Z(i, j) where bit (i*N + j) of add_mask
+  // is set (Z bf16 with row stride add_ld; N a multiple of 32).  LoRA dropout
+  // uses it to gate the adapter term of dX.
+  const uint16_t *add;
+  const uint32_t *add_mask;
+  float add_scale;
+  int64_t add_ld;
   int *err;
 };
+
+// v[j] += add_scale * Z(row, col0 + j) for the kept columns of a 32-column chunk.
+__device__ __forceinline__ void tc_add_masked(const TcGemmArgs &p, int row, int col0, float (&v)[32]) {
+  const uint32_t m = ld_dep_u32(p.add_mask + (((int64_t)row * p.N + col0) >> 5));
+  const uint16_t *z = p.add + (int64_t)row * p.add_ld + col0;
+  if ((p.add_ld & 7) == 0) {
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const uint4 w = ld_dep_v4(z + 8 * q);
+      const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+      for (int h = 0; h < 4; ++h) {
+        const int j = 8 * q + 2 * h;
+        if ((m >> j) & 1u) v[j] += p.add_scale * __uint_as_float(ww[h] << 16);
+        if ((m >> (j + 1)) & 1u) v[j + 1] += p.add_scale * __uint_as_float(ww[h] & 0xFFFF0000u);
+      }
+    }
+  } else {
+#pragma unroll
+    for (int j = 0; j < 32; ++j)
+      if ((m >> j) & 1u) v[j] += p.add_scale * __uint_as_float(ld_dep_u16(z + j) << 16);
+  }
+}
 
 // Fold-form store of 32 consecutive output columns col0.. of row `row` (the
 // values before alpha; split partials go to the dense [split][M][fold] buffer).
@@ -458,6 +489,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         } else {
           __nv_bfloat16 *o = reinterpret_cast<__nv_bfloat16 *>(p.out);
           const int64_t lo = p.lo_off;
+          float v[32];
+#pragma unroll
+          for (int j = 0; j < 32; ++j) v[j] = alpha * __uint_as_float(r[j]);
+          if (p.add) tc_add_masked(p, row, col0, v);
           if (p.ld_col == 1 && col0 + 32 <= p.N && (p.ld_row & 7) == 0 && (lo & 7) == 0) {
             uint4 *dst = reinterpret_cast<uint4 *>(o + (int64_t)row * p.ld_row + col0);
             uint4 *dst_lo = reinterpret_cast<uint4 *>(o + (int64_t)row * p.ld_row + col0 + lo);
@@ -466,8 +501,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
               uint32_t w[4], wl[4];
 #pragma unroll
               for (int h = 0; h < 4; ++h) {
-                const float v0 = alpha * __uint_as_float(r[8 * j + 2 * h]);
-                const float v1 = alpha * __uint_as_float(r[8 * j + 2 * h + 1]);
+                const float v0 = v[8 * j + 2 * h];
+                const float v1 = v[8 * j + 2 * h + 1];
                 const __nv_bfloat162 b2 = __floats2bfloat162_rn(v0, v1);
                 w[h] = *reinterpret_cast<const uint32_t *>(&b2);
                 const __nv_bfloat162 l2 = __floats2bfloat162_rn(v0 - __low2float(b2), v1 - __high2float(b2));
@@ -480,11 +515,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
             for (int j = 0; j < 32; ++j)
               if (col0 + j < p.N) {
-                const float v = alpha * __uint_as_float(r[j]);
-                const __nv_bfloat16 hb = __float2bfloat16_rn(v);
+                const __nv_bfloat16 hb = __float2bfloat16_rn(v[j]);
                 const int64_t off = (int64_t)row * p.ld_row + (int64_t)(col0 + j) * p.ld_col;
                 o[off] = hb;
-                if (lo > 0) o[off + lo] = __float2bfloat16_rn(v - __bfloat162float(hb));
+                if (lo > 0) o[off + lo] = __float2bfloat16_rn(v[j] - __bfloat162float(hb));
               }
           }
         }

@@ -187,6 +187,32 @@ QLORA_API int qlora_linear_bwd(const uint16_t *dY, const uint16_t *X, const uint
                      const qlora_nf4dq_t *W, const uint16_t *L1, const uint16_t *L2, int r, float s, uint16_t *dX,
                      void *dL1, void *dL2, int grad_dtype, void *ws, size_t ws_bytes, void *stream);
 
+/*
+ * LoRA dropout (QLoRA Appendix B.2 trains with LoRA dropout, p = 0.1 up to
+ * 13B and 0.05 at 33B and 65B).  It acts on the adapter's input only:
+ *   Y  = X W_hat^T + T L2,   T = s drop(X) L1,   drop(X) = X * m / (1 - p);
+ *   dX = dY W_hat + (G L1^T) * m / (1 - p),  G = s dY L2^T;
+ *   dL2 = T^T dY,  dL1 = drop(X)^T G.
+ * The keep mask m is an input: uint32 words over the row-major [M x K]
+ * elements of X, bit b of word w keeping element 32 w + b (so [M x K/32]
+ * words, 16-byte aligned; the same mask must be passed to the forward and
+ * the backward of a step).  0 <= p < 1; p = 0 with an all-ones mask computes
+ * the plain linear.  Other arguments, layouts and T_save are those of
+ * qlora_linear_fwd / qlora_linear_bwd.  Every token count takes the
+ * dequant + tensor-core path.  Workspace: *_dropout_workspace_size().
+ * Errors: as qlora_linear_fwd / _bwd, plus QLORA_ERR_INVALID_ARG for a NULL
+ * mask (M > 0) or p outside [0, 1).
+ */
+QLORA_API size_t qlora_linear_fwd_dropout_workspace_size(int64_t M, int64_t n_out, int64_t k_in, int r);
+QLORA_API size_t qlora_linear_bwd_dropout_workspace_size(int64_t M, int64_t n_out, int64_t k_in, int r);
+QLORA_API int qlora_linear_fwd_dropout(const uint16_t *X, int64_t M, const qlora_nf4dq_t *W, const uint16_t *L1,
+                                       const uint16_t *L2, int r, float s, const uint32_t *mask, float p,
+                                       uint16_t *Y, uint16_t *T_save, void *ws, size_t ws_bytes, void *stream);
+QLORA_API int qlora_linear_bwd_dropout(const uint16_t *dY, const uint16_t *X, const uint16_t *T_saved, int64_t M,
+                                       const qlora_nf4dq_t *W, const uint16_t *L1, const uint16_t *L2, int r,
+                                       float s, const uint32_t *mask, float p, uint16_t *dX, void *dL1, void *dL2,
+                                       int grad_dtype, void *ws, size_t ws_bytes, void *stream);
+
 /* ---- diagnostics ----------------------------------------------------------------- */
 
 /* Static description of a status code. */
@@ -219,9 +245,11 @@ QLORA_API int qlora_get_last_device_error(void *stream);
 #define QLORA_KERNEL_GEMM_DX 13     /* dX = dY W_hat + G L1^T */
 #define QLORA_KERNEL_GEMM_DL2 14    /* dL2 = T^T dY */
 #define QLORA_KERNEL_GEMM_DL1 15    /* dL1 = X^T G */
+#define QLORA_KERNEL_GEMM_Z 16      /* Z = G L1^T (dropout backward) */
 #define QLORA_KERNEL_SPLITK_FINALIZE 20
 #define QLORA_KERNEL_GEMV_FWD 30    /* fused decode + mma.sync product, up to 32 tokens */
 #define QLORA_KERNEL_FUSED_FWD 31   /* fused decode + tcgen05 product, up to 128 tokens */
+#define QLORA_KERNEL_DROPOUT_MASK 40 /* Xm = X * m (LoRA dropout) */
 QLORA_API int qlora_profile_start(int capacity);
 QLORA_API int qlora_profile_stop(void);
 QLORA_API int qlora_profile_read(int i, int *kind, float *ms);
