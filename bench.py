@@ -148,6 +148,18 @@ class Linear:
         self.T = torch.empty(M, 2 * r, dtype=torch.bfloat16, device=dev)
         self.dX = torch.empty(M, K, dtype=torch.bfloat16, device=dev)
         self.q = None
+        self.mask = None
+
+
+def device_dropout_mask(M, K, p, seed, dev):
+    """Keep mask of LoRA dropout drawn on the device (seeded): int32 words
+    [M, K/32], element 32 w + b kept in bit b of word w with probability 1 - p."""
+    g = torch.Generator(device=dev)
+    g.manual_seed(seed)
+    keep = (torch.rand((M, K // 32, 32), generator=g, device=dev) >= p).to(torch.int64)
+    words = (keep << torch.arange(32, device=dev, dtype=torch.int64)).sum(-1)
+    return words.to(torch.uint32).view(torch.int32) if hasattr(torch, "uint32") else (
+        torch.where(words >= 2 ** 31, words - 2 ** 32, words).to(torch.int32))
 
 
 def build_layer(dev, rank, wl=WL):
@@ -167,20 +179,23 @@ def build_layer(dev, rank, wl=WL):
     return lins, grads, [H, A, U] + [l.dY for l in lins]
 
 
-def make_step(qlora, lins, grads, world, wl=WL):
-    """One step; `ready(t)` (if given) is called before the step first reads input t."""
+def make_step(qlora, lins, grads, world, wl=WL, dropout=0.0):
+    """One step; `ready(t)` (if given) is called before the step first reads input t.
+    With `dropout` > 0 each linear applies LoRA dropout with its own keep mask."""
     def step(ready=None):
         for l in lins:
             l.q = qlora.quantize_nf4_dq(l.W, out=l.q)
         for l in lins:
             if ready:
                 ready(l.X)
-            qlora.linear_fwd(l.X, l.q, l.L1, l.L2, wl.s, Y=l.Y, T=l.T)
+                if l.mask is not None:
+                    ready(l.mask)
+            qlora.linear_fwd(l.X, l.q, l.L1, l.L2, wl.s, Y=l.Y, T=l.T, dropout_mask=l.mask, dropout_p=dropout)
         for l in reversed(lins):
             if ready:
                 ready(l.dY)
             qlora.linear_bwd(l.dY, l.X, l.T, l.q, l.L1, l.L2, wl.s, grad_dtype=torch.float32,
-                             dX=l.dX, dL1=l.dL1, dL2=l.dL2)
+                             dX=l.dX, dL1=l.dL1, dL2=l.dL2, dropout_mask=l.mask, dropout_p=dropout)
         grads.allreduce()
     return step
 
@@ -254,6 +269,8 @@ def run_ours(args, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     wl = TRAIN[args.workload]
+    if wl.layers > 1 and args.dropout > 0:
+        raise SystemExit("bench.py: --dropout applies to the single-layer training workloads")
     if wl.layers > 1:
         from bit_nf4_quantized_02_b200.stack import QLoRAStack, SEEDED_DY
         hidden, mlp = wl.linears[0].n_out, wl.linears[4].n_out
@@ -266,14 +283,26 @@ def run_ours(args, rank, world, local_rank):
         sel = wl.linears * wl.layers
     else:
         lins, grads, acts = build_layer(dev, rank, wl)
+        if args.dropout > 0:
+            for i, l in enumerate(lins):
+                l.mask = device_dropout_mask(wl.M, l.lin.k_in, args.dropout, wl.seed + 1000 * rank + 50 + i, dev)
         # copy order for the end-to-end run: the step's first read of each input
-        acts = acts[:3] + acts[3:][::-1]
+        # (with dropout each linear's keep mask right after its input)
+        if args.dropout > 0:
+            first = []
+            for l in lins:
+                if all(l.X.data_ptr() != a.data_ptr() for a in first):
+                    first.append(l.X)
+                first.append(l.mask)
+            acts = first + acts[3:][::-1]
+        else:
+            acts = acts[:3] + acts[3:][::-1]
         flat = grads.flat
         if args.linear:
             lins = [l for l in lins if l.lin.name == args.linear]
         for l in lins:  # allocate the quantized buffers once
             l.q = qlora.quantize_nf4_dq(l.W)
-        step = make_step(qlora, lins, grads, world, wl)
+        step = make_step(qlora, lins, grads, world, wl, dropout=args.dropout)
         sel = [l.lin for l in lins]
     for _ in range(args.warmup):
         step()
@@ -335,8 +364,11 @@ def run_ours(args, rank, world, local_rank):
         c[1] += kms
     dom_ms = per_kind.get("gemm_Y", [0, 0.0])[1] + per_kind.get("gemm_dX", [0, 0.0])[1]
     dom_n = per_kind.get("gemm_Y", [0, 0.0])[0] + per_kind.get("gemm_dX", [0, 0.0])[0]
+    # with LoRA dropout dX's adapter term runs as its own product (gemm_Z),
+    # so the dX launches do the base product alone
     dom_flops = args.steps * sum(linear_flops(wl.M, l.n_out, l.k_in, wl.r)["gemm_Y"] +
-                                 linear_flops(wl.M, l.n_out, l.k_in, wl.r)["gemm_dX"] for l in sel)
+                                 linear_flops(wl.M, l.n_out, l.k_in, wl.r)["gemm_dX"]
+                                 - (2 * wl.M * wl.r * l.k_in if args.dropout > 0 else 0) for l in sel)
     achieved = dom_flops / (dom_ms * 1e-3) / 1e12 if dom_ms > 0 else None
     # The burst GEMM peak while the SM clock held its maximum through the timed
     # region; the sustained (power-capped) one once the clock dropped.
@@ -366,7 +398,8 @@ def run_ours(args, rank, world, local_rank):
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": wl.name + (f"[{args.linear} only]" if args.linear else ""),
+        "config": {"workload": wl.name + (f"[{args.linear} only]" if args.linear else "")
+                               + (f"-lora-dropout{args.dropout:g}" if args.dropout > 0 else ""),
                    "model": {"llama7b-train": "llama7b-layer-linears", "llama65b-train": "llama65b-layer-linears",
                              "llama33b-stack": "llama33b-8-layer-stack"}[args.workload],
                    "global_batch": (16 if wl.M == 8192 and args.workload == "llama7b-train" else 4) * world,
@@ -376,7 +409,9 @@ def run_ours(args, rank, world, local_rank):
                    "step": f"quantize {7 * wl.layers} fp32 weights to NF4+DQ, fwd + bwd of the "
                            f"{7 * wl.layers} QLoRA linears"
                            + (" (layer to layer: H' = bf16(down(up(H)) + R))" if wl.layers > 1 else "")
-                           + (", all-reduce of adapter grads" if world > 1 else ""),
+                           + (", all-reduce of adapter grads" if world > 1 else "")
+                           + (f", LoRA dropout p = {args.dropout:g} on every adapter (one seeded keep mask per "
+                              f"linear, copied in with the inputs in e2e)" if args.dropout > 0 else ""),
                    "l2": "inputs larger than L2 (>1 GB touched per step), no flush"},
         "e2e": ({"value": flops / (ms_e2e * 1e-3) / 1e12, "unit": UNIT, "h2d_bytes_per_step": h2d,
                  "d2h_bytes_per_step": d2h,
@@ -669,6 +704,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end (host buffers) measurement")
+    ap.add_argument("--dropout", type=float, default=0.0,
+                    help="LoRA dropout probability on every adapter (single-layer training workloads)")
     ap.add_argument("--tokens", type=int, default=None,
                     help="llama65b-decode: tokens per step (default 16; 33..128 run the tcgen05 fused forward)")
     ap.add_argument("--linear", choices=[l.name for l in WL.linears], default=None,
