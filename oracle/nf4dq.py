@@ -74,6 +74,37 @@ E4M3_MAX = 448.0           # largest finite OCP E4M3 value
 # exact midpoints.
 NF4_MIDPOINTS = (NF4_VALUES[:-1].astype(np.float64) + NF4_VALUES[1:].astype(np.float64)) / 2.0
 
+# --------------------------------------------------------------------------
+# The 4-bit float FP4 (E2M1) that the paper compares NF4 against (§4,
+# Tables 2-4: "Float4 (E2M1)").  Its value set {0, 0.5, 1, 1.5, 2, 3, 4, 6}
+# and their negatives, normalised by the largest value 6 so that a block's
+# absmax maps to +-1 as for NF4, rounded to float32, in ascending order.  The
+# format has a positive and a negative zero; both codes hold +0 here, so code
+# 7 is the exact zero of either table.  (Its encoding: sign, a 2-bit exponent
+# with bias 1, a 1-bit mantissa; exponent 0 is subnormal: 0.5 * m.)
+# --------------------------------------------------------------------------
+def e2m1_value(bits: int) -> float:
+    """Value of a 4-bit E2M1 code (sign bit 3, exponent bits 2-1, mantissa bit 0)."""
+    sign = -1.0 if bits & 8 else 1.0
+    e, m = (bits >> 1) & 3, bits & 1
+    mag = 0.5 * m if e == 0 else (1.0 + 0.5 * m) * 2.0 ** (e - 1)
+    return sign * mag
+
+
+def _fp4_table() -> np.ndarray:
+    vals = sorted({e2m1_value(b) for b in range(16)})           # 15 distinct values, one zero
+    vals = vals[:7] + [0.0] + vals[7:]                          # both zero codes
+    return np.array([np.float32(v) / np.float32(6.0) for v in vals], dtype=np.float32)
+
+
+FP4_VALUES = _fp4_table()
+TABLES = {"nf4": NF4_VALUES, "fp4": FP4_VALUES}
+
+
+def midpoints(levels: np.ndarray) -> np.ndarray:
+    levels = np.asarray(levels, dtype=np.float32).astype(np.float64)
+    return (levels[:-1] + levels[1:]) / 2.0
+
 
 # --------------------------------------------------------------------------
 # Small exact-rounding helpers.
@@ -196,18 +227,19 @@ def e4m3_encode_rne_satfinite(x) -> np.ndarray:
 # --------------------------------------------------------------------------
 # First-level quantization: NF4 with absmax blocks of 64.
 # --------------------------------------------------------------------------
-def nf4_code(x32) -> np.ndarray:
-    """Nearest NF4 level for normalised inputs x in [-1, 1].
+def nf4_code(x32, levels: np.ndarray = NF4_VALUES) -> np.ndarray:
+    """Nearest level of a 16-level table (NF4 by default) for normalised inputs x in [-1, 1].
 
     code = number of exact midpoints that x lies strictly above, so an input
     exactly on a midpoint takes the lower level.
     """
+    mids = NF4_MIDPOINTS if levels is NF4_VALUES else midpoints(levels)
     x = f32(x32).astype(np.float64)
     flat = x.reshape(-1)
     out = np.empty(flat.size, dtype=np.uint8)
     step = 1 << 20                      # bounded temporaries only; no effect on the result
     for s in range(0, flat.size, step):
-        out[s:s + step] = (flat[s:s + step, None] > NF4_MIDPOINTS).sum(axis=-1)
+        out[s:s + step] = (flat[s:s + step, None] > mids).sum(axis=-1)
     return out.reshape(x.shape)
 
 
@@ -227,8 +259,9 @@ def block_absmax(flat32: np.ndarray, bs: int) -> np.ndarray:
     return out
 
 
-def quantize_nf4(w) -> tuple[np.ndarray, np.ndarray]:
-    """NF4-quantize a tensor in absmax blocks of 64 (§2 blocking, §3 NF4).
+def quantize_nf4(w, levels: np.ndarray = NF4_VALUES) -> tuple[np.ndarray, np.ndarray]:
+    """NF4-quantize (or, with ``levels``, quantize to another 16-level table) a
+    tensor in absmax blocks of 64 (§2 blocking, §3 NF4).
 
     w: any float array (float32 or bfloat16 values widened to float32); it is
     flattened row-major.  Returns (codes uint8 [numel], c2 float32 [nblocks]).
@@ -240,7 +273,7 @@ def quantize_nf4(w) -> tuple[np.ndarray, np.ndarray]:
     scale = np.repeat(c2, W_BLOCK)[: flat.size]
     with np.errstate(invalid="ignore", divide="ignore"):
         x = (flat / scale).astype(np.float32)      # IEEE float32 quotient
-    codes = nf4_code(np.where(scale == 0, np.float32(0), x))
+    codes = nf4_code(np.where(scale == 0, np.float32(0), x), levels)
     codes = np.where(scale == 0, NF4_ZERO_CODE, codes).astype(np.uint8)
     return codes, c2
 
@@ -310,7 +343,7 @@ def dequant_c2(code8, c1, mu) -> np.ndarray:
     return fma_f32(e4m3_decode(code8), c1_per, np.float32(mu))
 
 
-def double_dequant_bits(codes, code8, c1, mu, shape) -> np.ndarray:
+def double_dequant_bits(codes, code8, c1, mu, shape, levels: np.ndarray = NF4_VALUES) -> np.ndarray:
     """doubleDequant (Eq. 6) to bfloat16, returned as uint16 bit patterns.
 
     W_hat = bf16_rne(f32(NF4[code] * c2_hat[block])) with c2_hat from
@@ -319,11 +352,11 @@ def double_dequant_bits(codes, code8, c1, mu, shape) -> np.ndarray:
     codes = np.asarray(codes, dtype=np.uint8).reshape(-1)
     c2_hat = dequant_c2(code8, c1, mu)
     scale = np.repeat(c2_hat, W_BLOCK)[: codes.size]
-    prod = (NF4_VALUES[codes] * scale).astype(np.float32)
+    prod = (np.asarray(levels, np.float32)[codes] * scale).astype(np.float32)
     return bf16_rne_bits(prod).reshape(shape)
 
 
-def quantize_nf4_dq(w):
+def quantize_nf4_dq(w, levels: np.ndarray = NF4_VALUES):
     """The full quantizer of the QLoRA storage format.
 
     Returns a dict with the packed codes (uint8 [ceil(numel/2)]), the E4M3
@@ -331,7 +364,7 @@ def quantize_nf4_dq(w):
     (float32), plus the unpacked codes and the float32 c2 for checking.
     """
     w = np.asarray(w)
-    codes, c2 = quantize_nf4(w)
+    codes, c2 = quantize_nf4(w, levels)
     code8, c1, mu = double_quantize(c2)
     return {
         "shape": tuple(w.shape),
@@ -341,16 +374,17 @@ def quantize_nf4_dq(w):
         "c2_fp8": code8,
         "c1": c1,
         "mu": mu,
+        "levels": np.asarray(levels, np.float32),
     }
 
 
 def dequantize(q) -> np.ndarray:
     """doubleDequant of a ``quantize_nf4_dq`` result, as float32 values of bf16."""
-    bits = double_dequant_bits(q["codes"], q["c2_fp8"], q["c1"], q["mu"], q["shape"])
+    bits = double_dequant_bits(q["codes"], q["c2_fp8"], q["c1"], q["mu"], q["shape"], q.get("levels", NF4_VALUES))
     return bf16_bits_to_f32(bits)
 
 
-def dequantize_rows(w, rows) -> np.ndarray:
+def dequantize_rows(w, rows, levels: np.ndarray = NF4_VALUES) -> np.ndarray:
     """doubleDequant of selected rows of a 2-D weight, for sampled checks.
 
     The same steps as ``quantize_nf4_dq`` + ``dequantize``: every block's c2
@@ -372,14 +406,14 @@ def dequantize_rows(w, rows) -> np.ndarray:
         seg = c2[g0 * C2_BLOCK: min(c2.size, g1 * C2_BLOCK)]
         code8, c1, _ = double_quantize(seg, mu)
         c2_hat = dequant_c2(code8, c1, mu)[b0 - g0 * C2_BLOCK: b1 - g0 * C2_BLOCK]
-        codes, c2_row = quantize_nf4(w[row])
+        codes, c2_row = quantize_nf4(w[row], levels)
         assert np.array_equal(c2_row, c2[b0:b1])
-        prod = (NF4_VALUES[codes] * np.repeat(c2_hat, W_BLOCK)).astype(np.float32)
+        prod = (np.asarray(levels, np.float32)[codes] * np.repeat(c2_hat, W_BLOCK)).astype(np.float32)
         out[i] = bf16_bits_to_f32(bf16_rne_bits(prod))
     return out
 
 
-def dequantize_cols(w, cols) -> np.ndarray:
+def dequantize_cols(w, cols, levels: np.ndarray = NF4_VALUES) -> np.ndarray:
     """doubleDequant of selected columns of a 2-D weight: [n_out, len(cols)].
 
     The same steps as ``quantize_nf4_dq`` + ``dequantize``: every block's c2
@@ -399,9 +433,9 @@ def dequantize_cols(w, cols) -> np.ndarray:
     c2_sel = c2.reshape(n_out, bpr)[:, cols // W_BLOCK]
     with np.errstate(invalid="ignore", divide="ignore"):
         x = (w[:, cols] / c2_sel).astype(np.float32)      # IEEE float32 quotient
-    codes = nf4_code(np.where(c2_sel == 0, np.float32(0), x))
+    codes = nf4_code(np.where(c2_sel == 0, np.float32(0), x), levels)
     codes = np.where(c2_sel == 0, NF4_ZERO_CODE, codes).astype(np.uint8)
-    prod = (NF4_VALUES[codes] * c2_hat).astype(np.float32)
+    prod = (np.asarray(levels, np.float32)[codes] * c2_hat).astype(np.float32)
     return bf16_bits_to_f32(bf16_rne_bits(prod))
 
 
