@@ -63,6 +63,7 @@ class NF4Tensor:
     c2_fp8  uint8 [ceil(numel/64)]  E4M3 codes of the mean-centred block absmax
     c1      fp32  [ceil(nblk/256)]  second-level constants
     c2_mean fp32  [1]               mean of the first-level constants
+    table   "nf4" (Appendix E levels) or "fp4" (E2M1, the 4-bit float of §4)
     """
 
     n_out: int
@@ -71,6 +72,7 @@ class NF4Tensor:
     c2_fp8: torch.Tensor
     c1: torch.Tensor
     c2_mean: torch.Tensor
+    table: str = "nf4"
 
     @property
     def shape(self):
@@ -82,7 +84,7 @@ class NF4Tensor:
 
     def as_struct(self) -> _lib.NF4DQ:
         return _lib.NF4DQ(self.n_out, self.k_in, _ptr(self.codes), _ptr(self.c2_fp8), _ptr(self.c1),
-                          _ptr(self.c2_mean))
+                          _ptr(self.c2_mean), _lib.TABLES[self.table])
 
     def nbytes(self) -> int:
         return sum(t.numel() * t.element_size() for t in (self.codes, self.c2_fp8, self.c1, self.c2_mean))
@@ -100,8 +102,9 @@ def _empty_nf4(n_out: int, k_in: int, device) -> NF4Tensor:
     )
 
 
-def quantize_nf4_dq(W: torch.Tensor, out: NF4Tensor | None = None) -> NF4Tensor:
-    """Quantize a 2-D fp32 or bf16 CUDA weight [n_out, k_in] to NF4 + DQ."""
+def quantize_nf4_dq(W: torch.Tensor, out: NF4Tensor | None = None, table: str = "nf4") -> NF4Tensor:
+    """Quantize a 2-D fp32 or bf16 CUDA weight [n_out, k_in] to NF4 + DQ
+    (``table="fp4"``: the FP4 E2M1 code table instead of NF4)."""
     lib = _lib.load()
     if W.dim() != 2:
         raise ValueError("qlora: W must be 2-D [n_out, k_in]")
@@ -112,12 +115,15 @@ def quantize_nf4_dq(W: torch.Tensor, out: NF4Tensor | None = None) -> NF4Tensor:
     else:
         raise TypeError("qlora: W must be float32 or bfloat16")
     n_out, k_in = W.shape
+    if table not in _lib.TABLES:
+        raise ValueError(f"qlora: unknown code table {table!r}")
     q = out if out is not None else _empty_nf4(n_out, k_in, W.device)
+    q.table = table
     ws_bytes = lib.qlora_quantize_workspace_size(n_out * k_in)
     ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=W.device)
-    _lib.check(lib.qlora_quantize_nf4_dq(_ptr(W), wdt, n_out, k_in, _ptr(q.codes), _ptr(q.c2_fp8), _ptr(q.c1),
-                                         _ptr(q.c2_mean), _ptr(ws), ws_bytes, _stream(W.device)),
-               "qlora_quantize_nf4_dq")
+    _lib.check(lib.qlora_quantize_4bit_dq(_ptr(W), wdt, n_out, k_in, _lib.TABLES[table], _ptr(q.codes),
+                                          _ptr(q.c2_fp8), _ptr(q.c1), _ptr(q.c2_mean), _ptr(ws), ws_bytes,
+                                          _stream(W.device)), "qlora_quantize_4bit_dq")
     return q
 
 

@@ -43,7 +43,11 @@ class NF4DQ(ctypes.Structure):
         ("c2_fp8", c_void_p),
         ("c1", c_void_p),
         ("c2_mean", c_void_p),
+        ("table", ctypes.c_int32),
     ]
+
+
+TABLES = {"nf4": 0, "fp4": 1}   # QLORA_TABLE_NF4, QLORA_TABLE_FP4
 
 
 # name -> (restype, argtypes)
@@ -57,6 +61,8 @@ SIGNATURES = {
     "qlora_quantize_workspace_size": (c_size_t, [c_int64]),
     "qlora_quantize_nf4_dq": (c_int, [c_void_p, c_int, c_int64, c_int64, c_void_p, c_void_p, c_void_p, c_void_p,
                                       c_void_p, c_size_t, c_void_p]),
+    "qlora_quantize_4bit_dq": (c_int, [c_void_p, c_int, c_int64, c_int64, c_int, c_void_p, c_void_p, c_void_p,
+                                       c_void_p, c_void_p, c_size_t, c_void_p]),
     "qlora_quantize_nf4_dq_noalloc": (c_int, [c_void_p, c_int, c_int64, c_int64, c_void_p, c_void_p, c_void_p,
                                               c_void_p, c_void_p]),
     "qlora_dequant": (c_int, [POINTER(NF4DQ), c_void_p, c_void_p]),

@@ -71,6 +71,7 @@ struct GvArgs {
   const __nv_bfloat16 *L1;   // [K x r]
   const __nv_bfloat16 *L2;   // [r x N]
   float *acc;            // [M x N] fp32, zero at launch
+  int table;             // 16-level code table of the weight (kLevels)
   int *err;
 };
 
@@ -110,11 +111,11 @@ __device__ __forceinline__ void fence_acq_rel_gpu() { asm volatile("fence.acq_re
 // bytes.
 struct BlockTable {
   uint32_t lo[4], hi[4];
-  __device__ __forceinline__ void build(float c2h) {
+  __device__ __forceinline__ void build(float c2h, const float *levels) {
     uint32_t e[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-      const __nv_bfloat162 p = __floats2bfloat162_rn(__fmul_rn(kNF4[2 * i], c2h), __fmul_rn(kNF4[2 * i + 1], c2h));
+      const __nv_bfloat162 p = __floats2bfloat162_rn(__fmul_rn(levels[2 * i], c2h), __fmul_rn(levels[2 * i + 1], c2h));
       e[i] = *reinterpret_cast<const uint32_t *>(&p);
     }
 #pragma unroll
@@ -213,8 +214,8 @@ struct GvConsumer {
         for (int t = 0; t < NT; ++t) d[c][t][0] = d[c][t][1] = d[c][t][2] = d[c][t][3] = 0.f;
     }
     BlockTable tb0, tb1;
-    tb0.build(cur.c2hat(0, mu));
-    tb1.build(cur.c2hat(1, mu));
+    tb0.build(cur.c2hat(0, mu), kLevels[P.table]);
+    tb1.build(cur.c2hat(1, mu), kLevels[P.table]);
     int nu = u, nstn = st + 1;
     if (nstn == nst) {
       nu = u + gridDim.x;

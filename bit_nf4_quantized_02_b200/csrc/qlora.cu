@@ -47,7 +47,7 @@ int current_device_info(DeviceInfo **out) {
       if (cudaGetSymbolAddress(reinterpret_cast<void **>(&d.err), g_dev_err) != cudaSuccess) return QLORA_ERR_CUDA;
       // One-time fill of the quantizer's code table (a constant of the NF4
       // levels), completed before any library launch on this device.
-      code_lut_init_kernel<<<(kCodeLutBytes + 255) / 256, 256>>>();
+      code_lut_init_kernel<<<dim3((kCodeLutBytes + 255) / 256, kNumTables), 256>>>();
       if (cudaGetLastError() != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess) return QLORA_ERR_CUDA;
       d.init = true;
     }
@@ -411,11 +411,12 @@ int dequant_launch(const qlora_nf4dq_t *W, __nv_bfloat16 *out, cudaStream_t st, 
   const int grid = (int)std::max<int64_t>(1, std::min<int64_t>((n8 + 255) / 256, (int64_t)sms * 16));
   ProfScope prof(QLORA_KERNEL_DEQUANT, st);
   return launch_pdl(nf4_dequant_kernel, dim3(grid), dim3(256), 0, st, W->codes, W->c2_fp8, W->c1, W->c2_mean, numel,
-                    out);
+                    out, (int)W->table);
 }
 
 int check_weight(const qlora_nf4dq_t *W) {
   if (!W || !W->codes || !W->c2_fp8 || !W->c1 || !W->c2_mean) return QLORA_ERR_INVALID_ARG;
+  if (W->table < 0 || W->table >= kNumTables) return QLORA_ERR_INVALID_ARG;
   if (W->n_out < 0 || W->k_in < 0) return QLORA_ERR_INVALID_ARG;
   if (!aligned(W->codes, 16) || !aligned(W->c2_fp8, 16) || !aligned(W->c1, 16) || !aligned(W->c2_mean, 4))
     return QLORA_ERR_MISALIGNED;
@@ -506,6 +507,7 @@ int launch_fused_fwd(const qlora_nf4dq_t *W, const uint16_t *X, int64_t M, const
   }
   FtArgs a;
   std::memset(&a, 0, sizeof(a));
+  a.table = (int)W->table;
   a.M = (int)M;
   a.N = (int)N;
   a.K = (int)K;
@@ -567,6 +569,7 @@ int launch_gemv(const qlora_nf4dq_t *W, const uint16_t *X, int64_t M, const uint
     return QLORA_ERR_CUDA;
   GvArgs a;
   std::memset(&a, 0, sizeof(a));
+  a.table = (int)W->table;
   a.M = (int)M;
   a.N = (int)N;
   a.K = (int)K;
@@ -750,7 +753,14 @@ size_t qlora_quantize_workspace_size(int64_t numel) {
 
 int qlora_quantize_nf4_dq(const void *W, int w_dtype, int64_t n_out, int64_t k_in, uint8_t *codes, uint8_t *c2_fp8,
                           float *c1, float *c2_mean, void *ws, size_t ws_bytes, void *stream) {
+  return qlora_quantize_4bit_dq(W, w_dtype, n_out, k_in, QLORA_TABLE_NF4, codes, c2_fp8, c1, c2_mean, ws, ws_bytes,
+                                stream);
+}
+
+int qlora_quantize_4bit_dq(const void *W, int w_dtype, int64_t n_out, int64_t k_in, int table, uint8_t *codes,
+                           uint8_t *c2_fp8, float *c1, float *c2_mean, void *ws, size_t ws_bytes, void *stream) {
   if (n_out < 0 || k_in < 0) return QLORA_ERR_INVALID_ARG;
+  if (table < 0 || table >= kNumTables) return QLORA_ERR_INVALID_ARG;
   if (w_dtype != QLORA_DTYPE_F32 && w_dtype != QLORA_DTYPE_BF16) return QLORA_ERR_INVALID_ARG;
   if (k_in > 0 && n_out > INT64_MAX / k_in) return QLORA_ERR_UNSUPPORTED_SHAPE;
   const int64_t numel = n_out * k_in;
@@ -774,10 +784,10 @@ int qlora_quantize_nf4_dq(const void *W, int w_dtype, int64_t n_out, int64_t k_i
   ProfScope prof(QLORA_KERNEL_QUANTIZE, st);
   if (w_dtype == QLORA_DTYPE_F32)
     rc = launch_pdl(nf4_quantize_kernel<float>, dim3(grid1), dim3(kQuantThreads), 0, st,
-                    reinterpret_cast<const float *>(W), numel, codes, c2, partial);
+                    reinterpret_cast<const float *>(W), numel, codes, c2, partial, table);
   else
     rc = launch_pdl(nf4_quantize_kernel<__nv_bfloat16>, dim3(grid1), dim3(kQuantThreads), 0, st,
-                    reinterpret_cast<const __nv_bfloat16 *>(W), numel, codes, c2, partial);
+                    reinterpret_cast<const __nv_bfloat16 *>(W), numel, codes, c2, partial, table);
   }
   if (rc) return rc;
   const int64_t nb256 = (nblk + 255) / 256;
@@ -789,6 +799,7 @@ int qlora_quantize_nf4_dq(const void *W, int w_dtype, int64_t n_out, int64_t k_i
 
 int qlora_quantize_nf4_dq_noalloc(const void *W, int w_dtype, int64_t n_out, int64_t k_in, uint8_t *codes,
                                   uint8_t *c2_fp8, float *c1, float *c2_mean, void *stream) {
+  const int table = QLORA_TABLE_NF4;   // the no-allocation quantizer writes NF4 codes
   if (n_out < 0 || k_in < 0) return QLORA_ERR_INVALID_ARG;
   if (w_dtype != QLORA_DTYPE_F32 && w_dtype != QLORA_DTYPE_BF16) return QLORA_ERR_INVALID_ARG;
   if (k_in > 0 && n_out > QLORA_NOALLOC_MAX_NUMEL / k_in) return QLORA_ERR_SCRATCH_LIMIT;
@@ -812,10 +823,10 @@ int qlora_quantize_nf4_dq_noalloc(const void *W, int w_dtype, int64_t n_out, int
   const int grid1 = (int)std::max<int64_t>(1, std::min<int64_t>((ngroups + 7) / 8, std::min(kQuantMaxCtas, dev->sms * kQuantCtasPerSm)));
   if (w_dtype == QLORA_DTYPE_F32)
     rc = launch_pdl(nf4_quantize_kernel<float>, dim3(grid1), dim3(kQuantThreads), 0, st,
-                    reinterpret_cast<const float *>(W), numel, codes, c2, partial);
+                    reinterpret_cast<const float *>(W), numel, codes, c2, partial, table);
   else
     rc = launch_pdl(nf4_quantize_kernel<__nv_bfloat16>, dim3(grid1), dim3(kQuantThreads), 0, st,
-                    reinterpret_cast<const __nv_bfloat16 *>(W), numel, codes, c2, partial);
+                    reinterpret_cast<const __nv_bfloat16 *>(W), numel, codes, c2, partial, table);
   if (rc) return rc;
   const int64_t nb256 = (nblk + 255) / 256;
   const int grid2 = (int)std::max<int64_t>(1, std::min<int64_t>((nb256 + kDqWarps - 1) / kDqWarps, (int64_t)dev->sms * 4));

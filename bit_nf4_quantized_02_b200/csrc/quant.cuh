@@ -23,9 +23,15 @@
 
 namespace qlora {
 
-// The 16 NF4 levels of Appendix E, in code order (all exact in fp32).
-__constant__ float kNF4[16] = {
-    -1.0f,
+// The 16-level code tables, in code order (all exact in fp32):
+//   kLevels[QLORA_TABLE_NF4]: the NF4 levels of Appendix E;
+//   kLevels[QLORA_TABLE_FP4]: FP4 (E2M1), the 4-bit float of §4 (Tables 2-4)
+//     that NF4 is compared against: its values {0, 0.5, 1, 1.5, 2, 3, 4, 6}
+//     and their negatives divided by 6 (fp32 quotients), both zero codes +0.
+// Code 7 is the exact zero of either table.
+constexpr int kNumTables = 2;
+__constant__ float kLevels[kNumTables][16] = {
+    {-1.0f,
     -0.6961928009986877f,
     -0.5250730514526367f,
     -0.39491748809814453f,
@@ -40,7 +46,9 @@ __constant__ float kNF4[16] = {
     0.44070982933044434f,
     0.5626170039176941f,
     0.7229568362236023f,
-    1.0f,
+    1.0f},
+    {-1.0f, -0x1.555556p-1f, -0.5f, -0x1.555556p-2f, -0.25f, -0x1.555556p-3f, -0x1.555556p-4f, 0.0f,
+     0.0f, 0x1.555556p-4f, 0x1.555556p-3f, 0.25f, 0x1.555556p-2f, 0.5f, 0x1.555556p-1f, 1.0f},
 };
 
 constexpr int kQuantThreads = 256;
@@ -54,9 +62,10 @@ constexpr int kQuantMaxCtas = 148 * 8;
 // rounded toward -inf keeps the decision exact in fp32.
 struct NF4Thresholds {
   float t[15];
-  __device__ __forceinline__ void init() {
+  __device__ __forceinline__ void init(int table) {
 #pragma unroll
-    for (int j = 0; j < 15; ++j) t[j] = __double2float_rd(((double)kNF4[j] + (double)kNF4[j + 1]) * 0.5);
+    for (int j = 0; j < 15; ++j)
+      t[j] = __double2float_rd(((double)kLevels[table][j] + (double)kLevels[table][j + 1]) * 0.5);
   }
   // code = #{ j : x > m_j } by a 4-step binary search over the sorted thresholds.
   __device__ __forceinline__ uint32_t encode(float x) const {
@@ -97,14 +106,15 @@ constexpr uint32_t kCodeBoundary = 0x80;
 
 // The table, filled once per device from the same thresholds the exact path
 // uses (code_lut_init_kernel), and copied into shared memory by each CTA.
-__device__ __align__(16) uint8_t g_code_lut[kCodeLutBytes];
+__device__ __align__(16) uint8_t g_code_lut[kNumTables][kCodeLutBytes];
 
 __global__ void __launch_bounds__(256) code_lut_init_kernel() {
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  const int table = blockIdx.y;
   if (i >= kCodeLutBytes) return;
   const int b = min(max(i - 1, 0), kCodeBins - 1);
   NF4Thresholds th;
-  th.init();
+  th.init(table);
   uint32_t code = 0;
   int edge = -1;
 #pragma unroll
@@ -113,15 +123,15 @@ __global__ void __launch_bounds__(256) code_lut_init_kernel() {
     code += tb < b ? 1u : 0u;
     if (tb >= b - 2 && tb <= b + 2) edge = j;
   }
-  g_code_lut[i] = edge >= 0 ? (uint8_t)(kCodeBoundary | edge) : (uint8_t)code;
+  g_code_lut[table][i] = edge >= 0 ? (uint8_t)(kCodeBoundary | edge) : (uint8_t)code;
 }
 
 // Copy the table into shared memory and zero the rest of its span (all
 // threads of the CTA).
-__device__ __forceinline__ void load_code_lut(uint8_t *lut) {
+__device__ __forceinline__ void load_code_lut(uint8_t *lut, int table) {
   for (int i = threadIdx.x; i < kCodeLutSpan / 16; i += blockDim.x)
     reinterpret_cast<uint4 *>(lut)[i] =
-        i < kCodeLutBytes / 16 ? reinterpret_cast<const uint4 *>(g_code_lut)[i] : make_uint4(0, 0, 0, 0);
+        i < kCodeLutBytes / 16 ? reinterpret_cast<const uint4 *>(g_code_lut[table])[i] : make_uint4(0, 0, 0, 0);
 }
 
 // Table index of v given sc = (1/absmax) * kCodeBins/2: the fused multiply-add
@@ -223,15 +233,16 @@ template <typename TW>
 __global__ void __launch_bounds__(kQuantThreads, kQuantCtasPerSm) nf4_quantize_kernel(const TW *__restrict__ W, int64_t numel,
                                                                     uint8_t *__restrict__ codes,
                                                                     float *__restrict__ c2,
-                                                                    double *__restrict__ partial) {
+                                                                    double *__restrict__ partial, int table) {
   __shared__ double red[kQuantThreads / 32];
   __shared__ float thr[16];
   __shared__ __align__(16) uint8_t lut[kCodeLutSpan];
   NF4Thresholds th;
-  th.init();
+  th.init(table);
   if (threadIdx.x < 15)
-    thr[threadIdx.x] = __double2float_rd(((double)kNF4[threadIdx.x] + (double)kNF4[threadIdx.x + 1]) * 0.5);
-  load_code_lut(lut);
+    thr[threadIdx.x] =
+        __double2float_rd(((double)kLevels[table][threadIdx.x] + (double)kLevels[table][threadIdx.x + 1]) * 0.5);
+  load_code_lut(lut, table);
   __syncthreads();
   pdl_trigger();
   pdl_wait();
@@ -403,9 +414,9 @@ __global__ void __launch_bounds__(256) nf4_dequant_kernel(const uint8_t *__restr
                                                           const uint8_t *__restrict__ c2_fp8,
                                                           const float *__restrict__ c1,
                                                           const float *__restrict__ mu_p, int64_t numel,
-                                                          __nv_bfloat16 *__restrict__ out) {
+                                                          __nv_bfloat16 *__restrict__ out, int table) {
   __shared__ float lut[16];
-  if (threadIdx.x < 16) lut[threadIdx.x] = kNF4[threadIdx.x];
+  if (threadIdx.x < 16) lut[threadIdx.x] = kLevels[table][threadIdx.x];
   __syncthreads();
   pdl_trigger();
   pdl_wait();

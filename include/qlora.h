@@ -85,7 +85,19 @@ typedef struct {
   const uint8_t *c2_fp8;  /* [nblk] OCP E4M3 code of (c2_b - mean) / c1               */
   const float *c1;        /* [n1] second-level constants: absmax(c2 - mean) / 448    */
   const float *c2_mean;   /* [1] mean of the first-level constants c2                 */
+  int32_t table;          /* the 16-level code table: QLORA_TABLE_NF4 (0, the default
+                             of a zero-initialised struct) or QLORA_TABLE_FP4        */
 } qlora_nf4dq_t;
+
+/* 16-level code tables (code order; code 7 is the exact zero of both):
+ *   QLORA_TABLE_NF4  the NF4 levels of Appendix E;
+ *   QLORA_TABLE_FP4  FP4 (E2M1), the 4-bit float of §4 (Tables 2-4) that NF4
+ *                    is compared against: {0, 0.5, 1, 1.5, 2, 3, 4, 6} and
+ *                    their negatives divided by 6 (float32 quotients), with
+ *                    both zero codes holding +0.  Blocking, Double
+ *                    Quantization and doubleDequant are the same for both. */
+#define QLORA_TABLE_NF4 0
+#define QLORA_TABLE_FP4 1
 
 /* ---- quantizer -------------------------------------------------------------- */
 
@@ -107,6 +119,12 @@ QLORA_API size_t qlora_quantize_workspace_size(int64_t numel);
  *   Outputs: codes [ceil(n/2)], c2_fp8 [nblk], c1 [n1], c2_mean [1].
  *   Any n_out, k_in >= 0 (a final partial block uses only its real elements).
  */
+/* The same quantizer with the code table chosen by `table` (QLORA_TABLE_*);
+ * qlora_quantize_nf4_dq is table QLORA_TABLE_NF4.  Returns
+ * QLORA_ERR_INVALID_ARG for an unknown table. */
+QLORA_API int qlora_quantize_4bit_dq(const void *W, int w_dtype, int64_t n_out, int64_t k_in, int table,
+                                     uint8_t *codes, uint8_t *c2_fp8, float *c1, float *c2_mean, void *ws,
+                                     size_t ws_bytes, void *stream);
 QLORA_API int qlora_quantize_nf4_dq(const void *W, int w_dtype, int64_t n_out, int64_t k_in, uint8_t *codes,
                           uint8_t *c2_fp8, float *c1, float *c2_mean, void *ws, size_t ws_bytes, void *stream);
 
