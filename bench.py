@@ -576,7 +576,7 @@ def run_quantizer(args, rank, world, local_rank):
     nbytes_q = nbytes_d = 0
     for i, lin in enumerate(wl.linears):
         W = inputs.device_weight_with_outliers(lin.n_out, lin.k_in, wl.seed + 1000 * rank + i, dev)
-        q = qlora.quantize_nf4_dq(W)
+        q = qlora.quantize_nf4_dq(W, table=args.table)
         out = torch.empty_like(W)
         mats.append((W, q, out))
         nbytes_q += W.numel() * 2 + q.nbytes()
@@ -585,13 +585,24 @@ def run_quantizer(args, rank, world, local_rank):
 
     def step():
         for W, q, out in mats:
-            qlora.quantize_nf4_dq(W, out=q)
+            qlora.quantize_nf4_dq(W, out=q, table=args.table)
         for W, q, out in mats:
             qlora.dequant(q, out=out)
 
     ms, launches, clocks = _timed(qlora, step, args, dev, world, rank, local_rank)
     if rank != 0:
         return None
+    # Accuracy of the storage format (outside the timed region): RMS error of
+    # the dequantized weights against the originals, relative to their RMS,
+    # for both code tables on the same weights (the comparison of §4).
+    accuracy = {}
+    for t in ("nf4", "fp4"):
+        se = sq = 0.0
+        for W, _, _ in mats:
+            wh = qlora.dequant(qlora.quantize_nf4_dq(W, table=t)).float()
+            se += float((wh - W.float()).square().sum())
+            sq += float(W.float().square().sum())
+        accuracy[f"{t}_rel_rms_error"] = (se / sq) ** 0.5
     peaks, peak_src = load_peaks()
     per_kind, kernels = _kernel_table(launches, args.steps)
     peak = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
@@ -601,10 +612,11 @@ def run_quantizer(args, rank, world, local_rank):
     roof_q = nbytes_q * args.steps / (q_ms * 1e-3) / 1e9 if q_ms else None
     roof_d = nbytes_d * args.steps / (dk[1] * 1e-3) / 1e9 if dk[1] else None
     return {
-        "metric": "NF4+DQ quantize + dequantize GB/s", "value": (nbytes_q + nbytes_d) * world / (ms * 1e-3) / 1e9,
+        "metric": ("NF4" if args.table == "nf4" else "FP4 (E2M1)") + "+DQ quantize + dequantize GB/s", "value": (nbytes_q + nbytes_d) * world / (ms * 1e-3) / 1e9,
         "unit": "GB/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "u8", "data": "synthetic",
-        "config": {"workload": wl.name, "params": sum(l.n_out * l.k_in for l in wl.linears),
+        "config": {"workload": wl.name + ("" if args.table == "nf4" else "-fp4"),
+                   "code_table": args.table, "params": sum(l.n_out * l.k_in for l in wl.linears),
                    "bytes_quantize": nbytes_q, "bytes_dequant": nbytes_d,
                    "l2": "weights (667 MB bf16) larger than L2, no flush"},
         "gpu_launches": len(launches),
@@ -612,6 +624,7 @@ def run_quantizer(args, rank, world, local_rank):
                      "achieved": roof_q, "achieved_dequant": roof_d, "peak": peak, "unit": "GB/s",
                      "frac": roof_q / peak if roof_q else None, "frac_dequant": roof_d / peak if roof_d else None,
                      "traffic": None, "peak_source": f"{peak_src} hbm_gbs"},
+        "accuracy": accuracy,
         "kernels": kernels, "clocks": clocks,
     }
 
@@ -704,6 +717,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end (host buffers) measurement")
+    ap.add_argument("--table", choices=["nf4", "fp4"], default="nf4",
+                    help="4-bit code table of the quantizer workload (fp4: FP4 E2M1, compared against NF4)")
     ap.add_argument("--dropout", type=float, default=0.0,
                     help="LoRA dropout probability on every adapter (single-layer training workloads)")
     ap.add_argument("--tokens", type=int, default=None,
