@@ -149,6 +149,7 @@ class Linear:
         self.dX = torch.empty(M, K, dtype=torch.bfloat16, device=dev)
         self.q = None
         self.mask = None
+        self.Xm = None         # masked adapter input, saved by the forward (LoRA dropout)
 
 
 def device_dropout_mask(M, K, p, seed, dev):
@@ -190,12 +191,13 @@ def make_step(qlora, lins, grads, world, wl=WL, dropout=0.0):
                 ready(l.X)
                 if l.mask is not None:
                     ready(l.mask)
-            qlora.linear_fwd(l.X, l.q, l.L1, l.L2, wl.s, Y=l.Y, T=l.T, dropout_mask=l.mask, dropout_p=dropout)
+            qlora.linear_fwd(l.X, l.q, l.L1, l.L2, wl.s, Y=l.Y, T=l.T, dropout_mask=l.mask, dropout_p=dropout,
+                             Xm=l.Xm)
         for l in reversed(lins):
             if ready:
                 ready(l.dY)
             qlora.linear_bwd(l.dY, l.X, l.T, l.q, l.L1, l.L2, wl.s, grad_dtype=torch.float32,
-                             dX=l.dX, dL1=l.dL1, dL2=l.dL2, dropout_mask=l.mask, dropout_p=dropout)
+                             dX=l.dX, dL1=l.dL1, dL2=l.dL2, dropout_mask=l.mask, dropout_p=dropout, Xm=l.Xm)
         grads.allreduce()
     return step
 
@@ -286,6 +288,7 @@ def run_ours(args, rank, world, local_rank):
         if args.dropout > 0:
             for i, l in enumerate(lins):
                 l.mask = device_dropout_mask(wl.M, l.lin.k_in, args.dropout, wl.seed + 1000 * rank + 50 + i, dev)
+                l.Xm = torch.empty_like(l.X)
         # copy order for the end-to-end run: the step's first read of each input
         # (with dropout each linear's keep mask right after its input)
         if args.dropout > 0:

@@ -170,14 +170,15 @@ def _mask_arg(mask: torch.Tensor, M: int, K: int, dev) -> torch.Tensor:
 
 def linear_fwd(X: torch.Tensor, q: NF4Tensor, L1: torch.Tensor, L2: torch.Tensor, s: float,
                save_T: bool = True, Y: torch.Tensor | None = None, T: torch.Tensor | None = None,
-               dropout_mask: torch.Tensor | None = None, dropout_p: float = 0.0):
+               dropout_mask: torch.Tensor | None = None, dropout_p: float = 0.0, Xm: torch.Tensor | None = None):
     """Y = X doubleDequant(W)^T + s X L1 L2 (Eq. 3 / Eq. 5).  Returns (Y, T or None).
 
     X [M, K] bf16, L1 [K, r] bf16, L2 [r, N] bf16.  T [M, 2r] bf16 holds
     T = s X L1 as a hi/lo pair: T ~= T[:, :r] + T[:, r:] (see ``t_value``).
     With ``dropout_mask`` (keep bits, 32-bit words [M, K/32], element 32 w + b
     in bit b of word w) LoRA dropout acts on the adapter input:
-    T = s (X * m / (1 - dropout_p)) L1.
+    T = s (X * m / (1 - dropout_p)) L1; ``Xm`` ([M, K] bf16, optional)
+    receives the masked input X * m for the backward.
     """
     lib = _lib.load()
     M, K = X.shape
@@ -195,7 +196,8 @@ def linear_fwd(X: torch.Tensor, q: NF4Tensor, L1: torch.Tensor, L2: torch.Tensor
         ws = _WS.get(lib.qlora_linear_fwd_dropout_workspace_size(M, N, K, r), dev)
         _lib.check(lib.qlora_linear_fwd_dropout(_ptr(_bits(X)), M, q.as_struct(), _ptr(_bits(L1)), _ptr(_bits(L2)), r,
                                                 float(s), _ptr(dropout_mask), float(dropout_p), _ptr(_bits(Y)),
-                                                _ptr(T) if save_T else None, _ptr(ws), ws.numel(), _stream(dev)),
+                                                _ptr(T) if save_T else None, _ptr(Xm), _ptr(ws), ws.numel(),
+                                                _stream(dev)),
                    "qlora_linear_fwd_dropout")
         return Y, (T if save_T else None)
     ws_bytes = lib.qlora_linear_fwd_workspace_size(M, N, K, r)
@@ -215,11 +217,12 @@ def t_value(T: torch.Tensor) -> torch.Tensor:
 def linear_bwd(dY: torch.Tensor, X: torch.Tensor, T: torch.Tensor | None, q: NF4Tensor, L1: torch.Tensor,
                L2: torch.Tensor, s: float, need_dX: bool = True, grad_dtype=torch.bfloat16,
                dX: torch.Tensor | None = None, dL1: torch.Tensor | None = None, dL2: torch.Tensor | None = None,
-               dropout_mask: torch.Tensor | None = None, dropout_p: float = 0.0):
+               dropout_mask: torch.Tensor | None = None, dropout_p: float = 0.0, Xm: torch.Tensor | None = None):
     """Adapter-only backward.  Returns (dX or None, dL1 [K, r], dL2 [r, N]).
 
     With ``dropout_mask`` (the forward's mask) the adapter path goes through
     the mask: dX = dY W_hat + (G L1^T) m / (1 - p), dL1 = drop(X)^T G.
+    ``Xm`` is the forward's masked input (recomputed from X and the mask if None).
     """
     lib = _lib.load()
     M, N = dY.shape
@@ -243,7 +246,7 @@ def linear_bwd(dY: torch.Tensor, X: torch.Tensor, T: torch.Tensor | None, q: NF4
     if dropout_mask is not None:
         _mask_arg(dropout_mask, M, K, dev)
         ws = _WS.get(lib.qlora_linear_bwd_dropout_workspace_size(M, N, K, r), dev)
-        _lib.check(lib.qlora_linear_bwd_dropout(_ptr(_bits(dY)), _ptr(_bits(X)), _ptr(T), M, q.as_struct(),
+        _lib.check(lib.qlora_linear_bwd_dropout(_ptr(_bits(dY)), _ptr(_bits(X)), _ptr(T), _ptr(Xm), M, q.as_struct(),
                                                 _ptr(_bits(L1)), _ptr(_bits(L2)), r, float(s), _ptr(dropout_mask),
                                                 float(dropout_p), _ptr(dX) if need_dX else None, _ptr(dL1),
                                                 _ptr(dL2), gdt, _ptr(ws), ws.numel(), _stream(dev)),

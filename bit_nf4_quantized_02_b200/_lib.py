@@ -75,10 +75,11 @@ SIGNATURES = {
     "qlora_linear_fwd_dropout_workspace_size": (c_size_t, [c_int64, c_int64, c_int64, c_int]),
     "qlora_linear_bwd_dropout_workspace_size": (c_size_t, [c_int64, c_int64, c_int64, c_int]),
     "qlora_linear_fwd_dropout": (c_int, [c_void_p, c_int64, POINTER(NF4DQ), c_void_p, c_void_p, c_int, c_float,
-                                         c_void_p, c_float, c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]),
-    "qlora_linear_bwd_dropout": (c_int, [c_void_p, c_void_p, c_void_p, c_int64, POINTER(NF4DQ), c_void_p, c_void_p,
-                                         c_int, c_float, c_void_p, c_float, c_void_p, c_void_p, c_void_p, c_int,
-                                         c_void_p, c_size_t, c_void_p]),
+                                         c_void_p, c_float, c_void_p, c_void_p, c_void_p, c_void_p, c_size_t,
+                                         c_void_p]),
+    "qlora_linear_bwd_dropout": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_int64, POINTER(NF4DQ), c_void_p,
+                                         c_void_p, c_int, c_float, c_void_p, c_float, c_void_p, c_void_p, c_void_p,
+                                         c_int, c_void_p, c_size_t, c_void_p]),
 }
 
 _lib = None

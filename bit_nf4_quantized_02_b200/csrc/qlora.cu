@@ -1057,14 +1057,14 @@ size_t qlora_linear_bwd_dropout_workspace_size(int64_t M, int64_t n_out, int64_t
 
 int qlora_linear_fwd_dropout(const uint16_t *X, int64_t M, const qlora_nf4dq_t *W, const uint16_t *L1,
                              const uint16_t *L2, int r, float s, const uint32_t *mask, float p, uint16_t *Y,
-                             uint16_t *T_save, void *ws, size_t ws_bytes, void *stream) {
+                             uint16_t *T_save, uint16_t *Xm_save, void *ws, size_t ws_bytes, void *stream) {
   int rc = check_linear(M, W, r);
   if (rc) return rc;
   if (!(p >= 0.f && p < 1.f)) return QLORA_ERR_INVALID_ARG;
   if (M == 0) return QLORA_OK;
   if (!X || !L1 || !L2 || !Y || !mask) return QLORA_ERR_INVALID_ARG;
   if (!aligned(X, 16) || !aligned(L1, 16) || !aligned(L2, 16) || !aligned(Y, 16) || !aligned(mask, 16) ||
-      (T_save && !aligned(T_save, 16)))
+      (T_save && !aligned(T_save, 16)) || (Xm_save && !aligned(Xm_save, 16)))
     return QLORA_ERR_MISALIGNED;
   DeviceInfo *dev;
   rc = current_device_info(&dev);
@@ -1075,16 +1075,16 @@ int qlora_linear_fwd_dropout(const uint16_t *X, int64_t M, const qlora_nf4dq_t *
   if (!ws || ws_bytes < qlora_linear_fwd_dropout_workspace_size(M, N, K, r)) return QLORA_ERR_WORKSPACE;
   if (!aligned(ws, 256)) return QLORA_ERR_MISALIGNED;
   uint8_t *w8 = reinterpret_cast<uint8_t *>(ws);
-  uint16_t *Xm = reinterpret_cast<uint16_t *>(w8 + L.total);
+  uint16_t *Xm = Xm_save ? Xm_save : reinterpret_cast<uint16_t *>(w8 + L.total);
   rc = dropout_launch(X, mask, M * K, Xm, dev, st);
   if (rc) return rc;
   return fwd_large(X, Xm, s / (1.f - p), M, W, L1, L2, r, Y, T_save, w8, L, dev, st);
 }
 
-int qlora_linear_bwd_dropout(const uint16_t *dY, const uint16_t *X, const uint16_t *T_saved, int64_t M,
-                             const qlora_nf4dq_t *W, const uint16_t *L1, const uint16_t *L2, int r, float s,
-                             const uint32_t *mask, float p, uint16_t *dX, void *dL1, void *dL2, int grad_dtype,
-                             void *ws, size_t ws_bytes, void *stream) {
+int qlora_linear_bwd_dropout(const uint16_t *dY, const uint16_t *X, const uint16_t *T_saved,
+                             const uint16_t *Xm_saved, int64_t M, const qlora_nf4dq_t *W, const uint16_t *L1,
+                             const uint16_t *L2, int r, float s, const uint32_t *mask, float p, uint16_t *dX,
+                             void *dL1, void *dL2, int grad_dtype, void *ws, size_t ws_bytes, void *stream) {
   int rc = check_linear(M, W, r);
   if (rc) return rc;
   if (!(p >= 0.f && p < 1.f)) return QLORA_ERR_INVALID_ARG;
@@ -1093,7 +1093,7 @@ int qlora_linear_bwd_dropout(const uint16_t *dY, const uint16_t *X, const uint16
   if (M > 0 && (!dY || !X || !mask)) return QLORA_ERR_INVALID_ARG;
   if (!aligned(L1, 16) || !aligned(L2, 16) || !aligned(dL1, 16) || !aligned(dL2, 16) || (dY && !aligned(dY, 16)) ||
       (X && !aligned(X, 16)) || (dX && !aligned(dX, 16)) || (T_saved && !aligned(T_saved, 16)) ||
-      (mask && !aligned(mask, 16)))
+      (mask && !aligned(mask, 16)) || (Xm_saved && !aligned(Xm_saved, 16)))
     return QLORA_ERR_MISALIGNED;
   DeviceInfo *dev;
   rc = current_device_info(&dev);
@@ -1110,10 +1110,14 @@ int qlora_linear_bwd_dropout(const uint16_t *dY, const uint16_t *X, const uint16
   if (!ws || ws_bytes < qlora_linear_bwd_dropout_workspace_size(M, N, K, r)) return QLORA_ERR_WORKSPACE;
   if (!aligned(ws, 256)) return QLORA_ERR_MISALIGNED;
   uint8_t *w8 = reinterpret_cast<uint8_t *>(ws);
-  uint16_t *Xm = reinterpret_cast<uint16_t *>(w8 + L.total);
   uint16_t *Z = reinterpret_cast<uint16_t *>(w8 + L.total + align_up((size_t)M * K * 2));
-  rc = dropout_launch(X, mask, M * K, Xm, dev, st);
-  if (rc) return rc;
+  const uint16_t *Xm = Xm_saved;
+  if (!Xm) {   // recompute the masked input
+    uint16_t *Xw = reinterpret_cast<uint16_t *>(w8 + L.total);
+    rc = dropout_launch(X, mask, M * K, Xw, dev, st);
+    if (rc) return rc;
+    Xm = Xw;
+  }
   const BwdDropout drop = {Xm, 1.f / (1.f - p), mask, Z};
   return bwd_large(dY, X, T_saved, M, W, L1, L2, r, s, dX, dL1, dL2, grad_dtype == QLORA_DTYPE_F32, w8, L, &drop,
                    dev, st);

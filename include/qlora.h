@@ -215,9 +215,12 @@ QLORA_API int qlora_linear_bwd(const uint16_t *dY, const uint16_t *X, const uint
  * elements of X, bit b of word w keeping element 32 w + b (so [M x K/32]
  * words, 16-byte aligned; the same mask must be passed to the forward and
  * the backward of a step).  0 <= p < 1; p = 0 with an all-ones mask computes
- * the plain linear.  Other arguments, layouts and T_save are those of
- * qlora_linear_fwd / qlora_linear_bwd.  Every token count takes the
- * dequant + tensor-core path.  Workspace: *_dropout_workspace_size().
+ * the plain linear.  Xm_save [M x K] bf16 (out, may be NULL) receives the
+ * masked input X * m; passing it back as Xm_saved spares the backward its
+ * recomputation (NULL: recomputed from X and the mask).  Other arguments,
+ * layouts and T_save are those of qlora_linear_fwd / qlora_linear_bwd.  Every
+ * token count takes the dequant + tensor-core path.  Workspace:
+ * *_dropout_workspace_size().
  * Errors: as qlora_linear_fwd / _bwd, plus QLORA_ERR_INVALID_ARG for a NULL
  * mask (M > 0) or p outside [0, 1).
  */
@@ -225,11 +228,13 @@ QLORA_API size_t qlora_linear_fwd_dropout_workspace_size(int64_t M, int64_t n_ou
 QLORA_API size_t qlora_linear_bwd_dropout_workspace_size(int64_t M, int64_t n_out, int64_t k_in, int r);
 QLORA_API int qlora_linear_fwd_dropout(const uint16_t *X, int64_t M, const qlora_nf4dq_t *W, const uint16_t *L1,
                                        const uint16_t *L2, int r, float s, const uint32_t *mask, float p,
-                                       uint16_t *Y, uint16_t *T_save, void *ws, size_t ws_bytes, void *stream);
-QLORA_API int qlora_linear_bwd_dropout(const uint16_t *dY, const uint16_t *X, const uint16_t *T_saved, int64_t M,
-                                       const qlora_nf4dq_t *W, const uint16_t *L1, const uint16_t *L2, int r,
-                                       float s, const uint32_t *mask, float p, uint16_t *dX, void *dL1, void *dL2,
-                                       int grad_dtype, void *ws, size_t ws_bytes, void *stream);
+                                       uint16_t *Y, uint16_t *T_save, uint16_t *Xm_save, void *ws, size_t ws_bytes,
+                                       void *stream);
+QLORA_API int qlora_linear_bwd_dropout(const uint16_t *dY, const uint16_t *X, const uint16_t *T_saved,
+                                       const uint16_t *Xm_saved, int64_t M, const qlora_nf4dq_t *W,
+                                       const uint16_t *L1, const uint16_t *L2, int r, float s, const uint32_t *mask,
+                                       float p, uint16_t *dX, void *dL1, void *dL2, int grad_dtype, void *ws,
+                                       size_t ws_bytes, void *stream);
 
 /* ---- diagnostics ----------------------------------------------------------------- */
 

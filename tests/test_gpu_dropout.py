@@ -33,14 +33,17 @@ def _run(W, X, L1, L2, dY, words, s, p, grad_dtype=torch.float32):
     q = qlora.quantize_nf4_dq(W.cuda())
     mask = torch.from_numpy(words.view(np.int32)).cuda()
     Xd, L1d, L2d, dYd = X.cuda(), L1.cuda(), L2.cuda(), dY.cuda()
-    Y, T = qlora.linear_fwd(Xd, q, L1d, L2d, s, dropout_mask=mask, dropout_p=p)
+    Xm = torch.empty_like(Xd)
+    Y, T = qlora.linear_fwd(Xd, q, L1d, L2d, s, dropout_mask=mask, dropout_p=p, Xm=Xm)
     dX, dL1, dL2 = qlora.linear_bwd(dYd, Xd, T, q, L1d, L2d, s, grad_dtype=grad_dtype, dropout_mask=mask,
-                                    dropout_p=p)
-    # the backward also recomputes T when none is saved
+                                    dropout_p=p, Xm=Xm)
+    # the backward also recomputes T and the masked input when none is saved
     _, dL1b, dL2b = qlora.linear_bwd(dYd, Xd, None, q, L1d, L2d, s, need_dX=False, grad_dtype=grad_dtype,
                                      dropout_mask=mask, dropout_p=p)
     torch.cuda.synchronize()
     assert qlora.last_device_error() == 0
+    keep = torch.from_numpy(inputs.unpack_mask(words, X.shape[1])).cuda()
+    assert torch.equal(Xm.view(torch.int16), torch.where(keep, Xd, torch.zeros_like(Xd)).view(torch.int16))
     return q, Y, T, dX, dL1, dL2, dL1b, dL2b
 
 
