@@ -28,7 +28,7 @@ struct DeviceInfo {
   int sms = 0;
   int *err = nullptr;        // device address of g_dev_err
   bool gemm_attr[16] = {};   // [wide][fold][BN 64/128/256 or 3 = pair]: shared-memory limit set
-  int pair_clusters[2] = {0, 0};   // co-resident 2-CTA clusters of the pair GEMM [wide]
+  int pair_clusters[3] = {0, 0, 0};   // co-resident 2-CTA clusters of the pair GEMM [form]
   int gemv_smem_set[3] = {0, 0, 0};   // dynamic smem limit set per NT variant
   int gemv_per_sm[3] = {0, 0, 0};     // resident CTAs per SM per NT variant
   int fused_smem_set[4] = {0, 0, 0, 0};   // dynamic smem limit set per token-padding variant
@@ -263,11 +263,11 @@ int launch_gemm_bn(const CUtensorMap *maps, TcGemmArgs &args, int sms, DeviceInf
 
 // CTA-pair GEMM (256 x 256 tiles): a persistent grid of 2-CTA clusters, as
 // many as can be resident at once.
-template <bool WIDE>
+template <bool WIDE, bool DROPZ = false>
 int launch_gemm_pair(const CUtensorMap *maps, TcGemmArgs &args, DeviceInfo *dev, cudaStream_t st, int kind) {
   constexpr int BN = 256;
   using Cfg = TcCfg<BN, true, WIDE>;
-  auto kernel = tc_gemm_kernel<BN, true, false, WIDE>;
+  auto kernel = tc_gemm_kernel<BN, true, false, WIDE, DROPZ>;
   cudaLaunchConfig_t cfg;
   std::memset(&cfg, 0, sizeof(cfg));
   cudaLaunchAttribute attr[2];
@@ -282,18 +282,19 @@ int launch_gemm_pair(const CUtensorMap *maps, TcGemmArgs &args, DeviceInfo *dev,
   cfg.stream = st;
   cfg.attrs = attr;
   cfg.numAttrs = 1;   // the occupancy query takes the cluster shape alone
-  const int idx = 3 + (WIDE ? 8 : 0);
+  const int form = DROPZ ? 2 : (WIDE ? 1 : 0);
+  const int idx = DROPZ ? 15 : 3 + (WIDE ? 8 : 0);
   if (!dev->gemm_attr[idx]) {
     if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes) != cudaSuccess)
       return QLORA_ERR_CUDA;
     cfg.gridDim = dim3(2 * (unsigned)dev->sms, 1, 1);
     int clusters = 0;
     if (cudaOccupancyMaxActiveClusters(&clusters, kernel, &cfg) != cudaSuccess || clusters < 1) return QLORA_ERR_CUDA;
-    dev->pair_clusters[WIDE ? 1 : 0] = clusters;
+    dev->pair_clusters[form] = clusters;
     dev->gemm_attr[idx] = true;
   }
   const int units = args.m_tiles * args.n_tiles * args.splits;
-  const int clusters = std::max(1, std::min(units, dev->pair_clusters[WIDE ? 1 : 0]));
+  const int clusters = std::max(1, std::min(units, dev->pair_clusters[form]));
   cfg.gridDim = dim3(2 * (unsigned)clusters, 1, 1);
   cfg.numAttrs = g_prof.on ? 1 : 2;   // a programmatic dependent of the previous kernel, unless the event log records
   ProfScope prof(kind, st);
@@ -314,8 +315,11 @@ int tc_gemm(cudaStream_t st, DeviceInfo *dev, int64_t M, int64_t N, int nseg, co
             void *out, int64_t ld_row, int64_t ld_col, int out_f32, float *split_ws, int kind, int64_t lo_off = 0,
             bool split_all = false, int fold = 0, const GemmAddend *add = nullptr) {
   if (M <= 0 || N <= 0) return QLORA_OK;
-  // the addend is applied by the direct bf16 epilogue only
+  // the addend is applied by the direct bf16 epilogue only; add->z == nullptr
+  // asks for segment 1 as the masked term (the pair form's second accumulator)
   if (add && (split_ws || out_f32 || fold || N % 32)) return QLORA_ERR_UNSUPPORTED_SHAPE;
+  const bool dropz = add && !add->z;
+  if (dropz && nseg != 2) return QLORA_ERR_UNSUPPORTED_SHAPE;
   if (M > (int64_t)INT32_MAX / 2 || N > (int64_t)INT32_MAX / 2) return QLORA_ERR_UNSUPPORTED_SHAPE;
   const int bn = pick_bn(N);
   CUtensorMap maps[4];
@@ -376,7 +380,10 @@ int tc_gemm(cudaStream_t st, DeviceInfo *dev, int64_t M, int64_t N, int nseg, co
     a.out_f32 = out_f32;
   }
   int rc;
-  if (pair) {
+  if (dropz) {
+    if (!pair || !wide) return QLORA_ERR_UNSUPPORTED_SHAPE;
+    rc = launch_gemm_pair<true, true>(maps, a, dev, st, kind);
+  } else if (pair) {
     rc = wide ? launch_gemm_pair<true>(maps, a, dev, st, kind) : launch_gemm_pair<false>(maps, a, dev, st, kind);
   } else if (fold) {
     switch (bn) {
@@ -916,14 +923,24 @@ int bwd_large(const uint16_t *dY, const uint16_t *X, const uint16_t *T_saved, in
       GemmSeg sX[2] = {{{dY, M, N, N, 0}, {w_hat, K, N, K, 1}}, {{G, M, r, 2 * r, 0}, {L1, K, r, r, 0}}};
       rc = tc_gemm(st, dev, M, K, 2, sX, 1.f, dX, K, 1, 0, nullptr, QLORA_KERNEL_GEMM_DX);
     } else {
-      // With dropout the adapter term is gated by the mask: Z = G_hi L1^T
-      // first, then dX = dY W_hat + keep * m * Z, added before the rounding.
-      GemmSeg sZ = {{G, M, r, 2 * r, 0}, {L1, K, r, r, 0}};
-      rc = tc_gemm(st, dev, M, K, 1, &sZ, 1.f, drop->Z, K, 1, 0, nullptr, QLORA_KERNEL_GEMM_Z);
-      if (rc) return rc;
-      GemmSeg sX = {{dY, M, N, N, 0}, {w_hat, K, N, K, 1}};
-      const GemmAddend add = {drop->Z, drop->mask, keep, K};
-      rc = tc_gemm(st, dev, M, K, 1, &sX, 1.f, dX, K, 1, 0, nullptr, QLORA_KERNEL_GEMM_DX, 0, false, 0, &add);
+      // With dropout the adapter term is gated by the mask.  When dX runs in
+      // the wide pair form, G_hi L1^T accumulates in the tile's second TMEM
+      // accumulator and the epilogue stores D0 + keep * m * D1.  Otherwise
+      // Z = G_hi L1^T first, then dX = dY W_hat + keep * m * Z, added before
+      // the rounding.
+      const bool in_tile = M > kBM && K > 128 && N >= 128 && N % 64 == 0;
+      if (in_tile) {
+        GemmSeg sX[2] = {{{dY, M, N, N, 0}, {w_hat, K, N, K, 1}}, {{G, M, r, 2 * r, 0}, {L1, K, r, r, 0}}};
+        const GemmAddend add = {nullptr, drop->mask, keep, K};
+        rc = tc_gemm(st, dev, M, K, 2, sX, 1.f, dX, K, 1, 0, nullptr, QLORA_KERNEL_GEMM_DX, 0, false, 0, &add);
+      } else {
+        GemmSeg sZ = {{G, M, r, 2 * r, 0}, {L1, K, r, r, 0}};
+        rc = tc_gemm(st, dev, M, K, 1, &sZ, 1.f, drop->Z, K, 1, 0, nullptr, QLORA_KERNEL_GEMM_Z);
+        if (rc) return rc;
+        GemmSeg sX = {{dY, M, N, N, 0}, {w_hat, K, N, K, 1}};
+        const GemmAddend add = {drop->Z, drop->mask, keep, K};
+        rc = tc_gemm(st, dev, M, K, 1, &sX, 1.f, dX, K, 1, 0, nullptr, QLORA_KERNEL_GEMM_DX, 0, false, 0, &add);
+      }
     }
     if (rc) return rc;
   }

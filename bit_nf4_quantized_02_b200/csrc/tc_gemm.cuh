@@ -170,7 +170,11 @@ __device__ __forceinline__ void tc_seg_range(const TcGemmArgs &p, int s, int spl
   }
 }
 
-template <int BN, bool PAIR = false, bool FOLD = false, bool WIDE = false>
+// DROPZ (LoRA dropout in dX, pair form): segment 1 (the adapter term) goes
+// into the tile's second accumulator instead of the first, and the epilogue
+// stores alpha * D0 + add_scale * m * D1 with the keep mask m (add_mask).
+// The two accumulators then serve one tile, so tiles do not overlap.
+template <int BN, bool PAIR = false, bool FOLD = false, bool WIDE = false, bool DROPZ = false>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tA0, const __grid_constant__ CUtensorMap tB0,
                    const __grid_constant__ CUtensorMap tA1, const __grid_constant__ CUtensorMap tB1,
@@ -353,15 +357,20 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       for (int u = first_unit; u < units && ok; u += unit_stride, ++t) {
         int mt, nt, split;
         tc_unit_coords(u, p, mt, nt, split);
-        const int acc = t & 1;
-        const uint32_t use = (uint32_t)(t >> 1);
+        constexpr int kAccs = DROPZ ? 1 : 2;
+        const int acc = t % kAccs;
+        const uint32_t use = (uint32_t)(t / kAccs);
         if (!mbar_wait<PAIR>(smem_u32(tempty_bar + acc), (use & 1u) ^ 1u, p.err, DEV_TIMEOUT_MMA)) break;
         tc_fence_after();
-        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
+        uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
         uint32_t accumulate = 0;
         for (int s = 0; s < p.nseg && ok; ++s) {
           int kb0, kb1;
           tc_seg_range(p, s, split, kb0, kb1);
+          if (DROPZ && s == 1) {   // the adapter term into the second accumulator
+            d_tmem = tmem_base + (uint32_t)BN;
+            accumulate = 0;
+          }
           const int a_mn = p.seg[s].a_mn, b_mn = p.seg[s].b_mn;
           const int step = (WIDE && p.seg[s].wide) ? 2 : 1;
           for (int kb = kb0; kb < kb1; kb += step) {
@@ -419,8 +428,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     for (int u = first_unit; u < units; u += unit_stride, ++t) {
       int mt, nt, split;
       tc_unit_coords(u, p, mt, nt, split);
-      const int acc = t & 1;
-      const uint32_t use = (uint32_t)(t >> 1);
+      constexpr int kAccs = DROPZ ? 1 : 2;
+      const int acc = t % kAccs;
+      const uint32_t use = (uint32_t)(t / kAccs);
       // Warp-uniform wait: tcgen05.ld below must be executed by all 32 lanes.
       const bool got = mbar_wait(smem_u32(tfull_bar + acc), use & 1u, p.err, DEV_TIMEOUT_EPILOGUE);
       if (!__all_sync(0xFFFFFFFFu, got)) break;
@@ -457,6 +467,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       for (int c = 0; c < BN; c += 32) {
         uint32_t r[32];
         tmem_ld_32x32b_x32(tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN + c), r);
+        [[maybe_unused]] uint32_t r2[32];
+        if constexpr (DROPZ) tmem_ld_32x32b_x32(tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(BN + c), r2);
         tmem_wait_ld();
         const int col0 = nt * BN + c;
         if (!row_ok || col0 >= p.N) continue;
@@ -492,7 +504,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           float v[32];
 #pragma unroll
           for (int j = 0; j < 32; ++j) v[j] = alpha * __uint_as_float(r[j]);
-          if (p.add) tc_add_masked(p, row, col0, v);
+          if constexpr (DROPZ) {
+            const uint32_t m = ld_dep_u32(p.add_mask + (((int64_t)row * p.N + col0) >> 5));
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              if ((m >> j) & 1u) v[j] += p.add_scale * __uint_as_float(r2[j]);
+          } else if (p.add) {
+            tc_add_masked(p, row, col0, v);
+          }
           if (p.ld_col == 1 && col0 + 32 <= p.N && (p.ld_row & 7) == 0 && (lo & 7) == 0) {
             uint4 *dst = reinterpret_cast<uint4 *>(o + (int64_t)row * p.ld_row + col0);
             uint4 *dst_lo = reinterpret_cast<uint4 *>(o + (int64_t)row * p.ld_row + col0 + lo);
