@@ -85,7 +85,7 @@ struct FtArgs {
   const float *c1;
   const float *mu;
   float *acc;            // [M x N] fp32, zero at launch
-  int table;             // 16-level code table of the weight (kLevels)
+  float levels[16];      // the weight's 16-level code table
   int *err;
 };
 
@@ -359,7 +359,7 @@ __global__ void __launch_bounds__(FtCfg<MP>::kThreads, 1)
         const uint4 qb = lds128(sc + (((uint32_t)(2 * j + 1) << 4) ^ cswz));
         const uint32_t q[8] = {qa.x, qa.y, qa.z, qa.w, qb.x, qb.y, qb.z, qb.w};
         BlockTable tb;
-        tb.build(n < p.N ? ft_c2hat(raw, n, ks * 4, j, kblocks, mu) : 0.f, kLevels[p.table]);
+        tb.build(n < p.N ? ft_c2hat(raw, n, ks * 4, j, kblocks, mu) : 0.f, p.levels);
         // decode the row's 64 weights into registers, then wait for the slot
         uint32_t e[32];
 #pragma unroll

@@ -71,7 +71,7 @@ struct GvArgs {
   const __nv_bfloat16 *L1;   // [K x r]
   const __nv_bfloat16 *L2;   // [r x N]
   float *acc;            // [M x N] fp32, zero at launch
-  int table;             // 16-level code table of the weight (kLevels)
+  float levels[16];      // the weight's 16-level code table
   int *err;
 };
 
@@ -214,8 +214,8 @@ struct GvConsumer {
         for (int t = 0; t < NT; ++t) d[c][t][0] = d[c][t][1] = d[c][t][2] = d[c][t][3] = 0.f;
     }
     BlockTable tb0, tb1;
-    tb0.build(cur.c2hat(0, mu), kLevels[P.table]);
-    tb1.build(cur.c2hat(1, mu), kLevels[P.table]);
+    tb0.build(cur.c2hat(0, mu), P.levels);
+    tb1.build(cur.c2hat(1, mu), P.levels);
     int nu = u, nstn = st + 1;
     if (nstn == nst) {
       nu = u + gridDim.x;

@@ -514,7 +514,7 @@ int launch_fused_fwd(const qlora_nf4dq_t *W, const uint16_t *X, int64_t M, const
   }
   FtArgs a;
   std::memset(&a, 0, sizeof(a));
-  a.table = (int)W->table;
+  std::memcpy(a.levels, kLevelsHost[W->table], sizeof(a.levels));
   a.M = (int)M;
   a.N = (int)N;
   a.K = (int)K;
@@ -576,7 +576,7 @@ int launch_gemv(const qlora_nf4dq_t *W, const uint16_t *X, int64_t M, const uint
     return QLORA_ERR_CUDA;
   GvArgs a;
   std::memset(&a, 0, sizeof(a));
-  a.table = (int)W->table;
+  std::memcpy(a.levels, kLevelsHost[W->table], sizeof(a.levels));
   a.M = (int)M;
   a.N = (int)N;
   a.K = (int)K;

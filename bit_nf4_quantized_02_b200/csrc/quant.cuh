@@ -30,26 +30,30 @@ namespace qlora {
 //     and their negatives divided by 6 (fp32 quotients), both zero codes +0.
 // Code 7 is the exact zero of either table.
 constexpr int kNumTables = 2;
-__constant__ float kLevels[kNumTables][16] = {
-    {-1.0f,
-    -0.6961928009986877f,
-    -0.5250730514526367f,
-    -0.39491748809814453f,
-    -0.28444138169288635f,
-    -0.18477343022823334f,
-    -0.09105003625154495f,
-    0.0f,
-    0.07958029955625534f,
-    0.16093020141124725f,
-    0.24611230194568634f,
-    0.33791524171829224f,
-    0.44070982933044434f,
-    0.5626170039176941f,
-    0.7229568362236023f,
-    1.0f},
-    {-1.0f, -0x1.555556p-1f, -0.5f, -0x1.555556p-2f, -0.25f, -0x1.555556p-3f, -0x1.555556p-4f, 0.0f,
+#define QLORA_LEVEL_TABLES  \
+    {-1.0f, \
+    -0.6961928009986877f, \
+    -0.5250730514526367f, \
+    -0.39491748809814453f, \
+    -0.28444138169288635f, \
+    -0.18477343022823334f, \
+    -0.09105003625154495f, \
+    0.0f, \
+    0.07958029955625534f, \
+    0.16093020141124725f, \
+    0.24611230194568634f, \
+    0.33791524171829224f, \
+    0.44070982933044434f, \
+    0.5626170039176941f, \
+    0.7229568362236023f, \
+    1.0f}, \
+    {-1.0f, -0x1.555556p-1f, -0.5f, -0x1.555556p-2f, -0.25f, -0x1.555556p-3f, -0x1.555556p-4f, 0.0f, \
      0.0f, 0x1.555556p-4f, 0x1.555556p-3f, 0.25f, 0x1.555556p-2f, 0.5f, 0x1.555556p-1f, 1.0f},
-};
+__constant__ float kLevels[kNumTables][16] = {QLORA_LEVEL_TABLES};
+// The same tables on the host, to pass a weight's levels to the decode
+// kernels as launch arguments (constant offsets in the parameter space).
+static const float kLevelsHost[kNumTables][16] = {QLORA_LEVEL_TABLES};
+#undef QLORA_LEVEL_TABLES
 
 constexpr int kQuantThreads = 256;
 constexpr int kQuantCtasPerSm = 5;     // resident at 48 registers per thread
