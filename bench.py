@@ -421,7 +421,7 @@ def run_ours(args, rank, world, local_rank):
                  "copies": ("host->device copies on a copy stream in the order the step first reads them, "
                             "overlapping quantization and compute" if wl.layers == 1 else
                             "host->device copies before the step")} if ms_e2e else None),
-        "gpu_launches": len(launches),
+        "gpu_launches": _kernel_count(launches),
         "roofline": {"bound": "tensor", "kernel": "tc_gemm (Y = X W^T + T L2 and dX = dY W + G L1^T)",
                      "traffic_unit": "bytes per launch (DRAM read + write)",
                      "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
@@ -491,40 +491,17 @@ def _kernel_table(launches, steps):
                       for k, v in sorted(per_kind.items(), key=lambda kv: -kv[1][1])}
 
 
-def run_decode(args, rank, world, local_rank):
-    """LLaMA-65B layer forward at 16 tokens: the memory-bound few-token path."""
-    import bit_nf4_quantized_02_b200 as qlora
-    wl = workloads.LLAMA65B_LAYER
-    M, r, s = args.tokens or wl.extra["M_decode"], wl.r, wl.s
-    dev = torch.device("cuda", local_rank)
-    torch.cuda.set_device(dev)
-    base = wl.seed + 1000 * rank
-    H = inputs.device_normal((M, 8192), 1.0, base + 1, dev, torch.bfloat16)
-    A = inputs.device_normal((M, 8192), 1.0, base + 2, dev, torch.bfloat16)
-    U = inputs.device_normal((M, 22016), 1.0, base + 3, dev, torch.bfloat16)
-    xs = {"q": H, "k": H, "v": H, "o": A, "gate": H, "up": H, "down": U}
-    lins = []
-    nbytes = 0
-    for i, lin in enumerate(wl.linears):
-        N, K = lin.n_out, lin.k_in
-        W = inputs.device_normal((N, K), inputs.WEIGHT_STD, wl.seed + 100 * i, dev)
-        q = qlora.quantize_nf4_dq(W)
-        del W
-        L1 = inputs.device_normal((K, r), 1.0 / np.sqrt(K), wl.seed + 100 * i + 1, dev, torch.bfloat16)
-        L2 = inputs.device_normal((r, N), inputs.L2_STD, wl.seed + 100 * i + 2, dev, torch.bfloat16)
-        Y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
-        T = torch.empty(M, 2 * r, dtype=torch.bfloat16, device=dev)
-        lins.append((xs[lin.name], q, L1, L2, Y, T))
-        # algorithmic bytes: NF4+DQ weight, LoRA factors, X read, Y and T written
-        nbytes += q.nbytes() + 2 * r * (K + N) + 2 * M * K + 2 * M * N + 2 * M * 2 * r
-    torch.cuda.synchronize()
+# Kernels behind one entry of the library's event log: the few-token forward
+# logs its chain (T accumulation, product, epilogue) as one entry.
+KERNELS_PER_ENTRY = {"gemv_fwd": 3, "fused_fwd": 3}
 
-    def step():
-        for X, q, L1, L2, Y, T in lins:
-            qlora.linear_fwd(X, q, L1, L2, s, Y=Y, T=T)
 
-    ms, launches, clocks = _timed(qlora, step, args, dev, world, rank, local_rank)
-    # the same step captured in a CUDA graph (no host launch overhead)
+def _kernel_count(launches) -> int:
+    return sum(KERNELS_PER_ENTRY.get(kind, 1) for kind, _ in launches)
+
+
+def _graph_ms(step, dev, steps):
+    """Per-step ms of ``step`` captured once in a CUDA graph and replayed."""
     g = torch.cuda.CUDAGraph()
     side = torch.cuda.Stream(dev)
     side.wait_stream(torch.cuda.current_stream(dev))
@@ -537,11 +514,83 @@ def run_decode(args, rank, world, local_rank):
         g.replay()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record()
-    for _ in range(args.steps):
+    for _ in range(steps):
         g.replay()
     e1.record()
     torch.cuda.synchronize()
-    ms_graph = e0.elapsed_time(e1) / args.steps
+    return e0.elapsed_time(e1) / steps
+
+
+def _eager_ms(step, steps):
+    for _ in range(3):
+        step()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record()
+    for _ in range(steps):
+        step()
+    e1.record()
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / steps
+
+
+def run_decode(args, rank, world, local_rank):
+    """LLaMA-65B layer forward at 16 tokens: the memory-bound few-token path.
+
+    The seven projections run as the layer's data flow allows: q, k, v, gate
+    and up (which all read the layer input H) as one grouped call, then o
+    (reads the attention output A) and down (reads U).  The line also reports
+    the same step as seven single-linear calls and as one group of all seven.
+    """
+    import bit_nf4_quantized_02_b200 as qlora
+    wl = workloads.LLAMA65B_LAYER
+    M, r, s = args.tokens or wl.extra["M_decode"], wl.r, wl.s
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    base = wl.seed + 1000 * rank
+    H = inputs.device_normal((M, 8192), 1.0, base + 1, dev, torch.bfloat16)
+    A = inputs.device_normal((M, 8192), 1.0, base + 2, dev, torch.bfloat16)
+    U = inputs.device_normal((M, 22016), 1.0, base + 3, dev, torch.bfloat16)
+    xs = {"q": H, "k": H, "v": H, "o": A, "gate": H, "up": H, "down": U}
+    lins, members = [], {}
+    nbytes = 0
+    for i, lin in enumerate(wl.linears):
+        N, K = lin.n_out, lin.k_in
+        W = inputs.device_normal((N, K), inputs.WEIGHT_STD, wl.seed + 100 * i, dev)
+        q = qlora.quantize_nf4_dq(W)
+        del W
+        L1 = inputs.device_normal((K, r), 1.0 / np.sqrt(K), wl.seed + 100 * i + 1, dev, torch.bfloat16)
+        L2 = inputs.device_normal((r, N), inputs.L2_STD, wl.seed + 100 * i + 2, dev, torch.bfloat16)
+        Y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+        T = torch.empty(M, 2 * r, dtype=torch.bfloat16, device=dev)
+        lins.append((xs[lin.name], q, L1, L2, Y, T))
+        members[lin.name] = {"X": xs[lin.name], "q": q, "L1": L1, "L2": L2, "s": s, "Y": Y, "T": T}
+        # algorithmic bytes: NF4+DQ weight, LoRA factors, X read, Y and T written
+        nbytes += q.nbytes() + 2 * r * (K + N) + 2 * M * K + 2 * M * N + 2 * M * 2 * r
+    torch.cuda.synchronize()
+    groups = [[members[n] for n in ("q", "k", "v", "gate", "up")], [members["o"]], [members["down"]]]
+    everything = [members[l.name] for l in wl.linears]
+
+    def step():                       # the layer's data flow: three grouped calls
+        for grp in groups:
+            qlora.linear_fwd_group(grp)
+
+    def step_single():                # seven single-linear calls
+        for X, q, L1, L2, Y, T in lins:
+            qlora.linear_fwd(X, q, L1, L2, s, Y=Y, T=T)
+
+    def step_one_group():             # all seven in one launch chain
+        qlora.linear_fwd_group(everything)
+
+    ms, launches, clocks = _timed(qlora, step, args, dev, world, rank, local_rank)
+    ms_graph = _graph_ms(step, dev, args.steps)
+    variants = {}
+    for name, fn in (("seven_single_calls", step_single), ("one_group_of_seven", step_one_group)):
+        e, gms = _eager_ms(fn, args.steps), _graph_ms(fn, dev, args.steps)
+        variants[name] = {"ms_per_step": e, "value": nbytes / (e * 1e-3) / 1e9, "graph_ms_per_step": gms,
+                          "graph_value": nbytes / (gms * 1e-3) / 1e9}
+    if qlora.last_device_error() != 0:
+        raise RuntimeError("device error in the decode variants")
     if rank != 0:
         return None
     peaks, peak_src = load_peaks()
@@ -549,16 +598,21 @@ def run_decode(args, rank, world, local_rank):
     dom = per_kind.get("fused_fwd") or per_kind.get("gemv_fwd") or [0, 0.0]
     achieved = nbytes * args.steps / (dom[1] * 1e-3) / 1e9 if dom[1] > 0 else None
     peak = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+    for v in variants.values():
+        v["unit"] = "GB/s"
+        v["graph_frac_of_hbm"] = v["graph_value"] / peak
     return {
         "metric": "QLoRA NF4 linear forward, NF4-weight-bound GB/s", "value": nbytes * world / (ms * 1e-3) / 1e9,
         "unit": "GB/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": f"llama65b-layer-7-linears-forward-M{M}-r64", "tokens": M, "lora_r": r,
                    "bytes_per_step": nbytes, "l2": "weights (418 MB) larger than L2, no flush",
-                   "step": "forward of the 7 QLoRA linears (weights resident, quantized once)"},
+                   "step": "forward of the 7 QLoRA linears (weights resident, quantized once) as the layer's "
+                           "data flow groups them: {q, k, v, gate, up} on H, then o on A, then down on U"},
         "graph": {"ms_per_step": ms_graph, "value": nbytes * world / (ms_graph * 1e-3) / 1e9, "unit": "GB/s",
                   "frac_of_hbm": nbytes / (ms_graph * 1e-3) / 1e9 / peak},
-        "gpu_launches": len(launches),
+        "variants": variants,
+        "gpu_launches": _kernel_count(launches),
         "roofline": {"bound": "hbm", "kernel": ("few-token forward chain (lora_down_small + " +
                                                 ("gemv_fwd" if M <= 32 else "nf4_fused_fwd (tcgen05)") + " + epilogue)"),
                      "achieved": achieved, "peak": peak, "unit": "GB/s",
@@ -622,7 +676,7 @@ def run_quantizer(args, rank, world, local_rank):
                    "code_table": args.table, "params": sum(l.n_out * l.k_in for l in wl.linears),
                    "bytes_quantize": nbytes_q, "bytes_dequant": nbytes_d,
                    "l2": "weights (667 MB bf16) larger than L2, no flush"},
-        "gpu_launches": len(launches),
+        "gpu_launches": _kernel_count(launches),
         "roofline": {"bound": "hbm", "kernel": "quantize (K1 + K2) and dequant (K3)",
                      "achieved": roof_q, "achieved_dequant": roof_d, "peak": peak, "unit": "GB/s",
                      "frac": roof_q / peak if roof_q else None, "frac_dequant": roof_d / peak if roof_d else None,

@@ -14,6 +14,7 @@ Appendix E.
 
 from __future__ import annotations
 
+import ctypes
 from dataclasses import dataclass
 
 import torch
@@ -26,6 +27,7 @@ __all__ = [
     "quantize_nf4_dq",
     "dequant",
     "linear_fwd",
+    "linear_fwd_group",
     "linear_bwd",
     "last_device_error",
     "t_value",
@@ -206,6 +208,46 @@ def linear_fwd(X: torch.Tensor, q: NF4Tensor, L1: torch.Tensor, L2: torch.Tensor
                                     _ptr(_bits(Y)), _ptr(T) if save_T else None, _ptr(ws), ws.numel(),
                                     _stream(dev)), "qlora_linear_fwd")
     return Y, (T if save_T else None)
+
+
+def linear_fwd_group(members, save_T: bool = True) -> list:
+    """The forward of several linears that see the same tokens, in one call.
+
+    ``members``: a sequence of dicts with keys ``X`` [M, K_i], ``q``
+    (NF4Tensor), ``L1`` [K_i, r_i], ``L2`` [r_i, N_i], ``s`` and optionally the
+    outputs ``Y`` [M, N_i] and ``T`` [M, 2 r_i].  Every member computes what
+    ``linear_fwd`` computes; with at most 128 tokens the whole group runs as
+    one launch chain.  Returns [(Y, T or None)] in member order.
+    """
+    lib = _lib.load()
+    if not 0 < len(members) <= _lib.QLORA_MAX_GROUP:
+        raise ValueError(f"qlora: a group holds 1..{_lib.QLORA_MAX_GROUP} linears")
+    M = members[0]["X"].shape[0]
+    dev = members[0]["X"].device
+    arr = (_lib.FwdMember * len(members))()
+    keep, outs = [], []
+    for i, m in enumerate(members):
+        X, q, L1, L2 = m["X"], m["q"], m["L1"], m["L2"]
+        K, r, N = X.shape[1], L1.shape[1], q.n_out
+        if X.shape[0] != M or X.device != dev:
+            raise ValueError("qlora: the members of a group share the token count and the device")
+        if K != q.k_in or L1.shape[0] != K or tuple(L2.shape) != (r, N):
+            raise ValueError("qlora: shape mismatch")
+        Y = m.get("Y")
+        if Y is None:
+            Y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        T = m.get("T")
+        if save_T and T is None:
+            T = torch.empty((M, 2 * r), dtype=torch.bfloat16, device=dev)
+        w = q.as_struct()
+        keep.append(w)
+        arr[i] = _lib.FwdMember(_ptr(_bits(X)), ctypes.pointer(w), _ptr(_bits(L1)), _ptr(_bits(L2)), r,
+                                float(m["s"]), _ptr(_bits(Y)), _ptr(T) if save_T else None)
+        outs.append((Y, T if save_T else None))
+    ws = _WS.get(lib.qlora_linear_fwd_group_workspace_size(arr, len(members), M), dev)
+    _lib.check(lib.qlora_linear_fwd_group(arr, len(members), M, _ptr(ws), ws.numel(), _stream(dev)),
+               "qlora_linear_fwd_group")
+    return outs
 
 
 def t_value(T: torch.Tensor) -> torch.Tensor:

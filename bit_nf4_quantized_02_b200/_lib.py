@@ -49,6 +49,23 @@ class NF4DQ(ctypes.Structure):
 
 TABLES = {"nf4": 0, "fp4": 1}   # QLORA_TABLE_NF4, QLORA_TABLE_FP4
 
+QLORA_MAX_GROUP = 8
+
+
+class FwdMember(ctypes.Structure):
+    """Mirror of qlora_fwd_member_t (one linear of a grouped forward)."""
+
+    _fields_ = [
+        ("X", c_void_p),
+        ("W", POINTER(NF4DQ)),
+        ("L1", c_void_p),
+        ("L2", c_void_p),
+        ("r", ctypes.c_int32),
+        ("s", c_float),
+        ("Y", c_void_p),
+        ("T_save", c_void_p),
+    ]
+
 
 # name -> (restype, argtypes)
 SIGNATURES = {
@@ -72,6 +89,8 @@ SIGNATURES = {
                                  c_void_p, c_void_p, c_size_t, c_void_p]),
     "qlora_linear_bwd": (c_int, [c_void_p, c_void_p, c_void_p, c_int64, POINTER(NF4DQ), c_void_p, c_void_p, c_int,
                                  c_float, c_void_p, c_void_p, c_void_p, c_int, c_void_p, c_size_t, c_void_p]),
+    "qlora_linear_fwd_group_workspace_size": (c_size_t, [POINTER(FwdMember), c_int, c_int64]),
+    "qlora_linear_fwd_group": (c_int, [POINTER(FwdMember), c_int, c_int64, c_void_p, c_size_t, c_void_p]),
     "qlora_linear_fwd_dropout_workspace_size": (c_size_t, [c_int64, c_int64, c_int64, c_int]),
     "qlora_linear_bwd_dropout_workspace_size": (c_size_t, [c_int64, c_int64, c_int64, c_int]),
     "qlora_linear_fwd_dropout": (c_int, [c_void_p, c_int64, POINTER(NF4DQ), c_void_p, c_void_p, c_int, c_float,

@@ -38,7 +38,10 @@
 //                column = token) and red.global.add into acc.
 // Work: the (128-row tile, 256-K stage) items of the weight are split into
 // equal contiguous ranges, one per CTA; a CTA adds its partial sums into acc
-// whenever its range moves to the next row tile, and at its end.
+// whenever its range moves to the next row tile, and at its end.  A group of
+// linears that see the same tokens (GM > 1) concatenates their items, linear
+// after linear; a row tile never spans two linears, so the accumulator
+// hand-off is unchanged.
 #pragma once
 
 #include "common.cuh"
@@ -77,17 +80,46 @@ struct FtCfg {
   static_assert(kSmemBytes <= 232448, "shared memory per CTA");
 };
 
-struct FtArgs {
-  int M, N, K;
+struct FtMember {
+  int N, K;
   int kstages;           // ceil(K / 256)
-  int items;             // row tiles x kstages
   const uint8_t *c2_fp8;
   const float *c1;
   const float *mu;
   float *acc;            // [M x N] fp32, zero at launch
-  float levels[16];      // the weight's 16-level code table
+};
+
+// A group of linears that see the same tokens: their (row tile, stage) items
+// are concatenated, linear after linear (see the group note in gemv.cuh).
+template <int GM>
+struct FtArgs {
+  int M;
+  int count;             // linears in the group
+  int items;             // row tiles x kstages, summed over the group
+  int beg[GM];           // first item of each linear
+  FtMember m[GM];
+  float levels[16];      // the 16-level code table (shared by the group)
   int *err;
 };
+
+// Per linear: its packed codes in boxes of 128 rows x 128 bytes, and X as
+// [64-block][token][64] in boxes of the four atoms of a stage.
+template <int GM>
+struct FtMaps {
+  CUtensorMap codes[GM];
+  CUtensorMap x[GM];
+};
+
+// Item `it` of a group -> its linear l, row tile rt and stage ks.
+template <int GM>
+__device__ __forceinline__ const FtMember &ft_item(const FtArgs<GM> &p, int it, int &rt, int &ks) {
+  const int l = group_member<GM>(p.beg, p.count, it);
+  const FtMember &m = p.m[l];
+  const int li = it - p.beg[l];
+  rt = li / m.kstages;
+  ks = li - rt * m.kstages;
+  return m;
+}
 
 __device__ __forceinline__ void sts128(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
   asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
@@ -130,7 +162,8 @@ __device__ __forceinline__ void cp_async_arrive_noinc(uint32_t bar) {
 // E4M3 codes (byte (n * kblocks + kb0) & 3 of the first word is block kb0), and
 // c1 of the first and the last of those blocks (they differ when the row's
 // blocks straddle a 256-group).  Producer lane `lane` fills rows lane + 32 i.
-__device__ __forceinline__ void ft_copy_consts(const FtArgs &p, uint32_t area, int rt, int ks, int lane, int kblocks) {
+__device__ __forceinline__ void ft_copy_consts(const FtMember &p, uint32_t area, int rt, int ks, int lane) {
+  const int kblocks = p.K >> 6;
   const int kb0 = ks * 4;
   const int nb = min(4, kblocks - kb0);
   const int64_t nblk = (int64_t)p.N * kblocks;
@@ -172,10 +205,9 @@ __device__ __forceinline__ float ft_c2hat(uint4 raw, int n, int kb0, int j, int 
   return __fmaf_rn(e4m3_to_f32((uint8_t)code8), c1, mu);
 }
 
-template <int MP>
+template <int MP, int GM>
 __global__ void __launch_bounds__(FtCfg<MP>::kThreads, 1)
-    nf4_fused_fwd_kernel(const __grid_constant__ CUtensorMap tmCodes, const __grid_constant__ CUtensorMap tmX,
-                         const __grid_constant__ FtArgs p) {
+    nf4_fused_fwd_kernel(const __grid_constant__ FtMaps<GM> maps, const __grid_constant__ FtArgs<GM> p) {
   using Cfg = FtCfg<MP>;
   constexpr int S = Cfg::kStages;
   constexpr int G = Cfg::kGroups;
@@ -194,7 +226,6 @@ __global__ void __launch_bounds__(FtCfg<MP>::kThreads, 1)
 
   const int warp = warp_id();
   const int lane = lane_id();
-  const int kblocks = p.K >> 6;
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");  // the epilogue may launch and wait
 
   if (threadIdx.x == 0) {
@@ -230,30 +261,32 @@ __global__ void __launch_bounds__(FtCfg<MP>::kThreads, 1)
     // Lane 0 drives the TMA ring; every lane copies the raw block constants of
     // rows lane + 32 i of the stage into its constant area asynchronously and
     // arrives on the stage's full barrier when they have landed.
-    if (lane == 0) {
-      tma_prefetch_desc(&tmCodes);
-      tma_prefetch_desc(&tmX);
+    if (lane < p.count) {
+      tma_prefetch_desc(&maps.codes[lane]);
+      tma_prefetch_desc(&maps.x[lane]);
     }
     int stage = 0;
     uint32_t phase = 0, used = 0, last_parity = 0;
     for (int it = i0; it < i1; ++it) {
-      const int rt = it / p.kstages, ks = it - rt * p.kstages;
+      int rt, ks;
+      const FtMember &m = ft_item<GM>(p, it, rt, ks);
+      const int l = group_member<GM>(p.beg, p.count, it);
       const bool got = mbar_wait(smem_u32(empty_bar + stage), phase ^ 1, p.err, DEV_TIMEOUT_PRODUCER);
       if (!__all_sync(0xFFFFFFFFu, got)) break;
       const uint32_t fb = smem_u32(full_bar + stage);
       const uint32_t sc = smem_u32(smem + stage * Cfg::kStageBytes);
       if (lane == 0) {
         mbar_arrive_expect_tx(fb, Cfg::kCodeBytes + Cfg::kXBytes);
-        tma_load_2d(sc, &tmCodes, fb, ks * (kFtStageK / 2), rt * kFtRows);
+        tma_load_2d(sc, &maps.codes[l], fb, ks * (kFtStageK / 2), rt * kFtRows);
         asm volatile(
             "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5}], "
             "[%2];" ::"r"(sc + Cfg::kCodeBytes),
-            "l"(reinterpret_cast<uint64_t>(&tmX)), "r"(fb), "r"(0), "r"(0), "r"(ks * 4)
+            "l"(reinterpret_cast<uint64_t>(&maps.x[l])), "r"(fb), "r"(0), "r"(0), "r"(ks * 4)
             : "memory");
       }
       used |= 1u << stage;
       last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
-      ft_copy_consts(p, sc + Cfg::kCodeBytes + Cfg::kXBytes, rt, ks, lane, kblocks);
+      ft_copy_consts(m, sc + Cfg::kCodeBytes + Cfg::kXBytes, rt, ks, lane);
       cp_async_arrive_noinc(fb);
       if (++stage == S) {
         stage = 0;
@@ -281,9 +314,11 @@ __global__ void __launch_bounds__(FtCfg<MP>::kThreads, 1)
       bool ok = true;
       uint32_t accumulate = 0;
       for (int it = i0; it < i1 && ok; ++it) {
-        const int rt = it / p.kstages, ks = it - rt * p.kstages;
+        int rt, ks;
+        const FtMember &m = ft_item<GM>(p, it, rt, ks);
+        const int kblocks = m.K >> 6;
         const bool first = it == i0 || ks == 0;
-        const bool last = it == i1 - 1 || ks == p.kstages - 1;
+        const bool last = it == i1 - 1 || ks == m.kstages - 1;
         const int acc = t & 1;
         if (first) {
           if (!mbar_wait(smem_u32(tempty_bar + acc), ((t >> 1) & 1u) ^ 1u, p.err, DEV_TIMEOUT_MMA)) break;
@@ -337,12 +372,14 @@ __global__ void __launch_bounds__(FtCfg<MP>::kThreads, 1)
     const int t = (warp & 3) * 32 + lane;         // weight row within the tile
     const uint32_t sa0 = smem_u32(a_area) + g * R * Cfg::kABytes + (t >> 3) * 1024 + (t & 7) * 16;  // row t, chunk 0
     const uint32_t cswz = (uint32_t)(t & 7) << 4;
-    const float mu = __ldg(p.mu);
     int stage = 0;
     uint32_t phase = 0;
     uint32_t writes = 0;     // blocks this group has stored into its slot
     for (int it = i0; it < i1; ++it) {
-      const int rt = it / p.kstages, ks = it - rt * p.kstages;
+      int rt, ks;
+      const FtMember &m = ft_item<GM>(p, it, rt, ks);
+      const int kblocks = m.K >> 6;
+      const float mu = __ldg(m.mu);
       const int nkb = min(4, kblocks - ks * 4);
       const bool got = mbar_wait(smem_u32(full_bar + stage), phase, p.err, DEV_TIMEOUT_MMA);
       if (!__all_sync(0xFFFFFFFFu, got)) break;
@@ -359,7 +396,7 @@ __global__ void __launch_bounds__(FtCfg<MP>::kThreads, 1)
         const uint4 qb = lds128(sc + (((uint32_t)(2 * j + 1) << 4) ^ cswz));
         const uint32_t q[8] = {qa.x, qa.y, qa.z, qa.w, qb.x, qb.y, qb.z, qb.w};
         BlockTable tb;
-        tb.build(n < p.N ? ft_c2hat(raw, n, ks * 4, j, kblocks, mu) : 0.f, p.levels);
+        tb.build(n < m.N ? ft_c2hat(raw, n, ks * 4, j, kblocks, mu) : 0.f, p.levels);
         // decode the row's 64 weights into registers, then wait for the slot
         uint32_t e[32];
 #pragma unroll
@@ -396,8 +433,9 @@ __global__ void __launch_bounds__(FtCfg<MP>::kThreads, 1)
     const int q = warp & 3;          // TMEM lane quarter
     int t = 0;
     for (int it = i0; it < i1; ++it) {
-      const int rt = it / p.kstages, ks = it - rt * p.kstages;
-      if (!(it == i1 - 1 || ks == p.kstages - 1)) continue;   // not the end of a row-tile segment
+      int rt, ks;
+      const FtMember &m = ft_item<GM>(p, it, rt, ks);
+      if (!(it == i1 - 1 || ks == m.kstages - 1)) continue;   // not the end of a row-tile segment
       const int acc = t & 1;
       const bool got = mbar_wait(smem_u32(tfull_bar + acc), (t >> 1) & 1u, p.err, DEV_TIMEOUT_EPILOGUE);
       if (!__all_sync(0xFFFFFFFFu, got)) break;
@@ -408,10 +446,10 @@ __global__ void __launch_bounds__(FtCfg<MP>::kThreads, 1)
         uint32_t r[16];
         tmem_ld_32x32b_x16(tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * MP + cc), r);
         tmem_wait_ld();
-        if (n < p.N) {
+        if (n < m.N) {
 #pragma unroll
           for (int i = 0; i < 16; ++i)
-            if (cc + i < p.M) red_add_f32(p.acc + (int64_t)(cc + i) * p.N + n, __uint_as_float(r[i]));
+            if (cc + i < p.M) red_add_f32(m.acc + (int64_t)(cc + i) * m.N + n, __uint_as_float(r[i]));
         }
       }
       tc_fence_before();

@@ -33,6 +33,13 @@
 // The two accumulators must be zero at launch (the host clears them with one
 // memset in stream order).  Split-K additions make the low bits of Y depend
 // on the order in which CTAs finish.
+//
+// Groups: one chain of the three launches may serve up to kMaxGroup linears
+// that see the same tokens (GM > 1; e.g. the seven projections of a decoder
+// layer, whose launch gaps and per-linear tails it removes).  Their units
+// (T slices, weight units, output column slices) are concatenated into one
+// flat list per kernel; a unit finds its linear from the list's start
+// offsets.  A single linear is a group of one (GM = 1).
 #pragma once
 
 #include "common.cuh"
@@ -59,20 +66,44 @@ struct GvCfg {
   static constexpr int kSmemBytes = kStages * kStageBytes + 1024 + 256;
 };
 
-struct GvArgs {
-  int M, N, K, r;
+constexpr int kMaxGroup = 8;         // linears per group launch
+
+// The linear, among the `count` members of a group, of flat unit `u`:
+// beg[i] is the first unit of member i (beg[0] = 0, increasing).
+template <int GM>
+__device__ __forceinline__ int group_member(const int (&beg)[GM], int count, int u) {
+  int l = 0;
+#pragma unroll
+  for (int i = 1; i < GM; ++i) l += (i < count && u >= beg[i]) ? 1 : 0;
+  return l;
+}
+
+struct GvMember {
+  int N, K;
   int nks;               // units per 64-row block
-  int units;
-  float s;
   const uint8_t *c2_fp8;
   const float *c1;
   const float *mu;
-  const __nv_bfloat16 *X;    // [M x K]
-  const __nv_bfloat16 *L1;   // [K x r]
-  const __nv_bfloat16 *L2;   // [r x N]
   float *acc;            // [M x N] fp32, zero at launch
-  float levels[16];      // the weight's 16-level code table
+};
+
+template <int GM>
+struct GvArgs {
+  int M;
+  int count;             // linears in the group
+  int units;             // units of all of them
+  int beg[GM];           // first unit of each linear
+  GvMember m[GM];
+  float levels[16];      // the 16-level code table (shared by the group)
   int *err;
+};
+
+// Per linear: its packed codes [N x K/2] in boxes of 64 rows x 128 bytes, and
+// X as [token][64-block][64] in boxes of 8 NT tokens x 4 blocks.
+template <int GM>
+struct GvMaps {
+  CUtensorMap codes[GM];
+  CUtensorMap x[GM];
 };
 
 __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
@@ -143,51 +174,57 @@ struct BlockTable {
 struct ConstPrefetch {
   uint32_t code8[2];
   float c1[2];
+  float mu;
   bool ok[2];
-  __device__ __forceinline__ void load(const GvArgs &p, int u, int st, int r0, int j, int kblocks) {
+  template <int GM>
+  __device__ __forceinline__ void load(const GvArgs<GM> &p, int u, int st, int r0, int j) {
     ok[0] = ok[1] = false;
     code8[0] = code8[1] = 0;
     c1[0] = c1[1] = 0.f;
+    mu = 0.f;
     if (u >= p.units) return;
-    const int rb = u / p.nks, ks = u - rb * p.nks;
+    const int l = group_member<GM>(p.beg, p.count, u);
+    const GvMember &m = p.m[l];
+    const int lu = u - p.beg[l];
+    const int rb = lu / m.nks, ks = lu - rb * m.nks;
+    const int kblocks = m.K >> 6;
     const int kb = ((ks * kGvUnitK + st * kGvStageK) >> 6) + j;
     if (kb >= kblocks) return;
+    mu = __ldg(m.mu);
 #pragma unroll
     for (int i = 0; i < 2; ++i) {
       const int n = rb * kGvRows + r0 + 8 * i;
-      if (n < p.N) {
+      if (n < m.N) {
         const int64_t b = (int64_t)n * kblocks + kb;
-        code8[i] = __ldg(p.c2_fp8 + b);
-        c1[i] = __ldg(p.c1 + (b >> 8));
+        code8[i] = __ldg(m.c2_fp8 + b);
+        c1[i] = __ldg(m.c1 + (b >> 8));
         ok[i] = true;
       }
     }
   }
-  __device__ __forceinline__ float c2hat(int i, float mu) const {
+  __device__ __forceinline__ float c2hat(int i) const {
     return ok[i] ? __fmaf_rn(e4m3_to_f32((uint8_t)code8[i]), c1[i], mu) : 0.f;
   }
 };
 
 // State of one decode/MMA warp of gemv_fwd_kernel.
-template <int NT>
+template <int NT, int GM>
 struct GvConsumer {
   using Cfg = GvCfg<NT>;
-  const GvArgs *p;
+  const GvArgs<GM> *p;
   uint8_t *smem;
   uint64_t *full_bar, *empty_bar;
-  int kblocks, g, j, r0, lane;
+  int g, j, r0, lane;
   int stage;
   uint32_t phase;
   int u, st;
-  float mu;
   float d[2][NT][4];  // two accumulator chains (even / odd k-steps)
 
-  __device__ __forceinline__ void init(const GvArgs &pp, uint8_t *sm, uint64_t *fb, uint64_t *eb, int kb) {
+  __device__ __forceinline__ void init(const GvArgs<GM> &pp, uint8_t *sm, uint64_t *fb, uint64_t *eb) {
     p = &pp;
     smem = sm;
     full_bar = fb;
     empty_bar = eb;
-    kblocks = kb;
     lane = lane_id();
     g = lane >> 2;
     j = lane & 3;
@@ -196,16 +233,18 @@ struct GvConsumer {
     phase = 0;
     u = blockIdx.x;
     st = 0;
-    mu = __ldg(pp.mu);
   }
 
   // Process item (u, st) whose constants are in `cur`; start loading the next
   // item's constants into `nxt`.  Returns false on a pipeline timeout.
   __device__ __forceinline__ bool item(const ConstPrefetch &cur, ConstPrefetch &nxt) {
-    const GvArgs &P = *p;
-    const int rb = u / P.nks, ks = u - rb * P.nks;
+    const GvArgs<GM> &P = *p;
+    const int l = group_member<GM>(P.beg, P.count, u);
+    const GvMember &m = P.m[l];
+    const int lu = u - P.beg[l];
+    const int rb = lu / m.nks, ks = lu - rb * m.nks;
     const int kbeg = ks * kGvUnitK;
-    const int nst = min(kGvUnitK, P.K - kbeg) > kGvStageK ? 2 : 1;
+    const int nst = min(kGvUnitK, m.K - kbeg) > kGvStageK ? 2 : 1;
     const int n0 = rb * kGvRows + r0, n1 = n0 + 8;
     if (st == 0) {
 #pragma unroll
@@ -214,14 +253,14 @@ struct GvConsumer {
         for (int t = 0; t < NT; ++t) d[c][t][0] = d[c][t][1] = d[c][t][2] = d[c][t][3] = 0.f;
     }
     BlockTable tb0, tb1;
-    tb0.build(cur.c2hat(0, mu), P.levels);
-    tb1.build(cur.c2hat(1, mu), P.levels);
+    tb0.build(cur.c2hat(0), P.levels);
+    tb1.build(cur.c2hat(1), P.levels);
     int nu = u, nstn = st + 1;
     if (nstn == nst) {
       nu = u + gridDim.x;
       nstn = 0;
     }
-    nxt.load(P, nu, nstn, r0, j, kblocks);
+    nxt.load(P, nu, nstn, r0, j);
     if (!mbar_wait(smem_u32(full_bar + stage), phase, P.err, DEV_TIMEOUT_MMA)) return false;
     const uint32_t sc = smem_u32(smem + stage * Cfg::kStageBytes);
     const uint32_t sx = sc + Cfg::kCodeBytes;
@@ -268,18 +307,20 @@ struct GvConsumer {
     }
     if (st == nst - 1) {
       // the unit is complete: add its partial products into the accumulator
+      float *acc = m.acc;
+      const int N = m.N;
 #pragma unroll
       for (int t = 0; t < NT; ++t) {
         const int tok = 8 * t + 2 * j;
         const float v0 = d[0][t][0] + d[1][t][0], v1 = d[0][t][1] + d[1][t][1];
         const float v2 = d[0][t][2] + d[1][t][2], v3 = d[0][t][3] + d[1][t][3];
         if (tok < P.M) {
-          if (n0 < P.N) red_add_f32(P.acc + (int64_t)tok * P.N + n0, v0);
-          if (n1 < P.N) red_add_f32(P.acc + (int64_t)tok * P.N + n1, v2);
+          if (n0 < N) red_add_f32(acc + (int64_t)tok * N + n0, v0);
+          if (n1 < N) red_add_f32(acc + (int64_t)tok * N + n1, v2);
         }
         if (tok + 1 < P.M) {
-          if (n0 < P.N) red_add_f32(P.acc + (int64_t)(tok + 1) * P.N + n0, v1);
-          if (n1 < P.N) red_add_f32(P.acc + (int64_t)(tok + 1) * P.N + n1, v3);
+          if (n0 < N) red_add_f32(acc + (int64_t)(tok + 1) * N + n0, v1);
+          if (n1 < N) red_add_f32(acc + (int64_t)(tok + 1) * N + n1, v3);
         }
       }
     }
@@ -289,10 +330,9 @@ struct GvConsumer {
   }
 };
 
-template <int NT>
+template <int NT, int GM>
 __global__ void __launch_bounds__(kGvThreads, GvCfg<NT>::kCtasPerSm)
-    gemv_fwd_kernel(const __grid_constant__ CUtensorMap tmCodes, const __grid_constant__ CUtensorMap tmX,
-                    const __grid_constant__ GvArgs p) {
+    gemv_fwd_kernel(const __grid_constant__ GvMaps<GM> maps, const __grid_constant__ GvArgs<GM> p) {
   using Cfg = GvCfg<NT>;
   constexpr int S = Cfg::kStages;
   extern __shared__ uint8_t smem_raw[];
@@ -302,7 +342,6 @@ __global__ void __launch_bounds__(kGvThreads, GvCfg<NT>::kCtasPerSm)
 
   const int warp = warp_id();
   const int lane = lane_id();
-  const int kblocks = p.K >> 6;
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");  // the epilogue may launch and wait
 
   // ---------------------------------------------------------------- main loop
@@ -318,21 +357,25 @@ __global__ void __launch_bounds__(kGvThreads, GvCfg<NT>::kCtasPerSm)
   if (warp == 4) {
     // Lane 0 drives the TMA ring; all lanes prefetch the next stage's block
     // constants (one code8 run per weight row) into L2 for the decode warps.
-    if (lane == 0) {
-      tma_prefetch_desc(&tmCodes);
-      tma_prefetch_desc(&tmX);
+    if (lane < p.count) {
+      tma_prefetch_desc(&maps.codes[lane]);
+      tma_prefetch_desc(&maps.x[lane]);
     }
     int stage = 0;
     uint32_t phase = 0, used = 0, last_parity = 0;
     bool ok = true;
     for (int u = blockIdx.x; u < p.units && ok; u += gridDim.x) {
-      const int rb = u / p.nks, ks = u - rb * p.nks;
+      const int l = group_member<GM>(p.beg, p.count, u);
+      const GvMember &m = p.m[l];
+      const int lu = u - p.beg[l];
+      const int rb = lu / m.nks, ks = lu - rb * m.nks;
       const int kbeg = ks * kGvUnitK;
-      const int nst = min(kGvUnitK, p.K - kbeg) > kGvStageK ? 2 : 1;
+      const int nst = min(kGvUnitK, m.K - kbeg) > kGvStageK ? 2 : 1;
+      const int kblocks = m.K >> 6;
 #pragma unroll
       for (int i = 0; i < 2; ++i) {
         const int n = rb * kGvRows + lane + 32 * i;
-        if (n < p.N) asm volatile("prefetch.global.L2 [%0];" ::"l"(p.c2_fp8 + (int64_t)n * kblocks + (kbeg >> 6)));
+        if (n < m.N) asm volatile("prefetch.global.L2 [%0];" ::"l"(m.c2_fp8 + (int64_t)n * kblocks + (kbeg >> 6)));
       }
       for (int st = 0; st < nst; ++st) {
         bool got = true;
@@ -343,11 +386,11 @@ __global__ void __launch_bounds__(kGvThreads, GvCfg<NT>::kCtasPerSm)
             mbar_arrive_expect_tx(fb, Cfg::kStageBytes);
             const uint32_t sc = smem_u32(smem + stage * Cfg::kStageBytes);
             const int k0 = kbeg + st * kGvStageK;
-            tma_load_2d(sc, &tmCodes, fb, k0 >> 1, rb * kGvRows);
+            tma_load_2d(sc, &maps.codes[l], fb, k0 >> 1, rb * kGvRows);
             asm volatile(
                 "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, "
                 "%5}], [%2];" ::"r"(sc + Cfg::kCodeBytes),
-                "l"(reinterpret_cast<uint64_t>(&tmX)), "r"(fb), "r"(0), "r"(k0 >> 6), "r"(0)
+                "l"(reinterpret_cast<uint64_t>(&maps.x[l])), "r"(fb), "r"(0), "r"(k0 >> 6), "r"(0)
                 : "memory");
             used |= 1u << stage;
             last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
@@ -367,13 +410,13 @@ __global__ void __launch_bounds__(kGvThreads, GvCfg<NT>::kCtasPerSm)
       for (int i = 0; i < S; ++i)
         if (used & (1u << i)) mbar_wait(smem_u32(full_bar + i), (last_parity >> i) & 1u, p.err, DEV_TIMEOUT_DRAIN);
   } else {
-    GvConsumer<NT> c;
-    c.init(p, smem, full_bar, empty_bar, kblocks);
+    GvConsumer<NT, GM> c;
+    c.init(p, smem, full_bar, empty_bar);
     // Flat walk over this CTA's (unit, stage) items, unrolled by two so the
     // block constants of the next item load into the other buffer (no copies
     // of in-flight loads) while the current item is decoded.
     ConstPrefetch pa, pb;
-    pa.load(p, c.u, c.st, c.r0, c.j, kblocks);
+    pa.load(p, c.u, c.st, c.r0, c.j);
     while (c.u < p.units) {
       if (!c.item(pa, pb)) break;
       if (c.u >= p.units || !c.item(pb, pa)) break;
@@ -385,23 +428,43 @@ __global__ void __launch_bounds__(kGvThreads, GvCfg<NT>::kCtasPerSm)
 }
 
 // T accumulation for few tokens: tacc[M x r] += X[:, k-slice] L1[k-slice, :]
-// for a 64-wide K slice per CTA (blockIdx.x) and a 64-wide column slice
-// (blockIdx.y).  Inputs are staged in shared memory with coalesced loads (X in
-// chunks of 32 tokens), then each thread forms 4 tokens x 1 column over the
-// slice and adds it with red.global.add.  Lets its dependent launch start
-// immediately.
+// for a 64-wide K slice per CTA (blockIdx.x, flat over the group's linears)
+// and a 64-wide column slice (blockIdx.y).  Inputs are staged in shared
+// memory with coalesced loads (X in chunks of 32 tokens), then each thread
+// forms 4 tokens x 1 column over the slice and adds it with red.global.add.
+// Lets its dependent launch start immediately.
 constexpr int kTSliceK = 64;
 constexpr int kTokChunk = 32;
 
-__global__ void __launch_bounds__(256) lora_down_small_kernel(const __nv_bfloat16 *__restrict__ X,
-                                                              const __nv_bfloat16 *__restrict__ L1, int M, int K,
-                                                              int r, float *__restrict__ tacc) {
+struct TdMember {
+  const __nv_bfloat16 *X;    // [M x K]
+  const __nv_bfloat16 *L1;   // [K x r]
+  float *tacc;               // [M x r] fp32, zero at launch
+  int K, r;
+};
+
+template <int GM>
+struct TdArgs {
+  int M, count;
+  int beg[GM];               // first K slice of each linear
+  TdMember m[GM];
+};
+
+template <int GM>
+__global__ void __launch_bounds__(256) lora_down_small_kernel(const __grid_constant__ TdArgs<GM> a) {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   __shared__ float xs[kTokChunk][kTSliceK + 1];
   __shared__ float ls[kTSliceK][65];
-  const int k0 = blockIdx.x * kTSliceK;
+  const int l = group_member<GM>(a.beg, a.count, blockIdx.x);
+  const TdMember &mb = a.m[l];
+  const int K = mb.K, r = mb.r, M = a.M;
+  const __nv_bfloat16 *__restrict__ X = mb.X;
+  const __nv_bfloat16 *__restrict__ L1 = mb.L1;
+  float *__restrict__ tacc = mb.tacc;
+  const int k0 = (blockIdx.x - a.beg[l]) * kTSliceK;
   const int kn = min(kTSliceK, K - k0);
   const int j0 = blockIdx.y * 64;
+  if (j0 >= r) return;       // a column slice beyond this linear's rank
   const int jn = min(64, r - j0);
   for (int i = threadIdx.x; i < kTSliceK * 64; i += blockDim.x) {
     const int k = i >> 6, jj = i & 63;
@@ -419,9 +482,9 @@ __global__ void __launch_bounds__(256) lora_down_small_kernel(const __nv_bfloat1
     for (int m0 = (threadIdx.x >> 6) * 4; m0 < mn; m0 += 16) {
       float t[4] = {0.f, 0.f, 0.f, 0.f};
       for (int k = 0; k < kn; ++k) {
-        const float l = ls[k][jj];
+        const float lv = ls[k][jj];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) t[i] = __fmaf_rn(xs[m0 + i][k], l, t[i]);
+        for (int i = 0; i < 4; ++i) t[i] = __fmaf_rn(xs[m0 + i][k], lv, t[i]);
       }
       if (jj < jn) {
 #pragma unroll
@@ -433,21 +496,43 @@ __global__ void __launch_bounds__(256) lora_down_small_kernel(const __nv_bfloat1
 }
 
 // Y[tok][n] = bf16(acc[tok][n] + sum_j (s T)[tok][j] L2[j][n]).  A CTA owns 64
-// columns (blockIdx.x) of 32 tokens (blockIdx.y): it stages their L2 slice
-// (r x 64) before waiting for the product kernel (L2 is an input), then s T
-// of its tokens, then thread (column c, token group q) forms tokens q, q+4,
-// ..., q+28.  Blocks of the first column slice also write T = s X L1 of their
-// tokens as a bf16 hi/lo pair.  Launched as a programmatic dependent of the
-// product kernel.
-__global__ void __launch_bounds__(256) gemv_epilogue_kernel(const float *__restrict__ acc,
-                                                            const float *__restrict__ tacc,
-                                                            const __nv_bfloat16 *__restrict__ L2, int M, int N, int r,
-                                                            float s, __nv_bfloat16 *__restrict__ Y,
-                                                            __nv_bfloat16 *__restrict__ T_save) {
+// columns (blockIdx.x, flat over the group's linears) of 32 tokens
+// (blockIdx.y): it stages their L2 slice (r x 64) before waiting for the
+// product kernel (L2 is an input), then s T of its tokens, then thread
+// (column c, token group q) forms tokens q, q+4, ..., q+28.  Blocks of a
+// linear's first column slice also write T = s X L1 of their tokens as a bf16
+// hi/lo pair.  Launched as a programmatic dependent of the product kernel.
+struct EpMember {
+  const float *acc;          // [M x N] fp32
+  const float *tacc;         // [M x r] fp32 (X L1, unscaled)
+  const __nv_bfloat16 *L2;   // [r x N]
+  __nv_bfloat16 *Y;          // [M x N]
+  __nv_bfloat16 *T_save;     // [M x 2r] or null
+  int N, r;
+  float s;
+};
+
+template <int GM>
+struct EpArgs {
+  int M, count;
+  int beg[GM];               // first column slice of each linear
+  EpMember m[GM];
+};
+
+template <int GM>
+__global__ void __launch_bounds__(256) gemv_epilogue_kernel(const __grid_constant__ EpArgs<GM> a) {
   extern __shared__ float esm[];
+  const int l = group_member<GM>(a.beg, a.count, blockIdx.x);
+  const EpMember &me = a.m[l];
+  const int M = a.M, N = me.N, r = me.r;
+  const float s = me.s;
+  const float *__restrict__ acc = me.acc;
+  const float *__restrict__ tacc = me.tacc;
+  const __nv_bfloat16 *__restrict__ L2 = me.L2;
   float *ts = esm;                                                        // [32 x r] s*T
   __nv_bfloat16 *l2s = reinterpret_cast<__nv_bfloat16 *>(esm + kTokChunk * r);  // [r x 64]
-  const int nb = blockIdx.x * 64;
+  const int slice = blockIdx.x - a.beg[l];
+  const int nb = slice * 64;
   const int ncols = min(64, N - nb);
   const int mb = blockIdx.y * kTokChunk;
   const int mn = min(kTokChunk, M - mb);
@@ -460,7 +545,8 @@ __global__ void __launch_bounds__(256) gemv_epilogue_kernel(const float *__restr
   asm volatile("griddepcontrol.wait;" ::: "memory");
   for (int i = threadIdx.x; i < mn * r; i += blockDim.x) ts[i] = s * ld_dep_f32(tacc + (int64_t)mb * r + i);
   __syncthreads();
-  if (blockIdx.x == 0 && T_save) {
+  if (slice == 0 && me.T_save) {
+    __nv_bfloat16 *T_save = me.T_save;
     for (int i = threadIdx.x; i < mn * r; i += blockDim.x) {
       const float v = ts[i];
       const int m = mb + i / r, jj = i % r;
@@ -487,6 +573,7 @@ __global__ void __launch_bounds__(256) gemv_epilogue_kernel(const float *__restr
       if (m < mn) y[i] = __fmaf_rn(ts[m * r + jj], l2, y[i]);
     }
   }
+  __nv_bfloat16 *Y = me.Y;
 #pragma unroll
   for (int i = 0; i < kTok; ++i) {
     const int m = q + 4 * i;

@@ -29,9 +29,9 @@ struct DeviceInfo {
   int *err = nullptr;        // device address of g_dev_err
   bool gemm_attr[16] = {};   // [wide][fold][BN 64/128/256 or 3 = pair]: shared-memory limit set
   int pair_clusters[3] = {0, 0, 0};   // co-resident 2-CTA clusters of the pair GEMM [form]
-  int gemv_smem_set[3] = {0, 0, 0};   // dynamic smem limit set per NT variant
-  int gemv_per_sm[3] = {0, 0, 0};     // resident CTAs per SM per NT variant
-  int fused_smem_set[4] = {0, 0, 0, 0};   // dynamic smem limit set per token-padding variant
+  int gemv_smem_set[6] = {};    // dynamic smem limit set per [group form][NT variant]
+  int gemv_per_sm[6] = {};      // resident CTAs per SM per [group form][NT variant]
+  int fused_smem_set[8] = {};   // dynamic smem limit set per [group form][token-padding variant]
 };
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_mu;
@@ -452,156 +452,246 @@ int encode_tmap(CUtensorMap *m, CUtensorMapDataType dt, int rank, const void *pt
   return r == CUDA_SUCCESS ? QLORA_OK : QLORA_ERR_CUDA;
 }
 
-// Workspace of the few-token forward: [acc M*N f32 | tacc M*r f32], zeroed per call.
-struct GemvLayout {
-  size_t acc, tacc, zero_bytes, total;
+// One linear of a few-token forward group (host view of its arguments).
+struct FwdMember {
+  const qlora_nf4dq_t *W;
+  const uint16_t *X, *L1, *L2;
+  int r;
+  float s;
+  uint16_t *Y, *T_save;
 };
 
-GemvLayout gemv_layout(int64_t M, int64_t N, int r) {
+// Workspace of the few-token forward: per linear [acc M*N f32 | tacc M*r f32],
+// one linear after the other, all zeroed by one memset per call.
+struct GemvLayout {
+  size_t acc[kMaxGroup], tacc[kMaxGroup];
+  size_t zero_bytes, total;
+};
+
+GemvLayout gemv_layout(int64_t M, const FwdMember *mem, int count) {
   GemvLayout L;
-  L.acc = 0;
-  L.tacc = align_up((size_t)M * N * 4, 16);
-  L.zero_bytes = L.tacc + (size_t)M * r * 4;
-  L.total = align_up(L.zero_bytes);
+  size_t off = 0;
+  for (int i = 0; i < count; ++i) {
+    L.acc[i] = align_up(off, 16);
+    L.tacc[i] = align_up(L.acc[i] + (size_t)M * mem[i].W->n_out * 4, 16);
+    off = L.tacc[i] + (size_t)M * mem[i].r * 4;
+  }
+  L.zero_bytes = off;
+  L.total = align_up(off);
   return L;
 }
 
-// Y = bf16(acc + s T L2) and the T hi/lo pair, as a programmatic dependent of
-// the product kernel just launched.
-int launch_lora_epilogue(const float *acc, const float *tacc, const __nv_bfloat16 *L2, int64_t M, int64_t N, int r,
-                         float s, uint16_t *Y, uint16_t *T_save, cudaStream_t st) {
-  const size_t esmem = (size_t)kTokChunk * r * 4 + (size_t)r * 64 * 2;
-  if (esmem > 48 * 1024 &&
-      cudaFuncSetAttribute(gemv_epilogue_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)esmem) != cudaSuccess)
-    return QLORA_ERR_CUDA;
-  const dim3 grid((unsigned)((N + 63) / 64), (unsigned)((M + kTokChunk - 1) / kTokChunk));
-  return launch_pdl(gemv_epilogue_kernel, grid, dim3(256), esmem, st, acc, tacc, L2, (int)M, (int)N, r, s,
-                    reinterpret_cast<__nv_bfloat16 *>(Y), reinterpret_cast<__nv_bfloat16 *>(T_save));
+size_t gemv_ws_bytes(int64_t M, int64_t N, int r) {
+  qlora_nf4dq_t w;
+  std::memset(&w, 0, sizeof(w));
+  w.n_out = N;
+  FwdMember m;
+  std::memset(&m, 0, sizeof(m));
+  m.W = &w;
+  m.r = r;
+  return gemv_layout(M, &m, 1).total;
 }
 
-// Fused doubleDequant + tcgen05 forward for M <= 128 tokens (MP = padded M):
-// T accumulation, then the product (a programmatic dependent of it), then the
-// LoRA epilogue.
-template <int MP>
-int launch_fused_fwd(const qlora_nf4dq_t *W, const uint16_t *X, int64_t M, const uint16_t *L1, const uint16_t *L2,
-                     int r, float s, uint16_t *Y, uint16_t *T_save, uint8_t *ws, DeviceInfo *dev, cudaStream_t st) {
+// T accumulation of every linear of the group (a plain launch: it follows all
+// earlier work in the stream).
+template <int GM>
+int launch_lora_down(const FwdMember *mem, int count, int64_t M, const GemvLayout &L, uint8_t *ws, cudaStream_t st) {
+  TdArgs<GM> a;
+  std::memset(&a, 0, sizeof(a));
+  a.M = (int)M;
+  a.count = count;
+  int slices = 0, rmax = 0;
+  for (int i = 0; i < count; ++i) {
+    const int64_t K = mem[i].W->k_in;
+    a.beg[i] = slices;
+    a.m[i].X = reinterpret_cast<const __nv_bfloat16 *>(mem[i].X);
+    a.m[i].L1 = reinterpret_cast<const __nv_bfloat16 *>(mem[i].L1);
+    a.m[i].tacc = reinterpret_cast<float *>(ws + L.tacc[i]);
+    a.m[i].K = (int)K;
+    a.m[i].r = mem[i].r;
+    slices += (int)((K + kTSliceK - 1) / kTSliceK);
+    rmax = std::max(rmax, mem[i].r);
+  }
+  lora_down_small_kernel<GM><<<dim3((unsigned)slices, (unsigned)((rmax + 63) / 64)), 256, 0, st>>>(a);
+  return launch_status();
+}
+
+// Y = bf16(acc + s T L2) and the T hi/lo pair of every linear of the group,
+// as a programmatic dependent of the product kernel just launched.
+template <int GM>
+int launch_lora_epilogue(const FwdMember *mem, int count, int64_t M, const GemvLayout &L, uint8_t *ws,
+                         cudaStream_t st) {
+  EpArgs<GM> a;
+  std::memset(&a, 0, sizeof(a));
+  a.M = (int)M;
+  a.count = count;
+  int slices = 0, rmax = 0;
+  for (int i = 0; i < count; ++i) {
+    const int64_t N = mem[i].W->n_out;
+    a.beg[i] = slices;
+    a.m[i].acc = reinterpret_cast<const float *>(ws + L.acc[i]);
+    a.m[i].tacc = reinterpret_cast<const float *>(ws + L.tacc[i]);
+    a.m[i].L2 = reinterpret_cast<const __nv_bfloat16 *>(mem[i].L2);
+    a.m[i].Y = reinterpret_cast<__nv_bfloat16 *>(mem[i].Y);
+    a.m[i].T_save = reinterpret_cast<__nv_bfloat16 *>(mem[i].T_save);
+    a.m[i].N = (int)N;
+    a.m[i].r = mem[i].r;
+    a.m[i].s = mem[i].s;
+    slices += (int)((N + 63) / 64);
+    rmax = std::max(rmax, mem[i].r);
+  }
+  const size_t esmem = (size_t)kTokChunk * rmax * 4 + (size_t)rmax * 64 * 2;
+  if (esmem > 48 * 1024 && cudaFuncSetAttribute(gemv_epilogue_kernel<GM>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                (int)esmem) != cudaSuccess)
+    return QLORA_ERR_CUDA;
+  const dim3 grid((unsigned)slices, (unsigned)((M + kTokChunk - 1) / kTokChunk));
+  return launch_pdl(gemv_epilogue_kernel<GM>, grid, dim3(256), esmem, st, a);
+}
+
+// Fused doubleDequant + tcgen05 forward for M <= 128 tokens (MP = padded M)
+// of a group of linears sharing one code table: T accumulation, then the
+// product (a programmatic dependent of it), then the LoRA epilogue.  The
+// accumulators are zero (the caller's memset).
+template <int MP, int GM>
+int launch_fused_fwd(const FwdMember *mem, int count, int64_t M, const GemvLayout &L, uint8_t *ws, DeviceInfo *dev,
+                     cudaStream_t st) {
   using Cfg = FtCfg<MP>;
-  const int64_t N = W->n_out, K = W->k_in;
-  const GemvLayout L = gemv_layout(M, N, r);
-  if (cudaMemsetAsync(ws, 0, L.zero_bytes, st) != cudaSuccess) return QLORA_ERR_CUDA;
-  CUtensorMap tm_codes, tm_x;
-  {
-    const cuuint64_t dims[2] = {(cuuint64_t)(K / 2), (cuuint64_t)N};
-    const cuuint64_t strides[1] = {(cuuint64_t)(K / 2)};
-    const cuuint32_t box[2] = {128, (cuuint32_t)kFtRows};
-    int rc = encode_tmap(&tm_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, W->codes, dims, strides, box);
-    if (rc) return rc;
+  FtMaps<GM> maps;
+  FtArgs<GM> a;
+  std::memset(&maps, 0, sizeof(maps));
+  std::memset(&a, 0, sizeof(a));
+  std::memcpy(a.levels, kLevelsHost[mem[0].W->table], sizeof(a.levels));
+  a.M = (int)M;
+  a.count = count;
+  a.err = dev->err;
+  int items = 0;
+  for (int i = 0; i < count; ++i) {
+    const qlora_nf4dq_t *W = mem[i].W;
+    const int64_t N = W->n_out, K = W->k_in;
+    {
+      const cuuint64_t dims[2] = {(cuuint64_t)(K / 2), (cuuint64_t)N};
+      const cuuint64_t strides[1] = {(cuuint64_t)(K / 2)};
+      const cuuint32_t box[2] = {128, (cuuint32_t)kFtRows};
+      int rc = encode_tmap(&maps.codes[i], CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, W->codes, dims, strides, box);
+      if (rc) return rc;
+    }
+    {
+      // X as [64-block][token][64]: one box = the four K-major atoms of a stage
+      const cuuint64_t dims[3] = {64, (cuuint64_t)M, (cuuint64_t)(K / 64)};
+      const cuuint64_t strides[2] = {(cuuint64_t)K * 2, 128};
+      const cuuint32_t box[3] = {64, (cuuint32_t)MP, 4};
+      int rc = encode_tmap(&maps.x[i], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, mem[i].X, dims, strides, box);
+      if (rc) return rc;
+    }
+    FtMember &m = a.m[i];
+    m.N = (int)N;
+    m.K = (int)K;
+    m.kstages = (int)((K + kFtStageK - 1) / kFtStageK);
+    m.c2_fp8 = W->c2_fp8;
+    m.c1 = W->c1;
+    m.mu = W->c2_mean;
+    m.acc = reinterpret_cast<float *>(ws + L.acc[i]);
+    a.beg[i] = items;
+    items += (int)((N + kFtRows - 1) / kFtRows) * m.kstages;
   }
-  {
-    // X as [64-block][token][64]: one box = the four K-major atoms of a stage
-    const cuuint64_t dims[3] = {64, (cuuint64_t)M, (cuuint64_t)(K / 64)};
-    const cuuint64_t strides[2] = {(cuuint64_t)K * 2, 128};
-    const cuuint32_t box[3] = {64, (cuuint32_t)MP, 4};
-    int rc = encode_tmap(&tm_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, X, dims, strides, box);
-    if (rc) return rc;
-  }
-  const int idx = MP == 16 ? 0 : (MP == 32 ? 1 : (MP == 64 ? 2 : 3));
+  a.items = items;
+  const int idx = (GM > 1 ? 4 : 0) + (MP == 16 ? 0 : (MP == 32 ? 1 : (MP == 64 ? 2 : 3)));
   if (dev->fused_smem_set[idx] < Cfg::kSmemBytes) {
-    if (cudaFuncSetAttribute(nf4_fused_fwd_kernel<MP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (cudaFuncSetAttribute(nf4_fused_fwd_kernel<MP, GM>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              Cfg::kSmemBytes) != cudaSuccess)
       return QLORA_ERR_CUDA;
     dev->fused_smem_set[idx] = Cfg::kSmemBytes;
   }
-  FtArgs a;
-  std::memset(&a, 0, sizeof(a));
-  std::memcpy(a.levels, kLevelsHost[W->table], sizeof(a.levels));
-  a.M = (int)M;
-  a.N = (int)N;
-  a.K = (int)K;
-  a.kstages = (int)((K + kFtStageK - 1) / kFtStageK);
-  a.items = (int)((N + kFtRows - 1) / kFtRows) * a.kstages;
-  a.c2_fp8 = W->c2_fp8;
-  a.c1 = W->c1;
-  a.mu = W->c2_mean;
-  a.acc = reinterpret_cast<float *>(ws + L.acc);
-  a.err = dev->err;
-  float *tacc = reinterpret_cast<float *>(ws + L.tacc);
   const int grid = std::max(1, std::min(a.items, dev->sms));
   ProfScope prof(QLORA_KERNEL_FUSED_FWD, st);
   // 1. T accumulation; 2. the fused product, overlapping it; 3. the LoRA epilogue.
-  const dim3 tgrid((unsigned)((K + kTSliceK - 1) / kTSliceK), (unsigned)((r + 63) / 64));
-  lora_down_small_kernel<<<tgrid, 256, 0, st>>>(reinterpret_cast<const __nv_bfloat16 *>(X),
-                                                reinterpret_cast<const __nv_bfloat16 *>(L1), (int)M, (int)K, r, tacc);
-  int rc = launch_status();
+  int rc = launch_lora_down<GM>(mem, count, M, L, ws, st);
   if (rc) return rc;
-  rc = launch_pdl(nf4_fused_fwd_kernel<MP>, dim3(grid), dim3(Cfg::kThreads), (size_t)Cfg::kSmemBytes, st, tm_codes,
-                  tm_x, a);
+  rc = launch_pdl(nf4_fused_fwd_kernel<MP, GM>, dim3(grid), dim3(Cfg::kThreads), (size_t)Cfg::kSmemBytes, st, maps,
+                  a);
   if (rc) return rc;
-  return launch_lora_epilogue(a.acc, tacc, reinterpret_cast<const __nv_bfloat16 *>(L2), M, N, r, s, Y, T_save, st);
+  return launch_lora_epilogue<GM>(mem, count, M, L, ws, st);
 }
 
-template <int NT>
-int launch_gemv(const qlora_nf4dq_t *W, const uint16_t *X, int64_t M, const uint16_t *L1, const uint16_t *L2, int r,
-                float s, uint16_t *Y, uint16_t *T_save, uint8_t *ws, DeviceInfo *dev, cudaStream_t st) {
+// Fused doubleDequant + mma.sync forward for M <= 8 NT tokens of a group of
+// linears sharing one code table (three launches, as launch_fused_fwd).
+template <int NT, int GM>
+int launch_gemv(const FwdMember *mem, int count, int64_t M, const GemvLayout &L, uint8_t *ws, DeviceInfo *dev,
+                cudaStream_t st) {
   using Cfg = GvCfg<NT>;
-  const int64_t N = W->n_out, K = W->k_in;
-  const GemvLayout L = gemv_layout(M, N, r);
-  if (cudaMemsetAsync(ws, 0, L.zero_bytes, st) != cudaSuccess) return QLORA_ERR_CUDA;
-  CUtensorMap tm_codes, tm_x;
-  {
-    const cuuint64_t dims[2] = {(cuuint64_t)(K / 2), (cuuint64_t)N};
-    const cuuint64_t strides[1] = {(cuuint64_t)(K / 2)};
-    const cuuint32_t box[2] = {128, (cuuint32_t)kGvRows};
-    int rc = encode_tmap(&tm_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, W->codes, dims, strides, box);
-    if (rc) return rc;
+  GvMaps<GM> maps;
+  GvArgs<GM> a;
+  std::memset(&maps, 0, sizeof(maps));
+  std::memset(&a, 0, sizeof(a));
+  std::memcpy(a.levels, kLevelsHost[mem[0].W->table], sizeof(a.levels));
+  a.M = (int)M;
+  a.count = count;
+  a.err = dev->err;
+  int units = 0;
+  for (int i = 0; i < count; ++i) {
+    const qlora_nf4dq_t *W = mem[i].W;
+    const int64_t N = W->n_out, K = W->k_in;
+    {
+      const cuuint64_t dims[2] = {(cuuint64_t)(K / 2), (cuuint64_t)N};
+      const cuuint64_t strides[1] = {(cuuint64_t)(K / 2)};
+      const cuuint32_t box[2] = {128, (cuuint32_t)kGvRows};
+      int rc = encode_tmap(&maps.codes[i], CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, W->codes, dims, strides, box);
+      if (rc) return rc;
+    }
+    {
+      const cuuint64_t dims[3] = {64, (cuuint64_t)(K / 64), (cuuint64_t)M};
+      const cuuint64_t strides[2] = {128, (cuuint64_t)K * 2};
+      const cuuint32_t box[3] = {64, 4, (cuuint32_t)(8 * NT)};
+      int rc = encode_tmap(&maps.x[i], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, mem[i].X, dims, strides, box);
+      if (rc) return rc;
+    }
+    GvMember &m = a.m[i];
+    m.N = (int)N;
+    m.K = (int)K;
+    m.nks = (int)((K + kGvUnitK - 1) / kGvUnitK);
+    m.c2_fp8 = W->c2_fp8;
+    m.c1 = W->c1;
+    m.mu = W->c2_mean;
+    m.acc = reinterpret_cast<float *>(ws + L.acc[i]);
+    a.beg[i] = units;
+    units += (int)((N + kGvRows - 1) / kGvRows) * m.nks;
   }
-  {
-    const cuuint64_t dims[3] = {64, (cuuint64_t)(K / 64), (cuuint64_t)M};
-    const cuuint64_t strides[2] = {128, (cuuint64_t)K * 2};
-    const cuuint32_t box[3] = {64, 4, (cuuint32_t)(8 * NT)};
-    int rc = encode_tmap(&tm_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, X, dims, strides, box);
-    if (rc) return rc;
-  }
+  a.units = units;
   const int smem = Cfg::kSmemBytes;
-  const int idx = NT == 1 ? 0 : (NT == 2 ? 1 : 2);
+  const int idx = (GM > 1 ? 3 : 0) + (NT == 1 ? 0 : (NT == 2 ? 1 : 2));
   if (dev->gemv_smem_set[idx] < smem) {
-    if (cudaFuncSetAttribute(gemv_fwd_kernel<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+    if (cudaFuncSetAttribute(gemv_fwd_kernel<NT, GM>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+        cudaSuccess)
       return QLORA_ERR_CUDA;
     dev->gemv_smem_set[idx] = smem;
   }
   int &per_sm = dev->gemv_per_sm[idx];
-  if (per_sm < 1 &&
-      (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, gemv_fwd_kernel<NT>, kGvThreads, smem) != cudaSuccess ||
-       per_sm < 1))
+  if (per_sm < 1 && (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, gemv_fwd_kernel<NT, GM>, kGvThreads,
+                                                                    smem) != cudaSuccess ||
+                     per_sm < 1))
     return QLORA_ERR_CUDA;
-  GvArgs a;
-  std::memset(&a, 0, sizeof(a));
-  std::memcpy(a.levels, kLevelsHost[W->table], sizeof(a.levels));
-  a.M = (int)M;
-  a.N = (int)N;
-  a.K = (int)K;
-  a.r = r;
-  a.nks = (int)((K + kGvUnitK - 1) / kGvUnitK);
-  a.units = (int)((N + kGvRows - 1) / kGvRows) * a.nks;
-  a.s = s;
-  a.c2_fp8 = W->c2_fp8;
-  a.c1 = W->c1;
-  a.mu = W->c2_mean;
-  a.L2 = reinterpret_cast<const __nv_bfloat16 *>(L2);
-  a.acc = reinterpret_cast<float *>(ws + L.acc);
-  a.err = dev->err;
-  float *tacc = reinterpret_cast<float *>(ws + L.tacc);
   const int grid = std::max(1, std::min(a.units, per_sm * dev->sms));
   ProfScope prof(QLORA_KERNEL_GEMV_FWD, st);
   // 1. T accumulation; 2. the product, overlapping it; 3. the LoRA epilogue.
-  const dim3 tgrid((unsigned)((K + kTSliceK - 1) / kTSliceK), (unsigned)((r + 63) / 64));
-  lora_down_small_kernel<<<tgrid, 256, 0, st>>>(reinterpret_cast<const __nv_bfloat16 *>(X),
-                                                reinterpret_cast<const __nv_bfloat16 *>(L1), (int)M, (int)K, r, tacc);
-  int rc = launch_status();
+  int rc = launch_lora_down<GM>(mem, count, M, L, ws, st);
   if (rc) return rc;
-  rc = launch_pdl(gemv_fwd_kernel<NT>, dim3(grid), dim3(kGvThreads), (size_t)smem, st, tm_codes, tm_x, a);
+  rc = launch_pdl(gemv_fwd_kernel<NT, GM>, dim3(grid), dim3(kGvThreads), (size_t)smem, st, maps, a);
   if (rc) return rc;
-  return launch_lora_epilogue(a.acc, tacc, a.L2, M, N, r, s, Y, T_save, st);
+  return launch_lora_epilogue<GM>(mem, count, M, L, ws, st);
+}
+
+// The few-token forward of `count` linears sharing one code table, on a
+// zeroed workspace: the path by token count.
+template <int GM>
+int few_token_fwd(const FwdMember *mem, int count, int64_t M, const GemvLayout &L, uint8_t *ws, DeviceInfo *dev,
+                  cudaStream_t st) {
+  // up to 32 tokens: weight decoded straight into mma.sync fragments (each
+  // warp independent); 33..128: decoded into shared memory for tcgen05
+  if (M <= 8) return launch_gemv<1, GM>(mem, count, M, L, ws, dev, st);
+  if (M <= 16) return launch_gemv<2, GM>(mem, count, M, L, ws, dev, st);
+  if (M <= kGvMaxM) return launch_gemv<4, GM>(mem, count, M, L, ws, dev, st);
+  if (M <= 64) return launch_fused_fwd<64, GM>(mem, count, M, L, ws, dev, st);
+  return launch_fused_fwd<128, GM>(mem, count, M, L, ws, dev, st);
 }
 
 struct FwdLayout {
@@ -981,7 +1071,7 @@ extern "C" {
 
 size_t qlora_linear_fwd_workspace_size(int64_t M, int64_t n_out, int64_t k_in, int r) {
   if (M < 0 || n_out <= 0 || k_in <= 0 || r <= 0) return 0;
-  if (M <= kFtMaxM) return gemv_layout(M, n_out, r).total;
+  if (M <= kFtMaxM) return gemv_ws_bytes(M, n_out, r);
   DeviceInfo *dev;
   const int sms = current_device_info(&dev) == QLORA_OK ? dev->sms : 148;
   return fwd_layout(M, n_out, k_in, r, sms).total;
@@ -1009,21 +1099,110 @@ int qlora_linear_fwd(const uint16_t *X, int64_t M, const qlora_nf4dq_t *W, const
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   if (M <= kFtMaxM) {
     // Few tokens: the weight bytes dominate; one fused decode + product pass.
-    if (!ws || ws_bytes < gemv_layout(M, N, r).total) return QLORA_ERR_WORKSPACE;
+    const FwdMember mem = {W, X, L1, L2, r, s, Y, T_save};
+    const GemvLayout L = gemv_layout(M, &mem, 1);
+    if (!ws || ws_bytes < L.total) return QLORA_ERR_WORKSPACE;
     if (!aligned(ws, 256)) return QLORA_ERR_MISALIGNED;
     uint8_t *w8 = reinterpret_cast<uint8_t *>(ws);
-    // up to 32 tokens: weight decoded straight into mma.sync fragments (each
-    // warp independent); 33..128: decoded into shared memory for tcgen05
-    if (M <= 8) return launch_gemv<1>(W, X, M, L1, L2, r, s, Y, T_save, w8, dev, st);
-    if (M <= 16) return launch_gemv<2>(W, X, M, L1, L2, r, s, Y, T_save, w8, dev, st);
-    if (M <= kGvMaxM) return launch_gemv<4>(W, X, M, L1, L2, r, s, Y, T_save, w8, dev, st);
-    if (M <= 64) return launch_fused_fwd<64>(W, X, M, L1, L2, r, s, Y, T_save, w8, dev, st);
-    return launch_fused_fwd<128>(W, X, M, L1, L2, r, s, Y, T_save, w8, dev, st);
+    if (cudaMemsetAsync(w8, 0, L.zero_bytes, st) != cudaSuccess) return QLORA_ERR_CUDA;
+    return few_token_fwd<1>(&mem, 1, M, L, w8, dev, st);
   }
   const FwdLayout L = fwd_layout(M, N, K, r, dev->sms);
   if (!ws || ws_bytes < L.total) return QLORA_ERR_WORKSPACE;
   if (!aligned(ws, 256)) return QLORA_ERR_MISALIGNED;
   return fwd_large(X, X, s, M, W, L1, L2, r, Y, T_save, reinterpret_cast<uint8_t *>(ws), L, dev, st);
+}
+
+// ------------------------------------------------------------- grouped forward
+static_assert(kMaxGroup == QLORA_MAX_GROUP, "group size of the C ABI");
+// Members are validated as by qlora_linear_fwd; the few-token path runs one
+// launch chain per code table present (normally one for the whole group).
+static int check_fwd_group(const qlora_fwd_member_t *members, int count, int64_t M) {
+  if (count < 0 || count > QLORA_MAX_GROUP || (count > 0 && !members)) return QLORA_ERR_INVALID_ARG;
+  for (int i = 0; i < count; ++i) {
+    const qlora_fwd_member_t &m = members[i];
+    int rc = check_linear(M, m.W, m.r);
+    if (rc) return rc;
+    if (M == 0) continue;
+    if (!m.X || !m.L1 || !m.L2 || !m.Y) return QLORA_ERR_INVALID_ARG;
+    if (!aligned(m.X, 16) || !aligned(m.L1, 16) || !aligned(m.L2, 16) || !aligned(m.Y, 16) ||
+        (m.T_save && !aligned(m.T_save, 16)))
+      return QLORA_ERR_MISALIGNED;
+  }
+  return QLORA_OK;
+}
+
+static void fwd_members(const qlora_fwd_member_t *members, int count, FwdMember *mem) {
+  for (int i = 0; i < count; ++i) {
+    const qlora_fwd_member_t &m = members[i];
+    mem[i] = FwdMember{m.W, m.X, m.L1, m.L2, m.r, m.s, m.Y, m.T_save};
+  }
+}
+
+size_t qlora_linear_fwd_group_workspace_size(const qlora_fwd_member_t *members, int count, int64_t M) {
+  if (M < 0 || count < 0 || count > QLORA_MAX_GROUP || (count > 0 && !members)) return 0;
+  for (int i = 0; i < count; ++i)
+    if (!members[i].W || members[i].W->n_out <= 0 || members[i].W->k_in <= 0 || members[i].r <= 0) return 0;
+  FwdMember mem[kMaxGroup];
+  fwd_members(members, count, mem);
+  if (M <= kFtMaxM) return gemv_layout(M, mem, count).total;
+  DeviceInfo *dev;
+  const int sms = current_device_info(&dev) == QLORA_OK ? dev->sms : 148;
+  size_t need = 0;
+  for (int i = 0; i < count; ++i)
+    need = std::max(need, fwd_layout(M, mem[i].W->n_out, mem[i].W->k_in, mem[i].r, sms).total);
+  return need;
+}
+
+int qlora_linear_fwd_group(const qlora_fwd_member_t *members, int count, int64_t M, void *ws, size_t ws_bytes,
+                           void *stream) {
+  int rc = check_fwd_group(members, count, M);
+  if (rc) return rc;
+  if (count == 0 || M == 0) return QLORA_OK;
+  DeviceInfo *dev;
+  rc = current_device_info(&dev);
+  if (rc) return rc;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  FwdMember mem[kMaxGroup];
+  fwd_members(members, count, mem);
+  if (M <= kFtMaxM) {
+    const GemvLayout L = gemv_layout(M, mem, count);
+    if (!ws || ws_bytes < L.total) return QLORA_ERR_WORKSPACE;
+    if (!aligned(ws, 256)) return QLORA_ERR_MISALIGNED;
+    uint8_t *w8 = reinterpret_cast<uint8_t *>(ws);
+    if (cudaMemsetAsync(w8, 0, L.zero_bytes, st) != cudaSuccess) return QLORA_ERR_CUDA;
+    for (int t = 0; t < kNumTables; ++t) {
+      FwdMember sub[kMaxGroup];
+      GemvLayout SL = L;
+      int n = 0;
+      for (int i = 0; i < count; ++i)
+        if (mem[i].W->table == t) {
+          sub[n] = mem[i];
+          SL.acc[n] = L.acc[i];
+          SL.tacc[n] = L.tacc[i];
+          ++n;
+        }
+      if (n == 0) continue;
+      rc = n == 1 ? few_token_fwd<1>(sub, 1, M, SL, w8, dev, st) : few_token_fwd<kMaxGroup>(sub, n, M, SL, w8, dev, st);
+      if (rc) return rc;
+    }
+    return QLORA_OK;
+  }
+  // Many tokens: each linear is a full tensor-core pass of its own; they run
+  // in order on the shared workspace.
+  size_t need = 0;
+  for (int i = 0; i < count; ++i)
+    need = std::max(need, fwd_layout(M, mem[i].W->n_out, mem[i].W->k_in, mem[i].r, dev->sms).total);
+  if (!ws || ws_bytes < need) return QLORA_ERR_WORKSPACE;
+  if (!aligned(ws, 256)) return QLORA_ERR_MISALIGNED;
+  for (int i = 0; i < count; ++i) {
+    const FwdMember &m = mem[i];
+    const FwdLayout L = fwd_layout(M, m.W->n_out, m.W->k_in, m.r, dev->sms);
+    rc = fwd_large(m.X, m.X, m.s, M, m.W, m.L1, m.L2, m.r, m.Y, m.T_save, reinterpret_cast<uint8_t *>(ws), L, dev,
+                   st);
+    if (rc) return rc;
+  }
+  return QLORA_OK;
 }
 
 int qlora_linear_bwd(const uint16_t *dY, const uint16_t *X, const uint16_t *T_saved, int64_t M,

@@ -206,6 +206,45 @@ QLORA_API int qlora_linear_bwd(const uint16_t *dY, const uint16_t *X, const uint
                      void *dL1, void *dL2, int grad_dtype, void *ws, size_t ws_bytes, void *stream);
 
 /*
+ * Grouped forward: the forward of up to QLORA_MAX_GROUP linears that see the
+ * same M tokens, each exactly as qlora_linear_fwd computes it (§2 Eq. 3 / §3
+ * Eq. 5), e.g. the q, k, v, gate and up projections of a decoder layer, which
+ * all read the layer's normalised input.
+ *   members[count]: a HOST array; member i names its own X [M x K_i], weight
+ *   W_i (host pointer to the view), L1 [K_i x r_i], L2 [r_i x N_i], scale s_i,
+ *   output Y [M x N_i] and optional T_save [M x 2 r_i] (layouts, shape and
+ *   alignment rules of qlora_linear_fwd).  Members may share X (read only);
+ *   no output may overlap another member's input or output.
+ *   With M <= 128 the whole group runs as one chain of three kernels (T
+ *   accumulation, fused doubleDequant + product, LoRA epilogue) over the
+ *   concatenated work of all members, instead of one chain per linear: the
+ *   per-linear launch gaps and tails of the few-token path disappear.
+ *   Members of different code tables (W->table) run as one chain per table.
+ *   With M > 128 every member runs its own tensor-core pass, in order.
+ *   count = 0 or M = 0: nothing is done.  Workspace:
+ *   qlora_linear_fwd_group_workspace_size(), which returns 0 for invalid
+ *   arguments.
+ * Errors: those of qlora_linear_fwd for any member, and QLORA_ERR_INVALID_ARG
+ * for count outside [0, QLORA_MAX_GROUP] or a NULL members array.
+ */
+#define QLORA_MAX_GROUP 8
+
+typedef struct {
+  const uint16_t *X;          /* [M x W->k_in] bf16 */
+  const qlora_nf4dq_t *W;     /* host pointer to the weight view */
+  const uint16_t *L1;         /* [k_in x r] bf16 */
+  const uint16_t *L2;         /* [r x n_out] bf16 */
+  int32_t r;
+  float s;
+  uint16_t *Y;                /* [M x n_out] bf16, written */
+  uint16_t *T_save;           /* [M x 2r] bf16 hi/lo pair, written; or NULL */
+} qlora_fwd_member_t;
+
+QLORA_API size_t qlora_linear_fwd_group_workspace_size(const qlora_fwd_member_t *members, int count, int64_t M);
+QLORA_API int qlora_linear_fwd_group(const qlora_fwd_member_t *members, int count, int64_t M, void *ws,
+                                     size_t ws_bytes, void *stream);
+
+/*
  * LoRA dropout (QLoRA Appendix B.2 trains with LoRA dropout, p = 0.1 up to
  * 13B and 0.05 at 33B and 65B).  It acts on the adapter's input only:
  *   Y  = X W_hat^T + T L2,   T = s drop(X) L1,   drop(X) = X * m / (1 - p);

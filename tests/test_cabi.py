@@ -86,3 +86,43 @@ def test_workspace_sizes_are_host_only(lib):
     assert lib.qlora_quantize_workspace_size(1 << 20) >= (1 << 20) // 64 * 4
     assert lib.qlora_linear_fwd_workspace_size(8192, 4096, 4096, 64) >= 4096 * 4096 * 2
     assert lib.qlora_linear_bwd_workspace_size(8192, 4096, 4096, 64) >= 4096 * 4096 * 2 + 2 * 8192 * 64 * 2
+
+
+def test_group_forward_host_rules(lib):
+    from bit_nf4_quantized_02_b200 import _lib
+    fake = 1 << 20
+    # an empty group does nothing; a NULL array or more than QLORA_MAX_GROUP members is refused
+    assert lib.qlora_linear_fwd_group(None, 0, 8, None, 0, None) == _lib.QLORA_OK
+    assert lib.qlora_linear_fwd_group(None, 1, 8, None, 0, None) == _lib.QLORA_ERR_INVALID_ARG
+    big = (_lib.FwdMember * (_lib.QLORA_MAX_GROUP + 1))()
+    assert lib.qlora_linear_fwd_group(big, _lib.QLORA_MAX_GROUP + 1, 8, None, 0, None) == _lib.QLORA_ERR_INVALID_ARG
+    assert lib.qlora_linear_fwd_group_workspace_size(big, _lib.QLORA_MAX_GROUP + 1, 8) == 0
+    # a member breaking a shape rule fails the whole group before anything runs
+    good = _lib.NF4DQ(192, 192, fake, fake, fake, fake)
+    bad = _lib.NF4DQ(192, 100, fake, fake, fake, fake)
+    arr = (_lib.FwdMember * 2)(_lib.FwdMember(fake, ctypes.pointer(good), fake, fake, 16, 1.0, fake, None),
+                               _lib.FwdMember(fake, ctypes.pointer(bad), fake, fake, 16, 1.0, fake, None))
+    assert lib.qlora_linear_fwd_group(arr, 2, 8, fake, 1 << 30, None) == _lib.QLORA_ERR_UNSUPPORTED_SHAPE
+
+
+def test_group_workspace_sizes(lib):
+    from bit_nf4_quantized_02_b200 import _lib
+    fake = 1 << 20
+    shapes = [(192, 192, 16), (320, 192, 16), (192, 320, 8), (72, 320, 8)]
+    views = [_lib.NF4DQ(n, k, fake, fake, fake, fake) for n, k, _ in shapes]
+    arr = (_lib.FwdMember * len(shapes))(*[_lib.FwdMember(fake, ctypes.pointer(v), fake, fake, r, 1.0, fake, None)
+                                           for v, (_, _, r) in zip(views, shapes)])
+    for M in (1, 16, 128, 129, 4096):
+        # a group of one needs what the single call needs
+        for i, (n, k, r) in enumerate(shapes):
+            one = (_lib.FwdMember * 1)(arr[i])
+            assert lib.qlora_linear_fwd_group_workspace_size(one, 1, M) == lib.qlora_linear_fwd_workspace_size(M, n, k, r)
+        total = lib.qlora_linear_fwd_group_workspace_size(arr, len(shapes), M)
+        singles = [lib.qlora_linear_fwd_workspace_size(M, n, k, r) for n, k, r in shapes]
+        if M <= 128:
+            # few tokens: every member keeps its own fp32 accumulators [M x (N + r)]
+            assert total >= sum(M * (n + r) * 4 for n, _, r in shapes)
+            assert total <= sum(singles)
+        else:
+            # many tokens: members run in turn on one shared workspace
+            assert total == max(singles)
