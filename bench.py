@@ -568,19 +568,21 @@ def run_decode(args, rank, world, local_rank):
         # algorithmic bytes: NF4+DQ weight, LoRA factors, X read, Y and T written
         nbytes += q.nbytes() + 2 * r * (K + N) + 2 * M * K + 2 * M * N + 2 * M * 2 * r
     torch.cuda.synchronize()
-    groups = [[members[n] for n in ("q", "k", "v", "gate", "up")], [members["o"]], [members["down"]]]
-    everything = [members[l.name] for l in wl.linears]
+    # grouped calls with their arguments marshalled once (qlora.FwdGroup)
+    groups = [qlora.FwdGroup([members[n] for n in ("q", "k", "v", "gate", "up")]),
+              qlora.FwdGroup([members["o"]]), qlora.FwdGroup([members["down"]])]
+    everything = qlora.FwdGroup([members[l.name] for l in wl.linears])
 
     def step():                       # the layer's data flow: three grouped calls
         for grp in groups:
-            qlora.linear_fwd_group(grp)
+            grp()
 
     def step_single():                # seven single-linear calls
         for X, q, L1, L2, Y, T in lins:
             qlora.linear_fwd(X, q, L1, L2, s, Y=Y, T=T)
 
     def step_one_group():             # all seven in one launch chain
-        qlora.linear_fwd_group(everything)
+        everything()
 
     ms, launches, clocks = _timed(qlora, step, args, dev, world, rank, local_rank)
     ms_graph = _graph_ms(step, dev, args.steps)

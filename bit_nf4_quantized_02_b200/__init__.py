@@ -28,6 +28,7 @@ __all__ = [
     "dequant",
     "linear_fwd",
     "linear_fwd_group",
+    "FwdGroup",
     "linear_bwd",
     "last_device_error",
     "t_value",
@@ -210,6 +211,48 @@ def linear_fwd(X: torch.Tensor, q: NF4Tensor, L1: torch.Tensor, L2: torch.Tensor
     return Y, (T if save_T else None)
 
 
+class FwdGroup:
+    """A grouped forward whose arguments are marshalled once (see
+    ``linear_fwd_group``).  Calling it runs the group again on the same
+    tensors, which it keeps alive; only the C call is made per run."""
+
+    def __init__(self, members, save_T: bool = True):
+        lib = _lib.load()
+        if not 0 < len(members) <= _lib.QLORA_MAX_GROUP:
+            raise ValueError(f"qlora: a group holds 1..{_lib.QLORA_MAX_GROUP} linears")
+        M = members[0]["X"].shape[0]
+        dev = members[0]["X"].device
+        arr = (_lib.FwdMember * len(members))()
+        self._keep, self.outputs = [], []
+        for i, m in enumerate(members):
+            X, q, L1, L2 = m["X"], m["q"], m["L1"], m["L2"]
+            K, r, N = X.shape[1], L1.shape[1], q.n_out
+            if X.shape[0] != M or X.device != dev:
+                raise ValueError("qlora: the members of a group share the token count and the device")
+            if K != q.k_in or L1.shape[0] != K or tuple(L2.shape) != (r, N):
+                raise ValueError("qlora: shape mismatch")
+            Y = m.get("Y")
+            if Y is None:
+                Y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+            T = m.get("T")
+            if save_T and T is None:
+                T = torch.empty((M, 2 * r), dtype=torch.bfloat16, device=dev)
+            w = q.as_struct()
+            self._keep += [w, X, q, L1, L2]
+            arr[i] = _lib.FwdMember(_ptr(_bits(X)), ctypes.pointer(w), _ptr(_bits(L1)), _ptr(_bits(L2)), r,
+                                    float(m["s"]), _ptr(_bits(Y)), _ptr(T) if save_T else None)
+            self.outputs.append((Y, T if save_T else None))
+        self._arr, self._n, self._M, self._dev = arr, len(members), M, dev
+        self._ws_bytes = lib.qlora_linear_fwd_group_workspace_size(arr, len(members), M)
+        self._fn = lib.qlora_linear_fwd_group
+
+    def __call__(self) -> list:
+        ws = _WS.get(self._ws_bytes, self._dev)
+        _lib.check(self._fn(self._arr, self._n, self._M, ws.data_ptr(), ws.numel(), _stream(self._dev)),
+                   "qlora_linear_fwd_group")
+        return self.outputs
+
+
 def linear_fwd_group(members, save_T: bool = True) -> list:
     """The forward of several linears that see the same tokens, in one call.
 
@@ -217,37 +260,11 @@ def linear_fwd_group(members, save_T: bool = True) -> list:
     (NF4Tensor), ``L1`` [K_i, r_i], ``L2`` [r_i, N_i], ``s`` and optionally the
     outputs ``Y`` [M, N_i] and ``T`` [M, 2 r_i].  Every member computes what
     ``linear_fwd`` computes; with at most 128 tokens the whole group runs as
-    one launch chain.  Returns [(Y, T or None)] in member order.
+    one launch chain.  Returns [(Y, T or None)] in member order.  For repeated
+    calls on the same tensors, ``FwdGroup(members)`` marshals the arguments
+    once.
     """
-    lib = _lib.load()
-    if not 0 < len(members) <= _lib.QLORA_MAX_GROUP:
-        raise ValueError(f"qlora: a group holds 1..{_lib.QLORA_MAX_GROUP} linears")
-    M = members[0]["X"].shape[0]
-    dev = members[0]["X"].device
-    arr = (_lib.FwdMember * len(members))()
-    keep, outs = [], []
-    for i, m in enumerate(members):
-        X, q, L1, L2 = m["X"], m["q"], m["L1"], m["L2"]
-        K, r, N = X.shape[1], L1.shape[1], q.n_out
-        if X.shape[0] != M or X.device != dev:
-            raise ValueError("qlora: the members of a group share the token count and the device")
-        if K != q.k_in or L1.shape[0] != K or tuple(L2.shape) != (r, N):
-            raise ValueError("qlora: shape mismatch")
-        Y = m.get("Y")
-        if Y is None:
-            Y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
-        T = m.get("T")
-        if save_T and T is None:
-            T = torch.empty((M, 2 * r), dtype=torch.bfloat16, device=dev)
-        w = q.as_struct()
-        keep.append(w)
-        arr[i] = _lib.FwdMember(_ptr(_bits(X)), ctypes.pointer(w), _ptr(_bits(L1)), _ptr(_bits(L2)), r,
-                                float(m["s"]), _ptr(_bits(Y)), _ptr(T) if save_T else None)
-        outs.append((Y, T if save_T else None))
-    ws = _WS.get(lib.qlora_linear_fwd_group_workspace_size(arr, len(members), M), dev)
-    _lib.check(lib.qlora_linear_fwd_group(arr, len(members), M, _ptr(ws), ws.numel(), _stream(dev)),
-               "qlora_linear_fwd_group")
-    return outs
+    return FwdGroup(members, save_T)()
 
 
 def t_value(T: torch.Tensor) -> torch.Tensor:

@@ -114,6 +114,27 @@ def test_repeated_group_calls_reuse_workspace():
         _check(host, outs)
 
 
+def test_prepared_group_follows_its_inputs():
+    """A FwdGroup marshalled once and run again after its inputs were
+    overwritten in place computes the new inputs' forward."""
+    M = 16
+    host, dev = _layer_members(M, 7700)
+    grp = qlora.FwdGroup(dev)
+    grp()
+    torch.cuda.synchronize()
+    _check(host, grp.outputs)
+    g = inputs.rng(7701)
+    done = set()
+    for m in dev:                          # H is shared by five members: overwrite it once
+        if m["X"].data_ptr() not in done:
+            done.add(m["X"].data_ptr())
+            m["X"].copy_(inputs.normal_bf16(g, tuple(m["X"].shape)).cuda())
+    new_host = [(name, W, m["X"].cpu(), L1, L2, t) for m, (name, W, X, L1, L2, t) in zip(dev, host)]
+    grp()
+    torch.cuda.synchronize()
+    _check(new_host, grp.outputs)
+
+
 def test_single_member_group_matches_linear_fwd_path():
     """A group of one is the single-linear call (same kernels, same work split)."""
     M = 16
