@@ -414,11 +414,14 @@ int tc_gemm(cudaStream_t st, DeviceInfo *dev, int64_t M, int64_t N, int nseg, co
 int dequant_launch(const qlora_nf4dq_t *W, __nv_bfloat16 *out, cudaStream_t st, int sms) {
   const int64_t numel = W->n_out * W->k_in;
   if (numel == 0) return QLORA_OK;
-  const int64_t n8 = numel >> 3;
-  const int grid = (int)std::max<int64_t>(1, std::min<int64_t>((n8 + 255) / 256, (int64_t)sms * 16));
+  DeviceInfo *dev;
+  int rc = current_device_info(&dev);
+  if (rc) return rc;
+  const int64_t nchunks = numel / kDqChunk;
+  const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(nchunks, (int64_t)sms * kDqCtasPerSm));
   ProfScope prof(QLORA_KERNEL_DEQUANT, st);
-  return launch_pdl(nf4_dequant_kernel, dim3(grid), dim3(256), 0, st, W->codes, W->c2_fp8, W->c1, W->c2_mean, numel,
-                    out, (int)W->table);
+  return launch_pdl(nf4_dequant_kernel, dim3(grid), dim3(kDqThreads), 0, st, W->codes, W->c2_fp8, W->c1,
+                    W->c2_mean, numel, out, (int)W->table, dev->err);
 }
 
 int check_weight(const qlora_nf4dq_t *W) {

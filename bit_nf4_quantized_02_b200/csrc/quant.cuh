@@ -412,41 +412,119 @@ __global__ void __launch_bounds__(32 * kDqWarps) dq_constants_kernel(const float
 // K3: doubleDequant (Eq. 6) to bf16:
 //   c2_hat = fma(E4M3(code8_b), c1_beta, mu)   (one rounding)
 //   W_hat  = bf16_rne(fp32(NF4[code] * c2_hat))
-// Each thread converts 8 elements (one 32-bit word of nibbles -> one 16-byte
-// store); a scalar path finishes a numel that is not a multiple of 8.
-__global__ void __launch_bounds__(256) nf4_dequant_kernel(const uint8_t *__restrict__ codes,
-                                                          const uint8_t *__restrict__ c2_fp8,
-                                                          const float *__restrict__ c1,
-                                                          const float *__restrict__ mu_p, int64_t numel,
-                                                          __nv_bfloat16 *__restrict__ out, int table) {
+// Streamed in chunks of kDqChunk weights (128 blocks of 64, inside one
+// 256-block group, so one c1 per chunk).  CTA b takes chunks b, b + grid,
+// ...; thread 0 brings each chunk's packed codes (4 KB) and E4M3 block codes
+// (128 B) into a ring of shared-memory stages with bulk copies
+// (cp.async.bulk, completing on the stage's mbarrier), kDqStages chunks ahead,
+// so every SM keeps tens of KB of reads in flight.  Thread t decodes the
+// 32-bit code words t, t + 256, t + 512, ... of a stage (8 weights each), so
+// each warp's 16-byte stores cover 512 contiguous bytes.  The last CTA
+// converts the weights after the last whole chunk with plain loads.
+constexpr int kDqChunk = 8192;
+constexpr int kDqCodeBytes = kDqChunk / 2;
+constexpr int kDqC2Bytes = kDqChunk / 64;
+constexpr int kDqStageBytes = kDqCodeBytes + kDqC2Bytes;
+constexpr int kDqStages = 6;
+constexpr int kDqThreads = 256;
+constexpr int kDqCtasPerSm = 8;
+constexpr int kDqWordsPerThread = kDqCodeBytes / 4 / kDqThreads;
+static_assert(kDqCodeBytes == 4 * kDqWordsPerThread * kDqThreads, "whole code words per thread");
+static_assert(256 % (kDqChunk / 64) == 0, "a chunk lies inside one 256-block group");
+static_assert(kDqStageBytes % 16 == 0 && kDqC2Bytes % 16 == 0, "bulk-copy sizes and offsets");
+
+// Bulk copy global -> shared of `bytes` (multiple of 16; both addresses
+// 16-byte aligned), completing on mbarrier `bar`.
+__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+               "l"(src), "r"(bytes), "r"(bar)
+               : "memory");
+}
+
+// Eight weights from one 32-bit word of codes (element i in bits [4i, 4i+4)).
+__device__ __forceinline__ uint4 dq_decode8(uint32_t q, float c2h, const float *lut) {
+  uint32_t o[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float lo = __fmul_rn(lut[(q >> (8 * i)) & 0xF], c2h);
+    const float hi = __fmul_rn(lut[(q >> (8 * i + 4)) & 0xF], c2h);
+    const __nv_bfloat162 p = __floats2bfloat162_rn(lo, hi);
+    o[i] = *reinterpret_cast<const uint32_t *>(&p);
+  }
+  return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+__global__ void __launch_bounds__(kDqThreads, kDqCtasPerSm) nf4_dequant_kernel(
+    const uint8_t *__restrict__ codes, const uint8_t *__restrict__ c2_fp8, const float *__restrict__ c1,
+    const float *__restrict__ mu_p, int64_t numel, __nv_bfloat16 *__restrict__ out, int table, int *err) {
+  __shared__ __align__(128) uint8_t stage[kDqStages][kDqStageBytes];
+  __shared__ __align__(8) uint64_t full[kDqStages];
   __shared__ float lut[16];
   if (threadIdx.x < 16) lut[threadIdx.x] = kLevels[table][threadIdx.x];
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kDqStages; ++i) mbar_init(smem_u32(&full[i]), 1);
+    fence_mbar_init();
+  }
   __syncthreads();
   pdl_trigger();
   pdl_wait();
   const float mu = ld_dep_f32(mu_p);
-  const int64_t n8 = numel >> 3;
-  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-  for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < n8; e += stride) {
-    const uint32_t q = ld_dep_u32(codes + 4 * e);
-    const int64_t b = e >> 3;
-    const float c2h = __fmaf_rn(e4m3_to_f32((uint8_t)ld_dep_u8(c2_fp8 + b)), ld_dep_f32(c1 + (b >> 8)), mu);
-    uint32_t o[4];
+  const int64_t nchunks = numel / kDqChunk;
+  const int64_t step = gridDim.x;
+  const int64_t mine = (int64_t)blockIdx.x < nchunks ? (nchunks - 1 - blockIdx.x) / step + 1 : 0;
+  auto issue = [&](int64_t j) {   // thread 0: chunk number j of this CTA into stage j % kDqStages
+    const int64_t chunk = blockIdx.x + j * step;
+    const uint32_t bar = smem_u32(&full[j % kDqStages]);
+    const uint32_t dst = smem_u32(stage[j % kDqStages]);
+    mbar_arrive_expect_tx(bar, kDqStageBytes);
+    bulk_g2s(dst, codes + chunk * kDqCodeBytes, kDqCodeBytes, bar);
+    bulk_g2s(dst + kDqCodeBytes, c2_fp8 + chunk * kDqC2Bytes, kDqC2Bytes, bar);
+  };
+  int64_t issued = 0, done = 0;
+  if (threadIdx.x == 0)
+    for (; issued < mine && issued < kDqStages; ++issued) issue(issued);
+  const int t = threadIdx.x;
+  // c1 of a chunk (one per chunk), loaded a chunk ahead
+  auto c1_of = [&](int64_t j) { return ld_dep_f32(c1 + (((blockIdx.x + j * step) * (kDqChunk / 64)) >> 8)); };
+  float c1_next = mine > 0 ? c1_of(0) : 0.f;
+  for (; done < mine; ++done) {
+    const int st = (int)(done % kDqStages);
+    const bool got = mbar_wait(smem_u32(&full[st]), (uint32_t)((done / kDqStages) & 1), err, DEV_TIMEOUT_MMA);
+    if (__syncthreads_or(!got)) break;
+    const int64_t chunk = blockIdx.x + done * step;
+    const float c1v = c1_next;
+    if (done + 1 < mine) c1_next = c1_of(done + 1);
+    const uint8_t *sc = stage[st];
+    uint4 *dst = reinterpret_cast<uint4 *>(out + chunk * kDqChunk);
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const float lo = __fmul_rn(lut[(q >> (8 * i)) & 0xF], c2h);
-      const float hi = __fmul_rn(lut[(q >> (8 * i + 4)) & 0xF], c2h);
-      const __nv_bfloat162 p = __floats2bfloat162_rn(lo, hi);
-      o[i] = *reinterpret_cast<const uint32_t *>(&p);
+    for (int i = 0; i < kDqWordsPerThread; ++i) {
+      const int w = t + kDqThreads * i;                           // code word of the chunk
+      const uint32_t q = reinterpret_cast<const uint32_t *>(sc)[w];
+      const float c2h = __fmaf_rn(e4m3_to_f32(sc[kDqCodeBytes + (w >> 3)]), c1v, mu);
+      dst[w] = dq_decode8(q, c2h, lut);
     }
-    reinterpret_cast<uint4 *>(out)[e] = make_uint4(o[0], o[1], o[2], o[3]);
+    __syncthreads();   // stage st consumed by every thread
+    if (threadIdx.x == 0 && issued < mine) issue(issued++);
   }
-  if (blockIdx.x == 0 && threadIdx.x < (numel & 7)) {
-    const int64_t i = (n8 << 3) + threadIdx.x;
-    const int64_t b = i >> 6;
-    const float c2h = __fmaf_rn(e4m3_to_f32((uint8_t)ld_dep_u8(c2_fp8 + b)), ld_dep_f32(c1 + (b >> 8)), mu);
-    const uint32_t code = (ld_dep_u8(codes + (i >> 1)) >> ((i & 1) * 4)) & 0xF;
-    out[i] = __float2bfloat16_rn(__fmul_rn(lut[code], c2h));
+  // A CTA never exits with bulk copies into its shared memory in flight.
+  if (done < mine && threadIdx.x == 0)
+    for (int64_t j = done; j < issued; ++j)
+      if (!mbar_wait(smem_u32(&full[j % kDqStages]), (uint32_t)((j / kDqStages) & 1), err, DEV_TIMEOUT_DRAIN)) break;
+  // Weights after the last whole chunk: 8 per thread, then a scalar rest.
+  if (blockIdx.x == gridDim.x - 1) {
+    const int64_t n8 = numel >> 3;
+    for (int64_t e = nchunks * (kDqChunk / 8) + t; e < n8; e += kDqThreads) {
+      const int64_t b = e >> 3;
+      const float c2h = __fmaf_rn(e4m3_to_f32((uint8_t)ld_dep_u8(c2_fp8 + b)), ld_dep_f32(c1 + (b >> 8)), mu);
+      reinterpret_cast<uint4 *>(out)[e] = dq_decode8(ld_dep_u32(codes + 4 * e), c2h, lut);
+    }
+    if (t < (numel & 7)) {
+      const int64_t i = (n8 << 3) + t;
+      const int64_t b = i >> 6;
+      const float c2h = __fmaf_rn(e4m3_to_f32((uint8_t)ld_dep_u8(c2_fp8 + b)), ld_dep_f32(c1 + (b >> 8)), mu);
+      const uint32_t code = (ld_dep_u8(codes + (i >> 1)) >> ((i & 1) * 4)) & 0xF;
+      out[i] = __float2bfloat16_rn(__fmul_rn(lut[code], c2h));
+    }
   }
 }
 

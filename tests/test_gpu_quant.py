@@ -31,7 +31,7 @@ def _check_bit_exact(W_cpu: torch.Tensor):
 
 
 @pytest.mark.parametrize("shape", [(1, 64), (1, 1), (3, 100), (7, 333), (2, 256), (5, 320), (64, 4096),
-                                   (257, 64 * 257), (33, 1000)])
+                                   (257, 64 * 257), (33, 1000), (1, 8205), (3, 8192), (1, 8192 * 9 + 64)])
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
 def test_quantize_dequant_bit_exact_small(shape, dtype):
     g = inputs.rng(100 + shape[0] * 7 + shape[1])
