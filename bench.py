@@ -768,6 +768,87 @@ def run_reference(args, rank, world):
     }
 
 
+def run_cublas_compare(args, rank, world, local_rank):
+    """Context for the GEMM roofline: the library's Y and dX products (X W_hat^T
+    + T_hi L2 and dY W_hat + G_hi L1^T, event log of linear_fwd / linear_bwd)
+    against cuBLAS (torch.mm, bf16 in, fp32 accumulate, bf16 out) on the same
+    LLaMA-7B shapes at 8192 tokens."""
+    import bit_nf4_quantized_02_b200 as qlora
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    wl = WL
+    M, r, s = wl.M, wl.r, wl.s
+    rows = []
+    seen = set()
+    for i, lin in enumerate(wl.linears):
+        N, K = lin.n_out, lin.k_in
+        if (N, K) in seen:
+            continue
+        seen.add((N, K))
+        X = inputs.device_normal((M, K), 1.0, wl.seed + 7 * i, dev, torch.bfloat16)
+        W = inputs.device_normal((N, K), inputs.WEIGHT_STD, wl.seed + 7 * i + 1, dev)
+        q = qlora.quantize_nf4_dq(W)
+        Wb = qlora.dequant(q)
+        L1 = inputs.device_normal((K, r), 1.0 / np.sqrt(K), wl.seed + 7 * i + 2, dev, torch.bfloat16)
+        L2 = inputs.device_normal((r, N), inputs.L2_STD, wl.seed + 7 * i + 3, dev, torch.bfloat16)
+        Y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+        T = torch.empty(M, 2 * r, dtype=torch.bfloat16, device=dev)
+        for _ in range(args.warmup):
+            qlora.linear_fwd(X, q, L1, L2, s, Y=Y, T=T)
+            torch.mm(X, Wb.t(), out=Y)
+        torch.cuda.synchronize()
+        dY = inputs.device_normal((M, N), 1.0, wl.seed + 7 * i + 4, dev, torch.bfloat16)
+        dX = torch.empty(M, K, dtype=torch.bfloat16, device=dev)
+        for _ in range(args.warmup):
+            qlora.linear_bwd(dY, X, T, q, L1, L2, s, dX=dX)
+            torch.mm(dY, Wb, out=dX)
+        torch.cuda.synchronize()
+        qlora.profile_start(args.steps * 16 + 16)
+        for _ in range(args.steps):
+            qlora.linear_fwd(X, q, L1, L2, s, Y=Y, T=T)
+            qlora.linear_bwd(dY, X, T, q, L1, L2, s, dX=dX)
+        torch.cuda.synchronize()
+        log = qlora.profile_stop()
+        ours = [ms for kind, ms in log if kind == "gemm_Y"]
+        ours_dx = [ms for kind, ms in log if kind == "gemm_dX"]
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+        warm, cold, warm_dx, cold_dx = [], [], [], []
+        for _ in range(args.steps):
+            for lst, fl, fn in ((warm, False, lambda: torch.mm(X, Wb.t(), out=Y)),
+                                (cold, True, lambda: torch.mm(X, Wb.t(), out=Y)),
+                                (warm_dx, False, lambda: torch.mm(dY, Wb, out=dX)),
+                                (cold_dx, True, lambda: torch.mm(dY, Wb, out=dX))):
+                if fl:
+                    flush.fill_(1)    # evict the operands from L2 (256 MB written)
+                e0.record()
+                fn()
+                e1.record()
+                torch.cuda.synchronize()
+                lst.append(e0.elapsed_time(e1))
+        f_ours = linear_flops(M, N, K, r)["gemm_Y"]
+        f_mm = 2 * M * N * K
+        rows.append({"shape": f"{M}x{N}x{K}", "linears": [l.name for l in wl.linears if (l.n_out, l.k_in) == (N, K)],
+                     "ours_gemm_Y_ms": statistics.median(ours), "ours_tflops": f_ours / statistics.median(ours) / 1e9,
+                     "cublas_mm_ms_l2_warm": statistics.median(warm),
+                     "cublas_tflops_l2_warm": f_mm / statistics.median(warm) / 1e9,
+                     "cublas_mm_ms_l2_flushed": statistics.median(cold),
+                     "cublas_tflops_l2_flushed": f_mm / statistics.median(cold) / 1e9,
+                     "ours_gemm_dX_ms": statistics.median(ours_dx),
+                     "ours_dx_tflops": linear_flops(M, N, K, r)["gemm_dX"] / statistics.median(ours_dx) / 1e9,
+                     "cublas_dx_tflops_l2_warm": f_mm / statistics.median(warm_dx) / 1e9,
+                     "cublas_dx_tflops_l2_flushed": f_mm / statistics.median(cold_dx) / 1e9})
+        del flush, dY, dX
+        del X, W, q, Wb, L1, L2, Y, T
+    peaks, src = load_peaks()
+    return {"metric": "Y product TFLOP/s, library tcgen05 GEMM against cuBLAS on the same shapes", "unit": "TFLOP/s",
+            "rows": rows, "peak_bf16_tflops": peaks.get("bf16_tflops"), "peak_source": src,
+            "note": "median over --steps single calls; the library's time is its event-log time of the Y launch "
+                    "inside linear_fwd, right after the dequant and T launches (which also adds T_hi L2 as 2 M r N "
+                    "more FLOPs); cuBLAS via torch.mm on the dequantized weight, timed back to back (L2 warm) and "
+                    "after writing 256 MB (L2 flushed)"}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -782,6 +863,8 @@ def main():
                     help="LoRA dropout probability on every adapter (single-layer training workloads)")
     ap.add_argument("--tokens", type=int, default=None,
                     help="llama65b-decode: tokens per step (default 16; 33..128 run the tcgen05 fused forward)")
+    ap.add_argument("--cublas-compare", action="store_true",
+                    help="print the library's Y GEMM against cuBLAS (torch.mm) on the LLaMA-7B shapes, then exit")
     ap.add_argument("--linear", choices=[l.name for l in WL.linears], default=None,
                     help="restrict the step to one linear of the layer (profiling runs)")
     ap.add_argument("--workload", choices=list(TRAIN) + ["llama65b-decode", "quantizer"], default="llama7b-train",
@@ -804,7 +887,9 @@ def main():
             torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
                                                  device_id=torch.device("cuda", local_rank))
         try:
-            if args.workload == "llama65b-decode":
+            if args.cublas_compare:
+                out = run_cublas_compare(args, rank, world, local_rank)
+            elif args.workload == "llama65b-decode":
                 out = run_decode(args, rank, world, local_rank)
             elif args.workload == "quantizer":
                 out = run_quantizer(args, rank, world, local_rank)
