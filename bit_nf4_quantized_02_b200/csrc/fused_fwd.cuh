@@ -112,8 +112,8 @@ struct FtMaps {
 
 // Item `it` of a group -> its linear l, row tile rt and stage ks.
 template <int GM>
-__device__ __forceinline__ const FtMember &ft_item(const FtArgs<GM> &p, int it, int &rt, int &ks) {
-  const int l = group_member<GM>(p.beg, p.count, it);
+__device__ __forceinline__ const FtMember &ft_item(const FtArgs<GM> &p, int it, int &l, int &rt, int &ks) {
+  l = group_member<GM>(p.beg, p.count, it);
   const FtMember &m = p.m[l];
   const int li = it - p.beg[l];
   rt = li / m.kstages;
@@ -268,9 +268,8 @@ __global__ void __launch_bounds__(FtCfg<MP>::kThreads, 1)
     int stage = 0;
     uint32_t phase = 0, used = 0, last_parity = 0;
     for (int it = i0; it < i1; ++it) {
-      int rt, ks;
-      const FtMember &m = ft_item<GM>(p, it, rt, ks);
-      const int l = group_member<GM>(p.beg, p.count, it);
+      int l, rt, ks;
+      const FtMember &m = ft_item<GM>(p, it, l, rt, ks);
       const bool got = mbar_wait(smem_u32(empty_bar + stage), phase ^ 1, p.err, DEV_TIMEOUT_PRODUCER);
       if (!__all_sync(0xFFFFFFFFu, got)) break;
       const uint32_t fb = smem_u32(full_bar + stage);
@@ -314,8 +313,8 @@ __global__ void __launch_bounds__(FtCfg<MP>::kThreads, 1)
       bool ok = true;
       uint32_t accumulate = 0;
       for (int it = i0; it < i1 && ok; ++it) {
-        int rt, ks;
-        const FtMember &m = ft_item<GM>(p, it, rt, ks);
+        int l, rt, ks;
+        const FtMember &m = ft_item<GM>(p, it, l, rt, ks);
         const int kblocks = m.K >> 6;
         const bool first = it == i0 || ks == 0;
         const bool last = it == i1 - 1 || ks == m.kstages - 1;
@@ -376,8 +375,8 @@ __global__ void __launch_bounds__(FtCfg<MP>::kThreads, 1)
     uint32_t phase = 0;
     uint32_t writes = 0;     // blocks this group has stored into its slot
     for (int it = i0; it < i1; ++it) {
-      int rt, ks;
-      const FtMember &m = ft_item<GM>(p, it, rt, ks);
+      int l, rt, ks;
+      const FtMember &m = ft_item<GM>(p, it, l, rt, ks);
       const int kblocks = m.K >> 6;
       const float mu = __ldg(m.mu);
       const int nkb = min(4, kblocks - ks * 4);
@@ -433,8 +432,8 @@ __global__ void __launch_bounds__(FtCfg<MP>::kThreads, 1)
     const int q = warp & 3;          // TMEM lane quarter
     int t = 0;
     for (int it = i0; it < i1; ++it) {
-      int rt, ks;
-      const FtMember &m = ft_item<GM>(p, it, rt, ks);
+      int l, rt, ks;
+      const FtMember &m = ft_item<GM>(p, it, l, rt, ks);
       if (!(it == i1 - 1 || ks == m.kstages - 1)) continue;   // not the end of a row-tile segment
       const int acc = t & 1;
       const bool got = mbar_wait(smem_u32(tfull_bar + acc), (t >> 1) & 1u, p.err, DEV_TIMEOUT_EPILOGUE);

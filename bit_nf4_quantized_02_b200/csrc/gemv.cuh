@@ -12,7 +12,8 @@
 //                            overlaps the first kernel completely);
 //   gemv_epilogue_kernel     Y = bf16(acc + s T L2), and T = s X L1 as a bf16
 //                            hi/lo pair for the backward.
-// gemv_fwd_kernel, persistent, 160 threads per CTA (3 CTAs per SM):
+// gemv_fwd_kernel, persistent, 160 threads per CTA (4 CTAs per SM up to 16
+// tokens, 3 at 32):
 //   * warp 4 is a TMA producer: per stage, 64 weight rows x 256 K of packed
 //     codes (128-byte swizzle) and the matching X tile (3-D view of X,
 //     [token][64-block][64], 128-byte swizzle) into a ring of mbarrier stages;
