@@ -182,11 +182,26 @@ def build_layer(dev, rank, wl=WL):
 
 def make_step(qlora, lins, grads, world, wl=WL, dropout=0.0):
     """One step; `ready(t)` (if given) is called before the step first reads input t.
-    With `dropout` > 0 each linear applies LoRA dropout with its own keep mask."""
+    With `dropout` > 0 each linear applies LoRA dropout with its own keep mask.
+    Without dropout the forward runs the linears that read the same input as
+    one grouped call (q, k, v, gate and up on the layer input), in the order
+    of their first use."""
+    groups = []
+    if dropout == 0:
+        by_x = {}
+        for l in lins:
+            by_x.setdefault(l.X.data_ptr(), []).append(l)
+        groups = [(g[0].X, qlora.FwdGroup([{"X": l.X, "q": l.q, "L1": l.L1, "L2": l.L2, "s": wl.s, "Y": l.Y,
+                                             "T": l.T} for l in g])) for g in by_x.values()]
+
     def step(ready=None):
         for l in lins:
             l.q = qlora.quantize_nf4_dq(l.W, out=l.q)
-        for l in lins:
+        for X, grp in groups:
+            if ready:
+                ready(X)
+            grp()
+        for l in (lins if dropout > 0 else []):
             if ready:
                 ready(l.X)
                 if l.mask is not None:
@@ -411,6 +426,8 @@ def run_ours(args, rank, world, local_rank):
                    "parallelism": f"dp{world}" if world > 1 else "single",
                    "step": f"quantize {7 * wl.layers} fp32 weights to NF4+DQ, fwd + bwd of the "
                            f"{7 * wl.layers} QLoRA linears"
+                           + (" (forward of the linears that read the same input as one grouped call: q, k, v, "
+                              "gate, up on the layer input)" if wl.layers == 1 and args.dropout == 0 else "")
                            + (" (layer to layer: H' = bf16(down(up(H)) + R))" if wl.layers > 1 else "")
                            + (", all-reduce of adapter grads" if world > 1 else "")
                            + (f", LoRA dropout p = {args.dropout:g} on every adapter (one seeded keep mask per "

@@ -14,6 +14,7 @@
 #include "gemv.cuh"
 #include "fused_fwd.cuh"
 #include "dropout.cuh"
+#include "group.cuh"
 
 namespace qlora {
 
@@ -955,6 +956,18 @@ namespace {
 // Forward above the few-token sizes: dequant + tcgen05 GEMMs.  The adapter's
 // down-projection reads Xt with scale t_scale: T = t_scale Xt L1 (Xt = X and
 // t_scale = s without dropout).
+// doubleDequant of W into w_hat (Eq. 6), then Y = X W_hat^T + T_hi L2 (the
+// LoRA up-projection as extra K-steps of the same accumulation), given T as
+// a bf16 hi/lo pair [M x 2r].
+int fwd_y(const uint16_t *X, int64_t M, const qlora_nf4dq_t *W, const uint16_t *L2, int r, const uint16_t *T,
+          uint16_t *Y, __nv_bfloat16 *w_hat, DeviceInfo *dev, cudaStream_t st) {
+  const int64_t N = W->n_out, K = W->k_in;
+  int rc = dequant_launch(W, w_hat, st, dev->sms);
+  if (rc) return rc;
+  GemmSeg sY[2] = {{{X, M, K, K, 0}, {w_hat, N, K, K, 0}}, {{T, M, r, 2 * r, 0}, {L2, N, r, N, 1}}};
+  return tc_gemm(st, dev, M, N, 2, sY, 1.f, Y, N, 1, 0, nullptr, QLORA_KERNEL_GEMM_Y);
+}
+
 int fwd_large(const uint16_t *X, const uint16_t *Xt, float t_scale, int64_t M, const qlora_nf4dq_t *W,
               const uint16_t *L1, const uint16_t *L2, int r, uint16_t *Y, uint16_t *T_save, uint8_t *w8,
               const FwdLayout &L, DeviceInfo *dev, cudaStream_t st) {
@@ -1116,6 +1129,145 @@ int qlora_linear_fwd(const uint16_t *X, int64_t M, const qlora_nf4dq_t *W, const
   return fwd_large(X, X, s, M, W, L1, L2, r, Y, T_save, reinterpret_cast<uint8_t *>(ws), L, dev, st);
 }
 
+// ------------------------------------------------ grouped forward, many tokens
+// Sets of members that read the same X (same pointer and K), in order of
+// their first member: set_of[i] is member i's set.
+static int x_sets(const FwdMember *mem, int count, int *set_of) {
+  int n = 0;
+  for (int i = 0; i < count; ++i) {
+    set_of[i] = -1;
+    for (int j = 0; j < i; ++j)
+      if (mem[j].X == mem[i].X && mem[j].W->k_in == mem[i].W->k_in) {
+        set_of[i] = set_of[j];
+        break;
+      }
+    if (set_of[i] < 0) set_of[i] = n++;
+  }
+  return n;
+}
+
+// Workspace: the bf16 weight (largest member, reused member after member);
+// T_cat fp32 [M x R] and L1_cat bf16 [K x R] of the largest shared-input set;
+// each member's T pair [M x 2r] (used where it passes no T_save); the split-K
+// partials of the largest adapter product.
+struct GroupLargeLayout {
+  size_t w_hat, t_cat, l1_cat, t_own[kMaxGroup], split, total;
+};
+
+static GroupLargeLayout group_large_layout(int64_t M, const FwdMember *mem, int count, int sms) {
+  int set_of[kMaxGroup];
+  const int nsets = x_sets(mem, count, set_of);
+  size_t w = 0, tcat = 0, l1cat = 0, split = 0;
+  for (int i = 0; i < count; ++i) w = std::max(w, (size_t)mem[i].W->n_out * mem[i].W->k_in * 2);
+  for (int s = 0; s < nsets; ++s) {
+    int64_t R = 0, K = 0;
+    int members = 0;
+    for (int i = 0; i < count; ++i)
+      if (set_of[i] == s) {
+        R += mem[i].r;
+        K = mem[i].W->k_in;
+        ++members;
+        split = std::max(split, gemm_split_ws_bytes(M, mem[i].r, K, sms, true));
+      }
+    if (members > 1) {
+      tcat = std::max(tcat, (size_t)M * R * 4);
+      l1cat = std::max(l1cat, (size_t)K * R * 2);
+      split = std::max(split, gemm_split_ws_bytes(M, R, K, sms, true));
+    }
+  }
+  GroupLargeLayout L;
+  size_t off = 0;
+  L.w_hat = off;
+  off += align_up(w);
+  L.t_cat = off;
+  off += align_up(tcat);
+  L.l1_cat = off;
+  off += align_up(l1cat);
+  for (int i = 0; i < count; ++i) {
+    L.t_own[i] = off;
+    off += align_up((size_t)M * 2 * mem[i].r * 2);
+  }
+  L.split = off;
+  off += align_up(split);
+  L.total = off;
+  return L;
+}
+
+// The grouped forward at many tokens (M > 128) on a workspace laid out by
+// group_large_layout.
+static int group_large_fwd(int64_t M, const FwdMember *mem, int count, uint8_t *w8, const GroupLargeLayout &L,
+                           DeviceInfo *dev, cudaStream_t st) {
+  int set_of[kMaxGroup];
+  const int nsets = x_sets(mem, count, set_of);
+  __nv_bfloat16 *w_hat = reinterpret_cast<__nv_bfloat16 *>(w8 + L.w_hat);
+  float *split_ws = reinterpret_cast<float *>(w8 + L.split);
+  for (int s = 0; s < nsets; ++s) {
+    int idx[kMaxGroup], n = 0;
+    for (int i = 0; i < count; ++i)
+      if (set_of[i] == s) idx[n++] = i;
+    uint16_t *T[kMaxGroup];
+    for (int k = 0; k < n; ++k) {
+      const FwdMember &m = mem[idx[k]];
+      T[k] = m.T_save ? m.T_save : reinterpret_cast<uint16_t *>(w8 + L.t_own[idx[k]]);
+    }
+    int rc;
+    if (n == 1) {
+      const FwdMember &m = mem[idx[0]];
+      FwdLayout FL;
+      FL.w_hat = L.w_hat;
+      FL.t = L.t_own[idx[0]];
+      FL.split = L.split;
+      FL.total = L.total;
+      rc = fwd_large(m.X, m.X, m.s, M, m.W, m.L1, m.L2, m.r, m.Y, m.T_save, w8, FL, dev, st);
+      if (rc) return rc;
+      continue;
+    }
+    // The shared input's adapter product: X [L1_a | L1_b | ...] into T_cat.
+    const int64_t K = mem[idx[0]].W->k_in;
+    TScatterArgs a;
+    std::memset(&a, 0, sizeof(a));
+    int R = 0;
+    uint16_t *l1_cat = reinterpret_cast<uint16_t *>(w8 + L.l1_cat);
+    for (int k = 0; k < n; ++k) {
+      const FwdMember &m = mem[idx[k]];
+      a.off[k] = R;
+      a.r[k] = m.r;
+      a.s[k] = m.s;
+      a.T[k] = reinterpret_cast<__nv_bfloat16 *>(T[k]);
+      R += m.r;
+    }
+    // L1_cat [K x R]: member k's L1 [K x r_k] in columns off_k .. off_k + r_k.
+    for (int k = 0; k < n; ++k) {
+      const FwdMember &m = mem[idx[k]];
+      if (cudaMemcpy2DAsync(l1_cat + a.off[k], (size_t)R * 2, m.L1, (size_t)m.r * 2, (size_t)m.r * 2, (size_t)K,
+                            cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+        return QLORA_ERR_CUDA;
+    }
+    a.off[n] = R;
+    a.R = R;
+    a.M = M;
+    a.count = n;
+    float *t_cat = reinterpret_cast<float *>(w8 + L.t_cat);
+    a.t_cat = t_cat;
+    GemmSeg sT = {{mem[idx[0]].X, M, K, K, 0}, {l1_cat, R, K, R, 1}};
+    rc = tc_gemm(st, dev, M, R, 1, &sT, 1.f, t_cat, R, 1, 1, split_ws, QLORA_KERNEL_GEMM_T);
+    if (rc) return rc;
+    {
+      const int64_t cnt = M * R;
+      const int grid = (int)std::max<int64_t>(1, std::min<int64_t>((cnt + 255) / 256, (int64_t)dev->sms * 8));
+      ProfScope prof(QLORA_KERNEL_T_SCATTER, st);
+      rc = launch_pdl(t_scatter_kernel, dim3(grid), dim3(256), 0, st, a);
+      if (rc) return rc;
+    }
+    for (int k = 0; k < n; ++k) {
+      const FwdMember &m = mem[idx[k]];
+      rc = fwd_y(m.X, M, m.W, m.L2, m.r, T[k], m.Y, w_hat, dev, st);
+      if (rc) return rc;
+    }
+  }
+  return QLORA_OK;
+}
+
 // ------------------------------------------------------------- grouped forward
 static_assert(kMaxGroup == QLORA_MAX_GROUP, "group size of the C ABI");
 // Members are validated as by qlora_linear_fwd; the few-token path runs one
@@ -1151,10 +1303,7 @@ size_t qlora_linear_fwd_group_workspace_size(const qlora_fwd_member_t *members, 
   if (M <= kFtMaxM) return gemv_layout(M, mem, count).total;
   DeviceInfo *dev;
   const int sms = current_device_info(&dev) == QLORA_OK ? dev->sms : 148;
-  size_t need = 0;
-  for (int i = 0; i < count; ++i)
-    need = std::max(need, fwd_layout(M, mem[i].W->n_out, mem[i].W->k_in, mem[i].r, sms).total);
-  return need;
+  return group_large_layout(M, mem, count, sms).total;
 }
 
 int qlora_linear_fwd_group(const qlora_fwd_member_t *members, int count, int64_t M, void *ws, size_t ws_bytes,
@@ -1191,21 +1340,12 @@ int qlora_linear_fwd_group(const qlora_fwd_member_t *members, int count, int64_t
     }
     return QLORA_OK;
   }
-  // Many tokens: each linear is a full tensor-core pass of its own; they run
-  // in order on the shared workspace.
-  size_t need = 0;
-  for (int i = 0; i < count; ++i)
-    need = std::max(need, fwd_layout(M, mem[i].W->n_out, mem[i].W->k_in, mem[i].r, dev->sms).total);
-  if (!ws || ws_bytes < need) return QLORA_ERR_WORKSPACE;
+  // Many tokens: members that share X share one adapter down-projection; then
+  // each runs its own doubleDequant and tensor-core product, in order.
+  const GroupLargeLayout L = group_large_layout(M, mem, count, dev->sms);
+  if (!ws || ws_bytes < L.total) return QLORA_ERR_WORKSPACE;
   if (!aligned(ws, 256)) return QLORA_ERR_MISALIGNED;
-  for (int i = 0; i < count; ++i) {
-    const FwdMember &m = mem[i];
-    const FwdLayout L = fwd_layout(M, m.W->n_out, m.W->k_in, m.r, dev->sms);
-    rc = fwd_large(m.X, m.X, m.s, M, m.W, m.L1, m.L2, m.r, m.Y, m.T_save, reinterpret_cast<uint8_t *>(ws), L, dev,
-                   st);
-    if (rc) return rc;
-  }
-  return QLORA_OK;
+  return group_large_fwd(M, mem, count, reinterpret_cast<uint8_t *>(ws), L, dev, st);
 }
 
 int qlora_linear_bwd(const uint16_t *dY, const uint16_t *X, const uint16_t *T_saved, int64_t M,

@@ -220,7 +220,10 @@ QLORA_API int qlora_linear_bwd(const uint16_t *dY, const uint16_t *X, const uint
  *   concatenated work of all members, instead of one chain per linear: the
  *   per-linear launch gaps and tails of the few-token path disappear.
  *   Members of different code tables (W->table) run as one chain per table.
- *   With M > 128 every member runs its own tensor-core pass, in order.
+ *   With M > 128, members that read the same X (same pointer and K) share one
+ *   adapter down-projection, X [L1_a | L1_b | ...] (their L1 copied side by
+ *   side), split into each member's T; then every member runs its own
+ *   doubleDequant and tensor-core product, in order.
  *   count = 0 or M = 0: nothing is done.  Workspace:
  *   qlora_linear_fwd_group_workspace_size(), which returns 0 for invalid
  *   arguments.
@@ -312,6 +315,7 @@ QLORA_API int qlora_get_last_device_error(void *stream);
 #define QLORA_KERNEL_GEMV_FWD 30    /* fused decode + mma.sync product, up to 32 tokens */
 #define QLORA_KERNEL_FUSED_FWD 31   /* fused decode + tcgen05 product, up to 128 tokens */
 #define QLORA_KERNEL_DROPOUT_MASK 40 /* Xm = X * m (LoRA dropout) */
+#define QLORA_KERNEL_T_SCATTER 41   /* shared-input T split into each linear's hi/lo pair (grouped forward) */
 QLORA_API int qlora_profile_start(int capacity);
 QLORA_API int qlora_profile_stop(void);
 QLORA_API int qlora_profile_read(int i, int *kind, float *ms);

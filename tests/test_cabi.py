@@ -124,5 +124,9 @@ def test_group_workspace_sizes(lib):
             assert total >= sum(M * (n + r) * 4 for n, _, r in shapes)
             assert total <= sum(singles)
         else:
-            # many tokens: members run in turn on one shared workspace
-            assert total == max(singles)
+            # many tokens: one bf16 weight buffer reused member after member, every
+            # member's T pair, and the fp32 T of the largest set sharing an input
+            # (here members 0, 1 share X and K = 192, members 2, 3 share K = 320)
+            assert total >= max(singles)
+            assert total >= max(n * k * 2 for n, k, _ in shapes) + sum(M * 2 * r * 2 for _, _, r in shapes) \
+                + M * max(16 + 16, 8 + 8) * 4

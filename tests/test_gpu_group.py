@@ -199,3 +199,56 @@ def test_llama65b_layer_group_16_tokens_sampled():
         Y_ref, T_ref = qlora_linear.forward(Xf, w_rows, L1f, L2f[:, rows], s)
         assert_close(bf16_to_np(Y)[:, rows], Y_ref, f"{name} Y[:, sampled features]")
         assert_close(qlora.t_value(T).cpu().numpy(), T_ref, f"{name} T")
+
+
+@pytest.mark.parametrize("M", [129, 300])
+def test_shared_input_sets_many_tokens(M):
+    """Many tokens: members reading the same X share one adapter product, split
+    into each member's T with its own rank and scale; an unshared member and a
+    member without a saved T ride along."""
+    g = inputs.rng(7800 + M)
+    K1, K2 = 320, 192
+    Xa, Xb = inputs.normal_bf16(g, (M, K1)), inputs.normal_bf16(g, (M, K2))
+    spec = [("a0", Xa, 72, 8, 2.0), ("b0", Xb, 264, 16, 1.0), ("a1", Xa, 520, 64, 0.25),
+            ("a2", Xa, 136, 136, 0.5), ("b1", Xb, 64, 32, 1.5)]
+    xd = {id(Xa): Xa.cuda(), id(Xb): Xb.cuda()}
+    host, dev = [], []
+    for name, X, N, r, s in spec:
+        K = X.shape[1]
+        W = torch.from_numpy(inputs.weight_f32(g, N, K))
+        L1, L2 = inputs.lora_factors(g, K, N, r)
+        host.append((name, W, X, L1, L2, "nf4"))
+        m = {"X": xd[id(X)], "q": qlora.quantize_nf4_dq(W.cuda()), "L1": L1.cuda(), "L2": L2.cuda(), "s": s}
+        dev.append(m)
+    outs = qlora.linear_fwd_group(dev)
+    torch.cuda.synchronize()
+    assert qlora.last_device_error() == 0
+    _check(host, outs, s_of=lambda i: spec[i][4])
+    # without saved T (the pairs live in the workspace); Y unchanged up to rounding order
+    outs2 = qlora.linear_fwd_group(dev, save_T=False)
+    torch.cuda.synchronize()
+    _check(host, outs2, s_of=lambda i: spec[i][4])
+
+
+def test_layer_group_mid_size_full_check():
+    """A LLaMA-proportioned layer (hidden 1024, MLP 2816, r 64) at 1024 tokens,
+    grouped as a layer's data flow groups it, checked in full."""
+    M, hid, mlp, r, s = 1024, 1024, 2816, 64, 0.25
+    g = inputs.rng(7900)
+    xs = {"H": inputs.normal_bf16(g, (M, hid)), "A": inputs.normal_bf16(g, (M, hid)),
+          "U": inputs.normal_bf16(g, (M, mlp))}
+    shapes = [("q", hid, hid, "H"), ("k", hid, hid, "H"), ("v", hid, hid, "H"), ("o", hid, hid, "A"),
+              ("gate", mlp, hid, "H"), ("up", mlp, hid, "H"), ("down", hid, mlp, "U")]
+    xd = {k: v.cuda() for k, v in xs.items()}
+    host, dev = {}, {}
+    for name, N, K, src in shapes:
+        W = torch.from_numpy(inputs.weight_f32(g, N, K))
+        L1, L2 = inputs.lora_factors(g, K, N, r)
+        host[name] = (name, W, xs[src], L1, L2, "nf4")
+        dev[name] = {"X": xd[src], "q": qlora.quantize_nf4_dq(W.cuda()), "L1": L1.cuda(), "L2": L2.cuda(), "s": s}
+    groups = [["q", "k", "v", "gate", "up"], ["o"], ["down"]]
+    for grp in groups:
+        outs = qlora.linear_fwd_group([dev[n] for n in grp])
+        torch.cuda.synchronize()
+        assert qlora.last_device_error() == 0
+        _check([host[n] for n in grp], outs, s_of=lambda i: s)
