@@ -130,3 +130,24 @@ def test_group_workspace_sizes(lib):
             assert total >= max(singles)
             assert total >= max(n * k * 2 for n, k, _ in shapes) + sum(M * 2 * r * 2 for _, _, r in shapes) \
                 + M * max(16 + 16, 8 + 8) * 4
+
+
+def test_group_shared_input_workspace(lib):
+    """Many tokens: members that read the same X (same pointer and K) share one
+    adapter product, whose fp32 T_cat [M x sum r] and L1_cat [K x sum r] the
+    workspace then holds; members with distinct inputs need no such space."""
+    from bit_nf4_quantized_02_b200 import _lib
+    fake = 1 << 20
+    M, N, K, r = 4096, 512, 1024, 64
+    view = _lib.NF4DQ(N, K, fake, fake, fake, fake)
+
+    def size(xs):
+        arr = (_lib.FwdMember * len(xs))(*[_lib.FwdMember(x, ctypes.pointer(view), fake, fake, r, 1.0, fake, None)
+                                           for x in xs])
+        return lib.qlora_linear_fwd_group_workspace_size(arr, len(xs), M)
+
+    distinct = size([fake, fake * 2, fake * 3])
+    shared = size([fake, fake, fake])
+    assert shared - distinct >= M * 3 * r * 4 + K * 3 * r * 2 - 3 * 256
+    # one shared pair and one single member: the pair's T_cat and L1_cat only
+    assert size([fake, fake * 2, fake]) - distinct >= M * 2 * r * 4 + K * 2 * r * 2 - 3 * 256
