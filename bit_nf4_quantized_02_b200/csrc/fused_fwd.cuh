@@ -83,6 +83,7 @@ struct FtCfg {
 struct FtMember {
   int N, K;
   int kstages;           // ceil(K / 256)
+  DivU31 ks_div;         // division by kstages
   const uint8_t *c2_fp8;
   const float *c1;
   const float *mu;
@@ -116,7 +117,7 @@ __device__ __forceinline__ const FtMember &ft_item(const FtArgs<GM> &p, int it, 
   l = group_member<GM>(p.beg, p.count, it);
   const FtMember &m = p.m[l];
   const int li = it - p.beg[l];
-  rt = li / m.kstages;
+  rt = (int)m.ks_div.div((uint32_t)li);
   ks = li - rt * m.kstages;
   return m;
 }

@@ -79,9 +79,30 @@ __device__ __forceinline__ int group_member(const int (&beg)[GM], int count, int
   return l;
 }
 
+// Division of n (0 <= n < 2^31) by a divisor d >= 1 fixed at launch, as a
+// multiply-high and a shift (Granlund and Montgomery, "Division by invariant
+// integers using multiplication", 1994): with l = ceil(log2 d) and
+// mul = ceil(2^(31 + l) / d) (< 2^32 for d >= 2), n / d = umulhi(n, mul) >>
+// (l - 1); mul = 0 stands for d = 1.
+struct DivU31 {
+  uint32_t mul, shr;
+  __device__ __forceinline__ uint32_t div(uint32_t n) const { return mul ? (__umulhi(n, mul) >> shr) : n; }
+};
+
+inline DivU31 make_div_u31(uint32_t d) {
+  DivU31 r = {0u, 0u};
+  if (d <= 1) return r;
+  uint32_t l = 0;
+  while ((1ull << l) < d) ++l;
+  r.mul = (uint32_t)(((1ull << (31 + l)) + d - 1) / d);
+  r.shr = l - 1;
+  return r;
+}
+
 struct GvMember {
   int N, K;
   int nks;               // units per 64-row block
+  DivU31 nks_div;        // division by nks
   const uint8_t *c2_fp8;
   const float *c1;
   const float *mu;
@@ -187,7 +208,7 @@ struct ConstPrefetch {
     const int l = group_member<GM>(p.beg, p.count, u);
     const GvMember &m = p.m[l];
     const int lu = u - p.beg[l];
-    const int rb = lu / m.nks, ks = lu - rb * m.nks;
+    const int rb = (int)m.nks_div.div((uint32_t)lu), ks = lu - rb * m.nks;
     const int kblocks = m.K >> 6;
     const int kb = ((ks * kGvUnitK + st * kGvStageK) >> 6) + j;
     if (kb >= kblocks) return;
@@ -243,7 +264,7 @@ struct GvConsumer {
     const int l = group_member<GM>(P.beg, P.count, u);
     const GvMember &m = P.m[l];
     const int lu = u - P.beg[l];
-    const int rb = lu / m.nks, ks = lu - rb * m.nks;
+    const int rb = (int)m.nks_div.div((uint32_t)lu), ks = lu - rb * m.nks;
     const int kbeg = ks * kGvUnitK;
     const int nst = min(kGvUnitK, m.K - kbeg) > kGvStageK ? 2 : 1;
     const int n0 = rb * kGvRows + r0, n1 = n0 + 8;
@@ -369,7 +390,7 @@ __global__ void __launch_bounds__(kGvThreads, GvCfg<NT>::kCtasPerSm)
       const int l = group_member<GM>(p.beg, p.count, u);
       const GvMember &m = p.m[l];
       const int lu = u - p.beg[l];
-      const int rb = lu / m.nks, ks = lu - rb * m.nks;
+      const int rb = (int)m.nks_div.div((uint32_t)lu), ks = lu - rb * m.nks;
       const int kbeg = ks * kGvUnitK;
       const int nst = min(kGvUnitK, m.K - kbeg) > kGvStageK ? 2 : 1;
       const int kblocks = m.K >> 6;

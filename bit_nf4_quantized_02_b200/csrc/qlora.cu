@@ -591,6 +591,7 @@ int launch_fused_fwd(const FwdMember *mem, int count, int64_t M, const GemvLayou
     m.N = (int)N;
     m.K = (int)K;
     m.kstages = (int)((K + kFtStageK - 1) / kFtStageK);
+    m.ks_div = make_div_u31((uint32_t)m.kstages);
     m.c2_fp8 = W->c2_fp8;
     m.c1 = W->c1;
     m.mu = W->c2_mean;
@@ -653,6 +654,7 @@ int launch_gemv(const FwdMember *mem, int count, int64_t M, const GemvLayout &L,
     m.N = (int)N;
     m.K = (int)K;
     m.nks = (int)((K + kGvUnitK - 1) / kGvUnitK);
+    m.nks_div = make_div_u31((uint32_t)m.nks);
     m.c2_fp8 = W->c2_fp8;
     m.c1 = W->c1;
     m.mu = W->c2_mean;
