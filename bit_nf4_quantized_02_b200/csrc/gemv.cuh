@@ -5,7 +5,8 @@
 //
 //   Y[M x N] = bf16( X W_hat^T + (s X L1) L2 ),   M <= 8*NT (NT in {1, 2, 4})
 //
-// Three launches per linear, chained with programmatic dependent launch:
+// Three launches per call (one linear or a group of them, below), chained
+// with programmatic dependent launch:
 //   lora_down_small_kernel   adds K-slices of X L1 into an fp32 accumulator;
 //   gemv_fwd_kernel          streams the weight and adds X W_hat^T into an fp32
 //                            [M x N] accumulator (does not need T, so it
@@ -40,7 +41,8 @@
 // layer, whose launch gaps and per-linear tails it removes).  Their units
 // (T slices, weight units, output column slices) are concatenated into one
 // flat list per kernel; a unit finds its linear from the list's start
-// offsets.  A single linear is a group of one (GM = 1).
+// offsets, then its place in that linear with a multiply-high by a divisor
+// fixed at launch (DivU31).  A single linear is a group of one (GM = 1).
 #pragma once
 
 #include "common.cuh"
