@@ -207,9 +207,10 @@ QLORA_API int qlora_linear_bwd(const uint16_t *dY, const uint16_t *X, const uint
 
 /*
  * Grouped forward: the forward of up to QLORA_MAX_GROUP linears that see the
- * same M tokens, each exactly as qlora_linear_fwd computes it (§2 Eq. 3 / §3
- * Eq. 5), e.g. the q, k, v, gate and up projections of a decoder layer, which
- * all read the layer's normalised input.
+ * same M tokens, each computing what qlora_linear_fwd computes (§2 Eq. 3 / §3
+ * Eq. 5) up to the order of its fp32 additions, e.g. the q, k, v, gate and up
+ * projections of a decoder layer, which all read the layer's normalised
+ * input.
  *   members[count]: a HOST array; member i names its own X [M x K_i], weight
  *   W_i (host pointer to the view), L1 [K_i x r_i], L2 [r_i x N_i], scale s_i,
  *   output Y [M x N_i] and optional T_save [M x 2 r_i] (layouts, shape and
