@@ -225,7 +225,8 @@ QLORA_API int qlora_linear_bwd(const uint16_t *dY, const uint16_t *X, const uint
  *   adapter down-projection, X [L1_a | L1_b | ...] (their L1 copied side by
  *   side), split into each member's T; then every member runs its own
  *   doubleDequant and tensor-core product, in order.
- *   count = 0 or M = 0: nothing is done.  Workspace:
+ *   LoRA dropout is not part of the grouped forward (qlora_linear_fwd_dropout
+ *   runs it per linear).  count = 0 or M = 0: nothing is done.  Workspace:
  *   qlora_linear_fwd_group_workspace_size(), which returns 0 for invalid
  *   arguments.
  * Errors: those of qlora_linear_fwd for any member, and QLORA_ERR_INVALID_ARG
