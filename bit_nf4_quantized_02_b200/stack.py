@@ -2,13 +2,14 @@
 
 Every linear is an NF4 + Double-Quantization weight with a LoRA adapter
 (QLoRA, §3 Eq. 5), run forward and then backward in sequence through the
-library (quantize_nf4_dq, linear_fwd, linear_bwd).
+library (quantize_nf4_dq, FwdGroup, linear_fwd, linear_bwd).
 
 The pages give no model code, so the layer wiring is the plainest stack of the
 seven LLaMA linears that carries activations from layer to layer:
 
-* forward: q, k, v, o, gate and up all read the layer input H; down reads
-  U = up(H); the layer output is D = down(U).  The next layer's input is
+* forward: q, k, v, o, gate and up all read the layer input H (one grouped
+  call, which shares their adapter down-projection); down reads U = up(H);
+  the layer output is D = down(U).  The next layer's input is
   H' = bf16(D + R), with R a fixed N(0, 1) bf16 residual per layer;
 * backward, top to bottom: dD = dH'; dU = dX of down.  q, k, v, o and gate
   get fixed N(0, 1) bf16 output gradients.  dH = bf16 of the fp32 sum of the
@@ -16,8 +17,8 @@ seven LLaMA linears that carries activations from layer to layer:
 
 The residual add and the gradient sum are elementwise glue outside the QLoRA
 linear, done here with torch; every linear's work runs in the library.  The
-``ops`` argument takes any object with the three library functions, so that
-the wiring can be exercised on the host with a stand-in.
+``ops`` argument takes any object with those library functions, so that the
+wiring can be exercised on the host with a stand-in.
 """
 
 from __future__ import annotations
@@ -88,7 +89,10 @@ class QLoRAStack:
         self.dU = [torch.empty(M, mlp, dtype=bf, device=device) for _ in range(layers)]
         self.dH = [torch.empty(M, hidden, dtype=bf, device=device) for _ in range(layers)] + \
                   [make((M, hidden), 1.0, seed + 998_000, bf)]     # dH[layers]: gradient at the top
-        self._y = torch.empty(M, max(hidden, mlp), dtype=bf, device=device)    # discarded outputs
+        # discarded outputs (q, k, v, o, gate): one buffer each, since a grouped
+        # forward's members may not share an output
+        self._y = {name: torch.empty(M, shapes[name][0], dtype=bf, device=device) for name in SEEDED_DY}
+        self._groups, self._group_key = None, None
         self._dx = torch.empty(M, hidden, dtype=bf, device=device)
         self._acc = torch.empty(M, hidden, dtype=torch.float32, device=device)
         # adapter gradients: views of one flat buffer (one all-reduce per step)
@@ -105,15 +109,25 @@ class QLoRAStack:
         for x in self.linears():
             x.q = self.ops.quantize_nf4_dq(x.W, out=x.q)
 
+    def _fwd_groups(self):
+        """One grouped forward per layer over the six linears that read H (built
+        once per set of quantized weights)."""
+        key = tuple(id(self.lin[l][name].q) for l in range(self.layers) for name in READS_H)
+        if key != self._group_key:
+            self._groups = [
+                self.ops.FwdGroup([{"X": self.H[l], "q": row[name].q, "L1": row[name].L1, "L2": row[name].L2,
+                                    "s": self.s, "Y": self.U[l] if name == "up" else self._y[name],
+                                    "T": row[name].T} for name in READS_H])
+                for l, row in enumerate(self.lin)]
+            self._group_key = key
+        return self._groups
+
     def forward(self):
-        ops, s, M = self.ops, self.s, self.M
+        ops, s = self.ops, self.s
+        groups = self._fwd_groups()
         for l in range(self.layers):
-            H, row = self.H[l], self.lin[l]
-            for name in READS_H:
-                x = row[name]
-                n = x.L2.shape[1]
-                out = self.U[l] if name == "up" else self._y.view(-1)[:M * n].view(M, n)
-                ops.linear_fwd(H, x.q, x.L1, x.L2, s, Y=out, T=x.T)
+            row = self.lin[l]
+            groups[l]()          # q, k, v, o, gate and up on H[l]
             d = row["down"]
             ops.linear_fwd(self.U[l], d.q, d.L1, d.L2, s, Y=self.D[l], T=d.T)
             torch.add(self.D[l].float(), self.R[l].float(), out=self._acc)

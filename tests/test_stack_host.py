@@ -40,6 +40,13 @@ class OracleOps:
         self.calls.append(("fwd", X, Y.clone()))
         return Y, T
 
+    def FwdGroup(self, members):
+        """A grouped forward: each member as linear_fwd computes it, in member order."""
+        def run():
+            return [self.linear_fwd(m["X"], m["q"], m["L1"], m["L2"], m["s"], Y=m["Y"], T=m["T"])
+                    for m in members]
+        return run
+
     def linear_bwd(self, dY, X, T, q, L1, L2, s, grad_dtype=None, dX=None, dL1=None, dL2=None):
         dXr, dL1r, dL2r = qlora_linear.backward(_np(dY), _np(X), q["w_hat"], _np(L1), _np(L2), s)
         dX.copy_(torch.from_numpy(dXr.astype(np.float32)))
