@@ -58,6 +58,39 @@ def _bits(t: torch.Tensor) -> torch.Tensor:
     return t
 
 
+def _check_out(t: torch.Tensor | None, shape, dtype, dev, name: str) -> None:
+    """A caller-supplied output: exactly ``shape`` and ``dtype``, contiguous, on ``dev``.
+
+    The kernels write the full extent the shapes imply, so a smaller buffer
+    (or one of a narrower dtype) would be written past its end.
+    """
+    if t is None:
+        return
+    if tuple(t.shape) != tuple(shape) or t.dtype != dtype or t.device != dev or not t.is_contiguous():
+        raise ValueError(f"qlora: {name} must be a contiguous {dtype} tensor of shape {tuple(shape)} on {dev}, "
+                         f"got {t.dtype} {tuple(t.shape)} on {t.device}")
+
+
+def _check_device(dev, require_cuda: bool = True, **tensors) -> None:
+    """Every tensor on the one device ``dev``, a CUDA device (a kernel given
+    another GPU's memory would reach across devices)."""
+    for name, t in tensors.items():
+        if t is not None and t.device != dev:
+            raise ValueError(f"qlora: {name} is on {t.device}, expected {dev} (all tensors of a call share a device)")
+    if require_cuda and dev.type != "cuda":
+        raise ValueError("qlora: tensors must live on a CUDA device")
+
+
+def _span(t: torch.Tensor | None):
+    if t is None or t.numel() == 0:
+        return None
+    return (t.data_ptr(), t.data_ptr() + t.numel() * t.element_size())
+
+
+def _overlap(a, b) -> bool:
+    return a is not None and b is not None and a[0] < b[1] and b[0] < a[1]
+
+
 @dataclass
 class NF4Tensor:
     """A weight in the QLoRA storage format (device buffers owned by torch).
@@ -132,6 +165,8 @@ def quantize_nf4_dq(W: torch.Tensor, out: NF4Tensor | None = None, table: str = 
 
 def dequant(q: NF4Tensor, out: torch.Tensor | None = None) -> torch.Tensor:
     """doubleDequant (Eq. 6): the bf16 weight [n_out, k_in]."""
+    _check_out(out, q.shape, torch.bfloat16, q.device, "out")
+    _check_device(q.device, c2_fp8=q.c2_fp8, c1=q.c1, c2_mean=q.c2_mean)
     lib = _lib.load()
     if out is None:
         out = torch.empty(q.shape, dtype=torch.bfloat16, device=q.device)
@@ -183,13 +218,18 @@ def linear_fwd(X: torch.Tensor, q: NF4Tensor, L1: torch.Tensor, L2: torch.Tensor
     T = s (X * m / (1 - dropout_p)) L1; ``Xm`` ([M, K] bf16, optional)
     receives the masked input X * m for the backward.
     """
-    lib = _lib.load()
     M, K = X.shape
     r = L1.shape[1]
     N = q.n_out
     if K != q.k_in or L1.shape[0] != K or tuple(L2.shape) != (r, N):
         raise ValueError("qlora: shape mismatch")
     dev = X.device
+    _check_out(Y, (M, N), torch.bfloat16, dev, "Y")
+    if save_T:
+        _check_out(T, (M, 2 * r), torch.bfloat16, dev, "T")
+    _check_out(Xm, (M, K), torch.bfloat16, dev, "Xm")
+    _check_device(dev, L1=L1, L2=L2, codes=q.codes, c2_fp8=q.c2_fp8, c1=q.c1, c2_mean=q.c2_mean, mask=dropout_mask)
+    lib = _lib.load()
     if Y is None:
         Y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
     if save_T and T is None:
@@ -217,20 +257,39 @@ class FwdGroup:
     tensors, which it keeps alive; only the C call is made per run."""
 
     def __init__(self, members, save_T: bool = True):
-        lib = _lib.load()
         if not 0 < len(members) <= _lib.QLORA_MAX_GROUP:
             raise ValueError(f"qlora: a group holds 1..{_lib.QLORA_MAX_GROUP} linears")
         M = members[0]["X"].shape[0]
         dev = members[0]["X"].device
-        arr = (_lib.FwdMember * len(members))()
-        self._keep, self.outputs = [], []
-        for i, m in enumerate(members):
+        # every argument is checked before the library is loaded or a pointer taken
+        for m in members:
             X, q, L1, L2 = m["X"], m["q"], m["L1"], m["L2"]
             K, r, N = X.shape[1], L1.shape[1], q.n_out
             if X.shape[0] != M or X.device != dev:
                 raise ValueError("qlora: the members of a group share the token count and the device")
             if K != q.k_in or L1.shape[0] != K or tuple(L2.shape) != (r, N):
                 raise ValueError("qlora: shape mismatch")
+            _check_out(m.get("Y"), (M, N), torch.bfloat16, dev, "Y")
+            if save_T:
+                _check_out(m.get("T"), (M, 2 * r), torch.bfloat16, dev, "T")
+            _check_device(dev, False, L1=L1, L2=L2, codes=q.codes, c2_fp8=q.c2_fp8, c1=q.c1, c2_mean=q.c2_mean)
+        # caller-supplied outputs may not overlap any member's input X or output
+        outs = [(i, name, _span(m.get(name))) for i, m in enumerate(members)
+                for name in (("Y", "T") if save_T else ("Y",))]
+        for i, name, sp in outs:
+            for j, m in enumerate(members):
+                if _overlap(sp, _span(m["X"])):
+                    raise ValueError(f"qlora: member {i}'s {name} overlaps member {j}'s X")
+            for j, name2, sp2 in outs:
+                if (i, name) < (j, name2) and _overlap(sp, sp2):
+                    raise ValueError(f"qlora: member {i}'s {name} overlaps member {j}'s {name2}")
+        _check_device(dev)
+        lib = _lib.load()
+        arr = (_lib.FwdMember * len(members))()
+        self._keep, self.outputs = [], []
+        for i, m in enumerate(members):
+            X, q, L1, L2 = m["X"], m["q"], m["L1"], m["L2"]
+            r, N = L1.shape[1], q.n_out
             Y = m.get("Y")
             if Y is None:
                 Y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
@@ -283,11 +342,10 @@ def linear_bwd(dY: torch.Tensor, X: torch.Tensor, T: torch.Tensor | None, q: NF4
     the mask: dX = dY W_hat + (G L1^T) m / (1 - p), dL1 = drop(X)^T G.
     ``Xm`` is the forward's masked input (recomputed from X and the mask if None).
     """
-    lib = _lib.load()
     M, N = dY.shape
     K = q.k_in
     r = L1.shape[1]
-    if N != q.n_out or tuple(X.shape) != (M, K) or tuple(L2.shape) != (r, N):
+    if N != q.n_out or tuple(X.shape) != (M, K) or tuple(L2.shape) != (r, N) or L1.shape[0] != K:
         raise ValueError("qlora: shape mismatch")
     if grad_dtype == torch.bfloat16:
         gdt = _lib.QLORA_DTYPE_BF16
@@ -296,6 +354,15 @@ def linear_bwd(dY: torch.Tensor, X: torch.Tensor, T: torch.Tensor | None, q: NF4
     else:
         raise TypeError("qlora: grad_dtype must be bfloat16 or float32")
     dev = dY.device
+    if T is not None and (tuple(T.shape) != (M, 2 * r) or T.dtype != torch.bfloat16):
+        raise ValueError(f"qlora: T must be the forward's bf16 [M, 2r] = {(M, 2 * r)} hi/lo pair")
+    if need_dX:
+        _check_out(dX, (M, K), torch.bfloat16, dev, "dX")
+    _check_out(dL1, (K, r), grad_dtype, dev, "dL1")
+    _check_out(dL2, (r, N), grad_dtype, dev, "dL2")
+    _check_device(dev, X=X, T=T, L1=L1, L2=L2, codes=q.codes, c2_fp8=q.c2_fp8, c1=q.c1, c2_mean=q.c2_mean,
+                  mask=dropout_mask, Xm=Xm)
+    lib = _lib.load()
     if need_dX and dX is None:
         dX = torch.empty((M, K), dtype=torch.bfloat16, device=dev)
     if dL1 is None:

@@ -21,6 +21,8 @@ QLORA_ERR_DEVICE_TIMEOUT = -5
 QLORA_ERR_WORKSPACE = -6
 QLORA_ERR_SCRATCH_LIMIT = -7
 QLORA_NOALLOC_MAX_NUMEL = 1 << 28
+QLORA_DEFAULT_WAIT_LIMIT_NS = 4_000_000_000
+QLORA_MAX_WAIT_LIMIT_NS = 60_000_000_000
 
 QLORA_DTYPE_F32 = 0
 QLORA_DTYPE_BF16 = 1
@@ -75,6 +77,8 @@ SIGNATURES = {
     "qlora_profile_read": (c_int, [c_int, POINTER(c_int), POINTER(c_float)]),
     "qlora_status_str": (ctypes.c_char_p, [c_int]),
     "qlora_get_last_device_error": (c_int, [c_void_p]),
+    "qlora_set_wait_limit_ns": (c_int, [ctypes.c_uint64, c_void_p]),
+    "qlora_diag_expired_wait": (c_int, [c_void_p]),
     "qlora_quantize_workspace_size": (c_size_t, [c_int64]),
     "qlora_quantize_nf4_dq": (c_int, [c_void_p, c_int, c_int64, c_int64, c_void_p, c_void_p, c_void_p, c_void_p,
                                       c_void_p, c_size_t, c_void_p]),

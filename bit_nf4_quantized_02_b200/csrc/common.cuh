@@ -27,12 +27,16 @@ enum DeviceError : int {
   DEV_TIMEOUT_MMA = 2,        // MMA issuer waited too long for data or TMEM
   DEV_TIMEOUT_EPILOGUE = 3,   // epilogue waited too long for an accumulator
   DEV_TIMEOUT_DRAIN = 4,      // in-flight copies/MMAs did not finish during shutdown
+  DEV_TIMEOUT_DIAG = 5,       // the diagnostic wait of qlora_diag_expired_wait
 };
 
-// Bound on any single wait: far above the longest legitimate wait of a
-// pipeline stage (microseconds), short enough that a broken pipeline returns
-// control to the host within seconds.
-constexpr uint64_t kWaitLimitNs = 4000000000ull;
+// Bound on any single wait, per device: by default far above the longest
+// legitimate wait of a pipeline stage (microseconds), short enough that a
+// broken pipeline returns control to the host within seconds.  The host may
+// change it (qlora_set_wait_limit_ns); a wait reads it when it first fails
+// to complete at once.
+constexpr uint64_t kDefaultWaitLimitNs = 4000000000ull;
+__device__ unsigned long long g_wait_limit_ns = kDefaultWaitLimitNs;
 
 __device__ __forceinline__ uint64_t globaltimer_ns() {
   uint64_t t;
@@ -94,15 +98,16 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t par
 }
 
 // Wait for the phase with the given parity to complete.  Returns false (and
-// records `code`) if it does not complete within kWaitLimitNs.
+// records `code`) if it does not complete within the device's wait limit.
 template <bool kClusterScope = false>
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int *err, int code) {
   auto poll = [&]() { return kClusterScope ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity); };
   if (poll()) return true;
   const uint64_t t0 = globaltimer_ns();
+  const uint64_t limit = *reinterpret_cast<volatile unsigned long long *>(&g_wait_limit_ns);
   for (uint32_t i = 1;; ++i) {
     if (poll()) return true;
-    if ((i & 255u) == 0 && globaltimer_ns() - t0 > kWaitLimitNs) {
+    if ((i & 255u) == 0 && globaltimer_ns() - t0 > limit) {
       record_error(err, code);
       return false;
     }

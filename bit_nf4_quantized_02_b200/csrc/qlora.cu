@@ -4,6 +4,7 @@
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cstring>
 #include <mutex>
 
@@ -20,19 +21,36 @@ namespace qlora {
 
 __device__ int g_dev_err;
 
+// Sets the device's wait limit (stream-ordered, one thread).
+__global__ void set_wait_limit_kernel(unsigned long long ns) { g_wait_limit_ns = ns; }
+
+// Diagnostics: one thread waits, through the same bounded wait as every
+// pipeline, for the first phase of an mbarrier that nothing arrives on.  The
+// wait runs out after the device's wait limit, records DEV_TIMEOUT_DIAG and
+// returns.  No copy or MMA is issued, so nothing is in flight at exit.
+__global__ void diag_expired_wait_kernel(int *err) {
+  __shared__ __align__(8) uint64_t bar;
+  mbar_init(smem_u32(&bar), 1);
+  fence_mbar_init();
+  mbar_wait(smem_u32(&bar), 0, err, DEV_TIMEOUT_DIAG);
+}
+
 namespace {
 
 constexpr int kMaxDevices = 64;
 
+// Per-device state.  `sms` and `err` are written once, under g_mu, before
+// `init` is published with release order; readers check `init` with acquire
+// order first.  The per-kernel set-up slots (a shared-memory limit set, an
+// occupancy figure) are filled lazily by once(): 0 means not done yet.
 struct DeviceInfo {
-  bool init = false;
+  std::atomic<bool> init{false};
   int sms = 0;
-  int *err = nullptr;        // device address of g_dev_err
-  bool gemm_attr[16] = {};   // [wide][fold][BN 64/128/256 or 3 = pair]: shared-memory limit set
-  int pair_clusters[3] = {0, 0, 0};   // co-resident 2-CTA clusters of the pair GEMM [form]
-  int gemv_smem_set[6] = {};    // dynamic smem limit set per [group form][NT variant]
-  int gemv_per_sm[6] = {};      // resident CTAs per SM per [group form][NT variant]
-  int fused_smem_set[8] = {};   // dynamic smem limit set per [group form][token-padding variant]
+  int *err = nullptr;                    // device address of g_dev_err
+  std::atomic<int> gemm_attr[16];        // [wide][fold][BN 64/128/256 or 3 = pair]: 1 once the smem limit is set
+  std::atomic<int> pair_clusters[3];     // co-resident 2-CTA clusters of the pair GEMM [form]
+  std::atomic<int> gemv_per_sm[6];       // mma.sync few-token product: resident CTAs per SM [group form][NT]
+  std::atomic<int> fused_smem_set[8];    // tcgen05 few-token product: smem limit set [group form][token padding]
 };
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_mu;
@@ -41,20 +59,31 @@ int current_device_info(DeviceInfo **out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return QLORA_ERR_CUDA;
   DeviceInfo &d = g_dev[dev];
-  if (!d.init) {
+  if (!d.init.load(std::memory_order_acquire)) {
     std::lock_guard<std::mutex> lock(g_mu);
-    if (!d.init) {
+    if (!d.init.load(std::memory_order_relaxed)) {
       if (cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return QLORA_ERR_CUDA;
       if (cudaGetSymbolAddress(reinterpret_cast<void **>(&d.err), g_dev_err) != cudaSuccess) return QLORA_ERR_CUDA;
-      // One-time fill of the quantizer's code table (a constant of the NF4
-      // levels), completed before any library launch on this device.
-      code_lut_init_kernel<<<dim3((kCodeLutBytes + 255) / 256, kNumTables), 256>>>();
-      if (cudaGetLastError() != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess) return QLORA_ERR_CUDA;
-      d.init = true;
+      d.init.store(true, std::memory_order_release);
     }
   }
   *out = &d;
   return QLORA_OK;
+}
+
+// One-time set-up step of a device: runs f() (a positive result, or <= 0 on
+// failure) under the device mutex the first time, stores its result in
+// `slot` and returns it; later calls return the stored value.
+template <class F>
+int once(std::atomic<int> &slot, F &&f) {
+  int v = slot.load(std::memory_order_acquire);
+  if (v > 0) return v;
+  std::lock_guard<std::mutex> lock(g_mu);
+  v = slot.load(std::memory_order_relaxed);
+  if (v > 0) return v;
+  v = f();
+  if (v > 0) slot.store(v, std::memory_order_release);
+  return v;
 }
 
 // ---------------------------------------------------------------- event log
@@ -250,11 +279,13 @@ int launch_gemm_bn(const CUtensorMap *maps, TcGemmArgs &args, int sms, DeviceInf
   using Cfg = TcCfg<BN, false, WIDE>;
   auto kernel = tc_gemm_kernel<BN, false, FOLD, WIDE>;
   const int idx = (BN == 64 ? 0 : (BN == 128 ? 1 : 2)) + (FOLD ? 4 : 0) + (WIDE ? 8 : 0);
-  if (!dev->gemm_attr[idx]) {
-    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes) != cudaSuccess)
-      return QLORA_ERR_CUDA;
-    dev->gemm_attr[idx] = true;
-  }
+  if (once(dev->gemm_attr[idx], [&] {
+        return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes) ==
+                       cudaSuccess
+                   ? 1
+                   : 0;
+      }) <= 0)
+    return QLORA_ERR_CUDA;
   const int units = args.m_tiles * args.n_tiles * args.splits;
   const int grid = std::max(1, std::min(units, sms));
   ProfScope prof(kind, st);
@@ -284,18 +315,17 @@ int launch_gemm_pair(const CUtensorMap *maps, TcGemmArgs &args, DeviceInfo *dev,
   cfg.attrs = attr;
   cfg.numAttrs = 1;   // the occupancy query takes the cluster shape alone
   const int form = DROPZ ? 2 : (WIDE ? 1 : 0);
-  const int idx = DROPZ ? 15 : 3 + (WIDE ? 8 : 0);
-  if (!dev->gemm_attr[idx]) {
+  const int resident = once(dev->pair_clusters[form], [&] {
     if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes) != cudaSuccess)
-      return QLORA_ERR_CUDA;
+      return 0;
     cfg.gridDim = dim3(2 * (unsigned)dev->sms, 1, 1);
     int clusters = 0;
-    if (cudaOccupancyMaxActiveClusters(&clusters, kernel, &cfg) != cudaSuccess || clusters < 1) return QLORA_ERR_CUDA;
-    dev->pair_clusters[form] = clusters;
-    dev->gemm_attr[idx] = true;
-  }
+    if (cudaOccupancyMaxActiveClusters(&clusters, kernel, &cfg) != cudaSuccess) return 0;
+    return clusters;
+  });
+  if (resident <= 0) return QLORA_ERR_CUDA;
   const int units = args.m_tiles * args.n_tiles * args.splits;
-  const int clusters = std::max(1, std::min(units, dev->pair_clusters[form]));
+  const int clusters = std::max(1, std::min(units, resident));
   cfg.gridDim = dim3(2 * (unsigned)clusters, 1, 1);
   cfg.numAttrs = g_prof.on ? 1 : 2;   // a programmatic dependent of the previous kernel, unless the event log records
   ProfScope prof(kind, st);
@@ -601,12 +631,13 @@ int launch_fused_fwd(const FwdMember *mem, int count, int64_t M, const GemvLayou
   }
   a.items = items;
   const int idx = (GM > 1 ? 4 : 0) + (MP == 16 ? 0 : (MP == 32 ? 1 : (MP == 64 ? 2 : 3)));
-  if (dev->fused_smem_set[idx] < Cfg::kSmemBytes) {
-    if (cudaFuncSetAttribute(nf4_fused_fwd_kernel<MP, GM>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             Cfg::kSmemBytes) != cudaSuccess)
-      return QLORA_ERR_CUDA;
-    dev->fused_smem_set[idx] = Cfg::kSmemBytes;
-  }
+  if (once(dev->fused_smem_set[idx], [&] {
+        return cudaFuncSetAttribute(nf4_fused_fwd_kernel<MP, GM>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    Cfg::kSmemBytes) == cudaSuccess
+                   ? 1
+                   : 0;
+      }) <= 0)
+    return QLORA_ERR_CUDA;
   const int grid = std::max(1, std::min(a.items, dev->sms));
   ProfScope prof(QLORA_KERNEL_FUSED_FWD, st);
   // 1. T accumulation; 2. the fused product, overlapping it; 3. the LoRA epilogue.
@@ -665,17 +696,15 @@ int launch_gemv(const FwdMember *mem, int count, int64_t M, const GemvLayout &L,
   a.units = units;
   const int smem = Cfg::kSmemBytes;
   const int idx = (GM > 1 ? 3 : 0) + (NT == 1 ? 0 : (NT == 2 ? 1 : 2));
-  if (dev->gemv_smem_set[idx] < smem) {
+  const int per_sm = once(dev->gemv_per_sm[idx], [&] {
+    int n = 0;
     if (cudaFuncSetAttribute(gemv_fwd_kernel<NT, GM>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
-        cudaSuccess)
-      return QLORA_ERR_CUDA;
-    dev->gemv_smem_set[idx] = smem;
-  }
-  int &per_sm = dev->gemv_per_sm[idx];
-  if (per_sm < 1 && (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, gemv_fwd_kernel<NT, GM>, kGvThreads,
-                                                                    smem) != cudaSuccess ||
-                     per_sm < 1))
-    return QLORA_ERR_CUDA;
+            cudaSuccess ||
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, gemv_fwd_kernel<NT, GM>, kGvThreads, smem) != cudaSuccess)
+      return 0;
+    return n;
+  });
+  if (per_sm <= 0) return QLORA_ERR_CUDA;
   const int grid = std::max(1, std::min(a.units, per_sm * dev->sms));
   ProfScope prof(QLORA_KERNEL_GEMV_FWD, st);
   // 1. T accumulation; 2. the product, overlapping it; 3. the LoRA epilogue.
@@ -848,10 +877,55 @@ int qlora_get_last_device_error(void *stream) {
   return QLORA_OK;
 }
 
+int qlora_set_wait_limit_ns(uint64_t ns, void *stream) {
+  if (ns > QLORA_MAX_WAIT_LIMIT_NS) return QLORA_ERR_INVALID_ARG;
+  DeviceInfo *dev;
+  int rc = current_device_info(&dev);
+  if (rc) return rc;
+  set_wait_limit_kernel<<<1, 1, 0, reinterpret_cast<cudaStream_t>(stream)>>>(ns == 0 ? kDefaultWaitLimitNs : ns);
+  return launch_status();
+}
+
+int qlora_diag_expired_wait(void *stream) {
+  DeviceInfo *dev;
+  int rc = current_device_info(&dev);
+  if (rc) return rc;
+  diag_expired_wait_kernel<<<1, 1, 0, reinterpret_cast<cudaStream_t>(stream)>>>(dev->err);
+  return launch_status();
+}
+
 size_t qlora_quantize_workspace_size(int64_t numel) {
   if (numel < 0) return 0;
   const int64_t nblk = (numel + 63) / 64;
   return align_up((size_t)nblk * 4) + align_up((size_t)kQuantMaxCtas * 8);
+}
+
+// The quantizer's two launches (K1: absmax, codes and fp64 partial sums of
+// c2; K2: the Double-Quantization constants), with c2 and the partial sums
+// in the given scratch.
+static int quantize_launch(const void *W, int w_dtype, int64_t numel, int table, uint8_t *codes, uint8_t *c2_fp8,
+                           float *c1, float *c2_mean, float *c2, double *partial, DeviceInfo *dev, cudaStream_t st) {
+  const int64_t nblk = (numel + 63) / 64;
+  const int64_t ngroups = numel >> 9;   // 512-element groups, one per warp iteration
+  const int grid1 = (int)std::max<int64_t>(
+      1, std::min<int64_t>((ngroups + 7) / 8, std::min(kQuantMaxCtas, dev->sms * kQuantCtasPerSm)));
+  int rc;
+  {
+    ProfScope prof(QLORA_KERNEL_QUANTIZE, st);
+    if (w_dtype == QLORA_DTYPE_F32)
+      rc = launch_pdl(nf4_quantize_kernel<float>, dim3(grid1), dim3(kQuantThreads), 0, st,
+                      reinterpret_cast<const float *>(W), numel, codes, c2, partial, table);
+    else
+      rc = launch_pdl(nf4_quantize_kernel<__nv_bfloat16>, dim3(grid1), dim3(kQuantThreads), 0, st,
+                      reinterpret_cast<const __nv_bfloat16 *>(W), numel, codes, c2, partial, table);
+  }
+  if (rc) return rc;
+  const int64_t nb256 = (nblk + 255) / 256;
+  const int grid2 =
+      (int)std::max<int64_t>(1, std::min<int64_t>((nb256 + kDqWarps - 1) / kDqWarps, (int64_t)dev->sms * 4));
+  ProfScope prof(QLORA_KERNEL_DQ_CONSTANTS, st);
+  return launch_pdl(dq_constants_kernel, dim3(grid2), dim3(32 * kDqWarps), 0, st, (const float *)c2, nblk,
+                    (const double *)partial, grid1, c2_fp8, c1, c2_mean);
 }
 
 int qlora_quantize_nf4_dq(const void *W, int w_dtype, int64_t n_out, int64_t k_in, uint8_t *codes, uint8_t *c2_fp8,
@@ -881,23 +955,7 @@ int qlora_quantize_4bit_dq(const void *W, int w_dtype, int64_t n_out, int64_t k_
   const int64_t nblk = (numel + 63) / 64;
   float *c2 = reinterpret_cast<float *>(ws);
   double *partial = reinterpret_cast<double *>(reinterpret_cast<uint8_t *>(ws) + align_up((size_t)nblk * 4));
-  const int64_t ngroups = numel >> 9;   // 512-element groups, one per warp iteration
-  const int grid1 = (int)std::max<int64_t>(1, std::min<int64_t>((ngroups + 7) / 8, std::min(kQuantMaxCtas, dev->sms * kQuantCtasPerSm)));
-  {
-  ProfScope prof(QLORA_KERNEL_QUANTIZE, st);
-  if (w_dtype == QLORA_DTYPE_F32)
-    rc = launch_pdl(nf4_quantize_kernel<float>, dim3(grid1), dim3(kQuantThreads), 0, st,
-                    reinterpret_cast<const float *>(W), numel, codes, c2, partial, table);
-  else
-    rc = launch_pdl(nf4_quantize_kernel<__nv_bfloat16>, dim3(grid1), dim3(kQuantThreads), 0, st,
-                    reinterpret_cast<const __nv_bfloat16 *>(W), numel, codes, c2, partial, table);
-  }
-  if (rc) return rc;
-  const int64_t nb256 = (nblk + 255) / 256;
-  const int grid2 = (int)std::max<int64_t>(1, std::min<int64_t>((nb256 + kDqWarps - 1) / kDqWarps, (int64_t)dev->sms * 4));
-  ProfScope prof(QLORA_KERNEL_DQ_CONSTANTS, st);
-  return launch_pdl(dq_constants_kernel, dim3(grid2), dim3(32 * kDqWarps), 0, st, (const float *)c2, nblk,
-                    (const double *)partial, grid1, c2_fp8, c1, c2_mean);
+  return quantize_launch(W, w_dtype, numel, table, codes, c2_fp8, c1, c2_mean, c2, partial, dev, st);
 }
 
 int qlora_quantize_nf4_dq_noalloc(const void *W, int w_dtype, int64_t n_out, int64_t k_in, uint8_t *codes,
@@ -919,22 +977,9 @@ int qlora_quantize_nf4_dq_noalloc(const void *W, int w_dtype, int64_t n_out, int
   if (numel == 0) return cudaMemsetAsync(c2_mean, 0, sizeof(float), st) == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
   if (!W || !codes || !c2_fp8 || !c1) return QLORA_ERR_INVALID_ARG;
   if (!aligned(W, 16) || !aligned(codes, 16) || !aligned(c2_fp8, 16) || !aligned(c1, 16)) return QLORA_ERR_MISALIGNED;
-  const int64_t nblk = (numel + 63) / 64;
   float *c2 = reinterpret_cast<float *>(scratch);
   double *partial = reinterpret_cast<double *>(scratch + kNoallocC2Bytes);
-  const int64_t ngroups = numel >> 9;   // 512-element groups, one per warp iteration
-  const int grid1 = (int)std::max<int64_t>(1, std::min<int64_t>((ngroups + 7) / 8, std::min(kQuantMaxCtas, dev->sms * kQuantCtasPerSm)));
-  if (w_dtype == QLORA_DTYPE_F32)
-    rc = launch_pdl(nf4_quantize_kernel<float>, dim3(grid1), dim3(kQuantThreads), 0, st,
-                    reinterpret_cast<const float *>(W), numel, codes, c2, partial, table);
-  else
-    rc = launch_pdl(nf4_quantize_kernel<__nv_bfloat16>, dim3(grid1), dim3(kQuantThreads), 0, st,
-                    reinterpret_cast<const __nv_bfloat16 *>(W), numel, codes, c2, partial, table);
-  if (rc) return rc;
-  const int64_t nb256 = (nblk + 255) / 256;
-  const int grid2 = (int)std::max<int64_t>(1, std::min<int64_t>((nb256 + kDqWarps - 1) / kDqWarps, (int64_t)dev->sms * 4));
-  return launch_pdl(dq_constants_kernel, dim3(grid2), dim3(32 * kDqWarps), 0, st, (const float *)c2, nblk,
-                    (const double *)partial, grid1, c2_fp8, c1, c2_mean);
+  return quantize_launch(W, w_dtype, numel, table, codes, c2_fp8, c1, c2_mean, c2, partial, dev, st);
 }
 
 int qlora_dequant(const qlora_nf4dq_t *W, uint16_t *W_out, void *stream) {

@@ -104,38 +104,64 @@ struct NF4Thresholds {
 // included) can index outside it.
 constexpr int kCodeBins = 16384;
 constexpr int kCodeLutEntries = kCodeBins + 2;
-constexpr int kCodeLutBytes = (kCodeLutEntries + 15) / 16 * 16;
+
+// Each CTA builds the table in its shared memory from the same thresholds
+// the exact path uses, before it waits for the kernel ahead of it (so the
+// build overlaps that kernel's tail).  Entry i holds, for the bin b =
+// min(max(i - 1, 0), kCodeBins - 1), either kCodeBoundary | j when the
+// boundary bin tb_j = floor((t_j + 1) * kCodeBins / 2) of threshold j lies
+// within two bins of b, or else the code #{j : tb_j < b}.  Entries from
+// kCodeLutBytes on are zero.
+//
+// A warp fills 32 consecutive words (128 entries, lane l word l) per pass.
+// Consecutive thresholds are hundreds of bins apart, so at most one threshold
+// lies within two bins of the 128 entries of a pass: the warp counts the thresholds below its first bin
+// minus two with one ballot, and a lane whose four bins are clear of the
+// next threshold stores that count four times; the few lanes near a
+// threshold resolve their four entries one by one.
+constexpr int kCodeLutBytes = (kCodeLutEntries + 3) / 4 * 4;
 constexpr int kCodeLutSpan = 32768;
 constexpr uint32_t kCodeBoundary = 0x80;
 
-// The table, filled once per device from the same thresholds the exact path
-// uses (code_lut_init_kernel), and copied into shared memory by each CTA.
-__device__ __align__(16) uint8_t g_code_lut[kNumTables][kCodeLutBytes];
-
-__global__ void __launch_bounds__(256) code_lut_init_kernel() {
-  const int i = blockIdx.x * blockDim.x + threadIdx.x;
-  const int table = blockIdx.y;
-  if (i >= kCodeLutBytes) return;
-  const int b = min(max(i - 1, 0), kCodeBins - 1);
-  NF4Thresholds th;
-  th.init(table);
-  uint32_t code = 0;
-  int edge = -1;
-#pragma unroll
-  for (int j = 0; j < 15; ++j) {
-    const int tb = (int)floor(((double)th.t[j] + 1.0) * (kCodeBins / 2));
-    code += tb < b ? 1u : 0u;
-    if (tb >= b - 2 && tb <= b + 2) edge = j;
+__device__ __forceinline__ void build_code_lut(uint8_t *lut, int table, int *tb_s) {
+  if (threadIdx.x < 16) {
+    int tb = 0x7FFFFFFF;   // entry 15: past every bin
+    if (threadIdx.x < 15) {
+      const float t = __double2float_rd(((double)kLevels[table][threadIdx.x] + (double)kLevels[table][threadIdx.x + 1]) * 0.5);
+      tb = (int)floor(((double)t + 1.0) * (kCodeBins / 2));
+    }
+    tb_s[threadIdx.x] = tb;
   }
-  g_code_lut[table][i] = edge >= 0 ? (uint8_t)(kCodeBoundary | edge) : (uint8_t)code;
-}
-
-// Copy the table into shared memory and zero the rest of its span (all
-// threads of the CTA).
-__device__ __forceinline__ void load_code_lut(uint8_t *lut, int table) {
-  for (int i = threadIdx.x; i < kCodeLutSpan / 16; i += blockDim.x)
-    reinterpret_cast<uint4 *>(lut)[i] =
-        i < kCodeLutBytes / 16 ? reinterpret_cast<const uint4 *>(g_code_lut[table])[i] : make_uint4(0, 0, 0, 0);
+  __syncthreads();
+  const int lane = threadIdx.x & 31;
+  const int my_tb = lane < 15 ? tb_s[lane] : 0x7FFFFFFF;
+  uint32_t *lw = reinterpret_cast<uint32_t *>(lut);
+  for (int w0 = (threadIdx.x & ~31); w0 < kCodeLutSpan / 4; w0 += blockDim.x) {
+    const int w = w0 + lane;
+    const int first_bin = max(4 * w0 - 1, 0);
+    // thresholds more than two bins below the warp's first bin
+    const int c = __popc(__ballot_sync(0xFFFFFFFFu, my_tb < first_bin - 2));
+    uint32_t v = 0;
+    if (4 * w < kCodeLutBytes) {
+      const int bhi = min(4 * w + 2, kCodeBins - 1);
+      const int tc = tb_s[c];
+      if (tc > bhi + 2) {
+        v = (uint32_t)c * 0x01010101u;
+      } else {
+        const int tn = tb_s[min(c + 1, 15)];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const int b = min(max(4 * w + k - 1, 0), kCodeBins - 1);
+          const bool past = tc < b - 2;             // threshold c is behind this bin
+          const int j = c + (past ? 1 : 0);         // first threshold >= b - 2
+          const int tj = past ? tn : tc;
+          const uint32_t e = tj <= b + 2 ? (kCodeBoundary | (uint32_t)j) : (uint32_t)(j + (tj < b ? 1 : 0));
+          v |= e << (8 * k);
+        }
+      }
+    }
+    lw[w] = v;
+  }
 }
 
 // Table index of v given sc = (1/absmax) * kCodeBins/2: the fused multiply-add
@@ -240,13 +266,14 @@ __global__ void __launch_bounds__(kQuantThreads, kQuantCtasPerSm) nf4_quantize_k
                                                                     double *__restrict__ partial, int table) {
   __shared__ double red[kQuantThreads / 32];
   __shared__ float thr[16];
+  __shared__ int tb_s[16];
   __shared__ __align__(16) uint8_t lut[kCodeLutSpan];
   NF4Thresholds th;
   th.init(table);
   if (threadIdx.x < 15)
     thr[threadIdx.x] =
         __double2float_rd(((double)kLevels[table][threadIdx.x] + (double)kLevels[table][threadIdx.x + 1]) * 0.5);
-  load_code_lut(lut, table);
+  build_code_lut(lut, table, tb_s);
   __syncthreads();
   pdl_trigger();
   pdl_wait();

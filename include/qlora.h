@@ -20,22 +20,25 @@
  *     device memory: scratch space is passed in as (ws, ws_bytes) and must be
  *     at least the size the matching *_workspace_size() function returns.
  *   - Streams: `stream` is a cudaStream_t (NULL = legacy default stream).
- *     Every call only enqueues work on that stream and never synchronizes it;
- *     outputs are valid once the stream has reached that point.  The one
- *     exception is the first call on a device: it fills a constant table of
- *     the quantizer (a function of the NF4 levels only) and waits for the
- *     device once.  The kernels are launched as programmatic dependents of
- *     the kernel before them in the stream (they may start their set-up
- *     while it finishes) and wait for it before touching any memory, so the
- *     ordering is that of plain stream order.
+ *     Every call only enqueues work on that stream and never synchronizes
+ *     the stream or the device (the diagnostics below say where they do);
+ *     outputs are valid once the stream has reached that point.  The first
+ *     call on a device reads its SM count and the address of the
+ *     library's device error word, and enqueues nothing else.  The kernels
+ *     are launched as programmatic dependents of the kernel before them in
+ *     the stream (they may start their set-up while it finishes) and wait
+ *     for it before touching any memory, so the ordering is that of plain
+ *     stream order.
  *   - bfloat16 data is passed as uint16_t bit patterns.
  *   - Alignment: every device pointer must be 16-byte aligned (W->c2_mean and
  *     c2_mean only need 4 bytes).
  *   - Errors: every call returns an int status (QLORA_OK = 0 or a negative
  *     QLORA_ERR_*); argument errors are detected on the host before anything
  *     is enqueued.  A kernel never traps: if a pipeline wait inside a kernel
- *     exceeds its time bound the kernel records a device error and returns,
- *     which qlora_get_last_device_error() reports.
+ *     exceeds its time bound (qlora_set_wait_limit_ns) the kernel records a
+ *     device error and returns, which qlora_get_last_device_error() reports.
+ *     The device error word is one per device, not per stream: it holds the
+ *     first failure of any stream's kernels since it was last cleared.
  *   - Shapes: W is stored as [n_out x k_in] row-major (a PyTorch Linear.weight;
  *     the paper's W in R^{h x o} transposed).  Blocks of 64 run along the
  *     row-major flattening, so with k_in % 64 == 0 every block lies inside one
@@ -284,6 +287,32 @@ QLORA_API int qlora_linear_bwd_dropout(const uint16_t *dY, const uint16_t *X, co
 
 /* Static description of a status code. */
 QLORA_API const char *qlora_status_str(int status);
+
+/*
+ * Bound on every wait inside the library's kernels (a pipeline stage waiting
+ * for its data, a producer waiting for a free stage), for the current device.
+ * A wait that runs longer records QLORA_ERR_DEVICE_TIMEOUT in the device
+ * error word and the kernel returns without finishing its work (no trap, no
+ * copy or MMA left in flight).  The default is QLORA_DEFAULT_WAIT_LIMIT_NS
+ * (4 s), far above any legitimate wait.  The new limit is set by a one-thread
+ * kernel enqueued on `stream` and applies to kernels that start after it.
+ * ns = 0 restores the default; ns > QLORA_MAX_WAIT_LIMIT_NS (60 s) returns
+ * QLORA_ERR_INVALID_ARG.
+ */
+#define QLORA_DEFAULT_WAIT_LIMIT_NS 4000000000ull
+#define QLORA_MAX_WAIT_LIMIT_NS 60000000000ull
+QLORA_API int qlora_set_wait_limit_ns(uint64_t ns, void *stream);
+
+/*
+ * Diagnostics of the failure path: enqueues on `stream` one thread that
+ * waits, through the same bounded wait as every pipeline of the library, on
+ * a barrier that nothing completes.  The wait runs out after the device's
+ * wait limit; the kernel then records a device timeout and returns, so that
+ * the next qlora_get_last_device_error() returns QLORA_ERR_DEVICE_TIMEOUT.
+ * It touches no caller memory.  Meant for tests of error handling, with a
+ * short limit set first.
+ */
+QLORA_API int qlora_diag_expired_wait(void *stream);
 
 /*
  * Synchronizes `stream`, then returns and clears the device error word of the

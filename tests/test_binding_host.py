@@ -1,5 +1,7 @@
-"""Argument checks of the Python binding that run before any device pointer is
-taken (no GPU needed): the grouped forward's member count and shapes."""
+"""Argument checks of the Python binding that run before the library is loaded
+or any device pointer is taken (no GPU, no built library needed): member
+counts and shapes, caller-supplied outputs of the wrong shape or dtype,
+tensors on different devices, and grouped outputs that overlap inputs."""
 
 import pytest
 import torch
@@ -35,3 +37,67 @@ def test_host_tensors_are_refused():
     # a well-formed member on the host: the binding refuses to pass host memory as device pointers
     with pytest.raises(ValueError, match="CUDA device"):
         qlora.linear_fwd_group([_member()])
+
+
+def _linear_args(M=4, N=16, K=64, r=8):
+    m = _member(M, N, K, r)
+    return m["X"], m["q"], m["L1"], m["L2"]
+
+
+@pytest.mark.parametrize("name,bad", [
+    ("Y", lambda M, N, K, r: torch.zeros(M - 1, N, dtype=torch.bfloat16)),      # too small: written past its end
+    ("Y", lambda M, N, K, r: torch.zeros(M, N, dtype=torch.float32)),
+    ("T", lambda M, N, K, r: torch.zeros(M, r, dtype=torch.bfloat16)),          # T is the [M, 2r] hi/lo pair
+])
+def test_forward_outputs_are_checked(name, bad):
+    M, N, K, r = 4, 16, 64, 8
+    X, q, L1, L2 = _linear_args(M, N, K, r)
+    with pytest.raises(ValueError, match=f"{name} must be"):
+        qlora.linear_fwd(X, q, L1, L2, 1.0, **{name: bad(M, N, K, r)})
+
+
+@pytest.mark.parametrize("name,bad,kw", [
+    ("dX", lambda M, N, K, r: torch.zeros(M, K + 64, dtype=torch.bfloat16), {}),
+    ("dL1", lambda M, N, K, r: torch.zeros(K, r, dtype=torch.bfloat16), {"grad_dtype": torch.float32}),
+    ("dL2", lambda M, N, K, r: torch.zeros(r, N, dtype=torch.float32), {}),
+    ("dL2", lambda M, N, K, r: torch.zeros(r, N - 8, dtype=torch.bfloat16), {}),
+])
+def test_backward_outputs_are_checked(name, bad, kw):
+    M, N, K, r = 4, 16, 64, 8
+    X, q, L1, L2 = _linear_args(M, N, K, r)
+    dY = torch.zeros(M, N, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match=f"{name} must be"):
+        qlora.linear_bwd(dY, X, None, q, L1, L2, 1.0, **{name: bad(M, N, K, r)}, **kw)
+
+
+def test_backward_saved_T_shape_is_checked():
+    M, N, K, r = 4, 16, 64, 8
+    X, q, L1, L2 = _linear_args(M, N, K, r)
+    dY = torch.zeros(M, N, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="hi/lo pair"):
+        qlora.linear_bwd(dY, X, torch.zeros(M, r, dtype=torch.bfloat16), q, L1, L2, 1.0)
+
+
+def test_tensors_on_another_device_are_refused():
+    X, q, L1, L2 = _linear_args()
+    with pytest.raises(ValueError, match="L2 is on meta"):
+        qlora.linear_fwd(X, q, L1, L2.to("meta"), 1.0)
+    m = _member()
+    m["L1"] = m["L1"].to("meta")
+    with pytest.raises(ValueError, match="L1 is on meta"):
+        qlora.linear_fwd_group([m])
+
+
+def test_group_outputs_may_not_overlap_inputs_or_each_other():
+    M, N, K, r = 4, 16, 64, 8
+    a, b = _member(M, N, K, r), _member(M, N, K, r)
+    b["X"] = a["X"]                                        # shared input: allowed
+    a["Y"] = a["X"].view(-1)[:M * N].view(M, N)            # output aliasing the shared input
+    with pytest.raises(ValueError, match="member 0's Y overlaps member 0's X"):
+        qlora.linear_fwd_group([a, b])
+    a, b = _member(M, N, K, r), _member(M, N, K, r)
+    buf = torch.zeros(M * N + 8, dtype=torch.bfloat16)
+    a["Y"] = buf[:M * N].view(M, N)
+    b["Y"] = buf[8:].view(M, N)                            # two outputs sharing bytes
+    with pytest.raises(ValueError, match="member 0's Y overlaps member 1's Y"):
+        qlora.linear_fwd_group([a, b])
