@@ -24,7 +24,11 @@
  *     the stream or the device (the diagnostics below say where they do);
  *     outputs are valid once the stream has reached that point.  The first
  *     call on a device reads its SM count and the address of the
- *     library's device error word, and enqueues nothing else.  The kernels
+ *     library's device error word, and enqueues nothing else.  (The library
+ *     uses the process's shared CUDA runtime.  Under CUDA's default lazy
+ *     module loading, the runtime loads each kernel at its first launch in
+ *     the process and may wait for the device to do so; with
+ *     CUDA_MODULE_LOADING=EAGER it loads them with the context instead.)  The kernels
  *     are launched as programmatic dependents of the kernel before them in
  *     the stream (they may start their set-up while it finishes) and wait
  *     for it before touching any memory, so the ordering is that of plain

@@ -30,11 +30,11 @@ qlora = pytest.importorskip("bit_nf4_quantized_02_b200")
 # The child process: load the library before CUDA starts, put a ~2 s spin
 # kernel on one stream, then make the library's first call (the quantizer) on
 # another stream and record how long the call took on the host and whether
-# the spin kernel was still running when it returned.  CUDA_MODULE_LOADING is
-# EAGER in the child so that the library's kernels are loaded when the
-# context is created: with lazy loading the CUDA runtime itself may
-# synchronize the context to load a kernel on its first launch, which is not
-# the library's doing.
+# the spin kernel was still running when it returned and when the quantizer's
+# stream had finished.  CUDA_MODULE_LOADING is EAGER in the child so that the
+# library's kernels are loaded with the context: under lazy loading the CUDA
+# runtime loads a kernel at its first launch and may wait for the device to
+# do so, for any library's kernels, which is not the library's doing.
 _CHILD = r"""
 import json, sys, time
 import numpy as np
