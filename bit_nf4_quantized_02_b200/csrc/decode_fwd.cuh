@@ -1,0 +1,355 @@
+// Fused doubleDequant + tensor-core product for up to 128 tokens (QLoRA §3
+// Eq. 5 with the frozen weight decoded on the fly, Eq. 6): the NF4 weight is
+// streamed from HBM once and decoded straight into tensor memory, where
+// tcgen05 MMAs read it as their A operand -- no bf16 copy of the weight is
+// written to HBM or to shared memory.
+//
+//   acc[M x N] += X W_hat^T        (fp32, L2-resident; zero at launch)
+//
+// computed transposed, acc^T = W_hat X^T: the weight rows are the 128-row MMA M
+// dimension (TMEM lanes) and the tokens the MMA N dimension (MP = tokens
+// padded to 16, 32, 64 or 128).  The LoRA branch and the bf16 output come
+// from the kernels around it (lora_down_small_kernel before it, which it
+// overlaps as a programmatic dependent, and gemv_epilogue_kernel after).
+//
+// The decoded weight is exactly doubleDequant's bf16 weight (bit-identical to
+// qlora_dequant): W_hat = bf16(fp32(level[c] * c2_hat)) with c2_hat =
+// fma(E4M3(code8), c1, mu), the block constant of the weight's 64-block.
+// A byte of two codes looks up the fp32 pair (level[lo], level[hi]) in a
+// fixed 256-entry table; one packed fp32 multiply (mul.rn.f32x2) applies the
+// block's c2_hat and one conversion rounds the pair to bf16 -- the same two
+// roundings as the dequant kernel, with no per-block table to build.
+//
+// One persistent CTA per SM, 14 warps:
+//   warps 0..3    epilogue: tcgen05.ld of the accumulator (lane = weight row,
+//                 column = token) and red.global.add into acc;
+//   warps 4..11   two decoder warpgroups; group g decodes the items (row tile,
+//                 256-K stage) g, g + 2, ... of the CTA's range.  Thread t
+//                 of a group owns weight row t of the tile (TMEM lane t): it
+//                 reads its row's 128 code bytes from the stage (128-byte
+//                 swizzle, conflict-free 16-byte loads), and per byte
+//                 extracts it (one byte permute), forms the address of its
+//                 replica of the table entry (one multiply-add), loads the
+//                 fp32 pair (8 bytes; the table holds 16 replicas, so each
+//                 half-warp's lookups hit 32 distinct banks), multiplies it
+//                 by c2_hat (one packed fp32 multiply) and rounds it to a bf16
+//                 pair (one conversion).  Each 64-block's 32 pairs go to TMEM
+//                 with one tcgen05.st (32 columns of the group's A slot);
+//   warp 12       producer: lane 0 loads, per stage, 128 weight rows x 256 K
+//                 of packed codes (128-byte swizzle) and the stage's X as four
+//                 K-major 128-byte-swizzled atoms of MP tokens (one 3-D box)
+//                 with TMA; all lanes copy the stage's raw block constants
+//                 with cp.async;
+//   warp 13       allocates TMEM; one thread issues tcgen05.mma (M = 128,
+//                 N = MP, K = 16; A from the group's TMEM slot, B from the X
+//                 atoms) into one of two TMEM accumulators.
+// TMEM columns: [0, 2 MP) the two accumulators, then one 128-column A slot
+// per decoder group (K = 256 bf16 of 128 rows).
+// Work: the items are split into equal contiguous ranges, one per CTA; the
+// CTA adds its partial sums into acc whenever its range moves to the next
+// row tile, and at its end.  Groups of linears concatenate their items (see
+// the group note in gemv.cuh).
+#pragma once
+
+#include "common.cuh"
+#include "quant.cuh"
+#include "gemv.cuh"
+#include "fused_fwd.cuh"
+
+namespace qlora {
+
+constexpr int kDfRows = 128;                  // weight rows per tile (MMA M, TMEM lanes)
+constexpr int kDfStageK = 256;                // K per stage: four 64-blocks
+constexpr int kDfLutEntries = 256;            // one per code byte (two codes)
+constexpr int kDfLutReplicas = 16;            // one per lane of a half-warp (8-byte loads)
+constexpr int kDfLutBytes = kDfLutEntries * kDfLutReplicas * 8;
+
+template <int MP>
+struct DfCfg {
+  static_assert(MP == 16 || MP == 32 || MP == 64 || MP == 128, "MMA N");
+  static constexpr int kGroups = 2;                           // decoder warpgroups
+  static constexpr int kDecWarp0 = 4;
+  static constexpr int kProdWarp = kDecWarp0 + 4 * kGroups;
+  static constexpr int kMmaWarp = kProdWarp + 1;
+  static constexpr int kThreads = 32 * (kMmaWarp + 1);
+  static constexpr int kCodeBytes = kDfRows * 128;            // 128 rows x 256 codes
+  static constexpr int kXBytes = 4 * MP * 128;                // 4 atoms of MP rows x 64 bf16
+  static constexpr int kCstBytes = kDfRows * 16;              // raw block constants of 128 rows
+  static constexpr int kStageBytes = kCodeBytes + kXBytes + kCstBytes;
+  static constexpr int kBarBytes = 1024;
+  static constexpr int kMaxSmem = 232448;                     // per CTA on sm_100
+  static constexpr int kStagesFit = (kMaxSmem - 1024 - kDfLutBytes - kBarBytes) / kStageBytes;
+  static constexpr int kStages = kStagesFit > 8 ? 8 : kStagesFit;
+  static constexpr int kSmemBytes = kStages * kStageBytes + kDfLutBytes + kBarBytes + 1024;
+  static constexpr int kACols = kDfStageK / 2;                // 32-bit TMEM columns per A slot
+  static constexpr int kTmemCols = 512;
+  static_assert(kStages >= 2, "pipeline depth");
+  static_assert(kCodeBytes % 1024 == 0 && kXBytes % 1024 == 0, "128-byte-swizzle boxes start 1 KB aligned");
+  static_assert(2 * MP + kGroups * kACols <= kTmemCols, "TMEM columns");
+  static_assert(kSmemBytes <= kMaxSmem, "shared memory per CTA");
+};
+
+// The fp32 pair at a shared-memory address (8-byte aligned).
+__device__ __forceinline__ uint64_t lds64(uint32_t addr) {
+  uint64_t v;
+  asm("ld.shared.b64 %0, [%1];" : "=l"(v) : "r"(addr));
+  return v;
+}
+
+// {c, c} as a packed fp32 pair.
+__device__ __forceinline__ uint64_t f32x2_splat(float c) {
+  uint64_t v;
+  asm("mov.b64 %0, {%1, %1};" : "=l"(v) : "f"(c));
+  return v;
+}
+
+// bf16 pair (low half = element 0) of the fp32 products p * c, each rounded
+// to fp32 and then to bf16 (round to nearest even both times).
+__device__ __forceinline__ uint32_t mul_round_bf16x2(uint64_t p, uint64_t c) {
+  uint64_t y;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(y) : "l"(p), "l"(c));
+  float lo, hi;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(y));
+  uint32_t d;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(hi), "f"(lo));
+  return d;
+}
+
+template <int MP, int GM>
+__global__ void __launch_bounds__(DfCfg<MP>::kThreads, 1)
+    nf4_decode_fwd_kernel(const __grid_constant__ FtMaps<GM> maps, const __grid_constant__ FtArgs<GM> p) {
+  using Cfg = DfCfg<MP>;
+  constexpr int S = Cfg::kStages;
+  constexpr int G = Cfg::kGroups;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t *lut = smem + S * Cfg::kStageBytes;
+  uint64_t *full_bar = reinterpret_cast<uint64_t *>(smem + S * Cfg::kStageBytes + kDfLutBytes);
+  uint64_t *empty_bar = full_bar + S;
+  uint64_t *afull_bar = empty_bar + S;                  // [G]
+  uint64_t *aempty_bar = afull_bar + G;                 // [G]
+  uint64_t *tfull_bar = aempty_bar + G;                 // [2]
+  uint64_t *tempty_bar = tfull_bar + 2;                 // [2]
+  uint64_t *done_bar = tempty_bar + 2;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(done_bar + 1);
+
+  const int warp = warp_id();
+  const int lane = lane_id();
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");  // the epilogue may launch and wait
+
+  // The table: entry v (a code byte) holds the fp32 pair (level[v & 15],
+  // level[v >> 4]) in replica j at byte 128 v + 8 j.
+  for (int i = threadIdx.x; i < kDfLutEntries * kDfLutReplicas; i += blockDim.x) {
+    const int v = i / kDfLutReplicas;
+    reinterpret_cast<float2 *>(lut)[i] = make_float2(p.levels[v & 15], p.levels[v >> 4]);
+  }
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < S; ++i) {
+      mbar_init(smem_u32(full_bar + i), 1 + 32);             // TMA bytes + the producer lanes' constants
+      mbar_init(smem_u32(empty_bar + i), 4 + 1);             // the decoding group's warps + the MMAs on X
+    }
+    for (int i = 0; i < G; ++i) {
+      mbar_init(smem_u32(afull_bar + i), 4);                 // the four warps of a decoder group
+      mbar_init(smem_u32(aempty_bar + i), 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(smem_u32(tfull_bar + i), 1);
+      mbar_init(smem_u32(tempty_bar + i), 4);
+    }
+    mbar_init(smem_u32(done_bar), 1);
+    fence_mbar_init();
+  }
+  if (warp == Cfg::kMmaWarp) {
+    tmem_alloc(smem_u32(tmem_slot), Cfg::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  int i0, i1;
+  ft_range(p.items, blockIdx.x, gridDim.x, i0, i1);
+
+  if (warp == Cfg::kProdWarp) {
+    // ------------------------------------------------------------ producer
+    if (lane < p.count) {
+      tma_prefetch_desc(&maps.codes[lane]);
+      tma_prefetch_desc(&maps.x[lane]);
+    }
+    int stage = 0;
+    uint32_t phase = 0, used = 0, last_parity = 0;
+    for (int it = i0; it < i1; ++it) {
+      int l, rt, ks;
+      const FtMember &m = ft_item<GM>(p, it, l, rt, ks);
+      const bool got = mbar_wait(smem_u32(empty_bar + stage), phase ^ 1, p.err, DEV_TIMEOUT_PRODUCER);
+      if (!__all_sync(0xFFFFFFFFu, got)) break;
+      const uint32_t fb = smem_u32(full_bar + stage);
+      const uint32_t sc = smem_u32(smem + stage * Cfg::kStageBytes);
+      if (lane == 0) {
+        mbar_arrive_expect_tx(fb, Cfg::kCodeBytes + Cfg::kXBytes);
+        tma_load_2d(sc, &maps.codes[l], fb, ks * (kDfStageK / 2), rt * kDfRows);
+        tma_load_3d(sc + Cfg::kCodeBytes, &maps.x[l], fb, 0, 0, ks * 4);
+      }
+      used |= 1u << stage;
+      last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
+      ft_copy_consts(m, sc + Cfg::kCodeBytes + Cfg::kXBytes, rt, ks, lane);
+      cp_async_arrive_noinc(fb);
+      if (++stage == S) {
+        stage = 0;
+        phase ^= 1;
+      }
+    }
+    // Drain: every lane's copies and lane 0's tensor copies have landed once
+    // the last phase of each used stage has completed.
+    for (int i = 0; i < S; ++i)
+      if (used & (1u << i)) {
+        const bool done = mbar_wait(smem_u32(full_bar + i), (last_parity >> i) & 1u, p.err, DEV_TIMEOUT_DRAIN);
+        if (!__all_sync(0xFFFFFFFFu, done)) break;
+      }
+  } else if (warp == Cfg::kMmaWarp) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc = idesc_bf16_f32(kDfRows, MP, 0, 0);
+      int stage = 0;
+      uint32_t phase = 0;
+      int t = 0;               // row-tile segments started
+      uint32_t accumulate = 0;
+      for (int it = i0; it < i1; ++it) {
+        int l, rt, ks;
+        const FtMember &m = ft_item<GM>(p, it, l, rt, ks);
+        const int rel = it - i0;
+        const int g = rel % G;
+        const uint32_t use = (uint32_t)(rel / G);     // this group's item count before this one
+        const bool first = it == i0 || ks == 0;
+        const bool last = it == i1 - 1 || ks == m.kstages - 1;
+        const int acc = t & 1;
+        if (first) {
+          if (!mbar_wait(smem_u32(tempty_bar + acc), ((t >> 1) & 1u) ^ 1u, p.err, DEV_TIMEOUT_MMA)) break;
+          tc_fence_after();
+          accumulate = 0;
+        }
+        if (!mbar_wait(smem_u32(full_bar + stage), phase, p.err, DEV_TIMEOUT_MMA)) break;
+        if (!mbar_wait(smem_u32(afull_bar + g), use & 1u, p.err, DEV_TIMEOUT_MMA)) break;
+        tc_fence_after();
+        const uint32_t sx = smem_u32(smem + stage * Cfg::kStageBytes) + Cfg::kCodeBytes;
+        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * MP);
+        const uint32_t a_tmem = tmem_base + (uint32_t)(2 * MP + g * Cfg::kACols);
+        const int nk = 4 * min(4, (m.K >> 6) - ks * 4);   // 16-wide k-steps of the stage's real blocks
+        for (int k = 0; k < nk; ++k) {
+          // B: atom k / 4 of the stage's X (MP rows x 128 B), 32 bytes per k-step inside it
+          tc_mma_f16_ts(d_tmem, a_tmem + 8 * k, smem_desc_sw128(sx + (k >> 2) * (MP * 128) + (k & 3) * 32, 16, 1024),
+                        idesc, accumulate);
+          accumulate = 1;
+        }
+        tc_commit(smem_u32(aempty_bar + g));         // A slot free once these MMAs have read it
+        tc_commit(smem_u32(empty_bar + stage));      // X tile consumed
+        if (++stage == S) {
+          stage = 0;
+          phase ^= 1;
+        }
+        if (last) {
+          tc_commit(smem_u32(tfull_bar + acc));      // partial sums of this row tile ready
+          ++t;
+        }
+      }
+      tc_commit(smem_u32(done_bar));
+      mbar_wait(smem_u32(done_bar), 0, p.err, DEV_TIMEOUT_DRAIN);
+    }
+  } else if (warp >= Cfg::kDecWarp0 && warp < Cfg::kProdWarp) {
+    // ------------------------------------------------------------ decoders
+    const int g = (warp - Cfg::kDecWarp0) >> 2;
+    const int quad = warp & 3;                    // TMEM lane quarter of this warp
+    const int t = quad * 32 + lane;               // weight row within the tile
+    const uint32_t lut_lane = smem_u32(lut) + 8u * (uint32_t)(lane & (kDfLutReplicas - 1));
+    const uint32_t a_row = tmem_base + ((uint32_t)(quad * 32) << 16) + (uint32_t)(2 * MP + g * Cfg::kACols);
+    const uint32_t cswz = (uint32_t)(t & 7) << 4;
+    uint32_t use = 0;
+    for (int it = i0 + g; it < i1; it += G, ++use) {
+      const int rel = it - i0;
+      const int stage = rel % S;
+      const uint32_t phase = (uint32_t)(rel / S) & 1u;
+      int l, rt, ks;
+      const FtMember &m = ft_item<GM>(p, it, l, rt, ks);
+      const int kblocks = m.K >> 6;
+      const int nkb = min(4, kblocks - ks * 4);
+      const float mu = __ldg(m.mu);
+      if (!__all_sync(0xFFFFFFFFu, mbar_wait(smem_u32(full_bar + stage), phase, p.err, DEV_TIMEOUT_MMA))) break;
+      const uint8_t *sbase = smem + stage * Cfg::kStageBytes;
+      const uint4 raw = *reinterpret_cast<const uint4 *>(sbase + Cfg::kCodeBytes + Cfg::kXBytes + t * 16);
+      const int n = rt * kDfRows + t;
+      uint64_t c2[4];     // {c2_hat, c2_hat} of the stage's four blocks
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        c2[j] = f32x2_splat((j < nkb && n < m.N) ? ft_c2hat(raw, n, ks * 4, j, kblocks, mu) : 0.f);
+      // the MMAs of this group's previous item have read its A slot
+      if (!__all_sync(0xFFFFFFFFu, mbar_wait(smem_u32(aempty_bar + g), (use & 1u) ^ 1u, p.err, DEV_TIMEOUT_MMA)))
+        break;
+      tc_fence_after();
+      const uint32_t sc = smem_u32(sbase) + t * 128;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        if (j >= nkb) break;
+        // this row's 32 code bytes of block j: 16-byte chunks 2j, 2j+1 of its swizzled 128-byte line
+        const uint4 qa = lds128(sc + (((uint32_t)(2 * j) << 4) ^ cswz));
+        const uint4 qb = lds128(sc + (((uint32_t)(2 * j + 1) << 4) ^ cswz));
+        const uint32_t q[8] = {qa.x, qa.y, qa.z, qa.w, qb.x, qb.y, qb.z, qb.w};
+        uint32_t e[32];
+#pragma unroll
+        for (int w = 0; w < 8; ++w)
+#pragma unroll
+          for (int b = 0; b < 4; ++b) {
+            const uint32_t v = __byte_perm(q[w], 0u, 0x4440u | (uint32_t)b);   // code byte b, zero-extended
+            e[4 * w + b] = mul_round_bf16x2(lds64(lut_lane + v * 128u), c2[j]);
+          }
+        tmem_st_32x32b_x32(a_row + 32 * j, e);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(smem_u32(afull_bar + g));          // A slot written
+        mbar_arrive(smem_u32(empty_bar + stage));      // codes and constants of this stage consumed
+      }
+    }
+  } else if (warp < 4) {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp;              // TMEM lane quarter
+    int t = 0;
+    for (int it = i0; it < i1; ++it) {
+      int l, rt, ks;
+      const FtMember &m = ft_item<GM>(p, it, l, rt, ks);
+      if (!(it == i1 - 1 || ks == m.kstages - 1)) continue;   // not the end of a row-tile segment
+      const int acc = t & 1;
+      const bool got = mbar_wait(smem_u32(tfull_bar + acc), (t >> 1) & 1u, p.err, DEV_TIMEOUT_EPILOGUE);
+      if (!__all_sync(0xFFFFFFFFu, got)) break;
+      tc_fence_after();
+      const int n = rt * kDfRows + q * 32 + lane;
+#pragma unroll 1
+      for (int cc = 0; cc < MP; cc += 16) {
+        uint32_t r[16];
+        tmem_ld_32x32b_x16(tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * MP + cc), r);
+        tmem_wait_ld();
+        if (n < m.N) {
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            if (cc + i < p.M) red_add_f32(m.acc + (int64_t)(cc + i) * m.N + n, __uint_as_float(r[i]));
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(tempty_bar + acc));
+      ++t;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == Cfg::kMmaWarp) tmem_dealloc(tmem_base, Cfg::kTmemCols);
+  // Complete only after the T launch this grid overlapped has completed, so
+  // that the epilogue launched after this grid sees T.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+}  // namespace qlora

@@ -14,6 +14,7 @@
 #include "tc_gemm.cuh"
 #include "gemv.cuh"
 #include "fused_fwd.cuh"
+#include "decode_fwd.cuh"
 #include "dropout.cuh"
 #include "group.cuh"
 
@@ -51,6 +52,7 @@ struct DeviceInfo {
   std::atomic<int> pair_clusters[3];     // co-resident 2-CTA clusters of the pair GEMM [form]
   std::atomic<int> gemv_per_sm[6];       // mma.sync few-token product: resident CTAs per SM [group form][NT]
   std::atomic<int> fused_smem_set[8];    // tcgen05 few-token product: smem limit set [group form][token padding]
+  std::atomic<int> decode_smem_set[8];   // TMEM-decode few-token product: smem limit set [group form][token padding]
 };
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_mu;
@@ -649,6 +651,73 @@ int launch_fused_fwd(const FwdMember *mem, int count, int64_t M, const GemvLayou
   return launch_lora_epilogue<GM>(mem, count, M, L, ws, st);
 }
 
+// Fused doubleDequant + tcgen05 forward with the weight decoded into TMEM,
+// for M <= MP tokens of a group of linears sharing one code table: T
+// accumulation, the product (a programmatic dependent of it), then the LoRA
+// epilogue.  The accumulators are zero (the caller's memset).
+template <int MP, int GM>
+int launch_decode_fwd(const FwdMember *mem, int count, int64_t M, const GemvLayout &L, uint8_t *ws, DeviceInfo *dev,
+                      cudaStream_t st) {
+  using Cfg = DfCfg<MP>;
+  FtMaps<GM> maps;
+  FtArgs<GM> a;
+  std::memset(&maps, 0, sizeof(maps));
+  std::memset(&a, 0, sizeof(a));
+  std::memcpy(a.levels, kLevelsHost[mem[0].W->table], sizeof(a.levels));
+  a.M = (int)M;
+  a.count = count;
+  a.err = dev->err;
+  int items = 0;
+  for (int i = 0; i < count; ++i) {
+    const qlora_nf4dq_t *W = mem[i].W;
+    const int64_t N = W->n_out, K = W->k_in;
+    {
+      const cuuint64_t dims[2] = {(cuuint64_t)(K / 2), (cuuint64_t)N};
+      const cuuint64_t strides[1] = {(cuuint64_t)(K / 2)};
+      const cuuint32_t box[2] = {128, (cuuint32_t)kDfRows};
+      int rc = encode_tmap(&maps.codes[i], CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, W->codes, dims, strides, box);
+      if (rc) return rc;
+    }
+    {
+      // X as [64-block][token][64]: one box = the four K-major atoms of a stage
+      const cuuint64_t dims[3] = {64, (cuuint64_t)M, (cuuint64_t)(K / 64)};
+      const cuuint64_t strides[2] = {(cuuint64_t)K * 2, 128};
+      const cuuint32_t box[3] = {64, (cuuint32_t)MP, 4};
+      int rc = encode_tmap(&maps.x[i], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, mem[i].X, dims, strides, box);
+      if (rc) return rc;
+    }
+    FtMember &m = a.m[i];
+    m.N = (int)N;
+    m.K = (int)K;
+    m.kstages = (int)((K + kDfStageK - 1) / kDfStageK);
+    m.ks_div = make_div_u31((uint32_t)m.kstages);
+    m.c2_fp8 = W->c2_fp8;
+    m.c1 = W->c1;
+    m.mu = W->c2_mean;
+    m.acc = reinterpret_cast<float *>(ws + L.acc[i]);
+    a.beg[i] = items;
+    items += (int)((N + kDfRows - 1) / kDfRows) * m.kstages;
+  }
+  a.items = items;
+  const int idx = (GM > 1 ? 4 : 0) + (MP == 16 ? 0 : (MP == 32 ? 1 : (MP == 64 ? 2 : 3)));
+  if (once(dev->decode_smem_set[idx], [&] {
+        return cudaFuncSetAttribute(nf4_decode_fwd_kernel<MP, GM>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    Cfg::kSmemBytes) == cudaSuccess
+                   ? 1
+                   : 0;
+      }) <= 0)
+    return QLORA_ERR_CUDA;
+  const int grid = std::max(1, std::min(a.items, dev->sms));
+  ProfScope prof(QLORA_KERNEL_FUSED_FWD, st);
+  // 1. T accumulation; 2. the fused product, overlapping it; 3. the LoRA epilogue.
+  int rc = launch_lora_down<GM>(mem, count, M, L, ws, st);
+  if (rc) return rc;
+  rc = launch_pdl(nf4_decode_fwd_kernel<MP, GM>, dim3(grid), dim3(Cfg::kThreads), (size_t)Cfg::kSmemBytes, st, maps,
+                  a);
+  if (rc) return rc;
+  return launch_lora_epilogue<GM>(mem, count, M, L, ws, st);
+}
+
 // Fused doubleDequant + mma.sync forward for M <= 8 NT tokens of a group of
 // linears sharing one code table (three launches, as launch_fused_fwd).
 template <int NT, int GM>
@@ -722,11 +791,10 @@ int few_token_fwd(const FwdMember *mem, int count, int64_t M, const GemvLayout &
                   cudaStream_t st) {
   // up to 32 tokens: weight decoded straight into mma.sync fragments (each
   // warp independent); 33..128: decoded into shared memory for tcgen05
-  if (M <= 8) return launch_gemv<1, GM>(mem, count, M, L, ws, dev, st);
-  if (M <= 16) return launch_gemv<2, GM>(mem, count, M, L, ws, dev, st);
-  if (M <= kGvMaxM) return launch_gemv<4, GM>(mem, count, M, L, ws, dev, st);
-  if (M <= 64) return launch_fused_fwd<64, GM>(mem, count, M, L, ws, dev, st);
-  return launch_fused_fwd<128, GM>(mem, count, M, L, ws, dev, st);
+  if (M <= 16) return launch_decode_fwd<16, GM>(mem, count, M, L, ws, dev, st);
+  if (M <= 32) return launch_decode_fwd<32, GM>(mem, count, M, L, ws, dev, st);
+  if (M <= 64) return launch_decode_fwd<64, GM>(mem, count, M, L, ws, dev, st);
+  return launch_decode_fwd<128, GM>(mem, count, M, L, ws, dev, st);
 }
 
 struct FwdLayout {

@@ -1,7 +1,7 @@
 """GPU parity of the fused few-token forward (M <= 128 tokens: the weight is
-decoded into shared memory for the tensor core and never written to HBM as
-bf16) against the float64 oracle, and its consistency with the large-M
-path's dequantized weight."""
+decoded into tensor memory for the tensor core and never written to HBM as
+bf16) against the float64 oracle, and how close its decoded weight is to
+doubleDequant's exact bf16 weight."""
 
 import numpy as np
 import pytest
@@ -37,8 +37,8 @@ def test_few_token_forward_parity(M, N, K, r):
     Y_ref, T_ref = oracle_fwd(X, w_hat, L1, L2, s)
     assert_close(bf16_to_np(Y), Y_ref, "Y")
     assert_close(qlora.t_value(T).cpu().numpy(), T_ref, "T")
-    # the base product uses exactly the dequantized weight: with L2 = 0 it matches
-    # torch's GEMM on qlora_dequant's output to fp32-accumulation accuracy
+    # with L2 = 0 the product matches torch's GEMM on qlora_dequant's output up to
+    # fp32 accumulation and the decode's bf16 roundings (2^-7 relative per weight)
     Y0, _ = qlora.linear_fwd(X.cuda(), q, L1.cuda(), torch.zeros_like(L2).cuda(), s)
     ref0 = (X.cuda().float() @ qlora.dequant(q).float().T)
     assert (Y0.float() - ref0).abs().max().item() <= 1e-2 * (ref0.abs().max().item() + 1e-6) + 1e-6
@@ -96,3 +96,29 @@ def test_llama65b_linear_16_tokens_sampled(lin):
     Y_ref, T_ref = qlora_linear.forward(Xf, w_rows, L1f, L2f[:, rows], s)
     assert_close(bf16_to_np(Y)[:, rows], Y_ref, "Y[:, sampled features]")
     assert_close(qlora.t_value(T).cpu().numpy(), T_ref, "T")
+
+
+@pytest.mark.parametrize("M", [16, 48, 128])
+@pytest.mark.parametrize("table", ["nf4", "fp4"])
+def test_decoded_weight_is_double_dequant(M, table):
+    """One-hot token rows pick single input features, so with L2 = 0 each
+    output is one decoded weight (an fp32 sum of one product, exact in bf16):
+    the few-token product decodes exactly doubleDequant's bf16 weight, bit for
+    bit, zero codes included."""
+    N, K, r = 264, 1088, 8
+    g = inputs.rng(700 + M)
+    W = torch.from_numpy(inputs.weight_f32(g, N, K))
+    W[:, 5] = 0.0                                   # exact zeros inside nonzero blocks
+    ks = np.sort(np.random.default_rng(M).choice(K, M, replace=False))
+    ks[0] = 5
+    X = torch.zeros(M, K, dtype=torch.bfloat16)
+    X[np.arange(M), ks] = 1.0
+    L1 = torch.zeros(K, r, dtype=torch.bfloat16)
+    L2 = torch.zeros(r, N, dtype=torch.bfloat16)
+    q = qlora.quantize_nf4_dq(W.cuda(), table=table)
+    Y, _ = qlora.linear_fwd(X.cuda(), q, L1.cuda(), L2.cuda(), 1.0)
+    exact = qlora.dequant(q)[:, torch.as_tensor(ks, device="cuda")].T     # [M, N] bf16
+    torch.cuda.synchronize()
+    assert qlora.last_device_error() == 0
+    assert not Y[0].float().abs().any()
+    assert torch.equal(Y.view(torch.int16), exact.contiguous().view(torch.int16))
