@@ -20,11 +20,12 @@
 // block's c2_hat and one conversion rounds the pair to bf16 -- the same two
 // roundings as the dequant kernel, with no per-block table to build.
 //
-// One persistent CTA per SM, 14 warps:
+// One persistent CTA per SM, 4 + 4 G + 2 warps:
 //   warps 0..3    epilogue: tcgen05.ld of the accumulator (lane = weight row,
 //                 column = token) and red.global.add into acc;
-//   warps 4..11   two decoder warpgroups; group g decodes the items (row tile,
-//                 256-K stage) g, g + 2, ... of the CTA's range.  Thread t
+//   warps 4..    G decoder warpgroups (3 up to 64 tokens, 2 at 128, where
+//                 TMEM holds fewer A slots); group g decodes the items (row
+//                 tile, 256-K stage) g, g + G, ... of the CTA's range.  Thread t
 //                 of a group owns weight row t of the tile (TMEM lane t): it
 //                 reads its row's 128 code bytes from the stage (128-byte
 //                 swizzle, conflict-free 16-byte loads), and per byte
@@ -35,12 +36,15 @@
 //                 by c2_hat (one packed fp32 multiply) and rounds it to a bf16
 //                 pair (one conversion).  Each 64-block's 32 pairs go to TMEM
 //                 with one tcgen05.st (32 columns of the group's A slot);
-//   warp 12       producer: lane 0 loads, per stage, 128 weight rows x 256 K
+//   warp P        producer: lane 0 loads, per stage, 128 weight rows x 256 K
 //                 of packed codes (128-byte swizzle) and the stage's X as four
 //                 K-major 128-byte-swizzled atoms of MP tokens (one 3-D box)
-//                 with TMA; all lanes copy the stage's raw block constants
-//                 with cp.async;
-//   warp 13       allocates TMEM; one thread issues tcgen05.mma (M = 128,
+//                 with TMA.  The raw block constants of a row (its four E4M3
+//                 codes and c1) are loaded by the decoder thread that owns
+//                 the row, into registers, two of its items ahead: gathered
+//                 by one producer warp, 128 rows of scattered 4-byte copies
+//                 per stage set the pace of the whole kernel;
+//   warp P + 1    allocates TMEM; one thread issues tcgen05.mma (M = 128,
 //                 N = MP, K = 16; A from the group's TMEM slot, B from the X
 //                 atoms) into one of two TMEM accumulators.
 // TMEM columns: [0, 2 MP) the two accumulators, then one 128-column A slot
@@ -67,15 +71,14 @@ constexpr int kDfLutBytes = kDfLutEntries * kDfLutReplicas * 8;
 template <int MP>
 struct DfCfg {
   static_assert(MP == 16 || MP == 32 || MP == 64 || MP == 128, "MMA N");
-  static constexpr int kGroups = 2;                           // decoder warpgroups
+  static constexpr int kGroups = MP <= 64 ? 3 : 2;            // decoder warpgroups
   static constexpr int kDecWarp0 = 4;
   static constexpr int kProdWarp = kDecWarp0 + 4 * kGroups;
   static constexpr int kMmaWarp = kProdWarp + 1;
   static constexpr int kThreads = 32 * (kMmaWarp + 1);
   static constexpr int kCodeBytes = kDfRows * 128;            // 128 rows x 256 codes
   static constexpr int kXBytes = 4 * MP * 128;                // 4 atoms of MP rows x 64 bf16
-  static constexpr int kCstBytes = kDfRows * 16;              // raw block constants of 128 rows
-  static constexpr int kStageBytes = kCodeBytes + kXBytes + kCstBytes;
+  static constexpr int kStageBytes = kCodeBytes + kXBytes;
   static constexpr int kBarBytes = 1024;
   static constexpr int kMaxSmem = 232448;                     // per CTA on sm_100
   static constexpr int kStagesFit = (kMaxSmem - 1024 - kDfLutBytes - kBarBytes) / kStageBytes;
@@ -115,6 +118,39 @@ __device__ __forceinline__ uint32_t mul_round_bf16x2(uint64_t p, uint64_t c) {
   return d;
 }
 
+// Raw block constants of weight row n for stage ks, in registers, in the
+// layout ft_c2hat reads: the two aligned 32-bit words of c2_fp8 holding the
+// row's (up to) four E4M3 codes of the stage, then c1 of the first and of
+// the last of those blocks.  Words that reach past the end of c2_fp8 are
+// read byte by byte.  Rows past the weight read nothing.
+__device__ __forceinline__ uint4 df_load_raw(const FtMember &m, int n, int ks) {
+  uint4 raw = make_uint4(0, 0, 0, 0);
+  if (n >= m.N) return raw;
+  const int kblocks = m.K >> 6;
+  const int kb0 = ks * 4;
+  const int nb = min(4, kblocks - kb0);
+  const int64_t nblk = (int64_t)m.N * kblocks;
+  const int64_t b0 = (int64_t)n * kblocks + kb0;
+  const int64_t last = b0 + nb - 1;
+  const int64_t w0 = b0 >> 2;
+  uint32_t wv[2] = {0u, 0u};
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {
+    const int64_t w = w0 + k;
+    if (k == 1 && (last >> 2) == w0) break;
+    if (4 * w + 3 < nblk) {
+      wv[k] = __ldg(reinterpret_cast<const uint32_t *>(m.c2_fp8) + w);
+    } else {
+      for (int64_t b = 4 * w; b < nblk; ++b) wv[k] |= (uint32_t)__ldg(m.c2_fp8 + b) << (8 * (int)(b - 4 * w));
+    }
+  }
+  raw.x = wv[0];
+  raw.y = wv[1];
+  raw.z = __float_as_uint(__ldg(m.c1 + (b0 >> 8)));
+  raw.w = __float_as_uint(__ldg(m.c1 + (last >> 8)));
+  return raw;
+}
+
 template <int MP, int GM>
 __global__ void __launch_bounds__(DfCfg<MP>::kThreads, 1)
     nf4_decode_fwd_kernel(const __grid_constant__ FtMaps<GM> maps, const __grid_constant__ FtArgs<GM> p) {
@@ -145,7 +181,7 @@ __global__ void __launch_bounds__(DfCfg<MP>::kThreads, 1)
   }
   if (threadIdx.x == 0) {
     for (int i = 0; i < S; ++i) {
-      mbar_init(smem_u32(full_bar + i), 1 + 32);             // TMA bytes + the producer lanes' constants
+      mbar_init(smem_u32(full_bar + i), 1);                  // the TMA bytes
       mbar_init(smem_u32(empty_bar + i), 4 + 1);             // the decoding group's warps + the MMAs on X
     }
     for (int i = 0; i < G; ++i) {
@@ -181,7 +217,7 @@ __global__ void __launch_bounds__(DfCfg<MP>::kThreads, 1)
     uint32_t phase = 0, used = 0, last_parity = 0;
     for (int it = i0; it < i1; ++it) {
       int l, rt, ks;
-      const FtMember &m = ft_item<GM>(p, it, l, rt, ks);
+      ft_item<GM>(p, it, l, rt, ks);
       const bool got = mbar_wait(smem_u32(empty_bar + stage), phase ^ 1, p.err, DEV_TIMEOUT_PRODUCER);
       if (!__all_sync(0xFFFFFFFFu, got)) break;
       const uint32_t fb = smem_u32(full_bar + stage);
@@ -193,15 +229,13 @@ __global__ void __launch_bounds__(DfCfg<MP>::kThreads, 1)
       }
       used |= 1u << stage;
       last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
-      ft_copy_consts(m, sc + Cfg::kCodeBytes + Cfg::kXBytes, rt, ks, lane);
-      cp_async_arrive_noinc(fb);
       if (++stage == S) {
         stage = 0;
         phase ^= 1;
       }
     }
-    // Drain: every lane's copies and lane 0's tensor copies have landed once
-    // the last phase of each used stage has completed.
+    // Drain: lane 0's tensor copies have landed once the last phase of each
+    // used stage has completed.
     for (int i = 0; i < S; ++i)
       if (used & (1u << i)) {
         const bool done = mbar_wait(smem_u32(full_bar + i), (last_parity >> i) & 1u, p.err, DEV_TIMEOUT_DRAIN);
@@ -236,12 +270,23 @@ __global__ void __launch_bounds__(DfCfg<MP>::kThreads, 1)
         const uint32_t d_tmem = tmem_base + (uint32_t)(acc * MP);
         const uint32_t a_tmem = tmem_base + (uint32_t)(2 * MP + g * Cfg::kACols);
         const int nk = 4 * min(4, (m.K >> 6) - ks * 4);   // 16-wide k-steps of the stage's real blocks
-        for (int k = 0; k < nk; ++k) {
-          // B: atom k / 4 of the stage's X (MP rows x 128 B), 32 bytes per k-step inside it
-          tc_mma_f16_ts(d_tmem, a_tmem + 8 * k, smem_desc_sw128(sx + (k >> 2) * (MP * 128) + (k & 3) * 32, 16, 1024),
-                        idesc, accumulate);
-          accumulate = 1;
+        // The issuing thread is held for the duration of each MMA (tens of
+        // cycles at these sizes), so the k-step loop carries no arithmetic:
+        // k-step k reads A columns 8k and, as B, atom k / 4 of the stage's X
+        // (MP rows x 128 B) at byte 32 (k % 4) inside it -- a constant
+        // offset of the stage's descriptor (its address field counts 16 B).
+        const uint64_t b0 = smem_desc_sw128(sx, 16, 1024);
+        if (nk == 16) {
+          tc_mma_f16_ts(d_tmem, a_tmem, b0, idesc, accumulate);
+#pragma unroll
+          for (int k = 1; k < 16; ++k)
+            tc_mma_f16_ts(d_tmem, a_tmem + 8 * k, b0 + (uint64_t)(((k >> 2) * (MP * 128) + (k & 3) * 32) >> 4), idesc, 1u);
+        } else {
+          for (int k = 0; k < nk; ++k)
+            tc_mma_f16_ts(d_tmem, a_tmem + 8 * k, b0 + (uint64_t)(((k >> 2) * (MP * 128) + (k & 3) * 32) >> 4), idesc,
+                          k == 0 ? accumulate : 1u);
         }
+        accumulate = 1;
         tc_commit(smem_u32(aempty_bar + g));         // A slot free once these MMAs have read it
         tc_commit(smem_u32(empty_bar + stage));      // X tile consumed
         if (++stage == S) {
@@ -264,8 +309,18 @@ __global__ void __launch_bounds__(DfCfg<MP>::kThreads, 1)
     const uint32_t lut_lane = smem_u32(lut) + 8u * (uint32_t)(lane & (kDfLutReplicas - 1));
     const uint32_t a_row = tmem_base + ((uint32_t)(quad * 32) << 16) + (uint32_t)(2 * MP + g * Cfg::kACols);
     const uint32_t cswz = (uint32_t)(t & 7) << 4;
-    uint32_t use = 0;
-    for (int it = i0 + g; it < i1; it += G, ++use) {
+    // the raw constants of this group's item it + u G (none past the range)
+    auto raw_of = [&](int u) -> uint4 {
+      const int it = i0 + g + u * G;
+      if (it >= i1) return make_uint4(0, 0, 0, 0);
+      int l, rt, ks;
+      const FtMember &m = ft_item<GM>(p, it, l, rt, ks);
+      return df_load_raw(m, rt * kDfRows + t, ks);
+    };
+    // Decode the group's item u with its constants `raw`, then start loading
+    // the constants of item u + 2 into `raw`.  Returns false on a timeout.
+    auto item = [&](int u, uint4 &raw) -> bool {
+      const int it = i0 + g + u * G;
       const int rel = it - i0;
       const int stage = rel % S;
       const uint32_t phase = (uint32_t)(rel / S) & 1u;
@@ -273,20 +328,19 @@ __global__ void __launch_bounds__(DfCfg<MP>::kThreads, 1)
       const FtMember &m = ft_item<GM>(p, it, l, rt, ks);
       const int kblocks = m.K >> 6;
       const int nkb = min(4, kblocks - ks * 4);
-      const float mu = __ldg(m.mu);
-      if (!__all_sync(0xFFFFFFFFu, mbar_wait(smem_u32(full_bar + stage), phase, p.err, DEV_TIMEOUT_MMA))) break;
-      const uint8_t *sbase = smem + stage * Cfg::kStageBytes;
-      const uint4 raw = *reinterpret_cast<const uint4 *>(sbase + Cfg::kCodeBytes + Cfg::kXBytes + t * 16);
       const int n = rt * kDfRows + t;
+      const float mu = __ldg(m.mu);
       uint64_t c2[4];     // {c2_hat, c2_hat} of the stage's four blocks
 #pragma unroll
       for (int j = 0; j < 4; ++j)
         c2[j] = f32x2_splat((j < nkb && n < m.N) ? ft_c2hat(raw, n, ks * 4, j, kblocks, mu) : 0.f);
+      raw = raw_of(u + 2);
+      if (!__all_sync(0xFFFFFFFFu, mbar_wait(smem_u32(full_bar + stage), phase, p.err, DEV_TIMEOUT_MMA))) return false;
       // the MMAs of this group's previous item have read its A slot
-      if (!__all_sync(0xFFFFFFFFu, mbar_wait(smem_u32(aempty_bar + g), (use & 1u) ^ 1u, p.err, DEV_TIMEOUT_MMA)))
-        break;
+      if (!__all_sync(0xFFFFFFFFu, mbar_wait(smem_u32(aempty_bar + g), ((uint32_t)u & 1u) ^ 1u, p.err, DEV_TIMEOUT_MMA)))
+        return false;
       tc_fence_after();
-      const uint32_t sc = smem_u32(sbase) + t * 128;
+      const uint32_t sc = smem_u32(smem + stage * Cfg::kStageBytes) + t * 128;
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         if (j >= nkb) break;
@@ -309,8 +363,14 @@ __global__ void __launch_bounds__(DfCfg<MP>::kThreads, 1)
       __syncwarp();
       if (lane == 0) {
         mbar_arrive(smem_u32(afull_bar + g));          // A slot written
-        mbar_arrive(smem_u32(empty_bar + stage));      // codes and constants of this stage consumed
+        mbar_arrive(smem_u32(empty_bar + stage));      // codes of this stage consumed
       }
+      return true;
+    };
+    uint4 ra = raw_of(0), rb = raw_of(1);
+    for (int u = 0; i0 + g + u * G < i1; u += 2) {
+      if (!item(u, ra)) break;
+      if (i0 + g + (u + 1) * G >= i1 || !item(u + 1, rb)) break;
     }
   } else if (warp < 4) {
     // ------------------------------------------------------------ epilogue
