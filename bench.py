@@ -278,6 +278,27 @@ TRAIN = {"llama7b-train": workloads.LLAMA7B_LAYER, "llama65b-train": workloads.L
          "llama33b-stack": workloads.LLAMA33B_STACK}
 
 
+def train_config(args, wl, world):
+    """The `config` of a training-workload line (both arms print the same one)."""
+    return {"workload": wl.name + (f"[{args.linear} only]" if args.linear else "")
+                        + (f"-lora-dropout{args.dropout:g}" if args.dropout > 0 else ""),
+            "model": {"llama7b-train": "llama7b-layer-linears", "llama65b-train": "llama65b-layer-linears",
+                      "llama33b-stack": "llama33b-8-layer-stack"}[args.workload],
+            "global_batch": (16 if wl.M == 8192 and args.workload == "llama7b-train" else 4) * world,
+            "seq_len": 512 if args.workload == "llama7b-train" else 2048,
+            "tokens_per_rank": wl.M, "lora_r": wl.r, "lora_alpha": wl.alpha, "layers": wl.layers,
+            "parallelism": f"dp{world}" if world > 1 else "single",
+            "step": f"quantize {7 * wl.layers} fp32 weights to NF4+DQ, fwd + bwd of the "
+                    f"{7 * wl.layers} QLoRA linears"
+                    + (" (forward of the linears that read the same input as one grouped call: q, k, v, "
+                       "gate, up on the layer input)" if wl.layers == 1 and args.dropout == 0 else "")
+                    + (" (layer to layer: H' = bf16(down(up(H)) + R))" if wl.layers > 1 else "")
+                    + (", all-reduce of adapter grads" if world > 1 else "")
+                    + (f", LoRA dropout p = {args.dropout:g} on every adapter (one seeded keep mask per "
+                       f"linear, copied in with the inputs in e2e)" if args.dropout > 0 else ""),
+            "l2": "inputs larger than L2 (>1 GB touched per step), no flush"}
+
+
 def run_ours(args, rank, world, local_rank):
     import bit_nf4_quantized_02_b200 as qlora
     from bit_nf4_quantized_02_b200 import _lib
@@ -416,23 +437,7 @@ def run_ours(args, rank, world, local_rank):
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": wl.name + (f"[{args.linear} only]" if args.linear else "")
-                               + (f"-lora-dropout{args.dropout:g}" if args.dropout > 0 else ""),
-                   "model": {"llama7b-train": "llama7b-layer-linears", "llama65b-train": "llama65b-layer-linears",
-                             "llama33b-stack": "llama33b-8-layer-stack"}[args.workload],
-                   "global_batch": (16 if wl.M == 8192 and args.workload == "llama7b-train" else 4) * world,
-                   "seq_len": 512 if args.workload == "llama7b-train" else 2048,
-                   "tokens_per_rank": wl.M, "lora_r": wl.r, "lora_alpha": wl.alpha, "layers": wl.layers,
-                   "parallelism": f"dp{world}" if world > 1 else "single",
-                   "step": f"quantize {7 * wl.layers} fp32 weights to NF4+DQ, fwd + bwd of the "
-                           f"{7 * wl.layers} QLoRA linears"
-                           + (" (forward of the linears that read the same input as one grouped call: q, k, v, "
-                              "gate, up on the layer input)" if wl.layers == 1 and args.dropout == 0 else "")
-                           + (" (layer to layer: H' = bf16(down(up(H)) + R))" if wl.layers > 1 else "")
-                           + (", all-reduce of adapter grads" if world > 1 else "")
-                           + (f", LoRA dropout p = {args.dropout:g} on every adapter (one seeded keep mask per "
-                              f"linear, copied in with the inputs in e2e)" if args.dropout > 0 else ""),
-                   "l2": "inputs larger than L2 (>1 GB touched per step), no flush"},
+        "config": train_config(args, wl, world),
         "e2e": ({"value": flops / (ms_e2e * 1e-3) / 1e12, "unit": UNIT, "h2d_bytes_per_step": h2d,
                  "d2h_bytes_per_step": d2h,
                  "copies": ("host->device copies on a copy stream in the order the step first reads them, "
@@ -448,8 +453,17 @@ def run_ours(args, rank, world, local_rank):
         "kernels": kernels,
         "clocks": clocks,
     }
-    if world == 1 and not args.no_cpu_baseline and not args.linear and args.workload == "llama7b-train":
+    default_line = world == 1 and not args.linear and args.workload == "llama7b-train" and args.dropout == 0
+    if default_line and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline()
+    if default_line and not args.no_subrecords:
+        # the other targets, each timed on its own (CUDA events) after the headline:
+        # the decode-sized forward (LLaMA-65B layer at 16 tokens) and the quantizer
+        del lins, grads, acts, step, flat
+        torch.cuda.empty_cache()
+        out["decode"] = decode_subrecord(args, rank, world, local_rank)
+        torch.cuda.empty_cache()
+        out["quantizer"] = quantizer_subrecord(args, rank, world, local_rank)
     return out
 
 
@@ -633,7 +647,7 @@ def run_decode(args, rank, world, local_rank):
         "variants": variants,
         "gpu_launches": _kernel_count(launches),
         "roofline": {"bound": "hbm", "kernel": ("few-token forward chain (lora_down_small + " +
-                                                ("gemv_fwd" if M <= 32 else "nf4_fused_fwd (tcgen05)") + " + epilogue)"),
+                                                "nf4_decode_fwd: weight decoded into TMEM, tcgen05" + " + epilogue)"),
                      "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak if achieved else None, "traffic": None,
                      "peak_source": f"{peak_src} hbm_gbs", "launches_timed": dom[0],
@@ -705,6 +719,102 @@ def run_quantizer(args, rank, world, local_rank):
     }
 
 
+# --------------------------------------------------------------------------- sub-records
+def _subargs(args, **kw):
+    ns = argparse.Namespace(**vars(args))
+    ns.__dict__.update(kw)
+    return ns
+
+
+SUB_KEYS = ("metric", "value", "unit", "ms_per_step", "steps", "warmup", "config", "graph", "variants",
+            "roofline", "accuracy", "kernels", "gpu_launches", "clocks")
+
+
+def decode_subrecord(args, rank, world, local_rank):
+    """Config 4a in the default line: the LLaMA-65B layer forward at 16 tokens."""
+    sub = run_decode(_subargs(args, steps=20, warmup=3, tokens=workloads.LLAMA65B_LAYER.extra["M_decode"]),
+                     rank, world, local_rank)
+    rec = {k: sub[k] for k in SUB_KEYS if k in sub}
+    peak = sub["roofline"]["peak"]
+    rec["frac_of_hbm"] = sub["value"] / peak
+    if not args.no_cpu_baseline:
+        rec["cpu_baseline"] = decode_cpu_baseline()
+    return rec
+
+
+def quantizer_subrecord(args, rank, world, local_rank):
+    """Config 3 in the default line: NF4 + DQ quantize and dequantize of LLaMA-7B-shaped bf16 weights."""
+    sub = run_quantizer(_subargs(args, steps=20, warmup=3, table="nf4"), rank, world, local_rank)
+    rec = {k: sub[k] for k in SUB_KEYS if k in sub}
+    peak = sub["roofline"]["peak"]
+    rec["frac_of_hbm"] = sub["value"] / peak
+    if not args.no_cpu_baseline:
+        rec["cpu_baseline"] = quantizer_cpu_baseline()
+    return rec
+
+
+def nf4_nbytes(n_out: int, k_in: int) -> int:
+    """Bytes of a weight in the stored NF4 + DQ format (codes, E4M3 block codes, c1, mean)."""
+    n = n_out * k_in
+    nblk = (n + 63) // 64
+    return (n + 1) // 2 + nblk + 4 * ((nblk + 255) // 256) + 4
+
+
+def decode_step_bytes(M: int, r: int) -> int:
+    """Algorithmic bytes of the decode step: NF4 + DQ weights, LoRA factors, X read, Y and T written."""
+    return sum(nf4_nbytes(l.n_out, l.k_in) + 2 * r * (l.k_in + l.n_out) + 2 * M * l.k_in + 2 * M * l.n_out
+               + 2 * M * 2 * r for l in workloads.LLAMA65B_LAYER.linears)
+
+
+DECODE_SAMPLE = 8
+
+
+def decode_cpu_baseline():
+    """The oracle's doubleDequant + fp64 forward on 1/8 of each LLaMA-65B linear's
+    output rows at 16 tokens (the weights quantized beforehand, untimed), scaled x8."""
+    from oracle import nf4dq, qlora_linear
+    wl = workloads.LLAMA65B_LAYER
+    M, r, s = wl.extra["M_decode"], wl.r, wl.s
+    g = inputs.rng(wl.seed + 9)
+    data = []
+    for lin in wl.linears:
+        N, K = lin.n_out, lin.k_in
+        rows = N // DECODE_SAMPLE
+        oq = nf4dq.quantize_nf4_dq(inputs.weight_f32(g, rows, K))
+        L1, L2 = inputs.lora_factors(g, K, rows, r)
+        data.append((oq, inputs.normal_bf16(g, (M, K)).float().numpy().astype(np.float64),
+                     L1.float().numpy().astype(np.float64), L2.float().numpy().astype(np.float64)))
+    t0 = time.perf_counter()
+    for oq, X, L1, L2 in data:
+        qlora_linear.forward(X, nf4dq.dequantize(oq), L1, L2, s)
+    dt = time.perf_counter() - t0
+    return {"value": decode_step_bytes(M, r) / (dt * DECODE_SAMPLE) / 1e9, "unit": "GB/s", "cores": _cores(),
+            "kind": "oracle", "sample_seconds": dt,
+            "sample": f"doubleDequant + fp64 forward of 1/{DECODE_SAMPLE} of each linear's output rows at {M} "
+                      f"tokens (weights quantized beforehand); full-step time = {DECODE_SAMPLE} x sample"}
+
+
+QUANT_SAMPLE = 8
+
+
+def quantizer_cpu_baseline():
+    """The oracle's NF4 + DQ quantize and doubleDequant of 1/8 of each matrix's rows, scaled x8."""
+    from oracle import nf4dq
+    wl = workloads.QUANTIZER_7B
+    g = inputs.rng(wl.seed + 9)
+    mats = [inputs.weight_bf16_with_outliers(g, l.n_out // QUANT_SAMPLE, l.k_in).float().numpy()
+            for l in wl.linears]
+    t0 = time.perf_counter()
+    for W in mats:
+        nf4dq.dequantize(nf4dq.quantize_nf4_dq(W))
+    dt = time.perf_counter() - t0
+    nbytes = sum(2 * (2 * l.n_out * l.k_in + nf4_nbytes(l.n_out, l.k_in)) for l in wl.linears)
+    return {"value": nbytes / (dt * QUANT_SAMPLE) / 1e9, "unit": "GB/s", "cores": _cores(), "kind": "oracle",
+            "sample_seconds": dt,
+            "sample": f"NF4+DQ quantize and doubleDequant of 1/{QUANT_SAMPLE} of each matrix's rows; "
+                      f"full-step time = {QUANT_SAMPLE} x sample"}
+
+
 # --------------------------------------------------------------------------- oracle timing
 SAMPLE_SLICE = 64   # the CPU sample is 1/64 of a step: 128 of the 8192 tokens, 1/64 of each weight's rows
 
@@ -751,14 +861,26 @@ SAMPLE_DESC = (f"1/{SAMPLE_SLICE} of a step: NF4+DQ of 1/{SAMPLE_SLICE} of each 
 
 
 def cpu_baseline(reps=1):
+    """The oracle on the host cores (all BLAS threads), and again on one thread."""
     data = _oracle_sample_setup()
     t0 = time.perf_counter()
     for _ in range(reps):
         _oracle_sample_step(data)
     dt = (time.perf_counter() - t0) / reps
     step_s = dt * SAMPLE_SLICE
-    return {"value": step_flops() / step_s / 1e12, "unit": UNIT, "cores": _cores(), "kind": "oracle",
-            "sample": SAMPLE_DESC, "sample_seconds": dt}
+    out = {"value": step_flops() / step_s / 1e12, "unit": UNIT, "cores": _cores(), "kind": "oracle",
+           "sample": SAMPLE_DESC, "sample_seconds": dt}
+    try:
+        from threadpoolctl import threadpool_limits
+        with threadpool_limits(limits=1):
+            t0 = time.perf_counter()
+            _oracle_sample_step(data)
+            dt1 = time.perf_counter() - t0
+        out["single_thread"] = {"value": step_flops() / (dt1 * SAMPLE_SLICE) / 1e12, "unit": UNIT, "cores": 1,
+                                "sample_seconds": dt1}
+    except ImportError:
+        pass
+    return out
 
 
 def run_reference(args, rank, world):
@@ -778,9 +900,9 @@ def run_reference(args, rank, world):
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_s * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": WL.name, "model": "llama7b-layer-linears", "global_batch": 16, "seq_len": 512,
-                   "lora_r": WL.r, "lora_alpha": WL.alpha, "parallelism": "single (rank 0 only)"},
-        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": SAMPLE_DESC},
+        "config": train_config(_subargs(args, workload="llama7b-train", linear=None, dropout=0.0), WL, 1),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": SAMPLE_DESC,
+                         "sample_seconds": dt},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
 
@@ -874,6 +996,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end (host buffers) measurement")
+    ap.add_argument("--no-subrecords", action="store_true",
+                    help="default workload: skip the decode (16-token) and quantizer sub-records")
     ap.add_argument("--table", choices=["nf4", "fp4"], default="nf4",
                     help="4-bit code table of the quantizer workload (fp4: FP4 E2M1, compared against NF4)")
     ap.add_argument("--dropout", type=float, default=0.0,

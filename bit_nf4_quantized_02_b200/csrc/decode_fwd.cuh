@@ -20,12 +20,11 @@
 // block's c2_hat and one conversion rounds the pair to bf16 -- the same two
 // roundings as the dequant kernel, with no per-block table to build.
 //
-// One persistent CTA per SM, 4 + 4 G + 2 warps:
+// One persistent CTA per SM, 14 warps:
 //   warps 0..3    epilogue: tcgen05.ld of the accumulator (lane = weight row,
 //                 column = token) and red.global.add into acc;
-//   warps 4..    G decoder warpgroups (3 up to 64 tokens, 2 at 128, where
-//                 TMEM holds fewer A slots); group g decodes the items (row
-//                 tile, 256-K stage) g, g + G, ... of the CTA's range.  Thread t
+//   warps 4..11   two decoder warpgroups; group g decodes the items (row
+//                 tile, 256-K stage) g, g + 2, ... of the CTA's range.  Thread t
 //                 of a group owns weight row t of the tile (TMEM lane t): it
 //                 reads its row's 128 code bytes from the stage (128-byte
 //                 swizzle, conflict-free 16-byte loads), and per byte
@@ -36,15 +35,23 @@
 //                 by c2_hat (one packed fp32 multiply) and rounds it to a bf16
 //                 pair (one conversion).  Each 64-block's 32 pairs go to TMEM
 //                 with one tcgen05.st (32 columns of the group's A slot);
-//   warp P        producer: lane 0 loads, per stage, 128 weight rows x 256 K
-//                 of packed codes (128-byte swizzle) and the stage's X as four
-//                 K-major 128-byte-swizzled atoms of MP tokens (one 3-D box)
-//                 with TMA.  The raw block constants of a row (its four E4M3
+//   warp 12       producer: lane 0 loads, per stage, 128 weight rows x 256 K
+//                 of packed codes (128-byte swizzle) into the codes ring and
+//                 the stage's X as four K-major 128-byte-swizzled atoms of MP
+//                 tokens (one 3-D box) into the X ring, with TMA.  A decoder
+//                 thread copies its row's 128 code bytes into registers as
+//                 soon as they land and the slot goes back to the producer at
+//                 once, so nearly the whole codes ring (up to 8 x 16 KB) is
+//                 in flight: at HBM rate a stage takes thousands of cycles to
+//                 land, and slots held while their data is decoded starved
+//                 the memory pipeline.  The X ring is released by the MMAs'
+//                 one commit per item, which also frees the decoding group's
+//                 TMEM slot;  The raw block constants of a row (its four E4M3
 //                 codes and c1) are loaded by the decoder thread that owns
 //                 the row, into registers, two of its items ahead: gathered
 //                 by one producer warp, 128 rows of scattered 4-byte copies
 //                 per stage set the pace of the whole kernel;
-//   warp P + 1    allocates TMEM; one thread issues tcgen05.mma (M = 128,
+//   warp 13       allocates TMEM; one thread issues tcgen05.mma (M = 128,
 //                 N = MP, K = 16; A from the group's TMEM slot, B from the X
 //                 atoms) into one of two TMEM accumulators.
 // TMEM columns: [0, 2 MP) the two accumulators, then one 128-column A slot
@@ -71,24 +78,27 @@ constexpr int kDfLutBytes = kDfLutEntries * kDfLutReplicas * 8;
 template <int MP>
 struct DfCfg {
   static_assert(MP == 16 || MP == 32 || MP == 64 || MP == 128, "MMA N");
-  static constexpr int kGroups = MP <= 64 ? 3 : 2;            // decoder warpgroups
+  static constexpr int kGroups = 2;                           // decoder warpgroups
   static constexpr int kDecWarp0 = 4;
   static constexpr int kProdWarp = kDecWarp0 + 4 * kGroups;
   static constexpr int kMmaWarp = kProdWarp + 1;
   static constexpr int kThreads = 32 * (kMmaWarp + 1);
   static constexpr int kCodeBytes = kDfRows * 128;            // 128 rows x 256 codes
   static constexpr int kXBytes = 4 * MP * 128;                // 4 atoms of MP rows x 64 bf16
-  static constexpr int kStageBytes = kCodeBytes + kXBytes;
   static constexpr int kBarBytes = 1024;
   static constexpr int kMaxSmem = 232448;                     // per CTA on sm_100
-  static constexpr int kStagesFit = (kMaxSmem - 1024 - kDfLutBytes - kBarBytes) / kStageBytes;
-  static constexpr int kStages = kStagesFit > 8 ? 8 : kStagesFit;
-  static constexpr int kSmemBytes = kStages * kStageBytes + kDfLutBytes + kBarBytes + 1024;
+  static constexpr int kRingBytes = kMaxSmem - 1024 - kDfLutBytes - kBarBytes;
+  // X ring: 64 KB of stages (at least two); the codes ring takes the rest, up to 8 stages
+  static constexpr int kXStages = (65536 / kXBytes) < 2 ? 2 : (65536 / kXBytes > 8 ? 8 : 65536 / kXBytes);
+  static constexpr int kCodeStagesFit = (kRingBytes - kXStages * kXBytes) / kCodeBytes;
+  static constexpr int kCodeStages = kCodeStagesFit > 8 ? 8 : kCodeStagesFit;
+  static constexpr int kSmemBytes = kCodeStages * kCodeBytes + kXStages * kXBytes + kDfLutBytes + kBarBytes + 1024;
   static constexpr int kACols = kDfStageK / 2;                // 32-bit TMEM columns per A slot
   static constexpr int kTmemCols = 512;
-  static_assert(kStages >= 2, "pipeline depth");
+  static_assert(kCodeStages >= 2, "pipeline depth");
   static_assert(kCodeBytes % 1024 == 0 && kXBytes % 1024 == 0, "128-byte-swizzle boxes start 1 KB aligned");
   static_assert(2 * MP + kGroups * kACols <= kTmemCols, "TMEM columns");
+  static_assert(kXStages >= kGroups, "an item's completion barrier outlives its group's next item");
   static_assert(kSmemBytes <= kMaxSmem, "shared memory per CTA");
 };
 
@@ -155,16 +165,19 @@ template <int MP, int GM>
 __global__ void __launch_bounds__(DfCfg<MP>::kThreads, 1)
     nf4_decode_fwd_kernel(const __grid_constant__ FtMaps<GM> maps, const __grid_constant__ FtArgs<GM> p) {
   using Cfg = DfCfg<MP>;
-  constexpr int S = Cfg::kStages;
+  constexpr int SC = Cfg::kCodeStages;
+  constexpr int SX = Cfg::kXStages;
   constexpr int G = Cfg::kGroups;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t *lut = smem + S * Cfg::kStageBytes;
-  uint64_t *full_bar = reinterpret_cast<uint64_t *>(smem + S * Cfg::kStageBytes + kDfLutBytes);
-  uint64_t *empty_bar = full_bar + S;
-  uint64_t *afull_bar = empty_bar + S;                  // [G]
-  uint64_t *aempty_bar = afull_bar + G;                 // [G]
-  uint64_t *tfull_bar = aempty_bar + G;                 // [2]
+  uint8_t *xring = smem + SC * Cfg::kCodeBytes;
+  uint8_t *lut = xring + SX * Cfg::kXBytes;
+  uint64_t *cfull_bar = reinterpret_cast<uint64_t *>(lut + kDfLutBytes);   // [SC] codes landed
+  uint64_t *cempty_bar = cfull_bar + SC;                // [SC] codes copied out by the decoders
+  uint64_t *xfull_bar = cempty_bar + SC;                // [SX] X landed
+  uint64_t *idone_bar = xfull_bar + SX;                 // [SX] item rel's MMAs done (slot rel % SX)
+  uint64_t *afull_bar = idone_bar + SX;                 // [G]
+  uint64_t *tfull_bar = afull_bar + G;                  // [2]
   uint64_t *tempty_bar = tfull_bar + 2;                 // [2]
   uint64_t *done_bar = tempty_bar + 2;
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(done_bar + 1);
@@ -180,14 +193,15 @@ __global__ void __launch_bounds__(DfCfg<MP>::kThreads, 1)
     reinterpret_cast<float2 *>(lut)[i] = make_float2(p.levels[v & 15], p.levels[v >> 4]);
   }
   if (threadIdx.x == 0) {
-    for (int i = 0; i < S; ++i) {
-      mbar_init(smem_u32(full_bar + i), 1);                  // the TMA bytes
-      mbar_init(smem_u32(empty_bar + i), 4 + 1);             // the decoding group's warps + the MMAs on X
+    for (int i = 0; i < SC; ++i) {
+      mbar_init(smem_u32(cfull_bar + i), 1);                 // the TMA bytes
+      mbar_init(smem_u32(cempty_bar + i), 4);                // the four warps of the decoding group
     }
-    for (int i = 0; i < G; ++i) {
-      mbar_init(smem_u32(afull_bar + i), 4);                 // the four warps of a decoder group
-      mbar_init(smem_u32(aempty_bar + i), 1);
+    for (int i = 0; i < SX; ++i) {
+      mbar_init(smem_u32(xfull_bar + i), 1);                 // the TMA bytes
+      mbar_init(smem_u32(idone_bar + i), 1);                 // the MMAs' commit
     }
+    for (int i = 0; i < G; ++i) mbar_init(smem_u32(afull_bar + i), 4);   // the four warps of a decoder group
     for (int i = 0; i < 2; ++i) {
       mbar_init(smem_u32(tfull_bar + i), 1);
       mbar_init(smem_u32(tempty_bar + i), 4);
@@ -213,40 +227,44 @@ __global__ void __launch_bounds__(DfCfg<MP>::kThreads, 1)
       tma_prefetch_desc(&maps.codes[lane]);
       tma_prefetch_desc(&maps.x[lane]);
     }
-    int stage = 0;
-    uint32_t phase = 0, used = 0, last_parity = 0;
-    for (int it = i0; it < i1; ++it) {
-      int l, rt, ks;
-      ft_item<GM>(p, it, l, rt, ks);
-      const bool got = mbar_wait(smem_u32(empty_bar + stage), phase ^ 1, p.err, DEV_TIMEOUT_PRODUCER);
-      if (!__all_sync(0xFFFFFFFFu, got)) break;
-      const uint32_t fb = smem_u32(full_bar + stage);
-      const uint32_t sc = smem_u32(smem + stage * Cfg::kStageBytes);
-      if (lane == 0) {
-        mbar_arrive_expect_tx(fb, Cfg::kCodeBytes + Cfg::kXBytes);
-        tma_load_2d(sc, &maps.codes[l], fb, ks * (kDfStageK / 2), rt * kDfRows);
-        tma_load_3d(sc + Cfg::kCodeBytes, &maps.x[l], fb, 0, 0, ks * 4);
+    if (lane == 0) {
+      bool ok = true;
+      for (int it = i0; it < i1 && ok; ++it) {
+        const int rel = it - i0;
+        int l, rt, ks;
+        ft_item<GM>(p, it, l, rt, ks);
+        const int cs = rel % SC, xs = rel % SX;
+        if (!mbar_wait(smem_u32(cempty_bar + cs), ((uint32_t)(rel / SC) & 1u) ^ 1u, p.err, DEV_TIMEOUT_PRODUCER)) break;
+        const uint32_t cb = smem_u32(cfull_bar + cs);
+        mbar_arrive_expect_tx(cb, Cfg::kCodeBytes);
+        tma_load_2d(smem_u32(smem + cs * Cfg::kCodeBytes), &maps.codes[l], cb, ks * (kDfStageK / 2), rt * kDfRows);
+        // the X slot's previous item (rel - SX) has had its MMAs
+        if (!mbar_wait(smem_u32(idone_bar + xs), ((uint32_t)(rel / SX) & 1u) ^ 1u, p.err, DEV_TIMEOUT_PRODUCER)) {
+          ok = false;
+          break;
+        }
+        const uint32_t xb = smem_u32(xfull_bar + xs);
+        mbar_arrive_expect_tx(xb, Cfg::kXBytes);
+        tma_load_3d(smem_u32(xring + xs * Cfg::kXBytes), &maps.x[l], xb, 0, 0, ks * 4);
       }
-      used |= 1u << stage;
-      last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
-      if (++stage == S) {
-        stage = 0;
-        phase ^= 1;
-      }
+      // Drain: the copies of the last uses of every slot have landed.
+      const int n = i1 - i0;
+      for (int rel = n - SC > 0 ? n - SC : 0; rel < n; ++rel)
+        if (!mbar_wait(smem_u32(cfull_bar + rel % SC), (uint32_t)(rel / SC) & 1u, p.err, DEV_TIMEOUT_DRAIN)) break;
+      for (int rel = n - SX > 0 ? n - SX : 0; rel < n; ++rel)
+        if (!mbar_wait(smem_u32(xfull_bar + rel % SX), (uint32_t)(rel / SX) & 1u, p.err, DEV_TIMEOUT_DRAIN)) break;
     }
-    // Drain: lane 0's tensor copies have landed once the last phase of each
-    // used stage has completed.
-    for (int i = 0; i < S; ++i)
-      if (used & (1u << i)) {
-        const bool done = mbar_wait(smem_u32(full_bar + i), (last_parity >> i) & 1u, p.err, DEV_TIMEOUT_DRAIN);
-        if (!__all_sync(0xFFFFFFFFu, done)) break;
-      }
   } else if (warp == Cfg::kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
+    // Every synchronising operation of this thread between MMAs (an mbarrier
+    // wait, a tcgen05 fence, a commit) waits for the MMAs in flight, hundreds
+    // of cycles each at these sizes (measured), so an item costs it as few as
+    // possible: one wait (the decoder group signals its A slot only once the
+    // item's X tile has landed too), one fence and one commit.  Batching the
+    // items of both decoder groups under one wait was measured slower: with
+    // one TMEM slot per group, decoding then no longer overlaps the MMAs.
     if (lane == 0) {
       const uint32_t idesc = idesc_bf16_f32(kDfRows, MP, 0, 0);
-      int stage = 0;
-      uint32_t phase = 0;
       int t = 0;               // row-tile segments started
       uint32_t accumulate = 0;
       for (int it = i0; it < i1; ++it) {
@@ -255,27 +273,24 @@ __global__ void __launch_bounds__(DfCfg<MP>::kThreads, 1)
         const int rel = it - i0;
         const int g = rel % G;
         const uint32_t use = (uint32_t)(rel / G);     // this group's item count before this one
+        const int xs = rel % SX;
         const bool first = it == i0 || ks == 0;
         const bool last = it == i1 - 1 || ks == m.kstages - 1;
         const int acc = t & 1;
         if (first) {
           if (!mbar_wait(smem_u32(tempty_bar + acc), ((t >> 1) & 1u) ^ 1u, p.err, DEV_TIMEOUT_MMA)) break;
-          tc_fence_after();
           accumulate = 0;
         }
-        if (!mbar_wait(smem_u32(full_bar + stage), phase, p.err, DEV_TIMEOUT_MMA)) break;
         if (!mbar_wait(smem_u32(afull_bar + g), use & 1u, p.err, DEV_TIMEOUT_MMA)) break;
         tc_fence_after();
-        const uint32_t sx = smem_u32(smem + stage * Cfg::kStageBytes) + Cfg::kCodeBytes;
         const uint32_t d_tmem = tmem_base + (uint32_t)(acc * MP);
         const uint32_t a_tmem = tmem_base + (uint32_t)(2 * MP + g * Cfg::kACols);
         const int nk = 4 * min(4, (m.K >> 6) - ks * 4);   // 16-wide k-steps of the stage's real blocks
-        // The issuing thread is held for the duration of each MMA (tens of
-        // cycles at these sizes), so the k-step loop carries no arithmetic:
-        // k-step k reads A columns 8k and, as B, atom k / 4 of the stage's X
-        // (MP rows x 128 B) at byte 32 (k % 4) inside it -- a constant
-        // offset of the stage's descriptor (its address field counts 16 B).
-        const uint64_t b0 = smem_desc_sw128(sx, 16, 1024);
+        // k-step k reads A columns 8k and, as B, atom k / 4 of the item's X
+        // (MP rows x 128 B) at byte 32 (k % 4) inside it: a constant offset of
+        // the item's descriptor (its address field counts 16 B), so the loop
+        // carries no arithmetic.
+        const uint64_t b0 = smem_desc_sw128(smem_u32(xring + xs * Cfg::kXBytes), 16, 1024);
         if (nk == 16) {
           tc_mma_f16_ts(d_tmem, a_tmem, b0, idesc, accumulate);
 #pragma unroll
@@ -287,12 +302,8 @@ __global__ void __launch_bounds__(DfCfg<MP>::kThreads, 1)
                           k == 0 ? accumulate : 1u);
         }
         accumulate = 1;
-        tc_commit(smem_u32(aempty_bar + g));         // A slot free once these MMAs have read it
-        tc_commit(smem_u32(empty_bar + stage));      // X tile consumed
-        if (++stage == S) {
-          stage = 0;
-          phase ^= 1;
-        }
+        // the item's completion frees its X slot and its group's A slot
+        tc_commit(smem_u32(idone_bar + xs));
         if (last) {
           tc_commit(smem_u32(tfull_bar + acc));      // partial sums of this row tile ready
           ++t;
@@ -322,8 +333,7 @@ __global__ void __launch_bounds__(DfCfg<MP>::kThreads, 1)
     auto item = [&](int u, uint4 &raw) -> bool {
       const int it = i0 + g + u * G;
       const int rel = it - i0;
-      const int stage = rel % S;
-      const uint32_t phase = (uint32_t)(rel / S) & 1u;
+      const int cs = rel % SC;
       int l, rt, ks;
       const FtMember &m = ft_item<GM>(p, it, l, rt, ks);
       const int kblocks = m.K >> 6;
@@ -335,19 +345,33 @@ __global__ void __launch_bounds__(DfCfg<MP>::kThreads, 1)
       for (int j = 0; j < 4; ++j)
         c2[j] = f32x2_splat((j < nkb && n < m.N) ? ft_c2hat(raw, n, ks * 4, j, kblocks, mu) : 0.f);
       raw = raw_of(u + 2);
-      if (!__all_sync(0xFFFFFFFFu, mbar_wait(smem_u32(full_bar + stage), phase, p.err, DEV_TIMEOUT_MMA))) return false;
-      // the MMAs of this group's previous item have read its A slot
-      if (!__all_sync(0xFFFFFFFFu, mbar_wait(smem_u32(aempty_bar + g), ((uint32_t)u & 1u) ^ 1u, p.err, DEV_TIMEOUT_MMA)))
+      // the row's 128 code bytes into registers (16-byte chunks of its
+      // swizzled line), and the stage's codes slot back to the producer
+      if (!__all_sync(0xFFFFFFFFu, mbar_wait(smem_u32(cfull_bar + cs), (uint32_t)(rel / SC) & 1u, p.err,
+                                             DEV_TIMEOUT_MMA)))
         return false;
+      const uint32_t sc = smem_u32(smem + cs * Cfg::kCodeBytes) + t * 128;
+      uint4 qv[8];
+#pragma unroll
+      for (int c = 0; c < 8; ++c) qv[c] = lds128(sc + (((uint32_t)c << 4) ^ cswz));
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(cempty_bar + cs));
+      // the MMAs of this group's previous item (rel - G) have read its A
+      // slot.  The X ring has at least G slots, so that item's completion is
+      // the latest one the barrier can have seen: the next one on it needs
+      // this item's MMAs, which need this group's decode below.
+      if (rel >= G) {
+        const int prev = rel - G;
+        if (!__all_sync(0xFFFFFFFFu, mbar_wait(smem_u32(idone_bar + prev % SX), (uint32_t)(prev / SX) & 1u, p.err,
+                                               DEV_TIMEOUT_MMA)))
+          return false;
+      }
       tc_fence_after();
-      const uint32_t sc = smem_u32(smem + stage * Cfg::kStageBytes) + t * 128;
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         if (j >= nkb) break;
-        // this row's 32 code bytes of block j: 16-byte chunks 2j, 2j+1 of its swizzled 128-byte line
-        const uint4 qa = lds128(sc + (((uint32_t)(2 * j) << 4) ^ cswz));
-        const uint4 qb = lds128(sc + (((uint32_t)(2 * j + 1) << 4) ^ cswz));
-        const uint32_t q[8] = {qa.x, qa.y, qa.z, qa.w, qb.x, qb.y, qb.z, qb.w};
+        const uint32_t q[8] = {qv[2 * j].x, qv[2 * j].y, qv[2 * j].z, qv[2 * j].w,
+                               qv[2 * j + 1].x, qv[2 * j + 1].y, qv[2 * j + 1].z, qv[2 * j + 1].w};
         uint32_t e[32];
 #pragma unroll
         for (int w = 0; w < 8; ++w)
@@ -360,11 +384,13 @@ __global__ void __launch_bounds__(DfCfg<MP>::kThreads, 1)
       }
       tmem_wait_st();
       tc_fence_before();
+      // the item's X tile has landed too (the MMA issuer does not wait for it)
+      const int xs = rel % SX;
+      if (!__all_sync(0xFFFFFFFFu, mbar_wait(smem_u32(xfull_bar + xs), (uint32_t)(rel / SX) & 1u, p.err,
+                                             DEV_TIMEOUT_MMA)))
+        return false;
       __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(smem_u32(afull_bar + g));          // A slot written
-        mbar_arrive(smem_u32(empty_bar + stage));      // codes of this stage consumed
-      }
+      if (lane == 0) mbar_arrive(smem_u32(afull_bar + g));   // A slot written, X landed
       return true;
     };
     uint4 ra = raw_of(0), rb = raw_of(1);
