@@ -524,7 +524,7 @@ def _kernel_table(launches, steps):
 
 # Kernels behind one entry of the library's event log: the few-token forward
 # logs its chain (T accumulation, product, epilogue) as one entry.
-KERNELS_PER_ENTRY = {"gemv_fwd": 3, "fused_fwd": 3}
+KERNELS_PER_ENTRY = {"fused_fwd": 3}
 
 
 def _kernel_count(launches) -> int:
@@ -628,7 +628,7 @@ def run_decode(args, rank, world, local_rank):
         return None
     peaks, peak_src = load_peaks()
     per_kind, kernels = _kernel_table(launches, args.steps)
-    dom = per_kind.get("fused_fwd") or per_kind.get("gemv_fwd") or [0, 0.0]
+    dom = per_kind.get("fused_fwd") or [0, 0.0]
     achieved = nbytes * args.steps / (dom[1] * 1e-3) / 1e9 if dom[1] > 0 else None
     peak = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
     for v in variants.values():

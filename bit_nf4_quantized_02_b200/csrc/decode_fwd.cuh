@@ -10,7 +10,8 @@
 // dimension (TMEM lanes) and the tokens the MMA N dimension (MP = tokens
 // padded to 16, 32, 64 or 128).  The LoRA branch and the bf16 output come
 // from the kernels around it (lora_down_small_kernel before it, which it
-// overlaps as a programmatic dependent, and gemv_epilogue_kernel after).
+// overlaps as a programmatic dependent, and lora_epilogue_kernel after;
+// few_token.cuh).
 //
 // The decoded weight is exactly doubleDequant's bf16 weight (bit-identical to
 // qlora_dequant): W_hat = bf16(fp32(level[c] * c2_hat)) with c2_hat =
@@ -59,13 +60,12 @@
 // Work: the items are split into equal contiguous ranges, one per CTA; the
 // CTA adds its partial sums into acc whenever its range moves to the next
 // row tile, and at its end.  Groups of linears concatenate their items (see
-// the group note in gemv.cuh).
+// the group note in few_token.cuh).
 #pragma once
 
 #include "common.cuh"
 #include "quant.cuh"
-#include "gemv.cuh"
-#include "fused_fwd.cuh"
+#include "few_token.cuh"
 
 namespace qlora {
 
@@ -74,6 +74,76 @@ constexpr int kDfStageK = 256;                // K per stage: four 64-blocks
 constexpr int kDfLutEntries = 256;            // one per code byte (two codes)
 constexpr int kDfLutReplicas = 16;            // one per lane of a half-warp (8-byte loads)
 constexpr int kDfLutBytes = kDfLutEntries * kDfLutReplicas * 8;
+
+// One linear of a launch: its shape, block constants and accumulator.
+struct DfMember {
+  int N, K;
+  int kstages;           // ceil(K / 256)
+  DivU31 ks_div;         // division by kstages
+  const uint8_t *c2_fp8;
+  const float *c1;
+  const float *mu;
+  float *acc;            // [M x N] fp32, zero at launch
+};
+
+// A group of linears that see the same tokens: their (row tile, stage) items
+// are concatenated, linear after linear (see the group note in few_token.cuh).
+template <int GM>
+struct DfArgs {
+  int M;
+  int count;             // linears in the group
+  int items;             // row tiles x kstages, summed over the group
+  int beg[GM];           // first item of each linear
+  DfMember m[GM];
+  float levels[16];      // the 16-level code table (shared by the group)
+  int *err;
+};
+
+// Per linear: its packed codes in boxes of 128 rows x 128 bytes, and X as
+// [64-block][token][64] in boxes of the four atoms of a stage.
+template <int GM>
+struct DfMaps {
+  CUtensorMap codes[GM];
+  CUtensorMap x[GM];
+};
+
+// Item `it` of a group -> its linear l, row tile rt and stage ks.
+template <int GM>
+__device__ __forceinline__ const DfMember &df_item(const DfArgs<GM> &p, int it, int &l, int &rt, int &ks) {
+  l = group_member<GM>(p.beg, p.count, it);
+  const DfMember &m = p.m[l];
+  const int li = it - p.beg[l];
+  rt = (int)m.ks_div.div((uint32_t)li);
+  ks = li - rt * m.kstages;
+  return m;
+}
+
+// 32 lanes x 16 consecutive 32-bit columns.
+__device__ __forceinline__ void tmem_ld_32x32b_x16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr)
+      : "memory");
+}
+
+// The contiguous range of items [i0, i1) of CTA b among g.
+__device__ __forceinline__ void df_range(int items, int b, int g, int &i0, int &i1) {
+  i0 = (int)(((int64_t)items * b) / g);
+  i1 = (int)(((int64_t)items * (b + 1)) / g);
+}
+
+// c2_hat of block kb0 + j of weight row n from its raw constants (j < 4, the
+// block inside the weight).
+__device__ __forceinline__ float df_c2hat(uint4 raw, int n, int kb0, int j, int kblocks, float mu) {
+  const int64_t b0 = (int64_t)n * kblocks + kb0;
+  const int sh = (int)(b0 & 3) + j;                  // byte index in the 8-byte pair
+  const uint32_t code8 = (sh < 4 ? raw.x >> (8 * sh) : raw.y >> (8 * (sh - 4))) & 0xFFu;
+  const float c1 = ((b0 + j) >> 8) == (b0 >> 8) ? __uint_as_float(raw.z) : __uint_as_float(raw.w);
+  return __fmaf_rn(e4m3_to_f32((uint8_t)code8), c1, mu);
+}
 
 template <int MP>
 struct DfCfg {
@@ -129,11 +199,11 @@ __device__ __forceinline__ uint32_t mul_round_bf16x2(uint64_t p, uint64_t c) {
 }
 
 // Raw block constants of weight row n for stage ks, in registers, in the
-// layout ft_c2hat reads: the two aligned 32-bit words of c2_fp8 holding the
+// layout df_c2hat reads: the two aligned 32-bit words of c2_fp8 holding the
 // row's (up to) four E4M3 codes of the stage, then c1 of the first and of
 // the last of those blocks.  Words that reach past the end of c2_fp8 are
 // read byte by byte.  Rows past the weight read nothing.
-__device__ __forceinline__ uint4 df_load_raw(const FtMember &m, int n, int ks) {
+__device__ __forceinline__ uint4 df_load_raw(const DfMember &m, int n, int ks) {
   uint4 raw = make_uint4(0, 0, 0, 0);
   if (n >= m.N) return raw;
   const int kblocks = m.K >> 6;
@@ -163,7 +233,7 @@ __device__ __forceinline__ uint4 df_load_raw(const FtMember &m, int n, int ks) {
 
 template <int MP, int GM>
 __global__ void __launch_bounds__(DfCfg<MP>::kThreads, 1)
-    nf4_decode_fwd_kernel(const __grid_constant__ FtMaps<GM> maps, const __grid_constant__ FtArgs<GM> p) {
+    nf4_decode_fwd_kernel(const __grid_constant__ DfMaps<GM> maps, const __grid_constant__ DfArgs<GM> p) {
   using Cfg = DfCfg<MP>;
   constexpr int SC = Cfg::kCodeStages;
   constexpr int SX = Cfg::kXStages;
@@ -219,7 +289,7 @@ __global__ void __launch_bounds__(DfCfg<MP>::kThreads, 1)
   const uint32_t tmem_base = *tmem_slot;
 
   int i0, i1;
-  ft_range(p.items, blockIdx.x, gridDim.x, i0, i1);
+  df_range(p.items, blockIdx.x, gridDim.x, i0, i1);
 
   if (warp == Cfg::kProdWarp) {
     // ------------------------------------------------------------ producer
@@ -232,7 +302,7 @@ __global__ void __launch_bounds__(DfCfg<MP>::kThreads, 1)
       for (int it = i0; it < i1 && ok; ++it) {
         const int rel = it - i0;
         int l, rt, ks;
-        ft_item<GM>(p, it, l, rt, ks);
+        df_item<GM>(p, it, l, rt, ks);
         const int cs = rel % SC, xs = rel % SX;
         if (!mbar_wait(smem_u32(cempty_bar + cs), ((uint32_t)(rel / SC) & 1u) ^ 1u, p.err, DEV_TIMEOUT_PRODUCER)) break;
         const uint32_t cb = smem_u32(cfull_bar + cs);
@@ -269,7 +339,7 @@ __global__ void __launch_bounds__(DfCfg<MP>::kThreads, 1)
       uint32_t accumulate = 0;
       for (int it = i0; it < i1; ++it) {
         int l, rt, ks;
-        const FtMember &m = ft_item<GM>(p, it, l, rt, ks);
+        const DfMember &m = df_item<GM>(p, it, l, rt, ks);
         const int rel = it - i0;
         const int g = rel % G;
         const uint32_t use = (uint32_t)(rel / G);     // this group's item count before this one
@@ -325,7 +395,7 @@ __global__ void __launch_bounds__(DfCfg<MP>::kThreads, 1)
       const int it = i0 + g + u * G;
       if (it >= i1) return make_uint4(0, 0, 0, 0);
       int l, rt, ks;
-      const FtMember &m = ft_item<GM>(p, it, l, rt, ks);
+      const DfMember &m = df_item<GM>(p, it, l, rt, ks);
       return df_load_raw(m, rt * kDfRows + t, ks);
     };
     // Decode the group's item u with its constants `raw`, then start loading
@@ -335,7 +405,7 @@ __global__ void __launch_bounds__(DfCfg<MP>::kThreads, 1)
       const int rel = it - i0;
       const int cs = rel % SC;
       int l, rt, ks;
-      const FtMember &m = ft_item<GM>(p, it, l, rt, ks);
+      const DfMember &m = df_item<GM>(p, it, l, rt, ks);
       const int kblocks = m.K >> 6;
       const int nkb = min(4, kblocks - ks * 4);
       const int n = rt * kDfRows + t;
@@ -343,7 +413,7 @@ __global__ void __launch_bounds__(DfCfg<MP>::kThreads, 1)
       uint64_t c2[4];     // {c2_hat, c2_hat} of the stage's four blocks
 #pragma unroll
       for (int j = 0; j < 4; ++j)
-        c2[j] = f32x2_splat((j < nkb && n < m.N) ? ft_c2hat(raw, n, ks * 4, j, kblocks, mu) : 0.f);
+        c2[j] = f32x2_splat((j < nkb && n < m.N) ? df_c2hat(raw, n, ks * 4, j, kblocks, mu) : 0.f);
       raw = raw_of(u + 2);
       // the row's 128 code bytes into registers (16-byte chunks of its
       // swizzled line), and the stage's codes slot back to the producer
@@ -404,7 +474,7 @@ __global__ void __launch_bounds__(DfCfg<MP>::kThreads, 1)
     int t = 0;
     for (int it = i0; it < i1; ++it) {
       int l, rt, ks;
-      const FtMember &m = ft_item<GM>(p, it, l, rt, ks);
+      const DfMember &m = df_item<GM>(p, it, l, rt, ks);
       if (!(it == i1 - 1 || ks == m.kstages - 1)) continue;   // not the end of a row-tile segment
       const int acc = t & 1;
       const bool got = mbar_wait(smem_u32(tfull_bar + acc), (t >> 1) & 1u, p.err, DEV_TIMEOUT_EPILOGUE);

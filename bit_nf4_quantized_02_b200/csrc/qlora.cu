@@ -12,8 +12,7 @@
 #include "common.cuh"
 #include "quant.cuh"
 #include "tc_gemm.cuh"
-#include "gemv.cuh"
-#include "fused_fwd.cuh"
+#include "few_token.cuh"
 #include "decode_fwd.cuh"
 #include "dropout.cuh"
 #include "group.cuh"
@@ -50,9 +49,7 @@ struct DeviceInfo {
   int *err = nullptr;                    // device address of g_dev_err
   std::atomic<int> gemm_attr[16];        // [wide][fold][BN 64/128/256 or 3 = pair]: 1 once the smem limit is set
   std::atomic<int> pair_clusters[3];     // co-resident 2-CTA clusters of the pair GEMM [form]
-  std::atomic<int> gemv_per_sm[6];       // mma.sync few-token product: resident CTAs per SM [group form][NT]
-  std::atomic<int> fused_smem_set[8];    // tcgen05 few-token product: smem limit set [group form][token padding]
-  std::atomic<int> decode_smem_set[8];   // TMEM-decode few-token product: smem limit set [group form][token padding]
+  std::atomic<int> decode_smem_set[8];   // few-token product: smem limit set [group form][token padding]
 };
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_mu;
@@ -499,13 +496,13 @@ struct FwdMember {
 
 // Workspace of the few-token forward: per linear [acc M*N f32 | tacc M*r f32],
 // one linear after the other, all zeroed by one memset per call.
-struct GemvLayout {
+struct FewLayout {
   size_t acc[kMaxGroup], tacc[kMaxGroup];
   size_t zero_bytes, total;
 };
 
-GemvLayout gemv_layout(int64_t M, const FwdMember *mem, int count) {
-  GemvLayout L;
+FewLayout few_layout(int64_t M, const FwdMember *mem, int count) {
+  FewLayout L;
   size_t off = 0;
   for (int i = 0; i < count; ++i) {
     L.acc[i] = align_up(off, 16);
@@ -517,7 +514,7 @@ GemvLayout gemv_layout(int64_t M, const FwdMember *mem, int count) {
   return L;
 }
 
-size_t gemv_ws_bytes(int64_t M, int64_t N, int r) {
+size_t few_ws_bytes(int64_t M, int64_t N, int r) {
   qlora_nf4dq_t w;
   std::memset(&w, 0, sizeof(w));
   w.n_out = N;
@@ -525,13 +522,13 @@ size_t gemv_ws_bytes(int64_t M, int64_t N, int r) {
   std::memset(&m, 0, sizeof(m));
   m.W = &w;
   m.r = r;
-  return gemv_layout(M, &m, 1).total;
+  return few_layout(M, &m, 1).total;
 }
 
 // T accumulation of every linear of the group (a plain launch: it follows all
 // earlier work in the stream).
 template <int GM>
-int launch_lora_down(const FwdMember *mem, int count, int64_t M, const GemvLayout &L, uint8_t *ws, cudaStream_t st) {
+int launch_lora_down(const FwdMember *mem, int count, int64_t M, const FewLayout &L, uint8_t *ws, cudaStream_t st) {
   TdArgs<GM> a;
   std::memset(&a, 0, sizeof(a));
   a.M = (int)M;
@@ -555,7 +552,7 @@ int launch_lora_down(const FwdMember *mem, int count, int64_t M, const GemvLayou
 // Y = bf16(acc + s T L2) and the T hi/lo pair of every linear of the group,
 // as a programmatic dependent of the product kernel just launched.
 template <int GM>
-int launch_lora_epilogue(const FwdMember *mem, int count, int64_t M, const GemvLayout &L, uint8_t *ws,
+int launch_lora_epilogue(const FwdMember *mem, int count, int64_t M, const FewLayout &L, uint8_t *ws,
                          cudaStream_t st) {
   EpArgs<GM> a;
   std::memset(&a, 0, sizeof(a));
@@ -577,78 +574,11 @@ int launch_lora_epilogue(const FwdMember *mem, int count, int64_t M, const GemvL
     rmax = std::max(rmax, mem[i].r);
   }
   const size_t esmem = (size_t)kTokChunk * rmax * 4 + (size_t)rmax * 64 * 2;
-  if (esmem > 48 * 1024 && cudaFuncSetAttribute(gemv_epilogue_kernel<GM>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  if (esmem > 48 * 1024 && cudaFuncSetAttribute(lora_epilogue_kernel<GM>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                 (int)esmem) != cudaSuccess)
     return QLORA_ERR_CUDA;
   const dim3 grid((unsigned)slices, (unsigned)((M + kTokChunk - 1) / kTokChunk));
-  return launch_pdl(gemv_epilogue_kernel<GM>, grid, dim3(256), esmem, st, a);
-}
-
-// Fused doubleDequant + tcgen05 forward for M <= 128 tokens (MP = padded M)
-// of a group of linears sharing one code table: T accumulation, then the
-// product (a programmatic dependent of it), then the LoRA epilogue.  The
-// accumulators are zero (the caller's memset).
-template <int MP, int GM>
-int launch_fused_fwd(const FwdMember *mem, int count, int64_t M, const GemvLayout &L, uint8_t *ws, DeviceInfo *dev,
-                     cudaStream_t st) {
-  using Cfg = FtCfg<MP>;
-  FtMaps<GM> maps;
-  FtArgs<GM> a;
-  std::memset(&maps, 0, sizeof(maps));
-  std::memset(&a, 0, sizeof(a));
-  std::memcpy(a.levels, kLevelsHost[mem[0].W->table], sizeof(a.levels));
-  a.M = (int)M;
-  a.count = count;
-  a.err = dev->err;
-  int items = 0;
-  for (int i = 0; i < count; ++i) {
-    const qlora_nf4dq_t *W = mem[i].W;
-    const int64_t N = W->n_out, K = W->k_in;
-    {
-      const cuuint64_t dims[2] = {(cuuint64_t)(K / 2), (cuuint64_t)N};
-      const cuuint64_t strides[1] = {(cuuint64_t)(K / 2)};
-      const cuuint32_t box[2] = {128, (cuuint32_t)kFtRows};
-      int rc = encode_tmap(&maps.codes[i], CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, W->codes, dims, strides, box);
-      if (rc) return rc;
-    }
-    {
-      // X as [64-block][token][64]: one box = the four K-major atoms of a stage
-      const cuuint64_t dims[3] = {64, (cuuint64_t)M, (cuuint64_t)(K / 64)};
-      const cuuint64_t strides[2] = {(cuuint64_t)K * 2, 128};
-      const cuuint32_t box[3] = {64, (cuuint32_t)MP, 4};
-      int rc = encode_tmap(&maps.x[i], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, mem[i].X, dims, strides, box);
-      if (rc) return rc;
-    }
-    FtMember &m = a.m[i];
-    m.N = (int)N;
-    m.K = (int)K;
-    m.kstages = (int)((K + kFtStageK - 1) / kFtStageK);
-    m.ks_div = make_div_u31((uint32_t)m.kstages);
-    m.c2_fp8 = W->c2_fp8;
-    m.c1 = W->c1;
-    m.mu = W->c2_mean;
-    m.acc = reinterpret_cast<float *>(ws + L.acc[i]);
-    a.beg[i] = items;
-    items += (int)((N + kFtRows - 1) / kFtRows) * m.kstages;
-  }
-  a.items = items;
-  const int idx = (GM > 1 ? 4 : 0) + (MP == 16 ? 0 : (MP == 32 ? 1 : (MP == 64 ? 2 : 3)));
-  if (once(dev->fused_smem_set[idx], [&] {
-        return cudaFuncSetAttribute(nf4_fused_fwd_kernel<MP, GM>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    Cfg::kSmemBytes) == cudaSuccess
-                   ? 1
-                   : 0;
-      }) <= 0)
-    return QLORA_ERR_CUDA;
-  const int grid = std::max(1, std::min(a.items, dev->sms));
-  ProfScope prof(QLORA_KERNEL_FUSED_FWD, st);
-  // 1. T accumulation; 2. the fused product, overlapping it; 3. the LoRA epilogue.
-  int rc = launch_lora_down<GM>(mem, count, M, L, ws, st);
-  if (rc) return rc;
-  rc = launch_pdl(nf4_fused_fwd_kernel<MP, GM>, dim3(grid), dim3(Cfg::kThreads), (size_t)Cfg::kSmemBytes, st, maps,
-                  a);
-  if (rc) return rc;
-  return launch_lora_epilogue<GM>(mem, count, M, L, ws, st);
+  return launch_pdl(lora_epilogue_kernel<GM>, grid, dim3(256), esmem, st, a);
 }
 
 // Fused doubleDequant + tcgen05 forward with the weight decoded into TMEM,
@@ -656,11 +586,11 @@ int launch_fused_fwd(const FwdMember *mem, int count, int64_t M, const GemvLayou
 // accumulation, the product (a programmatic dependent of it), then the LoRA
 // epilogue.  The accumulators are zero (the caller's memset).
 template <int MP, int GM>
-int launch_decode_fwd(const FwdMember *mem, int count, int64_t M, const GemvLayout &L, uint8_t *ws, DeviceInfo *dev,
+int launch_decode_fwd(const FwdMember *mem, int count, int64_t M, const FewLayout &L, uint8_t *ws, DeviceInfo *dev,
                       cudaStream_t st) {
   using Cfg = DfCfg<MP>;
-  FtMaps<GM> maps;
-  FtArgs<GM> a;
+  DfMaps<GM> maps;
+  DfArgs<GM> a;
   std::memset(&maps, 0, sizeof(maps));
   std::memset(&a, 0, sizeof(a));
   std::memcpy(a.levels, kLevelsHost[mem[0].W->table], sizeof(a.levels));
@@ -686,7 +616,7 @@ int launch_decode_fwd(const FwdMember *mem, int count, int64_t M, const GemvLayo
       int rc = encode_tmap(&maps.x[i], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, mem[i].X, dims, strides, box);
       if (rc) return rc;
     }
-    FtMember &m = a.m[i];
+    DfMember &m = a.m[i];
     m.N = (int)N;
     m.K = (int)K;
     m.kstages = (int)((K + kDfStageK - 1) / kDfStageK);
@@ -718,79 +648,13 @@ int launch_decode_fwd(const FwdMember *mem, int count, int64_t M, const GemvLayo
   return launch_lora_epilogue<GM>(mem, count, M, L, ws, st);
 }
 
-// Fused doubleDequant + mma.sync forward for M <= 8 NT tokens of a group of
-// linears sharing one code table (three launches, as launch_fused_fwd).
-template <int NT, int GM>
-int launch_gemv(const FwdMember *mem, int count, int64_t M, const GemvLayout &L, uint8_t *ws, DeviceInfo *dev,
-                cudaStream_t st) {
-  using Cfg = GvCfg<NT>;
-  GvMaps<GM> maps;
-  GvArgs<GM> a;
-  std::memset(&maps, 0, sizeof(maps));
-  std::memset(&a, 0, sizeof(a));
-  std::memcpy(a.levels, kLevelsHost[mem[0].W->table], sizeof(a.levels));
-  a.M = (int)M;
-  a.count = count;
-  a.err = dev->err;
-  int units = 0;
-  for (int i = 0; i < count; ++i) {
-    const qlora_nf4dq_t *W = mem[i].W;
-    const int64_t N = W->n_out, K = W->k_in;
-    {
-      const cuuint64_t dims[2] = {(cuuint64_t)(K / 2), (cuuint64_t)N};
-      const cuuint64_t strides[1] = {(cuuint64_t)(K / 2)};
-      const cuuint32_t box[2] = {128, (cuuint32_t)kGvRows};
-      int rc = encode_tmap(&maps.codes[i], CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, W->codes, dims, strides, box);
-      if (rc) return rc;
-    }
-    {
-      const cuuint64_t dims[3] = {64, (cuuint64_t)(K / 64), (cuuint64_t)M};
-      const cuuint64_t strides[2] = {128, (cuuint64_t)K * 2};
-      const cuuint32_t box[3] = {64, 4, (cuuint32_t)(8 * NT)};
-      int rc = encode_tmap(&maps.x[i], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, mem[i].X, dims, strides, box);
-      if (rc) return rc;
-    }
-    GvMember &m = a.m[i];
-    m.N = (int)N;
-    m.K = (int)K;
-    m.nks = (int)((K + kGvUnitK - 1) / kGvUnitK);
-    m.nks_div = make_div_u31((uint32_t)m.nks);
-    m.c2_fp8 = W->c2_fp8;
-    m.c1 = W->c1;
-    m.mu = W->c2_mean;
-    m.acc = reinterpret_cast<float *>(ws + L.acc[i]);
-    a.beg[i] = units;
-    units += (int)((N + kGvRows - 1) / kGvRows) * m.nks;
-  }
-  a.units = units;
-  const int smem = Cfg::kSmemBytes;
-  const int idx = (GM > 1 ? 3 : 0) + (NT == 1 ? 0 : (NT == 2 ? 1 : 2));
-  const int per_sm = once(dev->gemv_per_sm[idx], [&] {
-    int n = 0;
-    if (cudaFuncSetAttribute(gemv_fwd_kernel<NT, GM>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
-            cudaSuccess ||
-        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, gemv_fwd_kernel<NT, GM>, kGvThreads, smem) != cudaSuccess)
-      return 0;
-    return n;
-  });
-  if (per_sm <= 0) return QLORA_ERR_CUDA;
-  const int grid = std::max(1, std::min(a.units, per_sm * dev->sms));
-  ProfScope prof(QLORA_KERNEL_GEMV_FWD, st);
-  // 1. T accumulation; 2. the product, overlapping it; 3. the LoRA epilogue.
-  int rc = launch_lora_down<GM>(mem, count, M, L, ws, st);
-  if (rc) return rc;
-  rc = launch_pdl(gemv_fwd_kernel<NT, GM>, dim3(grid), dim3(kGvThreads), (size_t)smem, st, maps, a);
-  if (rc) return rc;
-  return launch_lora_epilogue<GM>(mem, count, M, L, ws, st);
-}
-
 // The few-token forward of `count` linears sharing one code table, on a
 // zeroed workspace: the path by token count.
 template <int GM>
-int few_token_fwd(const FwdMember *mem, int count, int64_t M, const GemvLayout &L, uint8_t *ws, DeviceInfo *dev,
+int few_token_fwd(const FwdMember *mem, int count, int64_t M, const FewLayout &L, uint8_t *ws, DeviceInfo *dev,
                   cudaStream_t st) {
-  // up to 32 tokens: weight decoded straight into mma.sync fragments (each
-  // warp independent); 33..128: decoded into shared memory for tcgen05
+  // the weight decoded into TMEM for tcgen05 MMAs with N = tokens padded to
+  // 16, 32, 64 or 128
   if (M <= 16) return launch_decode_fwd<16, GM>(mem, count, M, L, ws, dev, st);
   if (M <= 32) return launch_decode_fwd<32, GM>(mem, count, M, L, ws, dev, st);
   if (M <= 64) return launch_decode_fwd<64, GM>(mem, count, M, L, ws, dev, st);
@@ -1202,7 +1066,7 @@ extern "C" {
 
 size_t qlora_linear_fwd_workspace_size(int64_t M, int64_t n_out, int64_t k_in, int r) {
   if (M < 0 || n_out <= 0 || k_in <= 0 || r <= 0) return 0;
-  if (M <= kFtMaxM) return gemv_ws_bytes(M, n_out, r);
+  if (M <= kFewMaxM) return few_ws_bytes(M, n_out, r);
   DeviceInfo *dev;
   const int sms = current_device_info(&dev) == QLORA_OK ? dev->sms : 148;
   return fwd_layout(M, n_out, k_in, r, sms).total;
@@ -1228,10 +1092,10 @@ int qlora_linear_fwd(const uint16_t *X, int64_t M, const qlora_nf4dq_t *W, const
   if (rc) return rc;
   const int64_t N = W->n_out, K = W->k_in;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  if (M <= kFtMaxM) {
+  if (M <= kFewMaxM) {
     // Few tokens: the weight bytes dominate; one fused decode + product pass.
     const FwdMember mem = {W, X, L1, L2, r, s, Y, T_save};
-    const GemvLayout L = gemv_layout(M, &mem, 1);
+    const FewLayout L = few_layout(M, &mem, 1);
     if (!ws || ws_bytes < L.total) return QLORA_ERR_WORKSPACE;
     if (!aligned(ws, 256)) return QLORA_ERR_MISALIGNED;
     uint8_t *w8 = reinterpret_cast<uint8_t *>(ws);
@@ -1415,7 +1279,7 @@ size_t qlora_linear_fwd_group_workspace_size(const qlora_fwd_member_t *members, 
     if (!members[i].W || members[i].W->n_out <= 0 || members[i].W->k_in <= 0 || members[i].r <= 0) return 0;
   FwdMember mem[kMaxGroup];
   fwd_members(members, count, mem);
-  if (M <= kFtMaxM) return gemv_layout(M, mem, count).total;
+  if (M <= kFewMaxM) return few_layout(M, mem, count).total;
   DeviceInfo *dev;
   const int sms = current_device_info(&dev) == QLORA_OK ? dev->sms : 148;
   return group_large_layout(M, mem, count, sms).total;
@@ -1432,15 +1296,15 @@ int qlora_linear_fwd_group(const qlora_fwd_member_t *members, int count, int64_t
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   FwdMember mem[kMaxGroup];
   fwd_members(members, count, mem);
-  if (M <= kFtMaxM) {
-    const GemvLayout L = gemv_layout(M, mem, count);
+  if (M <= kFewMaxM) {
+    const FewLayout L = few_layout(M, mem, count);
     if (!ws || ws_bytes < L.total) return QLORA_ERR_WORKSPACE;
     if (!aligned(ws, 256)) return QLORA_ERR_MISALIGNED;
     uint8_t *w8 = reinterpret_cast<uint8_t *>(ws);
     if (cudaMemsetAsync(w8, 0, L.zero_bytes, st) != cudaSuccess) return QLORA_ERR_CUDA;
     for (int t = 0; t < kNumTables; ++t) {
       FwdMember sub[kMaxGroup];
-      GemvLayout SL = L;
+      FewLayout SL = L;
       int n = 0;
       for (int i = 0; i < count; ++i)
         if (mem[i].W->table == t) {

@@ -347,8 +347,7 @@ QLORA_API int qlora_get_last_device_error(void *stream);
 #define QLORA_KERNEL_GEMM_DL1 15    /* dL1 = X^T G */
 #define QLORA_KERNEL_GEMM_Z 16      /* Z = G L1^T (dropout backward) */
 #define QLORA_KERNEL_SPLITK_FINALIZE 20
-#define QLORA_KERNEL_GEMV_FWD 30    /* fused decode + mma.sync product, up to 32 tokens */
-#define QLORA_KERNEL_FUSED_FWD 31   /* fused decode + tcgen05 product, up to 128 tokens */
+#define QLORA_KERNEL_FUSED_FWD 31   /* few-token forward chain (up to 128 tokens): T, fused decode + tcgen05 product, LoRA epilogue */
 #define QLORA_KERNEL_DROPOUT_MASK 40 /* Xm = X * m (LoRA dropout) */
 #define QLORA_KERNEL_T_SCATTER 41   /* shared-input T split into each linear's hi/lo pair (grouped forward) */
 QLORA_API int qlora_profile_start(int capacity);

@@ -1,12 +1,12 @@
 // Host check of the launch-time divisor constants of the few-token product
-// kernels (make_div_u31 in gemv.cuh): for every divisor tested, the
+// kernels (make_div_u31 in few_token.cuh): for every divisor tested, the
 // multiply-high-and-shift quotient equals n / d for numerators across
 // [0, 2^31).  Built and run by tests/test_host_div.py; needs no GPU.
 #include <cstdint>
 #include <cstdio>
 #include <random>
 
-#include "gemv.cuh"
+#include "few_token.cuh"
 
 static uint32_t quotient(const qlora::DivU31 &v, uint32_t n) {
   // the device form: __umulhi(n, mul) >> shr, with mul = 0 meaning d = 1

@@ -68,7 +68,7 @@ def _weights(N, K, seed):
 
 @pytest.mark.parametrize("M", [8, 16, 24, 48, 100, 200])
 def test_fp4_linear_forward_every_path(M):
-    """1-32 tokens (mma.sync decode), 33-128 (tcgen05 fused decode), above (dequant + GEMM)."""
+    """1-128 tokens (weight decoded into TMEM for tcgen05), above (dequant + GEMM)."""
     N, K, r, s = 256, 512, 16, 1.0
     g = inputs.rng(900 + M)
     W = _weights(N, K, 901 + M)

@@ -1,5 +1,5 @@
 """The launch-time divisor constants of the few-token product kernels
-(Granlund-Montgomery multiply-high and shift, make_div_u31 in gemv.cuh)
+(Granlund-Montgomery multiply-high and shift, make_div_u31 in few_token.cuh)
 against exact integer division, on the host: a small program built with nvcc
 from the library's own header (no GPU needed)."""
 
