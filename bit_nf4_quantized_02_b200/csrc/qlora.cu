@@ -50,6 +50,7 @@ struct DeviceInfo {
   std::atomic<int> gemm_attr[16];        // [wide][fold][BN 64/128/256 or 3 = pair]: 1 once the smem limit is set
   std::atomic<int> pair_clusters[3];     // co-resident 2-CTA clusters of the pair GEMM [form]
   std::atomic<int> decode_smem_set[8];   // few-token product: smem limit set [group form][token padding]
+  std::atomic<int> quant_smem_set[2];    // quantizer: smem limit set [bf16, fp32 input]
 };
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_mu;
@@ -838,18 +839,30 @@ size_t qlora_quantize_workspace_size(int64_t numel) {
 static int quantize_launch(const void *W, int w_dtype, int64_t numel, int table, uint8_t *codes, uint8_t *c2_fp8,
                            float *c1, float *c2_mean, float *c2, double *partial, DeviceInfo *dev, cudaStream_t st) {
   const int64_t nblk = (numel + 63) / 64;
-  const int64_t ngroups = numel >> 9;   // 512-element groups, one per warp iteration
-  const int grid1 = (int)std::max<int64_t>(
-      1, std::min<int64_t>((ngroups + 7) / 8, std::min(kQuantMaxCtas, dev->sms * kQuantCtasPerSm)));
+  // one persistent CTA per SM, each streaming whole chunks (fewer CTAs for a
+  // small tensor; the groups after the last whole chunk go to the last CTA)
+  const int64_t nchunks = numel / kQuantChunk;
+  const int grid1 = (int)std::max<int64_t>(1, std::min<int64_t>(nchunks, std::min(kQuantMaxCtas, dev->sms)));
+  const bool f32 = w_dtype == QLORA_DTYPE_F32;
+  const int smem = f32 ? QuantCfg<float>::kSmemBytes : QuantCfg<__nv_bfloat16>::kSmemBytes;
+  if (once(dev->quant_smem_set[f32 ? 1 : 0], [&] {
+        return (f32 ? cudaFuncSetAttribute(nf4_quantize_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           smem)
+                    : cudaFuncSetAttribute(nf4_quantize_kernel<__nv_bfloat16>,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) == cudaSuccess
+                   ? 1
+                   : 0;
+      }) <= 0)
+    return QLORA_ERR_CUDA;
   int rc;
   {
     ProfScope prof(QLORA_KERNEL_QUANTIZE, st);
-    if (w_dtype == QLORA_DTYPE_F32)
-      rc = launch_pdl(nf4_quantize_kernel<float>, dim3(grid1), dim3(kQuantThreads), 0, st,
-                      reinterpret_cast<const float *>(W), numel, codes, c2, partial, table);
+    if (f32)
+      rc = launch_pdl(nf4_quantize_kernel<float>, dim3(grid1), dim3(kQuantThreads), (size_t)smem, st,
+                      reinterpret_cast<const float *>(W), numel, codes, c2, partial, table, dev->err);
     else
-      rc = launch_pdl(nf4_quantize_kernel<__nv_bfloat16>, dim3(grid1), dim3(kQuantThreads), 0, st,
-                      reinterpret_cast<const __nv_bfloat16 *>(W), numel, codes, c2, partial, table);
+      rc = launch_pdl(nf4_quantize_kernel<__nv_bfloat16>, dim3(grid1), dim3(kQuantThreads), (size_t)smem, st,
+                      reinterpret_cast<const __nv_bfloat16 *>(W), numel, codes, c2, partial, table, dev->err);
   }
   if (rc) return rc;
   const int64_t nb256 = (nblk + 255) / 256;

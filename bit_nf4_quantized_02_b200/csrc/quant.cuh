@@ -55,9 +55,11 @@ __constant__ float kLevels[kNumTables][16] = {QLORA_LEVEL_TABLES};
 static const float kLevelsHost[kNumTables][16] = {QLORA_LEVEL_TABLES};
 #undef QLORA_LEVEL_TABLES
 
-constexpr int kQuantThreads = 256;
-constexpr int kQuantCtasPerSm = 5;     // resident at 48 registers per thread
-constexpr int kQuantMaxCtas = 148 * 8;
+constexpr int kQuantComputeWarps = 28;                       // warps that quantize groups
+constexpr int kQuantThreads = 32 * (kQuantComputeWarps + 1);  // + one producer warp
+constexpr int kQuantMaxCtas = 148 * 8;                        // bound on the partial sums (one per CTA)
+constexpr int kQuantChunk = 8192;                             // weights per bulk copy: 16 groups of 512
+constexpr int kQuantRingBytes = 160 * 1024;
 
 // Decision thresholds for the nearest-level search.  Level j+1 beats level j
 // exactly when x exceeds their midpoint m_j = (q_j + q_{j+1}) / 2, which is
@@ -87,14 +89,17 @@ struct NF4Thresholds {
 
 // Exact nearest-level codes without a division for almost every weight.
 // [-1, 1] is cut into kCodeBins bins of width 2^-13; bin(x) = floor((x + 1) *
-// kCodeBins / 2).  A bin with no decision threshold within two bins of it has
-// one code for every x in those five bins, so any estimate of
-// x = fp32(w / absmax) that is within one bin of x and lands in it (the
-// estimate w * (1/absmax) is within a few ulps, far below a bin) gives the
-// exact code.  The bins near a threshold (5 per threshold, 0.46% of them) hold
-// kCodeBoundary | j, j the index of that threshold (thresholds are hundreds of
-// bins apart, so there is one), and their weights take the exact division:
-// the code is then j + (x > t_j).
+// kCodeBins / 2).  The estimate of x = fp32(w / absmax) is e = w * sc with sc
+// = RN(1/absmax) * kCodeBins/2, taken with one fused multiply-add (below):
+// both sc and x carry one rounding of relative size <= 2^-24 and |w / absmax|
+// <= 1, so e differs from x * kCodeBins/2 by at most 2 * 8192 * 2^-24 = 2^-10
+// of a bin, and the estimated bin is bin(x) - 1, bin(x) or bin(x) + 1.  So a
+// bin b with no decision threshold in bins b - 1 .. b + 1 (kCodeMargin = 1)
+// holds the one code of every x that can land in it, and is exact.  The bins
+// next to a threshold (3 per threshold, 0.27% of them) hold kCodeBoundary |
+// j, j the index of that threshold (thresholds are at least 342 bins apart,
+// so there is one), and their weights take the exact division: the code is
+// then j + (x > t_j).
 //
 // The table is indexed by b + 1, b the estimated bin, so that the two
 // rounding overshoots b = -1 and b = kCodeBins (x within an ulp of -1 or 1)
@@ -104,21 +109,22 @@ struct NF4Thresholds {
 // included) can index outside it.
 constexpr int kCodeBins = 16384;
 constexpr int kCodeLutEntries = kCodeBins + 2;
+constexpr int kCodeMargin = 1;        // bins either side of a threshold's bin that are marked
 
 // Each CTA builds the table in its shared memory from the same thresholds
 // the exact path uses, before it waits for the kernel ahead of it (so the
 // build overlaps that kernel's tail).  Entry i holds, for the bin b =
 // min(max(i - 1, 0), kCodeBins - 1), either kCodeBoundary | j when the
 // boundary bin tb_j = floor((t_j + 1) * kCodeBins / 2) of threshold j lies
-// within two bins of b, or else the code #{j : tb_j < b}.  Entries from
-// kCodeLutBytes on are zero.
+// within kCodeMargin bins of b, or else the code #{j : tb_j < b}.  Entries
+// from kCodeLutBytes on are zero.
 //
 // A warp fills 32 consecutive words (128 entries, lane l word l) per pass.
 // Consecutive thresholds are hundreds of bins apart, so at most one threshold
-// lies within two bins of the 128 entries of a pass: the warp counts the thresholds below its first bin
-// minus two with one ballot, and a lane whose four bins are clear of the
-// next threshold stores that count four times; the few lanes near a
-// threshold resolve their four entries one by one.
+// lies within kCodeMargin bins of the 128 entries of a pass: the warp counts
+// the thresholds below its first bin minus the margin with one ballot, and a
+// lane whose four bins are clear of the next threshold stores that count four
+// times; the few lanes near a threshold resolve their four entries one by one.
 constexpr int kCodeLutBytes = (kCodeLutEntries + 3) / 4 * 4;
 constexpr int kCodeLutSpan = 32768;
 constexpr uint32_t kCodeBoundary = 0x80;
@@ -139,23 +145,23 @@ __device__ __forceinline__ void build_code_lut(uint8_t *lut, int table, int *tb_
   for (int w0 = (threadIdx.x & ~31); w0 < kCodeLutSpan / 4; w0 += blockDim.x) {
     const int w = w0 + lane;
     const int first_bin = max(4 * w0 - 1, 0);
-    // thresholds more than two bins below the warp's first bin
-    const int c = __popc(__ballot_sync(0xFFFFFFFFu, my_tb < first_bin - 2));
+    // thresholds more than kCodeMargin bins below the warp's first bin
+    const int c = __popc(__ballot_sync(0xFFFFFFFFu, my_tb < first_bin - kCodeMargin));
     uint32_t v = 0;
     if (4 * w < kCodeLutBytes) {
       const int bhi = min(4 * w + 2, kCodeBins - 1);
       const int tc = tb_s[c];
-      if (tc > bhi + 2) {
+      if (tc > bhi + kCodeMargin) {
         v = (uint32_t)c * 0x01010101u;
       } else {
         const int tn = tb_s[min(c + 1, 15)];
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
           const int b = min(max(4 * w + k - 1, 0), kCodeBins - 1);
-          const bool past = tc < b - 2;             // threshold c is behind this bin
-          const int j = c + (past ? 1 : 0);         // first threshold >= b - 2
+          const bool past = tc < b - kCodeMargin;   // threshold c is behind this bin
+          const int j = c + (past ? 1 : 0);         // first threshold >= b - kCodeMargin
           const int tj = past ? tn : tc;
-          const uint32_t e = tj <= b + 2 ? (kCodeBoundary | (uint32_t)j) : (uint32_t)(j + (tj < b ? 1 : 0));
+          const uint32_t e = tj <= b + kCodeMargin ? (kCodeBoundary | (uint32_t)j) : (uint32_t)(j + (tj < b ? 1 : 0));
           v |= e << (8 * k);
         }
       }
@@ -234,6 +240,19 @@ struct Raw16<__nv_bfloat16> {
   }
 };
 
+// Element i (0..15, a run-time index) of the sixteen unpacked weights, by a
+// select tree: the fix-up below reads it from registers instead of
+// reloading it from global memory.
+__device__ __forceinline__ float select16(const float (&v)[16], int i) {
+  float a[8], b[4];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) a[k] = (i & 1) ? v[2 * k + 1] : v[2 * k];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) b[k] = (i & 2) ? a[2 * k + 1] : a[2 * k];
+  const float c0 = (i & 4) ? b[1] : b[0], c1 = (i & 4) ? b[3] : b[2];
+  return (i & 8) ? c1 : c0;
+}
+
 __device__ __forceinline__ float load1(const float *p) { return ld_dep_f32(p); }
 __device__ __forceinline__ float load1(const __nv_bfloat16 *p) { return __uint_as_float(ld_dep_u16(p) << 16); }
 
@@ -253,107 +272,229 @@ __device__ __forceinline__ double cta_sum_f64(double v, double *scratch) {
 // K1: per 64-block absmax c2, nearest-level codes, nibble packing, and one
 // fp64 partial sum of c2 per CTA (for the Double-Quantization mean).
 //
-// A warp processes groups of eight 64-blocks (512 elements): lane l owns
-// elements [16l, 16l+16) of the group, i.e. 4 lanes per block; the block
-// absmax is reduced over those 4 lanes.  The (at most eight) blocks after the
-// last full group are handled by the last CTA, one warp per block.
+// Work is in groups of eight 64-blocks (512 weights): a warp quantizes a
+// group with lane l owning weights [16 l, 16 l + 16), i.e. 4 lanes per block,
+// the block absmax reduced over those 4 lanes.
+//
+// One persistent CTA per SM.  The weights stream through shared memory: one
+// producer thread keeps a ring of chunks (16 groups, 8192 weights) in flight
+// with bulk copies (cp.async.bulk, completing on the slot's mbarrier) -- about
+// 160 KB per SM, enough to keep HBM busy; loading each group into the
+// registers of the warp that quantizes it left too few bytes in flight.  The
+// 28 compute warps take the CTA's groups in turn (warp w: its groups w, w +
+// 28, ...), and a slot goes back to the producer once its 16 groups are done.
+// The groups after the last whole chunk are quantized by the last CTA from
+// global memory, and so are the (at most eight) blocks after the last whole
+// group, one warp per block.
 constexpr float kTinyAbsmax = 1e-30f;   // below this 1/absmax may overflow: exact division
 
+// Quantize one group's sixteen weights of this lane (v), whose 64-block has
+// the absmax `amax` (already reduced over the block's four lanes): two words
+// of packed nibble codes.
+__device__ __forceinline__ void quant_lane16(const float (&v)[16], float amax, const uint8_t *lut, const float *thr,
+                                             const NF4Thresholds &th, uint32_t &pk0, uint32_t &pk1) {
+  pk0 = pk1 = 0x77777777u;   // all-zero block: every element is the exact-zero level
+  if (amax >= kTinyAbsmax) {
+    const float sc = __frcp_rn(amax) * (float)(kCodeBins / 2);
+    uint32_t e[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) e[i] = lut[code_lut_index(v[i], sc)];
+    const uint32_t w0 = pack_entries(e[0], e[1], e[2], e[3]), w1 = pack_entries(e[4], e[5], e[6], e[7]);
+    const uint32_t w2 = pack_entries(e[8], e[9], e[10], e[11]), w3 = pack_entries(e[12], e[13], e[14], e[15]);
+    pk0 = pack_nibbles(w0, w1);
+    pk1 = pack_nibbles(w2, w3);
+    if ((w0 | w1 | w2 | w3) & 0x80808080u) {
+      // Boundary weights (a few per warp): exact division, code = j + (x > t_j).
+      uint32_t m = boundary_bits(w0) | (boundary_bits(w1) << 4) | (boundary_bits(w2) << 8) | (boundary_bits(w3) << 12);
+      while (m) {
+        const int i = __ffs(m) - 1;
+        m &= m - 1;
+        const int sh = 4 * (i & 7);
+        uint32_t &pk = i < 8 ? pk0 : pk1;
+        const uint32_t j = (pk >> sh) & 0xFu;
+        const uint32_t c = j + (__fdiv_rn(select16(v, i), amax) > thr[j] ? 1u : 0u);
+        pk = (pk & ~(0xFu << sh)) | (c << sh);
+      }
+    }
+  } else if (amax != 0.f) {
+    pk0 = pk1 = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      pk0 |= th.encode(__fdiv_rn(v[i], amax)) << (4 * i);
+      pk1 |= th.encode(__fdiv_rn(v[8 + i], amax)) << (4 * i);
+    }
+  }
+}
+
+// Group g of the tensor, this lane's sixteen weights in v: codes and c2 out,
+// the lane's share of the c2 sum into acc.
+__device__ __forceinline__ void quant_group(const float (&v)[16], int64_t g, const uint8_t *lut, const float *thr,
+                                            const NF4Thresholds &th, uint8_t *__restrict__ codes,
+                                            float *__restrict__ c2, double &acc) {
+  const int lane = lane_id();
+  float amax = 0.f;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(v[i]));
+  amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 1));
+  amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 2));
+  uint32_t pk0, pk1;
+  quant_lane16(v, amax, lut, thr, th, pk0, pk1);
+  reinterpret_cast<uint2 *>(codes)[(g << 5) + lane] = make_uint2(pk0, pk1);
+  if ((lane & 3) == 0) {
+    c2[(g << 3) + (lane >> 2)] = amax;
+    acc += (double)amax;
+  }
+}
+
+// Sixteen consecutive weights from shared memory (16-byte aligned).
 template <typename TW>
-__global__ void __launch_bounds__(kQuantThreads, kQuantCtasPerSm) nf4_quantize_kernel(const TW *__restrict__ W, int64_t numel,
+__device__ __forceinline__ void lds_unpack16(uint32_t addr, float (&v)[16]);
+template <>
+__device__ __forceinline__ void lds_unpack16<float>(uint32_t addr, float (&v)[16]) {
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    uint4 q;
+    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(q.x), "=r"(q.y), "=r"(q.z), "=r"(q.w) : "r"(addr + 16 * i));
+    v[4 * i] = __uint_as_float(q.x); v[4 * i + 1] = __uint_as_float(q.y);
+    v[4 * i + 2] = __uint_as_float(q.z); v[4 * i + 3] = __uint_as_float(q.w);
+  }
+}
+template <>
+__device__ __forceinline__ void lds_unpack16<__nv_bfloat16>(uint32_t addr, float (&v)[16]) {
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    uint32_t w[4];
+    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3]) : "r"(addr + 16 * h));
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      v[8 * h + 2 * i] = __uint_as_float(w[i] << 16);
+      v[8 * h + 2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+    }
+  }
+}
+
+// Bulk copy global -> shared of `bytes` (multiple of 16; both addresses
+// 16-byte aligned), completing on mbarrier `bar`.
+__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+               "l"(src), "r"(bytes), "r"(bar)
+               : "memory");
+}
+
+template <typename TW>
+struct QuantCfg {
+  static constexpr int kChunkBytes = kQuantChunk * (int)sizeof(TW);
+  static constexpr int kStages = kQuantRingBytes / kChunkBytes;     // 10 (bf16) or 5 (fp32)
+  static constexpr int kSmemBytes = kQuantRingBytes + 2 * kStages * 8 + 1024;   // + the static code table
+  static_assert(kStages >= 2 && kStages <= 16, "ring depth");
+};
+
+template <typename TW>
+__global__ void __launch_bounds__(kQuantThreads, 1) nf4_quantize_kernel(const TW *__restrict__ W, int64_t numel,
                                                                     uint8_t *__restrict__ codes,
                                                                     float *__restrict__ c2,
-                                                                    double *__restrict__ partial, int table) {
+                                                                    double *__restrict__ partial, int table,
+                                                                    int *err) {
+  using Cfg = QuantCfg<TW>;
+  constexpr int S = Cfg::kStages;
+  extern __shared__ uint8_t qsm_raw[];
+  uint8_t *ring = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(qsm_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t *full = reinterpret_cast<uint64_t *>(ring + kQuantRingBytes);
+  uint64_t *empty = full + S;
+  // The code table is a static shared array: its address is a constant of
+  // the kernel, so a lookup is one shared load with the index as its only
+  // register operand (through a pointer into dynamic shared memory it was a
+  // generic load with 64-bit address arithmetic, measured ALU-bound).
+  __shared__ __align__(16) uint8_t lut[kCodeLutSpan];
   __shared__ double red[kQuantThreads / 32];
   __shared__ float thr[16];
   __shared__ int tb_s[16];
-  __shared__ __align__(16) uint8_t lut[kCodeLutSpan];
   NF4Thresholds th;
   th.init(table);
   if (threadIdx.x < 15)
     thr[threadIdx.x] =
         __double2float_rd(((double)kLevels[table][threadIdx.x] + (double)kLevels[table][threadIdx.x + 1]) * 0.5);
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < S; ++i) {
+      mbar_init(smem_u32(full + i), 1);
+      mbar_init(smem_u32(empty + i), kQuantChunk / 512);      // one arrival per group of the chunk
+    }
+    fence_mbar_init();
+  }
   build_code_lut(lut, table, tb_s);
   __syncthreads();
   pdl_trigger();
   pdl_wait();
+  const int warp = warp_id();
   const int lane = lane_id();
   const int64_t ngroups = numel >> 9;
-  const int64_t nwarps = (int64_t)gridDim.x * (kQuantThreads / 32);
+  const int64_t nchunks = numel / kQuantChunk;
+  // this CTA's chunks: blockIdx.x + i * gridDim.x, i < mine
+  const int64_t mine = (int64_t)blockIdx.x < nchunks ? (nchunks - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+  constexpr int kGroupsPerChunk = kQuantChunk / 512;
   double acc = 0.0;
 
-  for (int64_t g = (int64_t)blockIdx.x * (kQuantThreads / 32) + warp_id(); g < ngroups; g += nwarps) {
-    const int64_t base = (g << 9) + (lane << 4);
-    Raw16<TW> cur;
-    cur.load(W + base);
-    float v[16];
-    cur.unpack(v);
-    float amax = 0.f;
+  if (warp == kQuantComputeWarps) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      for (int64_t i = 0; i < mine; ++i) {
+        const int st = (int)(i % S);
+        if (!mbar_wait(smem_u32(empty + st), ((uint32_t)(i / S) & 1u) ^ 1u, err, DEV_TIMEOUT_PRODUCER)) break;
+        const uint32_t fb = smem_u32(full + st);
+        mbar_arrive_expect_tx(fb, Cfg::kChunkBytes);
+        bulk_g2s(smem_u32(ring + st * Cfg::kChunkBytes), W + (blockIdx.x + i * gridDim.x) * (int64_t)kQuantChunk,
+                 Cfg::kChunkBytes, fb);
+      }
+      // A CTA never exits with bulk copies into its shared memory in flight.
+      for (int64_t i = mine > S ? mine - S : 0; i < mine; ++i)
+        if (!mbar_wait(smem_u32(full + (int)(i % S)), (uint32_t)(i / S) & 1u, err, DEV_TIMEOUT_DRAIN)) break;
+    }
+  } else {
+    // ------------------------------------------------------------ compute warps
+    for (int64_t q = warp; q < mine * kGroupsPerChunk; q += kQuantComputeWarps) {
+      const int64_t i = q / kGroupsPerChunk;
+      const int gi = (int)(q % kGroupsPerChunk);
+      const int st = (int)(i % S);
+      if (!__all_sync(0xFFFFFFFFu, mbar_wait(smem_u32(full + st), (uint32_t)(i / S) & 1u, err, DEV_TIMEOUT_MMA))) break;
+      float v[16];
+      lds_unpack16<TW>(smem_u32(ring + st * Cfg::kChunkBytes) + (uint32_t)((gi * 512 + lane * 16) * (int)sizeof(TW)), v);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(empty + st));   // this group's weights are in registers
+      const int64_t g = (blockIdx.x + i * gridDim.x) * kGroupsPerChunk + gi;
+      quant_group(v, g, lut, thr, th, codes, c2, acc);
+    }
+    // The last CTA: the groups after the last whole chunk, from global memory.
+    if (blockIdx.x == gridDim.x - 1) {
+      for (int64_t g = nchunks * kGroupsPerChunk + warp; g < ngroups; g += kQuantComputeWarps) {
+        Raw16<TW> cur;
+        cur.load(W + (g << 9) + (lane << 4));
+        float v[16];
+        cur.unpack(v);
+        quant_group(v, g, lut, thr, th, codes, c2, acc);
+      }
+      // Tail: blocks [8*ngroups, nblk), at most 8, one warp each.
+      const int64_t nblk = (numel + 63) >> 6;
+      const int64_t b = (ngroups << 3) + warp;
+      if (warp < 8 && b < nblk) {
+        const int64_t s = b << 6;
+        const int64_t i0 = s + 2 * lane, i1 = i0 + 1;
+        const float v0 = i0 < numel ? load1(W + i0) : 0.f;
+        const float v1 = i1 < numel ? load1(W + i1) : 0.f;
+        float amax = fmaxf(fabsf(v0), fabsf(v1));
 #pragma unroll
-    for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(v[i]));
-    amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 1));
-    amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 2));
-    uint32_t pk0 = 0x77777777u, pk1 = 0x77777777u;   // all-zero block: every element is the exact-zero level
-    if (amax >= kTinyAbsmax) {
-      const float sc = __frcp_rn(amax) * (float)(kCodeBins / 2);
-      uint32_t e[16];
-#pragma unroll
-      for (int i = 0; i < 16; ++i) e[i] = lut[code_lut_index(v[i], sc)];
-      const uint32_t w0 = pack_entries(e[0], e[1], e[2], e[3]), w1 = pack_entries(e[4], e[5], e[6], e[7]);
-      const uint32_t w2 = pack_entries(e[8], e[9], e[10], e[11]), w3 = pack_entries(e[12], e[13], e[14], e[15]);
-      pk0 = pack_nibbles(w0, w1);
-      pk1 = pack_nibbles(w2, w3);
-      if ((w0 | w1 | w2 | w3) & 0x80808080u) {
-        // Boundary weights (a few per warp): exact division, code = j + (x > t_j).
-        uint32_t m = boundary_bits(w0) | (boundary_bits(w1) << 4) | (boundary_bits(w2) << 8) | (boundary_bits(w3) << 12);
-        while (m) {
-          const int i = __ffs(m) - 1;
-          m &= m - 1;
-          const int sh = 4 * (i & 7);
-          uint32_t &pk = i < 8 ? pk0 : pk1;
-          const uint32_t j = (pk >> sh) & 0xFu;
-          const uint32_t c = j + (__fdiv_rn(load1(W + base + i), amax) > thr[j] ? 1u : 0u);
-          pk = (pk & ~(0xFu << sh)) | (c << sh);
+        for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
+        uint32_t k0 = 7, k1 = 7;
+        if (amax != 0.f) {
+          k0 = th.encode(__fdiv_rn(v0, amax));
+          k1 = i1 < numel ? th.encode(__fdiv_rn(v1, amax)) : 0u;
+        } else if (i1 >= numel) {
+          k1 = 0;
         }
-      }
-    } else if (amax != 0.f) {
-      pk0 = pk1 = 0;
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        pk0 |= th.encode(__fdiv_rn(v[i], amax)) << (4 * i);
-        pk1 |= th.encode(__fdiv_rn(v[8 + i], amax)) << (4 * i);
-      }
-    }
-    reinterpret_cast<uint2 *>(codes)[(g << 5) + lane] = make_uint2(pk0, pk1);
-    if ((lane & 3) == 0) {
-      c2[(g << 3) + (lane >> 2)] = amax;
-      acc += (double)amax;
-    }
-  }
-
-  // Tail: blocks [8*ngroups, nblk), at most 8, one warp each in the last CTA.
-  if (blockIdx.x == gridDim.x - 1) {
-    const int64_t nblk = (numel + 63) >> 6;
-    const int64_t b = (ngroups << 3) + warp_id();
-    if (b < nblk) {
-      const int64_t s = b << 6;
-      const int64_t i0 = s + 2 * lane, i1 = i0 + 1;
-      const float v0 = i0 < numel ? load1(W + i0) : 0.f;
-      const float v1 = i1 < numel ? load1(W + i1) : 0.f;
-      float amax = fmaxf(fabsf(v0), fabsf(v1));
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
-      uint32_t k0 = 7, k1 = 7;
-      if (amax != 0.f) {
-        k0 = th.encode(__fdiv_rn(v0, amax));
-        k1 = i1 < numel ? th.encode(__fdiv_rn(v1, amax)) : 0u;
-      } else if (i1 >= numel) {
-        k1 = 0;
-      }
-      if (i0 < numel) codes[i0 >> 1] = (uint8_t)(k0 | (k1 << 4));
-      if (lane == 0) {
-        c2[b] = amax;
-        acc += (double)amax;
+        if (i0 < numel) codes[i0 >> 1] = (uint8_t)(k0 | (k1 << 4));
+        if (lane == 0) {
+          c2[b] = amax;
+          acc += (double)amax;
+        }
       }
     }
   }
@@ -460,13 +601,6 @@ static_assert(kDqCodeBytes == 4 * kDqWordsPerThread * kDqThreads, "whole code wo
 static_assert(256 % (kDqChunk / 64) == 0, "a chunk lies inside one 256-block group");
 static_assert(kDqStageBytes % 16 == 0 && kDqC2Bytes % 16 == 0, "bulk-copy sizes and offsets");
 
-// Bulk copy global -> shared of `bytes` (multiple of 16; both addresses
-// 16-byte aligned), completing on mbarrier `bar`.
-__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar) {
-  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
-               "l"(src), "r"(bytes), "r"(bar)
-               : "memory");
-}
 
 // Eight weights from one 32-bit word of codes (element i in bits [4i, 4i+4)).
 __device__ __forceinline__ uint4 dq_decode8(uint32_t q, float c2h, const float *lut) {
