@@ -898,7 +898,9 @@ def run_reference(args, rank, world):
     cores = _cores()
     return {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_s * 1e3, "higher_is_better": True,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True,
+        "step_is_sample": f"each timed step is the 1/{SAMPLE_SLICE} sample below, so ms_per_step is the sample's "
+                          f"time; value = the sample's FLOPs / that time (full-step time {step_s * 1e3:.0f} ms)",
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": train_config(_subargs(args, workload="llama7b-train", linear=None, dropout=0.0), WL, 1),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": SAMPLE_DESC,
