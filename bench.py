@@ -180,19 +180,33 @@ def build_layer(dev, rank, wl=WL):
     return lins, grads, [H, A, U] + [l.dY for l in lins]
 
 
+BWD_GROUPS = (("down",), ("gate", "up"), ("o",), ("q", "k", "v"))
+
+
 def make_step(qlora, lins, grads, world, wl=WL, dropout=0.0):
     """One step; `ready(t)` (if given) is called before the step first reads input t.
     With `dropout` > 0 each linear applies LoRA dropout with its own keep mask.
     Without dropout the forward runs the linears that read the same input as
     one grouped call (q, k, v, gate and up on the layer input), in the order
-    of their first use."""
-    groups = []
+    of their first use, and the backward as grouped calls in the order a
+    layer's gradients arrive (BWD_GROUPS)."""
+    groups, bwd_groups = [], []
     if dropout == 0:
         by_x = {}
         for l in lins:
             by_x.setdefault(l.X.data_ptr(), []).append(l)
         groups = [(g[0].X, qlora.FwdGroup([{"X": l.X, "q": l.q, "L1": l.L1, "L2": l.L2, "s": wl.s, "Y": l.Y,
                                              "T": l.T} for l in g])) for g in by_x.values()]
+        # the backward as the layer's gradients arrive: down, then gate and up,
+        # then o, then q, k and v
+        by_name = {l.lin.name: l for l in lins}
+        order = [[by_name[n] for n in names if n in by_name] for names in BWD_GROUPS]
+        order = [g for g in order if g]
+        rest = [l for l in reversed(lins) if all(l not in g for g in order)]
+        order += [[l] for l in rest]
+        bwd_groups = [([l.dY for l in g], qlora.BwdGroup(
+            [{"dY": l.dY, "X": l.X, "T": l.T, "q": l.q, "L1": l.L1, "L2": l.L2, "s": wl.s, "dX": l.dX,
+              "dL1": l.dL1, "dL2": l.dL2} for l in g], grad_dtype=torch.float32)) for g in order]
 
     def step(ready=None):
         for l in lins:
@@ -208,7 +222,11 @@ def make_step(qlora, lins, grads, world, wl=WL, dropout=0.0):
                     ready(l.mask)
             qlora.linear_fwd(l.X, l.q, l.L1, l.L2, wl.s, Y=l.Y, T=l.T, dropout_mask=l.mask, dropout_p=dropout,
                              Xm=l.Xm)
-        for l in reversed(lins):
+        for dys, grp in bwd_groups:
+            for t in (dys if ready else []):
+                ready(t)
+            grp()
+        for l in (reversed(lins) if dropout > 0 else []):
             if ready:
                 ready(l.dY)
             qlora.linear_bwd(l.dY, l.X, l.T, l.q, l.L1, l.L2, wl.s, grad_dtype=torch.float32,
@@ -291,7 +309,8 @@ def train_config(args, wl, world):
             "step": f"quantize {7 * wl.layers} fp32 weights to NF4+DQ, fwd + bwd of the "
                     f"{7 * wl.layers} QLoRA linears"
                     + (" (forward of the linears that read the same input as one grouped call: q, k, v, "
-                       "gate, up on the layer input)" if wl.layers == 1 and args.dropout == 0 else "")
+                       "gate, up on the layer input; backward grouped as the gradients arrive: down, "
+                       "{gate, up}, o, {q, k, v})" if wl.layers == 1 and args.dropout == 0 else "")
                     + (" (layer to layer: H' = bf16(down(up(H)) + R))" if wl.layers > 1 else "")
                     + (", all-reduce of adapter grads" if world > 1 else "")
                     + (f", LoRA dropout p = {args.dropout:g} on every adapter (one seeded keep mask per "

@@ -386,6 +386,97 @@ def linear_bwd(dY: torch.Tensor, X: torch.Tensor, T: torch.Tensor | None, q: NF4
     return (dX if need_dX else None), dL1, dL2
 
 
+class BwdGroup:
+    """A grouped backward whose arguments are marshalled once (see
+    ``linear_bwd_group``).  Calling it runs the group again on the same
+    tensors, which it keeps alive; only the C call is made per run."""
+
+    def __init__(self, members, need_dX: bool = True, grad_dtype=torch.bfloat16):
+        if not 0 < len(members) <= _lib.QLORA_MAX_GROUP:
+            raise ValueError(f"qlora: a group holds 1..{_lib.QLORA_MAX_GROUP} linears")
+        if grad_dtype == torch.bfloat16:
+            gdt = _lib.QLORA_DTYPE_BF16
+        elif grad_dtype == torch.float32:
+            gdt = _lib.QLORA_DTYPE_F32
+        else:
+            raise TypeError("qlora: grad_dtype must be bfloat16 or float32")
+        M = members[0]["dY"].shape[0]
+        dev = members[0]["dY"].device
+        # every argument is checked before the library is loaded or a pointer taken
+        for m in members:
+            dY, X, T, q, L1, L2 = m["dY"], m["X"], m.get("T"), m["q"], m["L1"], m["L2"]
+            K, r, N = q.k_in, L1.shape[1], q.n_out
+            if dY.shape[0] != M or dY.device != dev:
+                raise ValueError("qlora: the members of a group share the token count and the device")
+            if tuple(dY.shape) != (M, N) or tuple(X.shape) != (M, K) or L1.shape[0] != K or tuple(L2.shape) != (r, N):
+                raise ValueError("qlora: shape mismatch")
+            if T is not None and (tuple(T.shape) != (M, 2 * r) or T.dtype != torch.bfloat16):
+                raise ValueError(f"qlora: T must be the forward's bf16 [M, 2r] = {(M, 2 * r)} hi/lo pair")
+            if need_dX:
+                _check_out(m.get("dX"), (M, K), torch.bfloat16, dev, "dX")
+            _check_out(m.get("dL1"), (K, r), grad_dtype, dev, "dL1")
+            _check_out(m.get("dL2"), (r, N), grad_dtype, dev, "dL2")
+            _check_device(dev, False, X=X, T=T, L1=L1, L2=L2, codes=q.codes, c2_fp8=q.c2_fp8, c1=q.c1,
+                          c2_mean=q.c2_mean)
+        # caller-supplied outputs may not overlap each other or any member's input
+        names = ("dX", "dL1", "dL2") if need_dX else ("dL1", "dL2")
+        outs = [(i, name, _span(m.get(name))) for i, m in enumerate(members) for name in names]
+        for i, name, sp in outs:
+            for j, m in enumerate(members):
+                for inp in ("dY", "X", "T"):
+                    if _overlap(sp, _span(m.get(inp))):
+                        raise ValueError(f"qlora: member {i}'s {name} overlaps member {j}'s {inp}")
+            for j, name2, sp2 in outs:
+                if (i, name) < (j, name2) and _overlap(sp, sp2):
+                    raise ValueError(f"qlora: member {i}'s {name} overlaps member {j}'s {name2}")
+        _check_device(dev)
+        lib = _lib.load()
+        arr = (_lib.BwdMember * len(members))()
+        self._keep, self.outputs = [], []
+        for i, m in enumerate(members):
+            dY, X, T, q, L1, L2 = m["dY"], m["X"], m.get("T"), m["q"], m["L1"], m["L2"]
+            K, r, N = q.k_in, L1.shape[1], q.n_out
+            dX = m.get("dX") if need_dX else None
+            if need_dX and dX is None:
+                dX = torch.empty((M, K), dtype=torch.bfloat16, device=dev)
+            dL1 = m.get("dL1")
+            if dL1 is None:
+                dL1 = torch.empty((K, r), dtype=grad_dtype, device=dev)
+            dL2 = m.get("dL2")
+            if dL2 is None:
+                dL2 = torch.empty((r, N), dtype=grad_dtype, device=dev)
+            w = q.as_struct()
+            self._keep += [w, dY, X, T, q, L1, L2]
+            arr[i] = _lib.BwdMember(_ptr(_bits(dY)), _ptr(_bits(X)), _ptr(T), ctypes.pointer(w), _ptr(_bits(L1)),
+                                    _ptr(_bits(L2)), r, float(m["s"]), _ptr(dX) if need_dX else None, _ptr(dL1),
+                                    _ptr(dL2))
+            self.outputs.append((dX if need_dX else None, dL1, dL2))
+        self._arr, self._n, self._M, self._dev, self._gdt = arr, len(members), M, dev, gdt
+        self._ws_bytes = lib.qlora_linear_bwd_group_workspace_size(arr, len(members), M)
+        self._fn = lib.qlora_linear_bwd_group
+
+    def __call__(self) -> list:
+        ws = _WS.get(self._ws_bytes, self._dev)
+        _lib.check(self._fn(self._arr, self._n, self._M, self._gdt, ws.data_ptr(), ws.numel(), _stream(self._dev)),
+                   "qlora_linear_bwd_group")
+        return self.outputs
+
+
+def linear_bwd_group(members, need_dX: bool = True, grad_dtype=torch.bfloat16) -> list:
+    """The backward of several linears whose output gradients are available
+    together, in one call.
+
+    ``members``: a sequence of dicts with keys ``dY`` [M, N_i], ``X`` [M, K_i],
+    ``T`` (the forward's [M, 2 r_i] pair, or None to recompute), ``q``
+    (NF4Tensor), ``L1`` [K_i, r_i], ``L2`` [r_i, N_i], ``s`` and optionally the
+    outputs ``dX``, ``dL1``, ``dL2``.  Every member computes what
+    ``linear_bwd`` computes; the rank-r products of all members run as two
+    launches, and members that read the same X share one pass over it for
+    dL1.  Returns [(dX or None, dL1, dL2)] in member order.
+    """
+    return BwdGroup(members, need_dX, grad_dtype)()
+
+
 def profile_start(capacity: int = 4096) -> None:
     """Start logging the library's kernel launches with CUDA events (diagnostics)."""
     _lib.check(_lib.load().qlora_profile_start(capacity), "qlora_profile_start")

@@ -31,6 +31,7 @@ QLORA_MAX_RANK = 256
 KERNEL_KINDS = {
     1: "quantize", 2: "dq_constants", 3: "dequant",
     10: "gemm_T", 11: "gemm_Y", 12: "gemm_G", 13: "gemm_dX", 14: "gemm_dL2", 15: "gemm_dL1", 16: "gemm_Z",
+    17: "rank_G_dL2", 18: "rank_dL1",
     20: "splitk_finalize", 31: "fused_fwd", 40: "dropout_mask", 41: "t_scatter",
 }
 
@@ -69,6 +70,24 @@ class FwdMember(ctypes.Structure):
     ]
 
 
+class BwdMember(ctypes.Structure):
+    """Mirror of qlora_bwd_member_t (one linear of a grouped backward)."""
+
+    _fields_ = [
+        ("dY", c_void_p),
+        ("X", c_void_p),
+        ("T_saved", c_void_p),
+        ("W", POINTER(NF4DQ)),
+        ("L1", c_void_p),
+        ("L2", c_void_p),
+        ("r", ctypes.c_int32),
+        ("s", c_float),
+        ("dX", c_void_p),
+        ("dL1", c_void_p),
+        ("dL2", c_void_p),
+    ]
+
+
 # name -> (restype, argtypes)
 SIGNATURES = {
     "qlora_version": (c_int, []),
@@ -95,6 +114,8 @@ SIGNATURES = {
                                  c_float, c_void_p, c_void_p, c_void_p, c_int, c_void_p, c_size_t, c_void_p]),
     "qlora_linear_fwd_group_workspace_size": (c_size_t, [POINTER(FwdMember), c_int, c_int64]),
     "qlora_linear_fwd_group": (c_int, [POINTER(FwdMember), c_int, c_int64, c_void_p, c_size_t, c_void_p]),
+    "qlora_linear_bwd_group_workspace_size": (c_size_t, [POINTER(BwdMember), c_int, c_int64]),
+    "qlora_linear_bwd_group": (c_int, [POINTER(BwdMember), c_int, c_int64, c_int, c_void_p, c_size_t, c_void_p]),
     "qlora_linear_fwd_dropout_workspace_size": (c_size_t, [c_int64, c_int64, c_int64, c_int]),
     "qlora_linear_bwd_dropout_workspace_size": (c_size_t, [c_int64, c_int64, c_int64, c_int]),
     "qlora_linear_fwd_dropout": (c_int, [c_void_p, c_int64, POINTER(NF4DQ), c_void_p, c_void_p, c_int, c_float,

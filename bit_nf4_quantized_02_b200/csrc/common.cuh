@@ -67,6 +67,16 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t byt
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
 }
 
+// Proxy fence for shared memory.  A stage that threads read with ordinary
+// loads (the generic proxy) and that a bulk or tensor copy (the async proxy)
+// then refills needs one on each side: the readers issue it after their loads
+// and before they release the stage (so the loads have completed), and the
+// copying thread issues it after it has seen the release and before the copy.
+// Without them a refill was seen to overtake reads still in flight.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }

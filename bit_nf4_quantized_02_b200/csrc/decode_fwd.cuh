@@ -305,6 +305,7 @@ __global__ void __launch_bounds__(DfCfg<MP>::kThreads, 1)
         df_item<GM>(p, it, l, rt, ks);
         const int cs = rel % SC, xs = rel % SX;
         if (!mbar_wait(smem_u32(cempty_bar + cs), ((uint32_t)(rel / SC) & 1u) ^ 1u, p.err, DEV_TIMEOUT_PRODUCER)) break;
+        fence_proxy_async_smem();   // the decoders' loads of this slot before the copy's writes
         const uint32_t cb = smem_u32(cfull_bar + cs);
         mbar_arrive_expect_tx(cb, Cfg::kCodeBytes);
         tma_load_2d(smem_u32(smem + cs * Cfg::kCodeBytes), &maps.codes[l], cb, ks * (kDfStageK / 2), rt * kDfRows);
@@ -424,6 +425,7 @@ __global__ void __launch_bounds__(DfCfg<MP>::kThreads, 1)
       uint4 qv[8];
 #pragma unroll
       for (int c = 0; c < 8; ++c) qv[c] = lds128(sc + (((uint32_t)c << 4) ^ cswz));
+      fence_proxy_async_smem();   // the loads complete before the slot is released
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(cempty_bar + cs));
       // the MMAs of this group's previous item (rel - G) have read its A

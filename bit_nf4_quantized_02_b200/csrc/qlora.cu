@@ -6,7 +6,9 @@
 #include <algorithm>
 #include <atomic>
 #include <cstring>
+#include <map>
 #include <mutex>
+#include <vector>
 
 #include "qlora.h"
 #include "common.cuh"
@@ -16,6 +18,7 @@
 #include "decode_fwd.cuh"
 #include "dropout.cuh"
 #include "group.cuh"
+#include "rank_gemm.cuh"
 
 namespace qlora {
 
@@ -51,6 +54,7 @@ struct DeviceInfo {
   std::atomic<int> pair_clusters[3];     // co-resident 2-CTA clusters of the pair GEMM [form]
   std::atomic<int> decode_smem_set[8];   // few-token product: smem limit set [group form][token padding]
   std::atomic<int> quant_smem_set[2];    // quantizer: smem limit set [bf16, fp32 input]
+  std::atomic<int> rank_smem_set{0};     // grouped rank-r products: smem limit set
 };
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_mu;
@@ -440,6 +444,208 @@ int tc_gemm(cudaStream_t st, DeviceInfo *dev, int64_t M, int64_t N, int nseg, co
   ProfScope prof(QLORA_KERNEL_SPLITK_FINALIZE, st);
   return launch_pdl(splitk_finalize_kernel, dim3(grid), dim3(256), 0, st, (const float *)split_ws, splits, (int)M,
                     (int)W, alpha, out, ld_row, ld_col, lo_off, out_f32);
+}
+
+// ---------------------------------------------------- grouped rank-r products
+// Host side of rank_gemm_kernel: one problem per RankJob.
+struct RankJob {
+  Operand A, B;
+  int bn;                    // 64 or 128: B rows per n-tile (the MMA N)
+  int n_tiles;
+  int ncols;                 // valid output columns per n-tile, before the fold
+  int fold;
+  RankOut outs[kMaxGroup];   // one per n-tile (part is filled at launch)
+  int width() const { return fold ? fold : ncols; }
+};
+
+struct RankShape {
+  int64_t m_tiles, tiles, nkb;
+};
+
+RankShape rank_shape(const RankJob &j) {
+  RankShape s;
+  s.m_tiles = (j.A.rows + kBM - 1) / kBM;
+  s.tiles = s.m_tiles * j.n_tiles;
+  s.nkb = (j.A.kext + kBK - 1) / kBK;
+  return s;
+}
+
+// Splits of each problem's reduction, chosen by simulating the kernel's walk:
+// units in order of decreasing length, CTA c taking unit kG + c in even rounds
+// and kG + G - 1 - c in odd ones.  A unit costs its k-blocks plus one (the
+// hand-over between units); a split unit three more (its partial's store and
+// the finalize's read, each 32 KB at r = 64 against 16 KB of A per k-block).
+// The plan with the smallest largest CTA load wins.  Plans are cached by shape.
+constexpr int kRankMinKb = 4;
+
+void plan_rank(const RankShape *sh, int n, int sms, int *splits) {
+  static std::mutex mu;
+  static std::map<std::vector<int64_t>, std::vector<int>> cache;
+  std::vector<int64_t> key{sms, n};
+  for (int i = 0; i < n; ++i) key.insert(key.end(), {sh[i].tiles, sh[i].nkb});
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    auto it = cache.find(key);
+    if (it != cache.end()) {
+      std::copy(it->second.begin(), it->second.end(), splits);
+      return;
+    }
+  }
+  std::vector<int64_t> cand;
+  for (int i = 0; i < n; ++i)
+    for (int s = 1; s <= 32; ++s) {
+      const int64_t L = (sh[i].nkb + s - 1) / s;
+      if (L >= kRankMinKb || s == 1) cand.push_back(L);
+    }
+  std::sort(cand.begin(), cand.end());
+  cand.erase(std::unique(cand.begin(), cand.end()), cand.end());
+  std::vector<int> best(n, 1), cur(n);
+  int64_t best_span = INT64_MAX, best_units = INT64_MAX;
+  std::vector<int64_t> load;
+  std::vector<std::pair<int64_t, int64_t>> runs;   // (cost, count), longest first
+  for (int64_t L : cand) {
+    runs.clear();
+    int64_t units = 0;
+    for (int i = 0; i < n; ++i) {
+      int64_t s = std::max<int64_t>(1, (sh[i].nkb + L - 1) / L);
+      const int64_t kbps = (sh[i].nkb + s - 1) / s;
+      s = (sh[i].nkb + kbps - 1) / kbps;
+      cur[i] = (int)s;
+      runs.push_back({kbps + 1 + (s > 1 ? 3 : 0), sh[i].tiles * s});
+      units += sh[i].tiles * s;
+    }
+    std::stable_sort(runs.begin(), runs.end(), [](auto &a, auto &b) { return a.first > b.first; });
+    const int64_t G = std::max<int64_t>(1, std::min<int64_t>(units, sms));
+    load.assign((size_t)G, 0);
+    int64_t u = 0;
+    for (auto &rc : runs)
+      for (int64_t c = 0; c < rc.second; ++c, ++u) {
+        const int64_t k = u / G, pos = u - k * G;
+        load[(size_t)((k & 1) ? G - 1 - pos : pos)] += rc.first;
+      }
+    const int64_t span = *std::max_element(load.begin(), load.end());
+    if (span < best_span || (span == best_span && units < best_units)) {
+      best_span = span;
+      best_units = units;
+      best = cur;
+    }
+  }
+  std::copy(best.begin(), best.end(), splits);
+  std::lock_guard<std::mutex> lock(mu);
+  cache.emplace(std::move(key), std::move(best));
+}
+
+// fp32 partial bytes of a launch of these problems.
+size_t rank_part_bytes(const RankJob *jobs, int n, int sms) {
+  if (n <= 0) return 0;
+  RankShape sh[kRankMaxProbs];
+  int splits[kRankMaxProbs];
+  for (int i = 0; i < n; ++i) sh[i] = rank_shape(jobs[i]);
+  plan_rank(sh, n, sms, splits);
+  size_t b = 0;
+  for (int i = 0; i < n; ++i)
+    if (splits[i] > 1) b += (size_t)jobs[i].n_tiles * align_up((size_t)splits[i] * jobs[i].A.rows * jobs[i].width() * 4);
+  return b;
+}
+
+// Runs the problems as one rank_gemm_kernel launch (then, if any is split,
+// one rank_finalize_kernel launch).  `part` holds rank_part_bytes() bytes.
+int rank_launch(const RankJob *jobs, int n, uint8_t *part, DeviceInfo *dev, cudaStream_t st, int kind) {
+  if (n <= 0) return QLORA_OK;
+  if (n > kRankMaxProbs) return QLORA_ERR_UNSUPPORTED_SHAPE;
+  RankShape sh[kRankMaxProbs];
+  int splits[kRankMaxProbs], order[kRankMaxProbs];
+  int64_t kbps[kRankMaxProbs];
+  for (int i = 0; i < n; ++i) sh[i] = rank_shape(jobs[i]);
+  plan_rank(sh, n, dev->sms, splits);
+  for (int i = 0; i < n; ++i) {
+    kbps[i] = (sh[i].nkb + splits[i] - 1) / splits[i];
+    order[i] = i;
+  }
+  // longest units first, as the plan assumed
+  std::stable_sort(order, order + n, [&](int a, int b) {
+    return kbps[a] + (splits[a] > 1 ? 3 : 0) > kbps[b] + (splits[b] > 1 ? 3 : 0);
+  });
+  RankMaps maps;
+  RankArgs a;
+  RankFinArgs fin;
+  std::memset(&maps, 0, sizeof(maps));
+  std::memset(&a, 0, sizeof(a));
+  std::memset(&fin, 0, sizeof(fin));
+  int64_t units = 0, elem = 0;
+  size_t part_off = 0;
+  for (int oi = 0; oi < n; ++oi) {
+    const int i = order[oi];
+    const RankJob &j = jobs[i];
+    if (a.nout + j.n_tiles > kRankMaxOuts || j.n_tiles < 1) return QLORA_ERR_UNSUPPORTED_SHAPE;
+    if (j.A.rows > INT32_MAX / 2 || j.A.kext > INT32_MAX / 2) return QLORA_ERR_UNSUPPORTED_SHAPE;
+    RankProb &q = a.prob[a.nprob];
+    q.rows = (int)j.A.rows;
+    q.m_tiles = (int)sh[i].m_tiles;
+    q.n_tiles = j.n_tiles;
+    q.bn = j.bn;
+    q.ncols = j.ncols;
+    q.fold = j.fold;
+    q.nkb = (int)sh[i].nkb;
+    q.splits = splits[i];
+    q.kb_per_split = (int)kbps[i];
+    q.a_mn = j.A.mn_major;
+    q.b_mn = j.B.mn_major;
+    q.wide = q.nkb >= 2 && wide_ok(j.A) && wide_ok(j.B);
+    q.unit0 = (int)units;
+    q.out0 = a.nout;
+    int rc = q.wide ? make_tmap3(&maps.m[2 * a.nprob], j.A, kBM) : make_tmap(&maps.m[2 * a.nprob], j.A, kBM);
+    if (rc) return rc;
+    rc = q.wide ? make_tmap3(&maps.m[2 * a.nprob + 1], j.B, j.bn) : make_tmap(&maps.m[2 * a.nprob + 1], j.B, j.bn);
+    if (rc) return rc;
+    for (int t = 0; t < j.n_tiles; ++t) {
+      RankOut o = j.outs[t];
+      o.part = nullptr;
+      if (q.splits > 1) {
+        if (fin.njobs == kRankMaxOuts) return QLORA_ERR_UNSUPPORTED_SHAPE;
+        o.part = reinterpret_cast<float *>(part + part_off);
+        part_off += align_up((size_t)q.splits * q.rows * j.width() * 4);
+        RankFinJob &f = fin.job[fin.njobs++];
+        f.part = o.part;
+        f.out = o.ptr;
+        f.ld_row = o.ld_row;
+        f.ld_col = o.ld_col;
+        f.lo_off = o.lo_off;
+        f.elem0 = elem;
+        f.splits = q.splits;
+        f.rows = q.rows;
+        f.width = j.width();
+        f.out_f32 = o.out_f32;
+        f.alpha = o.alpha;
+        elem += (int64_t)q.rows * j.width();
+      }
+      a.out[a.nout + t] = o;
+    }
+    a.nout += j.n_tiles;
+    units += sh[i].tiles * q.splits;
+    ++a.nprob;
+  }
+  if (units > INT32_MAX / 2) return QLORA_ERR_UNSUPPORTED_SHAPE;
+  a.units = (int)units;
+  a.err = dev->err;
+  if (once(dev->rank_smem_set, [&] {
+        return cudaFuncSetAttribute(rank_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    kRankSmemBytes) == cudaSuccess
+                   ? 1
+                   : 0;
+      }) <= 0)
+    return QLORA_ERR_CUDA;
+  const int grid = (int)std::min<int64_t>(units, dev->sms);
+  int rc;
+  {
+    ProfScope prof(kind, st);
+    rc = launch_pdl(rank_gemm_kernel, dim3(grid), dim3(kGemmThreads), kRankSmemBytes, st, maps, a);
+  }
+  if (rc || fin.njobs == 0) return rc;
+  fin.total = elem;
+  const int fgrid = (int)std::min<int64_t>((elem + 255) / 256, (int64_t)dev->sms * 8);
+  ProfScope prof(QLORA_KERNEL_SPLITK_FINALIZE, st);
+  return launch_pdl(rank_finalize_kernel, dim3(fgrid), dim3(256), 0, st, fin);
 }
 
 int dequant_launch(const qlora_nf4dq_t *W, __nv_bfloat16 *out, cudaStream_t st, int sms) {
@@ -1063,6 +1269,212 @@ int bwd_large(const uint16_t *dY, const uint16_t *X, const uint16_t *T_saved, in
   return tc_gemm(st, dev, K, r, 2, s1, keep, dL1, r, 1, out_f32, split_ws, QLORA_KERNEL_GEMM_DL1, 0, true);
 }
 
+// ------------------------------------------ grouped backward (many tokens)
+struct BwdMember {
+  const uint16_t *dY, *X, *T;   // X: what the adapter reads (the masked input under LoRA dropout)
+  const qlora_nf4dq_t *W;
+  const uint16_t *L1, *L2;
+  int r;
+  float s;
+  uint16_t *dX;
+  void *dL1, *dL2;
+  float keep = 1.f;             // LoRA dropout's 1 / (1 - p): scales T's recomputation and dL1
+};
+
+// The grouped rank kernel serves ranks whose [hi | lo] pair fits one
+// 128-column tile with the fold's chunking.
+bool rank_group_ok(int r) { return r <= 64 && can_fold(r); }
+
+// Workspace of a grouped backward.  G holds every member's hi/lo pair side by
+// side ([M x sum 2r] bf16), the members that share X (same pointer, K and r)
+// next to each other, so that their dL1 products read one [M x 2r*n] operand.
+struct BwdGroupLayout {
+  size_t g = 0, t = 0, w_hat = 0, part = 0, total = 0;
+  int64_t g_ld = 0;
+  int64_t g_col[kMaxGroup] = {};
+  size_t t_off[kMaxGroup] = {};
+  int set_of[kMaxGroup] = {};   // X set of each member
+  int nsets = 0;
+  int set_first[kMaxGroup] = {}, set_size[kMaxGroup] = {};
+};
+
+// The rank problems of the three launches: T (members without T_saved), G and
+// dL2 (every member), dL1 (one problem per X set when its n-tiles line up with
+// the members' pairs, else one per member).  Pointers into the workspace are
+// taken relative to `w8` (nullptr when only sizing).
+struct BwdGroupJobs {
+  RankJob t[kMaxGroup], gl2[2 * kMaxGroup], l1[kMaxGroup];
+  int nt = 0, ngl2 = 0, nl1 = 0;
+};
+
+void bwd_group_jobs(int64_t M, const BwdMember *mem, int count, const BwdGroupLayout &L, uint8_t *w8, bool f32,
+                    bool t_all, BwdGroupJobs &J) {
+  auto at = [w8](size_t off) { return reinterpret_cast<uint16_t *>(reinterpret_cast<uintptr_t>(w8) + off); };
+  uint16_t *G = at(L.g);
+  for (int i = 0; i < count; ++i) {
+    const BwdMember &m = mem[i];
+    const int64_t N = m.W->n_out, K = m.W->k_in;
+    const int r = m.r;
+    const uint16_t *T = m.T;
+    if (!T || t_all) {   // T = s X L1 as a hi/lo pair
+      uint16_t *Tw = at(L.t + L.t_off[i]);
+      RankJob &j = J.t[J.nt++];
+      j.A = {m.X, M, K, K, 0};
+      j.B = {m.L1, r, K, r, 1};
+      j.bn = 64;
+      j.n_tiles = 1;
+      j.ncols = r;
+      j.fold = 0;
+      j.outs[0] = RankOut{Tw, nullptr, 2 * r, 1, r, m.s * m.keep, 0};
+      T = Tw;
+    }
+    RankJob &jg = J.gl2[J.ngl2++];   // G = s dY L2^T (L2 [r x N] is K-major here)
+    jg.A = {m.dY, M, N, N, 0};
+    jg.B = {m.L2, r, N, N, 0};
+    jg.bn = 64;
+    jg.n_tiles = 1;
+    jg.ncols = r;
+    jg.fold = 0;
+    jg.outs[0] = RankOut{G + L.g_col[i], nullptr, L.g_ld, 1, r, m.s, 0};
+    RankJob &j2 = J.gl2[J.ngl2++];   // dL2^T = dY^T [T_hi | T_lo], folded, written transposed
+    j2.A = {m.dY, N, M, N, 1};
+    j2.B = {T, 2 * r, M, 2 * r, 1};
+    j2.bn = 2 * r <= 64 ? 64 : 128;
+    j2.n_tiles = 1;
+    j2.ncols = 2 * r;
+    j2.fold = r;
+    j2.outs[0] = RankOut{m.dL2, nullptr, 1, N, 0, 1.f, f32 ? 1 : 0};
+  }
+  for (int sidx = 0; sidx < L.nsets; ++sidx) {
+    const int first = L.set_first[sidx], n = L.set_size[sidx];
+    const BwdMember &m0 = mem[first];
+    const int64_t K = m0.W->k_in;
+    const int r = m0.r;
+    const bool joint = 2 * r == 64 || 2 * r == 128;   // n-tile t = member t's [hi | lo]
+    int members[kMaxGroup], k = 0;
+    for (int i = 0; i < count; ++i)
+      if (L.set_of[i] == sidx) members[k++] = i;
+    if (joint) {
+      RankJob &j = J.l1[J.nl1++];   // dL1 = X^T [G_hi | G_lo] of every member of the set
+      j.A = {m0.X, K, M, K, 1};
+      j.B = {G + L.g_col[first], (int64_t)n * 2 * r, M, L.g_ld, 1};
+      j.bn = 2 * r;
+      j.n_tiles = n;
+      j.ncols = 2 * r;
+      j.fold = r;
+      for (int t = 0; t < n; ++t) j.outs[t] = RankOut{mem[members[t]].dL1, nullptr, r, 1, 0, mem[members[t]].keep, f32 ? 1 : 0};
+    } else {
+      for (int t = 0; t < n; ++t) {
+        const int i = members[t];
+        RankJob &j = J.l1[J.nl1++];
+        j.A = {m0.X, K, M, K, 1};
+        j.B = {G + L.g_col[i], 2 * r, M, L.g_ld, 1};
+        j.bn = 64;
+        j.n_tiles = 1;
+        j.ncols = 2 * r;
+        j.fold = r;
+        j.outs[0] = RankOut{mem[i].dL1, nullptr, r, 1, 0, mem[i].keep, f32 ? 1 : 0};
+      }
+    }
+  }
+}
+
+BwdGroupLayout bwd_group_layout(int64_t M, const BwdMember *mem, int count, int sms) {
+  BwdGroupLayout L;
+  // X sets, in order of first appearance
+  for (int i = 0; i < count; ++i) {
+    int s = -1;
+    for (int k = 0; k < L.nsets && s < 0; ++k) {
+      const BwdMember &f = mem[L.set_first[k]];
+      if (f.X == mem[i].X && f.W->k_in == mem[i].W->k_in && f.r == mem[i].r && f.keep == mem[i].keep) s = k;
+    }
+    if (s < 0) {
+      s = L.nsets++;
+      L.set_first[s] = i;
+    }
+    L.set_of[i] = s;
+    ++L.set_size[s];
+  }
+  int64_t col = 0;
+  for (int s = 0; s < L.nsets; ++s)
+    for (int i = 0; i < count; ++i)
+      if (L.set_of[i] == s) {
+        L.g_col[i] = col;
+        col += 2 * mem[i].r;
+      }
+  L.g_ld = col;
+  size_t t_bytes = 0, w_bytes = 0;
+  for (int i = 0; i < count; ++i) {
+    L.t_off[i] = t_bytes;
+    t_bytes += align_up((size_t)M * 2 * mem[i].r * 2);
+    w_bytes = std::max(w_bytes, (size_t)mem[i].W->n_out * mem[i].W->k_in * 2);
+  }
+  L.g = 0;
+  L.t = align_up((size_t)M * L.g_ld * 2);
+  L.w_hat = L.t + t_bytes;
+  L.part = L.w_hat + align_up(w_bytes);
+  // T space for every member: the size does not depend on which T_saved are given
+  BwdGroupJobs J;
+  bwd_group_jobs(M, mem, count, L, nullptr, false, true, J);
+  size_t pb = 0;
+  for (int i = 0; i < J.nt; ++i) pb = std::max(pb, rank_part_bytes(&J.t[i], 1, sms));   // one launch each
+  pb = std::max(pb, rank_part_bytes(J.gl2, J.ngl2, sms));
+  pb = std::max(pb, rank_part_bytes(J.l1, J.nl1, sms));
+  L.total = L.part + pb;
+  return L;
+}
+
+// The backward of linears whose rank products run grouped (rank_group_ok):
+// [T of members without T_saved] -> G and dL2 of all -> dL1 per X set ->
+// per member doubleDequant and dX = dY W_hat + G_hi L1^T.
+// With LoRA dropout (`drop`, a group of one whose X is the masked input) the
+// adapter term of dX goes through the mask as in bwd_large.
+int bwd_group_large(int64_t M, const BwdMember *mem, int count, bool f32, uint8_t *w8, const BwdGroupLayout &L,
+                    DeviceInfo *dev, cudaStream_t st, const BwdDropout *drop = nullptr) {
+  if (drop && count != 1) return QLORA_ERR_UNSUPPORTED_SHAPE;
+  BwdGroupJobs J;
+  bwd_group_jobs(M, mem, count, L, w8, f32, false, J);
+  uint8_t *part = w8 + L.part;
+  int rc;
+  for (int i = 0; i < J.nt; ++i) {   // a member without T_saved: recompute it alone
+    rc = rank_launch(&J.t[i], 1, part, dev, st, QLORA_KERNEL_GEMM_T);
+    if (rc) return rc;
+  }
+  rc = rank_launch(J.gl2, J.ngl2, part, dev, st, QLORA_KERNEL_RANK_G_DL2);
+  if (rc) return rc;
+  rc = rank_launch(J.l1, J.nl1, part, dev, st, QLORA_KERNEL_RANK_DL1);
+  if (rc) return rc;
+  __nv_bfloat16 *w_hat = reinterpret_cast<__nv_bfloat16 *>(w8 + L.w_hat);
+  const uint16_t *G = reinterpret_cast<const uint16_t *>(w8 + L.g);
+  for (int i = 0; i < count; ++i) {
+    const BwdMember &m = mem[i];
+    if (!m.dX) continue;
+    const int64_t N = m.W->n_out, K = m.W->k_in;
+    rc = dequant_launch(m.W, w_hat, st, dev->sms);
+    if (rc) return rc;
+    const Operand g_hi = {G + L.g_col[i], M, m.r, L.g_ld, 0};
+    const Operand l1t = {m.L1, K, m.r, m.r, 0};
+    if (!drop) {
+      GemmSeg sX[2] = {{{m.dY, M, N, N, 0}, {w_hat, K, N, K, 1}}, {g_hi, l1t}};
+      rc = tc_gemm(st, dev, M, K, 2, sX, 1.f, m.dX, K, 1, 0, nullptr, QLORA_KERNEL_GEMM_DX);
+    } else if (M > kBM && K > 128 && N >= 128 && N % 64 == 0) {
+      // the masked adapter term in the pair tile's second accumulator
+      GemmSeg sX[2] = {{{m.dY, M, N, N, 0}, {w_hat, K, N, K, 1}}, {g_hi, l1t}};
+      const GemmAddend add = {nullptr, drop->mask, drop->keep, K};
+      rc = tc_gemm(st, dev, M, K, 2, sX, 1.f, m.dX, K, 1, 0, nullptr, QLORA_KERNEL_GEMM_DX, 0, false, 0, &add);
+    } else {
+      GemmSeg sZ = {g_hi, l1t};
+      rc = tc_gemm(st, dev, M, K, 1, &sZ, 1.f, drop->Z, K, 1, 0, nullptr, QLORA_KERNEL_GEMM_Z);
+      if (rc) return rc;
+      GemmSeg sX = {{m.dY, M, N, N, 0}, {w_hat, K, N, K, 1}};
+      const GemmAddend add = {drop->Z, drop->mask, drop->keep, K};
+      rc = tc_gemm(st, dev, M, K, 1, &sX, 1.f, m.dX, K, 1, 0, nullptr, QLORA_KERNEL_GEMM_DX, 0, false, 0, &add);
+    }
+    if (rc) return rc;
+  }
+  return QLORA_OK;
+}
+
 // Xm = X * m into the workspace.
 int dropout_launch(const uint16_t *X, const uint32_t *mask, int64_t numel, uint16_t *Xm, DeviceInfo *dev,
                    cudaStream_t st) {
@@ -1089,6 +1501,14 @@ size_t qlora_linear_bwd_workspace_size(int64_t M, int64_t n_out, int64_t k_in, i
   if (M < 0 || n_out <= 0 || k_in <= 0 || r <= 0) return 0;
   DeviceInfo *dev;
   const int sms = current_device_info(&dev) == QLORA_OK ? dev->sms : 148;
+  if (M > 0 && rank_group_ok(r)) {   // the single-linear backward runs as a group of one
+    qlora_nf4dq_t w;
+    std::memset(&w, 0, sizeof(w));
+    w.n_out = n_out;
+    w.k_in = k_in;
+    const BwdMember m = {nullptr, nullptr, nullptr, &w, nullptr, nullptr, r, 1.f, nullptr, nullptr, nullptr};
+    return bwd_group_layout(M, &m, 1, sms).total;
+  }
   return bwd_layout(M, n_out, k_in, r, sms).total;
 }
 
@@ -1362,11 +1782,103 @@ int qlora_linear_bwd(const uint16_t *dY, const uint16_t *X, const uint16_t *T_sa
     if (cudaMemsetAsync(dL2, 0, (size_t)r * N * gsz, st) != cudaSuccess) return QLORA_ERR_CUDA;
     return QLORA_OK;
   }
+  if (rank_group_ok(r)) {   // a group of one: G and dL2 in one launch, then dL1
+    const BwdMember m = {dY, X, T_saved, W, L1, L2, r, s, dX, dL1, dL2};
+    const BwdGroupLayout L = bwd_group_layout(M, &m, 1, dev->sms);
+    if (!ws || ws_bytes < L.total) return QLORA_ERR_WORKSPACE;
+    if (!aligned(ws, 256)) return QLORA_ERR_MISALIGNED;
+    return bwd_group_large(M, &m, 1, grad_dtype == QLORA_DTYPE_F32, reinterpret_cast<uint8_t *>(ws), L, dev, st);
+  }
   const BwdLayout L = bwd_layout(M, N, K, r, dev->sms);
   if (!ws || ws_bytes < L.total) return QLORA_ERR_WORKSPACE;
   if (!aligned(ws, 256)) return QLORA_ERR_MISALIGNED;
   return bwd_large(dY, X, T_saved, M, W, L1, L2, r, s, dX, dL1, dL2, grad_dtype == QLORA_DTYPE_F32,
                    reinterpret_cast<uint8_t *>(ws), L, nullptr, dev, st);
+}
+
+static int check_bwd_member(const qlora_bwd_member_t &m, int64_t M) {
+  int rc = check_linear(M, m.W, m.r);
+  if (rc) return rc;
+  if (!m.L1 || !m.L2 || !m.dL1 || !m.dL2) return QLORA_ERR_INVALID_ARG;
+  if (M > 0 && (!m.dY || !m.X)) return QLORA_ERR_INVALID_ARG;
+  if (!aligned(m.L1, 16) || !aligned(m.L2, 16) || !aligned(m.dL1, 16) || !aligned(m.dL2, 16) ||
+      (m.dY && !aligned(m.dY, 16)) || (m.X && !aligned(m.X, 16)) || (m.dX && !aligned(m.dX, 16)) ||
+      (m.T_saved && !aligned(m.T_saved, 16)))
+    return QLORA_ERR_MISALIGNED;
+  return QLORA_OK;
+}
+
+static BwdMember bwd_member(const qlora_bwd_member_t &m) {
+  return BwdMember{m.dY, m.X, m.T_saved, m.W, m.L1, m.L2, m.r, m.s, m.dX, m.dL1, m.dL2};
+}
+
+// Grouped members first (one layout), the others one at a time after them.
+static size_t bwd_group_ws(int64_t M, const qlora_bwd_member_t *members, int count, int sms) {
+  BwdMember grp[kMaxGroup];
+  int ng = 0;
+  size_t other = 0;
+  for (int i = 0; i < count; ++i) {
+    const qlora_bwd_member_t &m = members[i];
+    if (rank_group_ok(m.r)) grp[ng++] = bwd_member(m);
+    else other = std::max(other, bwd_layout(M, m.W->n_out, m.W->k_in, m.r, sms).total);
+  }
+  return std::max(other, ng ? bwd_group_layout(M, grp, ng, sms).total : (size_t)0);
+}
+
+size_t qlora_linear_bwd_group_workspace_size(const qlora_bwd_member_t *members, int count, int64_t M) {
+  if (M < 0 || count < 0 || count > QLORA_MAX_GROUP || (count > 0 && !members)) return 0;
+  for (int i = 0; i < count; ++i)
+    if (!members[i].W || members[i].W->n_out <= 0 || members[i].W->k_in <= 0 || members[i].r <= 0) return 0;
+  if (M == 0) return 0;
+  DeviceInfo *dev;
+  const int sms = current_device_info(&dev) == QLORA_OK ? dev->sms : 148;
+  return bwd_group_ws(M, members, count, sms);
+}
+
+int qlora_linear_bwd_group(const qlora_bwd_member_t *members, int count, int64_t M, int grad_dtype, void *ws,
+                           size_t ws_bytes, void *stream) {
+  if (count < 0 || count > QLORA_MAX_GROUP || (count > 0 && !members) || M < 0) return QLORA_ERR_INVALID_ARG;
+  if (grad_dtype != QLORA_DTYPE_F32 && grad_dtype != QLORA_DTYPE_BF16) return QLORA_ERR_INVALID_ARG;
+  for (int i = 0; i < count; ++i) {
+    const int rc = check_bwd_member(members[i], M);
+    if (rc) return rc;
+  }
+  if (count == 0) return QLORA_OK;
+  DeviceInfo *dev;
+  int rc = current_device_info(&dev);
+  if (rc) return rc;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const bool f32 = grad_dtype == QLORA_DTYPE_F32;
+  if (M == 0) {  // no tokens: the adapter gradients are zero
+    const size_t gsz = f32 ? 4 : 2;
+    for (int i = 0; i < count; ++i) {
+      const qlora_bwd_member_t &m = members[i];
+      if (cudaMemsetAsync(m.dL1, 0, (size_t)m.W->k_in * m.r * gsz, st) != cudaSuccess) return QLORA_ERR_CUDA;
+      if (cudaMemsetAsync(m.dL2, 0, (size_t)m.r * m.W->n_out * gsz, st) != cudaSuccess) return QLORA_ERR_CUDA;
+    }
+    return QLORA_OK;
+  }
+  if (!ws || ws_bytes < bwd_group_ws(M, members, count, dev->sms)) return QLORA_ERR_WORKSPACE;
+  if (!aligned(ws, 256)) return QLORA_ERR_MISALIGNED;
+  uint8_t *w8 = reinterpret_cast<uint8_t *>(ws);
+  BwdMember grp[kMaxGroup];
+  int ng = 0;
+  for (int i = 0; i < count; ++i)
+    if (rank_group_ok(members[i].r)) grp[ng++] = bwd_member(members[i]);
+  if (ng) {
+    const BwdGroupLayout L = bwd_group_layout(M, grp, ng, dev->sms);
+    rc = bwd_group_large(M, grp, ng, f32, w8, L, dev, st);
+    if (rc) return rc;
+  }
+  for (int i = 0; i < count; ++i) {
+    const qlora_bwd_member_t &m = members[i];
+    if (rank_group_ok(m.r)) continue;
+    const BwdLayout L = bwd_layout(M, m.W->n_out, m.W->k_in, m.r, dev->sms);
+    rc = bwd_large(m.dY, m.X, m.T_saved, M, m.W, m.L1, m.L2, m.r, m.s, m.dX, m.dL1, m.dL2, f32, w8, L, nullptr,
+                   dev, st);
+    if (rc) return rc;
+  }
+  return QLORA_OK;
 }
 
 // ---------------------------------------------------------------- LoRA dropout
@@ -1379,11 +1891,25 @@ size_t qlora_linear_fwd_dropout_workspace_size(int64_t M, int64_t n_out, int64_t
   return fwd_layout(M, n_out, k_in, r, sms).total + align_up((size_t)M * k_in * 2);
 }
 
+// The backward's own layout (that of a group of one where the rank-r products
+// run grouped), then Xm [M x K] and Z [M x K] bf16.
+static size_t bwd_dropout_base(int64_t M, int64_t n_out, int64_t k_in, int r, int sms) {
+  if (M > 0 && rank_group_ok(r)) {
+    qlora_nf4dq_t w;
+    std::memset(&w, 0, sizeof(w));
+    w.n_out = n_out;
+    w.k_in = k_in;
+    BwdMember m = {nullptr, nullptr, nullptr, &w, nullptr, nullptr, r, 1.f, nullptr, nullptr, nullptr};
+    return bwd_group_layout(M, &m, 1, sms).total;
+  }
+  return bwd_layout(M, n_out, k_in, r, sms).total;
+}
+
 size_t qlora_linear_bwd_dropout_workspace_size(int64_t M, int64_t n_out, int64_t k_in, int r) {
   if (M < 0 || n_out <= 0 || k_in <= 0 || r <= 0) return 0;
   DeviceInfo *dev;
   const int sms = current_device_info(&dev) == QLORA_OK ? dev->sms : 148;
-  return bwd_layout(M, n_out, k_in, r, sms).total + 2 * align_up((size_t)M * k_in * 2);
+  return bwd_dropout_base(M, n_out, k_in, r, sms) + 2 * align_up((size_t)M * k_in * 2);
 }
 
 int qlora_linear_fwd_dropout(const uint16_t *X, int64_t M, const qlora_nf4dq_t *W, const uint16_t *L1,
@@ -1437,21 +1963,28 @@ int qlora_linear_bwd_dropout(const uint16_t *dY, const uint16_t *X, const uint16
     if (cudaMemsetAsync(dL2, 0, (size_t)r * N * gsz, st) != cudaSuccess) return QLORA_ERR_CUDA;
     return QLORA_OK;
   }
-  const BwdLayout L = bwd_layout(M, N, K, r, dev->sms);
-  if (!ws || ws_bytes < qlora_linear_bwd_dropout_workspace_size(M, N, K, r)) return QLORA_ERR_WORKSPACE;
+  const size_t base = bwd_dropout_base(M, N, K, r, dev->sms);
+  if (!ws || ws_bytes < base + 2 * align_up((size_t)M * K * 2)) return QLORA_ERR_WORKSPACE;
   if (!aligned(ws, 256)) return QLORA_ERR_MISALIGNED;
   uint8_t *w8 = reinterpret_cast<uint8_t *>(ws);
-  uint16_t *Z = reinterpret_cast<uint16_t *>(w8 + L.total + align_up((size_t)M * K * 2));
+  uint16_t *Z = reinterpret_cast<uint16_t *>(w8 + base + align_up((size_t)M * K * 2));
   const uint16_t *Xm = Xm_saved;
   if (!Xm) {   // recompute the masked input
-    uint16_t *Xw = reinterpret_cast<uint16_t *>(w8 + L.total);
+    uint16_t *Xw = reinterpret_cast<uint16_t *>(w8 + base);
     rc = dropout_launch(X, mask, M * K, Xw, dev, st);
     if (rc) return rc;
     Xm = Xw;
   }
   const BwdDropout drop = {Xm, 1.f / (1.f - p), mask, Z};
-  return bwd_large(dY, X, T_saved, M, W, L1, L2, r, s, dX, dL1, dL2, grad_dtype == QLORA_DTYPE_F32, w8, L, &drop,
-                   dev, st);
+  const bool f32 = grad_dtype == QLORA_DTYPE_F32;
+  if (rank_group_ok(r)) {   // the rank-r products as in the plain backward, on the masked input
+    BwdMember m = {dY, Xm, T_saved, W, L1, L2, r, s, dX, dL1, dL2};
+    m.keep = drop.keep;
+    const BwdGroupLayout L = bwd_group_layout(M, &m, 1, dev->sms);
+    return bwd_group_large(M, &m, 1, f32, w8, L, dev, st, &drop);
+  }
+  const BwdLayout L = bwd_layout(M, N, K, r, dev->sms);
+  return bwd_large(dY, X, T_saved, M, W, L1, L2, r, s, dX, dL1, dL2, f32, w8, L, &drop, dev, st);
 }
 
 }  // extern "C"

@@ -257,6 +257,44 @@ QLORA_API int qlora_linear_fwd_group(const qlora_fwd_member_t *members, int coun
                                      size_t ws_bytes, void *stream);
 
 /*
+ * Grouped backward: the backward of up to QLORA_MAX_GROUP linears whose output
+ * gradients are available together (a layer's q, k and v after the attention
+ * backward; gate and up after the SwiGLU backward), each computing exactly
+ * what qlora_linear_bwd computes (same formulas, layouts and shape rules, all
+ * members on the same M tokens).  For members with r in {8, 16, 32, 64}:
+ *   - G and dL2 of all of them run as one launch of the grouped rank-r
+ *     kernel, dL1 as a second one, where members that read the same X (same
+ *     pointer, k_in and r) share one pass over X;
+ *   - then each member's doubleDequant and dX = dY W_hat + G_hi L1^T.
+ * Members with other ranks run the single-linear backward one after another.
+ * Split reductions are summed in a fixed order: results are reproducible run
+ * to run, but may differ in the last bits from a call on a different group
+ * (a different split of the same reduction).
+ * Outputs of different members must not overlap each other or any input.
+ * Workspace: qlora_linear_bwd_group_workspace_size() bytes (the same members
+ * and M; independent of which T_saved are NULL), 256-byte aligned.
+ * Errors: as qlora_linear_bwd, for the first failing member; QLORA_ERR_INVALID_ARG
+ * for count outside [0, QLORA_MAX_GROUP] or a NULL member array with count > 0.
+ */
+typedef struct {
+  const uint16_t *dY;         /* [M x n_out] bf16 */
+  const uint16_t *X;          /* [M x k_in] bf16 */
+  const uint16_t *T_saved;    /* [M x 2r] bf16 hi/lo pair from the forward, or NULL to recompute */
+  const qlora_nf4dq_t *W;
+  const uint16_t *L1;         /* [k_in x r] bf16 */
+  const uint16_t *L2;         /* [r x n_out] bf16 */
+  int r;
+  float s;
+  uint16_t *dX;               /* [M x k_in] bf16, written; or NULL to skip */
+  void *dL1;                  /* [k_in x r], grad_dtype, written */
+  void *dL2;                  /* [r x n_out], grad_dtype, written */
+} qlora_bwd_member_t;
+
+QLORA_API size_t qlora_linear_bwd_group_workspace_size(const qlora_bwd_member_t *members, int count, int64_t M);
+QLORA_API int qlora_linear_bwd_group(const qlora_bwd_member_t *members, int count, int64_t M, int grad_dtype,
+                                     void *ws, size_t ws_bytes, void *stream);
+
+/*
  * LoRA dropout (QLoRA Appendix B.2 trains with LoRA dropout, p = 0.1 up to
  * 13B and 0.05 at 33B and 65B).  It acts on the adapter's input only:
  *   Y  = X W_hat^T + T L2,   T = s drop(X) L1,   drop(X) = X * m / (1 - p);
@@ -346,6 +384,8 @@ QLORA_API int qlora_get_last_device_error(void *stream);
 #define QLORA_KERNEL_GEMM_DL2 14    /* dL2 = T^T dY */
 #define QLORA_KERNEL_GEMM_DL1 15    /* dL1 = X^T G */
 #define QLORA_KERNEL_GEMM_Z 16      /* Z = G L1^T (dropout backward) */
+#define QLORA_KERNEL_RANK_G_DL2 17  /* G = s dY L2^T and dL2 = T^T dY of every linear of a backward, one launch */
+#define QLORA_KERNEL_RANK_DL1 18    /* dL1 = X^T G of every linear of a backward, one launch */
 #define QLORA_KERNEL_SPLITK_FINALIZE 20
 #define QLORA_KERNEL_FUSED_FWD 31   /* few-token forward chain (up to 128 tokens): T, fused decode + tcgen05 product, LoRA epilogue */
 #define QLORA_KERNEL_DROPOUT_MASK 40 /* Xm = X * m (LoRA dropout) */

@@ -143,3 +143,29 @@ def test_config3_full_size_sampled():
         assert np.array_equal(got_bits, ref_bits)
         del Wd, q, w_hat
     assert qlora.last_device_error() == 0
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("dtype,shape", [(torch.float32, (4096, 4096)), (torch.bfloat16, (8192, 4096))])
+def test_streamed_ring_reuse_repeated(dtype, shape):
+    """Weights large enough that every CTA of the quantizer refills each slot of
+    its shared-memory ring many times (fp32 16.7 M and bf16 33.5 M weights
+    against 148 CTAs of 5 and 10 slots of 8192 weights), quantized repeatedly:
+    bit-exact every time.  A refill that overtook the reads of a slot gave a
+    few groups the codes of the chunk five slots later."""
+    g = inputs.rng(4242 + shape[0])
+    W = torch.from_numpy(inputs.weight_f32(g, *shape)).to(dtype)
+    oq = oracle_quant(W)
+    Wd = W.cuda()
+    for _ in range(4):
+        q = qlora.quantize_nf4_dq(Wd)
+        got = gpu_quant_to_np(q)
+        assert got["mu"] == oq["mu"]
+        assert np.array_equal(got["packed"], oq["packed"])
+        assert np.array_equal(got["c2_fp8"], oq["c2_fp8"])
+        assert np.array_equal(got["c1"].view(np.uint32), oq["c1"].view(np.uint32))
+    ref_bits = nf4dq.double_dequant_bits(oq["codes"], oq["c2_fp8"], oq["c1"], oq["mu"], oq["shape"])
+    for _ in range(3):
+        got_bits = qlora.dequant(q).cpu().view(torch.int16).numpy().view(np.uint16)
+        assert np.array_equal(got_bits, ref_bits)
+    assert qlora.last_device_error() == 0
