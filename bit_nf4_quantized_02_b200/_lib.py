@@ -32,7 +32,7 @@ KERNEL_KINDS = {
     1: "quantize", 2: "dq_constants", 3: "dequant",
     10: "gemm_T", 11: "gemm_Y", 12: "gemm_G", 13: "gemm_dX", 14: "gemm_dL2", 15: "gemm_dL1", 16: "gemm_Z",
     17: "rank_G_dL2", 18: "rank_dL1",
-    20: "splitk_finalize", 31: "fused_fwd", 40: "dropout_mask", 41: "t_scatter",
+    20: "splitk_finalize", 31: "fused_fwd", 40: "dropout_mask",
 }
 
 

@@ -21,7 +21,7 @@ LIB_NAME = "libqlora.so"
 LIB_PATH = os.path.join(PKG_DIR, LIB_NAME)
 
 SOURCES = ["qlora.cu"]
-DEPENDS = ["qlora.cu", "common.cuh", "quant.cuh", "tc_gemm.cuh", "few_token.cuh", "decode_fwd.cuh", "dropout.cuh", "group.cuh"]
+DEPENDS = ["qlora.cu", "common.cuh", "quant.cuh", "tc_gemm.cuh", "few_token.cuh", "decode_fwd.cuh", "dropout.cuh", "rank_gemm.cuh"]
 
 NVCC_FLAGS = [
     "-O3",

@@ -69,10 +69,10 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t byt
 
 // Proxy fence for shared memory.  A stage that threads read with ordinary
 // loads (the generic proxy) and that a bulk or tensor copy (the async proxy)
-// then refills needs one on each side: the readers issue it after their loads
-// and before they release the stage (so the loads have completed), and the
-// copying thread issues it after it has seen the release and before the copy.
-// Without them a refill was seen to overtake reads still in flight.
+// then refills: the mbarrier (or bar.sync) release/acquire orders the reads
+// before the copying thread's later accesses in the generic proxy only, so
+// that thread issues this fence after it has seen the release and before the
+// copy.  Without it a refill was seen to overtake reads still in flight.
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }

@@ -425,7 +425,6 @@ __global__ void __launch_bounds__(DfCfg<MP>::kThreads, 1)
       uint4 qv[8];
 #pragma unroll
       for (int c = 0; c < 8; ++c) qv[c] = lds128(sc + (((uint32_t)c << 4) ^ cswz));
-      fence_proxy_async_smem();   // the loads complete before the slot is released
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(cempty_bar + cs));
       // the MMAs of this group's previous item (rel - G) have read its A

@@ -17,7 +17,6 @@
 #include "few_token.cuh"
 #include "decode_fwd.cuh"
 #include "dropout.cuh"
-#include "group.cuh"
 #include "rank_gemm.cuh"
 
 namespace qlora {
@@ -648,6 +647,20 @@ int rank_launch(const RankJob *jobs, int n, uint8_t *part, DeviceInfo *dev, cuda
   return launch_pdl(rank_finalize_kernel, dim3(fgrid), dim3(256), 0, st, fin);
 }
 
+// The adapter's down-projection T = alpha Xt L1 (L1 read MN-major) as a bf16
+// hi/lo pair [M x 2r], as one problem of the rank kernel (r <= 128).
+RankJob t_job(const uint16_t *Xt, int64_t M, int64_t K, const uint16_t *L1, int r, float alpha, uint16_t *T) {
+  RankJob j;
+  j.A = {Xt, M, K, K, 0};
+  j.B = {L1, r, K, r, 1};
+  j.bn = r <= 64 ? 64 : 128;
+  j.n_tiles = 1;
+  j.ncols = r;
+  j.fold = 0;
+  j.outs[0] = RankOut{T, nullptr, 2 * r, 1, r, alpha, 0};
+  return j;
+}
+
 int dequant_launch(const qlora_nf4dq_t *W, __nv_bfloat16 *out, cudaStream_t st, int sms) {
   const int64_t numel = W->n_out * W->k_in;
   if (numel == 0) return QLORA_OK;
@@ -877,7 +890,12 @@ FwdLayout fwd_layout(int64_t M, int64_t N, int64_t K, int r, int sms) {
   L.w_hat = 0;
   L.t = align_up((size_t)N * K * 2);
   L.split = L.t + align_up((size_t)M * 2 * r * 2);
-  L.total = L.split + gemm_split_ws_bytes(M, r, K, sms, true);
+  size_t part = gemm_split_ws_bytes(M, r, K, sms, true);
+  if (r <= 128) {
+    const RankJob tj = t_job(nullptr, M, K, nullptr, r, 1.f, nullptr);
+    part = std::max(part, rank_part_bytes(&tj, 1, sms));
+  }
+  L.total = L.split + part;
   return L;
 }
 
@@ -1178,8 +1196,13 @@ int fwd_large(const uint16_t *X, const uint16_t *Xt, float t_scale, int64_t M, c
   if (rc) return rc;
   // 2. T = s X L1 (the adapter's down-projection; L1 read MN-major), stored
   //    as a bf16 hi/lo pair [M x 2r]: T ~= T[:, :r] + T[:, r:].
-  GemmSeg sT = {{Xt, M, K, K, 0}, {L1, r, K, r, 1}};
-  rc = tc_gemm(st, dev, M, r, 1, &sT, t_scale, T, 2 * r, 1, 0, split_ws, QLORA_KERNEL_GEMM_T, r);
+  if (r <= 128) {
+    const RankJob tj = t_job(Xt, M, K, L1, r, t_scale, T);
+    rc = rank_launch(&tj, 1, reinterpret_cast<uint8_t *>(split_ws), dev, st, QLORA_KERNEL_GEMM_T);
+  } else {
+    GemmSeg sT = {{Xt, M, K, K, 0}, {L1, r, K, r, 1}};
+    rc = tc_gemm(st, dev, M, r, 1, &sT, t_scale, T, 2 * r, 1, 0, split_ws, QLORA_KERNEL_GEMM_T, r);
+  }
   if (rc) return rc;
   // 3. Y = X W_hat^T + T_hi L2 (the LoRA up-projection as extra K-steps).
   GemmSeg sY[2] = {{{X, M, K, K, 0}, {w_hat, N, K, K, 0}}, {{T, M, r, 2 * r, 0}, {L2, N, r, N, 1}}};
@@ -1563,36 +1586,74 @@ static int x_sets(const FwdMember *mem, int count, int *set_of) {
 // each member's T pair [M x 2r] (used where it passes no T_save); the split-K
 // partials of the largest adapter product.
 struct GroupLargeLayout {
-  size_t w_hat, t_cat, l1_cat, t_own[kMaxGroup], split, total;
+  size_t w_hat, l1_cat, t_own[kMaxGroup], split, total;
 };
+
+// The adapter down-projections of the members of one X set (same input
+// pointer and K) as problems of one rank launch: with equal ranks of 64 or 128
+// one problem over L1_cat = [L1_a | L1_b | ...] whose n-tile k is member k
+// (each 128-row strip of X is read for all members on neighbouring CTAs),
+// otherwise one problem per member.  Returns false when a rank is above 128.
+static bool fwd_set_jobs(int64_t M, const FwdMember *mem, const int *idx, int n, uint16_t *const *T,
+                         const uint16_t *l1_cat, RankJob *jobs, int *njobs, bool *joint) {
+  const FwdMember &m0 = mem[idx[0]];
+  const int64_t K = m0.W->k_in;
+  bool same = true;
+  for (int k = 0; k < n; ++k) {
+    if (mem[idx[k]].r > 128) return false;
+    same = same && mem[idx[k]].r == m0.r;
+  }
+  *joint = same && n > 1 && (m0.r == 64 || m0.r == 128);
+  if (*joint) {
+    RankJob &j = jobs[0];
+    j.A = {m0.X, M, K, K, 0};
+    j.B = {l1_cat, (int64_t)n * m0.r, K, (int64_t)n * m0.r, 1};
+    j.bn = m0.r;
+    j.n_tiles = n;
+    j.ncols = m0.r;
+    j.fold = 0;
+    for (int k = 0; k < n; ++k) j.outs[k] = RankOut{T[k], nullptr, 2 * m0.r, 1, m0.r, mem[idx[k]].s, 0};
+    *njobs = 1;
+  } else {
+    for (int k = 0; k < n; ++k) {
+      const FwdMember &m = mem[idx[k]];
+      jobs[k] = t_job(m.X, M, K, m.L1, m.r, m.s, T[k]);
+    }
+    *njobs = n;
+  }
+  return true;
+}
 
 static GroupLargeLayout group_large_layout(int64_t M, const FwdMember *mem, int count, int sms) {
   int set_of[kMaxGroup];
   const int nsets = x_sets(mem, count, set_of);
-  size_t w = 0, tcat = 0, l1cat = 0, split = 0;
+  size_t w = 0, l1cat = 0, split = 0;
   for (int i = 0; i < count; ++i) w = std::max(w, (size_t)mem[i].W->n_out * mem[i].W->k_in * 2);
   for (int s = 0; s < nsets; ++s) {
-    int64_t R = 0, K = 0;
-    int members = 0;
+    int idx[kMaxGroup], n = 0;
     for (int i = 0; i < count; ++i)
-      if (set_of[i] == s) {
-        R += mem[i].r;
-        K = mem[i].W->k_in;
-        ++members;
-        split = std::max(split, gemm_split_ws_bytes(M, mem[i].r, K, sms, true));
+      if (set_of[i] == s) idx[n++] = i;
+    int64_t R = 0;
+    for (int k = 0; k < n; ++k) R += mem[idx[k]].r;
+    uint16_t *T[kMaxGroup] = {};
+    RankJob jobs[kMaxGroup];
+    int nj = 0;
+    bool joint = false;
+    if (n > 1 && fwd_set_jobs(M, mem, idx, n, T, nullptr, jobs, &nj, &joint)) {
+      split = std::max(split, rank_part_bytes(jobs, nj, sms));
+      if (joint) l1cat = std::max(l1cat, (size_t)mem[idx[0]].W->k_in * R * 2);
+    } else {
+      for (int k = 0; k < n; ++k) {
+        const FwdMember &m = mem[idx[k]];
+        const FwdLayout FL = fwd_layout(M, m.W->n_out, m.W->k_in, m.r, sms);
+        split = std::max(split, FL.total - FL.split);
       }
-    if (members > 1) {
-      tcat = std::max(tcat, (size_t)M * R * 4);
-      l1cat = std::max(l1cat, (size_t)K * R * 2);
-      split = std::max(split, gemm_split_ws_bytes(M, R, K, sms, true));
     }
   }
   GroupLargeLayout L;
   size_t off = 0;
   L.w_hat = off;
   off += align_up(w);
-  L.t_cat = off;
-  off += align_up(tcat);
   L.l1_cat = off;
   off += align_up(l1cat);
   for (int i = 0; i < count; ++i) {
@@ -1606,13 +1667,13 @@ static GroupLargeLayout group_large_layout(int64_t M, const FwdMember *mem, int 
 }
 
 // The grouped forward at many tokens (M > 128) on a workspace laid out by
-// group_large_layout.
+// group_large_layout: per X set one rank launch for the members' T, then each
+// member's doubleDequant and Y product.
 static int group_large_fwd(int64_t M, const FwdMember *mem, int count, uint8_t *w8, const GroupLargeLayout &L,
                            DeviceInfo *dev, cudaStream_t st) {
   int set_of[kMaxGroup];
   const int nsets = x_sets(mem, count, set_of);
   __nv_bfloat16 *w_hat = reinterpret_cast<__nv_bfloat16 *>(w8 + L.w_hat);
-  float *split_ws = reinterpret_cast<float *>(w8 + L.split);
   for (int s = 0; s < nsets; ++s) {
     int idx[kMaxGroup], n = 0;
     for (int i = 0; i < count; ++i)
@@ -1623,54 +1684,33 @@ static int group_large_fwd(int64_t M, const FwdMember *mem, int count, uint8_t *
       T[k] = m.T_save ? m.T_save : reinterpret_cast<uint16_t *>(w8 + L.t_own[idx[k]]);
     }
     int rc;
-    if (n == 1) {
-      const FwdMember &m = mem[idx[0]];
-      FwdLayout FL;
-      FL.w_hat = L.w_hat;
-      FL.t = L.t_own[idx[0]];
-      FL.split = L.split;
-      FL.total = L.total;
-      rc = fwd_large(m.X, m.X, m.s, M, m.W, m.L1, m.L2, m.r, m.Y, m.T_save, w8, FL, dev, st);
-      if (rc) return rc;
+    uint16_t *l1_cat = reinterpret_cast<uint16_t *>(w8 + L.l1_cat);
+    RankJob jobs[kMaxGroup];
+    int nj = 0;
+    bool joint = false;
+    if (n == 1 || !fwd_set_jobs(M, mem, idx, n, T, l1_cat, jobs, &nj, &joint)) {
+      for (int k = 0; k < n; ++k) {
+        const FwdMember &m = mem[idx[k]];
+        FwdLayout FL;
+        FL.w_hat = L.w_hat;
+        FL.t = L.t_own[idx[k]];
+        FL.split = L.split;
+        FL.total = L.total;
+        rc = fwd_large(m.X, m.X, m.s, M, m.W, m.L1, m.L2, m.r, m.Y, m.T_save, w8, FL, dev, st);
+        if (rc) return rc;
+      }
       continue;
     }
-    // The shared input's adapter product: X [L1_a | L1_b | ...] into T_cat.
-    const int64_t K = mem[idx[0]].W->k_in;
-    TScatterArgs a;
-    std::memset(&a, 0, sizeof(a));
-    int R = 0;
-    uint16_t *l1_cat = reinterpret_cast<uint16_t *>(w8 + L.l1_cat);
-    for (int k = 0; k < n; ++k) {
-      const FwdMember &m = mem[idx[k]];
-      a.off[k] = R;
-      a.r[k] = m.r;
-      a.s[k] = m.s;
-      a.T[k] = reinterpret_cast<__nv_bfloat16 *>(T[k]);
-      R += m.r;
+    if (joint) {   // L1_cat [K x n r]: member k's L1 [K x r] in columns k r .. k r + r
+      const int64_t K = mem[idx[0]].W->k_in;
+      const int r = mem[idx[0]].r;
+      for (int k = 0; k < n; ++k)
+        if (cudaMemcpy2DAsync(l1_cat + (int64_t)k * r, (size_t)n * r * 2, mem[idx[k]].L1, (size_t)r * 2,
+                              (size_t)r * 2, (size_t)K, cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+          return QLORA_ERR_CUDA;
     }
-    // L1_cat [K x R]: member k's L1 [K x r_k] in columns off_k .. off_k + r_k.
-    for (int k = 0; k < n; ++k) {
-      const FwdMember &m = mem[idx[k]];
-      if (cudaMemcpy2DAsync(l1_cat + a.off[k], (size_t)R * 2, m.L1, (size_t)m.r * 2, (size_t)m.r * 2, (size_t)K,
-                            cudaMemcpyDeviceToDevice, st) != cudaSuccess)
-        return QLORA_ERR_CUDA;
-    }
-    a.off[n] = R;
-    a.R = R;
-    a.M = M;
-    a.count = n;
-    float *t_cat = reinterpret_cast<float *>(w8 + L.t_cat);
-    a.t_cat = t_cat;
-    GemmSeg sT = {{mem[idx[0]].X, M, K, K, 0}, {l1_cat, R, K, R, 1}};
-    rc = tc_gemm(st, dev, M, R, 1, &sT, 1.f, t_cat, R, 1, 1, split_ws, QLORA_KERNEL_GEMM_T);
+    rc = rank_launch(jobs, nj, w8 + L.split, dev, st, QLORA_KERNEL_GEMM_T);
     if (rc) return rc;
-    {
-      const int64_t cnt = M * R;
-      const int grid = (int)std::max<int64_t>(1, std::min<int64_t>((cnt + 255) / 256, (int64_t)dev->sms * 8));
-      ProfScope prof(QLORA_KERNEL_T_SCATTER, st);
-      rc = launch_pdl(t_scatter_kernel, dim3(grid), dim3(256), 0, st, a);
-      if (rc) return rc;
-    }
     for (int k = 0; k < n; ++k) {
       const FwdMember &m = mem[idx[k]];
       rc = fwd_y(m.X, M, m.W, m.L2, m.r, T[k], m.Y, w_hat, dev, st);

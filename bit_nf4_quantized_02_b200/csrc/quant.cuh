@@ -459,7 +459,6 @@ __global__ void __launch_bounds__(kQuantThreads, 1) nf4_quantize_kernel(const TW
       if (!__all_sync(0xFFFFFFFFu, mbar_wait(smem_u32(full + st), (uint32_t)(i / S) & 1u, err, DEV_TIMEOUT_MMA))) break;
       float v[16];
       lds_unpack16<TW>(smem_u32(ring + st * Cfg::kChunkBytes) + (uint32_t)((gi * 512 + lane * 16) * (int)sizeof(TW)), v);
-      fence_proxy_async_smem();   // the loads complete before the slot is released
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(empty + st));   // this group's weights are in registers
       const int64_t g = (blockIdx.x + i * gridDim.x) * kGroupsPerChunk + gi;
@@ -666,10 +665,9 @@ __global__ void __launch_bounds__(kDqThreads, kDqCtasPerSm) nf4_dequant_kernel(
       const float c2h = __fmaf_rn(e4m3_to_f32(sc[kDqCodeBytes + (w >> 3)]), c1v, mu);
       dst[w] = dq_decode8(q, c2h, lut);
     }
-    fence_proxy_async_smem();   // this thread's loads of the stage before its refill
-    __syncthreads();            // stage st consumed by every thread
+    __syncthreads();   // stage st consumed by every thread
     if (threadIdx.x == 0 && issued < mine) {
-      fence_proxy_async_smem();
+      fence_proxy_async_smem();   // those reads before the refill's writes
       issue(issued++);
     }
   }

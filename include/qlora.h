@@ -389,7 +389,6 @@ QLORA_API int qlora_get_last_device_error(void *stream);
 #define QLORA_KERNEL_SPLITK_FINALIZE 20
 #define QLORA_KERNEL_FUSED_FWD 31   /* few-token forward chain (up to 128 tokens): T, fused decode + tcgen05 product, LoRA epilogue */
 #define QLORA_KERNEL_DROPOUT_MASK 40 /* Xm = X * m (LoRA dropout) */
-#define QLORA_KERNEL_T_SCATTER 41   /* shared-input T split into each linear's hi/lo pair (grouped forward) */
 QLORA_API int qlora_profile_start(int capacity);
 QLORA_API int qlora_profile_stop(void);
 QLORA_API int qlora_profile_read(int i, int *kind, float *ms);

@@ -252,3 +252,24 @@ def test_layer_group_mid_size_full_check():
         torch.cuda.synchronize()
         assert qlora.last_device_error() == 0
         _check([host[n] for n in grp], outs, s_of=lambda i: s)
+
+
+@pytest.mark.parametrize("r", [64, 128])
+def test_shared_input_equal_ranks_many_tokens(r):
+    """Many tokens, members on one input with equal ranks of 64 or 128: one
+    adapter product whose n-tile k is member k's L1, each T scaled on its own."""
+    M, K = 300, 320
+    g = inputs.rng(7950 + r)
+    X = inputs.normal_bf16(g, (M, K))
+    Xd = X.cuda()
+    host, dev = [], []
+    scales = [0.5, 1.0, 2.0]
+    for i, N in enumerate((136, 264, 72)):
+        W = torch.from_numpy(inputs.weight_f32(g, N, K))
+        L1, L2 = inputs.lora_factors(g, K, N, r)
+        host.append((f"m{i}", W, X, L1, L2, "nf4"))
+        dev.append({"X": Xd, "q": qlora.quantize_nf4_dq(W.cuda()), "L1": L1.cuda(), "L2": L2.cuda(), "s": scales[i]})
+    outs = qlora.linear_fwd_group(dev)
+    torch.cuda.synchronize()
+    assert qlora.last_device_error() == 0
+    _check(host, outs, s_of=lambda i: scales[i])
