@@ -311,7 +311,8 @@ def train_config(args, wl, world):
                     + (" (forward of the linears that read the same input as one grouped call: q, k, v, "
                        "gate, up on the layer input; backward grouped as the gradients arrive: down, "
                        "{gate, up}, o, {q, k, v})" if wl.layers == 1 and args.dropout == 0 else "")
-                    + (" (layer to layer: H' = bf16(down(up(H)) + R))" if wl.layers > 1 else "")
+                    + (" (layer to layer: H' = bf16(down(up(H)) + R); each layer's six linears on H as one "
+                       "grouped forward and one grouped backward)" if wl.layers > 1 else "")
                     + (", all-reduce of adapter grads" if world > 1 else "")
                     + (f", LoRA dropout p = {args.dropout:g} on every adapter (one seeded keep mask per "
                        f"linear, copied in with the inputs in e2e)" if args.dropout > 0 else ""),

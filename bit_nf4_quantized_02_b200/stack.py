@@ -2,7 +2,7 @@
 
 Every linear is an NF4 + Double-Quantization weight with a LoRA adapter
 (QLoRA, §3 Eq. 5), run forward and then backward in sequence through the
-library (quantize_nf4_dq, FwdGroup, linear_fwd, linear_bwd).
+library (quantize_nf4_dq, FwdGroup, linear_fwd, BwdGroup, linear_bwd).
 
 The pages give no model code, so the layer wiring is the plainest stack of the
 seven LLaMA linears that carries activations from layer to layer:
@@ -12,8 +12,9 @@ seven LLaMA linears that carries activations from layer to layer:
   the layer output is D = down(U).  The next layer's input is
   H' = bf16(D + R), with R a fixed N(0, 1) bf16 residual per layer;
 * backward, top to bottom: dD = dH'; dU = dX of down.  q, k, v, o and gate
-  get fixed N(0, 1) bf16 output gradients.  dH = bf16 of the fp32 sum of the
-  six dX that read H, taken in the order q, k, v, o, gate, up.
+  get fixed N(0, 1) bf16 output gradients; the six linears on H then run as
+  one grouped backward (their adapter products in two launches).  dH = bf16
+  of the fp32 sum of the six dX, taken in the order q, k, v, o, gate, up.
 
 The residual add and the gradient sum are elementwise glue outside the QLoRA
 linear, done here with torch; every linear's work runs in the library.  The
@@ -93,7 +94,10 @@ class QLoRAStack:
         # forward's members may not share an output
         self._y = {name: torch.empty(M, shapes[name][0], dtype=bf, device=device) for name in SEEDED_DY}
         self._groups, self._group_key = None, None
-        self._dx = torch.empty(M, hidden, dtype=bf, device=device)
+        self._bgroups, self._bgroup_key = None, None
+        # the dX of the six linears on H: one buffer each (a grouped backward's
+        # members may not share an output), summed into dH
+        self._dx = {name: torch.empty(M, hidden, dtype=bf, device=device) for name in READS_H}
         self._acc = torch.empty(M, hidden, dtype=torch.float32, device=device)
         # adapter gradients: views of one flat buffer (one all-reduce per step)
         order = [self.lin[l][name] for l in range(layers) for name in NAMES]
@@ -122,6 +126,19 @@ class QLoRAStack:
             self._group_key = key
         return self._groups
 
+    def _bwd_groups(self):
+        """One grouped backward per layer over the six linears that read H."""
+        key = tuple(id(self.lin[l][name].q) for l in range(self.layers) for name in READS_H)
+        if key != self._bgroup_key:
+            self._bgroups = [
+                self.ops.BwdGroup([{"dY": self.dU[l] if name == "up" else row[name].dY, "X": self.H[l],
+                                    "T": row[name].T, "q": row[name].q, "L1": row[name].L1, "L2": row[name].L2,
+                                    "s": self.s, "dX": self._dx[name], "dL1": row[name].dL1,
+                                    "dL2": row[name].dL2} for name in READS_H], grad_dtype=self.grad_dtype)
+                for l, row in enumerate(self.lin)]
+            self._bgroup_key = key
+        return self._bgroups
+
     def forward(self):
         ops, s = self.ops, self.s
         groups = self._fwd_groups()
@@ -135,20 +152,17 @@ class QLoRAStack:
 
     def backward(self):
         ops, s = self.ops, self.s
+        groups = self._bwd_groups()
         for l in reversed(range(self.layers)):
-            H, row = self.H[l], self.lin[l]
-            d = row["down"]
+            d = self.lin[l]["down"]
             ops.linear_bwd(self.dH[l + 1], self.U[l], d.T, d.q, d.L1, d.L2, s, grad_dtype=self.grad_dtype,
                            dX=self.dU[l], dL1=d.dL1, dL2=d.dL2)
+            groups[l]()          # q, k, v, o, gate and up on H[l]
             for j, name in enumerate(READS_H):
-                x = row[name]
-                dY = self.dU[l] if name == "up" else x.dY
-                ops.linear_bwd(dY, H, x.T, x.q, x.L1, x.L2, s, grad_dtype=self.grad_dtype,
-                               dX=self._dx, dL1=x.dL1, dL2=x.dL2)
                 if j == 0:
-                    self._acc.copy_(self._dx)
+                    self._acc.copy_(self._dx[name])
                 else:
-                    self._acc.add_(self._dx.float())
+                    self._acc.add_(self._dx[name].float())
             self.dH[l].copy_(self._acc)
 
     def step(self, group=None):

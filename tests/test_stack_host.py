@@ -20,7 +20,7 @@ def _np(t):
 
 
 class OracleOps:
-    """quantize_nf4_dq / linear_fwd / linear_bwd on CPU tensors via the oracle."""
+    """quantize_nf4_dq / linear_fwd / linear_bwd (and their grouped forms) on CPU tensors via the oracle."""
 
     def __init__(self):
         self.calls = []
@@ -45,6 +45,13 @@ class OracleOps:
         def run():
             return [self.linear_fwd(m["X"], m["q"], m["L1"], m["L2"], m["s"], Y=m["Y"], T=m["T"])
                     for m in members]
+        return run
+
+    def BwdGroup(self, members, grad_dtype=None):
+        """A grouped backward: each member as linear_bwd computes it, in member order."""
+        def run():
+            return [self.linear_bwd(m["dY"], m["X"], m["T"], m["q"], m["L1"], m["L2"], m["s"], dX=m["dX"],
+                                    dL1=m["dL1"], dL2=m["dL2"]) for m in members]
         return run
 
     def linear_bwd(self, dY, X, T, q, L1, L2, s, grad_dtype=None, dX=None, dL1=None, dL2=None):
