@@ -25,7 +25,7 @@ def _case(M, N, K, r, seed):
 
 
 @pytest.mark.parametrize("M", [1, 5, 8, 9, 16, 17, 32, 33, 64, 65, 100, 128])
-@pytest.mark.parametrize("N,K,r", [(72, 320, 8), (520, 1088, 64), (1032, 2048, 136), (264, 64, 16)])
+@pytest.mark.parametrize("N,K,r", [(72, 320, 8), (520, 1088, 64), (1032, 2048, 136), (264, 64, 16), (136, 1280, 16)])
 def test_few_token_forward_parity(M, N, K, r):
     W, X, L1, L2 = _case(M, N, K, r, 500 + M + N + K + r)
     s = 16.0 / r
@@ -98,14 +98,16 @@ def test_llama65b_linear_16_tokens_sampled(lin):
     assert_close(qlora.t_value(T).cpu().numpy(), T_ref, "T")
 
 
+@pytest.mark.parametrize("K", [1088, 1280])
 @pytest.mark.parametrize("M", [16, 48, 128])
 @pytest.mark.parametrize("table", ["nf4", "fp4"])
-def test_decoded_weight_is_double_dequant(M, table):
+def test_decoded_weight_is_double_dequant(M, table, K):
     """One-hot token rows pick single input features, so with L2 = 0 each
     output is one decoded weight (an fp32 sum of one product, exact in bf16):
     the few-token product decodes exactly doubleDequant's bf16 weight, bit for
-    bit, zero codes included."""
-    N, K, r = 264, 1088, 8
+    bit, zero codes included (K = 1088 ends on a stage of one 64-block, K =
+    1280 on a whole stage)."""
+    N, r = 264, 8
     g = inputs.rng(700 + M)
     W = torch.from_numpy(inputs.weight_f32(g, N, K))
     W[:, 5] = 0.0                                   # exact zeros inside nonzero blocks
