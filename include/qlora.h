@@ -193,6 +193,11 @@ QLORA_API size_t qlora_linear_bwd_workspace_size(int64_t M, int64_t n_out, int64
  *   reduction over tokens does not amplify a bf16 rounding of T.
  *   K = W->k_in (multiple of 64), N = W->n_out (multiple of 8), r a multiple of
  *   8 in [8, 256].  All products accumulate in fp32 on the tensor cores.
+ *   Reproducibility: above 128 tokens every reduction is summed in a fixed
+ *   order, so equal inputs give equal bits run to run.  At 1-128 tokens the
+ *   partial sums of Y and T over K are added with fp32 atomics (red.add), so
+ *   Y and T may differ in their last bits between runs (always within the
+ *   stated tolerance); the decoded weight itself is exact.
  */
 QLORA_API int qlora_linear_fwd(const uint16_t *X, int64_t M, const qlora_nf4dq_t *W, const uint16_t *L1, const uint16_t *L2,
                      int r, float s, uint16_t *Y, uint16_t *T_save, void *ws, size_t ws_bytes, void *stream);
