@@ -326,15 +326,27 @@ __device__ __forceinline__ void quant_lane16(const float (&v)[16], float amax, c
   }
 }
 
+// max(a, b, c) in one instruction (three-input max.f32, sm_100); a NaN input
+// is ignored as by fmaxf.
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
 // Group g of the tensor, this lane's sixteen weights in v: codes and c2 out,
 // the lane's share of the c2 sum into acc.
 __device__ __forceinline__ void quant_group(const float (&v)[16], int64_t g, const uint8_t *lut, const float *thr,
                                             const NF4Thresholds &th, uint8_t *__restrict__ codes,
                                             float *__restrict__ c2, double &acc) {
   const int lane = lane_id();
-  float amax = 0.f;
-#pragma unroll
-  for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(v[i]));
+  const float m0 = fmax3(fabsf(v[0]), fabsf(v[1]), fabsf(v[2]));
+  const float m1 = fmax3(fabsf(v[3]), fabsf(v[4]), fabsf(v[5]));
+  const float m2 = fmax3(fabsf(v[6]), fabsf(v[7]), fabsf(v[8]));
+  const float m3 = fmax3(fabsf(v[9]), fabsf(v[10]), fabsf(v[11]));
+  const float m4 = fmax3(fabsf(v[12]), fabsf(v[13]), fabsf(v[14]));
+  // (a block of NaN weights keeps c2 = 0, as the running fmaxf from 0 gave)
+  float amax = fmax3(fmax3(m0, m1, m2), fmax3(m3, m4, fabsf(v[15])), 0.f);
   amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 1));
   amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 2));
   uint32_t pk0, pk1;
@@ -452,17 +464,37 @@ __global__ void __launch_bounds__(kQuantThreads, 1) nf4_quantize_kernel(const TW
     }
   } else {
     // ------------------------------------------------------------ compute warps
-    for (int64_t q = warp; q < mine * kGroupsPerChunk; q += kQuantComputeWarps) {
-      const int64_t i = q / kGroupsPerChunk;
-      const int gi = (int)(q % kGroupsPerChunk);
-      const int st = (int)(i % S);
-      if (!__all_sync(0xFFFFFFFFu, mbar_wait(smem_u32(full + st), (uint32_t)(i / S) & 1u, err, DEV_TIMEOUT_MMA))) break;
+    // This warp's groups q = warp, warp + 28, ...: chunk i = q / 16 (of this
+    // CTA), group gi = q % 16 in it, ring slot i % S with phase (i / S) & 1,
+    // all tracked incrementally in 32-bit integers (a 64-bit division per
+    // group cost the ALU-bound loop measurably).
+    constexpr int kStepChunks = kQuantComputeWarps / kGroupsPerChunk;
+    constexpr int kStepGroups = kQuantComputeWarps % kGroupsPerChunk;
+    static_assert(kStepChunks + 1 < S, "a step crosses at most one ring wrap");
+    const int nq = (int)(mine * kGroupsPerChunk);
+    int i = warp / kGroupsPerChunk, gi = warp % kGroupsPerChunk;
+    int st = i % S;
+    uint32_t ph = (uint32_t)(i / S) & 1u;
+    for (int q = warp; q < nq; q += kQuantComputeWarps) {
+      if (!__all_sync(0xFFFFFFFFu, mbar_wait(smem_u32(full + st), ph, err, DEV_TIMEOUT_MMA))) break;
       float v[16];
       lds_unpack16<TW>(smem_u32(ring + st * Cfg::kChunkBytes) + (uint32_t)((gi * 512 + lane * 16) * (int)sizeof(TW)), v);
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(empty + st));   // this group's weights are in registers
-      const int64_t g = (blockIdx.x + i * gridDim.x) * kGroupsPerChunk + gi;
+      const int64_t g = ((int64_t)blockIdx.x + (int64_t)i * gridDim.x) * kGroupsPerChunk + gi;
       quant_group(v, g, lut, thr, th, codes, c2, acc);
+      int di = kStepChunks;
+      gi += kStepGroups;
+      if (gi >= kGroupsPerChunk) {
+        gi -= kGroupsPerChunk;
+        ++di;
+      }
+      i += di;
+      st += di;
+      if (st >= S) {
+        st -= S;
+        ph ^= 1u;
+      }
     }
     // The last CTA: the groups after the last whole chunk, from global memory.
     if (blockIdx.x == gridDim.x - 1) {
