@@ -101,3 +101,50 @@ def test_group_outputs_may_not_overlap_inputs_or_each_other():
     b["Y"] = buf[8:].view(M, N)                            # two outputs sharing bytes
     with pytest.raises(ValueError, match="member 0's Y overlaps member 1's Y"):
         qlora.linear_fwd_group([a, b])
+
+
+def _bwd_member(M=4, N=16, K=64, r=8, **kw):
+    m = _member(M, N, K, r)
+    m.update({"dY": torch.zeros(M, N, dtype=torch.bfloat16), "T": None})
+    m.update(kw)
+    return m
+
+
+def test_bwd_group_size_and_shapes():
+    with pytest.raises(ValueError, match="group holds"):
+        qlora.linear_bwd_group([])
+    with pytest.raises(ValueError, match="group holds"):
+        qlora.linear_bwd_group([_bwd_member() for _ in range(9)])
+    with pytest.raises(ValueError, match="shape mismatch"):
+        qlora.linear_bwd_group([_bwd_member(dY=torch.zeros(4, 24, dtype=torch.bfloat16))])
+    with pytest.raises(ValueError, match="T must be"):
+        qlora.linear_bwd_group([_bwd_member(T=torch.zeros(4, 8, dtype=torch.bfloat16))])
+    with pytest.raises(ValueError, match="share the token count"):
+        qlora.linear_bwd_group([_bwd_member(), _bwd_member(M=8)])
+
+
+@pytest.mark.parametrize("name,bad", [
+    ("dX", torch.zeros(4, 128, dtype=torch.bfloat16)),
+    ("dL1", torch.zeros(64, 8, dtype=torch.float32)),     # grad_dtype is bf16
+    ("dL2", torch.zeros(8, 24, dtype=torch.bfloat16)),
+])
+def test_bwd_group_outputs_are_checked(name, bad):
+    with pytest.raises(ValueError, match=f"{name} must be"):
+        qlora.linear_bwd_group([_bwd_member(**{name: bad})])
+
+
+def test_bwd_group_outputs_may_not_overlap():
+    a, b = _bwd_member(), _bwd_member()
+    shared = torch.zeros(64, 8, dtype=torch.bfloat16)
+    a["dL1"], b["dL1"] = shared, shared
+    with pytest.raises(ValueError, match="overlaps"):
+        qlora.linear_bwd_group([a, b])
+    c = _bwd_member()
+    c["dX"] = c["X"]                                        # an output on top of an input
+    with pytest.raises(ValueError, match="overlaps"):
+        qlora.linear_bwd_group([c])
+
+
+def test_bwd_group_host_tensors_are_refused():
+    with pytest.raises(ValueError, match="CUDA device"):
+        qlora.linear_bwd_group([_bwd_member()])
