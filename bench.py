@@ -700,6 +700,10 @@ def run_quantizer(args, rank, world, local_rank):
             qlora.dequant(q, out=out)
 
     ms, launches, clocks = _timed(qlora, step, args, dev, world, rank, local_rank)
+    # the same step replayed from a CUDA graph: the launches without the host's per-call cost
+    ms_graph = _graph_ms(step, dev, args.steps)
+    if qlora.last_device_error() != 0:
+        raise RuntimeError("device error in the graph replay of the quantizer step")
     if rank != 0:
         return None
     # Accuracy of the storage format (outside the timed region): RMS error of
@@ -730,6 +734,9 @@ def run_quantizer(args, rank, world, local_rank):
                    "bytes_quantize": nbytes_q, "bytes_dequant": nbytes_d,
                    "l2": "weights (667 MB bf16) larger than L2, no flush"},
         "gpu_launches": _kernel_count(launches),
+        "graph": {"ms_per_step": ms_graph, "value": (nbytes_q + nbytes_d) * world / (ms_graph * 1e-3) / 1e9,
+                  "unit": "GB/s", "frac_of_hbm": (nbytes_q + nbytes_d) / (ms_graph * 1e-3) / 1e9
+                  / load_peaks()[0].get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])},
         "roofline": {"bound": "hbm", "kernel": "quantize (K1 + K2) and dequant (K3)",
                      "achieved": roof_q, "achieved_dequant": roof_d, "peak": peak, "unit": "GB/s",
                      "frac": roof_q / peak if roof_q else None, "frac_dequant": roof_d / peak if roof_d else None,
