@@ -457,81 +457,12 @@ struct RankJob {
   int width() const { return fold ? fold : ncols; }
 };
 
-struct RankShape {
-  int64_t m_tiles, tiles, nkb;
-};
-
 RankShape rank_shape(const RankJob &j) {
   RankShape s;
   s.m_tiles = (j.A.rows + kBM - 1) / kBM;
   s.tiles = s.m_tiles * j.n_tiles;
   s.nkb = (j.A.kext + kBK - 1) / kBK;
   return s;
-}
-
-// Splits of each problem's reduction, chosen by simulating the kernel's walk:
-// units in order of decreasing length, CTA c taking unit kG + c in even rounds
-// and kG + G - 1 - c in odd ones.  A unit costs its k-blocks plus one (the
-// hand-over between units); a split unit three more (its partial's store and
-// the finalize's read, each 32 KB at r = 64 against 16 KB of A per k-block).
-// The plan with the smallest largest CTA load wins.  Plans are cached by shape.
-constexpr int kRankMinKb = 4;
-
-void plan_rank(const RankShape *sh, int n, int sms, int *splits) {
-  static std::mutex mu;
-  static std::map<std::vector<int64_t>, std::vector<int>> cache;
-  std::vector<int64_t> key{sms, n};
-  for (int i = 0; i < n; ++i) key.insert(key.end(), {sh[i].tiles, sh[i].nkb});
-  {
-    std::lock_guard<std::mutex> lock(mu);
-    auto it = cache.find(key);
-    if (it != cache.end()) {
-      std::copy(it->second.begin(), it->second.end(), splits);
-      return;
-    }
-  }
-  std::vector<int64_t> cand;
-  for (int i = 0; i < n; ++i)
-    for (int s = 1; s <= 32; ++s) {
-      const int64_t L = (sh[i].nkb + s - 1) / s;
-      if (L >= kRankMinKb || s == 1) cand.push_back(L);
-    }
-  std::sort(cand.begin(), cand.end());
-  cand.erase(std::unique(cand.begin(), cand.end()), cand.end());
-  std::vector<int> best(n, 1), cur(n);
-  int64_t best_span = INT64_MAX, best_units = INT64_MAX;
-  std::vector<int64_t> load;
-  std::vector<std::pair<int64_t, int64_t>> runs;   // (cost, count), longest first
-  for (int64_t L : cand) {
-    runs.clear();
-    int64_t units = 0;
-    for (int i = 0; i < n; ++i) {
-      int64_t s = std::max<int64_t>(1, (sh[i].nkb + L - 1) / L);
-      const int64_t kbps = (sh[i].nkb + s - 1) / s;
-      s = (sh[i].nkb + kbps - 1) / kbps;
-      cur[i] = (int)s;
-      runs.push_back({kbps + 1 + (s > 1 ? 3 : 0), sh[i].tiles * s});
-      units += sh[i].tiles * s;
-    }
-    std::stable_sort(runs.begin(), runs.end(), [](auto &a, auto &b) { return a.first > b.first; });
-    const int64_t G = std::max<int64_t>(1, std::min<int64_t>(units, sms));
-    load.assign((size_t)G, 0);
-    int64_t u = 0;
-    for (auto &rc : runs)
-      for (int64_t c = 0; c < rc.second; ++c, ++u) {
-        const int64_t k = u / G, pos = u - k * G;
-        load[(size_t)((k & 1) ? G - 1 - pos : pos)] += rc.first;
-      }
-    const int64_t span = *std::max_element(load.begin(), load.end());
-    if (span < best_span || (span == best_span && units < best_units)) {
-      best_span = span;
-      best_units = units;
-      best = cur;
-    }
-  }
-  std::copy(best.begin(), best.end(), splits);
-  std::lock_guard<std::mutex> lock(mu);
-  cache.emplace(std::move(key), std::move(best));
 }
 
 // fp32 partial bytes of a launch of these problems.
@@ -557,14 +488,7 @@ int rank_launch(const RankJob *jobs, int n, uint8_t *part, DeviceInfo *dev, cuda
   int64_t kbps[kRankMaxProbs];
   for (int i = 0; i < n; ++i) sh[i] = rank_shape(jobs[i]);
   plan_rank(sh, n, dev->sms, splits);
-  for (int i = 0; i < n; ++i) {
-    kbps[i] = (sh[i].nkb + splits[i] - 1) / splits[i];
-    order[i] = i;
-  }
-  // longest units first, as the plan assumed
-  std::stable_sort(order, order + n, [&](int a, int b) {
-    return kbps[a] + (splits[a] > 1 ? 3 : 0) > kbps[b] + (splits[b] > 1 ? 3 : 0);
-  });
+  rank_order(sh, splits, n, kbps, order);
   RankMaps maps;
   RankArgs a;
   RankFinArgs fin;

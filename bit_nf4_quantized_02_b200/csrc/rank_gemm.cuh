@@ -30,6 +30,12 @@
 // stage width (one or two 64-wide k-blocks per TMA box) are per problem.
 #pragma once
 
+#include <algorithm>
+#include <climits>
+#include <map>
+#include <mutex>
+#include <vector>
+
 #include "common.cuh"
 #include "tc_gemm.cuh"
 
@@ -86,7 +92,7 @@ struct RankUnit {
   int p, mt, nt, split;
 };
 
-__device__ __forceinline__ RankUnit rank_unit(const RankArgs &a, int u) {
+__host__ __device__ __forceinline__ RankUnit rank_unit(const RankArgs &a, int u) {
   RankUnit r;
   int p = 0;
   while (p + 1 < a.nprob && u >= a.prob[p + 1].unit0) ++p;
@@ -100,10 +106,12 @@ __device__ __forceinline__ RankUnit rank_unit(const RankArgs &a, int u) {
   return r;
 }
 
-// The unit of this CTA in round k: boustrophedon over the grid.
-__device__ __forceinline__ int rank_unit_of(int k, int G) {
-  return k * G + ((k & 1) ? (G - 1 - (int)blockIdx.x) : (int)blockIdx.x);
+// The unit of CTA b of G in round k: boustrophedon over the grid.
+__host__ __device__ __forceinline__ int rank_unit_at(int k, int G, int b) {
+  return k * G + ((k & 1) ? (G - 1 - b) : b);
 }
+
+__device__ __forceinline__ int rank_unit_of(int k, int G) { return rank_unit_at(k, G, (int)blockIdx.x); }
 
 // Store 32 consecutive columns col0.. of row `row` (values before alpha).
 __device__ __forceinline__ void rank_store(const RankOut &o, const RankProb &q, int row, int col0, int width,
@@ -435,6 +443,94 @@ __global__ void __launch_bounds__(256) rank_finalize_kernel(const __grid_constan
       if (f.lo_off > 0) o[off + f.lo_off] = __float2bfloat16_rn(s - __bfloat162float(hb));
     }
   }
+}
+
+
+// ------------------------------------------------------------------ host side
+// Scheduling of a launch, shared by the library's launcher and the host check
+// of the walk (tests/host/rank_walk_check.cu).
+
+// One problem as the planner sees it: its tiles (128-row tiles times n-tiles)
+// and the 64-wide k-blocks of its reduction.
+struct RankShape {
+  int64_t m_tiles, tiles, nkb;
+};
+
+// Splits of each problem's reduction, chosen by simulating the kernel's walk:
+// units in order of decreasing length, CTA c taking unit kG + c in even rounds
+// and kG + G - 1 - c in odd ones.  A unit costs its k-blocks plus one (the
+// hand-over between units); a split unit three more (its partial's store and
+// the finalize's read, each 32 KB at r = 64 against 16 KB of A per k-block).
+// The plan with the smallest largest CTA load wins.  Plans are cached by shape.
+constexpr int kRankMinKb = 4;
+
+inline void plan_rank(const RankShape *sh, int n, int sms, int *splits) {
+  static std::mutex mu;
+  static std::map<std::vector<int64_t>, std::vector<int>> cache;
+  std::vector<int64_t> key{sms, n};
+  for (int i = 0; i < n; ++i) key.insert(key.end(), {sh[i].tiles, sh[i].nkb});
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    auto it = cache.find(key);
+    if (it != cache.end()) {
+      std::copy(it->second.begin(), it->second.end(), splits);
+      return;
+    }
+  }
+  std::vector<int64_t> cand;
+  for (int i = 0; i < n; ++i)
+    for (int s = 1; s <= 32; ++s) {
+      const int64_t L = (sh[i].nkb + s - 1) / s;
+      if (L >= kRankMinKb || s == 1) cand.push_back(L);
+    }
+  std::sort(cand.begin(), cand.end());
+  cand.erase(std::unique(cand.begin(), cand.end()), cand.end());
+  std::vector<int> best(n, 1), cur(n);
+  int64_t best_span = INT64_MAX, best_units = INT64_MAX;
+  std::vector<int64_t> load;
+  std::vector<std::pair<int64_t, int64_t>> runs;   // (cost, count), longest first
+  for (int64_t L : cand) {
+    runs.clear();
+    int64_t units = 0;
+    for (int i = 0; i < n; ++i) {
+      int64_t s = std::max<int64_t>(1, (sh[i].nkb + L - 1) / L);
+      const int64_t kbps = (sh[i].nkb + s - 1) / s;
+      s = (sh[i].nkb + kbps - 1) / kbps;
+      cur[i] = (int)s;
+      runs.push_back({kbps + 1 + (s > 1 ? 3 : 0), sh[i].tiles * s});
+      units += sh[i].tiles * s;
+    }
+    std::stable_sort(runs.begin(), runs.end(), [](auto &a, auto &b) { return a.first > b.first; });
+    const int64_t G = std::max<int64_t>(1, std::min<int64_t>(units, sms));
+    load.assign((size_t)G, 0);
+    int64_t u = 0;
+    for (auto &rc : runs)
+      for (int64_t c = 0; c < rc.second; ++c, ++u) {
+        const int64_t k = u / G, pos = u - k * G;
+        load[(size_t)((k & 1) ? G - 1 - pos : pos)] += rc.first;
+      }
+    const int64_t span = *std::max_element(load.begin(), load.end());
+    if (span < best_span || (span == best_span && units < best_units)) {
+      best_span = span;
+      best_units = units;
+      best = cur;
+    }
+  }
+  std::copy(best.begin(), best.end(), splits);
+  std::lock_guard<std::mutex> lock(mu);
+  cache.emplace(std::move(key), std::move(best));
+}
+
+// The order of the problems in a launch, as the plan assumed: longest units
+// first (stable).  kbps receives each problem's k-blocks per split.
+inline void rank_order(const RankShape *sh, const int *splits, int n, int64_t *kbps, int *order) {
+  for (int i = 0; i < n; ++i) {
+    kbps[i] = (sh[i].nkb + splits[i] - 1) / splits[i];
+    order[i] = i;
+  }
+  std::stable_sort(order, order + n, [&](int a, int b) {
+    return kbps[a] + (splits[a] > 1 ? 3 : 0) > kbps[b] + (splits[b] > 1 ? 3 : 0);
+  });
 }
 
 }  // namespace qlora
