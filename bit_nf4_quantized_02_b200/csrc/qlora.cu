@@ -1506,9 +1506,9 @@ static int x_sets(const FwdMember *mem, int count, int *set_of) {
 }
 
 // Workspace: the bf16 weight (largest member, reused member after member);
-// T_cat fp32 [M x R] and L1_cat bf16 [K x R] of the largest shared-input set;
-// each member's T pair [M x 2r] (used where it passes no T_save); the split-K
-// partials of the largest adapter product.
+// L1_cat bf16 [K x R] of the largest set that shares X with equal ranks of 64
+// or 128; each member's T pair [M x 2r] (used where it passes no T_save); the
+// split partials of the largest adapter launch.
 struct GroupLargeLayout {
   size_t w_hat, l1_cat, t_own[kMaxGroup], split, total;
 };
