@@ -159,3 +159,59 @@ def test_llama7b_qkv_full_size_sampled():
         dL1_ref, dL2_ref = qlora_linear.adapter_grads(dYn, Xn, bf16_to_np(L1), bf16_to_np(L2), s)
         assert_close(dL1.float().cpu().numpy(), dL1_ref, f"{lin.name} dL1")
         assert_close(dL2.float().cpu().numpy(), dL2_ref, f"{lin.name} dL2")
+
+
+@pytest.mark.slow
+def test_llama7b_layer_groups_full_size_sampled():
+    """The training benchmark's launch configuration at full size: q, k, v,
+    gate and up on the layer input as one grouped forward (one adapter launch
+    over their L1 side by side), then gate and up as one grouped backward (its
+    G and dL2 problems split across the grid).  Y on 64 sampled output
+    features of every member, T in full; dX of gate and up on 256 sampled
+    token rows, dL1 and dL2 in full."""
+    from oracle import nf4dq
+    wl = workloads.LLAMA7B_LAYER
+    M, r, s = wl.M, wl.r, wl.s
+    lins = {l.name: l for l in wl.linears}
+    names = ("q", "k", "v", "gate", "up")
+    g = inputs.rng(wl.seed + 91)
+    H = inputs.normal_bf16(g, (M, lins["q"].k_in))
+    Hd = H.cuda()
+    host, dev = {}, {}
+    for i, name in enumerate(names):
+        N, K = lins[name].n_out, lins[name].k_in
+        Wd = inputs.device_normal((N, K), inputs.WEIGHT_STD, wl.seed + 300 + 10 * i, "cuda")
+        L1, L2 = inputs.lora_factors(inputs.rng(wl.seed + 301 + 10 * i), K, N, r)
+        host[name] = (Wd, L1, L2)
+        dev[name] = {"X": Hd, "q": qlora.quantize_nf4_dq(Wd), "L1": L1.cuda(), "L2": L2.cuda(), "s": s}
+    outs = qlora.linear_fwd_group([dev[n] for n in names])
+    torch.cuda.synchronize()
+    assert qlora.last_device_error() == 0
+    Hf = bf16_to_np(H).astype(np.float64)
+    for name, (Y, T) in zip(names, outs):
+        Wd, L1, L2 = host[name]
+        N = Wd.shape[0]
+        cols = np.sort(np.random.default_rng(N + len(name)).choice(N, 64, replace=False))
+        w_rows = nf4dq.dequantize_rows(Wd.cpu().numpy(), cols)
+        L1f, L2f = bf16_to_np(L1).astype(np.float64), bf16_to_np(L2).astype(np.float64)
+        Y_ref, T_ref = qlora_linear.forward(Hf, w_rows, L1f, L2f[:, cols], s)
+        assert_close(bf16_to_np(Y)[:, cols], Y_ref, f"{name} Y[:, sampled features]")
+        assert_close(qlora.t_value(T).cpu().numpy(), T_ref, f"{name} T")
+        dev[name]["T"] = T
+    dys = {}
+    for name in ("gate", "up"):
+        dys[name] = inputs.normal_bf16(g, (M, lins[name].n_out))
+        dev[name]["dY"] = dys[name].cuda()
+    bouts = qlora.linear_bwd_group([dev["gate"], dev["up"]])
+    torch.cuda.synchronize()
+    assert qlora.last_device_error() == 0
+    rows = np.sort(np.random.default_rng(3).choice(M, 256, replace=False))
+    for name, (dX, dL1, dL2) in zip(("gate", "up"), bouts):
+        Wd, L1, L2 = host[name]
+        w_hat = oracle_w_hat(oracle_quant(Wd.cpu()))
+        dYn = bf16_to_np(dys[name])
+        dX_ref = qlora_linear.backward_dx_rows(dYn[rows], w_hat, bf16_to_np(L1), bf16_to_np(L2), s)
+        assert_close(bf16_to_np(dX)[rows], dX_ref, f"{name} dX[rows]")
+        dL1_ref, dL2_ref = qlora_linear.adapter_grads(dYn, Hf, bf16_to_np(L1), bf16_to_np(L2), s)
+        assert_close(dL1.float().cpu().numpy(), dL1_ref, f"{name} dL1")
+        assert_close(dL2.float().cpu().numpy(), dL2_ref, f"{name} dL2")
