@@ -88,81 +88,87 @@ struct NF4Thresholds {
 };
 
 // Exact nearest-level codes without a division for almost every weight.
-// [-1, 1] is cut into kCodeBins bins of width 2^-13; bin(x) = floor((x + 1) *
-// kCodeBins / 2).  The estimate of x = fp32(w / absmax) is e = w * sc with sc
-// = RN(1/absmax) * kCodeBins/2, taken with one fused multiply-add (below):
-// both sc and x carry one rounding of relative size <= 2^-24 and |w / absmax|
-// <= 1, so e differs from x * kCodeBins/2 by at most 2 * 8192 * 2^-24 = 2^-10
-// of a bin, and the estimated bin is bin(x) - 1, bin(x) or bin(x) + 1.  So a
-// bin b with no decision threshold in bins b - 1 .. b + 1 (kCodeMargin = 1)
-// holds the one code of every x that can land in it, and is exact.  The bins
-// next to a threshold (3 per threshold, 0.27% of them) hold kCodeBoundary |
-// j, j the index of that threshold (thresholds are at least 342 bins apart,
-// so there is one), and their weights take the exact division: the code is
-// then j + (x > t_j).
+// [-1, 1] is cut into kCodeBins bins of width 2^-13; in bin units x sits at
+// X = (x + 1) * kCodeBins / 2 and threshold t_j at P_j = (t_j + 1) *
+// kCodeBins / 2.  The estimate of x = fp32(w / absmax) is E = w * sc +
+// kCodeBins / 2 with sc = RN(1/absmax) * kCodeBins/2 (a power-of-two
+// scaling, exact), taken with one fused multiply-add (below): w * RN(1/absmax)
+// and x each carry one rounding of relative size <= 2^-24 of w / absmax,
+// whose magnitude is <= 1, so |E - X| <= 8192 * 2 * 2^-24 = 2^-10.  The
+// estimated bin e = floor(E) therefore puts X in (e - 2^-10, e + 1 + 2^-10).
+// A bin e whose widened interval [e - d, e + 1 + d] (d = 2^-8, four times
+// that bound) holds no threshold gives every x that can land in it the same
+// code, #{j : P_j < e}, and that code is the table entry.  A bin whose
+// widened interval holds a threshold j (thresholds are at least 341 bins
+// apart, so at most one) holds kCodeBoundary | j, and its weights take the
+// exact division: the code is then j + (x > t_j).  That is the bin holding
+// P_j, and its neighbour only when P_j lies within d of their common edge:
+// one bin per threshold in almost every case, 0.09% of the bins.
 //
-// The table is indexed by b + 1, b the estimated bin, so that the two
-// rounding overshoots b = -1 and b = kCodeBins (x within an ulp of -1 or 1)
-// need no clamp: entry i holds the code of bin min(max(i - 1, 0), kCodeBins - 1).
-// In shared memory it is followed by zeros up to kCodeLutSpan entries, the
-// range of the 15-bit index below, so that no value of a weight (a NaN
-// included) can index outside it.
+// The table is indexed by e + 1 so that the rounding overshoots e = -1 and
+// e = kCodeBins (x within an ulp of -1 or 1) stay inside it; both hold the
+// code of the end they lie at.  In shared memory it is followed by zeros up
+// to kCodeLutSpan entries, the range of the 15-bit index below, so that no
+// value of a weight (a NaN included) can index outside it.
 constexpr int kCodeBins = 16384;
 constexpr int kCodeLutEntries = kCodeBins + 2;
-constexpr int kCodeMargin = 1;        // bins either side of a threshold's bin that are marked
+// Positions in fixed point, 2^16 units per bin: P_j * 2^16 = (t_j + 1) * 2^29
+// is an integer below 2^30 for every threshold of magnitude >= 2^-6 or zero
+// (all of both tables'), and (e + 1) * 2^16 + d stays below 2^31.
+constexpr int kCodeFixBits = 16;
+constexpr int kCodeFixMargin = 1 << (kCodeFixBits - 8);   // d = 2^-8 of a bin
 
 // Each CTA builds the table in its shared memory from the same thresholds
 // the exact path uses, before it waits for the kernel ahead of it (so the
-// build overlaps that kernel's tail).  Entry i holds, for the bin b =
-// min(max(i - 1, 0), kCodeBins - 1), either kCodeBoundary | j when the
-// boundary bin tb_j = floor((t_j + 1) * kCodeBins / 2) of threshold j lies
-// within kCodeMargin bins of b, or else the code #{j : tb_j < b}.  Entries
-// from kCodeLutBytes on are zero.
+// build overlaps that kernel's tail).  Entries from kCodeLutBytes on are
+// zero.
 //
 // A warp fills 32 consecutive words (128 entries, lane l word l) per pass.
-// Consecutive thresholds are hundreds of bins apart, so at most one threshold
-// lies within kCodeMargin bins of the 128 entries of a pass: the warp counts
-// the thresholds below its first bin minus the margin with one ballot, and a
-// lane whose four bins are clear of the next threshold stores that count four
-// times; the few lanes near a threshold resolve their four entries one by one.
+// The 128 bins of a pass with their margins span less than the gap between
+// two thresholds, so at most one threshold matters to a pass: the warp
+// counts the thresholds below its first bin's widened interval with one
+// ballot, and a lane whose four bins lie wholly below the next threshold
+// (margins included) stores that count four times; the few lanes near a
+// threshold resolve their four entries one by one.
 constexpr int kCodeLutBytes = (kCodeLutEntries + 3) / 4 * 4;
 constexpr int kCodeLutSpan = 32768;
 constexpr uint32_t kCodeBoundary = 0x80;
 
-__device__ __forceinline__ void build_code_lut(uint8_t *lut, int table, int *tb_s) {
+__device__ __forceinline__ void build_code_lut(uint8_t *lut, int table, int *pos_s) {
   if (threadIdx.x < 16) {
-    int tb = 0x7FFFFFFF;   // entry 15: past every bin
+    int p = 0x7FFFFFFF;   // entry 15: past every bin
     if (threadIdx.x < 15) {
       const float t = __double2float_rd(((double)kLevels[table][threadIdx.x] + (double)kLevels[table][threadIdx.x + 1]) * 0.5);
-      tb = (int)floor(((double)t + 1.0) * (kCodeBins / 2));
+      p = (int)floor(((double)t + 1.0) * (double)(1 << (13 + kCodeFixBits)));
     }
-    tb_s[threadIdx.x] = tb;
+    pos_s[threadIdx.x] = p;
   }
   __syncthreads();
   const int lane = threadIdx.x & 31;
-  const int my_tb = lane < 15 ? tb_s[lane] : 0x7FFFFFFF;
+  const int my_p = lane < 15 ? pos_s[lane] : 0x7FFFFFFF;
   uint32_t *lw = reinterpret_cast<uint32_t *>(lut);
   for (int w0 = (threadIdx.x & ~31); w0 < kCodeLutSpan / 4; w0 += blockDim.x) {
     const int w = w0 + lane;
-    const int first_bin = max(4 * w0 - 1, 0);
-    // thresholds more than kCodeMargin bins below the warp's first bin
-    const int c = __popc(__ballot_sync(0xFFFFFFFFu, my_tb < first_bin - kCodeMargin));
+    // bin of entry i is i - 1; the pass starts at bin 4 * w0 - 1
+    const int pass_lo = (4 * w0 - 1) * (1 << kCodeFixBits) - kCodeFixMargin;
+    const int c = __popc(__ballot_sync(0xFFFFFFFFu, my_p < pass_lo));
     uint32_t v = 0;
     if (4 * w < kCodeLutBytes) {
-      const int bhi = min(4 * w + 2, kCodeBins - 1);
-      const int tc = tb_s[c];
-      if (tc > bhi + kCodeMargin) {
+      const int pc = pos_s[c];
+      const int lane_hi = (4 * w + 3) * (1 << kCodeFixBits) + kCodeFixMargin;   // last bin 4w + 2, its upper edge
+      if (pc > lane_hi) {
         v = (uint32_t)c * 0x01010101u;
       } else {
-        const int tn = tb_s[min(c + 1, 15)];
+        const int pn = pos_s[min(c + 1, 15)];
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
-          const int b = min(max(4 * w + k - 1, 0), kCodeBins - 1);
-          const bool past = tc < b - kCodeMargin;   // threshold c is behind this bin
-          const int j = c + (past ? 1 : 0);         // first threshold >= b - kCodeMargin
-          const int tj = past ? tn : tc;
-          const uint32_t e = tj <= b + kCodeMargin ? (kCodeBoundary | (uint32_t)j) : (uint32_t)(j + (tj < b ? 1 : 0));
-          v |= e << (8 * k);
+          const int e = 4 * w + k - 1;
+          const int lo = e * (1 << kCodeFixBits) - kCodeFixMargin, hi = (e + 1) * (1 << kCodeFixBits) + kCodeFixMargin;
+          const bool past = pc < lo;            // threshold c lies below this bin's interval
+          const int j = c + (past ? 1 : 0);     // the first threshold not below it
+          const int pj = past ? pn : pc;
+          const uint32_t ent = pj <= hi ? (kCodeBoundary | (uint32_t)j) : (uint32_t)j;
+          v |= ent << (8 * k);
         }
       }
     }
@@ -195,9 +201,18 @@ __device__ __forceinline__ uint32_t pack_nibbles(uint32_t a, uint32_t b) {
   return __byte_perm(a, b, 0x6420);
 }
 
-// Bit q of the result: entry q of the word is a boundary entry.
-__device__ __forceinline__ uint32_t boundary_bits(uint32_t w) {
-  return (((w & 0x80808080u) >> 7) * 0x01020408u) >> 24;
+// The boundary entries of four entry words in one mask: entry k of word w
+// (element 4w + k of the sixteen) at bit 8k + 7 - 4 (w & 1) - (w >> 1), i.e.
+// the words' flag bits 7, 3, 6 and 2 of each byte.
+__device__ __forceinline__ uint32_t boundary_mask(uint32_t w0, uint32_t w1, uint32_t w2, uint32_t w3) {
+  const uint32_t a = (w0 & 0x80808080u) | ((w2 & 0x80808080u) >> 1);
+  const uint32_t b = (w1 & 0x80808080u) | ((w3 & 0x80808080u) >> 1);
+  return a | (b >> 4);
+}
+
+// The element (0..15) of bit p of boundary_mask.
+__device__ __forceinline__ int boundary_element(int p) {
+  return (p >> 3) | (~p & 4) | ((~p & 1) << 3);
 }
 
 // Sixteen consecutive weights as loaded (two or four 16-byte loads).  Issuing
@@ -305,9 +320,9 @@ __device__ __forceinline__ void quant_lane16(const float (&v)[16], float amax, c
     pk1 = pack_nibbles(w2, w3);
     if ((w0 | w1 | w2 | w3) & 0x80808080u) {
       // Boundary weights (a few per warp): exact division, code = j + (x > t_j).
-      uint32_t m = boundary_bits(w0) | (boundary_bits(w1) << 4) | (boundary_bits(w2) << 8) | (boundary_bits(w3) << 12);
+      uint32_t m = boundary_mask(w0, w1, w2, w3);
       while (m) {
-        const int i = __ffs(m) - 1;
+        const int i = boundary_element(__ffs(m) - 1);
         m &= m - 1;
         const int sh = 4 * (i & 7);
         uint32_t &pk = i < 8 ? pk0 : pk1;
@@ -420,7 +435,7 @@ __global__ void __launch_bounds__(kQuantThreads, 1) nf4_quantize_kernel(const TW
   __shared__ __align__(16) uint8_t lut[kCodeLutSpan];
   __shared__ double red[kQuantThreads / 32];
   __shared__ float thr[16];
-  __shared__ int tb_s[16];
+  __shared__ int pos_s[16];
   NF4Thresholds th;
   th.init(table);
   if (threadIdx.x < 15)
@@ -433,7 +448,7 @@ __global__ void __launch_bounds__(kQuantThreads, 1) nf4_quantize_kernel(const TW
     }
     fence_mbar_init();
   }
-  build_code_lut(lut, table, tb_s);
+  build_code_lut(lut, table, pos_s);
   __syncthreads();
   pdl_trigger();
   pdl_wait();
