@@ -215,10 +215,9 @@ __device__ __forceinline__ int boundary_element(int p) {
   return (p >> 3) | (~p & 4) | ((~p & 1) << 3);
 }
 
-// Sixteen consecutive weights as loaded (two or four 16-byte loads).  Issuing
-// the next group's loads before processing this one (one more group in
-// flight per warp) was measured slower: the registers it needs drop the
-// kernel from five to four resident CTAs per SM.
+// Sixteen consecutive weights loaded from global memory (two or four 16-byte
+// loads): the groups after the last whole chunk, which the last CTA
+// quantizes without the ring.
 template <typename TW>
 struct Raw16;
 template <>
@@ -256,8 +255,9 @@ struct Raw16<__nv_bfloat16> {
 };
 
 // Element i (0..15, a run-time index) of the sixteen unpacked weights, by a
-// select tree: the fix-up below reads it from registers instead of
-// reloading it from global memory.
+// select tree: the fix-up below reads it from registers, since the ring slot
+// the weights came from may already be refilled (and the tail groups come
+// from global memory).
 __device__ __forceinline__ float select16(const float (&v)[16], int i) {
   float a[8], b[4];
 #pragma unroll
