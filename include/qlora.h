@@ -233,10 +233,14 @@ QLORA_API int qlora_linear_bwd(const uint16_t *dY, const uint16_t *X, const uint
  *   concatenated work of all members, instead of one chain per linear: the
  *   per-linear launch gaps and tails of the few-token path disappear.
  *   Members of different code tables (W->table) run as one chain per table.
- *   With M > 128, members that read the same X (same pointer and K) share one
- *   adapter down-projection, X [L1_a | L1_b | ...] (their L1 copied side by
- *   side), split into each member's T; then every member runs its own
- *   doubleDequant and tensor-core product, in order.
+ *   With M > 128, the adapter down-projections T_i = s_i X L1_i of members
+ *   that read the same X (same pointer and K) run as one launch of the
+ *   grouped rank-r kernel (ranks up to 128; a set holding a larger rank runs
+ *   each member's own forward); with equal ranks of 64 or 128 their L1 are first
+ *   copied side by side, X [L1_a | L1_b | ...], so that each strip of X is
+ *   read for all of them together.  Every member's T is written as its hi/lo
+ *   pair; then every member runs its own doubleDequant and tensor-core
+ *   product, in order.
  *   LoRA dropout is not part of the grouped forward (qlora_linear_fwd_dropout
  *   runs it per linear).  count = 0 or M = 0: nothing is done.  Workspace:
  *   qlora_linear_fwd_group_workspace_size(), which returns 0 for invalid
