@@ -1,7 +1,7 @@
 """GPU parity of the fused few-token forward (M <= 128 tokens: the weight is
 decoded into tensor memory for the tensor core and never written to HBM as
-bf16) against the float64 oracle, and how close its decoded weight is to
-doubleDequant's exact bf16 weight."""
+bf16) against the float64 oracle, and its decoded weight against
+doubleDequant's exact bf16 weight, bit for bit."""
 
 import numpy as np
 import pytest
