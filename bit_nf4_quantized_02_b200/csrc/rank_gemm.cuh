@@ -1,9 +1,13 @@
-// Grouped rank-r products of the QLoRA backward (QLoRA §3, the paragraph
-// after Eq. 6: gradients flow to the adapter only):
+// Grouped rank-r products of the QLoRA linear: the backward's (QLoRA §3, the
+// paragraph after Eq. 6: gradients flow to the adapter only)
 //
 //   G_i   = s_i dY_i L2_i^T          [M x r]   contraction over n_out
 //   dL2_i = T_i^T dY_i               [r x N]   contraction over the tokens
 //   dL1_i = X_i^T G_i                [K x r]   contraction over the tokens
+//
+// and the forward's adapter down-projection (§2 Eq. 3, §3 Eq. 5)
+//
+//   T_i   = s_i X_i L1_i             [M x r]   contraction over k_in
 //
 // Each is a skinny product that streams one big operand (dY or X) once; one
 // launch per product spends a large share of its time in launch ramp, first
