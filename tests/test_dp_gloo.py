@@ -77,3 +77,60 @@ def test_two_rank_allreduce_matches_full_batch():
     assert all(r[1] for r in results), results
     assert sum(r[2] for r in results) == 37
     assert all(p.exitcode == 0 for p in procs)
+
+
+def _leaver(rank, world, port, q, steps_before_leaving, stall=0.0):
+    """Rank 1 takes part in `steps_before_leaving` exchanges, then leaves
+    between steps: it exits without its next all-reduce, or (stall > 0) stays
+    alive that many seconds without joining it.  Rank 0 keeps stepping and
+    must get an error from its next exchange, not wait for ever."""
+    import datetime
+    import time
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=5))
+    grads = FlatGrads([(64, 24, 8)], device="cpu")
+    for step in range(steps_before_leaving):
+        grads.flat.fill_(float(rank + 1))
+        grads.allreduce()
+        assert grads.flat.eq(3.0).all()
+    if rank == 1:
+        q.put((rank, "left", 0.0))
+        time.sleep(stall)
+        q.close()
+        q.join_thread()        # the message is out before the process goes
+        os._exit(0)            # no destroy, no further collective: the process is gone
+    t0 = time.monotonic()
+    try:
+        grads.allreduce()
+        q.put((rank, "no error", time.monotonic() - t0))
+    except Exception as e:    # gloo reports the lost peer (or the timeout) as an error
+        q.put((rank, type(e).__name__, time.monotonic() - t0))
+    q.close()
+    q.join_thread()
+    os._exit(0)
+
+
+@pytest.mark.parametrize("stall", [0.0, 15.0])
+def test_rank_leaving_between_steps_ends_the_next_exchange_with_an_error(stall):
+    """A rank that exits (stall 0) or stops taking part (stall 15 s, three
+    times the 5 s process-group timeout) between steps: the other rank's next
+    gradient exchange ends with an error, the peer loss at once, the silent
+    rank at the timeout."""
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_leaver, args=(r, 2, port, q, 2, stall)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=120)
+    alive = [p for p in procs if p.is_alive()]
+    for p in alive:
+        p.kill()
+    assert not alive, "a rank was still waiting after 120 s"
+    results = dict((r, (what, dt)) for r, what, dt in (q.get(timeout=10) for _ in range(2)))
+    assert results[1][0] == "left"
+    what, dt = results[0]
+    assert what != "no error", "the exchange with a departed rank completed"
+    assert dt < (14.0 if stall else 4.0), f"the error came after {dt:.1f} s"
