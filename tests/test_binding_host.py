@@ -1,7 +1,8 @@
 """Argument checks of the Python binding that run before the library is loaded
 or any device pointer is taken (no GPU, no built library needed): member
 counts and shapes, caller-supplied outputs of the wrong shape or dtype,
-tensors on different devices, and grouped outputs that overlap inputs."""
+tensors on different devices, and grouped outputs that overlap inputs; and
+that without the built library the binding raises instead of computing."""
 
 import pytest
 import torch
@@ -148,3 +149,17 @@ def test_bwd_group_outputs_may_not_overlap():
 def test_bwd_group_host_tensors_are_refused():
     with pytest.raises(ValueError, match="CUDA device"):
         qlora.linear_bwd_group([_bwd_member()])
+
+
+def test_missing_library_fails_loudly(monkeypatch, tmp_path):
+    """Without libqlora.so the binding raises; it has no other way to compute."""
+    from bit_nf4_quantized_02_b200 import _lib
+    monkeypatch.setattr(_lib, "LIB_PATH", str(tmp_path / "libqlora.so"))
+    monkeypatch.setattr(_lib, "_lib", None)
+    with pytest.raises(RuntimeError, match="not built"):
+        _lib.load()
+    # public calls reach the loader and stop there
+    with pytest.raises(RuntimeError, match="not built"):
+        qlora.last_device_error()
+    with pytest.raises(RuntimeError, match="not built"):
+        qlora.profile_start(16)
